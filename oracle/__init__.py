@@ -1,0 +1,232 @@
+"""CPU oracle for the QLoRA frozen-NF4 linear layer.
+
+TEST INFRASTRUCTURE ONLY: the tests, ``__graft_entry__.smoke()`` and the
+``cpu_baseline`` leg of ``bench.py`` are the only callers.  The product
+library never imports, links or runs anything here, and nothing here imports
+the product package.
+
+Two parts:
+
+* ``nf4_oracle.c`` (built into ``liboracle_nf4.so`` with gcc, loaded through
+  ctypes): the codebook, block absmax, NF4 encoding, double quantization and
+  dequantization, bit for bit, in plain loops.
+* the forward and backward of the linear layer below, written out as their
+  definitions in fp64 with numpy matrix products as the only library step.
+
+Page citations (title, section):
+
+* "QLoRA Guide" (dataaihub.co), "How QLoRA Works / Forward pass" and its
+  "Dequant + LoRA path" diagram: the input goes both through the dequantized
+  frozen weight and through LoRA A then B, and the two are summed; only A and
+  B get gradients, the dequantized weight is a constant for autograd.
+* "QLoRA Implementation Details (2025 Edition)", "Step 4: Apply LoRA
+  Adapters": the LoRA scaling is alpha / r.
+* "QLORA: Efficient Finetuning of Quantized LLMs" (imaddabbura.github.io),
+  "Notes": every forward/backward loads the 4-bit weights, dequantizes to
+  BF16, multiplies, and computes gradients only for the adapters, which are
+  stored and trained in BF16.
+
+Parity unpinned (no value on the pages to pin against, only self-consistency
+and mathematics): the codebook values themselves (reading R1), the tie rule
+(R2), the nibble order (R3) and the int8 form of the double quantization
+(R4).  Everything else is pinned by the tests in ``tests/test_oracle_*.py``.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "nf4_oracle.c")
+_LIB = os.path.join(_HERE, "liboracle_nf4.so")
+
+NF4_BLOCK = 64
+DQ_GROUP = 256
+
+
+def build(force: bool = False) -> str:
+    """Compile the C oracle with gcc (no fused multiply-add contraction)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        cmd = ["gcc", "-O2", "-std=c11", "-ffp-contract=off", "-fno-fast-math", "-fPIC", "-shared",
+               _SRC, "-o", _LIB + ".tmp", "-lm"]
+        subprocess.check_call(cmd)
+        os.replace(_LIB + ".tmp", _LIB)
+    return _LIB
+
+
+_lib = None
+
+
+def lib():
+    global _lib
+    if _lib is None:
+        build()
+        L = ctypes.CDLL(_LIB)
+        P = ctypes.c_void_p
+        i64 = ctypes.c_int64
+        L.oracle_ppnd16.restype = ctypes.c_double
+        L.oracle_ppnd16.argtypes = [ctypes.c_double]
+        L.oracle_nf4_codebook.argtypes = [P, P]
+        L.oracle_nf4_midpoints.argtypes = [P, P]
+        L.oracle_nf4_encode_value.restype = ctypes.c_int
+        L.oracle_nf4_encode_value.argtypes = [ctypes.c_float, P]
+        L.oracle_bf16_to_f32.restype = ctypes.c_float
+        L.oracle_bf16_to_f32.argtypes = [ctypes.c_uint16]
+        L.oracle_f32_to_bf16.restype = ctypes.c_uint16
+        L.oracle_f32_to_bf16.argtypes = [ctypes.c_float]
+        L.oracle_block_absmax.argtypes = [P, i64, P]
+        L.oracle_double_quant.argtypes = [P, i64, P, P, P]
+        L.oracle_quantize_dq.restype = ctypes.c_int
+        L.oracle_quantize_dq.argtypes = [P, i64, i64, P, P, P, P, P]
+        L.oracle_block_constant.restype = ctypes.c_float
+        L.oracle_block_constant.argtypes = [ctypes.c_int8, ctypes.c_float, ctypes.c_float]
+        L.oracle_dequant.restype = ctypes.c_int
+        L.oracle_dequant.argtypes = [P, P, P, P, i64, i64, P]
+        L.oracle_dequant_rows.restype = ctypes.c_int
+        L.oracle_dequant_rows.argtypes = [P, P, P, P, i64, i64, P, i64, P]
+        _lib = L
+    return _lib
+
+
+def _ptr(a: np.ndarray):
+    assert a.flags["C_CONTIGUOUS"]
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+# --------------------------------------------------------------------------
+# codebook and scalar encoding
+# --------------------------------------------------------------------------
+def ppnd16(p: float) -> float:
+    """Inverse standard normal CDF (Wichura 1988, AS 241)."""
+    return lib().oracle_ppnd16(float(p))
+
+
+def codebook():
+    """The 16 NF4 levels: (fp64 before rounding, fp32 as used)."""
+    v64 = np.zeros(16, np.float64)
+    v32 = np.zeros(16, np.float32)
+    lib().oracle_nf4_codebook(_ptr(v64), _ptr(v32))
+    return v64, v32
+
+
+def midpoints(L32: np.ndarray | None = None) -> np.ndarray:
+    if L32 is None:
+        L32 = codebook()[1]
+    L32 = np.ascontiguousarray(L32, np.float32)
+    m = np.zeros(15, np.float32)
+    lib().oracle_nf4_midpoints(_ptr(L32), _ptr(m))
+    return m
+
+
+def encode_value(x: float, m: np.ndarray | None = None) -> int:
+    if m is None:
+        m = midpoints()
+    m = np.ascontiguousarray(m, np.float32)
+    return lib().oracle_nf4_encode_value(ctypes.c_float(float(x)), _ptr(m))
+
+
+def bf16_to_f32(bits: np.ndarray) -> np.ndarray:
+    """Exact widening of raw bf16 bit patterns (uint16) to fp32."""
+    return (np.asarray(bits, np.uint16).astype(np.uint32) << 16).view(np.float32)
+
+
+def f32_to_bf16_scalar(f: float) -> int:
+    return int(lib().oracle_f32_to_bf16(ctypes.c_float(f)))
+
+
+# --------------------------------------------------------------------------
+# quantize / double-quant / dequant
+# --------------------------------------------------------------------------
+def quantize_dq(W_bits: np.ndarray):
+    """bf16 W [N, K] (raw uint16 bits) -> dict(packed, codes, scale, mean, absmax)."""
+    W_bits = np.ascontiguousarray(W_bits, np.uint16)
+    N, K = W_bits.shape
+    nblocks = N * K // NF4_BLOCK
+    G = (nblocks + DQ_GROUP - 1) // DQ_GROUP
+    packed = np.zeros((N, K // 2), np.uint8)
+    codes = np.zeros(nblocks, np.int8)
+    scale = np.zeros(G, np.float32)
+    mean = np.zeros(G, np.float32)
+    absmax = np.zeros(nblocks, np.float32)
+    rc = lib().oracle_quantize_dq(_ptr(W_bits), N, K, _ptr(packed), _ptr(codes), _ptr(scale), _ptr(mean),
+                                  _ptr(absmax))
+    if rc != 0:
+        raise ValueError(f"oracle_quantize_dq rejected shape {W_bits.shape}")
+    return dict(packed=packed, codes=codes, scale=scale, mean=mean, absmax=absmax, N=N, K=K)
+
+
+def double_quant(absmax: np.ndarray):
+    absmax = np.ascontiguousarray(absmax, np.float32)
+    nb = absmax.size
+    G = (nb + DQ_GROUP - 1) // DQ_GROUP
+    codes = np.zeros(nb, np.int8)
+    scale = np.zeros(G, np.float32)
+    mean = np.zeros(G, np.float32)
+    lib().oracle_double_quant(_ptr(absmax), nb, _ptr(codes), _ptr(scale), _ptr(mean))
+    return codes, scale, mean
+
+
+def block_constant(code: int, scale: float, mean: float) -> float:
+    return float(lib().oracle_block_constant(ctypes.c_int8(int(code)), ctypes.c_float(scale),
+                                             ctypes.c_float(mean)))
+
+
+def dequant(q: dict) -> np.ndarray:
+    """NF4-DQ -> bf16 W' [N, K] as raw uint16 bits."""
+    N, K = q["N"], q["K"]
+    out = np.zeros((N, K), np.uint16)
+    rc = lib().oracle_dequant(_ptr(q["packed"]), _ptr(q["codes"]), _ptr(q["scale"]), _ptr(q["mean"]),
+                              N, K, _ptr(out))
+    if rc != 0:
+        raise ValueError("oracle_dequant rejected its arguments")
+    return out
+
+
+def dequant_rows(q: dict, rows) -> np.ndarray:
+    N, K = q["N"], q["K"]
+    rows = np.ascontiguousarray(np.asarray(rows, np.int64))
+    out = np.zeros((rows.size, K), np.uint16)
+    rc = lib().oracle_dequant_rows(_ptr(q["packed"]), _ptr(q["codes"]), _ptr(q["scale"]), _ptr(q["mean"]),
+                                   N, K, _ptr(rows), rows.size, _ptr(out))
+    if rc != 0:
+        raise ValueError("oracle_dequant_rows rejected its arguments")
+    return out
+
+
+# --------------------------------------------------------------------------
+# linear layer forward / backward, fp64 definitions
+# --------------------------------------------------------------------------
+def lora_scaling(r: int, alpha: float) -> float:
+    """LoRA scaling alpha / r ("Step 4: Apply LoRA Adapters": r=64, alpha=16 -> 0.25)."""
+    return float(alpha) / float(r)
+
+
+def linear_fwd(X, Wd, A, B, s):
+    """Y = X W'^T + s (X A^T) B^T and T = X A^T, all fp64.
+
+    X [M, K], Wd = W' [N, K] (already dequantized), A [r, K], B [N, r].
+    """
+    X = np.asarray(X, np.float64)
+    T = X @ np.asarray(A, np.float64).T
+    Y = X @ np.asarray(Wd, np.float64).T + s * (T @ np.asarray(B, np.float64).T)
+    return Y, T
+
+
+def linear_bwd(X, dY, Wd, A, B, s):
+    """Gradients of <Y, dY> for the layer above; the frozen W' gets none.
+
+    U = dY B, dX = dY W' + s U A, dA = s U^T X, dB = s dY^T T with T = X A^T.
+    """
+    X = np.asarray(X, np.float64)
+    dY = np.asarray(dY, np.float64)
+    A = np.asarray(A, np.float64)
+    B = np.asarray(B, np.float64)
+    T = X @ A.T
+    U = dY @ B
+    dX = dY @ np.asarray(Wd, np.float64) + s * (U @ A)
+    dA = s * (U.T @ X)
+    dB = s * (dY.T @ T)
+    return dX, dA, dB

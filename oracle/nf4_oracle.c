@@ -1,0 +1,305 @@
+/*
+ * nf4_oracle.c -- plain, slow, obviously-correct CPU oracle for the NF4 +
+ * double-quantization encoding of a frozen QLoRA base weight.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing in the product library links, loads or
+ * calls this file; only the tests, the smoke check and the CPU-baseline leg of
+ * the benchmark do.  It shares no code, header, table or constant generator
+ * with the CUDA library: the codebook here comes from Wichura's AS 241
+ * inverse-normal, the library computes its own by bisection on erfc.
+ *
+ * What the pages fix, and where:
+ *   - "QLoRA Guide" (dataaihub.co), section "NF4 vs uniform INT4": NF4 places
+ *     its 16 levels at quantiles of the standard normal; quantization is
+ *     block-wise so an outlier only spoils its own block.
+ *   - "Qlora Expert" (skillsdirectory.com), section "Core Concept": levels at
+ *     N(0,1) quantiles; double quantization re-quantizes the per-block fp32
+ *     constants to 8 bit; section "Memory Math" / "Hyperparameter Guidance":
+ *     the saving is about 0.37 bit per parameter.
+ *   - "QLoRA Implementation Details (2025 Edition)" (spritualkrishna.cloud),
+ *     section "Step 1: 4-bit Quantization with NF4", "NF4 Math": 64 values
+ *     per block.
+ *   - "QLoRA: The 4-bit Revolution" (shshell.com), section "2. Double
+ *     Quantization": the scaling factors go from 32-bit to 8-bit.
+ * Readings taken where the pages are silent (each listed in the design doc):
+ *   R1 codebook construction (asymmetric 8 positive / 7 negative quantiles,
+ *      offset delta = ((1-1/32)+(1-1/30))/2, normalised by the largest level);
+ *   R2 nearest level with ties to the lower index, via fp32 midpoints;
+ *   R3 nibble order: element 2j in the high nibble of byte j;
+ *   R4 double quantization: groups of 256 block constants, fp32 mean and a
+ *      symmetric int8 code of (c - mean) with scale = max|c - mean| / 127;
+ *      the group sum is taken in fp64 over a pairwise tree (stride 128..1);
+ *   R5 dequantized weight = bf16_rne(L[q] * fmaf(code, scale, mean)).
+ *
+ * Compile with -ffp-contract=off: every fp32 operation below is meant to be
+ * one IEEE-rounded operation, exactly as written.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <string.h>
+
+#define NF4_BLOCK 64
+#define DQ_GROUP 256
+
+/* ---------------------------------------------------------------------------
+ * Inverse standard normal CDF, Wichura (1988), Applied Statistics algorithm
+ * AS 241 "PPND16" (rational approximations, about 1e-16 relative accuracy).
+ * Returns the x with Phi(x) = p for 0 < p < 1.
+ * ------------------------------------------------------------------------- */
+double oracle_ppnd16(double p)
+{
+    double q = p - 0.5;
+    double r, val;
+    if (fabs(q) <= 0.425) {
+        r = 0.180625 - q * q;
+        val = q * (((((((r * 2509.0809287301226727 + 33430.575583588128105) * r +
+                        67265.770927008700853) * r + 45921.953931549871457) * r +
+                      13731.693765509461125) * r + 1971.5909503065514427) * r +
+                    133.14166789178437745) * r + 3.387132872796366608) /
+              (((((((r * 5226.495278852545925 + 28729.085735721942674) * r +
+                    39307.89580009271061) * r + 21213.794301586595867) * r +
+                  5394.1960214247511077) * r + 687.1870074920579083) * r +
+                42.313330701600911252) * r + 1.0);
+        return val;
+    }
+    r = (q < 0.0) ? p : 1.0 - p;
+    r = sqrt(-log(r));
+    if (r <= 5.0) {
+        r -= 1.6;
+        val = (((((((r * 7.7454501427834140764e-4 + 0.0227238449892691845833) * r +
+                    0.24178072517745061177) * r + 1.27045825245236838258) * r +
+                  3.64784832476320460504) * r + 5.7694972214606914055) * r +
+                4.6303378461565452959) * r + 1.42343711074968357734) /
+              (((((((r * 1.05075007164441684324e-9 + 5.475938084995344946e-4) * r +
+                    0.0151986665636164571966) * r + 0.14810397642748007459) * r +
+                  0.68976733498510000455) * r + 1.6763848301838038494) * r +
+                2.05319162663775882187) * r + 1.0);
+    } else {
+        r -= 5.0;
+        val = (((((((r * 2.01033439929228813265e-7 + 2.71155556874348757815e-5) * r +
+                    0.0012426609473880784386) * r + 0.026532189526576123093) * r +
+                  0.29656057182850489123) * r + 1.7848265399172913358) * r +
+                5.4637849111641143699) * r + 6.6579046435011037772) /
+              (((((((r * 2.04426310338993978564e-15 + 1.4215117583164458887e-7) * r +
+                    1.8463183175100546818e-5) * r + 7.868691311456132591e-4) * r +
+                  0.0148753612908506148525) * r + 0.13692988092273580531) * r +
+                0.59983220655588793769) * r + 1.0);
+    }
+    return (q < 0.0) ? -val : val;
+}
+
+/* ---------------------------------------------------------------------------
+ * Reading R1: the 16 NF4 levels.  8 positive quantiles at the first 8 of 9
+ * evenly spaced probabilities from delta down to 1/2, 7 negative ones at the
+ * first 7 of 8 evenly spaced probabilities, plus an exact zero; sorted and
+ * divided (in fp64) by the largest, then rounded once to fp32.  The top and
+ * bottom levels are both Phi^-1(delta) before normalisation, so they come out
+ * as exactly +1 and -1.
+ * ------------------------------------------------------------------------- */
+void oracle_nf4_codebook(double out64[16], float out32[16])
+{
+    const double delta = 0.5 * ((1.0 - 1.0 / 32.0) + (1.0 - 1.0 / 30.0));
+    double v[16];
+    int n = 0;
+    for (int i = 0; i < 7; ++i) {          /* negative side, largest magnitude first */
+        double p = delta + (0.5 - delta) * (double)i / 7.0;
+        v[n++] = -oracle_ppnd16(p);
+    }
+    v[n++] = 0.0;
+    for (int i = 7; i >= 0; --i) {         /* positive side, ascending */
+        double p = delta + (0.5 - delta) * (double)i / 8.0;
+        v[n++] = oracle_ppnd16(p);
+    }
+    /* v is already ascending: -Phi^-1 is increasing in i on the negative side,
+     * Phi^-1 is decreasing in i on the positive side and walked backwards. */
+    double vmax = v[15];
+    for (int i = 0; i < 16; ++i) {
+        out64[i] = v[i] / vmax;
+        out32[i] = (float)out64[i];
+    }
+}
+
+/* Reading R2: decision thresholds m_i = fl32((L_i + L_{i+1}) / 2). */
+void oracle_nf4_midpoints(const float L[16], float m[15])
+{
+    for (int i = 0; i < 15; ++i) m[i] = (L[i] + L[i + 1]) * 0.5f;
+}
+
+/* Reading R2: the level index of a normalised value is the number of
+ * thresholds it lies strictly above (a value exactly on a threshold takes the
+ * lower level). */
+int oracle_nf4_encode_value(float x, const float m[15])
+{
+    int q = 0;
+    for (int i = 0; i < 15; ++i)
+        if (x > m[i]) ++q;
+    return q;
+}
+
+/* bf16 <-> fp32 from the IEEE-754 definitions (bf16 is the top half of an
+ * fp32 word; fp32 -> bf16 rounds to nearest, ties to even). */
+float oracle_bf16_to_f32(uint16_t h)
+{
+    uint32_t u = (uint32_t)h << 16;
+    float f;
+    memcpy(&f, &u, 4);
+    return f;
+}
+
+uint16_t oracle_f32_to_bf16(float f)
+{
+    uint32_t u;
+    memcpy(&u, &f, 4);
+    if ((u & 0x7fffffffu) > 0x7f800000u) return (uint16_t)((u >> 16) | 0x0040u); /* NaN stays NaN */
+    uint32_t lsb = (u >> 16) & 1u;
+    u += 0x7fffu + lsb;
+    return (uint16_t)(u >> 16);
+}
+
+/* ---------------------------------------------------------------------------
+ * Block absmax (one fp32 constant per 64 consecutive weights in flattened
+ * row-major order).  Exact: a bf16 magnitude is an fp32 value.
+ * ------------------------------------------------------------------------- */
+void oracle_block_absmax(const uint16_t* W, int64_t nblocks, float* absmax)
+{
+    for (int64_t b = 0; b < nblocks; ++b) {
+        float c = 0.0f;
+        for (int j = 0; j < NF4_BLOCK; ++j) {
+            float a = fabsf(oracle_bf16_to_f32(W[b * NF4_BLOCK + j]));
+            if (a > c) c = a;
+        }
+        absmax[b] = c;
+    }
+}
+
+/* ---------------------------------------------------------------------------
+ * Reading R4: second-level quantization of the block constants.
+ * For the group g of blocks [256 g, 256 g + n_g):
+ *   S       = fp64 pairwise sum of the constants (256 slots, empty slots 0,
+ *             slot i += slot i + stride for stride = 128, 64, ..., 1)
+ *   mean_g  = fl32(S / n_g)
+ *   d_b     = fl32(c_b - mean_g)
+ *   scale_g = fl32(max_b |d_b| / 127)
+ *   code_b  = clamp(rint(fl32(d_b / scale_g)), -127, 127), or 0 if scale_g = 0
+ * ------------------------------------------------------------------------- */
+void oracle_double_quant(const float* absmax, int64_t nblocks, int8_t* codes, float* scale, float* mean)
+{
+    int64_t ngroups = (nblocks + DQ_GROUP - 1) / DQ_GROUP;
+    for (int64_t g = 0; g < ngroups; ++g) {
+        int64_t b0 = g * DQ_GROUP;
+        int64_t n = nblocks - b0;
+        if (n > DQ_GROUP) n = DQ_GROUP;
+        double slot[DQ_GROUP];
+        for (int i = 0; i < DQ_GROUP; ++i) slot[i] = (i < n) ? (double)absmax[b0 + i] : 0.0;
+        for (int stride = DQ_GROUP / 2; stride >= 1; stride /= 2)
+            for (int i = 0; i < stride; ++i) slot[i] = slot[i] + slot[i + stride];
+        float mu = (float)(slot[0] / (double)n);
+        float dmax = 0.0f;
+        for (int64_t i = 0; i < n; ++i) {
+            float d = absmax[b0 + i] - mu;
+            if (fabsf(d) > dmax) dmax = fabsf(d);
+        }
+        float sc = dmax / 127.0f;
+        for (int64_t i = 0; i < n; ++i) {
+            int code = 0;
+            if (sc != 0.0f) {
+                float d = absmax[b0 + i] - mu;
+                float t = rintf(d / sc);
+                if (t > 127.0f) t = 127.0f;
+                if (t < -127.0f) t = -127.0f;
+                code = (int)t;
+            }
+            codes[b0 + i] = (int8_t)code;
+        }
+        scale[g] = sc;
+        mean[g] = mu;
+    }
+}
+
+/* ---------------------------------------------------------------------------
+ * Quantize + double-quantize a bf16 weight W [N, K] (row-major, K % 64 == 0).
+ * Outputs: packed [N, K/2] (reading R3), codes [N*K/64], scale/mean [G].
+ * The nibbles are encoded with the true block absmax c_b (quantization
+ * happens first, the constants are compressed after).
+ * ------------------------------------------------------------------------- */
+int oracle_quantize_dq(const uint16_t* W, int64_t N, int64_t K, uint8_t* packed, int8_t* codes,
+                       float* scale, float* mean, float* absmax_scratch)
+{
+    if (N <= 0 || K <= 0 || (K % NF4_BLOCK) != 0) return -1;
+    double L64[16];
+    float L[16], m[15];
+    oracle_nf4_codebook(L64, L);
+    oracle_nf4_midpoints(L, m);
+    int64_t nblocks = N * K / NF4_BLOCK;
+    oracle_block_absmax(W, nblocks, absmax_scratch);
+    for (int64_t b = 0; b < nblocks; ++b) {
+        float c = absmax_scratch[b];
+        for (int j = 0; j < NF4_BLOCK; j += 2) {
+            int q[2];
+            for (int h = 0; h < 2; ++h) {
+                if (c == 0.0f) {
+                    q[h] = 7;                        /* the exact-zero level */
+                } else {
+                    float x = oracle_bf16_to_f32(W[b * NF4_BLOCK + j + h]) / c;
+                    q[h] = oracle_nf4_encode_value(x, m);
+                }
+            }
+            packed[(b * NF4_BLOCK + j) / 2] = (uint8_t)((q[0] << 4) | q[1]);
+        }
+    }
+    oracle_double_quant(absmax_scratch, nblocks, codes, scale, mean);
+    return 0;
+}
+
+/* Reading R5: the block constant recovered from its int8 code. */
+float oracle_block_constant(int8_t code, float scale, float mean)
+{
+    return fmaf((float)code, scale, mean);
+}
+
+/* Reading R5: W' = bf16_rne(L[q] * c'_b) for every weight. */
+int oracle_dequant(const uint8_t* packed, const int8_t* codes, const float* scale, const float* mean,
+                   int64_t N, int64_t K, uint16_t* Wout)
+{
+    if (N <= 0 || K <= 0 || (K % NF4_BLOCK) != 0) return -1;
+    double L64[16];
+    float L[16];
+    oracle_nf4_codebook(L64, L);
+    int64_t nblocks = N * K / NF4_BLOCK;
+    for (int64_t b = 0; b < nblocks; ++b) {
+        int64_t g = b / DQ_GROUP;
+        float cp = oracle_block_constant(codes[b], scale[g], mean[g]);
+        for (int j = 0; j < NF4_BLOCK; ++j) {
+            int64_t e = b * NF4_BLOCK + j;
+            uint8_t byte = packed[e / 2];
+            int q = (e % 2 == 0) ? (byte >> 4) : (byte & 0x0f);
+            float w = L[q] * cp;
+            Wout[e] = oracle_f32_to_bf16(w);
+        }
+    }
+    return 0;
+}
+
+/* Dequantize only the listed rows of W' (for sampled parity on large shapes). */
+int oracle_dequant_rows(const uint8_t* packed, const int8_t* codes, const float* scale, const float* mean,
+                        int64_t N, int64_t K, const int64_t* rows, int64_t nrows, uint16_t* Wout)
+{
+    if (N <= 0 || K <= 0 || (K % NF4_BLOCK) != 0) return -1;
+    double L64[16];
+    float L[16];
+    oracle_nf4_codebook(L64, L);
+    for (int64_t ri = 0; ri < nrows; ++ri) {
+        int64_t n = rows[ri];
+        if (n < 0 || n >= N) return -2;
+        for (int64_t k = 0; k < K; ++k) {
+            int64_t e = n * K + k;
+            int64_t b = e / NF4_BLOCK;
+            int64_t g = b / DQ_GROUP;
+            float cp = oracle_block_constant(codes[b], scale[g], mean[g]);
+            uint8_t byte = packed[e / 2];
+            int q = (e % 2 == 0) ? (byte >> 4) : (byte & 0x0f);
+            Wout[ri * K + k] = oracle_f32_to_bf16(L[q] * cp);
+        }
+    }
+    return 0;
+}
