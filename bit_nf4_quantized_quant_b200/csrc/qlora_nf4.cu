@@ -1,0 +1,491 @@
+// qlora_nf4.cu -- the extern "C" entry points of libqlora_nf4.so (single
+// translation unit: the kernels are pulled in from the .cuh files).
+//
+// The ABI is documented in include/qlora_nf4.h.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "common.cuh"
+#include "quant.cuh"
+#include "small.cuh"
+#include "lora.cuh"
+
+using namespace qnf4;
+
+namespace {
+
+// ---------------------------------------------------------------------------
+// Codebook on the host: inverse normal CDF by bisection on libm's erfc,
+// Phi(x) = erfc(-x / sqrt 2) / 2, to the resolution of a double.  The
+// construction of the 16 levels is the one documented at nf4_codebook().
+// ---------------------------------------------------------------------------
+double phi(double x) { return 0.5 * std::erfc(-x / std::sqrt(2.0)); }
+
+double inv_phi_bisect(double p) {
+    double lo = -40.0, hi = 40.0;
+    for (int it = 0; it < 2000; ++it) {
+        const double mid = 0.5 * (lo + hi);
+        if (mid <= lo || mid >= hi) break;
+        if (phi(mid) < p) lo = mid; else hi = mid;
+    }
+    return 0.5 * (lo + hi);
+}
+
+NF4Tables g_tables;
+std::once_flag g_tables_once;
+
+void init_tables() {
+    const double delta = 0.5 * ((1.0 - 1.0 / 32.0) + (1.0 - 1.0 / 30.0));
+    double pos[8], neg[7];
+    for (int i = 0; i < 8; ++i) pos[i] = inv_phi_bisect(delta - (delta - 0.5) * i / 8.0);   // descending
+    for (int i = 0; i < 7; ++i) neg[i] = -inv_phi_bisect(delta - (delta - 0.5) * i / 7.0);  // ascending
+    double v[16];
+    for (int i = 0; i < 7; ++i) v[i] = neg[i];
+    v[7] = 0.0;
+    for (int i = 0; i < 8; ++i) v[8 + i] = pos[7 - i];
+    const double top = v[15];
+    for (int i = 0; i < 16; ++i) g_tables.L[i] = (float)(v[i] / top);
+    for (int i = 0; i < 15; ++i) g_tables.m[i] = (g_tables.L[i] + g_tables.L[i + 1]) * 0.5f;
+    g_tables.pad = 0.f;
+}
+
+const NF4Tables& tables() {
+    std::call_once(g_tables_once, init_tables);
+    return g_tables;
+}
+
+thread_local int t_last_path = 0;
+
+int g_sm_count[64];
+std::atomic<int> g_dev_ok[64];   // 0 unknown, 1 sm_100, -1 other
+
+int check_device(int* sm_count) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return QLORA_ERR_DEVICE;
+    if (dev < 0 || dev >= 64) return QLORA_ERR_DEVICE;
+    int st = g_dev_ok[dev].load();
+    if (st == 0) {
+        int major = 0, minor = 0, sms = 0;
+        if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+            return QLORA_ERR_DEVICE;
+        g_sm_count[dev] = sms;
+        st = (major == 10 && minor == 0) ? 1 : -1;
+        if (st == 1) {
+            // opt in to more than 48 KB of dynamic shared memory, once per device
+            const cudaError_t e = [&] {
+                cudaError_t r = cudaFuncSetAttribute(k_fwd_small<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                     fwd_small_smem_bytes<1>());
+                if (r == cudaSuccess) r = cudaFuncSetAttribute(k_fwd_small<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                               fwd_small_smem_bytes<2>());
+                if (r == cudaSuccess) r = cudaFuncSetAttribute(k_fwd_small<4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                               fwd_small_smem_bytes<4>());
+                if (r == cudaSuccess) r = cudaFuncSetAttribute(k_bwd_small<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                               bwd_small_smem_bytes<1>());
+                if (r == cudaSuccess) r = cudaFuncSetAttribute(k_bwd_small<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                               bwd_small_smem_bytes<2>());
+                return r;
+            }();
+            if (e != cudaSuccess) return QLORA_ERR_LAUNCH;
+        }
+        g_dev_ok[dev].store(st);
+    }
+    if (st != 1) return QLORA_ERR_DEVICE;
+    if (sm_count) *sm_count = g_sm_count[dev];
+    return QLORA_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int launch_status() {
+    const cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? QLORA_OK : QLORA_ERR_LAUNCH;
+}
+
+// ---------------------------------------------------------------------------
+// Workspace plan: every region 256-byte aligned; regions used one after the
+// other on a stream may share the "partials" region.
+// ---------------------------------------------------------------------------
+struct Plan {
+    int64_t M, N, K;
+    int r, rp;
+    // split-K choices
+    int zT, zU, zA, zB;
+    int64_t kT, kU, kA, kB;         // k per split
+    int S_bwd;                      // small-path N splits for dX
+    int64_t rows_per_split;
+    // byte offsets
+    size_t off_part, off_T32, off_U32, off_Tp, off_Ubf, off_sT, off_sU, off_Bp, off_At, total;
+};
+
+size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+// Tile of the skinny GEMM for an I x J output: (BI, BJ).
+void gemm_tile(int64_t I, int64_t J, int64_t* bi, int64_t* bj) {
+    if (J <= 16) { *bi = 64; *bj = 16; }
+    else if (I <= 16) { *bi = 16; *bj = 64; }
+    else { *bi = 64; *bj = 64; }
+}
+
+// Bytes of fp32 split-K partials for an I x J output with z splits.
+size_t gemm_part_bytes(int64_t I, int64_t J, int z) {
+    int64_t bi, bj;
+    gemm_tile(I, J, &bi, &bj);
+    return (size_t)z * rup(I, bi) * rup(J, bj) * 4;
+}
+
+int choose_splits(int64_t tiles, int64_t kd, int64_t target) {
+    int64_t z = cdiv(target, tiles > 0 ? tiles : 1);
+    const int64_t zmax = cdiv(kd, 256);
+    if (z > zmax) z = zmax;
+    if (z < 1) z = 1;
+    return (int)z;
+}
+
+Plan make_plan(int64_t M, int64_t N, int64_t K, int r, int sms) {
+    Plan p{};
+    p.M = M; p.N = N; p.K = K; p.r = r;
+    p.rp = (int)rup(r, 16);
+    const int64_t target = 2 * (int64_t)sms;
+    const int64_t bj = p.rp == 16 ? 16 : 64;
+    // T = X A^T: I = M (BI 64), J = rp, Kd = K
+    p.zT = choose_splits(cdiv(M, 64) * cdiv(p.rp, bj), K, target);
+    p.kT = rup(cdiv(K, p.zT), 32);
+    p.zT = (int)cdiv(K, p.kT);
+    // U = dY B: Kd = N
+    p.zU = choose_splits(cdiv(M, 64) * cdiv(p.rp, bj), N, target);
+    p.kU = rup(cdiv(N, p.zU), 32);
+    p.zU = (int)cdiv(N, p.kU);
+    // dA = U^T X: I = rp, J = K (BJ 64), Kd = M
+    const int64_t bi = p.rp == 16 ? 16 : 64;
+    p.zA = choose_splits(cdiv(p.rp, bi) * cdiv(K, 64), M, target);
+    p.kA = rup(cdiv(M, p.zA), 32);
+    p.zA = (int)cdiv(M, p.kA);
+    // dB = dY^T T: I = N (BI 64), J = rp, Kd = M
+    p.zB = choose_splits(cdiv(N, 64) * cdiv(p.rp, bj), M, target);
+    p.kB = rup(cdiv(M, p.zB), 32);
+    p.zB = (int)cdiv(M, p.kB);
+    // small-path dX: units = ceil(K/64/4) * S
+    {
+        const int64_t nkg = cdiv(K / kBlock, kBwdKW);
+        int64_t S = cdiv(target, nkg);
+        int64_t rps = rup(cdiv(N, S < 1 ? 1 : S), 64);
+        if (rps < 64) rps = 64;
+        p.rows_per_split = rps;
+        p.S_bwd = (int)cdiv(N, rps);
+    }
+    size_t part = 0;
+    auto upd = [&](size_t b) { if (b > part) part = b; };
+    upd(gemm_part_bytes(M, p.rp, p.zT));
+    upd(gemm_part_bytes(M, p.rp, p.zU));
+    upd(gemm_part_bytes(p.rp, K, p.zA));
+    upd(gemm_part_bytes(N, p.rp, p.zB));
+    if (M <= 32) upd((size_t)p.S_bwd * M * K * 4);
+    else upd((size_t)p.S_bwd * 32 * K * 4);   // large M processes 32-token chunks
+    size_t off = 0;
+    auto take = [&](size_t b) { const size_t o = off; off = align256(off + b); return o; };
+    p.off_part = take(part);
+    p.off_T32 = take((size_t)M * p.rp * 4);
+    p.off_U32 = take((size_t)M * p.rp * 4);
+    p.off_Tp = take((size_t)M * p.rp * 2);
+    p.off_Ubf = take((size_t)M * p.rp * 2);
+    p.off_sT = take((size_t)M * p.rp * 2);
+    p.off_sU = take((size_t)M * p.rp * 2);
+    p.off_Bp = take((size_t)N * p.rp * 2);
+    p.off_At = take((size_t)K * p.rp * 2);
+    p.total = off;
+    return p;
+}
+
+int grid_for(int64_t work, int per, int sms, int64_t cap_mult = 8) {
+    int64_t g = cdiv(work, per);
+    if (g > (int64_t)sms * cap_mult) g = (int64_t)sms * cap_mult;
+    if (g < 1) g = 1;
+    return (int)g;
+}
+
+// Split-K skinny GEMM + finish.
+template <bool AK, bool BK>
+int run_gemm(const uint16_t* A, int64_t lda, const uint16_t* B, int64_t ldb, int64_t I, int64_t J, int64_t Kd,
+             int64_t Ilim, int64_t Jlim, int z, int64_t kps, float* part, const FinishArgs& fin_in, int sms,
+             cudaStream_t st) {
+    GemmArgs g{};
+    g.A = A; g.B = B; g.C = part; g.lda = lda; g.ldb = ldb;
+    g.Kd = Kd; g.Ilim = Ilim; g.Jlim = Jlim; g.k_per_split = kps;
+    FinishArgs f = fin_in;
+    f.C = part; f.splits = z;
+    int64_t bi, bj;
+    gemm_tile(I, J, &bi, &bj);
+    g.I = rup(I, bi); g.J = rup(J, bj);
+    dim3 grid((unsigned)(g.I / bi), (unsigned)(g.J / bj), (unsigned)z);
+    if (bj == 16) k_gemm_mma<AK, BK, 64, 16, 4, 1><<<grid, 128, 0, st>>>(g);
+    else if (bi == 16) k_gemm_mma<AK, BK, 16, 64, 1, 4><<<grid, 128, 0, st>>>(g);
+    else k_gemm_mma<AK, BK, 64, 64, 2, 2><<<grid, 128, 0, st>>>(g);
+    f.I = g.I; f.J = g.J;
+    if (f.Iout > I) f.Iout = I;
+    if (f.Jout > J) f.Jout = J;
+    k_gemm_finish<<<grid_for(f.Iout * f.Jout, 256, sms), 256, 0, st>>>(f);
+    return launch_status();
+}
+
+FinishArgs fin_none() {
+    FinishArgs f{};
+    return f;
+}
+
+int validate_weight(const nf4dq_weight* w) {
+    if (!w || !w->packed || !w->codes || !w->scale || !w->mean) return QLORA_ERR_NULL;
+    if (w->N <= 0 || w->K <= 0 || (w->K % kBlock) != 0 || (w->N % 8) != 0) return QLORA_ERR_SHAPE;
+    if (w->N > (int64_t)1 << 31 || w->K > (int64_t)1 << 31 || w->N * w->K > ((int64_t)1 << 40)) return QLORA_ERR_SHAPE;
+    if (!aligned16(w->packed)) return QLORA_ERR_ALIGN;
+    return QLORA_OK;
+}
+
+// T (fp32 into ws, optional bf16 T_out [M, r], bf16 padded Tp and s*T) from X, A.
+int compute_T(const Plan& p, const uint16_t* X, const uint16_t* A, float s, uint16_t* T_out, uint8_t* ws, int sms,
+              cudaStream_t st) {
+    FinishArgs f = fin_none();
+    f.Iout = p.M; f.Jout = p.rp;
+    f.f32 = reinterpret_cast<float*>(ws + p.off_T32); f.ld_f32 = p.rp;
+    f.o1 = reinterpret_cast<uint16_t*>(ws + p.off_Tp); f.s1i = p.rp; f.s1j = 1; f.J1 = p.r; f.J1pad = p.rp; f.alpha1 = 1.f;
+    f.o2 = reinterpret_cast<uint16_t*>(ws + p.off_sT); f.s2i = p.rp; f.s2j = 1; f.J2 = p.r; f.J2pad = p.rp; f.alpha2 = s;
+    int rc = run_gemm<true, true>(X, p.K, A, p.K, p.M, p.rp, p.K, p.M, p.r, p.zT, p.kT,
+                                  reinterpret_cast<float*>(ws + p.off_part), f, sms, st);
+    if (rc != QLORA_OK) return rc;
+    if (T_out) {
+        // bf16 copy in the caller's unpadded [M, r] layout
+        k_pad_cols<<<grid_for(p.M * p.r, 256, sms), 256, 0, st>>>(reinterpret_cast<uint16_t*>(ws + p.off_Tp), p.M,
+                                                                   p.rp, T_out, p.r);
+        rc = launch_status();
+    }
+    return rc;
+}
+
+}  // namespace
+
+// ===========================================================================
+// extern "C" entry points
+// ===========================================================================
+extern "C" {
+
+int nf4_codebook(float out16[16]) {
+    if (!out16) return QLORA_ERR_NULL;
+    const NF4Tables& t = tables();
+    for (int i = 0; i < 16; ++i) out16[i] = t.L[i];
+    return QLORA_OK;
+}
+
+int nf4dq_sizes(int64_t N, int64_t K, int64_t* packed_bytes, int64_t* n_blocks, int64_t* n_groups) {
+    if (N <= 0 || K <= 0 || (K % kBlock) != 0) return QLORA_ERR_SHAPE;
+    if (N > ((int64_t)1 << 40) / K) return QLORA_ERR_SHAPE;
+    const int64_t nb = N * K / kBlock;
+    if (packed_bytes) *packed_bytes = N * K / 2;
+    if (n_blocks) *n_blocks = nb;
+    if (n_groups) *n_groups = cdiv(nb, kGroup);
+    return QLORA_OK;
+}
+
+int nf4_quantize_dq(const qlora_bf16* W, int64_t N, int64_t K, uint8_t* packed, int8_t* codes, float* scale,
+                    float* mean, qlora_stream_t stream) {
+    if (!W || !packed || !codes || !scale || !mean) return QLORA_ERR_NULL;
+    int64_t nb = 0, ng = 0;
+    if (nf4dq_sizes(N, K, nullptr, &nb, &ng) != QLORA_OK) return QLORA_ERR_SHAPE;
+    if (!aligned16(W) || !aligned16(packed)) return QLORA_ERR_ALIGN;
+    int sms = 0;
+    int rc = check_device(&sms);
+    if (rc != QLORA_OK) return rc;
+    const NF4Tables& tab = tables();
+    int grid = (int)(ng < (int64_t)sms * 8 ? ng : (int64_t)sms * 8);
+    k_quantize_dq<<<grid, 256, 0, (cudaStream_t)stream>>>(W, nb, packed, codes, scale, mean, tab);
+    return launch_status();
+}
+
+int nf4_dequant(const nf4dq_weight* w, qlora_bf16* W_out, qlora_stream_t stream) {
+    int rc = (!w || !W_out) ? QLORA_ERR_NULL : QLORA_OK;
+    if (rc != QLORA_OK) return rc;
+    if (!w->packed || !w->codes || !w->scale || !w->mean) return QLORA_ERR_NULL;
+    if (nf4dq_sizes(w->N, w->K, nullptr, nullptr, nullptr) != QLORA_OK) return QLORA_ERR_SHAPE;
+    if (!aligned16(w->packed) || !aligned16(W_out)) return QLORA_ERR_ALIGN;
+    int sms = 0;
+    rc = check_device(&sms);
+    if (rc != QLORA_OK) return rc;
+    const int64_t nchunks = w->N * w->K / 32;
+    k_dequant<<<grid_for(nchunks, 256, sms), 256, 0, (cudaStream_t)stream>>>(w->packed, w->codes, w->scale, w->mean,
+                                                                            nchunks, W_out, tables());
+    return launch_status();
+}
+
+size_t qlora_workspace_bytes(int64_t M, int64_t N, int64_t K, int r) {
+    if (M <= 0 || N <= 0 || K <= 0 || (K % kBlock) != 0 || (N % 8) != 0) return 0;
+    if (r < 1 || r > QLORA_MAX_RANK) return 0;
+    return make_plan(M, N, K, r, 148).total;
+}
+
+int qlora_linear_fwd(const qlora_bf16* X, int64_t M, const nf4dq_weight* w, const qlora_bf16* A,
+                     const qlora_bf16* B, int r, float scaling, qlora_bf16* Y, qlora_bf16* T_out, void* ws,
+                     size_t ws_bytes, qlora_stream_t stream) {
+    if (!X || !A || !B || !Y) return QLORA_ERR_NULL;
+    int rc = validate_weight(w);
+    if (rc != QLORA_OK) return rc;
+    if (M <= 0 || M > ((int64_t)1 << 31)) return QLORA_ERR_SHAPE;
+    if (r < 1 || r > QLORA_MAX_RANK) return QLORA_ERR_RANK;
+    if (!std::isfinite(scaling)) return QLORA_ERR_VALUE;
+    if (!aligned16(X) || !aligned16(Y) || !aligned16(A)) return QLORA_ERR_ALIGN;
+    if (!ws || (reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return ws ? QLORA_ERR_ALIGN : QLORA_ERR_WORKSPACE;
+    int sms = 0;
+    rc = check_device(&sms);
+    if (rc != QLORA_OK) return rc;
+    const Plan p = make_plan(M, w->N, w->K, r, 148);
+    if (ws_bytes < p.total) return QLORA_ERR_WORKSPACE;
+    cudaStream_t st = (cudaStream_t)stream;
+    uint8_t* wsb = static_cast<uint8_t*>(ws);
+
+    rc = compute_T(p, X, A, scaling, T_out, wsb, sms, st);
+    if (rc != QLORA_OK) return rc;
+
+    SmallFwdArgs a{};
+    a.X = X; a.packed = w->packed; a.codes = w->codes; a.scale = w->scale; a.mean = w->mean;
+    a.T32 = reinterpret_cast<const float*>(wsb + p.off_T32); a.B = B; a.Y = Y;
+    a.M = M; a.N = w->N; a.K = w->K; a.rp = p.rp; a.r = r; a.s = scaling;
+    const int64_t ntiles = cdiv(w->N, 16);
+    const int grid = (int)(ntiles < 2LL * sms ? ntiles : 2LL * sms);
+    if (M <= 8) {
+        k_fwd_small<1><<<grid, kSmallThreads, fwd_small_smem_bytes<1>(), st>>>(a, tables());
+    } else if (M <= 16) {
+        k_fwd_small<2><<<grid, kSmallThreads, fwd_small_smem_bytes<2>(), st>>>(a, tables());
+    } else {
+        k_fwd_small<4><<<grid, kSmallThreads, fwd_small_smem_bytes<4>(), st>>>(a, tables());
+    }
+    rc = launch_status();
+    if (rc == QLORA_OK) t_last_path = 1;
+    return rc;
+}
+
+int qlora_linear_bwd(const qlora_bf16* X, const qlora_bf16* dY, int64_t M, const nf4dq_weight* w,
+                     const qlora_bf16* A, const qlora_bf16* B, int r, float scaling, const qlora_bf16* T,
+                     qlora_bf16* dX, qlora_bf16* dA, qlora_bf16* dB, void* ws, size_t ws_bytes,
+                     qlora_stream_t stream) {
+    if (!X || !dY || !A || !B || !dX || !dA || !dB) return QLORA_ERR_NULL;
+    int rc = validate_weight(w);
+    if (rc != QLORA_OK) return rc;
+    if (M <= 0 || M > ((int64_t)1 << 31)) return QLORA_ERR_SHAPE;
+    if (r < 1 || r > QLORA_MAX_RANK) return QLORA_ERR_RANK;
+    if (!std::isfinite(scaling)) return QLORA_ERR_VALUE;
+    if (!aligned16(X) || !aligned16(dY) || !aligned16(A) || !aligned16(dX) || !aligned16(B)) return QLORA_ERR_ALIGN;
+    if (T && !aligned16(T)) return QLORA_ERR_ALIGN;
+    if (!ws || (reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return ws ? QLORA_ERR_ALIGN : QLORA_ERR_WORKSPACE;
+    int sms = 0;
+    rc = check_device(&sms);
+    if (rc != QLORA_OK) return rc;
+    const int64_t N = w->N, K = w->K;
+    const Plan p = make_plan(M, N, K, r, 148);
+    if (ws_bytes < p.total) return QLORA_ERR_WORKSPACE;
+    cudaStream_t st = (cudaStream_t)stream;
+    uint8_t* wsb = static_cast<uint8_t*>(ws);
+    float* part = reinterpret_cast<float*>(wsb + p.off_part);
+    uint16_t* Tp = reinterpret_cast<uint16_t*>(wsb + p.off_Tp);
+    uint16_t* Ubf = reinterpret_cast<uint16_t*>(wsb + p.off_Ubf);
+    uint16_t* Bp = reinterpret_cast<uint16_t*>(wsb + p.off_Bp);
+
+    // T: recompute, or take the caller's bf16 copy (padded to rp columns)
+    if (T == nullptr) {
+        rc = compute_T(p, X, A, scaling, nullptr, wsb, sms, st);
+    } else {
+        k_pad_cols<<<grid_for(M * p.rp, 256, sms), 256, 0, st>>>(T, M, r, Tp, p.rp);
+        rc = launch_status();
+    }
+    if (rc != QLORA_OK) return rc;
+
+    // U = dY B  ->  U32 (fp32), Ubf (bf16, unscaled), sU (bf16, scaled)
+    const uint16_t* Bop = B;
+    int64_t ldb = r;
+    if (r % 8 != 0) {
+        k_pad_cols<<<grid_for(N * p.rp, 256, sms), 256, 0, st>>>(B, N, r, Bp, p.rp);
+        Bop = Bp; ldb = p.rp;
+    }
+    {
+        FinishArgs f = fin_none();
+        f.Iout = M; f.Jout = p.rp;
+        f.f32 = reinterpret_cast<float*>(wsb + p.off_U32); f.ld_f32 = p.rp;
+        f.o1 = Ubf; f.s1i = p.rp; f.s1j = 1; f.J1 = r; f.J1pad = p.rp; f.alpha1 = 1.f;
+        f.o2 = reinterpret_cast<uint16_t*>(wsb + p.off_sU); f.s2i = p.rp; f.s2j = 1; f.J2 = r; f.J2pad = p.rp;
+        f.alpha2 = scaling;
+        rc = run_gemm<true, false>(dY, N, Bop, ldb, M, p.rp, N, M, r, p.zU, p.kU, part, f, sms, st);
+        if (rc != QLORA_OK) return rc;
+    }
+    // dB = s dY^T T  [N, r]
+    {
+        FinishArgs f = fin_none();
+        f.Iout = N; f.Jout = r;
+        f.o1 = dB; f.s1i = r; f.s1j = 1; f.J1 = r; f.J1pad = r; f.alpha1 = scaling;
+        rc = run_gemm<false, false>(dY, N, Tp, p.rp, N, p.rp, M, N, p.rp, p.zB, p.kB, part, f, sms, st);
+        if (rc != QLORA_OK) return rc;
+    }
+    // dA = s U^T X  [r, K]
+    {
+        FinishArgs f = fin_none();
+        f.Iout = r; f.Jout = K;
+        f.o1 = dA; f.s1i = K; f.s1j = 1; f.J1 = K; f.J1pad = K; f.alpha1 = scaling;
+        rc = run_gemm<false, false>(Ubf, p.rp, X, K, p.rp, K, M, p.rp, K, p.zA, p.kA, part, f, sms, st);
+        if (rc != QLORA_OK) return rc;
+    }
+    // dX = dY W' + s U A
+    {
+        const int64_t MC = 16;
+        for (int64_t m0 = 0; m0 < M; m0 += (M <= 16 ? M : MC)) {
+            const int64_t mc = (M <= 16) ? M : (M - m0 < MC ? M - m0 : MC);
+            SmallBwdArgs a{};
+            a.dY = dY + m0 * N; a.packed = w->packed; a.codes = w->codes; a.scale = w->scale; a.mean = w->mean;
+            a.part = part; a.M = mc; a.N = N; a.K = K; a.rows_per_split = p.rows_per_split; a.S = p.S_bwd;
+            const int64_t units = cdiv(K / kBlock, kBwdKW) * p.S_bwd;
+            const int grid = (int)(units < 2LL * sms ? units : 2LL * sms);
+            if (mc <= 8) k_bwd_small<1><<<grid, kSmallThreads, bwd_small_smem_bytes<1>(), st>>>(a, tables());
+            else k_bwd_small<2><<<grid, kSmallThreads, bwd_small_smem_bytes<2>(), st>>>(a, tables());
+            k_bwd_small_finish<<<grid_for(mc * K, 256, sms), 256, 0, st>>>(
+                part, p.S_bwd, mc, K, reinterpret_cast<const float*>(wsb + p.off_U32) + m0 * p.rp, p.rp, A, r,
+                scaling, dX + m0 * K);
+            rc = launch_status();
+            if (rc != QLORA_OK) return rc;
+        }
+    }
+    t_last_path = 1;
+    return QLORA_OK;
+}
+
+const char* qlora_status_string(int status) {
+    switch (status) {
+        case QLORA_OK: return "ok";
+        case QLORA_ERR_NULL: return "a required pointer is NULL";
+        case QLORA_ERR_SHAPE: return "invalid shape (M, N, K must be > 0, K % 64 == 0, N % 8 == 0)";
+        case QLORA_ERR_RANK: return "LoRA rank r outside [1, 256]";
+        case QLORA_ERR_ALIGN: return "pointer not 16-byte aligned (workspace: 256-byte)";
+        case QLORA_ERR_WORKSPACE: return "workspace missing or smaller than qlora_workspace_bytes()";
+        case QLORA_ERR_DEVICE: return "current CUDA device is not compute capability 10.0 (B200)";
+        case QLORA_ERR_LAUNCH: return "CUDA launch or runtime call failed";
+        case QLORA_ERR_TIMEOUT: return "a device-side bounded wait gave up";
+        case QLORA_ERR_VALUE: return "a scalar argument is not finite";
+        default: return "unknown status";
+    }
+}
+
+int qlora_device_status(int reset) {
+    if (cudaDeviceSynchronize() != cudaSuccess) return QLORA_ERR_LAUNCH;
+    int v = 0;
+    if (cudaMemcpyFromSymbol(&v, g_status, sizeof(int)) != cudaSuccess) return QLORA_ERR_LAUNCH;
+    if (reset) {
+        const int z = 0;
+        if (cudaMemcpyToSymbol(g_status, &z, sizeof(int)) != cudaSuccess) return QLORA_ERR_LAUNCH;
+    }
+    return v;
+}
+
+int qlora_last_path(void) { return t_last_path; }
+
+}  // extern "C"

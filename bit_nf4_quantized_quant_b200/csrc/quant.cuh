@@ -1,0 +1,174 @@
+// quant.cuh -- NF4 quantize + double-quantize and dense dequantize kernels.
+//
+// Both are HBM-bound streaming kernels (2 B read + 0.516 B written per weight,
+// and the reverse).  Layout of the quantized weight: see nf4dq_weight in
+// include/qlora_nf4.h.
+#pragma once
+#include "common.cuh"
+
+namespace qnf4 {
+
+// Nearest NF4 level of a normalised value x in [-1, 1]: the number of decision
+// thresholds that x lies strictly above, found by a 4-step binary search over
+// the sorted thresholds (the result equals the count exactly; a value on a
+// threshold takes the lower level).  Thresholds 3, 7 and 11 come from the
+// parameter bank, the last two steps index a 15-entry shared-memory copy
+// (16 distinct words in 16 banks: no bank conflicts).
+__device__ __forceinline__ uint32_t nf4_encode(float x, const NF4Tables& tab, const float* s_m) {
+    uint32_t q = (x > tab.m[7]) ? 8u : 0u;
+    float t = q ? tab.m[11] : tab.m[3];
+    q += (x > t) ? 4u : 0u;
+    q += (x > s_m[q + 1]) ? 2u : 0u;
+    q += (x > s_m[q]) ? 1u : 0u;
+    return q;
+}
+
+// One CTA (8 warps) per double-quant group of 256 blocks (16384 weights),
+// grid-stride over groups.  Warp w owns blocks [32w, 32w+32) of the group; a
+// block is handled by 8 lanes of 8 weights each (16-byte loads, coalesced
+// 512 B per warp instruction).  Warp 0 then runs the group's second-level
+// quantization with the fp64 pairwise tree held in registers: lane l keeps
+// slots l, l+32, ..., l+224, so strides 128, 64, 32 are in-register adds and
+// strides 16..1 are shuffles -- the same association order as the definition.
+__global__ void __launch_bounds__(256) k_quantize_dq(const uint16_t* __restrict__ W, int64_t nblocks,
+                                                     uint8_t* __restrict__ packed, int8_t* __restrict__ codes,
+                                                     float* __restrict__ scale, float* __restrict__ mean,
+                                                     NF4Tables tab) {
+    __shared__ float s_c[kGroup];
+    __shared__ float s_m[16];
+    if (threadIdx.x < 15) s_m[threadIdx.x] = tab.m[threadIdx.x];
+    if (threadIdx.x == 15) s_m[15] = INFINITY;
+    __syncthreads();
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int part = lane & 7, sub = lane >> 3;
+    const int64_t ngroups = cdiv(nblocks, kGroup);
+
+    for (int64_t g = blockIdx.x; g < ngroups; g += gridDim.x) {
+        const int64_t b0 = g * kGroup;
+        const int nb = (int)((nblocks - b0) < kGroup ? (nblocks - b0) : kGroup);
+
+        uint4 v[8];
+#pragma unroll
+        for (int it = 0; it < 8; ++it) {
+            const int bl = warp * 32 + it * 4 + sub;
+            if (bl < nb) v[it] = ldg_nc_v4(W + (b0 + bl) * kBlock + part * 8);
+            else v[it] = make_uint4(0, 0, 0, 0);
+        }
+#pragma unroll
+        for (int it = 0; it < 8; ++it) {
+            const int bl = warp * 32 + it * 4 + sub;
+            const uint32_t wv[4] = {v[it].x, v[it].y, v[it].z, v[it].w};
+            float w[8];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                w[2 * j] = bf16lo_to_f32(wv[j]);
+                w[2 * j + 1] = bf16hi_to_f32(wv[j]);
+            }
+            float c = 0.f;
+#pragma unroll
+            for (int j = 0; j < 8; ++j) c = fmaxf(c, fabsf(w[j]));
+            c = fmaxf(c, __shfl_xor_sync(0xffffffffu, c, 1));
+            c = fmaxf(c, __shfl_xor_sync(0xffffffffu, c, 2));
+            c = fmaxf(c, __shfl_xor_sync(0xffffffffu, c, 4));
+            if (bl < nb) {
+                uint32_t word = 0;
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    uint32_t q = 7u;
+                    if (c != 0.f) q = nf4_encode(__fdiv_rn(w[j], c), tab, s_m);
+                    // element 2i -> high nibble of byte i (little-endian word)
+                    word |= q << ((j >> 1) * 8 + ((j & 1) ? 0 : 4));
+                }
+                *reinterpret_cast<uint32_t*>(packed + ((b0 + bl) * kBlock + part * 8) / 2) = word;
+                if (part == 0) s_c[bl] = c;
+            }
+        }
+        __syncthreads();
+
+        if (warp == 0) {
+            double s[8];
+            float cv[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                const int idx = j * 32 + lane;
+                cv[j] = (idx < nb) ? s_c[idx] : 0.f;
+                s[j] = (double)cv[j];
+            }
+#pragma unroll
+            for (int j = 0; j < 4; ++j) s[j] = __dadd_rn(s[j], s[j + 4]);   // stride 128
+#pragma unroll
+            for (int j = 0; j < 2; ++j) s[j] = __dadd_rn(s[j], s[j + 2]);   // stride 64
+            double acc = __dadd_rn(s[0], s[1]);                              // stride 32
+#pragma unroll
+            for (int off = 16; off >= 1; off >>= 1)                          // strides 16..1
+                acc = __dadd_rn(acc, __shfl_down_sync(0xffffffffu, acc, off));
+            acc = __shfl_sync(0xffffffffu, acc, 0);
+            const float mu = __double2float_rn(__ddiv_rn(acc, (double)nb));
+            float d[8], dmax = 0.f;
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                d[j] = __fsub_rn(cv[j], mu);
+                if (j * 32 + lane < nb) dmax = fmaxf(dmax, fabsf(d[j]));
+            }
+#pragma unroll
+            for (int off = 16; off >= 1; off >>= 1) dmax = fmaxf(dmax, __shfl_xor_sync(0xffffffffu, dmax, off));
+            const float sc = __fdiv_rn(dmax, 127.0f);
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                const int idx = j * 32 + lane;
+                if (idx < nb) {
+                    int code = 0;
+                    if (sc != 0.f) {
+                        float t = rintf(__fdiv_rn(d[j], sc));
+                        t = fminf(fmaxf(t, -127.f), 127.f);
+                        code = (int)t;
+                    }
+                    codes[b0 + idx] = (int8_t)code;
+                }
+            }
+            if (lane == 0) {
+                scale[g] = sc;
+                mean[g] = mu;
+            }
+        }
+        __syncthreads();
+    }
+}
+
+// Dense dequantization: one thread per 16 packed bytes (32 weights = half a
+// block), grid-stride.  W' = bf16_rne(L[q] * c'_b), c'_b = fmaf(code, scale, mean).
+__global__ void __launch_bounds__(256) k_dequant(const uint8_t* __restrict__ packed,
+                                                 const int8_t* __restrict__ codes,
+                                                 const float* __restrict__ scale, const float* __restrict__ mean,
+                                                 int64_t nchunks, uint16_t* __restrict__ out, NF4Tables tab) {
+    __shared__ float s_L[16];
+    if (threadIdx.x < 16) s_L[threadIdx.x] = tab.L[threadIdx.x];
+    __syncthreads();
+    for (int64_t ch = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; ch < nchunks;
+         ch += (int64_t)gridDim.x * blockDim.x) {
+        const uint4 p = ldg_nc_v4(packed + ch * 16);
+        const int64_t b = ch >> 1;
+        const int64_t g = b / kGroup;
+        const float cp = __fmaf_rn((float)codes[b], __ldg(scale + g), __ldg(mean + g));
+        const uint32_t pw[4] = {p.x, p.y, p.z, p.w};
+        uint32_t o[16];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const uint32_t byte = (pw[j] >> (8 * k)) & 0xffu;
+                const float hi = __fmul_rn(s_L[byte >> 4], cp);     // element 2i
+                const float lo = __fmul_rn(s_L[byte & 15u], cp);    // element 2i+1
+                o[j * 4 + k] = pack_bf16x2(hi, lo);
+            }
+        }
+        uint4* dst = reinterpret_cast<uint4*>(out + ch * 32);
+        dst[0] = make_uint4(o[0], o[1], o[2], o[3]);
+        dst[1] = make_uint4(o[4], o[5], o[6], o[7]);
+        dst[2] = make_uint4(o[8], o[9], o[10], o[11]);
+        dst[3] = make_uint4(o[12], o[13], o[14], o[15]);
+    }
+}
+
+}  // namespace qnf4

@@ -1,0 +1,175 @@
+/*
+ * qlora_nf4.h -- C ABI of libqlora_nf4.so: the QLoRA frozen-NF4 linear layer
+ * on NVIDIA B200 (sm_100a).
+ *
+ * The layer (page citations give the page title and section):
+ *   - The frozen base weight W [N, K] (PyTorch Linear layout, out x in) is
+ *     stored as 4-bit NormalFloat: 16 levels at N(0,1) quantiles normalised
+ *     to [-1, 1] ("QLoRA Guide", NF4 vs uniform INT4; "Qlora Expert", Core
+ *     Concept), one absmax constant per block of 64 consecutive weights
+ *     ("QLoRA Implementation Details (2025 Edition)", Step 1, NF4 Math), and
+ *     the block constants themselves quantized to 8 bit ("QLoRA: The 4-bit
+ *     Revolution", 2. Double Quantization), here as int8 codes with an fp32
+ *     scale and mean per group of 256 block constants.
+ *   - Every forward and backward dequantizes to bf16 on the fly inside the
+ *     matrix product; the bf16 copy is never stored ("QLORA: Efficient
+ *     Finetuning of Quantized LLMs", Notes).
+ *   - A bf16 LoRA branch is added: Y = X W'^T + s (X A^T) B^T with
+ *     s = alpha / r ("QLoRA Guide", Forward pass; "QLoRA Implementation
+ *     Details (2025 Edition)", Step 4).  Only A and B receive gradients
+ *     ("QLoRA Guide", Forward pass: the dequantized W is a constant for
+ *     autograd), so the backward returns dX, dA and dB and never dW.
+ *
+ * Conventions for every entry point:
+ *   - bf16 values are passed as raw 16-bit patterns (qlora_bf16).
+ *   - Every tensor is dense row-major.  Pointers marked "device" must be
+ *     device (or managed) memory of the current CUDA device; the caller owns
+ *     all memory, the library never allocates or frees and holds no state
+ *     except a per-process copy of the codebook it computes on first use.
+ *   - Work is enqueued on `stream` (NULL = the legacy default stream) and
+ *     the call returns without synchronizing.  Results are valid once the
+ *     stream reaches that point.
+ *   - The return value is QLORA_OK (0) or a negative QLORA_ERR_* code.  All
+ *     argument checks run before anything is launched; a rejected call
+ *     launches nothing and writes nothing.  No C++ exception crosses the ABI.
+ *   - Weights and activations must be finite.
+ *   - Device-side waits are bounded: a kernel that gives up sets a sticky
+ *     status word read by qlora_device_status() instead of hanging.
+ */
+#ifndef QLORA_NF4_H
+#define QLORA_NF4_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define QLORA_API __attribute__((visibility("default")))
+#else
+#define QLORA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef uint16_t qlora_bf16;            /* raw bf16 bit pattern */
+typedef struct CUstream_st* qlora_stream_t;   /* a cudaStream_t */
+
+#define QLORA_NF4_BLOCK 64              /* weights per absmax block */
+#define QLORA_DQ_GROUP 256              /* block constants per double-quant group */
+#define QLORA_MAX_RANK 256              /* largest LoRA rank accepted */
+
+enum {
+    QLORA_OK = 0,
+    QLORA_ERR_NULL = -1,        /* a required pointer is NULL */
+    QLORA_ERR_SHAPE = -2,       /* M, N or K <= 0, K % 64 != 0, or a size overflows */
+    QLORA_ERR_RANK = -3,        /* r outside [1, QLORA_MAX_RANK] */
+    QLORA_ERR_ALIGN = -4,       /* a pointer is not 16-byte aligned */
+    QLORA_ERR_WORKSPACE = -5,   /* workspace NULL or smaller than qlora_workspace_bytes() */
+    QLORA_ERR_DEVICE = -6,      /* current device is not compute capability 10.0 */
+    QLORA_ERR_LAUNCH = -7,      /* a CUDA launch or runtime call failed */
+    QLORA_ERR_TIMEOUT = -8,     /* a device-side bounded wait gave up (see qlora_device_status) */
+    QLORA_ERR_VALUE = -9        /* a scalar argument is not finite */
+};
+
+/* Quantized weight: all device pointers, caller-owned.
+ *   packed [N, K/2] uint8: byte j of row n holds element 2j in its high
+ *                          nibble and element 2j+1 in its low nibble; a
+ *                          nibble is the index of an NF4 level (0..15).
+ *   codes  [N*K/64] int8 : code of block b = flat weights [64b, 64b+64)
+ *   scale  [G] fp32, mean [G] fp32, G = ceil(N*K/64 / 256): group g covers
+ *                          blocks [256g, 256g+256) of the flattened weight.
+ *   The constant of block b is c'_b = fmaf((float)codes[b], scale[b/256],
+ *   mean[b/256]) and the dequantized weight is bf16_rne(L[nibble] * c'_b). */
+typedef struct {
+    const uint8_t* packed;
+    const int8_t* codes;
+    const float* scale;
+    const float* mean;
+    int64_t N;
+    int64_t K;
+} nf4dq_weight;
+
+/* The 16 NF4 levels in fp32, ascending (out16[0] = -1, out16[7] = 0,
+ * out16[15] = +1): 8 positive normal quantiles at the first 8 of 9 evenly
+ * spaced probabilities from delta = ((1-1/32)+(1-1/30))/2 down to 1/2, 7
+ * negative ones at the first 7 of 8, and an exact zero, divided by the
+ * largest (the pages give only "levels at N(0,1) quantiles"; this is the
+ * construction of the QLoRA paper they cite).  Host memory; no GPU needed. */
+QLORA_API int nf4_codebook(float out16[16]);
+
+/* Element counts of a quantized [N, K] weight (host only, no GPU needed).
+ * Any output pointer may be NULL. */
+QLORA_API int nf4dq_sizes(int64_t N, int64_t K, int64_t* packed_bytes, int64_t* n_blocks, int64_t* n_groups);
+
+/* Quantize a bf16 weight W [N, K] (device) to NF4 with double-quantized
+ * constants ("Qlora Expert", Core Concept 1-2; "QLoRA Implementation
+ * Details (2025 Edition)", Step 1).  Per block: c_b = max |w|; each weight
+ * goes to the level nearest w / c_b (IEEE fp32 division; exactly halfway
+ * goes to the lower level; c_b = 0 gives the zero level 7).  Per group:
+ * mean_g = fl32(S / n_g) with S the fp64 pairwise sum (stride 128..1) of
+ * the group's constants, scale_g = fl32(max |c_b - mean_g| / 127),
+ * code_b = clamp(rint((c_b - mean_g) / scale_g), -127, 127) (0 when
+ * scale_g = 0).  Outputs (device, caller-allocated, sizes from
+ * nf4dq_sizes): packed, codes, scale, mean.  W and packed must be 16-byte
+ * aligned.  Requires K % 64 == 0. */
+QLORA_API int nf4_quantize_dq(const qlora_bf16* W, int64_t N, int64_t K, uint8_t* packed, int8_t* codes,
+                    float* scale, float* mean, qlora_stream_t stream);
+
+/* Dequantize to a dense bf16 W' [N, K] (device, 16-byte aligned)
+ * ("QLORA: Efficient Finetuning of Quantized LLMs", Notes: dequantize to
+ * BF16).  Bit-exact with the definition under nf4dq_weight. */
+QLORA_API int nf4_dequant(const nf4dq_weight* w, qlora_bf16* W_out, qlora_stream_t stream);
+
+/* Bytes of device workspace that qlora_linear_fwd / qlora_linear_bwd need
+ * for these sizes (0 is never returned for valid sizes; returns 0 for
+ * invalid ones).  The same workspace may be reused by calls that run one
+ * after another on one stream; calls that overlap on the GPU need separate
+ * workspaces. */
+QLORA_API size_t qlora_workspace_bytes(int64_t M, int64_t N, int64_t K, int r);
+
+/* Forward ("QLoRA Guide", Forward pass / Dequant + LoRA path):
+ *   T = X A^T            [M, r]  (fp32 accumulation)
+ *   Y = X W'^T + s T B^T [M, N]  (fp32 accumulation, one bf16 rounding)
+ * X [M, K] bf16, A [r, K] bf16, B [N, r] bf16, Y [M, N] bf16 (all device).
+ * T_out [M, r] bf16 may be NULL; when given it receives bf16(T) for reuse
+ * by the backward.  s = scaling (alpha / r).  ws: device workspace of at
+ * least qlora_workspace_bytes(M, N, K, r) bytes, 256-byte aligned.
+ * X, Y must be 16-byte aligned. */
+QLORA_API int qlora_linear_fwd(const qlora_bf16* X, int64_t M, const nf4dq_weight* w, const qlora_bf16* A,
+                     const qlora_bf16* B, int r, float scaling, qlora_bf16* Y, qlora_bf16* T_out,
+                     void* ws, size_t ws_bytes, qlora_stream_t stream);
+
+/* Backward of <Y, dY> ("QLoRA Guide", Forward pass: only A and B receive
+ * gradients; "QLORA: Efficient Finetuning of Quantized LLMs", Notes):
+ *   U  = dY B                    [M, r]
+ *   dX = dY W' + s U A           [M, K]
+ *   dA = s U^T X                 [r, K]
+ *   dB = s dY^T T, T = X A^T     [N, r]
+ * No gradient is computed for the frozen base weight.  T may be NULL (it is
+ * then recomputed from X and A) or the bf16 T_out of the forward.
+ * dX, dA, dB: device bf16 outputs (fp32 accumulation).  Same alignment and
+ * workspace rules as qlora_linear_fwd. */
+QLORA_API int qlora_linear_bwd(const qlora_bf16* X, const qlora_bf16* dY, int64_t M, const nf4dq_weight* w,
+                     const qlora_bf16* A, const qlora_bf16* B, int r, float scaling, const qlora_bf16* T,
+                     qlora_bf16* dX, qlora_bf16* dA, qlora_bf16* dB, void* ws, size_t ws_bytes,
+                     qlora_stream_t stream);
+
+/* Human-readable text for a status code (static storage). */
+QLORA_API const char* qlora_status_string(int status);
+
+/* Sticky device status of the current device: QLORA_OK, or QLORA_ERR_TIMEOUT
+ * if a kernel's bounded wait gave up since the last reset.  Synchronizes the
+ * current device.  reset != 0 clears it afterwards. */
+QLORA_API int qlora_device_status(int reset);
+
+/* Which kernel family the last successful fwd/bwd call on this thread
+ * dispatched to (for tests and benchmarks): 1 = small-M split-K tensor-core
+ * GEMV path, 2 = tcgen05 fused dequant-GEMM path. */
+QLORA_API int qlora_last_path(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* QLORA_NF4_H */

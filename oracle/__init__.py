@@ -230,3 +230,12 @@ def linear_bwd(X, dY, Wd, A, B, s):
     dA = s * (U.T @ X)
     dB = s * (dY.T @ T)
     return dX, dA, dB
+
+
+def linear_bwd_adapters(X, dY, A, B, s):
+    """The adapter gradients alone (dA, dB) of linear_bwd, without dX."""
+    X = np.asarray(X, np.float64)
+    dY = np.asarray(dY, np.float64)
+    T = X @ np.asarray(A, np.float64).T
+    U = dY @ np.asarray(B, np.float64)
+    return s * (U.T @ X), s * (dY.T @ T)

@@ -1,0 +1,145 @@
+"""GPU parity of qlora_linear_fwd / qlora_linear_bwd against the fp64 oracle.
+
+Tolerance |err| <= 1e-2 * max(1, |ref|) per element.  The weight the GPU
+multiplies with is first checked to be the oracle's bit for bit (see
+test_gpu_quant.py), so the oracle's W' is the exact operand.
+"""
+import numpy as np
+import pytest
+import torch
+
+from bit_nf4_quantized_quant_b200 import inputs
+from bit_nf4_quantized_quant_b200 import _ops as ops
+
+pytestmark = pytest.mark.gpu
+
+TOL = 1e-2
+
+
+def _close(got, ref, what):
+    got = np.asarray(got, np.float64)
+    ref = np.asarray(ref, np.float64)
+    assert got.shape == ref.shape, (what, got.shape, ref.shape)
+    err = np.abs(got - ref)
+    lim = TOL * np.maximum(1.0, np.abs(ref))
+    bad = err > lim
+    assert not bad.any(), (f"{what}: {bad.sum()} of {bad.size} outside tolerance; worst err "
+                           f"{err.max():.4g} at {np.unravel_index(np.argmax(err - lim), err.shape)}")
+
+
+def _setup(oracle_mod, M, N, K, r, seed, w_std=0.02, x_std=1.0):
+    W = inputs.weight(50 + seed, 0, N, K, w_std)
+    X = inputs.normal(60 + seed, (M, K), x_std)
+    A = inputs.uniform(61 + seed, (r, K), 1.0 / np.sqrt(K))
+    B = inputs.normal(62 + seed, (N, r), 0.01 * 10)    # larger than the workloads' so the LoRA term matters
+    dY = inputs.normal(63 + seed, (M, N), 1.0)
+    q = oracle_mod.quantize_dq(inputs.bf16_bits(W))
+    Wd = oracle_mod.bf16_to_f32(oracle_mod.dequant(q)).astype(np.float64)
+    w = ops.nf4_quantize_dq(W.cuda())
+    assert np.array_equal(w.packed.cpu().numpy(), q["packed"])
+    return W, X, A, B, dY, Wd, w
+
+
+CASES = [
+    # M, N, K, r
+    (1, 64, 64, 16),
+    (3, 136, 192, 4),
+    (8, 256, 1024, 16),
+    (16, 512, 512, 64),
+    (17, 200, 320, 24),
+    (32, 1024, 1024, 16),
+    (33, 128, 256, 16),
+    (100, 264, 640, 8),
+    (257, 384, 448, 64),
+    (5, 4096, 4096, 16),
+]
+
+
+@pytest.mark.parametrize("M,N,K,r", CASES)
+def test_fwd_bwd_parity(oracle_mod, M, N, K, r):
+    s = 32.0 / r
+    W, X, A, B, dY, Wd, w = _setup(oracle_mod, M, N, K, r, seed=M + N + K + r)
+    Xc, Ac, Bc, dYc = X.cuda(), A.cuda(), B.cuda(), dY.cuda()
+    T_out = torch.empty((M, r), dtype=torch.bfloat16, device="cuda")
+    Y = ops.qlora_linear_fwd(Xc, w, Ac, Bc, s, T_out=T_out)
+    dX, dA, dB = ops.qlora_linear_bwd(Xc, dYc, w, Ac, Bc, s)
+    dX2, dA2, dB2 = ops.qlora_linear_bwd(Xc, dYc, w, Ac, Bc, s, T=T_out)
+    torch.cuda.synchronize()
+    assert ops.qlora_device_status() == 0
+    X64, A64, B64, dY64 = (inputs.to_f64(t) for t in (X, A, B, dY))
+    Yr, Tr = oracle_mod.linear_fwd(X64, Wd, A64, B64, s)
+    dXr, dAr, dBr = oracle_mod.linear_bwd(X64, dY64, Wd, A64, B64, s)
+    _close(inputs.to_f64(Y), Yr, "Y")
+    _close(inputs.to_f64(T_out), Tr, "T")
+    _close(inputs.to_f64(dX), dXr, "dX")
+    _close(inputs.to_f64(dA), dAr, "dA")
+    _close(inputs.to_f64(dB), dBr, "dB")
+    _close(inputs.to_f64(dX2), dXr, "dX (T given)")
+    _close(inputs.to_f64(dA2), dAr, "dA (T given)")
+    _close(inputs.to_f64(dB2), dBr, "dB (T given)")
+
+
+def test_zero_B_is_plain_dequant_matmul(oracle_mod):
+    M, N, K, r = 24, 512, 1024, 16
+    W, X, A, B, dY, Wd, w = _setup(oracle_mod, M, N, K, r, seed=3)
+    Bz = torch.zeros_like(B)
+    Y = ops.qlora_linear_fwd(X.cuda(), w, A.cuda(), Bz.cuda(), 2.0)
+    Wdq = ops.nf4_dequant(w)
+    ref = (X.cuda().float() @ Wdq.float().T)
+    torch.cuda.synchronize()
+    _close(inputs.to_f64(Y), ref.double().cpu().numpy(), "Y vs torch.matmul on nf4_dequant")
+
+
+def test_repeatable(oracle_mod):
+    M, N, K, r = 16, 1024, 2048, 16
+    W, X, A, B, dY, Wd, w = _setup(oracle_mod, M, N, K, r, seed=4)
+    outs = []
+    for _ in range(2):
+        Y = ops.qlora_linear_fwd(X.cuda(), w, A.cuda(), B.cuda(), 2.0)
+        dX, dA, dB = ops.qlora_linear_bwd(X.cuda(), dY.cuda(), w, A.cuda(), B.cuda(), 2.0)
+        outs.append([t.cpu() for t in (Y, dX, dA, dB)])
+    for a, b in zip(*outs):
+        assert torch.equal(a, b)        # fixed reduction orders: bit-identical reruns
+
+
+def _sampled_rows_parity(oracle_mod, wl, proj, M, rows_n=16, bwd=True):
+    p = wl.projections[proj]
+    s = wl.scaling
+    W = inputs.layer_weight(wl, proj, device="cuda")
+    X, A, B, dY = inputs.layer_inputs(wl, proj, M, device="cuda", with_dy=bwd)
+    w = ops.nf4_quantize_dq(W)
+    Y = ops.qlora_linear_fwd(X, w, A, B, s)
+    if bwd:
+        dX, dA, dB = ops.qlora_linear_bwd(X, dY, w, A, B, s)
+    torch.cuda.synchronize()
+    assert ops.qlora_device_status() == 0
+    rng = np.random.default_rng(1000 * wl.index + proj + M)
+    rows_m = np.unique(np.concatenate([rng.choice(M, size=min(rows_n, M), replace=False), [0, M - 1]]))
+    # oracle weight rows (output features) and columns needed
+    Wbits = inputs.bf16_bits(W)
+    X64 = inputs.to_f64(X)
+    A64, B64 = inputs.to_f64(A), inputs.to_f64(B)
+    # Y rows: need the whole W'
+    q_full = oracle_mod.quantize_dq(Wbits)
+    Wd = oracle_mod.bf16_to_f32(oracle_mod.dequant(q_full)).astype(np.float64)
+    assert np.array_equal(w.packed.cpu().numpy(), q_full["packed"])
+    Yr, _ = oracle_mod.linear_fwd(X64[rows_m], Wd, A64, B64, s)
+    _close(inputs.to_f64(Y)[rows_m], Yr, "Y rows")
+    if bwd:
+        dY64 = inputs.to_f64(dY)
+        dXr, _, _ = oracle_mod.linear_bwd(X64[rows_m], dY64[rows_m], Wd, A64, B64, s)
+        _close(inputs.to_f64(dX)[rows_m], dXr, "dX rows")
+        # dA, dB need every row: computed in full by the oracle
+        dAr, dBr = oracle_mod.linear_bwd_adapters(X64, dY64, A64, B64, s)
+        _close(inputs.to_f64(dA), dAr, "dA")
+        _close(inputs.to_f64(dB), dBr, "dB")
+
+
+@pytest.mark.parametrize("proj", [0])
+def test_workload1_full(oracle_mod, proj):
+    _sampled_rows_parity(oracle_mod, inputs.WORKLOADS[1], proj, 16, rows_n=16)
+
+
+@pytest.mark.parametrize("proj,M", [(0, 1), (0, 4), (1, 8), (1, 32)])
+def test_workload2_decode(oracle_mod, proj, M):
+    _sampled_rows_parity(oracle_mod, inputs.WORKLOADS[2], proj, M, rows_n=M, bwd=False)

@@ -105,3 +105,10 @@ def test_linearity_and_scaling(oracle_mod):
     Y0, _ = oracle_mod.linear_fwd(X, Wd, A, B, 0.0)
     Y4, _ = oracle_mod.linear_fwd(X, Wd, A, B, 4.0)
     assert np.allclose(Y4 - Y0, 2 * (Y1 - Y0), atol=1e-12)
+
+
+def test_adapter_only_backward_matches_full(oracle_mod):
+    X, Wd, A, B, dY = _case(oracle_mod, M=6, N=9, K=128, r=3, seed=12)
+    _, dA, dB = oracle_mod.linear_bwd(X, dY, Wd, A, B, 0.5)
+    dA2, dB2 = oracle_mod.linear_bwd_adapters(X, dY, A, B, 0.5)
+    assert np.array_equal(dA, dA2) and np.array_equal(dB, dB2)
