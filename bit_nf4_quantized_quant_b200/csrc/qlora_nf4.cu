@@ -85,8 +85,6 @@ int check_device(int* sm_count) {
                                                      fwd_small_smem_bytes<1>());
                 if (r == cudaSuccess) r = cudaFuncSetAttribute(k_fwd_small<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                                                fwd_small_smem_bytes<2>());
-                if (r == cudaSuccess) r = cudaFuncSetAttribute(k_fwd_small<4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                               fwd_small_smem_bytes<4>());
                 if (r == cudaSuccess) r = cudaFuncSetAttribute(k_bwd_small<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                                                bwd_small_smem_bytes<1>());
                 if (r == cudaSuccess) r = cudaFuncSetAttribute(k_bwd_small<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -172,12 +170,12 @@ Plan make_plan(int64_t M, int64_t N, int64_t K, int r, int sms) {
     p.zB = choose_splits(cdiv(N, 64) * cdiv(p.rp, bj), M, target);
     p.kB = rup(cdiv(M, p.zB), 32);
     p.zB = (int)cdiv(M, p.kB);
-    // small-path dX: units = ceil(K/64/4) * S
+    // small-path dX: units = (K/64) * S, rows per split a multiple of 256
     {
-        const int64_t nkg = cdiv(K / kBlock, kBwdKW);
-        int64_t S = cdiv(target, nkg);
-        int64_t rps = rup(cdiv(N, S < 1 ? 1 : S), 64);
-        if (rps < 64) rps = 64;
+        const int64_t nblk = K / kBlock;
+        int64_t S = cdiv(target, nblk);
+        if (S < 1) S = 1;
+        int64_t rps = rup(cdiv(N, S), kBwdChunk);
         p.rows_per_split = rps;
         p.S_bwd = (int)cdiv(N, rps);
     }
@@ -187,8 +185,7 @@ Plan make_plan(int64_t M, int64_t N, int64_t K, int r, int sms) {
     upd(gemm_part_bytes(M, p.rp, p.zU));
     upd(gemm_part_bytes(p.rp, K, p.zA));
     upd(gemm_part_bytes(N, p.rp, p.zB));
-    if (M <= 32) upd((size_t)p.S_bwd * M * K * 4);
-    else upd((size_t)p.S_bwd * 32 * K * 4);   // large M processes 32-token chunks
+    upd((size_t)p.S_bwd * (M < 32 ? M : 32) * K * 4);   // small-path dX partials, 32-token chunks
     size_t off = 0;
     auto take = [&](size_t b) { const size_t o = off; off = align256(off + b); return o; };
     p.off_part = take(part);
@@ -356,13 +353,8 @@ int qlora_linear_fwd(const qlora_bf16* X, int64_t M, const nf4dq_weight* w, cons
     a.M = M; a.N = w->N; a.K = w->K; a.rp = p.rp; a.r = r; a.s = scaling;
     const int64_t ntiles = cdiv(w->N, 16);
     const int grid = (int)(ntiles < 2LL * sms ? ntiles : 2LL * sms);
-    if (M <= 8) {
-        k_fwd_small<1><<<grid, kSmallThreads, fwd_small_smem_bytes<1>(), st>>>(a, tables());
-    } else if (M <= 16) {
-        k_fwd_small<2><<<grid, kSmallThreads, fwd_small_smem_bytes<2>(), st>>>(a, tables());
-    } else {
-        k_fwd_small<4><<<grid, kSmallThreads, fwd_small_smem_bytes<4>(), st>>>(a, tables());
-    }
+    if (M <= 16) k_fwd_small<1><<<grid, kSmallThreads, fwd_small_smem_bytes<1>(), st>>>(a, tables());
+    else k_fwd_small<2><<<grid, kSmallThreads, fwd_small_smem_bytes<2>(), st>>>(a, tables());
     rc = launch_status();
     if (rc == QLORA_OK) t_last_path = 1;
     return rc;
@@ -436,24 +428,21 @@ int qlora_linear_bwd(const qlora_bf16* X, const qlora_bf16* dY, int64_t M, const
         rc = run_gemm<false, false>(Ubf, p.rp, X, K, p.rp, K, M, p.rp, K, p.zA, p.kA, part, f, sms, st);
         if (rc != QLORA_OK) return rc;
     }
-    // dX = dY W' + s U A
-    {
-        const int64_t MC = 16;
-        for (int64_t m0 = 0; m0 < M; m0 += (M <= 16 ? M : MC)) {
-            const int64_t mc = (M <= 16) ? M : (M - m0 < MC ? M - m0 : MC);
-            SmallBwdArgs a{};
-            a.dY = dY + m0 * N; a.packed = w->packed; a.codes = w->codes; a.scale = w->scale; a.mean = w->mean;
-            a.part = part; a.M = mc; a.N = N; a.K = K; a.rows_per_split = p.rows_per_split; a.S = p.S_bwd;
-            const int64_t units = cdiv(K / kBlock, kBwdKW) * p.S_bwd;
-            const int grid = (int)(units < 2LL * sms ? units : 2LL * sms);
-            if (mc <= 8) k_bwd_small<1><<<grid, kSmallThreads, bwd_small_smem_bytes<1>(), st>>>(a, tables());
-            else k_bwd_small<2><<<grid, kSmallThreads, bwd_small_smem_bytes<2>(), st>>>(a, tables());
-            k_bwd_small_finish<<<grid_for(mc * K, 256, sms), 256, 0, st>>>(
-                part, p.S_bwd, mc, K, reinterpret_cast<const float*>(wsb + p.off_U32) + m0 * p.rp, p.rp, A, r,
-                scaling, dX + m0 * K);
-            rc = launch_status();
-            if (rc != QLORA_OK) return rc;
-        }
+    // dX = dY W' + s U A, 32 tokens per pass
+    for (int64_t m0 = 0; m0 < M; m0 += 32) {
+        const int64_t mc = (M - m0 < 32) ? M - m0 : 32;
+        SmallBwdArgs a{};
+        a.dY = dY + m0 * N; a.packed = w->packed; a.codes = w->codes; a.scale = w->scale; a.mean = w->mean;
+        a.part = part; a.M = mc; a.N = N; a.K = K; a.rows_per_split = p.rows_per_split; a.S = p.S_bwd;
+        const int64_t units = (K / kBlock) * p.S_bwd;
+        const int grid = (int)(units < 2LL * sms ? units : 2LL * sms);
+        if (mc <= 16) k_bwd_small<1><<<grid, kBwdThreads, bwd_small_smem_bytes<1>(), st>>>(a, tables());
+        else k_bwd_small<2><<<grid, kBwdThreads, bwd_small_smem_bytes<2>(), st>>>(a, tables());
+        k_bwd_small_finish<<<grid_for(mc * K, 256, sms), 256, 0, st>>>(
+            part, p.S_bwd, mc, K, reinterpret_cast<const float*>(wsb + p.off_U32) + m0 * p.rp, p.rp, A, r, scaling,
+            dX + m0 * K);
+        rc = launch_status();
+        if (rc != QLORA_OK) return rc;
     }
     t_last_path = 1;
     return QLORA_OK;

@@ -1,45 +1,32 @@
 // small.cuh -- small-M (decode / GEMV-shaped) forward and backward-dX kernels.
 //
 // For a few tokens the layer is bound by streaming the 4.13-bit weight from
-// HBM, so the kernels are built around the cost of turning nibbles into bf16
-// MMA operands:
-//   * a shared-memory "pair table" maps a packed byte (two nibbles) straight to
-//     a bf16x2 register holding the two *unscaled* NF4 levels; it is replicated
-//     once per lane (entry v of lane l at word 32 v + l), so a warp-wide lookup
-//     never has a bank conflict;
-//   * the per-block constant c'_b is folded out of the inner product: each
-//     64-wide block is reduced on the tensor cores (mma.sync m16n8k16, fp32)
-//     into a fresh accumulator that is then added with one FMA per output,
-//     y += c'_b * sum_{k in b} L[q_k] x_k   (forward), or applied to the other
-//     operand (backward: dY[m, n] * c'_{n, b} rounded to bf16).
-// The k order inside one m16n8k16 MMA is permuted so that each lane's
-// fragment comes from contiguous packed bytes; the activation fragment is
-// loaded with the same permutation, so the sum is unchanged.
+// HBM, and the work per weight is the exact dequantization itself (see
+// nf4_decode.cuh: one 16-entry table per 64-weight block, byte-permute
+// lookups).  Both kernels let one thread own one row-block (64 consecutive
+// weights of a row), so the table is built once per 64 weights.
+//
+// Forward: Y^T = W' X^T on mma.sync m16n8k16 with the tokens as the MMA rows
+// and W' as the B operand.  The B fragment of lane (g, t) is two pairs of one
+// row (g) of W, so lane (g, t) can own row n0+g, block 4*ms + t, and feed the
+// 16 MMAs of a macro-step (4 blocks, 256 k) straight from registers: in MMA s
+// its logical k {2t, 2t+1} are elements 4s, 4s+1 of its block and {2t+8,
+// 2t+9} are 4s+2, 4s+3.  The activation fragment is loaded with the same k
+// permutation.  No shared memory is touched by the weights.
+//
+// Backward: dX = dY W' reduces over the rows of W, so the MMA B operand needs
+// pairs along n; each thread dequantizes its row-block into a swizzled
+// shared-memory tile and the MMA warps read it with ldmatrix.trans.
 #pragma once
 #include "common.cuh"
+#include "nf4_decode.cuh"
 
 namespace qnf4 {
 
-constexpr int kPairTableWords = 256 * 32;
 constexpr int kSmallThreads = 512;
 constexpr int kSmallWarps = kSmallThreads / 32;
-
-__device__ __forceinline__ void build_pair_table(uint32_t* s_tab, float* s_L, const NF4Tables& tab) {
-    if (threadIdx.x < 16) s_L[threadIdx.x] = tab.L[threadIdx.x];
-    __syncthreads();
-    for (int i = threadIdx.x; i < kPairTableWords; i += blockDim.x) {
-        const int v = i >> 5;
-        s_tab[i] = pack_bf16x2(s_L[v >> 4], s_L[v & 15]);
-    }
-    __syncthreads();
-}
-
-// bf16x2 (L[hi nibble], L[lo nibble]) of byte `j` of `w`; lane_base = smem
-// address of this lane's column of the pair table.
-__device__ __forceinline__ uint32_t pair_lookup(uint32_t lane_base, uint32_t w, int j) {
-    const uint32_t v = prmt(w, 0u, 0x4440u + (uint32_t)j);
-    return lds_u32(lane_base + v * 128u);
-}
+constexpr int kFwdRowGroups = 2;                          // 8-row groups per CTA
+constexpr int kFwdKSplits = kSmallWarps / kFwdRowGroups;  // warps sharing a row group
 
 __device__ __forceinline__ float block_constant(const int8_t* codes, const float* scale, const float* mean,
                                                 int64_t b) {
@@ -62,107 +49,104 @@ struct SmallFwdArgs {
 };
 
 template <int MT>
-constexpr int fwd_small_smem_bytes() { return kPairTableWords * 4 + kSmallWarps * 16 * (8 * MT + 4) * 4; }
+constexpr int fwd_small_smem_bytes() { return kFwdKSplits * 16 * (16 * MT + 1) * 4; }
 
-// Forward.  One CTA per 16-row tile of W (persistent, grid-stride over
-// tiles); its 16 warps split the K blocks.  Per warp and 64-wide block:
-//   lane (g, t) holds 8 packed bytes of rows g and g+8 (k in [16t, 16t+16)),
-//   MMA i uses bytes 2i, 2i+1: logical k {2t, 2t+1} <-> physical
-//   16t + 4i + {0, 1} and logical {2t+8, 2t+9} <-> 16t + 4i + {2, 3}.
-// Partial tiles are summed across warps in shared memory in a fixed order,
-// then s * T[m,:] . B[n,:] is added and Y is written once in bf16.
+// One CTA per 16-row tile (grid-stride).  Warp w: row group w % 2 (8 rows),
+// k-split w / 2 (every 8th macro-step).  Tokens in chunks of 16 * MT.
 template <int MT>
 __global__ void __launch_bounds__(kSmallThreads) k_fwd_small(SmallFwdArgs a, NF4Tables tab) {
-    constexpr int MC = 8 * MT;
-    constexpr int RS = MC + 4;                       // padded row stride of the reduction buffer
-    extern __shared__ __align__(16) uint8_t smem[];
-    uint32_t* s_tab = reinterpret_cast<uint32_t*>(smem);
-    float* s_red = reinterpret_cast<float*>(smem + kPairTableWords * 4);   // [warps][16][RS]
-    __shared__ float s_L[16];
-    build_pair_table(s_tab, s_L, tab);
+    constexpr int MC = 16 * MT;
+    constexpr int RS = MC + 1;
+    extern __shared__ __align__(1024) uint8_t smem[];
+    float* s_red = reinterpret_cast<float*>(smem);       // [ksplit][16 rows][RS]
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int g = lane >> 2, t = lane & 3;
-    const uint32_t lane_base = smem_u32(s_tab) + lane * 4;
+    const int rg = warp % kFwdRowGroups, ks = warp / kFwdRowGroups;
     const int64_t nblk = a.K / kBlock;
+    const int64_t nms = cdiv(nblk, 4);
     const int64_t ntiles = cdiv(a.N, 16);
     const int64_t rowbytes = a.K / 2;
 
     for (int64_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
         const int64_t n0 = tile * 16;
-        const int64_t row0 = min(n0 + g, a.N - 1), row1 = min(n0 + g + 8, a.N - 1);
-        const uint8_t* p0 = a.packed + row0 * rowbytes + 8 * t;
-        const uint8_t* p1 = a.packed + row1 * rowbytes + 8 * t;
+        const int64_t n = n0 + rg * 8 + g;
+        const bool nvalid = n < a.N;
         for (int64_t mc = 0; mc < a.M; mc += MC) {
             float acc[MT][4];
 #pragma unroll
-            for (int nt = 0; nt < MT; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
-            for (int64_t b = warp; b < nblk; b += kSmallWarps) {
-                const uint2 w0 = ldg_nc_v2(p0 + 32 * b);
-                const uint2 w1 = ldg_nc_v2(p1 + 32 * b);
-                uint32_t xf[MT][8];
-#pragma unroll
-                for (int nt = 0; nt < MT; ++nt) {
-                    const int64_t m = mc + nt * 8 + g;
-                    if (m < a.M) {
-                        const uint4* xp = reinterpret_cast<const uint4*>(a.X + m * a.K + 64 * b + 16 * t);
-                        const uint4 u0 = __ldg(xp), u1 = __ldg(xp + 1);
-                        xf[nt][0] = u0.x; xf[nt][1] = u0.y; xf[nt][2] = u0.z; xf[nt][3] = u0.w;
-                        xf[nt][4] = u1.x; xf[nt][5] = u1.y; xf[nt][6] = u1.z; xf[nt][7] = u1.w;
-                    } else {
-#pragma unroll
-                        for (int j = 0; j < 8; ++j) xf[nt][j] = 0u;
-                    }
+            for (int mt = 0; mt < MT; ++mt) acc[mt][0] = acc[mt][1] = acc[mt][2] = acc[mt][3] = 0.f;
+            for (int64_t ms = ks; ms < nms; ms += kFwdKSplits) {
+                const int64_t b = ms * 4 + t;
+                const bool valid = nvalid && b < nblk;
+                uint4 p0 = make_uint4(0, 0, 0, 0), p1 = p0;
+                float c = 0.f;
+                if (valid) {
+                    const uint8_t* pp = a.packed + n * rowbytes + 32 * b;
+                    p0 = ldg_nc_v4(pp);
+                    p1 = ldg_nc_v4(pp + 16);
+                    c = block_constant(a.codes, a.scale, a.mean, n * nblk + b);
                 }
-                const float c0 = block_constant(a.codes, a.scale, a.mean, row0 * nblk + b);
-                const float c1 = block_constant(a.codes, a.scale, a.mean, row1 * nblk + b);
-                float tmp[MT][4];
+                const BlockTable tb = make_block_table(tab, c);
+                const uint32_t pw[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
+                // 4 groups of 16 weights: group u feeds MMAs s = 4u .. 4u+3
 #pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const uint32_t u0 = (i < 2) ? w0.x : w0.y;
-                    const uint32_t u1 = (i < 2) ? w1.x : w1.y;
-                    const int j0 = (2 * i) & 3, j1 = (2 * i + 1) & 3;
-                    const uint32_t a0 = pair_lookup(lane_base, u0, j0);
-                    const uint32_t a1 = pair_lookup(lane_base, u1, j0);
-                    const uint32_t a2 = pair_lookup(lane_base, u0, j1);
-                    const uint32_t a3 = pair_lookup(lane_base, u1, j1);
+                for (int u = 0; u < 4; ++u) {
+                    uint32_t wa[4], wb[4];
+                    decode8(tb, pw[2 * u], wa);
+                    decode8(tb, pw[2 * u + 1], wb);
+                    const uint32_t wv[8] = {wa[0], wa[1], wa[2], wa[3], wb[0], wb[1], wb[2], wb[3]};
 #pragma unroll
-                    for (int nt = 0; nt < MT; ++nt) {
-                        if (i == 0) mma_bf16_16816_zero(tmp[nt], a0, a1, a2, a3, xf[nt][0], xf[nt][1]);
-                        else mma_bf16_16816(tmp[nt], a0, a1, a2, a3, xf[nt][2 * i], xf[nt][2 * i + 1]);
+                    for (int mt = 0; mt < MT; ++mt) {
+                        const int64_t m0 = mc + mt * 16 + g, m1 = m0 + 8;
+                        uint4 x00 = make_uint4(0, 0, 0, 0), x01 = x00, x10 = x00, x11 = x00;
+                        if (b < nblk) {
+                            if (m0 < a.M) {
+                                const uint4* xp = reinterpret_cast<const uint4*>(a.X + m0 * a.K + 64 * b + 16 * u);
+                                x00 = __ldg(xp);
+                                x01 = __ldg(xp + 1);
+                            }
+                            if (m1 < a.M) {
+                                const uint4* xp = reinterpret_cast<const uint4*>(a.X + m1 * a.K + 64 * b + 16 * u);
+                                x10 = __ldg(xp);
+                                x11 = __ldg(xp + 1);
+                            }
+                        }
+                        const uint32_t xa[8] = {x00.x, x00.y, x00.z, x00.w, x01.x, x01.y, x01.z, x01.w};
+                        const uint32_t xb[8] = {x10.x, x10.y, x10.z, x10.w, x11.x, x11.y, x11.z, x11.w};
+#pragma unroll
+                        for (int s4 = 0; s4 < 4; ++s4)
+                            mma_bf16_16816(acc[mt], xa[2 * s4], xb[2 * s4], xa[2 * s4 + 1], xb[2 * s4 + 1],
+                                           wv[2 * s4], wv[2 * s4 + 1]);
                     }
-                }
-#pragma unroll
-                for (int nt = 0; nt < MT; ++nt) {
-                    acc[nt][0] = __fmaf_rn(c0, tmp[nt][0], acc[nt][0]);
-                    acc[nt][1] = __fmaf_rn(c0, tmp[nt][1], acc[nt][1]);
-                    acc[nt][2] = __fmaf_rn(c1, tmp[nt][2], acc[nt][2]);
-                    acc[nt][3] = __fmaf_rn(c1, tmp[nt][3], acc[nt][3]);
                 }
             }
-            float* red = s_red + warp * 16 * RS;
+            // acc[mt]: c0,c1 -> (token mt*16+g, row 2t, 2t+1), c2,c3 -> (token +8)
+            float* red = s_red + ks * 16 * RS;
 #pragma unroll
-            for (int nt = 0; nt < MT; ++nt) {
-                red[g * RS + nt * 8 + 2 * t] = acc[nt][0];
-                red[g * RS + nt * 8 + 2 * t + 1] = acc[nt][1];
-                red[(g + 8) * RS + nt * 8 + 2 * t] = acc[nt][2];
-                red[(g + 8) * RS + nt * 8 + 2 * t + 1] = acc[nt][3];
+            for (int mt = 0; mt < MT; ++mt) {
+                const int r0 = rg * 8 + 2 * t;
+                red[r0 * RS + mt * 16 + g] = acc[mt][0];
+                red[(r0 + 1) * RS + mt * 16 + g] = acc[mt][1];
+                red[r0 * RS + mt * 16 + g + 8] = acc[mt][2];
+                red[(r0 + 1) * RS + mt * 16 + g + 8] = acc[mt][3];
             }
             __syncthreads();
             for (int idx = threadIdx.x; idx < 16 * MC; idx += blockDim.x) {
                 const int row = idx & 15, ml = idx >> 4;
-                const int64_t m = mc + ml, n = n0 + row;
-                if (m < a.M && n < a.N) {
+                const int64_t m = mc + ml, nn = n0 + row;
+                if (m < a.M && nn < a.N) {
                     float v = 0.f;
-                    for (int w = 0; w < kSmallWarps; ++w) v += s_red[w * 16 * RS + row * RS + ml];
+#pragma unroll
+                    for (int w = 0; w < kFwdKSplits; ++w) v += s_red[w * 16 * RS + row * RS + ml];
                     if (a.T32 != nullptr) {
                         const float* tr = a.T32 + m * a.rp;
-                        const uint16_t* br = a.B + n * a.r;
+                        const uint16_t* br = a.B + nn * a.r;
                         float l = 0.f;
                         for (int i = 0; i < a.r; ++i) l = __fmaf_rn(tr[i], bf16lo_to_f32(br[i]), l);
                         v = __fmaf_rn(a.s, l, v);
                     }
-                    a.Y[m * a.N + n] = (uint16_t)(pack_bf16x2(v, 0.f) & 0xffffu);
+                    a.Y[m * a.N + nn] = (uint16_t)(pack_bf16x2(v, 0.f) & 0xffffu);
                 }
             }
             __syncthreads();
@@ -178,122 +162,133 @@ struct SmallBwdArgs {
     const float* mean;
     float* part;              // [S][M][K] fp32 partial dY W' (no LoRA term)
     int64_t M, N, K;
-    int64_t rows_per_split;   // multiple of 64
+    int64_t rows_per_split;   // multiple of 256
     int S;
 };
 
-constexpr int kBwdKW = 4;     // k-blocks per CTA
-constexpr int kBwdNSUB = 4;   // n sub-ranges per CTA (kBwdKW * kBwdNSUB = 16 warps)
+constexpr int kBwdThreads = 256;
+constexpr int kBwdWarps = kBwdThreads / 32;
+constexpr int kBwdChunk = 256;        // W rows dequantized per pass (one per thread)
 
 template <int MT>
-constexpr int bwd_small_smem_bytes() { return kPairTableWords * 4 + kSmallWarps * 64 * (8 * MT + 4) * 4; }
+constexpr int bwd_small_smem_bytes() {
+    return kBwdChunk * 128 + kBwdWarps * 64 * (16 * MT + 1) * 4;
+}
 
-// Backward dX = dY W' without the LoRA term.  Work unit = (4 consecutive
-// 64-wide k-blocks, one split of the N rows); warp w takes k-block w % 4 and
-// every 4th 16-row step of the split.  Per step, lane (g, t) reads 4 packed
-// bytes (k in [8g, 8g+8) of its block) of rows n0 + {2t, 2t+1, 2t+8, 2t+9};
-// MMA j (0..3) maps logical row g <-> k = 8g + 2j, row g+8 <-> 8g + 2j + 1,
-// and logical reduction index {2t, 2t+1, 2t+8, 2t+9} <-> those rows.  The
-// pair lookups give (k even, k odd) of one row; two byte-permutes transpose
-// them into (row n, row n+1) operand pairs.  The per-(row, block) constant
-// multiplies dY before it is rounded to bf16.
+// Backward dX = dY W' (the LoRA term is added by k_bwd_small_finish).  Work
+// unit = (one 64-wide k-block kb, one split of the N rows).  Per pass of 256
+// rows: thread d dequantizes row nc + d, block kb into the swizzled tile
+// (16-byte chunk c of tile row r stored at chunk c ^ (r & 7)); then warp w
+// multiplies tile rows [32w, 32w+32): dY fragments from global memory, W'
+// fragments with ldmatrix.trans, 8 n8-tiles covering the 64 k of the block.
 template <int MT>
-__global__ void __launch_bounds__(kSmallThreads) k_bwd_small(SmallBwdArgs a, NF4Tables tab) {
-    constexpr int MC = 8 * MT;
-    constexpr int RS = MC + 4;
-    extern __shared__ __align__(16) uint8_t smem[];
-    uint32_t* s_tab = reinterpret_cast<uint32_t*>(smem);
-    float* s_red = reinterpret_cast<float*>(smem + kPairTableWords * 4);   // [warps][64][RS]
-    __shared__ float s_L[16];
-    build_pair_table(s_tab, s_L, tab);
+__global__ void __launch_bounds__(kBwdThreads) k_bwd_small(SmallBwdArgs a, NF4Tables tab) {
+    constexpr int MC = 16 * MT;
+    constexpr int RS = MC + 1;
+    extern __shared__ __align__(1024) uint8_t smem[];
+    uint8_t* s_tile = smem;                                               // [256][128 B]
+    float* s_red = reinterpret_cast<float*>(smem + kBwdChunk * 128);      // [warps][64][RS]
 
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int g = lane >> 2, t = lane & 3;
-    const int kw = warp % kBwdKW, sub = warp / kBwdKW;
-    const uint32_t lane_base = smem_u32(s_tab) + lane * 4;
     const int64_t nblk = a.K / kBlock;
-    const int64_t nkg = cdiv(nblk, kBwdKW);
-    const int64_t units = nkg * a.S;
+    const int64_t units = nblk * a.S;
     const int64_t rowbytes = a.K / 2;
+    const uint32_t tile_base = smem_u32(s_tile);
 
     for (int64_t u = blockIdx.x; u < units; u += gridDim.x) {
-        const int64_t kg = u / a.S, split = u % a.S;
-        const int64_t kb = kg * kBwdKW + kw;
-        const bool kvalid = kb < nblk;
+        const int64_t kb = u / a.S, split = u % a.S;
         const int64_t n_lo = split * a.rows_per_split;
         const int64_t n_hi = min(a.N, n_lo + a.rows_per_split);
         for (int64_t mc = 0; mc < a.M; mc += MC) {
-            float acc[4][MT][4];
+            float acc[MT][8][4];
 #pragma unroll
-            for (int j = 0; j < 4; ++j)
+            for (int mt = 0; mt < MT; ++mt)
 #pragma unroll
-                for (int nt = 0; nt < MT; ++nt) acc[j][nt][0] = acc[j][nt][1] = acc[j][nt][2] = acc[j][nt][3] = 0.f;
-            if (kvalid) {
-                for (int64_t n0 = n_lo + sub * 16; n0 < n_hi; n0 += 16 * kBwdNSUB) {
-                    // block constants of rows n0 .. n0+15, one per lane, then shuffled
-                    float cl = 0.f;
-                    if (lane < 16 && n0 + lane < n_hi)
-                        cl = block_constant(a.codes, a.scale, a.mean, (n0 + lane) * nblk + kb);
-                    const int64_t nA = n0 + 2 * t, nC = nA + 8;
-                    const float cA = __shfl_sync(0xffffffffu, cl, 2 * t);
-                    const float cB = __shfl_sync(0xffffffffu, cl, 2 * t + 1);
-                    const float cC = __shfl_sync(0xffffffffu, cl, 2 * t + 8);
-                    const float cD = __shfl_sync(0xffffffffu, cl, 2 * t + 9);
-                    const bool vA = nA < n_hi, vC = nC < n_hi;   // nA even and N % 8 == 0: nA+1 valid too
-                    const uint8_t* pk = a.packed + 32 * kb + 4 * g;
-                    const uint32_t wA = vA ? ldg_nc_u32(pk + nA * rowbytes) : 0u;
-                    const uint32_t wB = vA ? ldg_nc_u32(pk + (nA + 1) * rowbytes) : 0u;
-                    const uint32_t wC = vC ? ldg_nc_u32(pk + nC * rowbytes) : 0u;
-                    const uint32_t wD = vC ? ldg_nc_u32(pk + (nC + 1) * rowbytes) : 0u;
-                    uint32_t b0[MT], b1[MT];
-#pragma unroll
-                    for (int nt = 0; nt < MT; ++nt) {
-                        const int64_t m = mc + nt * 8 + g;
-                        uint32_t d01 = 0u, d89 = 0u;
-                        if (m < a.M) {
-                            const uint16_t* dyr = a.dY + m * a.N;
-                            if (vA) d01 = __ldg(reinterpret_cast<const unsigned int*>(dyr + nA));
-                            if (vC) d89 = __ldg(reinterpret_cast<const unsigned int*>(dyr + nC));
-                        }
-                        b0[nt] = pack_bf16x2(bf16lo_to_f32(d01) * cA, bf16hi_to_f32(d01) * cB);
-                        b1[nt] = pack_bf16x2(bf16lo_to_f32(d89) * cC, bf16hi_to_f32(d89) * cD);
+                for (int j = 0; j < 8; ++j) acc[mt][j][0] = acc[mt][j][1] = acc[mt][j][2] = acc[mt][j][3] = 0.f;
+            for (int64_t nc = n_lo; nc < n_hi; nc += kBwdChunk) {
+                // ---- dequantize row nc + tid, block kb, into the tile
+                {
+                    const int64_t n = nc + tid;
+                    uint4 p0 = make_uint4(0, 0, 0, 0), p1 = p0;
+                    float c = 0.f;
+                    if (n < n_hi) {
+                        const uint8_t* pp = a.packed + n * rowbytes + 32 * kb;
+                        p0 = ldg_nc_v4(pp);
+                        p1 = ldg_nc_v4(pp + 16);
+                        c = block_constant(a.codes, a.scale, a.mean, n * nblk + kb);
                     }
+                    const BlockTable tb = make_block_table(tab, c);
+                    const uint32_t pw[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
+                    const uint32_t row_addr = tile_base + tid * 128;
 #pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        const uint32_t PA = pair_lookup(lane_base, wA, j);
-                        const uint32_t PB = pair_lookup(lane_base, wB, j);
-                        const uint32_t PC = pair_lookup(lane_base, wC, j);
-                        const uint32_t PD = pair_lookup(lane_base, wD, j);
-                        const uint32_t a0 = prmt(PA, PB, 0x5410u);
-                        const uint32_t a1 = prmt(PA, PB, 0x7632u);
-                        const uint32_t a2 = prmt(PC, PD, 0x5410u);
-                        const uint32_t a3 = prmt(PC, PD, 0x7632u);
-#pragma unroll
-                        for (int nt = 0; nt < MT; ++nt) mma_bf16_16816(acc[j][nt], a0, a1, a2, a3, b0[nt], b1[nt]);
+                    for (int ch = 0; ch < 8; ++ch) {
+                        uint32_t o[4];
+                        decode8(tb, pw[ch], o);
+                        const uint32_t addr = row_addr + ((ch ^ (tid & 7)) << 4);
+                        asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};" ::"r"(addr), "r"(o[0]), "r"(o[1]),
+                                     "r"(o[2]), "r"(o[3]));
                     }
                 }
+                __syncthreads();
+                // ---- multiply: warp w takes tile rows [32w, 32w+32)
+#pragma unroll
+                for (int s2 = 0; s2 < 2; ++s2) {
+                    const int rbase = warp * 32 + s2 * 16;
+                    const int64_t nA = nc + rbase + 2 * t;          // reduction index of a0 / a1
+                    uint32_t af[MT][4];
+#pragma unroll
+                    for (int mt = 0; mt < MT; ++mt) {
+                        const int64_t m0 = mc + mt * 16 + g, m1 = m0 + 8;
+                        af[mt][0] = af[mt][1] = af[mt][2] = af[mt][3] = 0u;
+                        if (nA < n_hi) {
+                            if (m0 < a.M) af[mt][0] = __ldg(reinterpret_cast<const unsigned int*>(a.dY + m0 * a.N + nA));
+                            if (m1 < a.M) af[mt][1] = __ldg(reinterpret_cast<const unsigned int*>(a.dY + m1 * a.N + nA));
+                        }
+                        if (nA + 8 < n_hi) {
+                            if (m0 < a.M) af[mt][2] = __ldg(reinterpret_cast<const unsigned int*>(a.dY + m0 * a.N + nA + 8));
+                            if (m1 < a.M) af[mt][3] = __ldg(reinterpret_cast<const unsigned int*>(a.dY + m1 * a.N + nA + 8));
+                        }
+                    }
+                    const int mi = lane >> 3, rr = lane & 7;
+                    const int row = rbase + (mi & 1) * 8 + rr;
+#pragma unroll
+                    for (int jp = 0; jp < 4; ++jp) {
+                        const int ch = 2 * jp + (mi >> 1);
+                        const uint32_t addr = tile_base + row * 128 + ((ch ^ (row & 7)) << 4);
+                        uint32_t b00, b01, b10, b11;
+                        asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+                                     : "=r"(b00), "=r"(b01), "=r"(b10), "=r"(b11) : "r"(addr));
+#pragma unroll
+                        for (int mt = 0; mt < MT; ++mt) {
+                            mma_bf16_16816(acc[mt][2 * jp], af[mt][0], af[mt][1], af[mt][2], af[mt][3], b00, b01);
+                            mma_bf16_16816(acc[mt][2 * jp + 1], af[mt][0], af[mt][1], af[mt][2], af[mt][3], b10, b11);
+                        }
+                    }
+                }
+                __syncthreads();
             }
+            // acc[mt][j]: c0,c1 -> (token mt*16+g, k 8j+2t, +1), c2,c3 -> (token +8)
             float* red = s_red + warp * 64 * RS;
 #pragma unroll
-            for (int j = 0; j < 4; ++j)
+            for (int mt = 0; mt < MT; ++mt)
 #pragma unroll
-                for (int nt = 0; nt < MT; ++nt) {
-                    const int ke = 8 * g + 2 * j;
-                    red[ke * RS + nt * 8 + 2 * t] = acc[j][nt][0];
-                    red[ke * RS + nt * 8 + 2 * t + 1] = acc[j][nt][1];
-                    red[(ke + 1) * RS + nt * 8 + 2 * t] = acc[j][nt][2];
-                    red[(ke + 1) * RS + nt * 8 + 2 * t + 1] = acc[j][nt][3];
+                for (int j = 0; j < 8; ++j) {
+                    const int k0 = 8 * j + 2 * t;
+                    red[k0 * RS + mt * 16 + g] = acc[mt][j][0];
+                    red[(k0 + 1) * RS + mt * 16 + g] = acc[mt][j][1];
+                    red[k0 * RS + mt * 16 + g + 8] = acc[mt][j][2];
+                    red[(k0 + 1) * RS + mt * 16 + g + 8] = acc[mt][j][3];
                 }
             __syncthreads();
-            for (int idx = threadIdx.x; idx < kBwdKW * 64 * MC; idx += blockDim.x) {
-                const int kl = idx % (kBwdKW * 64), ml = idx / (kBwdKW * 64);
-                const int kwi = kl / 64, ke = kl % 64;
-                const int64_t k = (kg * kBwdKW + kwi) * 64 + ke, m = mc + ml;
-                if (k < a.K && m < a.M) {
+            for (int idx = tid; idx < 64 * MC; idx += kBwdThreads) {
+                const int kl = idx & 63, ml = idx >> 6;
+                const int64_t m = mc + ml;
+                if (m < a.M) {
                     float v = 0.f;
 #pragma unroll
-                    for (int s = 0; s < kBwdNSUB; ++s) v += s_red[(s * kBwdKW + kwi) * 64 * RS + ke * RS + ml];
-                    a.part[(split * a.M + m) * a.K + k] = v;
+                    for (int w = 0; w < kBwdWarps; ++w) v += s_red[w * 64 * RS + kl * RS + ml];
+                    a.part[(split * a.M + m) * a.K + kb * 64 + kl] = v;
                 }
             }
             __syncthreads();
