@@ -146,17 +146,26 @@ __global__ void __launch_bounds__(128) k_gemm_mma(GemmArgs p) {
 }
 
 // Sum of the split-K partials in split order, then up to three outputs, for
-// i < Iout and j < Jout (Jout <= J):
-//   f32 [i * ld_f32 + j]            = v
-//   o1  [i * s1i + j * s1j]  (bf16) = alpha1 * v  for j < J1, 0 for J1 <= j < J1pad
+// i < Iout and j < Jiter (columns at or beyond the partial extent J read as 0):
+//   f32 [i * ld_f32 + j]            = v                            (j < Jf)
+//   o1  [i * s1i + j * s1j]  (bf16) = alpha1 * v for j < J1, 0 for J1 <= j < J1pad
 //   o2  likewise with alpha2, J2, J2pad.
+//   hl  [i * hl_ld + j] = bf16(v), hl[i * hl_ld + hl_off + j] = bf16(v - bf16(v))
+//       for j < J1 (zero for J1 <= j < hl_off): a hi + lo pair that carries
+//       v to about 16 significant bits into a later bf16 product.
+// With row_pair (col_pair) > 0 the value is the sum of partial rows i and
+// i + row_pair (columns j and j + col_pair): the hi and lo halves of a
+// product computed with a hi + lo operand.
 struct FinishArgs {
     const float* C;
     int splits;
     int64_t I, J;            // partial layout [splits][I][J]
-    int64_t Iout, Jout;
+    int64_t row_pair, col_pair;
+    uint16_t* hl;
+    int64_t hl_ld, hl_off;
+    int64_t Iout, Jiter;
     float* f32;
-    int64_t ld_f32;
+    int64_t ld_f32, Jf;
     uint16_t* o1;
     int64_t s1i, s1j, J1, J1pad;
     float alpha1;
@@ -166,12 +175,27 @@ struct FinishArgs {
 };
 
 __global__ void __launch_bounds__(256) k_gemm_finish(FinishArgs f) {
-    const int64_t total = f.Iout * f.Jout;
+    const int64_t total = f.Iout * f.Jiter;
     for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < total; e += (int64_t)gridDim.x * blockDim.x) {
-        const int64_t i = e / f.Jout, j = e % f.Jout;
+        const int64_t i = e / f.Jiter, j = e % f.Jiter;
         float v = 0.f;
-        for (int z = 0; z < f.splits; ++z) v += f.C[(z * f.I + i) * f.J + j];
-        if (f.f32) f.f32[i * f.ld_f32 + j] = v;
+        if (j < f.J) {
+            for (int z = 0; z < f.splits; ++z) v += f.C[(z * f.I + i) * f.J + j];
+            if (f.row_pair > 0)
+                for (int z = 0; z < f.splits; ++z) v += f.C[(z * f.I + i + f.row_pair) * f.J + j];
+            if (f.col_pair > 0)
+                for (int z = 0; z < f.splits; ++z) v += f.C[(z * f.I + i) * f.J + j + f.col_pair];
+        }
+        if (f.f32 && j < f.Jf) f.f32[i * f.ld_f32 + j] = v;
+        if (f.hl && j < f.hl_off) {
+            uint16_t hi = 0, lo = 0;
+            if (j < f.J1) {
+                hi = (uint16_t)(pack_bf16x2(v, 0.f) & 0xffffu);
+                lo = (uint16_t)(pack_bf16x2(v - bf16lo_to_f32(hi), 0.f) & 0xffffu);
+            }
+            f.hl[i * f.hl_ld + j] = hi;
+            f.hl[i * f.hl_ld + f.hl_off + j] = lo;
+        }
         if (f.o1 && j < f.J1pad) f.o1[i * f.s1i + j * f.s1j] = (j < f.J1) ? (uint16_t)(pack_bf16x2(f.alpha1 * v, 0.f) & 0xffffu) : (uint16_t)0;
         if (f.o2 && j < f.J2pad) f.o2[i * f.s2i + j * f.s2j] = (j < f.J2) ? (uint16_t)(pack_bf16x2(f.alpha2 * v, 0.f) & 0xffffu) : (uint16_t)0;
     }

@@ -15,6 +15,7 @@
 #include "quant.cuh"
 #include "small.cuh"
 #include "lora.cuh"
+#include "tc_gemm.cuh"
 
 using namespace qnf4;
 
@@ -113,7 +114,7 @@ int launch_status() {
 // ---------------------------------------------------------------------------
 struct Plan {
     int64_t M, N, K;
-    int r, rp;
+    int r, rp, rp64;
     // split-K choices
     int zT, zU, zA, zB;
     int64_t kT, kU, kA, kB;         // k per split
@@ -151,6 +152,7 @@ Plan make_plan(int64_t M, int64_t N, int64_t K, int r, int sms) {
     Plan p{};
     p.M = M; p.N = N; p.K = K; p.r = r;
     p.rp = (int)rup(r, 16);
+    p.rp64 = (int)rup(r, 64);
     const int64_t target = 2 * (int64_t)sms;
     const int64_t bj = p.rp == 16 ? 16 : 64;
     // T = X A^T: I = M (BI 64), J = rp, Kd = K
@@ -183,18 +185,18 @@ Plan make_plan(int64_t M, int64_t N, int64_t K, int r, int sms) {
     auto upd = [&](size_t b) { if (b > part) part = b; };
     upd(gemm_part_bytes(M, p.rp, p.zT));
     upd(gemm_part_bytes(M, p.rp, p.zU));
-    upd(gemm_part_bytes(p.rp, K, p.zA));
-    upd(gemm_part_bytes(N, p.rp, p.zB));
-    upd((size_t)p.S_bwd * (M < 32 ? M : 32) * K * 4);   // small-path dX partials, 32-token chunks
+    upd(gemm_part_bytes(2 * p.rp, K, p.zA));
+    upd(gemm_part_bytes(N, 2 * p.rp, p.zB));
+    if (M <= 32) upd((size_t)p.S_bwd * M * K * 4);     // small-path dX partials
     size_t off = 0;
     auto take = [&](size_t b) { const size_t o = off; off = align256(off + b); return o; };
     p.off_part = take(part);
     p.off_T32 = take((size_t)M * p.rp * 4);
     p.off_U32 = take((size_t)M * p.rp * 4);
-    p.off_Tp = take((size_t)M * p.rp * 2);
-    p.off_Ubf = take((size_t)M * p.rp * 2);
-    p.off_sT = take((size_t)M * p.rp * 2);
-    p.off_sU = take((size_t)M * p.rp * 2);
+    p.off_Tp = take((size_t)M * 2 * p.rp * 2);     // T hi | lo
+    p.off_Ubf = take((size_t)M * 2 * p.rp * 2);    // U hi | lo
+    p.off_sT = take((size_t)M * p.rp64 * 2);
+    p.off_sU = take((size_t)M * p.rp64 * 2);
     p.off_Bp = take((size_t)N * p.rp * 2);
     p.off_At = take((size_t)K * p.rp * 2);
     p.total = off;
@@ -227,8 +229,7 @@ int run_gemm(const uint16_t* A, int64_t lda, const uint16_t* B, int64_t ldb, int
     else k_gemm_mma<AK, BK, 64, 64, 2, 2><<<grid, 128, 0, st>>>(g);
     f.I = g.I; f.J = g.J;
     if (f.Iout > I) f.Iout = I;
-    if (f.Jout > J) f.Jout = J;
-    k_gemm_finish<<<grid_for(f.Iout * f.Jout, 256, sms), 256, 0, st>>>(f);
+    k_gemm_finish<<<grid_for(f.Iout * f.Jiter, 256, sms), 256, 0, st>>>(f);
     return launch_status();
 }
 
@@ -245,25 +246,111 @@ int validate_weight(const nf4dq_weight* w) {
     return QLORA_OK;
 }
 
-// T (fp32 into ws, optional bf16 T_out [M, r], bf16 padded Tp and s*T) from X, A.
+// ---------------------------------------------------------------------------
+// TMA tensor maps (driver entry point fetched through the runtime, so the
+// library does not link libcuda directly)
+// ---------------------------------------------------------------------------
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(ptr);
+    });
+    return fn;
+}
+
+// 2-D row-major tensor [outer, inner] with the given row pitch; box [box_outer, box_inner].
+bool make_map_2d(CUtensorMap* m, CUtensorMapDataType dt, const void* ptr, uint64_t inner, uint64_t outer,
+                 uint64_t pitch_bytes, uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle sw) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[2] = {inner, outer};
+    const cuuint64_t strides[1] = {pitch_bytes};
+    const cuuint32_t box[2] = {box_inner, box_outer};
+    const cuuint32_t estr[2] = {1, 1};
+    return fn(m, dt, 2, const_cast<void*>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool g_tc_attr_set[64];
+std::mutex g_tc_mu;
+
+int ensure_tc_attrs() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return QLORA_ERR_DEVICE;
+    std::lock_guard<std::mutex> lk(g_tc_mu);
+    if (!g_tc_attr_set[dev]) {
+        if (cudaFuncSetAttribute(tc::k_tc_gemm<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, tc::SMEM_ALLOC) !=
+                cudaSuccess ||
+            cudaFuncSetAttribute(tc::k_tc_gemm<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, tc::SMEM_ALLOC) !=
+                cudaSuccess)
+            return QLORA_ERR_LAUNCH;
+        g_tc_attr_set[dev] = true;
+    }
+    return QLORA_OK;
+}
+
+// Fused dequant-GEMM on the tcgen05 path.  act [M, n_red] bf16 activations,
+// lact [M, rp64] bf16 scaled LoRA activations, lora_w / ldl the LoRA weight
+// rows (B for the forward, A for the backward).
+template <bool BWD>
+int launch_tc(const nf4dq_weight* w, const uint16_t* act, int64_t M, const uint16_t* lact, int rp64,
+              const uint16_t* lora_w, int64_t ldl, int r, uint16_t* out, int sms, cudaStream_t st) {
+    int rc = ensure_tc_attrs();
+    if (rc != QLORA_OK) return rc;
+    const int64_t N = w->N, K = w->K;
+    const int64_t n_red = BWD ? N : K, n_out = BWD ? K : N;
+    CUtensorMap tmA, tmL, tmP;
+    if (!make_map_2d(&tmA, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, act, n_red, M, n_red * 2, 64, 128,
+                     CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_map_2d(&tmL, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, lact, rp64, M, (uint64_t)rp64 * 2, 64, 128,
+                     CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_map_2d(&tmP, CU_TENSOR_MAP_DATA_TYPE_UINT8, w->packed, K / 2, N, K / 2, BWD ? 128 : 32,
+                     BWD ? 64 : 256, CU_TENSOR_MAP_SWIZZLE_NONE))
+        return QLORA_ERR_LAUNCH;
+    tc::Args a{};
+    a.codes = w->codes; a.scale = w->scale; a.mean = w->mean;
+    a.lora_w = lora_w; a.ldl = ldl; a.r = r; a.nlora = (int)cdiv(r, 64);
+    a.out = out; a.M = M; a.N = N; a.K = K; a.n_out = n_out; a.n_red = n_red;
+    const int64_t ntiles = cdiv(M, tc::BM) * cdiv(n_out, tc::BN);
+    const int grid = (int)(ntiles < sms ? ntiles : sms);
+    tc::k_tc_gemm<BWD><<<grid, tc::kThreads, tc::SMEM_ALLOC, st>>>(tmA, tmL, tmP, a, tables());
+    return launch_status();
+}
+
+// Tokens at or below this count take the small-M (GEMV-shaped) kernels.
+constexpr int64_t kSmallMaxM = 32;
+
+// T = X A^T: T32 (fp32 [M, rp]), Thl (bf16 hi|lo [M, 2 rp]), sT (bf16 s*T, [M, rp64]),
+// and the caller's T_out (bf16 [M, r]) when given.
 int compute_T(const Plan& p, const uint16_t* X, const uint16_t* A, float s, uint16_t* T_out, uint8_t* ws, int sms,
               cudaStream_t st) {
     FinishArgs f = fin_none();
-    f.Iout = p.M; f.Jout = p.rp;
-    f.f32 = reinterpret_cast<float*>(ws + p.off_T32); f.ld_f32 = p.rp;
-    f.o1 = reinterpret_cast<uint16_t*>(ws + p.off_Tp); f.s1i = p.rp; f.s1j = 1; f.J1 = p.r; f.J1pad = p.rp; f.alpha1 = 1.f;
-    f.o2 = reinterpret_cast<uint16_t*>(ws + p.off_sT); f.s2i = p.rp; f.s2j = 1; f.J2 = p.r; f.J2pad = p.rp; f.alpha2 = s;
+    f.Iout = p.M; f.Jiter = p.rp64;
+    f.f32 = reinterpret_cast<float*>(ws + p.off_T32); f.ld_f32 = p.rp; f.Jf = p.rp;
+    f.J1 = p.r;
+    f.hl = reinterpret_cast<uint16_t*>(ws + p.off_Tp); f.hl_ld = 2 * p.rp; f.hl_off = p.rp;
+    f.o2 = reinterpret_cast<uint16_t*>(ws + p.off_sT); f.s2i = p.rp64; f.s2j = 1; f.J2 = p.r; f.J2pad = p.rp64; f.alpha2 = s;
     int rc = run_gemm<true, true>(X, p.K, A, p.K, p.M, p.rp, p.K, p.M, p.r, p.zT, p.kT,
                                   reinterpret_cast<float*>(ws + p.off_part), f, sms, st);
     if (rc != QLORA_OK) return rc;
     if (T_out) {
-        // bf16 copy in the caller's unpadded [M, r] layout
+        // bf16 T in the caller's [M, r] layout: the hi half of Thl
         k_pad_cols<<<grid_for(p.M * p.r, 256, sms), 256, 0, st>>>(reinterpret_cast<uint16_t*>(ws + p.off_Tp), p.M,
-                                                                   p.rp, T_out, p.r);
+                                                                   2 * p.rp, T_out, p.r);
         rc = launch_status();
     }
     return rc;
 }
+
 
 }  // namespace
 
@@ -347,16 +434,32 @@ int qlora_linear_fwd(const qlora_bf16* X, int64_t M, const nf4dq_weight* w, cons
     rc = compute_T(p, X, A, scaling, T_out, wsb, sms, st);
     if (rc != QLORA_OK) return rc;
 
-    SmallFwdArgs a{};
-    a.X = X; a.packed = w->packed; a.codes = w->codes; a.scale = w->scale; a.mean = w->mean;
-    a.T32 = reinterpret_cast<const float*>(wsb + p.off_T32); a.B = B; a.Y = Y;
-    a.M = M; a.N = w->N; a.K = w->K; a.rp = p.rp; a.r = r; a.s = scaling;
-    const int64_t ntiles = cdiv(w->N, 16);
-    const int grid = (int)(ntiles < 2LL * sms ? ntiles : 2LL * sms);
-    if (M <= 16) k_fwd_small<1><<<grid, kSmallThreads, fwd_small_smem_bytes<1>(), st>>>(a, tables());
-    else k_fwd_small<2><<<grid, kSmallThreads, fwd_small_smem_bytes<2>(), st>>>(a, tables());
-    rc = launch_status();
-    if (rc == QLORA_OK) t_last_path = 1;
+    if (M <= kSmallMaxM) {
+        SmallFwdArgs a{};
+        a.X = X; a.packed = w->packed; a.codes = w->codes; a.scale = w->scale; a.mean = w->mean;
+        a.T32 = reinterpret_cast<const float*>(wsb + p.off_T32); a.B = B; a.Y = Y;
+        a.M = M; a.N = w->N; a.K = w->K; a.rp = p.rp; a.r = r; a.s = scaling;
+        const int64_t ntiles = cdiv(w->N, 16);
+        const int grid = (int)(ntiles < 2LL * sms ? ntiles : 2LL * sms);
+        if (M <= 16) k_fwd_small<1><<<grid, kSmallThreads, fwd_small_smem_bytes<1>(), st>>>(a, tables());
+        else k_fwd_small<2><<<grid, kSmallThreads, fwd_small_smem_bytes<2>(), st>>>(a, tables());
+        rc = launch_status();
+        if (rc == QLORA_OK) t_last_path = 1;
+        return rc;
+    }
+    // tcgen05 path: LoRA weight rows must be 16-byte granular (r % 8 == 0) or padded
+    const uint16_t* lw = B;
+    int64_t ldl = r;
+    if (r % 8 != 0) {
+        uint16_t* Bp = reinterpret_cast<uint16_t*>(wsb + p.off_Bp);
+        k_pad_cols<<<grid_for(w->N * p.rp, 256, sms), 256, 0, st>>>(B, w->N, r, Bp, p.rp);
+        lw = Bp;
+        ldl = p.rp;
+    } else if (!aligned16(B)) {
+        return QLORA_ERR_ALIGN;
+    }
+    rc = launch_tc<false>(w, X, M, reinterpret_cast<const uint16_t*>(wsb + p.off_sT), p.rp64, lw, ldl, r, Y, sms, st);
+    if (rc == QLORA_OK) t_last_path = 2;
     return rc;
 }
 
@@ -370,8 +473,7 @@ int qlora_linear_bwd(const qlora_bf16* X, const qlora_bf16* dY, int64_t M, const
     if (M <= 0 || M > ((int64_t)1 << 31)) return QLORA_ERR_SHAPE;
     if (r < 1 || r > QLORA_MAX_RANK) return QLORA_ERR_RANK;
     if (!std::isfinite(scaling)) return QLORA_ERR_VALUE;
-    if (!aligned16(X) || !aligned16(dY) || !aligned16(A) || !aligned16(dX) || !aligned16(B)) return QLORA_ERR_ALIGN;
-    if (T && !aligned16(T)) return QLORA_ERR_ALIGN;
+    if (!aligned16(X) || !aligned16(dY) || !aligned16(A) || !aligned16(dX)) return QLORA_ERR_ALIGN;
     if (!ws || (reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return ws ? QLORA_ERR_ALIGN : QLORA_ERR_WORKSPACE;
     int sms = 0;
     rc = check_device(&sms);
@@ -382,71 +484,77 @@ int qlora_linear_bwd(const qlora_bf16* X, const qlora_bf16* dY, int64_t M, const
     cudaStream_t st = (cudaStream_t)stream;
     uint8_t* wsb = static_cast<uint8_t*>(ws);
     float* part = reinterpret_cast<float*>(wsb + p.off_part);
-    uint16_t* Tp = reinterpret_cast<uint16_t*>(wsb + p.off_Tp);
-    uint16_t* Ubf = reinterpret_cast<uint16_t*>(wsb + p.off_Ubf);
+    uint16_t* Thl = reinterpret_cast<uint16_t*>(wsb + p.off_Tp);
+    uint16_t* Uhl = reinterpret_cast<uint16_t*>(wsb + p.off_Ubf);
     uint16_t* Bp = reinterpret_cast<uint16_t*>(wsb + p.off_Bp);
 
-    // T: recompute, or take the caller's bf16 copy (padded to rp columns)
+    // T: recompute (hi + lo pair), or take the caller's bf16 copy as it is (lo = 0)
     if (T == nullptr) {
         rc = compute_T(p, X, A, scaling, nullptr, wsb, sms, st);
     } else {
-        k_pad_cols<<<grid_for(M * p.rp, 256, sms), 256, 0, st>>>(T, M, r, Tp, p.rp);
+        k_pad_cols<<<grid_for(M * 2 * p.rp, 256, sms), 256, 0, st>>>(T, M, r, Thl, 2 * p.rp);
         rc = launch_status();
     }
     if (rc != QLORA_OK) return rc;
 
-    // U = dY B  ->  U32 (fp32), Ubf (bf16, unscaled), sU (bf16, scaled)
+    // U = dY B  ->  U32 (fp32), Uhl (bf16 hi | lo), sU (bf16 s*U, [M, rp64])
     const uint16_t* Bop = B;
     int64_t ldb = r;
-    if (r % 8 != 0) {
+    if (r % 8 != 0 || !aligned16(B)) {
         k_pad_cols<<<grid_for(N * p.rp, 256, sms), 256, 0, st>>>(B, N, r, Bp, p.rp);
         Bop = Bp; ldb = p.rp;
     }
     {
         FinishArgs f = fin_none();
-        f.Iout = M; f.Jout = p.rp;
-        f.f32 = reinterpret_cast<float*>(wsb + p.off_U32); f.ld_f32 = p.rp;
-        f.o1 = Ubf; f.s1i = p.rp; f.s1j = 1; f.J1 = r; f.J1pad = p.rp; f.alpha1 = 1.f;
-        f.o2 = reinterpret_cast<uint16_t*>(wsb + p.off_sU); f.s2i = p.rp; f.s2j = 1; f.J2 = r; f.J2pad = p.rp;
+        f.Iout = M; f.Jiter = p.rp64;
+        f.f32 = reinterpret_cast<float*>(wsb + p.off_U32); f.ld_f32 = p.rp; f.Jf = p.rp;
+        f.J1 = r;
+        f.hl = Uhl; f.hl_ld = 2 * p.rp; f.hl_off = p.rp;
+        f.o2 = reinterpret_cast<uint16_t*>(wsb + p.off_sU); f.s2i = p.rp64; f.s2j = 1; f.J2 = r; f.J2pad = p.rp64;
         f.alpha2 = scaling;
         rc = run_gemm<true, false>(dY, N, Bop, ldb, M, p.rp, N, M, r, p.zU, p.kU, part, f, sms, st);
         if (rc != QLORA_OK) return rc;
     }
-    // dB = s dY^T T  [N, r]
+    // dB = s dY^T T  [N, r]   (T as hi | lo columns, summed in the finish)
     {
         FinishArgs f = fin_none();
-        f.Iout = N; f.Jout = r;
+        f.Iout = N; f.Jiter = r; f.col_pair = p.rp;
         f.o1 = dB; f.s1i = r; f.s1j = 1; f.J1 = r; f.J1pad = r; f.alpha1 = scaling;
-        rc = run_gemm<false, false>(dY, N, Tp, p.rp, N, p.rp, M, N, p.rp, p.zB, p.kB, part, f, sms, st);
+        rc = run_gemm<false, false>(dY, N, Thl, 2 * p.rp, N, 2 * p.rp, M, N, 2 * p.rp, p.zB, p.kB, part, f, sms, st);
         if (rc != QLORA_OK) return rc;
     }
-    // dA = s U^T X  [r, K]
+    // dA = s U^T X  [r, K]   (U as hi | lo rows, summed in the finish)
     {
         FinishArgs f = fin_none();
-        f.Iout = r; f.Jout = K;
+        f.Iout = r; f.Jiter = K; f.row_pair = p.rp;
         f.o1 = dA; f.s1i = K; f.s1j = 1; f.J1 = K; f.J1pad = K; f.alpha1 = scaling;
-        rc = run_gemm<false, false>(Ubf, p.rp, X, K, p.rp, K, M, p.rp, K, p.zA, p.kA, part, f, sms, st);
+        rc = run_gemm<false, false>(Uhl, 2 * p.rp, X, K, 2 * p.rp, K, M, 2 * p.rp, K, p.zA, p.kA, part, f, sms, st);
         if (rc != QLORA_OK) return rc;
     }
-    // dX = dY W' + s U A, 32 tokens per pass
-    for (int64_t m0 = 0; m0 < M; m0 += 32) {
-        const int64_t mc = (M - m0 < 32) ? M - m0 : 32;
+    // dX = dY W' + s U A
+    if (M > kSmallMaxM) {
+        rc = launch_tc<true>(w, dY, M, reinterpret_cast<const uint16_t*>(wsb + p.off_sU), p.rp64, A, K, r, dX, sms,
+                             st);
+        if (rc == QLORA_OK) t_last_path = 2;
+        return rc;
+    }
+    {
         SmallBwdArgs a{};
-        a.dY = dY + m0 * N; a.packed = w->packed; a.codes = w->codes; a.scale = w->scale; a.mean = w->mean;
-        a.part = part; a.M = mc; a.N = N; a.K = K; a.rows_per_split = p.rows_per_split; a.S = p.S_bwd;
+        a.dY = dY; a.packed = w->packed; a.codes = w->codes; a.scale = w->scale; a.mean = w->mean;
+        a.part = part; a.M = M; a.N = N; a.K = K; a.rows_per_split = p.rows_per_split; a.S = p.S_bwd;
         const int64_t units = (K / kBlock) * p.S_bwd;
         const int grid = (int)(units < 2LL * sms ? units : 2LL * sms);
-        if (mc <= 16) k_bwd_small<1><<<grid, kBwdThreads, bwd_small_smem_bytes<1>(), st>>>(a, tables());
+        if (M <= 16) k_bwd_small<1><<<grid, kBwdThreads, bwd_small_smem_bytes<1>(), st>>>(a, tables());
         else k_bwd_small<2><<<grid, kBwdThreads, bwd_small_smem_bytes<2>(), st>>>(a, tables());
-        k_bwd_small_finish<<<grid_for(mc * K, 256, sms), 256, 0, st>>>(
-            part, p.S_bwd, mc, K, reinterpret_cast<const float*>(wsb + p.off_U32) + m0 * p.rp, p.rp, A, r, scaling,
-            dX + m0 * K);
+        k_bwd_small_finish<<<grid_for(M * K, 256, sms), 256, 0, st>>>(
+            part, p.S_bwd, M, K, reinterpret_cast<const float*>(wsb + p.off_U32), p.rp, A, r, scaling, dX);
         rc = launch_status();
         if (rc != QLORA_OK) return rc;
     }
     t_last_path = 1;
     return QLORA_OK;
 }
+
 
 const char* qlora_status_string(int status) {
     switch (status) {

@@ -41,17 +41,21 @@ def _setup(oracle_mod, M, N, K, r, seed, w_std=0.02, x_std=1.0):
 
 
 CASES = [
-    # M, N, K, r
+    # M, N, K, r            small-M kernels for M <= 32, tcgen05 kernels above
     (1, 64, 64, 16),
     (3, 136, 192, 4),
     (8, 256, 1024, 16),
     (16, 512, 512, 64),
     (17, 200, 320, 24),
     (32, 1024, 1024, 16),
+    (5, 4096, 4096, 16),
     (33, 128, 256, 16),
     (100, 264, 640, 8),
+    (128, 256, 256, 16),
+    (200, 520, 448, 24),
     (257, 384, 448, 64),
-    (5, 4096, 4096, 16),
+    (300, 768, 1216, 100),
+    (512, 1024, 2048, 16),
 ]
 
 
@@ -74,9 +78,12 @@ def test_fwd_bwd_parity(oracle_mod, M, N, K, r):
     _close(inputs.to_f64(dX), dXr, "dX")
     _close(inputs.to_f64(dA), dAr, "dA")
     _close(inputs.to_f64(dB), dBr, "dB")
+    # with T supplied, the bf16 T is an input of the backward: dB = s dY^T T_given
+    dBr_given = s * (dY64.T @ inputs.to_f64(T_out))
     _close(inputs.to_f64(dX2), dXr, "dX (T given)")
     _close(inputs.to_f64(dA2), dAr, "dA (T given)")
-    _close(inputs.to_f64(dB2), dBr, "dB (T given)")
+    _close(inputs.to_f64(dB2), dBr_given, "dB (T given)")
+    assert ops.qlora_last_path() == (1 if M <= 32 else 2)
 
 
 def test_zero_B_is_plain_dequant_matmul(oracle_mod):
