@@ -55,6 +55,8 @@ def lib():
             "qlora_status_string": (ctypes.c_char_p, [i32]),
             "qlora_device_status": (i32, [i32]),
             "qlora_last_path": (i32, []),
+            "qlora_launch_count": (ctypes.c_longlong, []),
+            "qlora_set_kernel_events": (i32, [P, P]),
         }
         for name, (res, args) in sig.items():
             fn = getattr(L, name)
@@ -196,3 +198,14 @@ def qlora_device_status(reset: bool = True) -> int:
 
 def qlora_last_path() -> int:
     return int(lib().qlora_last_path())
+
+
+def qlora_launch_count() -> int:
+    return int(lib().qlora_launch_count())
+
+
+def qlora_set_kernel_events(before, after) -> None:
+    """Record torch.cuda.Event `before`/`after` around the next fused dequant-GEMM launch on this thread."""
+    b = ctypes.c_void_p(before.cuda_event) if before is not None else None
+    a = ctypes.c_void_p(after.cuda_event) if after is not None else None
+    _check("qlora_set_kernel_events", lib().qlora_set_kernel_events(b, a))

@@ -63,6 +63,23 @@ const NF4Tables& tables() {
 
 thread_local int t_last_path = 0;
 
+// Kernel launches made by this library (all threads), for benchmarks.
+std::atomic<long long> g_launches{0};
+inline void note_launch(int n = 1) { g_launches.fetch_add(n, std::memory_order_relaxed); }
+
+// One-shot events recorded around the next fused dequant-GEMM launch.
+thread_local cudaEvent_t t_ev_before = nullptr;
+thread_local cudaEvent_t t_ev_after = nullptr;
+
+inline void hook_before(cudaStream_t st) {
+    if (t_ev_before) cudaEventRecord(t_ev_before, st);
+}
+inline void hook_after(cudaStream_t st) {
+    if (t_ev_after) cudaEventRecord(t_ev_after, st);
+    t_ev_before = nullptr;
+    t_ev_after = nullptr;
+}
+
 int g_sm_count[64];
 std::atomic<int> g_dev_ok[64];   // 0 unknown, 1 sm_100, -1 other
 
@@ -227,9 +244,11 @@ int run_gemm(const uint16_t* A, int64_t lda, const uint16_t* B, int64_t ldb, int
     if (bj == 16) k_gemm_mma<AK, BK, 64, 16, 4, 1><<<grid, 128, 0, st>>>(g);
     else if (bi == 16) k_gemm_mma<AK, BK, 16, 64, 1, 4><<<grid, 128, 0, st>>>(g);
     else k_gemm_mma<AK, BK, 64, 64, 2, 2><<<grid, 128, 0, st>>>(g);
+    note_launch();
     f.I = g.I; f.J = g.J;
     if (f.Iout > I) f.Iout = I;
     k_gemm_finish<<<grid_for(f.Iout * f.Jiter, 256, sms), 256, 0, st>>>(f);
+    note_launch();
     return launch_status();
 }
 
@@ -322,7 +341,10 @@ int launch_tc(const nf4dq_weight* w, const uint16_t* act, int64_t M, const uint1
     a.out = out; a.M = M; a.N = N; a.K = K; a.n_out = n_out; a.n_red = n_red;
     const int64_t ntiles = cdiv(M, tc::BM) * cdiv(n_out, tc::BN);
     const int grid = (int)(ntiles < sms ? ntiles : sms);
+    hook_before(st);
     tc::k_tc_gemm<BWD><<<grid, tc::kThreads, tc::SMEM_ALLOC, st>>>(tmA, tmL, tmP, a, tables());
+    hook_after(st);
+    note_launch();
     return launch_status();
 }
 
@@ -346,6 +368,7 @@ int compute_T(const Plan& p, const uint16_t* X, const uint16_t* A, float s, uint
         // bf16 T in the caller's [M, r] layout: the hi half of Thl
         k_pad_cols<<<grid_for(p.M * p.r, 256, sms), 256, 0, st>>>(reinterpret_cast<uint16_t*>(ws + p.off_Tp), p.M,
                                                                    2 * p.rp, T_out, p.r);
+        note_launch();
         rc = launch_status();
     }
     return rc;
@@ -388,6 +411,7 @@ int nf4_quantize_dq(const qlora_bf16* W, int64_t N, int64_t K, uint8_t* packed, 
     const NF4Tables& tab = tables();
     int grid = (int)(ng < (int64_t)sms * 8 ? ng : (int64_t)sms * 8);
     k_quantize_dq<<<grid, 256, 0, (cudaStream_t)stream>>>(W, nb, packed, codes, scale, mean, tab);
+    note_launch();
     return launch_status();
 }
 
@@ -403,6 +427,7 @@ int nf4_dequant(const nf4dq_weight* w, qlora_bf16* W_out, qlora_stream_t stream)
     const int64_t nchunks = w->N * w->K / 32;
     k_dequant<<<grid_for(nchunks, 256, sms), 256, 0, (cudaStream_t)stream>>>(w->packed, w->codes, w->scale, w->mean,
                                                                             nchunks, W_out, tables());
+    note_launch();
     return launch_status();
 }
 
@@ -441,8 +466,11 @@ int qlora_linear_fwd(const qlora_bf16* X, int64_t M, const nf4dq_weight* w, cons
         a.M = M; a.N = w->N; a.K = w->K; a.rp = p.rp; a.r = r; a.s = scaling;
         const int64_t ntiles = cdiv(w->N, 16);
         const int grid = (int)(ntiles < 2LL * sms ? ntiles : 2LL * sms);
+        hook_before(st);
         if (M <= 16) k_fwd_small<1><<<grid, kSmallThreads, fwd_small_smem_bytes<1>(), st>>>(a, tables());
         else k_fwd_small<2><<<grid, kSmallThreads, fwd_small_smem_bytes<2>(), st>>>(a, tables());
+        hook_after(st);
+        note_launch();
         rc = launch_status();
         if (rc == QLORA_OK) t_last_path = 1;
         return rc;
@@ -453,6 +481,7 @@ int qlora_linear_fwd(const qlora_bf16* X, int64_t M, const nf4dq_weight* w, cons
     if (r % 8 != 0) {
         uint16_t* Bp = reinterpret_cast<uint16_t*>(wsb + p.off_Bp);
         k_pad_cols<<<grid_for(w->N * p.rp, 256, sms), 256, 0, st>>>(B, w->N, r, Bp, p.rp);
+        note_launch();
         lw = Bp;
         ldl = p.rp;
     } else if (!aligned16(B)) {
@@ -493,6 +522,7 @@ int qlora_linear_bwd(const qlora_bf16* X, const qlora_bf16* dY, int64_t M, const
         rc = compute_T(p, X, A, scaling, nullptr, wsb, sms, st);
     } else {
         k_pad_cols<<<grid_for(M * 2 * p.rp, 256, sms), 256, 0, st>>>(T, M, r, Thl, 2 * p.rp);
+        note_launch();
         rc = launch_status();
     }
     if (rc != QLORA_OK) return rc;
@@ -502,6 +532,7 @@ int qlora_linear_bwd(const qlora_bf16* X, const qlora_bf16* dY, int64_t M, const
     int64_t ldb = r;
     if (r % 8 != 0 || !aligned16(B)) {
         k_pad_cols<<<grid_for(N * p.rp, 256, sms), 256, 0, st>>>(B, N, r, Bp, p.rp);
+        note_launch();
         Bop = Bp; ldb = p.rp;
     }
     {
@@ -544,10 +575,14 @@ int qlora_linear_bwd(const qlora_bf16* X, const qlora_bf16* dY, int64_t M, const
         a.part = part; a.M = M; a.N = N; a.K = K; a.rows_per_split = p.rows_per_split; a.S = p.S_bwd;
         const int64_t units = (K / kBlock) * p.S_bwd;
         const int grid = (int)(units < 2LL * sms ? units : 2LL * sms);
+        hook_before(st);
         if (M <= 16) k_bwd_small<1><<<grid, kBwdThreads, bwd_small_smem_bytes<1>(), st>>>(a, tables());
         else k_bwd_small<2><<<grid, kBwdThreads, bwd_small_smem_bytes<2>(), st>>>(a, tables());
+        hook_after(st);
+        note_launch();
         k_bwd_small_finish<<<grid_for(M * K, 256, sms), 256, 0, st>>>(
             part, p.S_bwd, M, K, reinterpret_cast<const float*>(wsb + p.off_U32), p.rp, A, r, scaling, dX);
+        note_launch();
         rc = launch_status();
         if (rc != QLORA_OK) return rc;
     }
@@ -584,5 +619,14 @@ int qlora_device_status(int reset) {
 }
 
 int qlora_last_path(void) { return t_last_path; }
+
+long long qlora_launch_count(void) { return g_launches.load(); }
+
+int qlora_set_kernel_events(void* before, void* after) {
+    if ((before == nullptr) != (after == nullptr)) return QLORA_ERR_NULL;
+    t_ev_before = static_cast<cudaEvent_t>(before);
+    t_ev_after = static_cast<cudaEvent_t>(after);
+    return QLORA_OK;
+}
 
 }  // extern "C"

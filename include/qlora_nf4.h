@@ -168,6 +168,15 @@ QLORA_API int qlora_device_status(int reset);
  * GEMV path, 2 = tcgen05 fused dequant-GEMM path. */
 QLORA_API int qlora_last_path(void);
 
+/* Measurement hooks (no counterpart on the pages; used by benchmarks).
+ * qlora_launch_count: number of kernels this library has launched in this
+ * process so far (all threads).  qlora_set_kernel_events: the next
+ * qlora_linear_fwd / qlora_linear_bwd call on this thread records `before`
+ * (a cudaEvent_t) on its stream right before its fused dequant-GEMM kernel
+ * and `after` right after it, then forgets both; pass NULL, NULL to clear. */
+QLORA_API long long qlora_launch_count(void);
+QLORA_API int qlora_set_kernel_events(void* before, void* after);
+
 #ifdef __cplusplus
 }
 #endif
