@@ -1,0 +1,471 @@
+#!/usr/bin/env python
+"""Benchmark of the QLoRA NF4 linear layer on B200.
+
+Default workload: the 7 projections of a Llama-7B-shaped decoder block
+(q, k, v, o 4096x4096; gate, up 4096->11008; down 11008->4096), frozen base
+weights in NF4 with double-quantized constants, 2048 tokens, LoRA r=16,
+alpha=32.  One step = forward + backward of all 7 projections through the
+C ABI (qlora_linear_fwd with T kept, qlora_linear_bwd with that T): the
+dequantization runs inside the fused GEMMs every step; quantization of the
+weights happens once, before timing, as at model load.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload 1..5] [--M m]
+
+Prints one JSON line (rank 0).  With N > 1 (launched by torch.distributed.run)
+every rank runs its own batch of the same workload (data parallel, weak
+scaling) and the adapter gradients dA, dB of all projections are summed over
+the ranks with one NCCL all-reduce per step.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "QLoRA linear fwd+bwd TFLOP/s & NF4 weight-stream GB/s; % of roofline, 1×B200"
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+# dram__bytes_read.sum + dram__bytes_write.sum per launch of the fused
+# dequant-GEMM, from an ncu capture (see profiles/), keyed by the hash of the
+# CUDA sources it was taken on; null once the kernel sources change.
+TRAFFIC = {}
+
+
+def src_hash() -> str:
+    h = hashlib.sha1()
+    d = os.path.join(ROOT, "bit_nf4_quantized_quant_b200", "csrc")
+    for f in sorted(os.listdir(d)):
+        with open(os.path.join(d, f), "rb") as fh:
+            h.update(f.encode())
+            h.update(fh.read())
+    return h.hexdigest()[:12]
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(PEAKS_FALLBACK), "fallback"
+
+
+# ---------------------------------------------------------------------------
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower().startswith("active")})
+        loaded = [v for v in sm if mx and v >= 0.5 * max(mx)] or sm
+        return {"sm_mhz": statistics.median(loaded) if loaded else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons, "samples": len(rows)}
+
+
+# ---------------------------------------------------------------------------
+def flops_fwd_bwd(M, N, K, r):
+    # fwd: 2MNK + 2MKr (T) + 2MNr (up); bwd: 2MNK (dX) + 2MKr (U A) + 2MNr (U) + 2MKr (dA) + 2MNr (dB)
+    return 4 * M * N * K + 6 * M * r * (K + N)
+
+
+def main_kernel_flops(M, N, K, r):
+    """Algorithmic flops of the two fused dequant-GEMM launches (fwd, bwd) of one projection."""
+    return 2 * M * N * K + 2 * M * N * r, 2 * M * N * K + 2 * M * K * r
+
+
+def nf4_bytes(N, K):
+    nb = N * K // 64
+    return N * K // 2 + nb + 8 * math.ceil(nb / 256)
+
+
+def build_lib():
+    from bit_nf4_quantized_quant_b200 import build as lib_build
+    lib_build.build()
+
+
+# ---------------------------------------------------------------------------
+def run_ours(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+
+    from bit_nf4_quantized_quant_b200 import _ops as ops
+    from bit_nf4_quantized_quant_b200 import inputs
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    wl = inputs.WORKLOADS[args.workload]
+    M = args.M or (wl.Ms[-1] if wl.Ms else 0)
+    r, s = wl.r, wl.scaling
+    projs = wl.projections
+    peaks, peak_src = load_peaks()
+
+    # ---- setup: weights quantized once, inputs resident in HBM
+    layers = []
+    for i, p in enumerate(projs):
+        W = inputs.layer_weight(wl, i, device=dev)
+        w = ops.nf4_quantize_dq(W)
+        del W
+        X, A, B, dY = inputs.layer_inputs(wl, i, M, device=dev)
+        if world > 1:   # each rank its own batch
+            X = inputs.normal(inputs.seed_of(wl.index, i, inputs.ROLE_X) + 7919 * rank, (M, p.K), 1.0, dev)
+            dY = inputs.normal(inputs.seed_of(wl.index, i, inputs.ROLE_DY) + 7919 * rank, (M, p.N), 1.0, dev)
+        L = dict(p=p, w=w, X=X, A=A, B=B, dY=dY,
+                 Y=torch.empty((M, p.N), dtype=torch.bfloat16, device=dev),
+                 T=torch.empty((M, r), dtype=torch.bfloat16, device=dev),
+                 dX=torch.empty((M, p.K), dtype=torch.bfloat16, device=dev))
+        layers.append(L)
+    # adapter gradients of all projections in one flat buffer (one all-reduce per step)
+    sizes = [(r * L["p"].K, L["p"].N * r) for L in layers]
+    gbuf = torch.empty(sum(a + b for a, b in sizes), dtype=torch.bfloat16, device=dev)
+    off = 0
+    for L, (na, nb) in zip(layers, sizes):
+        L["dA"] = gbuf[off:off + na].view(r, L["p"].K)
+        off += na
+        L["dB"] = gbuf[off:off + nb].view(L["p"].N, r)
+        off += nb
+    ws = torch.empty(max(ops.qlora_workspace_bytes(M, L["p"].N, L["p"].K, r) for L in layers), dtype=torch.uint8,
+                     device=dev)
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream()
+
+    def step(events=None):
+        for j, L in enumerate(layers):
+            if events is not None:
+                ops.qlora_set_kernel_events(*events[2 * j])
+            ops.qlora_linear_fwd(L["X"], L["w"], L["A"], L["B"], s, Y=L["Y"], T_out=L["T"], ws=ws)
+            if events is not None:
+                ops.qlora_set_kernel_events(*events[2 * j + 1])
+            ops.qlora_linear_bwd(L["X"], L["dY"], L["w"], L["A"], L["B"], s, T=L["T"], dX=L["dX"], dA=L["dA"],
+                                 dB=L["dB"], ws=ws)
+        if world > 1:
+            dist.all_reduce(gbuf)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+
+    # ---- timed region
+    kev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+            for _ in range(2 * len(layers))] for _ in range(args.steps)]
+    for evs in kev:                 # torch creates the CUDA events lazily: record once so they exist
+        for a, b in evs:
+            a.record(stream)
+            b.record(stream)
+    torch.cuda.synchronize()
+    clocks = ClockSampler(local_rank)
+    clocks.start()
+    launches0 = ops.qlora_launch_count()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    t0.record(stream)
+    for k in range(args.steps):
+        step(kev[k])
+    t1.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    launches = ops.qlora_launch_count() - launches0
+    clk = clocks.stop()
+    ms = t0.elapsed_time(t1)
+    if world > 1:
+        tt = torch.tensor([ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        ms = float(tt.item())
+    assert ops.qlora_device_status() == 0, "device-side wait timed out"
+    ms_per_step = ms / args.steps
+
+    flops_step = sum(flops_fwd_bwd(M, L["p"].N, L["p"].K, r) for L in layers)
+    bytes_step = sum(2 * nf4_bytes(L["p"].N, L["p"].K) for L in layers)
+    # roofline of the dominant kernel (the fused dequant-GEMM), from its own launch events
+    kflops, kms, nlaunch = 0.0, 0.0, 0
+    for k in range(args.steps):
+        for j, L in enumerate(layers):
+            f_fwd, f_bwd = main_kernel_flops(M, L["p"].N, L["p"].K, r)
+            for h, f in ((0, f_fwd), (1, f_bwd)):
+                a, b = kev[k][2 * j + h]
+                kms += a.elapsed_time(b)
+                kflops += f
+                nlaunch += 1
+    small = M <= 32
+    if small:
+        kbytes = sum(2 * nf4_bytes(L["p"].N, L["p"].K) for L in layers) * args.steps
+        achieved = kbytes / (kms * 1e-3) / 1e9
+        peak = peaks["hbm_gbs"]
+        roof = {"bound": "hbm", "unit": "GB/s"}
+    else:
+        achieved = kflops / (kms * 1e-3) / 1e12
+        peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
+        roof = {"bound": "tensor", "unit": "TFLOP/s"}
+    tr = TRAFFIC.get(f"workload{args.workload}_M{M}")
+    roof.update({"achieved": round(achieved, 2), "peak": peak, "frac": round(achieved / peak, 4),
+                 "traffic": tr["bytes_per_launch"] if tr and tr.get("src") == src_hash() else None,
+                 "peak_source": f"{peak_src} ({'hbm copy' if small else 'cuBLAS bf16 sustained'})",
+                 "kernel": "k_fwd_small/k_bwd_small" if small else "k_tc_gemm (fwd + bwd dX)",
+                 "launches_timed": nlaunch, "avg_launch_us": round(kms / nlaunch * 1e3, 2)})
+
+    if small:
+        value = bytes_step * world / (ms_per_step * 1e-3) / 1e9
+        unit = "GB/s"
+    else:
+        value = flops_step * world / (ms_per_step * 1e-3) / 1e12
+        unit = "TFLOP/s"
+
+    # ---- end to end through the C ABI with host buffers: H2D of X, dY, D2H of Y, dX, dA, dB each step
+    hX = [torch.empty_like(L["X"], device="cpu").pin_memory() for L in layers]
+    hdY = [torch.empty_like(L["dY"], device="cpu").pin_memory() for L in layers]
+    for h, L in zip(hX, layers):
+        h.copy_(L["X"])
+    for h, L in zip(hdY, layers):
+        h.copy_(L["dY"])
+    hout = [[torch.empty_like(L[k], device="cpu").pin_memory() for k in ("Y", "dX")] for L in layers]
+    hg = torch.empty_like(gbuf, device="cpu").pin_memory()
+    h2d = sum(h.numel() * 2 for h in hX) + sum(h.numel() * 2 for h in hdY)
+    d2h = sum(o.numel() * 2 for os_ in hout for o in os_) + hg.numel() * 2
+
+    def e2e_step():
+        for j, L in enumerate(layers):
+            L["X"].copy_(hX[j], non_blocking=True)
+            L["dY"].copy_(hdY[j], non_blocking=True)
+            ops.qlora_linear_fwd(L["X"], L["w"], L["A"], L["B"], s, Y=L["Y"], T_out=L["T"], ws=ws)
+            ops.qlora_linear_bwd(L["X"], L["dY"], L["w"], L["A"], L["B"], s, T=L["T"], dX=L["dX"], dA=L["dA"],
+                                 dB=L["dB"], ws=ws)
+            hout[j][0].copy_(L["Y"], non_blocking=True)
+            hout[j][1].copy_(L["dX"], non_blocking=True)
+        if world > 1:
+            dist.all_reduce(gbuf)
+        hg.copy_(gbuf, non_blocking=True)
+
+    for _ in range(max(1, args.warmup // 2)):
+        e2e_step()
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    e0.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ems = e0.elapsed_time(e1)
+    if world > 1:
+        tt = torch.tensor([ems], device=dev, dtype=torch.float64)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        ems = float(tt.item())
+    e2e_val = (flops_step if not small else bytes_step) * world / (ems / args.steps * 1e-3) / (1e12 if not small else 1e9)
+
+    cfg = {"workload": wl.name, "projections": [f"{p.name} {p.N}x{p.K}" for p in projs], "M_per_gpu": M,
+           "global_batch_tokens": M * world, "r": r, "alpha": wl.alpha, "weights": "NF4 + double-quant (64/256)",
+           "step": "qlora_linear_fwd + qlora_linear_bwd for every projection" +
+                   (" + NCCL all-reduce of dA,dB" if world > 1 else ""),
+           "l2": f"inputs larger than L2: {(bytes_step / 2 + sum(L['X'].numel() + L['dY'].numel() for L in layers) * 2) / 1e6:.0f} MB touched per step",
+           "parallelism": f"dp{world}"}
+    out = {"metric": METRIC, "value": round(value, 3), "unit": unit, "n_gpus": world, "steps": args.steps,
+           "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4), "higher_is_better": True,
+           "scaling": "weak", "vs_baseline": None, "dtype": "bf16 (NF4 weights, fp32 accumulate)",
+           "data": "synthetic (seeded)", "config": cfg, "roofline": roof,
+           "e2e": {"value": round(e2e_val, 3), "unit": unit, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+           "gpu_launches": launches, "clocks": clk}
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        out["cpu_baseline"] = cpu_baseline(wl, M, budget_s=args.cpu_seconds)
+    return out
+
+
+# ---------------------------------------------------------------------------
+def _threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info()]
+        return max(n + [1])
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def oracle_sample_step(wl, proj, rows, state):
+    """One bounded sample of a step on the CPU oracle: dequantize the
+    projection's full weight, then fp64 forward + backward on `rows` tokens.
+    Returns the algorithmic flops of the sampled rows."""
+    import numpy as np
+
+    import oracle
+    from bit_nf4_quantized_quant_b200 import inputs
+
+    p = wl.projections[proj]
+    if proj not in state:
+        W = inputs.layer_weight(wl, proj)
+        q = oracle.quantize_dq(inputs.bf16_bits(W))
+        X, A, B, dY = inputs.layer_inputs(wl, proj, rows)
+        state[proj] = (q, inputs.to_f64(X), inputs.to_f64(A), inputs.to_f64(B), inputs.to_f64(dY))
+    q, X, A, B, dY = state[proj]
+    Wd = oracle.bf16_to_f32(oracle.dequant(q)).astype(np.float64)
+    oracle.linear_fwd(X, Wd, A, B, wl.scaling)
+    oracle.linear_bwd(X, dY, Wd, A, B, wl.scaling)
+    return flops_fwd_bwd(rows, p.N, p.K, wl.r)
+
+
+def _distinct_shapes(wl):
+    seen, out = set(), []
+    for i, p in enumerate(wl.projections):
+        if (p.N, p.K) not in seen:
+            seen.add((p.N, p.K))
+            out.append(i)
+    return out
+
+
+def _sample_value(wl, M, projs_done, flops, dt):
+    if M <= 32:
+        b = sum(2 * nf4_bytes(wl.projections[i].N, wl.projections[i].K) for i in projs_done)
+        return b / dt / 1e9, "GB/s"
+    return flops / dt / 1e12, "TFLOP/s"
+
+
+def cpu_baseline(wl, M, budget_s=20.0):
+    """The oracle, as it stands, on the host cores over a bounded sample."""
+    rows = min(64, max(1, M))
+    shapes = _distinct_shapes(wl)
+    state = {}
+    for i in shapes:                               # quantize + inputs: load time, untimed
+        oracle_sample_step(wl, i, rows, state)
+    t0 = time.perf_counter()
+    flops, done = 0, []
+    while True:
+        i = shapes[len(done) % len(shapes)]
+        flops += oracle_sample_step(wl, i, rows, state)
+        done.append(i)
+        if len(done) >= len(shapes) and time.perf_counter() - t0 > budget_s / 2:
+            break
+    dt = time.perf_counter() - t0
+    v, unit = _sample_value(wl, M, done, flops, dt)
+    return {"value": round(v, 6), "unit": unit, "cores": _threads(), "kind": "oracle",
+            "sample": f"{len(done)} projection passes over the {len(shapes)} distinct shapes: oracle dequant of the "
+                      f"full NF4 weight (C, 1 thread) + fp64 fwd+bwd (numpy) on {rows} of {M} tokens; {dt:.1f} s"}
+
+
+def run_reference(args):
+    """The oracle as the reference arm: host cores, one bounded sample per step."""
+    from bit_nf4_quantized_quant_b200 import inputs
+    wl = inputs.WORKLOADS[args.workload]
+    M = args.M or (wl.Ms[-1] if wl.Ms else 0)
+    rows = min(64, max(1, M))
+    shapes = _distinct_shapes(wl)
+    state = {}
+    for i in shapes:
+        oracle_sample_step(wl, i, rows, state)
+    for k in range(args.warmup):
+        oracle_sample_step(wl, shapes[k % len(shapes)], rows, state)
+    t0 = time.perf_counter()
+    flops, done = 0, []
+    for k in range(args.steps):
+        i = shapes[k % len(shapes)]
+        flops += oracle_sample_step(wl, i, rows, state)
+        done.append(i)
+    dt = time.perf_counter() - t0
+    value, unit = _sample_value(wl, M, done, flops, dt)
+    sample = (f"each step: one projection shape (rotating over {len(shapes)}): oracle dequant of its full NF4 "
+              f"weight + fp64 fwd+bwd on {rows} of {M} tokens")
+    return {"impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": unit, "n_gpus": 1,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(dt / args.steps * 1e3, 3),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64 (oracle)",
+            "data": "synthetic (seeded)", "config": {"workload": wl.name, "M": M, "r": wl.r, "alpha": wl.alpha},
+            "cpu_baseline": {"value": round(value, 6), "unit": unit, "cores": _threads(), "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": round(value, 6), "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", type=int, default=3, choices=[1, 2, 3, 4])
+    ap.add_argument("--M", type=int, default=0, help="tokens per GPU (default: the workload's largest)")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=20.0)
+    args = ap.parse_args()
+    args.warmup = max(3, args.warmup)
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args)), flush=True)
+        return
+
+    import torch
+    import torch.distributed as dist
+    if world > 1:
+        import datetime
+        os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    build_lib()
+    try:
+        out = run_ours(args, rank, world, local_rank)
+        if rank == 0:
+            print(json.dumps(out), flush=True)
+    finally:
+        if world > 1:
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()
