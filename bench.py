@@ -128,6 +128,30 @@ def nf4_bytes(N, K):
     return N * K // 2 + nb + 8 * math.ceil(nb / 256)
 
 
+def rank_batch(wl, i, M, rank, world, device):
+    """Rank-local activations X [M, K] and upstream gradient dY [M, N] of projection i
+    (data parallel: every rank draws its own batch; rank 0 of a 1-GPU run draws the
+    workload's canonical inputs)."""
+    from bit_nf4_quantized_quant_b200 import inputs
+    p = wl.projections[i]
+    if world == 1:
+        X, _, _, dY = inputs.layer_inputs(wl, i, M, device=device)
+        return X, dY
+    X = inputs.normal(inputs.seed_of(wl.index, i, inputs.ROLE_X) + 7919 * rank, (M, p.K), 1.0, device)
+    dY = inputs.normal(inputs.seed_of(wl.index, i, inputs.ROLE_DY) + 7919 * rank, (M, p.N), 1.0, device)
+    return X, dY
+
+
+def grad_layout(shapes, r):
+    """Offsets of dA [r, K] and dB [N, r] of every projection in the flat gradient
+    buffer that is all-reduced once per step; returns ([(offA, offB)], total)."""
+    offs, off = [], 0
+    for N, K in shapes:
+        offs.append((off, off + r * K))
+        off += r * K + N * r
+    return offs, off
+
+
 def build_lib():
     from bit_nf4_quantized_quant_b200 import build as lib_build
     lib_build.build()
@@ -149,45 +173,55 @@ def run_ours(args, rank, world, local_rank):
     projs = wl.projections
     peaks, peak_src = load_peaks()
 
-    # ---- setup: weights quantized once, inputs resident in HBM
+    bwd = wl.backward
+    small = M <= 32
+    # ---- setup: weights quantized once, inputs resident in HBM.  For the
+    # memory-bound sizes the weight set is replicated so that one rotation
+    # through it streams more than twice the L2 capacity from HBM.
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    wset = sum(nf4_bytes(p.N, p.K) for p in projs)
+    copies = max(1, math.ceil(2 * l2 / wset)) if small else 1
     layers = []
     for i, p in enumerate(projs):
         W = inputs.layer_weight(wl, i, device=dev)
         w = ops.nf4_quantize_dq(W)
+        ws_copies = [w] + [ops.nf4_quantize_dq(W) for _ in range(copies - 1)]
         del W
-        X, A, B, dY = inputs.layer_inputs(wl, i, M, device=dev)
-        if world > 1:   # each rank its own batch
-            X = inputs.normal(inputs.seed_of(wl.index, i, inputs.ROLE_X) + 7919 * rank, (M, p.K), 1.0, dev)
-            dY = inputs.normal(inputs.seed_of(wl.index, i, inputs.ROLE_DY) + 7919 * rank, (M, p.N), 1.0, dev)
-        L = dict(p=p, w=w, X=X, A=A, B=B, dY=dY,
+        _, A, B, _ = inputs.layer_inputs(wl, i, M, device=dev, with_dy=False)
+        X, dY = rank_batch(wl, i, M, rank, world, dev)
+        L = dict(p=p, w=w, wc=ws_copies, X=X, A=A, B=B, dY=dY,
                  Y=torch.empty((M, p.N), dtype=torch.bfloat16, device=dev),
                  T=torch.empty((M, r), dtype=torch.bfloat16, device=dev),
                  dX=torch.empty((M, p.K), dtype=torch.bfloat16, device=dev))
         layers.append(L)
     # adapter gradients of all projections in one flat buffer (one all-reduce per step)
-    sizes = [(r * L["p"].K, L["p"].N * r) for L in layers]
-    gbuf = torch.empty(sum(a + b for a, b in sizes), dtype=torch.bfloat16, device=dev)
-    off = 0
-    for L, (na, nb) in zip(layers, sizes):
-        L["dA"] = gbuf[off:off + na].view(r, L["p"].K)
-        off += na
-        L["dB"] = gbuf[off:off + nb].view(L["p"].N, r)
-        off += nb
+    offs, total = grad_layout([(L["p"].N, L["p"].K) for L in layers], r)
+    gbuf = torch.empty(total, dtype=torch.bfloat16, device=dev)
+    for L, (oa, ob) in zip(layers, offs):
+        L["dA"] = gbuf[oa:oa + r * L["p"].K].view(r, L["p"].K)
+        L["dB"] = gbuf[ob:ob + L["p"].N * r].view(L["p"].N, r)
     ws = torch.empty(max(ops.qlora_workspace_bytes(M, L["p"].N, L["p"].K, r) for L in layers), dtype=torch.uint8,
                      device=dev)
     torch.cuda.synchronize()
     stream = torch.cuda.current_stream()
 
+    it = [0]
+
     def step(events=None):
+        c = it[0] % copies
+        it[0] += 1
         for j, L in enumerate(layers):
+            w = L["wc"][c]
             if events is not None:
                 ops.qlora_set_kernel_events(*events[2 * j])
-            ops.qlora_linear_fwd(L["X"], L["w"], L["A"], L["B"], s, Y=L["Y"], T_out=L["T"], ws=ws)
+            ops.qlora_linear_fwd(L["X"], w, L["A"], L["B"], s, Y=L["Y"], T_out=L["T"], ws=ws)
+            if not bwd:
+                continue
             if events is not None:
                 ops.qlora_set_kernel_events(*events[2 * j + 1])
-            ops.qlora_linear_bwd(L["X"], L["dY"], L["w"], L["A"], L["B"], s, T=L["T"], dX=L["dX"], dA=L["dA"],
+            ops.qlora_linear_bwd(L["X"], L["dY"], w, L["A"], L["B"], s, T=L["T"], dX=L["dX"], dA=L["dA"],
                                  dB=L["dB"], ws=ws)
-        if world > 1:
+        if world > 1 and bwd:
             dist.all_reduce(gbuf)
 
     for _ in range(args.warmup):
@@ -212,10 +246,12 @@ def run_ours(args, rank, world, local_rank):
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
+    torch.cuda.nvtx.range_push("timed")
     t0.record(stream)
     for k in range(args.steps):
         step(kev[k])
     t1.record(stream)
+    torch.cuda.nvtx.range_pop()
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
@@ -229,21 +265,34 @@ def run_ours(args, rank, world, local_rank):
     assert ops.qlora_device_status() == 0, "device-side wait timed out"
     ms_per_step = ms / args.steps
 
-    flops_step = sum(flops_fwd_bwd(M, L["p"].N, L["p"].K, r) for L in layers)
-    bytes_step = sum(2 * nf4_bytes(L["p"].N, L["p"].K) for L in layers)
+    npass = 2 if bwd else 1
+    flops_step = sum(flops_fwd_bwd(M, L["p"].N, L["p"].K, r) if bwd else
+                     2 * M * L["p"].N * L["p"].K + 2 * M * r * (L["p"].K + L["p"].N) for L in layers)
+    # algorithmic HBM bytes of one step: the NF4 weight once per pass, plus the
+    # activations, adapters and outputs each pass reads or writes once
+    bytes_step = 0
+    for L in layers:
+        N_, K_ = L["p"].N, L["p"].K
+        bytes_step += npass * nf4_bytes(N_, K_) + 2 * (M * K_ + r * K_ + N_ * r + M * N_)      # fwd: X, A, B, Y
+        if bwd:
+            bytes_step += 2 * (M * N_ + M * K_ + M * K_ + r * K_ + N_ * r + M * r)           # dY, X, dX, dA, dB, T
     # roofline of the dominant kernel (the fused dequant-GEMM), from its own launch events
     kflops, kms, nlaunch = 0.0, 0.0, 0
+    kbytes = 0
     for k in range(args.steps):
         for j, L in enumerate(layers):
-            f_fwd, f_bwd = main_kernel_flops(M, L["p"].N, L["p"].K, r)
-            for h, f in ((0, f_fwd), (1, f_bwd)):
+            N_, K_ = L["p"].N, L["p"].K
+            f_fwd, f_bwd = main_kernel_flops(M, N_, K_, r)
+            # the small-M kernels read the NF4 weight and the activations and write their output once
+            b_fwd = nf4_bytes(N_, K_) + 2 * (M * K_ + M * N_)
+            b_bwd = nf4_bytes(N_, K_) + 2 * (M * N_) + 4 * M * K_
+            for h, f, bb in ((0, f_fwd, b_fwd), (1, f_bwd, b_bwd))[:npass]:
                 a, b = kev[k][2 * j + h]
                 kms += a.elapsed_time(b)
                 kflops += f
+                kbytes += bb
                 nlaunch += 1
-    small = M <= 32
     if small:
-        kbytes = sum(2 * nf4_bytes(L["p"].N, L["p"].K) for L in layers) * args.steps
         achieved = kbytes / (kms * 1e-3) / 1e9
         peak = peaks["hbm_gbs"]
         roof = {"bound": "hbm", "unit": "GB/s"}
@@ -258,6 +307,7 @@ def run_ours(args, rank, world, local_rank):
                  "kernel": "k_fwd_small/k_bwd_small" if small else "k_tc_gemm (fwd + bwd dX)",
                  "launches_timed": nlaunch, "avg_launch_us": round(kms / nlaunch * 1e3, 2)})
 
+    roof["weight_copies_rotated"] = copies
     if small:
         value = bytes_step * world / (ms_per_step * 1e-3) / 1e9
         unit = "GB/s"
@@ -274,21 +324,23 @@ def run_ours(args, rank, world, local_rank):
         h.copy_(L["dY"])
     hout = [[torch.empty_like(L[k], device="cpu").pin_memory() for k in ("Y", "dX")] for L in layers]
     hg = torch.empty_like(gbuf, device="cpu").pin_memory()
-    h2d = sum(h.numel() * 2 for h in hX) + sum(h.numel() * 2 for h in hdY)
-    d2h = sum(o.numel() * 2 for os_ in hout for o in os_) + hg.numel() * 2
+    h2d = sum(h.numel() * 2 for h in hX) + (sum(h.numel() * 2 for h in hdY) if bwd else 0)
+    d2h = sum(os_[0].numel() * 2 + (os_[1].numel() * 2 if bwd else 0) for os_ in hout) + (hg.numel() * 2 if bwd else 0)
 
     def e2e_step():
         for j, L in enumerate(layers):
             L["X"].copy_(hX[j], non_blocking=True)
             L["dY"].copy_(hdY[j], non_blocking=True)
             ops.qlora_linear_fwd(L["X"], L["w"], L["A"], L["B"], s, Y=L["Y"], T_out=L["T"], ws=ws)
-            ops.qlora_linear_bwd(L["X"], L["dY"], L["w"], L["A"], L["B"], s, T=L["T"], dX=L["dX"], dA=L["dA"],
-                                 dB=L["dB"], ws=ws)
             hout[j][0].copy_(L["Y"], non_blocking=True)
-            hout[j][1].copy_(L["dX"], non_blocking=True)
-        if world > 1:
+            if bwd:
+                ops.qlora_linear_bwd(L["X"], L["dY"], L["w"], L["A"], L["B"], s, T=L["T"], dX=L["dX"],
+                                     dA=L["dA"], dB=L["dB"], ws=ws)
+                hout[j][1].copy_(L["dX"], non_blocking=True)
+        if world > 1 and bwd:
             dist.all_reduce(gbuf)
-        hg.copy_(gbuf, non_blocking=True)
+        if bwd:
+            hg.copy_(gbuf, non_blocking=True)
 
     for _ in range(max(1, args.warmup // 2)):
         e2e_step()
@@ -313,7 +365,8 @@ def run_ours(args, rank, world, local_rank):
            "global_batch_tokens": M * world, "r": r, "alpha": wl.alpha, "weights": "NF4 + double-quant (64/256)",
            "step": "qlora_linear_fwd + qlora_linear_bwd for every projection" +
                    (" + NCCL all-reduce of dA,dB" if world > 1 else ""),
-           "l2": f"inputs larger than L2: {(bytes_step / 2 + sum(L['X'].numel() + L['dY'].numel() for L in layers) * 2) / 1e6:.0f} MB touched per step",
+           "l2": (f"inputs larger than L2: {bytes_step / 1e6:.0f} MB of algorithmic traffic per step" if not small else
+                  f"weights rotated over {copies} copies ({copies * wset / 1e6:.0f} MB > 2x L2)"),
            "parallelism": f"dp{world}"}
     out = {"metric": METRIC, "value": round(value, 3), "unit": unit, "n_gpus": world, "steps": args.steps,
            "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4), "higher_is_better": True,
@@ -327,6 +380,106 @@ def run_ours(args, rank, world, local_rank):
 
 
 # ---------------------------------------------------------------------------
+def run_bulk(args, rank, world, local_rank):
+    """Workload 5: quantize + double-quantize all 224 tensors of a 32-layer
+    7B-shaped model, then dequantize them all back (one step = both passes)."""
+    import torch
+
+    from bit_nf4_quantized_quant_b200 import _ops as ops
+    from bit_nf4_quantized_quant_b200 import inputs
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    wl = inputs.WORKLOADS[5]
+    peaks, peak_src = load_peaks()
+    layers = args.layers or wl.repeat
+    tensors = []
+    for c in range(layers):
+        for i, p in enumerate(wl.projections):
+            W = inputs.layer_weight(wl, i, device=dev, copy=c + 1000 * rank)
+            tensors.append((W, ops.NF4Weight.empty(p.N, p.K, dev), torch.empty_like(W)))
+    params = sum(W.numel() for W, _, _ in tensors)
+    nb = sum(w.codes.numel() for _, w, _ in tensors)
+    ng = sum(w.scale.numel() for _, w, _ in tensors)
+    qbytes = params // 2 + nb + 8 * ng
+    stream = torch.cuda.current_stream()
+
+    def step(ev=None):
+        for j, (W, w, out) in enumerate(tensors):
+            if ev: ev[0][j][0].record(stream)
+            ops.nf4_quantize_dq(W, out=w)
+            if ev: ev[0][j][1].record(stream)
+        for j, (W, w, out) in enumerate(tensors):
+            if ev: ev[1][j][0].record(stream)
+            ops.nf4_dequant(w, out=out)
+            if ev: ev[1][j][1].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    ev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in tensors]
+          for _ in range(2)]
+    clocks = ClockSampler(local_rank)
+    clocks.start()
+    l0 = ops.qlora_launch_count()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    torch.cuda.nvtx.range_push("timed")
+    t0.record(stream)
+    for k in range(args.steps):
+        step(ev if k == args.steps - 1 else None)
+    t1.record(stream)
+    torch.cuda.nvtx.range_pop()
+    torch.cuda.synchronize()
+    launches = ops.qlora_launch_count() - l0
+    clk = clocks.stop()
+    assert ops.qlora_device_status() == 0
+    ms = t0.elapsed_time(t1) / args.steps
+    step_bytes = 2 * (2 * params + qbytes)           # quantize: read bf16, write NF4; dequant: the reverse
+    value = step_bytes / (ms * 1e-3) / 1e9
+    tq = sum(a.elapsed_time(b) for a, b in ev[0])
+    td = sum(a.elapsed_time(b) for a, b in ev[1])
+    kq = (2 * params + qbytes) / (tq * 1e-3) / 1e9
+    kd = (2 * params + qbytes) / (td * 1e-3) / 1e9
+    dom = ("k_quantize_dq", kq, tq) if tq >= td else ("k_dequant", kd, td)
+    roof = {"bound": "hbm", "unit": "GB/s", "achieved": round(dom[1], 1), "peak": peaks["hbm_gbs"],
+            "frac": round(dom[1] / peaks["hbm_gbs"], 4), "traffic": None,
+            "peak_source": f"{peak_src} (hbm copy)", "kernel": dom[0], "launches_timed": len(tensors),
+            "avg_launch_us": round(dom[2] / len(tensors) * 1e3, 2),
+            "other": {"k_quantize_dq_GBps": round(kq, 1), "k_dequant_GBps": round(kd, 1)}}
+    # e2e: host bf16 weights in, NF4 + dequantized weights out, for one layer (7 tensors) per step
+    hW = [W.cpu().pin_memory() for W, _, _ in tensors[:7]]
+    hout = [torch.empty_like(W, device="cpu").pin_memory() for W, _, _ in tensors[:7]]
+    hq = [(torch.empty_like(w.packed, device="cpu").pin_memory(), torch.empty_like(w.codes, device="cpu").pin_memory())
+          for _, w, _ in tensors[:7]]
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for k in range(args.steps):
+        for j, (W, w, out) in enumerate(tensors[:7]):
+            W.copy_(hW[j], non_blocking=True)
+            ops.nf4_quantize_dq(W, out=w)
+            ops.nf4_dequant(w, out=out)
+            hq[j][0].copy_(w.packed, non_blocking=True)
+            hq[j][1].copy_(w.codes, non_blocking=True)
+            hout[j].copy_(out, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    p7 = sum(W.numel() for W, _, _ in tensors[:7])
+    q7 = sum(w.packed.numel() + w.codes.numel() + 8 * w.scale.numel() for _, w, _ in tensors[:7])
+    e2e = 2 * (2 * p7 + q7) / (e0.elapsed_time(e1) / args.steps * 1e-3) / 1e9
+    return {"metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(ms, 4), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16 -> NF4 + int8/fp32 constants -> bf16", "data": "synthetic (seeded)",
+            "config": {"workload": wl.name, "tensors": len(tensors), "params": params,
+                       "step": "nf4_quantize_dq then nf4_dequant over every tensor",
+                       "l2": f"inputs larger than L2: {step_bytes / 1e9:.1f} GB per step"},
+            "roofline": roof,
+            "e2e": {"value": round(e2e, 1), "unit": "GB/s", "h2d_bytes_per_step": 2 * p7,
+                    "d2h_bytes_per_step": 2 * p7 + sum(w.packed.numel() + w.codes.numel() for _, w, _ in tensors[:7])},
+            "gpu_launches": launches, "clocks": clk}
+
+
 def _threads():
     try:
         from threadpoolctl import threadpool_info
@@ -433,7 +586,8 @@ def main():
     ap.add_argument("--steps", type=int, default=10)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", type=int, default=3, choices=[1, 2, 3, 4])
+    ap.add_argument("--workload", type=int, default=3, choices=[1, 2, 3, 4, 5])
+    ap.add_argument("--layers", type=int, default=0, help="workload 5: number of 7-tensor layers (default 32)")
     ap.add_argument("--M", type=int, default=0, help="tokens per GPU (default: the workload's largest)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=20.0)
@@ -459,7 +613,7 @@ def main():
                                 device_id=torch.device("cuda", local_rank))
     build_lib()
     try:
-        out = run_ours(args, rank, world, local_rank)
+        out = run_bulk(args, rank, world, local_rank) if args.workload == 5 else run_ours(args, rank, world, local_rank)
         if rank == 0:
             print(json.dumps(out), flush=True)
     finally:

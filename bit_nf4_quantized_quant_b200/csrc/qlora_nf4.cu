@@ -333,7 +333,7 @@ int launch_tc(const nf4dq_weight* w, const uint16_t* act, int64_t M, const uint1
         !make_map_2d(&tmL, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, lact, rp64, M, (uint64_t)rp64 * 2, 64, 128,
                      CU_TENSOR_MAP_SWIZZLE_128B) ||
         !make_map_2d(&tmP, CU_TENSOR_MAP_DATA_TYPE_UINT8, w->packed, K / 2, N, K / 2, BWD ? 128 : 32,
-                     BWD ? 64 : 256, CU_TENSOR_MAP_SWIZZLE_NONE))
+                     BWD ? 64 : 256, BWD ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_32B))
         return QLORA_ERR_LAUNCH;
     tc::Args a{};
     a.codes = w->codes; a.scale = w->scale; a.mean = w->mean;

@@ -6,9 +6,12 @@
 //
 // One persistent CTA per SM walks 128 x 256 output tiles (128 tokens x 256
 // output features), tokens fastest so that the CTAs running at the same time
-// share the same weight tile in L2.  Warp roles (448 threads):
-//   warp 0      TMA producer: activation tiles (128 x 64 bf16, 128-byte
-//               swizzle) and packed NF4 tiles into shared-memory rings;
+// share the same weight tile in L2.  Warp roles (480 threads):
+//   warp 0      TMA producer of the activation tiles (128 x 64 bf16, 128-byte
+//               swizzle);
+//   warp 14     TMA producer of the packed NF4 tiles, on its own 8-deep ring
+//               so that the HBM latency of the weight stream stays off the
+//               MMA's critical path;
 //   warp 1      TMEM allocator and MMA issuer (one thread): 4 MMAs of
 //               128 x 256 x 16 per 64-wide reduction step;
 //   warps 2-9   dequantizers: one thread per 64-weight row-block per step;
@@ -36,13 +39,13 @@ namespace qnf4 {
 namespace tc {
 
 constexpr int BM = 128, BN = 256, BK = 64;
-constexpr int SA = 4;                         // activation ring stages (16 KB)
+constexpr int SA = 3;                         // activation ring stages (16 KB)
 constexpr int SW = 3;                         // dequantized weight ring stages (32 KB)
-constexpr int SP = 4;                         // packed weight ring stages (8 KB)
+constexpr int SP = 8;                         // packed weight ring stages (8 KB)
 constexpr int A_BYTES = BM * BK * 2;          // 16384
 constexpr int W_BYTES = BN * BK * 2;          // 32768
 constexpr int P_BYTES = BN * BK / 2;          // 8192
-constexpr int kThreads = 448;
+constexpr int kThreads = 480;
 constexpr int kDeqThreads = 256;
 constexpr int kEpiThreads = 128;
 constexpr int kTmemCols = 512;
@@ -184,16 +187,38 @@ __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t
     asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
 }
 
+// Which row-block dequantizer thread d (0..255) owns in one reduction step:
+//   forward : tile row d (output feature c0 + d), the step's 64-wide k-block;
+//   backward: reduction row n = 8 (d / 32) + d % 8 of the step's 64 W rows,
+//             output block j = (d / 8) % 4 of the tile's 256 columns.
+// In the backward the 8 lanes of a quarter-warp hold 8 different rows, so
+// their 16-byte stores land in 8 different bank groups of the swizzled tile.
+template <bool BWD>
+__device__ __forceinline__ int deq_row(int d) { return BWD ? 8 * (d >> 5) + (d & 7) : d; }
+template <bool BWD>
+__device__ __forceinline__ int deq_blk(int d) { return BWD ? (d >> 3) & 3 : 0; }
+
 // Byte offset, inside one stage of the weight ring, of 16-byte chunk `ch`
-// (8 consecutive weights of one row-block) for the dequantizer thread d.
-//   forward  (K-major): row d of the 256-row tile, chunk ch of its 128 bytes;
-//   backward (MN-major): W row n = d / 4 of the 64-row step is the reduction
-//     index, block j = d % 4 of the 256 output columns is the MN atom.
+// (8 consecutive weights) of the row-block of thread d:
+//   forward  (K-major, 128-byte rows): row d, chunk ch at position ch ^ (d & 7);
+//   backward (MN-major): atom j = block (8 KB apart), 8-row group n / 8
+//     (1 KB apart), row n % 8 (128 B apart), chunk ch ^ (n % 8).
 template <bool BWD>
 __device__ __forceinline__ uint32_t w_chunk_offset(int d, int ch) {
     if (!BWD) return (uint32_t)(d * 128 + ((ch ^ (d & 7)) << 4));
-    const int n = d >> 2, j = d & 3;
+    const int n = deq_row<true>(d), j = deq_blk<true>(d);
     return (uint32_t)(j * 8192 + (n >> 3) * 1024 + (n & 7) * 128 + ((ch ^ (n & 7)) << 4));
+}
+
+// Byte offsets of the two 16-byte packed chunks of thread d's row-block in a
+// stage of the packed ring.  The forward tile (256 rows x 32 B) is written by
+// TMA with 32-byte swizzle (chunk ^= address bit 7), the backward tile
+// (64 rows x 128 B) with 128-byte swizzle (chunk ^= row % 8).
+template <bool BWD>
+__device__ __forceinline__ uint32_t p_chunk_offset(int d, int c) {
+    if (!BWD) return (uint32_t)(d * 32 + ((c ^ ((d >> 2) & 1)) << 4));
+    const int n = deq_row<true>(d), j = deq_blk<true>(d);
+    return (uint32_t)(n * 128 + (((2 * j + c) ^ (n & 7)) << 4));
 }
 
 // ----------------------------------------------------------------------------
@@ -244,42 +269,42 @@ k_tc_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
     const uint32_t tmem_base = *s_tmem;
 
     if (warp == 0) {
-        // ------------------------------------------------------------ TMA producer
+        // ------------------------------------------------------------ TMA producer: activations
         if (lane == 0) {
-            int sa = 0, pa = 0, sp = 0, pp = 0;
-            int issuedA = 0, issuedP = 0;
+            int sa = 0, pa = 0, issued = 0;
             bool ok = true;
             for (int64_t tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
                 const int m0 = (int)((tile % mtiles) * BM);
-                const int c0 = (int)((tile / mtiles) * BN);
                 for (int step = 0; step < nsteps && ok; ++step) {
                     if (!(ok = mbar_wait(emptyA(sa), pa ^ 1, s_abort))) break;
                     mbar_expect_tx(fullA(sa), A_BYTES);
                     if (step < nks) tma_load_2d(sbase + OFF_A + sa * A_BYTES, &tmA, fullA(sa), step * BK, m0);
                     else tma_load_2d(sbase + OFF_A + sa * A_BYTES, &tmL, fullA(sa), (step - nks) * BK, m0);
-                    ++issuedA;
+                    ++issued;
                     if (++sa == SA) { sa = 0; pa ^= 1; }
-                    if (step < nks) {
-                        if (!(ok = mbar_wait(emptyP(sp), pp ^ 1, s_abort))) break;
-                        mbar_expect_tx(fullP(sp), P_BYTES);
-                        if (!BWD) tma_load_2d(sbase + OFF_P + sp * P_BYTES, &tmP, fullP(sp), step * (BK / 2), c0);
-                        else tma_load_2d(sbase + OFF_P + sp * P_BYTES, &tmP, fullP(sp), c0 / 2, step * BK);
-                        ++issuedP;
-                        if (++sp == SP) { sp = 0; pp ^= 1; }
-                    }
                 }
             }
-            if (!ok) {
-                // wait for the copies this thread put in flight (the last SA / SP of them)
-                for (int i = 1; i <= SA && i <= issuedA; ++i) {
-                    const int k = issuedA - i;
-                    mbar_drain(fullA(k % SA), (k / SA) & 1);
-                }
-                for (int i = 1; i <= SP && i <= issuedP; ++i) {
-                    const int k = issuedP - i;
-                    mbar_drain(fullP(k % SP), (k / SP) & 1);
+            if (!ok)   // wait for the copies this thread put in flight (the last SA of them)
+                for (int i = 1; i <= SA && i <= issued; ++i) mbar_drain(fullA((issued - i) % SA), ((issued - i) / SA) & 1);
+        }
+    } else if (warp == 14) {
+        // ------------------------------------------------------------ TMA producer: packed weights
+        if (lane == 0) {
+            int sp = 0, pp = 0, issued = 0;
+            bool ok = true;
+            for (int64_t tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
+                const int c0 = (int)((tile / mtiles) * BN);
+                for (int step = 0; step < nks && ok; ++step) {
+                    if (!(ok = mbar_wait(emptyP(sp), pp ^ 1, s_abort))) break;
+                    mbar_expect_tx(fullP(sp), P_BYTES);
+                    if (!BWD) tma_load_2d(sbase + OFF_P + sp * P_BYTES, &tmP, fullP(sp), step * (BK / 2), c0);
+                    else tma_load_2d(sbase + OFF_P + sp * P_BYTES, &tmP, fullP(sp), c0 / 2, step * BK);
+                    ++issued;
+                    if (++sp == SP) { sp = 0; pp ^= 1; }
                 }
             }
+            if (!ok)
+                for (int i = 1; i <= SP && i <= issued; ++i) mbar_drain(fullP((issued - i) % SP), ((issued - i) / SP) & 1);
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
@@ -320,70 +345,87 @@ k_tc_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
     } else if (warp < 10) {
         // ------------------------------------------------------------ dequantizers
         const int d = tid - 64;
+        const int drow = deq_row<BWD>(d), dblk = deq_blk<BWD>(d);
         int sw = 0, pw = 0, sp = 0, pp = 0;
         bool ok = true;
+        // block constant inputs of reduction step `st` for this thread, fetched two steps ahead
+        auto fetch = [&](int64_t c0, int st, int& code, float& sc, float& mu) {
+            int64_t n, kb;
+            if (!BWD) { n = c0 + drow; kb = st; }
+            else { n = (int64_t)st * BK + drow; kb = c0 / kBlock + dblk; }
+            code = 0; sc = 0.f; mu = 0.f;
+            if (st < nks && n < a.N && kb < nblk) {
+                const int64_t b = n * nblk + kb;
+                const int64_t g = b >> 8;
+                code = __ldg(a.codes + b);
+                sc = __ldg(a.scale + g);
+                mu = __ldg(a.mean + g);
+            }
+        };
+        // one reduction step; (code, sc, mu) hold this step's block-constant inputs on
+        // entry and are refilled with those of step + 2 (two slots alternate, so the
+        // loads have two steps to land before anything reads the registers)
+        auto do_step = [&](int64_t c0, int step, int& code, float& sc, float& mu) {
+            uint32_t o[8][4];
+            if (step < nks) {
+                const float c = __fmaf_rn((float)code, sc, mu);
+                fetch(c0, step + 2, code, sc, mu);
+                if (!(ok = mbar_wait(fullP(sp), pp, s_abort))) return;
+                uint4 p0, p1;
+                const uint32_t pst = sbase + OFF_P + sp * P_BYTES;
+                const uint32_t src0 = pst + p_chunk_offset<BWD>(d, 0), src1 = pst + p_chunk_offset<BWD>(d, 1);
+                asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(p0.x), "=r"(p0.y), "=r"(p0.z), "=r"(p0.w) : "r"(src0));
+                asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(p1.x), "=r"(p1.y), "=r"(p1.z), "=r"(p1.w) : "r"(src1));
+                mbar_arrive(emptyP(sp));
+                if (++sp == SP) { sp = 0; pp ^= 1; }
+                const BlockTable tb = make_block_table(tab, c);
+                const uint32_t pwd[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
+#pragma unroll
+                for (int ch = 0; ch < 8; ++ch) decode8(tb, pwd[ch], o[ch]);
+            } else {
+                // LoRA step: rows of B (forward) or A (backward), zero beyond r / the output edge
+                const int lc = step - nks;
+                const uint16_t* src;
+                int64_t col0;
+                bool rowok;
+                if (!BWD) {
+                    const int64_t n = c0 + drow;
+                    rowok = n < a.N;
+                    src = a.lora_w + n * a.ldl;
+                    col0 = (int64_t)lc * BK;        // rank index of chunk 0
+                } else {
+                    const int64_t i = (int64_t)lc * BK + drow;
+                    rowok = i < a.r;
+                    src = a.lora_w + i * a.ldl;
+                    col0 = c0 + dblk * 64;          // output column of chunk 0
+                }
+#pragma unroll
+                for (int ch = 0; ch < 8; ++ch) {
+                    const int64_t col = col0 + ch * 8;
+                    const bool v = rowok && (BWD ? (col < a.K) : (col < a.r));
+                    uint4 q = make_uint4(0, 0, 0, 0);
+                    if (v) q = __ldg(reinterpret_cast<const uint4*>(src + col));
+                    o[ch][0] = q.x; o[ch][1] = q.y; o[ch][2] = q.z; o[ch][3] = q.w;
+                }
+            }
+            if (!(ok = mbar_wait(emptyW(sw), pw ^ 1, s_abort))) return;
+            const uint32_t wbase = sbase + OFF_W + sw * W_BYTES;
+#pragma unroll
+            for (int ch = 0; ch < 8; ++ch)
+                st_shared_v4(wbase + w_chunk_offset<BWD>(d, ch), o[ch][0], o[ch][1], o[ch][2], o[ch][3]);
+            fence_proxy_async();
+            mbar_arrive(fullW(sw));
+            if (++sw == SW) { sw = 0; pw ^= 1; }
+        };
         for (int64_t tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
             const int64_t c0 = (tile / mtiles) * BN;
-            for (int step = 0; step < nsteps && ok; ++step) {
-                uint32_t o[8][4];
-                if (step < nks) {
-                    // the block this thread owns in this step
-                    int64_t n, kb;
-                    uint32_t poff;
-                    if (!BWD) { n = c0 + d; kb = step; poff = (uint32_t)(d * 32); }
-                    else { n = (int64_t)step * BK + (d >> 2); kb = c0 / kBlock + (d & 3); poff = (uint32_t)((d >> 2) * 128 + (d & 3) * 32); }
-                    const bool valid = n < a.N && kb < nblk;
-                    float c = 0.f;
-                    if (valid) {
-                        const int64_t b = n * nblk + kb;
-                        const int64_t g = b >> 8;
-                        c = __fmaf_rn((float)__ldg(a.codes + b), __ldg(a.scale + g), __ldg(a.mean + g));
-                    }
-                    if (!(ok = mbar_wait(fullP(sp), pp, s_abort))) break;
-                    uint4 p0, p1;
-                    const uint32_t src = sbase + OFF_P + sp * P_BYTES + poff;
-                    asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(p0.x), "=r"(p0.y), "=r"(p0.z), "=r"(p0.w) : "r"(src));
-                    asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(p1.x), "=r"(p1.y), "=r"(p1.z), "=r"(p1.w) : "r"(src + 16));
-                    mbar_arrive(emptyP(sp));
-                    if (++sp == SP) { sp = 0; pp ^= 1; }
-                    const BlockTable tb = make_block_table(tab, c);
-                    const uint32_t pwd[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
-#pragma unroll
-                    for (int ch = 0; ch < 8; ++ch) decode8(tb, pwd[ch], o[ch]);
-                } else {
-                    // LoRA step: rows of B (forward) or A (backward), zero beyond r / the output edge
-                    const int lc = step - nks;
-                    const uint16_t* src;
-                    int64_t col0;
-                    bool rowok;
-                    if (!BWD) {
-                        const int64_t n = c0 + d;
-                        rowok = n < a.N;
-                        src = a.lora_w + n * a.ldl;
-                        col0 = (int64_t)lc * BK;        // rank index of chunk 0
-                    } else {
-                        const int64_t i = (int64_t)lc * BK + (d >> 2);
-                        rowok = i < a.r;
-                        src = a.lora_w + i * a.ldl;
-                        col0 = c0 + (d & 3) * 64;       // output column of chunk 0
-                    }
-#pragma unroll
-                    for (int ch = 0; ch < 8; ++ch) {
-                        const int64_t col = col0 + ch * 8;
-                        const bool v = rowok && (BWD ? (col < a.K) : (col < a.r));
-                        uint4 q = make_uint4(0, 0, 0, 0);
-                        if (v) q = __ldg(reinterpret_cast<const uint4*>(src + col));
-                        o[ch][0] = q.x; o[ch][1] = q.y; o[ch][2] = q.z; o[ch][3] = q.w;
-                    }
-                }
-                if (!(ok = mbar_wait(emptyW(sw), pw ^ 1, s_abort))) break;
-                const uint32_t wbase = sbase + OFF_W + sw * W_BYTES;
-#pragma unroll
-                for (int ch = 0; ch < 8; ++ch)
-                    st_shared_v4(wbase + w_chunk_offset<BWD>(d, ch), o[ch][0], o[ch][1], o[ch][2], o[ch][3]);
-                fence_proxy_async();
-                mbar_arrive(fullW(sw));
-                if (++sw == SW) { sw = 0; pw ^= 1; }
+            int codeA, codeB;
+            float scA, scB, muA, muB;
+            fetch(c0, 0, codeA, scA, muA);
+            fetch(c0, 1, codeB, scB, muB);
+            for (int step = 0; step < nsteps && ok; step += 2) {
+                do_step(c0, step, codeA, scA, muA);
+                if (ok && step + 1 < nsteps) do_step(c0, step + 1, codeB, scB, muB);
             }
         }
     } else {
