@@ -16,6 +16,7 @@
 #include "small.cuh"
 #include "lora.cuh"
 #include "tc_gemm.cuh"
+#include "tc2_gemm.cuh"
 
 using namespace qnf4;
 
@@ -99,11 +100,7 @@ int check_device(int* sm_count) {
         if (st == 1) {
             // opt in to more than 48 KB of dynamic shared memory, once per device
             const cudaError_t e = [&] {
-                cudaError_t r = cudaFuncSetAttribute(k_fwd_small<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                     fwd_small_smem_bytes<1>());
-                if (r == cudaSuccess) r = cudaFuncSetAttribute(k_fwd_small<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                               fwd_small_smem_bytes<2>());
-                if (r == cudaSuccess) r = cudaFuncSetAttribute(k_bwd_small<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                cudaError_t r = cudaFuncSetAttribute(k_bwd_small<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                                                bwd_small_smem_bytes<1>());
                 if (r == cudaSuccess) r = cudaFuncSetAttribute(k_bwd_small<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                                                bwd_small_smem_bytes<2>());
@@ -137,8 +134,9 @@ struct Plan {
     int64_t kT, kU, kA, kB;         // k per split
     int S_bwd;                      // small-path N splits for dX
     int64_t rows_per_split;
+    int KS, J;                      // small-path forward: K splits, macro-steps per split
     // byte offsets
-    size_t off_part, off_T32, off_U32, off_Tp, off_Ubf, off_sT, off_sU, off_Bp, off_At, total;
+    size_t off_part, off_cnt, off_T32, off_U32, off_Tp, off_Ubf, off_sT, off_sU, off_Bp, off_At, total;
 };
 
 size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
@@ -198,8 +196,19 @@ Plan make_plan(int64_t M, int64_t N, int64_t K, int r, int sms) {
         p.rows_per_split = rps;
         p.S_bwd = (int)cdiv(N, rps);
     }
+    // small-path forward: about 16 resident warps per SM, each owning 8 rows x J macro-steps
+    {
+        const int64_t nms = cdiv(K / kBlock, 4), nrg = cdiv(N, 8);
+        const int64_t slots = 16LL * sms;
+        int64_t ks = (slots + nrg / 2) / nrg;
+        if (ks < 1) ks = 1;
+        if (ks > nms) ks = nms;
+        p.J = (int)cdiv(nms, ks);
+        p.KS = (int)cdiv(nms, p.J);
+    }
     size_t part = 0;
     auto upd = [&](size_t b) { if (b > part) part = b; };
+    if (M <= 32) upd((size_t)p.KS * M * N * 4);          // small-path forward partials
     upd(gemm_part_bytes(M, p.rp, p.zT));
     upd(gemm_part_bytes(M, p.rp, p.zU));
     upd(gemm_part_bytes(2 * p.rp, K, p.zA));
@@ -208,6 +217,7 @@ Plan make_plan(int64_t M, int64_t N, int64_t K, int r, int sms) {
     size_t off = 0;
     auto take = [&](size_t b) { const size_t o = off; off = align256(off + b); return o; };
     p.off_part = take(part);
+    p.off_cnt = take((size_t)cdiv(N, 8) * 4);
     p.off_T32 = take((size_t)M * p.rp * 4);
     p.off_U32 = take((size_t)M * p.rp * 4);
     p.off_Tp = take((size_t)M * 2 * p.rp * 2);     // T hi | lo
@@ -300,6 +310,7 @@ bool make_map_2d(CUtensorMap* m, CUtensorMapDataType dt, const void* ptr, uint64
 }
 
 bool g_tc_attr_set[64];
+int g_pairs[64];            // co-resident SM pairs for the cta_group::2 kernel (0: not available)
 std::mutex g_tc_mu;
 
 int ensure_tc_attrs() {
@@ -310,8 +321,33 @@ int ensure_tc_attrs() {
         if (cudaFuncSetAttribute(tc::k_tc_gemm<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, tc::SMEM_ALLOC) !=
                 cudaSuccess ||
             cudaFuncSetAttribute(tc::k_tc_gemm<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, tc::SMEM_ALLOC) !=
-                cudaSuccess)
+                cudaSuccess ||
+            cudaFuncSetAttribute(tc2::k_tc2_gemm<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 tc2::SMEM_ALLOC) != cudaSuccess ||
+            cudaFuncSetAttribute(tc2::k_tc2_gemm<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 tc2::SMEM_ALLOC) != cudaSuccess)
             return QLORA_ERR_LAUNCH;
+        // pairs of SMs that can hold one cluster each at the same time
+        cudaLaunchConfig_t cfg = {};
+        cudaLaunchAttribute attr;
+        attr.id = cudaLaunchAttributeClusterDimension;
+        attr.val.clusterDim.x = 2; attr.val.clusterDim.y = 1; attr.val.clusterDim.z = 1;
+        cfg.gridDim = dim3(2 * 74, 1, 1);
+        cfg.blockDim = dim3(tc2::kThreads, 1, 1);
+        cfg.dynamicSmemBytes = tc2::SMEM_ALLOC;
+        cfg.attrs = nullptr;
+        cfg.numAttrs = 0;               // the kernel carries its cluster shape (__cluster_dims__)
+        int nclusters = 0;
+        if (cudaOccupancyMaxActiveClusters(&nclusters, tc2::k_tc2_gemm<false>, &cfg) != cudaSuccess) {
+            cudaGetLastError();
+            cfg.attrs = &attr;
+            cfg.numAttrs = 1;
+            if (cudaOccupancyMaxActiveClusters(&nclusters, tc2::k_tc2_gemm<false>, &cfg) != cudaSuccess) {
+                cudaGetLastError();
+                nclusters = 0;
+            }
+        }
+        g_pairs[dev] = nclusters;
         g_tc_attr_set[dev] = true;
     }
     return QLORA_OK;
@@ -348,6 +384,42 @@ int launch_tc(const nf4dq_weight* w, const uint16_t* act, int64_t M, const uint1
     return launch_status();
 }
 
+// The same on SM pairs (cta_group::2), 256 x 256 tiles.
+template <bool BWD>
+int launch_tc2(const nf4dq_weight* w, const uint16_t* act, int64_t M, const uint16_t* lact, int rp64,
+               const uint16_t* lora_w, int64_t ldl, int r, uint16_t* out, int pairs, cudaStream_t st) {
+    const int64_t N = w->N, K = w->K;
+    const int64_t n_red = BWD ? N : K, n_out = BWD ? K : N;
+    CUtensorMap tmA, tmL, tmP;
+    if (!make_map_2d(&tmA, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, act, n_red, M, n_red * 2, 64, 128,
+                     CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_map_2d(&tmL, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, lact, rp64, M, (uint64_t)rp64 * 2, 64, 128,
+                     CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_map_2d(&tmP, CU_TENSOR_MAP_DATA_TYPE_UINT8, w->packed, K / 2, N, K / 2, BWD ? 64 : 32,
+                     BWD ? 64 : 128, BWD ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B))
+        return QLORA_ERR_LAUNCH;
+    tc::Args a{};
+    a.codes = w->codes; a.scale = w->scale; a.mean = w->mean;
+    a.lora_w = lora_w; a.ldl = ldl; a.r = r; a.nlora = (int)cdiv(r, 64);
+    a.out = out; a.M = M; a.N = N; a.K = K; a.n_out = n_out; a.n_red = n_red;
+    const int64_t ntiles = cdiv(M, tc2::BM) * cdiv(n_out, tc2::BN);
+    const int np = (int)(ntiles < pairs ? ntiles : pairs);
+    hook_before(st);
+    tc2::k_tc2_gemm<BWD><<<2 * np, tc2::kThreads, tc2::SMEM_ALLOC, st>>>(tmA, tmL, tmP, a, tables());
+    hook_after(st);
+    note_launch();
+    return launch_status();
+}
+
+// Tokens above this count use the SM-pair kernel.
+constexpr int64_t kPairMinM = 128;
+
+int current_pairs() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
+    return g_pairs[dev];
+}
+
 // Tokens at or below this count take the small-M (GEMV-shaped) kernels.
 constexpr int64_t kSmallMaxM = 32;
 
@@ -361,6 +433,7 @@ int compute_T(const Plan& p, const uint16_t* X, const uint16_t* A, float s, uint
     f.J1 = p.r;
     f.hl = reinterpret_cast<uint16_t*>(ws + p.off_Tp); f.hl_ld = 2 * p.rp; f.hl_off = p.rp;
     f.o2 = reinterpret_cast<uint16_t*>(ws + p.off_sT); f.s2i = p.rp64; f.s2j = 1; f.J2 = p.r; f.J2pad = p.rp64; f.alpha2 = s;
+    f.zero = reinterpret_cast<int*>(ws + p.off_cnt); f.zero_n = cdiv(p.N, 8);
     int rc = run_gemm<true, true>(X, p.K, A, p.K, p.M, p.rp, p.K, p.M, p.r, p.zT, p.kT,
                                   reinterpret_cast<float*>(ws + p.off_part), f, sms, st);
     if (rc != QLORA_OK) return rc;
@@ -463,12 +536,15 @@ int qlora_linear_fwd(const qlora_bf16* X, int64_t M, const nf4dq_weight* w, cons
         SmallFwdArgs a{};
         a.X = X; a.packed = w->packed; a.codes = w->codes; a.scale = w->scale; a.mean = w->mean;
         a.T32 = reinterpret_cast<const float*>(wsb + p.off_T32); a.B = B; a.Y = Y;
-        a.M = M; a.N = w->N; a.K = w->K; a.rp = p.rp; a.r = r; a.s = scaling;
-        const int64_t ntiles = cdiv(w->N, 16);
-        const int grid = (int)(ntiles < 2LL * sms ? ntiles : 2LL * sms);
+        a.part = reinterpret_cast<float*>(wsb + p.off_part);
+        a.counters = reinterpret_cast<int*>(wsb + p.off_cnt);
+        a.M = M; a.N = w->N; a.K = w->K; a.rp = p.rp; a.r = r; a.s = scaling; a.KS = p.KS; a.J = p.J;
+        const int64_t items = cdiv(w->N, 8) * p.KS;
+        const int64_t warps = items < 16LL * sms ? items : 16LL * sms;
+        const int grid = (int)cdiv(warps, kGemvThreads / 32);
         hook_before(st);
-        if (M <= 16) k_fwd_small<1><<<grid, kSmallThreads, fwd_small_smem_bytes<1>(), st>>>(a, tables());
-        else k_fwd_small<2><<<grid, kSmallThreads, fwd_small_smem_bytes<2>(), st>>>(a, tables());
+        if (M <= 16) k_fwd_gemv<1><<<grid, kGemvThreads, 0, st>>>(a, tables());
+        else k_fwd_gemv<2><<<grid, kGemvThreads, 0, st>>>(a, tables());
         hook_after(st);
         note_launch();
         rc = launch_status();
@@ -486,6 +562,15 @@ int qlora_linear_fwd(const qlora_bf16* X, int64_t M, const nf4dq_weight* w, cons
         ldl = p.rp;
     } else if (!aligned16(B)) {
         return QLORA_ERR_ALIGN;
+    }
+    rc = ensure_tc_attrs();
+    if (rc != QLORA_OK) return rc;
+    const int pairs = current_pairs();
+    if (M > kPairMinM && pairs > 0) {
+        rc = launch_tc2<false>(w, X, M, reinterpret_cast<const uint16_t*>(wsb + p.off_sT), p.rp64, lw, ldl, r, Y,
+                               pairs, st);
+        if (rc == QLORA_OK) t_last_path = 3;
+        return rc;
     }
     rc = launch_tc<false>(w, X, M, reinterpret_cast<const uint16_t*>(wsb + p.off_sT), p.rp64, lw, ldl, r, Y, sms, st);
     if (rc == QLORA_OK) t_last_path = 2;
@@ -564,6 +649,15 @@ int qlora_linear_bwd(const qlora_bf16* X, const qlora_bf16* dY, int64_t M, const
     }
     // dX = dY W' + s U A
     if (M > kSmallMaxM) {
+        rc = ensure_tc_attrs();
+        if (rc != QLORA_OK) return rc;
+        const int pairs = current_pairs();
+        if (M > kPairMinM && pairs > 0) {
+            rc = launch_tc2<true>(w, dY, M, reinterpret_cast<const uint16_t*>(wsb + p.off_sU), p.rp64, A, K, r, dX,
+                                  pairs, st);
+            if (rc == QLORA_OK) t_last_path = 3;
+            return rc;
+        }
         rc = launch_tc<true>(w, dY, M, reinterpret_cast<const uint16_t*>(wsb + p.off_sU), p.rp64, A, K, r, dX, sms,
                              st);
         if (rc == QLORA_OK) t_last_path = 2;

@@ -1,0 +1,427 @@
+// tc2_gemm.cuh -- the fused NF4 dequant + GEMM on a pair of SMs
+// (tcgen05.mma.cta_group::2), for M > 128 tokens.
+//
+// Same computation as tc_gemm.cuh (forward Y = X W'^T + s T B^T, backward
+// dX = dY W' + s U A), but a cluster of two CTAs computes one 256-token x
+// 256-output tile with 256 x 256 x 16 MMAs issued by the leader CTA (rank 0):
+//   - each CTA holds its 128 tokens of the activation tile (A operand) and
+//     its 128 output features of the weight tile (B operand) in its own
+//     shared memory, at the same offsets;
+//   - each CTA's TMEM holds the accumulator rows of its own 128 tokens;
+//   - each CTA dequantizes only its half of W' per reduction step, so the
+//     decode work per MMA flop is half that of the single-SM kernel, which is
+//     what bounds the single-SM kernel (its ALU pipe runs ~60% busy at ~32%
+//     tensor activity).
+// Synchronisation across the pair:
+//   - activation tiles of both CTAs are loaded with cta_group::2 TMA whose
+//     transaction bytes complete on the leader's barrier (the leader arms it
+//     for both halves);
+//   - the dequantizers and the epilogue of both CTAs arrive on the leader's
+//     barriers (mapa + release at cluster scope); the leader's waits acquire
+//     at cluster scope;
+//   - MMA completion is multicast to the "empty" and "accumulator full"
+//     barriers of both CTAs (tcgen05.commit ... multicast::cluster, mask 0b11).
+// No TMA load uses multicast.  All waits are bounded as in tc_gemm.cuh; a
+// cluster barrier before TMEM is freed keeps either CTA from leaving while
+// the other may still touch its shared memory.
+#pragma once
+#include <cuda.h>
+#include "common.cuh"
+#include "nf4_decode.cuh"
+#include "tc_gemm.cuh"
+
+namespace qnf4 {
+namespace tc2 {
+
+using tc::Args;
+
+constexpr int BM = 256, BN = 256, BK = 64;       // pair tile
+constexpr int HM = 128, HN = 128;                // per-CTA halves
+constexpr int SA = 5, SW = 5, SP = 8;
+constexpr int A_BYTES = HM * BK * 2;             // 16 KB
+constexpr int W_BYTES = HN * BK * 2;             // 16 KB
+constexpr int P_BYTES = HN * BK / 2;             // 4 KB
+constexpr int kThreads = 480;
+constexpr int kGroupThreads = 128;               // dequantizers per step (one group of two)
+constexpr int kGroupWarps = kGroupThreads / 32;
+constexpr int kEpiWarps = 4;
+constexpr int kTmemCols = 512;
+
+constexpr int OFF_A = 0;
+constexpr int OFF_W = OFF_A + SA * A_BYTES;
+constexpr int OFF_P = OFF_W + SW * W_BYTES;
+constexpr int OFF_BAR = OFF_P + SP * P_BYTES;
+constexpr int NBAR = 2 * SA + 2 * SW + 2 * SP + 4 + 1;
+constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
+constexpr int SMEM_BYTES = OFF_MISC + 16;
+constexpr int SMEM_ALLOC = SMEM_BYTES + 1024;
+
+__device__ __forceinline__ uint32_t cluster_rank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+
+// shared::cluster address of the same variable in CTA `rank` of the cluster
+__device__ __forceinline__ uint32_t mapa(uint32_t saddr, uint32_t rank) {
+    uint32_t d;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(d) : "r"(saddr), "r"(rank));
+    return d;
+}
+
+__device__ __forceinline__ void cluster_sync() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_cl(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok) : "r"(bar), "r"(parity) : "memory");
+    return ok != 0;
+}
+
+// bounded wait, cluster-scope acquire
+__device__ __forceinline__ bool mbar_wait_cl(uint32_t bar, uint32_t parity, volatile int* abort_flag) {
+    if (mbar_try_cl(bar, parity)) return true;
+    const uint64_t t0 = tc::globaltimer();
+    while (true) {
+        if (mbar_try_cl(bar, parity)) return true;
+        if (*abort_flag) return false;
+        if (tc::globaltimer() - t0 > tc::kWaitTimeoutNs) {
+            *abort_flag = 1;
+            report_timeout();
+            return false;
+        }
+    }
+}
+
+__device__ __forceinline__ void mbar_drain_cl(uint32_t bar, uint32_t parity) {
+    const uint64_t t0 = tc::globaltimer();
+    while (!mbar_try_cl(bar, parity)) {
+        if (tc::globaltimer() - t0 > tc::kWaitTimeoutNs) { report_timeout(); return; }
+    }
+}
+
+// arrive on a barrier given by its shared::cluster address (own CTA or the peer)
+__device__ __forceinline__ void mbar_arrive_cl(uint32_t cl_addr) {
+    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cl_addr) : "memory");
+}
+
+__device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap* map, uint32_t cl_bar, int x, int y) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];"
+        ::"r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(cl_bar)
+        : "memory");
+}
+
+__device__ __forceinline__ void tc2_commit_both(uint32_t bar) {
+    asm volatile(
+        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;"
+        ::"r"(bar), "h"((unsigned short)0x3) : "memory");
+}
+
+__device__ __forceinline__ void tc2_commit_local(uint32_t bar) {
+    asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar) : "memory");
+}
+
+__device__ __forceinline__ void tc2_mma(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                        uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}"
+        ::"r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+__host__ __device__ constexpr uint32_t make_idesc2(bool b_mn_major) {
+    return (1u << 4) | (1u << 7) | (1u << 10) | ((b_mn_major ? 1u : 0u) << 16) | ((uint32_t)(BN >> 3) << 17) |
+           ((uint32_t)(BM >> 4) << 24);
+}
+
+// Row-block of dequantizer thread t (0..127 within its group) in one step:
+//   forward : row t of this CTA's 128 W rows, the step's k-block;
+//   backward: reduction row n = 16 (t / 32) + 8 ((t / 16) % 2) + t % 8 of the
+//             step's 64 W rows, output block j = (t / 8) % 2 of this CTA's
+//             128 columns (8 distinct n % 8 per quarter-warp, one j).
+template <bool BWD>
+__device__ __forceinline__ int deq_row(int t) {
+    return BWD ? 16 * (t >> 5) + 8 * ((t >> 4) & 1) + (t & 7) : t;
+}
+template <bool BWD>
+__device__ __forceinline__ int deq_blk(int t) { return BWD ? (t >> 3) & 1 : 0; }
+
+template <bool BWD>
+__device__ __forceinline__ uint32_t w_chunk_offset(int t, int ch) {
+    if (!BWD) return (uint32_t)(t * 128 + ((ch ^ (t & 7)) << 4));
+    const int n = deq_row<true>(t), j = deq_blk<true>(t);
+    return (uint32_t)(j * 8192 + (n >> 3) * 1024 + (n & 7) * 128 + ((ch ^ (n & 7)) << 4));
+}
+
+// packed tile: forward 128 rows x 32 B (32-byte swizzle), backward 64 rows x
+// 64 B (64-byte swizzle: chunk ^= (address / 128) % 4 = (row / 2) % 4)
+template <bool BWD>
+__device__ __forceinline__ uint32_t p_chunk_offset(int t, int c) {
+    if (!BWD) return (uint32_t)(t * 32 + ((c ^ ((t >> 2) & 1)) << 4));
+    const int n = deq_row<true>(t), j = deq_blk<true>(t);
+    return (uint32_t)(n * 64 + (((2 * j + c) ^ ((n >> 1) & 3)) << 4));
+}
+
+template <bool BWD>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
+k_tc2_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmL,
+           const __grid_constant__ CUtensorMap tmP, Args a, NF4Tables tab) {
+    extern __shared__ __align__(1024) uint8_t smem[];
+    uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem) + 1023) & ~(uintptr_t)1023);
+    const uint32_t sbase = smem_u32(base);
+    const uint32_t bar0 = sbase + OFF_BAR;
+    auto fullA = [&](int i) { return bar0 + 8 * i; };
+    auto emptyA = [&](int i) { return bar0 + 8 * (SA + i); };
+    auto fullW = [&](int i) { return bar0 + 8 * (2 * SA + i); };
+    auto emptyW = [&](int i) { return bar0 + 8 * (2 * SA + SW + i); };
+    auto fullP = [&](int i) { return bar0 + 8 * (2 * SA + 2 * SW + i); };
+    auto emptyP = [&](int i) { return bar0 + 8 * (2 * SA + 2 * SW + SP + i); };
+    auto tfull = [&](int i) { return bar0 + 8 * (2 * SA + 2 * SW + 2 * SP + i); };
+    auto tempty = [&](int i) { return bar0 + 8 * (2 * SA + 2 * SW + 2 * SP + 2 + i); };
+    const uint32_t drain = bar0 + 8 * (2 * SA + 2 * SW + 2 * SP + 4);
+    uint32_t* s_tmem = reinterpret_cast<uint32_t*>(base + OFF_MISC);
+    volatile int* s_abort = reinterpret_cast<volatile int*>(base + OFF_MISC + 4);
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const uint32_t crank = cluster_rank();
+    const bool leader = crank == 0;
+    const int64_t pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
+    const int64_t mtiles = cdiv(a.M, BM), ntiles_n = cdiv(a.n_out, BN);
+    const int64_t ntiles = mtiles * ntiles_n;
+    const int nks = (int)cdiv(a.n_red, BK);
+    const int nsteps = nks + a.nlora;
+    const int64_t nblk = a.K / kBlock;
+
+    if (tid == 0) {
+        for (int i = 0; i < SA; ++i) { tc::mbar_init(fullA(i), 1); tc::mbar_init(emptyA(i), 1); }
+        for (int i = 0; i < SW; ++i) { tc::mbar_init(fullW(i), 2 * kGroupWarps); tc::mbar_init(emptyW(i), 1); }
+        for (int i = 0; i < SP; ++i) { tc::mbar_init(fullP(i), 1); tc::mbar_init(emptyP(i), kGroupWarps); }
+        for (int i = 0; i < 2; ++i) { tc::mbar_init(tfull(i), 1); tc::mbar_init(tempty(i), 2 * kEpiWarps); }
+        tc::mbar_init(drain, 1);
+        *s_abort = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    __syncthreads();
+    cluster_sync();                      // the leader's barriers exist before anyone signals them
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(s_tmem)),
+                     "r"(kTmemCols));
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;");
+        tc::tc_fence_before();
+    }
+    __syncthreads();
+    tc::tc_fence_after();
+    const uint32_t tmem_base = *s_tmem;
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ activations (both CTAs)
+        if (lane == 0) {
+            int sa = 0, pa = 0, issued = 0;
+            bool ok = true;
+            for (int64_t tile = pair; tile < ntiles && ok; tile += npairs) {
+                const int m0 = (int)((tile % mtiles) * BM + crank * HM);
+                for (int step = 0; step < nsteps && ok; ++step) {
+                    if (!(ok = tc::mbar_wait(emptyA(sa), pa ^ 1, s_abort))) break;
+                    if (leader) tc::mbar_expect_tx(fullA(sa), 2 * A_BYTES);     // both halves land here
+                    const uint32_t bar = mapa(fullA(sa), 0);
+                    if (step < nks) tma_load_2d_pair(sbase + OFF_A + sa * A_BYTES, &tmA, bar, step * BK, m0);
+                    else tma_load_2d_pair(sbase + OFF_A + sa * A_BYTES, &tmL, bar, (step - nks) * BK, m0);
+                    ++issued;
+                    if (++sa == SA) { sa = 0; pa ^= 1; }
+                }
+            }
+            if (!ok && leader)
+                for (int i = 1; i <= SA && i <= issued; ++i) mbar_drain_cl(fullA((issued - i) % SA), ((issued - i) / SA) & 1);
+        }
+    } else if (warp == 14) {
+        // ------------------------------------------------------------ packed weights (own half)
+        if (lane == 0) {
+            int sp = 0, pp = 0, issued = 0;
+            bool ok = true;
+            for (int64_t tile = pair; tile < ntiles && ok; tile += npairs) {
+                const int c0 = (int)((tile / mtiles) * BN + crank * HN);
+                for (int step = 0; step < nks && ok; ++step) {
+                    if (!(ok = tc::mbar_wait(emptyP(sp), pp ^ 1, s_abort))) break;
+                    tc::mbar_expect_tx(fullP(sp), P_BYTES);
+                    if (!BWD) tc::tma_load_2d(sbase + OFF_P + sp * P_BYTES, &tmP, fullP(sp), step * (BK / 2), c0);
+                    else tc::tma_load_2d(sbase + OFF_P + sp * P_BYTES, &tmP, fullP(sp), c0 / 2, step * BK);
+                    ++issued;
+                    if (++sp == SP) { sp = 0; pp ^= 1; }
+                }
+            }
+            if (!ok)
+                for (int i = 1; i <= SP && i <= issued; ++i) tc::mbar_drain(fullP((issued - i) % SP), ((issued - i) / SP) & 1);
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer (leader only)
+        if (leader && lane == 0) {
+            constexpr uint32_t idesc = make_idesc2(BWD);
+            int sa = 0, pa = 0, sw = 0, pw = 0;
+            bool ok = true;
+            int it = 0;
+            for (int64_t tile = pair; tile < ntiles && ok; tile += npairs, ++it) {
+                const int acc = it & 1, aph = (it >> 1) & 1;
+                if (!(ok = mbar_wait_cl(tempty(acc), aph ^ 1, s_abort))) break;
+                tc::tc_fence_after();
+                const uint32_t d_tmem = tmem_base + acc * BN;
+                for (int step = 0; step < nsteps && ok; ++step) {
+                    if (!(ok = mbar_wait_cl(fullA(sa), pa, s_abort))) break;
+                    if (!(ok = mbar_wait_cl(fullW(sw), pw, s_abort))) break;
+                    tc::tc_fence_after();
+                    const uint32_t a_addr = sbase + OFF_A + sa * A_BYTES;
+                    const uint32_t w_addr = sbase + OFF_W + sw * W_BYTES;
+#pragma unroll
+                    for (int kk = 0; kk < BK / 16; ++kk) {
+                        const uint64_t adesc = tc::smem_desc_sw128(a_addr + kk * 32, 16, 1024);
+                        const uint64_t bdesc = BWD ? tc::smem_desc_sw128(w_addr + kk * 2048, 8192, 1024)
+                                                   : tc::smem_desc_sw128(w_addr + kk * 32, 16, 1024);
+                        tc2_mma(d_tmem, adesc, bdesc, idesc, (step > 0 || kk > 0) ? 1u : 0u);
+                    }
+                    tc2_commit_both(emptyA(sa));
+                    tc2_commit_both(emptyW(sw));
+                    if (++sa == SA) { sa = 0; pa ^= 1; }
+                    if (++sw == SW) { sw = 0; pw ^= 1; }
+                }
+                if (ok) tc2_commit_both(tfull(acc));
+            }
+            tc2_commit_local(drain);
+            mbar_drain_cl(drain, 0);
+        }
+    } else if (warp < 10) {
+        // ------------------------------------------------------------ dequantizers: two groups, alternate steps
+        const int grp = (warp - 2) >> 2;               // 0: even steps, 1: odd steps
+        const int t = ((warp - 2) & 3) * 32 + lane;    // 0..127
+        const int drow = deq_row<BWD>(t), dblk = deq_blk<BWD>(t);
+        bool ok = true;
+        auto fetch = [&](int64_t c0, int st, int& code, float& sc, float& mu) {
+            int64_t n, kb;
+            if (!BWD) { n = c0 + drow; kb = st; }
+            else { n = (int64_t)st * BK + drow; kb = c0 / kBlock + dblk; }
+            code = 0; sc = 0.f; mu = 0.f;
+            if (st < nks && n < a.N && kb < nblk) {
+                const int64_t b = n * nblk + kb;
+                const int64_t g = b >> 8;
+                code = __ldg(a.codes + b);
+                sc = __ldg(a.scale + g);
+                mu = __ldg(a.mean + g);
+            }
+        };
+        int it = 0;
+        for (int64_t tile = pair; tile < ntiles && ok; tile += npairs, ++it) {
+            const int64_t c0 = (tile / mtiles) * BN + crank * HN;   // this CTA's first output column
+            int code;
+            float sc, mu;
+            fetch(c0, grp, code, sc, mu);
+            for (int step = grp; step < nsteps && ok; step += 2) {
+                const int gs = it * nsteps + step;             // global step: W ring position
+                const int sw = gs % SW, pw = (gs / SW) & 1;
+                uint32_t o[8][4];
+                if (step < nks) {
+                    const float c = __fmaf_rn((float)code, sc, mu);
+                    fetch(c0, step + 2, code, sc, mu);
+                    const int gp = it * nks + step;            // global main step: P ring position
+                    const int sp = gp % SP, pp = (gp / SP) & 1;
+                    if (!(ok = tc::mbar_wait(fullP(sp), pp, s_abort))) break;
+                    uint4 p0, p1;
+                    const uint32_t pst = sbase + OFF_P + sp * P_BYTES;
+                    const uint32_t src0 = pst + p_chunk_offset<BWD>(t, 0), src1 = pst + p_chunk_offset<BWD>(t, 1);
+                    asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(p0.x), "=r"(p0.y), "=r"(p0.z), "=r"(p0.w) : "r"(src0));
+                    asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(p1.x), "=r"(p1.y), "=r"(p1.z), "=r"(p1.w) : "r"(src1));
+                    __syncwarp();
+                    if (lane == 0) tc::mbar_arrive(emptyP(sp));
+                    const BlockTable tb = make_block_table(tab, c);
+                    const uint32_t pwd[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
+#pragma unroll
+                    for (int ch = 0; ch < 8; ++ch) decode8(tb, pwd[ch], o[ch]);
+                } else {
+                    const int lc = step - nks;
+                    const uint16_t* src;
+                    int64_t col0;
+                    bool rowok;
+                    if (!BWD) {
+                        const int64_t n = c0 + drow;
+                        rowok = n < a.N;
+                        src = a.lora_w + n * a.ldl;
+                        col0 = (int64_t)lc * BK;
+                    } else {
+                        const int64_t i = (int64_t)lc * BK + drow;
+                        rowok = i < a.r;
+                        src = a.lora_w + i * a.ldl;
+                        col0 = c0 + dblk * 64;
+                    }
+#pragma unroll
+                    for (int ch = 0; ch < 8; ++ch) {
+                        const int64_t col = col0 + ch * 8;
+                        const bool v = rowok && (BWD ? (col < a.K) : (col < a.r));
+                        uint4 q = make_uint4(0, 0, 0, 0);
+                        if (v) q = __ldg(reinterpret_cast<const uint4*>(src + col));
+                        o[ch][0] = q.x; o[ch][1] = q.y; o[ch][2] = q.z; o[ch][3] = q.w;
+                    }
+                }
+                if (!(ok = tc::mbar_wait(emptyW(sw), pw ^ 1, s_abort))) break;
+                const uint32_t wbase = sbase + OFF_W + sw * W_BYTES;
+#pragma unroll
+                for (int ch = 0; ch < 8; ++ch)
+                    tc::st_shared_v4(wbase + w_chunk_offset<BWD>(t, ch), o[ch][0], o[ch][1], o[ch][2], o[ch][3]);
+                tc::fence_proxy_async();                  // this thread's tile writes -> async proxy
+                __syncwarp();
+                if (lane == 0) mbar_arrive_cl(mapa(fullW(sw), 0));
+            }
+        }
+    } else {
+        // ------------------------------------------------------------ epilogue (own 128 tokens)
+        const int q = warp & 3;
+        const int row = q * 32 + lane;
+        bool ok = true;
+        int it = 0;
+        for (int64_t tile = pair; tile < ntiles && ok; tile += npairs, ++it) {
+            const int acc = it & 1, aph = (it >> 1) & 1;
+            const int64_t m = (tile % mtiles) * BM + crank * HM + row;
+            const int64_t c0 = (tile / mtiles) * BN;
+            if (!(ok = tc::mbar_wait(tfull(acc), aph, s_abort))) break;
+            tc::tc_fence_after();
+#pragma unroll 1
+            for (int cc = 0; cc < BN / 32; ++cc) {
+                uint32_t r[32];
+                const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN + cc * 32);
+                TC_LD32(taddr, r);
+                asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+                if (m < a.M) {
+                    uint16_t* dst = a.out + m * a.n_out + c0 + cc * 32;
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        if (c0 + cc * 32 + j * 8 < a.n_out) {
+                            uint4 v;
+                            v.x = pack_bf16x2(__uint_as_float(r[8 * j + 0]), __uint_as_float(r[8 * j + 1]));
+                            v.y = pack_bf16x2(__uint_as_float(r[8 * j + 2]), __uint_as_float(r[8 * j + 3]));
+                            v.z = pack_bf16x2(__uint_as_float(r[8 * j + 4]), __uint_as_float(r[8 * j + 5]));
+                            v.w = pack_bf16x2(__uint_as_float(r[8 * j + 6]), __uint_as_float(r[8 * j + 7]));
+                            *reinterpret_cast<uint4*>(dst + j * 8) = v;
+                        }
+                    }
+                }
+            }
+            tc::tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cl(mapa(tempty(acc), 0));
+        }
+    }
+
+    __syncthreads();
+    cluster_sync();                      // neither CTA leaves while the pair may still use its memory
+    if (warp == 1) {
+        tc::tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(kTmemCols));
+    }
+}
+
+}  // namespace tc2
+}  // namespace qnf4

@@ -251,9 +251,9 @@ k_tc_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
 
     if (tid == 0) {
         for (int i = 0; i < SA; ++i) { mbar_init(fullA(i), 1); mbar_init(emptyA(i), 1); }
-        for (int i = 0; i < SW; ++i) { mbar_init(fullW(i), kDeqThreads); mbar_init(emptyW(i), 1); }
-        for (int i = 0; i < SP; ++i) { mbar_init(fullP(i), 1); mbar_init(emptyP(i), kDeqThreads); }
-        for (int i = 0; i < 2; ++i) { mbar_init(tfull(i), 1); mbar_init(tempty(i), kEpiThreads); }
+        for (int i = 0; i < SW; ++i) { mbar_init(fullW(i), kDeqThreads / 32); mbar_init(emptyW(i), 1); }
+        for (int i = 0; i < SP; ++i) { mbar_init(fullP(i), 1); mbar_init(emptyP(i), kDeqThreads / 32); }
+        for (int i = 0; i < 2; ++i) { mbar_init(tfull(i), 1); mbar_init(tempty(i), kEpiThreads / 32); }
         mbar_init(drain, 1);
         *s_abort = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -376,7 +376,8 @@ k_tc_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
                 const uint32_t src0 = pst + p_chunk_offset<BWD>(d, 0), src1 = pst + p_chunk_offset<BWD>(d, 1);
                 asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(p0.x), "=r"(p0.y), "=r"(p0.z), "=r"(p0.w) : "r"(src0));
                 asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(p1.x), "=r"(p1.y), "=r"(p1.z), "=r"(p1.w) : "r"(src1));
-                mbar_arrive(emptyP(sp));
+                __syncwarp();
+                if (lane == 0) mbar_arrive(emptyP(sp));
                 if (++sp == SP) { sp = 0; pp ^= 1; }
                 const BlockTable tb = make_block_table(tab, c);
                 const uint32_t pwd[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
@@ -414,7 +415,8 @@ k_tc_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
             for (int ch = 0; ch < 8; ++ch)
                 st_shared_v4(wbase + w_chunk_offset<BWD>(d, ch), o[ch][0], o[ch][1], o[ch][2], o[ch][3]);
             fence_proxy_async();
-            mbar_arrive(fullW(sw));
+            __syncwarp();
+            if (lane == 0) mbar_arrive(fullW(sw));
             if (++sw == SW) { sw = 0; pw ^= 1; }
         };
         for (int64_t tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
@@ -462,7 +464,8 @@ k_tc_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
                 }
             }
             tc_fence_before();
-            mbar_arrive(tempty(acc));
+            __syncwarp();
+            if (lane == 0) mbar_arrive(tempty(acc));
         }
     }
 

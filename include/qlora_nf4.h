@@ -164,8 +164,9 @@ QLORA_API const char* qlora_status_string(int status);
 QLORA_API int qlora_device_status(int reset);
 
 /* Which kernel family the last successful fwd/bwd call on this thread
- * dispatched to (for tests and benchmarks): 1 = small-M split-K tensor-core
- * GEMV path, 2 = tcgen05 fused dequant-GEMM path. */
+ * dispatched to (for tests and benchmarks): 1 = small-M tensor-core GEMV
+ * kernels (M <= 32), 2 = tcgen05 fused dequant-GEMM on one SM per tile
+ * (32 < M <= 128), 3 = the same on SM pairs (cta_group::2, M > 128). */
 QLORA_API int qlora_last_path(void);
 
 /* Measurement hooks (no counterpart on the pages; used by benchmarks).

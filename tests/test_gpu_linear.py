@@ -56,6 +56,9 @@ CASES = [
     (257, 384, 448, 64),
     (300, 768, 1216, 100),
     (512, 1024, 2048, 16),
+    (129, 256, 512, 16),
+    (640, 1280, 1024, 32),
+    (1000, 520, 1088, 64),
 ]
 
 
@@ -83,7 +86,7 @@ def test_fwd_bwd_parity(oracle_mod, M, N, K, r):
     _close(inputs.to_f64(dX2), dXr, "dX (T given)")
     _close(inputs.to_f64(dA2), dAr, "dA (T given)")
     _close(inputs.to_f64(dB2), dBr_given, "dB (T given)")
-    assert ops.qlora_last_path() == (1 if M <= 32 else 2)
+    assert ops.qlora_last_path() == (1 if M <= 32 else 2 if M <= 128 else 3)
 
 
 def test_zero_B_is_plain_dequant_matmul(oracle_mod):
