@@ -57,6 +57,7 @@ def lib():
             "qlora_last_path": (i32, []),
             "qlora_launch_count": (ctypes.c_longlong, []),
             "qlora_set_kernel_events": (i32, [P, P]),
+            "qlora_linear_fwd_noalloc": (i32, [P, i64, WP, P, P, i32, f32, P, P, P]),
         }
         for name, (res, args) in sig.items():
             fn = getattr(L, name)
@@ -209,3 +210,15 @@ def qlora_set_kernel_events(before, after) -> None:
     b = ctypes.c_void_p(before.cuda_event) if before is not None else None
     a = ctypes.c_void_p(after.cuda_event) if after is not None else None
     _check("qlora_set_kernel_events", lib().qlora_set_kernel_events(b, a))
+
+
+def qlora_linear_fwd_noalloc(X, w: NF4Weight, A, B, scaling: float, Y=None, T_out=None, stream=None):
+    """qlora_linear_fwd on the library's fixed static scratch (no workspace argument)."""
+    M = X.shape[0]
+    if Y is None:
+        Y = torch.empty((M, w.N), dtype=torch.bfloat16, device=X.device)
+    st = w.c_struct()
+    _check("qlora_linear_fwd_noalloc", lib().qlora_linear_fwd_noalloc(
+        _ptr(_bits(X)), M, ctypes.byref(st), _ptr(_bits(A)), _ptr(_bits(B)), A.shape[0], float(scaling),
+        _ptr(Y), _ptr(T_out), _stream(stream)))
+    return Y

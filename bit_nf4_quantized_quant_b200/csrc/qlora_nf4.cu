@@ -697,6 +697,7 @@ const char* qlora_status_string(int status) {
         case QLORA_ERR_LAUNCH: return "CUDA launch or runtime call failed";
         case QLORA_ERR_TIMEOUT: return "a device-side bounded wait gave up";
         case QLORA_ERR_VALUE: return "a scalar argument is not finite";
+        case QLORA_ERR_SCRATCH: return "needs more scratch than the fixed no-alloc scratch (QLORA_NOALLOC_SCRATCH_BYTES)";
         default: return "unknown status";
     }
 }
@@ -724,3 +725,49 @@ int qlora_set_kernel_events(void* before, void* after) {
 }
 
 }  // extern "C"
+
+// ===========================================================================
+// Allocation-free forward: the workspace is a fixed static device array.
+// ===========================================================================
+namespace {
+
+// Scratch of qlora_linear_fwd_noalloc; every device that loads the library
+// holds it until the process exits.
+static __device__ __align__(256) uint8_t g_noalloc_scratch[QLORA_NOALLOC_SCRATCH_BYTES];
+
+void* g_noalloc_ptr[64];
+std::mutex g_noalloc_mu;
+
+// Device address of the scratch on the current device, looked up once per
+// device with that device current (the host-side symbol is not a device
+// address and must never be handed to a kernel).
+int noalloc_scratch(void** out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return QLORA_ERR_DEVICE;
+    std::lock_guard<std::mutex> lk(g_noalloc_mu);
+    if (g_noalloc_ptr[dev] == nullptr) {
+        void* ptr = nullptr;
+        if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || ptr == nullptr) return QLORA_ERR_LAUNCH;
+        g_noalloc_ptr[dev] = ptr;
+    }
+    *out = g_noalloc_ptr[dev];
+    return QLORA_OK;
+}
+
+}  // namespace
+
+extern "C" int qlora_linear_fwd_noalloc(const qlora_bf16* X, int64_t M, const nf4dq_weight* w, const qlora_bf16* A,
+                                        const qlora_bf16* B, int r, float scaling, qlora_bf16* Y, qlora_bf16* T_out,
+                                        qlora_stream_t stream) {
+    if (w != nullptr) {
+        const size_t need = qlora_workspace_bytes(M, w->N, w->K, r);
+        if (need > (size_t)QLORA_NOALLOC_SCRATCH_BYTES) return QLORA_ERR_SCRATCH;
+    }
+    void* ws = nullptr;
+    if (w != nullptr && qlora_workspace_bytes(M, w->N, w->K, r) != 0) {
+        const int rc = noalloc_scratch(&ws);
+        if (rc != QLORA_OK) return rc;
+    }
+    // invalid arguments are reported by the regular forward before anything is launched
+    return qlora_linear_fwd(X, M, w, A, B, r, scaling, Y, T_out, ws, QLORA_NOALLOC_SCRATCH_BYTES, stream);
+}

@@ -69,7 +69,8 @@ enum {
     QLORA_ERR_DEVICE = -6,      /* current device is not compute capability 10.0 */
     QLORA_ERR_LAUNCH = -7,      /* a CUDA launch or runtime call failed */
     QLORA_ERR_TIMEOUT = -8,     /* a device-side bounded wait gave up (see qlora_device_status) */
-    QLORA_ERR_VALUE = -9        /* a scalar argument is not finite */
+    QLORA_ERR_VALUE = -9,       /* a scalar argument is not finite */
+    QLORA_ERR_SCRATCH = -10     /* needs more than QLORA_NOALLOC_SCRATCH_BYTES (no-alloc entry point) */
 };
 
 /* Quantized weight: all device pointers, caller-owned.
@@ -177,6 +178,32 @@ QLORA_API int qlora_last_path(void);
  * and `after` right after it, then forgets both; pass NULL, NULL to clear. */
 QLORA_API long long qlora_launch_count(void);
 QLORA_API int qlora_set_kernel_events(void* before, void* after);
+
+/* qlora_linear_fwd_noalloc -- the paper has no counterpart; this is a
+ * convenience of this library.
+ *
+ * The same forward as qlora_linear_fwd, for callers that cannot allocate
+ * device memory: code running where another allocator owns all of the
+ * device's memory (a serving engine that reserved its pool at start-up),
+ * or code called back from inside a framework that forbids allocating on
+ * its hot path.  Instead of a caller-provided workspace it uses one scratch
+ * array of QLORA_NOALLOC_SCRATCH_BYTES that the library defines statically
+ * in device memory; every GPU that loads the library holds that array until
+ * the process exits.  Nothing is allocated or freed by this call.
+ *   - The first call on a device looks up the array's device address
+ *     (cudaGetSymbolAddress) with that device current; make that first call
+ *     before any stream capture.
+ *   - Calls whose workspace need (qlora_workspace_bytes) exceeds
+ *     QLORA_NOALLOC_SCRATCH_BYTES return QLORA_ERR_SCRATCH and launch
+ *     nothing; decode-sized calls (M <= 32 with 70B-model projections) fit.
+ *   - All calls share the one array: calls that overlap on the GPU (other
+ *     streams, other host threads) race on it and must be serialized by the
+ *     caller.  What the forward needs zeroed it zeroes itself each call.
+ * Arguments, layouts and the other errors are those of qlora_linear_fwd. */
+#define QLORA_NOALLOC_SCRATCH_BYTES (8u << 20)
+QLORA_API int qlora_linear_fwd_noalloc(const qlora_bf16* X, int64_t M, const nf4dq_weight* w, const qlora_bf16* A,
+                                       const qlora_bf16* B, int r, float scaling, qlora_bf16* Y, qlora_bf16* T_out,
+                                       qlora_stream_t stream);
 
 #ifdef __cplusplus
 }
