@@ -207,7 +207,7 @@ def run_ours(args, rank, world, local_rank):
 
     it = [0]
 
-    def step(events=None):
+    def step(events=None, collective=True):
         c = it[0] % copies
         it[0] += 1
         for j, L in enumerate(layers):
@@ -221,16 +221,21 @@ def run_ours(args, rank, world, local_rank):
                 ops.qlora_set_kernel_events(*events[2 * j + 1])
             ops.qlora_linear_bwd(L["X"], L["dY"], w, L["A"], L["B"], s, T=L["T"], dX=L["dX"], dA=L["dA"],
                                  dB=L["dB"], ws=ws)
-        if world > 1 and bwd:
+        if world > 1 and bwd and collective:
             dist.all_reduce(gbuf)
 
     for _ in range(args.warmup):
         step()
+    c0 = ops.qlora_launch_count()
+    step()
+    per_step_launches = ops.qlora_launch_count() - c0
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
 
-    # ---- timed region
+    # ---- timed region: one CUDA graph per timed step (the library calls are
+    # asynchronous and allocation-free, so a step captures as is); each graph
+    # records its own per-launch events around the fused dequant-GEMM kernels
     kev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
             for _ in range(2 * len(layers))] for _ in range(args.steps)]
     for evs in kev:                 # torch creates the CUDA events lazily: record once so they exist
@@ -238,6 +243,19 @@ def run_ours(args, rank, world, local_rank):
             a.record(stream)
             b.record(stream)
     torch.cuda.synchronize()
+    graphs = []
+    if not args.no_graph:
+        for k in range(args.steps):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                step(kev[k], collective=False)
+            graphs.append(g)
+        for g in graphs:            # upload + warm
+            g.replay()
+            if world > 1:
+                dist.all_reduce(gbuf)
+        torch.cuda.synchronize()
+        stream = torch.cuda.current_stream()
     clocks = ClockSampler(local_rank)
     clocks.start()
     launches0 = ops.qlora_launch_count()
@@ -249,13 +267,20 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.nvtx.range_push("timed")
     t0.record(stream)
     for k in range(args.steps):
-        step(kev[k])
+        if graphs:
+            graphs[k].replay()
+            if world > 1 and bwd:
+                dist.all_reduce(gbuf)
+        else:
+            step(kev[k])
     t1.record(stream)
     torch.cuda.nvtx.range_pop()
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
     launches = ops.qlora_launch_count() - launches0
+    if graphs:   # a replayed graph launches the kernels captured from one step
+        launches = per_step_launches * args.steps
     clk = clocks.stop()
     ms = t0.elapsed_time(t1)
     if world > 1:
@@ -279,13 +304,26 @@ def run_ours(args, rank, world, local_rank):
     # roofline of the dominant kernel (the fused dequant-GEMM), from its own launch events
     kflops, kms, nlaunch = 0.0, 0.0, 0
     kbytes = 0
+    kev_src = "graph replay" if graphs else "timed steps"
+    try:
+        kev[0][0][0].elapsed_time(kev[0][0][1])
+    except RuntimeError:
+        # events inside a replayed graph could not be timed: time the kernels
+        # over the same number of steps launched eagerly on the same stream
+        torch.cuda.synchronize()
+        for k in range(args.steps):
+            step(kev[k], collective=False)
+        torch.cuda.synchronize()
+        kev_src = "eager pass after the timed steps"
     for k in range(args.steps):
         for j, L in enumerate(layers):
             N_, K_ = L["p"].N, L["p"].K
             f_fwd, f_bwd = main_kernel_flops(M, N_, K_, r)
-            # the small-M kernels read the NF4 weight and the activations and write their output once
-            b_fwd = nf4_bytes(N_, K_) + 2 * (M * K_ + M * N_)
-            b_bwd = nf4_bytes(N_, K_) + 2 * (M * N_) + 4 * M * K_
+            # small M: the timed pair in the forward is T = X A^T + the GEMV (NF4 weight, X, A, B
+            # read, Y and T written once); in the backward the U / dB kernel + the dX GEMV
+            # (NF4 weight, dY, B and T read, dB written once; split partials not counted)
+            b_fwd = nf4_bytes(N_, K_) + 2 * (M * K_ + M * N_ + r * K_ + N_ * r + M * r)
+            b_bwd = nf4_bytes(N_, K_) + 2 * (M * N_ + 2 * N_ * r + M * r)
             for h, f, bb in ((0, f_fwd, b_fwd), (1, f_bwd, b_bwd))[:npass]:
                 a, b = kev[k][2 * j + h]
                 kms += a.elapsed_time(b)
@@ -304,8 +342,10 @@ def run_ours(args, rank, world, local_rank):
     roof.update({"achieved": round(achieved, 2), "peak": peak, "frac": round(achieved / peak, 4),
                  "traffic": tr["bytes_per_launch"] if tr and tr.get("src") == src_hash() else None,
                  "peak_source": f"{peak_src} ({'hbm copy' if small else 'cuBLAS bf16 sustained'})",
-                 "kernel": "k_fwd_small/k_bwd_small" if small else "k_tc_gemm (fwd + bwd dX)",
-                 "launches_timed": nlaunch, "avg_launch_us": round(kms / nlaunch * 1e3, 2)})
+                 "kernel": ("k_lora_down_small + k_nf4_gemv / k_lora_bwd_small + k_tcs_gemm (programmatic-launch pairs)"
+                            if small else "k_tc_gemm / k_tc2_gemm (fwd + bwd dX)"),
+                 "launches_timed": nlaunch, "avg_launch_us": round(kms / nlaunch * 1e3, 2),
+                 "events_from": kev_src})
 
     roof["weight_copies_rotated"] = copies
     if small:
@@ -367,7 +407,8 @@ def run_ours(args, rank, world, local_rank):
                    (" + NCCL all-reduce of dA,dB" if world > 1 else ""),
            "l2": (f"inputs larger than L2: {bytes_step / 1e6:.0f} MB of algorithmic traffic per step" if not small else
                   f"weights rotated over {copies} copies ({copies * wset / 1e6:.0f} MB > 2x L2)"),
-           "parallelism": f"dp{world}"}
+           "parallelism": f"dp{world}",
+           "launch": "eager" if args.no_graph else "one CUDA graph per step (library calls captured as issued)"}
     out = {"metric": METRIC, "value": round(value, 3), "unit": unit, "n_gpus": world, "steps": args.steps,
            "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4), "higher_is_better": True,
            "scaling": "weak", "vs_baseline": None, "dtype": "bf16 (NF4 weights, fp32 accumulate)",
@@ -590,6 +631,7 @@ def main():
     ap.add_argument("--layers", type=int, default=0, help="workload 5: number of 7-tensor layers (default 32)")
     ap.add_argument("--M", type=int, default=0, help="tokens per GPU (default: the workload's largest)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-graph", action="store_true", help="launch the timed steps eagerly instead of as CUDA graphs")
     ap.add_argument("--cpu-seconds", type=float, default=20.0)
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)

@@ -99,6 +99,13 @@ __device__ __forceinline__ void mma_bf16_16816_zero(float (&d)[4], uint32_t a0, 
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "f"(z));
 }
 
+// Programmatic dependent launch: a kernel launched with programmatic stream
+// serialization may start once every CTA of the kernel before it has called
+// grid_dep_launch(); grid_dep_wait() then blocks until that kernel has
+// completed and its writes are visible.  Both are no-ops for a normal launch.
+__device__ __forceinline__ void grid_dep_launch() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+__device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 __host__ __device__ __forceinline__ int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
 __host__ __device__ __forceinline__ int64_t rup(int64_t a, int64_t b) { return cdiv(a, b) * b; }
 

@@ -1,0 +1,328 @@
+// gemv_mma.cuh -- small-M forward (M <= 32 tokens): fused exact NF4 decode +
+// mma.sync, with the packed weight staged by TMA and the work split evenly
+// over one CTA per SM.
+//
+//   Y [M, N] = X [M, K] . W'^T + s T B^T,   W' = bf16_rne(L[q] c')
+//
+// At a few tokens the layer is bound by the integer-pipe work of the exact
+// decode (a 16-entry bf16 table per 64-weight block and byte permutes, see
+// nf4_decode.cuh), so the kernel is built around keeping that pipe busy:
+//
+//  * The decoded bf16 pairs are the A operand of mma.sync m16n8k16 straight
+//    from registers (W rows are the MMA rows, tokens its 8-wide columns), so
+//    the weight never goes back to shared memory.  A lane (g, t) of the MMA
+//    holds rows g and g + 8 and, in MMA s, the logical k {2t, 2t+1, 2t+8,
+//    2t+9}; these are mapped to elements 4s .. 4s+3 of 64-weight block t of a
+//    256-wide step, so over the 16 MMAs of a step every lane decodes exactly
+//    two whole blocks (rows g and g + 8) and builds two tables.
+//  * Work unit = (128 rows, 256 reduction) = 8 warps x 16 rows.  The units
+//    are split evenly over the CTAs in (tile, step) order; in a CTA two
+//    groups of 8 warps take alternate units.  Partial sums of a tile that
+//    spans several (CTA, group) pairs are written to per-pair slots; the warp
+//    that arrives last on the (tile, warp row-slice) counter sums them in
+//    (CTA, group) order -- the result does not depend on arrival order -- and
+//    adds s T B^T.
+//  * Warp 0 lane 0 loads each unit's packed tile (128 rows x 128 B, 128-byte
+//    swizzle) with TMA; the 32 lanes of warp 0 copy the unit's activation
+//    slice with cp.async into a fragment-native layout ([j][token][t] 16-byte
+//    chunks: the 16 bytes lane (g, t) feeds to MMAs 2j and 2j+1), so the
+//    consumers' shared loads are conflict-free; both complete on the stage's
+//    mbarrier.  Rows of the slice beyond M are zeroed once and never copied.
+#pragma once
+#include <cuda.h>
+#include "common.cuh"
+#include "nf4_decode.cuh"
+#include "tc_gemm.cuh"
+
+namespace qnf4 {
+namespace gmv {
+
+constexpr int TR = 128;                          // rows of a unit
+constexpr int KSTEP = 256;                       // reduction of a unit
+constexpr int P_BYTES = TR * KSTEP / 2;          // 16384
+constexpr int kGroupWarps = 8;
+constexpr int kThreads = 32 * (1 + 2 * kGroupWarps);   // 544
+
+template <int NTT>
+struct Cfg {
+    static constexpr int NT = 8 * NTT;                  // token columns (zero beyond M)
+    static constexpr int X_BYTES = NT * KSTEP * 2;      // 4096 * NTT
+    static constexpr int STAGE = P_BYTES + X_BYTES;     // a multiple of 1024
+    static constexpr int SP = NTT == 4 ? 4 : 8;         // stages (half per group), a power of 2
+    static constexpr int OFF_BAR = SP * STAGE;
+    static constexpr int SMEM_ALLOC = OFF_BAR + 2 * SP * 8 + 16 + 1024;
+};
+
+struct Args {
+    const uint16_t* X;         // [M, K] bf16
+    const int8_t* codes;
+    const float* scale;
+    const float* mean;
+    int64_t M, N, K;
+    int tiles, nks;            // ceil(N / 128), ceil(K / 256)
+    int64_t units;             // tiles * nks
+    int ctas;
+    float* slots;              // [(ctas + tiles) * 2][NT][128] fp32 partials
+    int* counters;             // [tiles][8], zero on entry, left zero
+    const float* T32;          // [M, rp] fp32 LoRA down-projection
+    int rp, r;
+    const uint16_t* lora_B;    // [N, r]
+    float s;
+    uint16_t* Y;               // [M, N]
+};
+
+__host__ __device__ __forceinline__ int64_t unit_begin(int64_t c, int64_t U, int64_t C) { return c * U / C; }
+__host__ __device__ __forceinline__ int64_t unit_owner(int64_t u, int64_t U, int64_t C) {
+    return ((u + 1) * C + U - 1) / U - 1;
+}
+__device__ __forceinline__ void unit_advance(int& tile, int& ks, int n, int nks) {
+    ks += n;
+    while (ks >= nks) { ks -= nks; ++tile; }
+}
+
+// Units of CTA c inside tile [tu0, tu1), and which of its two groups took
+// them: bit 0 = group 0, bit 1 = group 1 (its CTA-local unit indices are even
+// for group 0 and odd for group 1).
+__device__ __forceinline__ int groups_in_tile(int64_t c, int64_t U, int64_t C, int64_t tu0, int64_t tu1) {
+    const int64_t b0 = unit_begin(c, U, C), b1 = unit_begin(c + 1, U, C);
+    const int64_t lo = b0 > tu0 ? b0 : tu0, hi = b1 < tu1 ? b1 : tu1;
+    if (hi - lo >= 2) return 3;
+    if (hi - lo == 1) return 1 << ((lo - b0) & 1);
+    return 0;
+}
+
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, int src_bytes) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
+}
+
+template <int NTT>
+__global__ void __launch_bounds__(kThreads, 1) k_nf4_gemv(const __grid_constant__ CUtensorMap tmP, Args a,
+                                                        NF4Tables tab) {
+    using C = Cfg<NTT>;
+    constexpr int NT = C::NT;
+    constexpr int SP = C::SP;
+    extern __shared__ __align__(1024) uint8_t smem[];
+    uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem) + 1023) & ~(uintptr_t)1023);
+    const uint32_t sbase = smem_u32(base);
+    const uint32_t bar0 = sbase + C::OFF_BAR;
+    auto full = [&](int i) { return bar0 + 8 * i; };
+    auto empty = [&](int i) { return bar0 + 8 * (SP + i); };
+    volatile int* s_abort = reinterpret_cast<volatile int*>(base + C::OFF_BAR + 2 * SP * 8);
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int64_t U = a.units;
+    const int u0 = (int)unit_begin(blockIdx.x, U, a.ctas), u1 = (int)unit_begin(blockIdx.x + 1, U, a.ctas);
+    const int nu = u1 - u0;
+    const int nks = a.nks;
+    const int tile0 = u0 / nks, ks0 = u0 - tile0 * nks;
+    const uint32_t nblk32 = (uint32_t)(a.K / kBlock), N32 = (uint32_t)a.N;
+
+    // token rows >= M of every stage's activation slice stay zero
+    for (int e = tid; e < SP * NT * 32; e += kThreads) {
+        const int st = e / (NT * 32), c = e % (NT * 32);
+        if ((c / 4) % NT >= a.M) {
+            const uint32_t dst = sbase + st * C::STAGE + P_BYTES + c * 16;
+            asm volatile("st.shared.v4.u32 [%0], {%1,%1,%1,%1};" ::"r"(dst), "r"(0u) : "memory");
+        }
+    }
+    if (tid == 0) {
+        for (int i = 0; i < SP; ++i) {
+            tc::mbar_init(full(i), 1 + 32);              // TMA expect-tx arrival + 32 cp.async arrivals
+            tc::mbar_init(empty(i), kGroupWarps);
+        }
+        *s_abort = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    __syncthreads();
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ producer
+        int tile = tile0, ks = ks0, issued = 0;
+        bool ok = true;
+        const int64_t mrows = a.M < NT ? a.M : NT;
+        for (int i = 0; i < nu; ++i) {
+            const int st = i % SP, ph = (i / SP) & 1;
+            int w_ok = 1;
+            if (lane == 0) w_ok = tc::mbar_wait(empty(st), ph ^ 1, s_abort) ? 1 : 0;
+            ok = __shfl_sync(0xffffffffu, w_ok, 0) != 0;
+            if (!ok) break;
+            const uint32_t sdst = sbase + st * C::STAGE;
+            if (lane == 0) {
+                tc::mbar_expect_tx(full(st), P_BYTES);
+                tc::tma_load_2d(sdst, &tmP, full(st), ks * (KSTEP / 2), tile * TR);
+            }
+            // activation chunks (m, t, j): 16 bytes of row m at k = 256 ks + 64 t + 8 j,
+            // stored at chunk (j * NT + m) * 4 + t of the slice; zero beyond K
+            for (int c = lane; c < mrows * 32; c += 32) {
+                const int m = c >> 5, t = (c >> 3) & 3, j = c & 7;
+                const int64_t k = (int64_t)ks * KSTEP + 64 * t + 8 * j;
+                const bool in = k < a.K;
+                const uint16_t* src = a.X + (in ? (int64_t)m * a.K + k : 0);
+                cp_async16(sdst + P_BYTES + ((j * NT + m) * 4 + t) * 16, src, in ? 16 : 0);
+            }
+            asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(full(st)) : "memory");
+            ++issued;
+            unit_advance(tile, ks, 1, nks);
+        }
+        // on abort: let the copies in flight land before the CTA exits
+        asm volatile("cp.async.wait_all;" ::: "memory");
+        if (!ok && lane == 0)
+            for (int k = 1; k <= SP && k <= issued; ++k)
+                tc::mbar_drain(full((issued - k) % SP), ((issued - k) / SP) & 1);
+    } else {
+        // ------------------------------------------------------------ decode + MMA warps
+        const int grp = (warp - 1) / kGroupWarps;        // units i = grp, grp + 2, ...
+        const int w8 = (warp - 1) % kGroupWarps;         // rows 16 w8 .. 16 w8 + 15 of a unit
+        const int g = lane >> 2, t = lane & 3;
+        const int r0 = 16 * w8 + g;                      // rows r0 and r0 + 8 of the tile
+        bool ok = true, waited = false;
+
+        // block-constant inputs of rows r0, r0 + 8, block 4 ks + t of the next unit to
+        // fetch (zero beyond the weight); fetches run two group-units ahead
+        int fi = grp, ft = tile0, fk = ks0;
+        unit_advance(ft, fk, grp, nks);
+        struct BC { int c0, c1; float s0, s1, m0, m1; };
+        auto fetch = [&](BC& b) {
+            b.c0 = b.c1 = 0; b.s0 = b.s1 = b.m0 = b.m1 = 0.f;
+            const int tile = ft, ks = fk;
+            const bool in = fi < nu;
+            fi += 2;
+            unit_advance(ft, fk, 2, nks);
+            // block indices fit 32 bits (the weight has fewer than 2^38 elements)
+            const uint32_t kb = (uint32_t)ks * 4u + (uint32_t)t;
+            if (!in || kb >= nblk32) return;
+            const uint32_t n0 = (uint32_t)tile * TR + (uint32_t)r0, n1 = n0 + 8u;
+            if (n0 < N32) {
+                const uint32_t bb = n0 * nblk32 + kb;
+                b.c0 = __ldg(a.codes + bb); b.s0 = __ldg(a.scale + (bb >> 8)); b.m0 = __ldg(a.mean + (bb >> 8));
+            }
+            if (n1 < N32) {
+                const uint32_t bb = n1 * nblk32 + kb;
+                b.c1 = __ldg(a.codes + bb); b.s1 = __ldg(a.scale + (bb >> 8)); b.m1 = __ldg(a.mean + (bb >> 8));
+            }
+        };
+
+        float acc[NTT][4];
+#pragma unroll
+        for (int nt = 0; nt < NTT; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
+
+        // finish (or publish) this warp's 16 rows of `tile` after the group's last unit of it
+        auto fixup = [&](int tile) {
+            if (!waited) { grid_dep_wait(); waited = true; }   // T and the zeroed counters
+            const int64_t tu0 = (int64_t)tile * nks, tu1 = tu0 + nks;
+            const int64_t c_first = unit_owner(tu0, U, a.ctas), c_last = unit_owner(tu1 - 1, U, a.ctas);
+            int expected = 0;
+            for (int64_t c2 = c_first; c2 <= c_last; ++c2) expected += __popc(groups_in_tile(c2, U, a.ctas, tu0, tu1));
+            bool finish = expected == 1;
+            if (!finish) {
+                float* sp = a.slots + (((int64_t)blockIdx.x + tile) * 2 + grp) * (NT * TR);
+#pragma unroll
+                for (int nt = 0; nt < NTT; ++nt) {
+                    const int m = 8 * nt + 2 * t;
+                    sp[m * TR + r0] = acc[nt][0];
+                    sp[(m + 1) * TR + r0] = acc[nt][1];
+                    sp[m * TR + r0 + 8] = acc[nt][2];
+                    sp[(m + 1) * TR + r0 + 8] = acc[nt][3];
+                }
+                __threadfence();
+                __syncwarp();
+                int last = 0;
+                if (lane == 0) {
+                    int* cnt = a.counters + (int64_t)tile * kGroupWarps + w8;
+                    last = atomicAdd(cnt, 1) == expected - 1;
+                    if (last) *cnt = 0;                        // ready for the next call
+                }
+                finish = __shfl_sync(0xffffffffu, last, 0) != 0;
+                if (finish) {
+                    __threadfence();
+#pragma unroll
+                    for (int nt = 0; nt < NTT; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
+                    for (int64_t c2 = c_first; c2 <= c_last; ++c2) {
+                        const int gm = groups_in_tile(c2, U, a.ctas, tu0, tu1);
+                        for (int g2 = 0; g2 < 2; ++g2) {
+                            if (!((gm >> g2) & 1)) continue;
+                            const float* p2 = a.slots + ((c2 + tile) * 2 + g2) * (NT * TR);
+#pragma unroll
+                            for (int nt = 0; nt < NTT; ++nt) {
+                                const int m = 8 * nt + 2 * t;
+                                acc[nt][0] += __ldcg(p2 + m * TR + r0);
+                                acc[nt][1] += __ldcg(p2 + (m + 1) * TR + r0);
+                                acc[nt][2] += __ldcg(p2 + m * TR + r0 + 8);
+                                acc[nt][3] += __ldcg(p2 + (m + 1) * TR + r0 + 8);
+                            }
+                        }
+                    }
+                }
+            }
+            if (finish) {
+#pragma unroll
+                for (int e = 0; e < 4 * NTT; ++e) {
+                    const int nt = e >> 2, q = e & 3;
+                    const int64_t m = 8 * nt + 2 * t + (q & 1);
+                    const int64_t n = (int64_t)tile * TR + r0 + 8 * (q >> 1);
+                    if (m < a.M && n < a.N) {
+                        const float* tr = a.T32 + m * a.rp;
+                        const uint16_t* br = a.lora_B + n * a.r;
+                        float l = 0.f;
+                        for (int i = 0; i < a.r; ++i) l = __fmaf_rn(tr[i], bf16lo_to_f32(br[i]), l);
+                        a.Y[m * a.N + n] = (uint16_t)(pack_bf16x2(__fmaf_rn(a.s, l, acc[nt][q]), 0.f) & 0xffffu);
+                    }
+                }
+            }
+#pragma unroll
+            for (int nt = 0; nt < NTT; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
+        };
+
+        BC bA, bB;
+        fetch(bA);
+        fetch(bB);
+        int tile = tile0, ks = ks0;
+        unit_advance(tile, ks, grp, nks);
+        // swizzled offsets of this lane's packed chunks (row r0; row r0 + 8 has the same swizzle)
+        const uint32_t pch0 = (uint32_t)(r0 * 128 + (((2 * t) ^ (r0 & 7)) << 4));
+        const uint32_t pch1 = (uint32_t)(r0 * 128 + (((2 * t + 1) ^ (r0 & 7)) << 4));
+        auto do_unit = [&](int i, BC& b) {
+            const float c0 = __fmaf_rn((float)b.c0, b.s0, b.m0), c1 = __fmaf_rn((float)b.c1, b.s1, b.m1);
+            fetch(b);
+            const int st = i % SP, ph = (i / SP) & 1;
+            if (!(ok = tc::mbar_wait(full(st), ph, s_abort))) return;
+            const uint32_t sst = sbase + st * C::STAGE;
+            uint32_t pa[8], pb[8];
+            asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(pa[0]), "=r"(pa[1]), "=r"(pa[2]), "=r"(pa[3]) : "r"(sst + pch0));
+            asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(pa[4]), "=r"(pa[5]), "=r"(pa[6]), "=r"(pa[7]) : "r"(sst + pch1));
+            asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(pb[0]), "=r"(pb[1]), "=r"(pb[2]), "=r"(pb[3]) : "r"(sst + pch0 + 1024));
+            asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(pb[4]), "=r"(pb[5]), "=r"(pb[6]), "=r"(pb[7]) : "r"(sst + pch1 + 1024));
+            const BlockTable ta = make_block_table(tab, c0), tb = make_block_table(tab, c1);
+            const uint32_t xb = sst + P_BYTES + (uint32_t)(lane * 16);
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                uint32_t oa[4], ob[4];
+                decode8(ta, pa[j], oa);
+                decode8(tb, pb[j], ob);
+#pragma unroll
+                for (int nt = 0; nt < NTT; ++nt) {
+                    uint32_t x0, x1, x2, x3;
+                    asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];"
+                                 : "=r"(x0), "=r"(x1), "=r"(x2), "=r"(x3)
+                                 : "r"(xb + (uint32_t)((j * NT + 8 * nt) * 64)));
+                    mma_bf16_16816(acc[nt], oa[0], ob[0], oa[1], ob[1], x0, x1);
+                    mma_bf16_16816(acc[nt], oa[2], ob[2], oa[3], ob[3], x2, x3);
+                }
+            }
+            __syncwarp();
+            if (lane == 0) tc::mbar_arrive(empty(st));
+        };
+        for (int i = grp; i < nu && ok; i += 2) {
+            do_unit(i, ((i >> 1) & 1) ? bB : bA);
+            if (!ok) break;
+            // the group's next unit is i + 2: finish this tile's segment when it leaves the tile
+            const int cur = tile;
+            unit_advance(tile, ks, 2, nks);
+            if (tile != cur || i + 2 >= nu) fixup(cur);
+        }
+    }
+    __syncthreads();
+}
+
+}  // namespace gmv
+}  // namespace qnf4

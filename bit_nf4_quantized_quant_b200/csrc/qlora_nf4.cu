@@ -13,7 +13,9 @@
 
 #include "common.cuh"
 #include "quant.cuh"
-#include "small.cuh"
+#include "small_lora.cuh"
+#include "tcs_gemm.cuh"
+#include "gemv_mma.cuh"
 #include "lora.cuh"
 #include "tc_gemm.cuh"
 #include "tc2_gemm.cuh"
@@ -72,11 +74,20 @@ inline void note_launch(int n = 1) { g_launches.fetch_add(n, std::memory_order_r
 thread_local cudaEvent_t t_ev_before = nullptr;
 thread_local cudaEvent_t t_ev_after = nullptr;
 
+// Under stream capture the record becomes an event-record node of the graph
+// (external record), so each replay of the graph re-records it.
+inline void record_hook(cudaEvent_t ev, cudaStream_t st) {
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(st, &cs) == cudaSuccess && cs == cudaStreamCaptureStatusActive)
+        cudaEventRecordWithFlags(ev, st, cudaEventRecordExternal);
+    else
+        cudaEventRecord(ev, st);
+}
 inline void hook_before(cudaStream_t st) {
-    if (t_ev_before) cudaEventRecord(t_ev_before, st);
+    if (t_ev_before) record_hook(t_ev_before, st);
 }
 inline void hook_after(cudaStream_t st) {
-    if (t_ev_after) cudaEventRecord(t_ev_after, st);
+    if (t_ev_after) record_hook(t_ev_after, st);
     t_ev_before = nullptr;
     t_ev_after = nullptr;
 }
@@ -100,10 +111,17 @@ int check_device(int* sm_count) {
         if (st == 1) {
             // opt in to more than 48 KB of dynamic shared memory, once per device
             const cudaError_t e = [&] {
-                cudaError_t r = cudaFuncSetAttribute(k_bwd_small<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                               bwd_small_smem_bytes<1>());
-                if (r == cudaSuccess) r = cudaFuncSetAttribute(k_bwd_small<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                               bwd_small_smem_bytes<2>());
+                cudaError_t r = cudaSuccess;
+                // the small adapter kernels run next to (or just before) the fused kernels,
+                // which need most of shared memory: keep the SM in its shared-memory-heavy
+                // configuration so that the next kernel's CTAs need no reconfiguration
+                const void* smalls[] = {(const void*)k_lora_down_small<1>, (const void*)k_lora_down_small<2>,
+                                        (const void*)k_lora_down_small<4>, (const void*)k_lora_down_small<8>,
+                                        (const void*)k_lora_bwd_small, (const void*)k_bwd_small_end};
+                for (const void* f : smalls)
+                    if (r == cudaSuccess)
+                        r = cudaFuncSetAttribute(f, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                                 (int)cudaSharedmemCarveoutMaxShared);
                 return r;
             }();
             if (e != cudaSuccess) return QLORA_ERR_LAUNCH;
@@ -132,11 +150,12 @@ struct Plan {
     // split-K choices
     int zT, zU, zA, zB;
     int64_t kT, kU, kA, kB;         // k per split
-    int S_bwd;                      // small-path N splits for dX
-    int64_t rows_per_split;
-    int KS, J;                      // small-path forward: K splits, macro-steps per split
+    int US;                         // small-path U = dY B: N splits
+    int64_t rows_u;                 //   rows of B per split
+    int NT;                         // small-path token tile of the tcgen05 kernel (16 or 32)
+    int64_t ncnt;                   // arrival counters in the workspace
     // byte offsets
-    size_t off_part, off_cnt, off_T32, off_U32, off_Tp, off_Ubf, off_sT, off_sU, off_Bp, off_At, total;
+    size_t off_slots, off_lslots, off_Upart, off_part, off_cnt, off_T32, off_U32, off_Tp, off_Ubf, off_sT, off_sU, off_Bp, total;
 };
 
 size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
@@ -163,6 +182,9 @@ int choose_splits(int64_t tiles, int64_t kd, int64_t target) {
     return (int)z;
 }
 
+// CTAs of the small-M tcgen05 kernel: at most one per SM of a B200.
+constexpr int64_t kMaxCtas = 148;
+
 Plan make_plan(int64_t M, int64_t N, int64_t K, int r, int sms) {
     Plan p{};
     p.M = M; p.N = N; p.K = K; p.r = r;
@@ -187,45 +209,60 @@ Plan make_plan(int64_t M, int64_t N, int64_t K, int r, int sms) {
     p.zB = choose_splits(cdiv(N, 64) * cdiv(p.rp, bj), M, target);
     p.kB = rup(cdiv(M, p.zB), 32);
     p.zB = (int)cdiv(M, p.kB);
-    // small-path dX: units = (K/64) * S, rows per split a multiple of 256
+    // small-path U partials: up to 64 splits of at least 128 rows
     {
-        const int64_t nblk = K / kBlock;
-        int64_t S = cdiv(target, nblk);
-        if (S < 1) S = 1;
-        int64_t rps = rup(cdiv(N, S), kBwdChunk);
-        p.rows_per_split = rps;
-        p.S_bwd = (int)cdiv(N, rps);
+        int64_t us = cdiv(N, 128);
+        if (us > 64) us = 64;
+        p.rows_u = rup(cdiv(N, us), 8);
+        p.US = (int)cdiv(N, p.rows_u);
     }
-    // small-path forward: about 16 resident warps per SM, each owning 8 rows x J macro-steps
-    {
-        const int64_t nms = cdiv(K / kBlock, 4), nrg = cdiv(N, 8);
-        const int64_t slots = 16LL * sms;
-        int64_t ks = (slots + nrg / 2) / nrg;
-        if (ks < 1) ks = 1;
-        if (ks > nms) ks = nms;
-        p.J = (int)cdiv(nms, ks);
-        p.KS = (int)cdiv(nms, p.J);
-    }
+    // regions of the path this M takes (the other path's are left empty)
+    const bool small = M <= 32;
     size_t part = 0;
     auto upd = [&](size_t b) { if (b > part) part = b; };
-    if (M <= 32) upd((size_t)p.KS * M * N * 4);          // small-path forward partials
-    upd(gemm_part_bytes(M, p.rp, p.zT));
-    upd(gemm_part_bytes(M, p.rp, p.zU));
-    upd(gemm_part_bytes(2 * p.rp, K, p.zA));
-    upd(gemm_part_bytes(N, 2 * p.rp, p.zB));
-    if (M <= 32) upd((size_t)p.S_bwd * M * K * 4);     // small-path dX partials
+    if (small) {
+    } else {
+        upd(gemm_part_bytes(M, p.rp, p.zT));
+        upd(gemm_part_bytes(M, p.rp, p.zU));
+        upd(gemm_part_bytes(2 * p.rp, K, p.zA));
+        upd(gemm_part_bytes(N, 2 * p.rp, p.zB));
+    }
+    // small-path tcgen05 kernel: per-CTA partial tiles of 128 x NT fp32 (slot = CTA + tile)
+    // and one arrival counter per output tile, forward (tiles over N) and backward (over K)
+    size_t slots = 0, ncnt = (size_t)cdiv(N, 8);
+    p.NT = M <= 16 ? 16 : 32;
+    if (small) {
+        for (int bwd = 0; bwd < 2; ++bwd) {
+            const int64_t tiles = cdiv(bwd ? K : N, tcs::TR), units = tiles * cdiv(bwd ? N : K, tcs::KSTEP);
+            const int64_t ctas = units < kMaxCtas ? units : kMaxCtas;
+            const size_t b = (size_t)(ctas + tiles) * p.NT * tcs::TR * 4;
+            if (b > slots) slots = b;
+            if ((size_t)(4 * tiles) > ncnt) ncnt = (size_t)(4 * tiles);
+        }
+        upd((size_t)M * K * 4);                    // backward dY W' sum
+        // forward GEMV: partial tiles of 128 x NT per (CTA + tile, group), counters [tiles][8]
+        const int64_t tiles = cdiv(N, gmv::TR), units = tiles * cdiv(K, gmv::KSTEP);
+        const int64_t ctas = units < kMaxCtas ? units : kMaxCtas;
+        const size_t b = (size_t)(ctas + tiles) * 2 * p.NT * gmv::TR * 4;
+        if (b > slots) slots = b;
+        if ((size_t)(tiles * gmv::kGroupWarps) > ncnt) ncnt = (size_t)(tiles * gmv::kGroupWarps);
+    }
+    const size_t big = small ? 0 : 1;
     size_t off = 0;
     auto take = [&](size_t b) { const size_t o = off; off = align256(off + b); return o; };
+    p.off_slots = take(slots);
+    p.off_lslots = take(small ? (size_t)cdiv(N, tcs::TR) * p.NT * tcs::TR * 4 : 0);
+    p.off_Upart = take(small ? (size_t)p.US * M * p.rp * 4 : 0);
     p.off_part = take(part);
-    p.off_cnt = take((size_t)cdiv(N, 8) * 4);
+    p.off_cnt = take(ncnt * 4);
+    p.ncnt = (int64_t)ncnt;
     p.off_T32 = take((size_t)M * p.rp * 4);
-    p.off_U32 = take((size_t)M * p.rp * 4);
-    p.off_Tp = take((size_t)M * 2 * p.rp * 2);     // T hi | lo
-    p.off_Ubf = take((size_t)M * 2 * p.rp * 2);    // U hi | lo
-    p.off_sT = take((size_t)M * p.rp64 * 2);
-    p.off_sU = take((size_t)M * p.rp64 * 2);
-    p.off_Bp = take((size_t)N * p.rp * 2);
-    p.off_At = take((size_t)K * p.rp * 2);
+    p.off_U32 = take(big * M * p.rp * 4);
+    p.off_Tp = take(big * M * 2 * p.rp * 2);     // T hi | lo
+    p.off_Ubf = take(big * M * 2 * p.rp * 2);    // U hi | lo
+    p.off_sT = take(big * M * p.rp64 * 2);
+    p.off_sU = take(big * M * p.rp64 * 2);
+    p.off_Bp = take(big * N * p.rp * 2);
     p.total = off;
     return p;
 }
@@ -270,7 +307,7 @@ FinishArgs fin_none() {
 int validate_weight(const nf4dq_weight* w) {
     if (!w || !w->packed || !w->codes || !w->scale || !w->mean) return QLORA_ERR_NULL;
     if (w->N <= 0 || w->K <= 0 || (w->K % kBlock) != 0 || (w->N % 8) != 0) return QLORA_ERR_SHAPE;
-    if (w->N > (int64_t)1 << 31 || w->K > (int64_t)1 << 31 || w->N * w->K > ((int64_t)1 << 40)) return QLORA_ERR_SHAPE;
+    if (w->N > (int64_t)1 << 31 || w->K > (int64_t)1 << 31 || w->N * w->K >= ((int64_t)1 << 38)) return QLORA_ERR_SHAPE;
     if (!aligned16(w->packed)) return QLORA_ERR_ALIGN;
     return QLORA_OK;
 }
@@ -325,7 +362,15 @@ int ensure_tc_attrs() {
             cudaFuncSetAttribute(tc2::k_tc2_gemm<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  tc2::SMEM_ALLOC) != cudaSuccess ||
             cudaFuncSetAttribute(tc2::k_tc2_gemm<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 tc2::SMEM_ALLOC) != cudaSuccess)
+                                 tc2::SMEM_ALLOC) != cudaSuccess ||
+            cudaFuncSetAttribute(tcs::k_tcs_gemm<false, 16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 tcs::SMEM_ALLOC) != cudaSuccess ||
+            cudaFuncSetAttribute(tcs::k_tcs_gemm<false, 32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 tcs::SMEM_ALLOC) != cudaSuccess ||
+            cudaFuncSetAttribute(tcs::k_tcs_gemm<true, 16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 tcs::SMEM_ALLOC) != cudaSuccess ||
+            cudaFuncSetAttribute(tcs::k_tcs_gemm<true, 32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 tcs::SMEM_ALLOC) != cudaSuccess)
             return QLORA_ERR_LAUNCH;
         // pairs of SMs that can hold one cluster each at the same time
         cudaLaunchConfig_t cfg = {};
@@ -448,6 +493,172 @@ int compute_T(const Plan& p, const uint16_t* X, const uint16_t* A, float s, uint
 }
 
 
+// Launch with programmatic stream serialization: the kernel may start while
+// the kernel before it on the stream is still running (that kernel calls
+// grid_dep_launch() first; this one calls grid_dep_wait() before it reads
+// anything the other writes).
+template <typename... KArgs, typename... Args>
+int launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st, Args... args) {
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    at[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, args...);
+    note_launch();
+    return e == cudaSuccess ? QLORA_OK : QLORA_ERR_LAUNCH;
+}
+
+// Small-M T = X A^T into T32 (and the caller's bf16 T_out); clears `zero`.
+int small_T(const Plan& p, const uint16_t* X, const uint16_t* A, uint16_t* T_out, int* zero, int zero_n,
+            uint8_t* ws, cudaStream_t st) {
+    LoraDownArgs d{};
+    d.X = X; d.A = A; d.M = p.M; d.K = p.K; d.r = p.r; d.rp = p.rp;
+    d.T32 = reinterpret_cast<float*>(ws + p.off_T32);
+    d.T_out = T_out; d.zero = zero; d.zero_n = zero_n;
+    const int mg = p.M <= 1 ? 1 : p.M <= 2 ? 2 : p.M <= 4 ? 4 : 8;
+    const dim3 grid((unsigned)p.r, (unsigned)cdiv(p.M, mg));
+    switch (mg) {
+        case 1: k_lora_down_small<1><<<grid, kLoraThreads, 0, st>>>(d); break;
+        case 2: k_lora_down_small<2><<<grid, kLoraThreads, 0, st>>>(d); break;
+        case 4: k_lora_down_small<4><<<grid, kLoraThreads, 0, st>>>(d); break;
+        default: k_lora_down_small<8><<<grid, kLoraThreads, 0, st>>>(d); break;
+    }
+    note_launch();
+    return launch_status();
+}
+
+// Small-M fused dequant-GEMM on tcgen05 (stream-K over one CTA per SM),
+// launched programmatically after the adapter kernel before it.
+template <bool BWD>
+int launch_tcs(const Plan& p, const nf4dq_weight* w, const uint16_t* act, const uint16_t* Bl, float s,
+               uint16_t* Y, float* dxsum, uint8_t* wsb, int sms, cudaStream_t st) {
+    int rc = ensure_tc_attrs();
+    if (rc != QLORA_OK) return rc;
+    const int64_t M = p.M, N = p.N, K = p.K;
+    const int64_t n_out = BWD ? K : N, n_red = BWD ? N : K;
+    CUtensorMap tmX, tmP;
+    if (!make_map_2d(&tmX, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, act, n_red, M, n_red * 2, 64, p.NT,
+                     CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_map_2d(&tmP, CU_TENSOR_MAP_DATA_TYPE_UINT8, w->packed, K / 2, N, K / 2, 64, tcs::TR,
+                     CU_TENSOR_MAP_SWIZZLE_64B))
+        return QLORA_ERR_LAUNCH;
+    tcs::Args a{};
+    a.codes = w->codes; a.scale = w->scale; a.mean = w->mean;
+    a.M = M; a.N = N; a.K = K; a.n_out = n_out; a.n_red = n_red;
+    a.tiles = (int)cdiv(n_out, tcs::TR);
+    a.nks = (int)cdiv(n_red, tcs::KSTEP);
+    a.units = (int64_t)a.tiles * a.nks;
+    int64_t ctas = sms < kMaxCtas ? sms : kMaxCtas;
+    if (ctas > a.units) ctas = a.units;
+    a.ctas = (int)ctas;
+    a.slots = reinterpret_cast<float*>(wsb + p.off_slots);
+    a.lslots = reinterpret_cast<float*>(wsb + p.off_lslots);
+    a.counters = reinterpret_cast<int*>(wsb + p.off_cnt);
+    a.T32 = reinterpret_cast<const float*>(wsb + p.off_T32); a.rp = p.rp; a.r = p.r;
+    a.lora_B = Bl; a.s = s; a.Y = Y; a.dxsum = dxsum;
+    a.b_vec = (Bl != nullptr && p.r % 8 == 0 && aligned16(Bl)) ? 1 : 0;
+    const dim3 grid((unsigned)ctas), block(tcs::kThreads);
+    if (p.NT == 16) return launch_pdl(tcs::k_tcs_gemm<BWD, 16>, grid, block, tcs::SMEM_ALLOC, st, tmX, tmP, a, tables());
+    return launch_pdl(tcs::k_tcs_gemm<BWD, 32>, grid, block, tcs::SMEM_ALLOC, st, tmX, tmP, a, tables());
+}
+
+// Small-M forward GEMV (mma.sync, stream-K over one CTA per SM), launched
+// programmatically after the T kernel.
+template <int NTT>
+int launch_gemv_ntt(const Plan& p, const nf4dq_weight* w, const uint16_t* X, const uint16_t* B, float s, uint16_t* Y,
+                    uint8_t* wsb, int sms, cudaStream_t st) {
+    using C = gmv::Cfg<NTT>;
+    static bool attr_set[64];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return QLORA_ERR_DEVICE;
+    if (!attr_set[dev]) {
+        std::lock_guard<std::mutex> lk(g_tc_mu);
+        if (cudaFuncSetAttribute(gmv::k_nf4_gemv<NTT>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_ALLOC) !=
+            cudaSuccess)
+            return QLORA_ERR_LAUNCH;
+        attr_set[dev] = true;
+    }
+    const int64_t N = p.N, K = p.K;
+    CUtensorMap tmP;
+    if (!make_map_2d(&tmP, CU_TENSOR_MAP_DATA_TYPE_UINT8, w->packed, K / 2, N, K / 2, gmv::KSTEP / 2, gmv::TR,
+                     CU_TENSOR_MAP_SWIZZLE_128B))
+        return QLORA_ERR_LAUNCH;
+    gmv::Args a{};
+    a.X = X; a.codes = w->codes; a.scale = w->scale; a.mean = w->mean;
+    a.M = p.M; a.N = N; a.K = K;
+    a.tiles = (int)cdiv(N, gmv::TR);
+    a.nks = (int)cdiv(K, gmv::KSTEP);
+    a.units = (int64_t)a.tiles * a.nks;
+    int64_t ctas = sms < kMaxCtas ? sms : kMaxCtas;
+    if (ctas > a.units) ctas = a.units;
+    a.ctas = (int)ctas;
+    a.slots = reinterpret_cast<float*>(wsb + p.off_slots);
+    a.counters = reinterpret_cast<int*>(wsb + p.off_cnt);
+    a.T32 = reinterpret_cast<const float*>(wsb + p.off_T32); a.rp = p.rp; a.r = p.r;
+    a.lora_B = B; a.s = s; a.Y = Y;
+    return launch_pdl(gmv::k_nf4_gemv<NTT>, dim3((unsigned)ctas), dim3(gmv::kThreads), (size_t)C::SMEM_ALLOC, st, tmP,
+                      a, tables());
+}
+
+int launch_gemv(const Plan& p, const nf4dq_weight* w, const uint16_t* X, const uint16_t* B, float s, uint16_t* Y,
+                uint8_t* wsb, int sms, cudaStream_t st) {
+    if (p.M <= 8) return launch_gemv_ntt<1>(p, w, X, B, s, Y, wsb, sms, st);
+    if (p.M <= 16) return launch_gemv_ntt<2>(p, w, X, B, s, Y, wsb, sms, st);
+    return launch_gemv_ntt<4>(p, w, X, B, s, Y, wsb, sms, st);
+}
+
+// Small-M forward: T = X A^T, then the fused GEMV, which overlaps the T
+// kernel and adds s T B^T when it finishes a tile.
+int small_fwd(const Plan& p, const uint16_t* X, const nf4dq_weight* w, const uint16_t* A, const uint16_t* B,
+              float scaling, uint16_t* Y, uint16_t* T_out, uint8_t* wsb, int sms, cudaStream_t st) {
+    hook_before(st);
+    int rc = small_T(p, X, A, T_out, reinterpret_cast<int*>(wsb + p.off_cnt), (int)p.ncnt, wsb, st);
+    if (rc != QLORA_OK) return rc;
+    rc = launch_gemv(p, w, X, B, scaling, Y, wsb, sms, st);
+    hook_after(st);
+    return rc;
+}
+
+// Small-M backward: [T], U partials + dB (and the counters cleared), the fused
+// dY W' kernel (overlapping the U / dB kernel), then dX = dY W' + s U A and dA.
+int small_bwd(const Plan& p, const uint16_t* X, const uint16_t* dY, const nf4dq_weight* w, const uint16_t* A,
+              const uint16_t* B, float scaling, const uint16_t* T, uint16_t* dX, uint16_t* dA, uint16_t* dB,
+              uint8_t* wsb, int sms, cudaStream_t st) {
+    int rc = QLORA_OK;
+    const float* T32 = nullptr;
+    if (T == nullptr) {
+        rc = small_T(p, X, A, nullptr, nullptr, 0, wsb, st);
+        if (rc != QLORA_OK) return rc;
+        T32 = reinterpret_cast<const float*>(wsb + p.off_T32);
+    }
+    hook_before(st);
+    LoraBwdArgs b{};
+    b.dY = dY; b.B = B; b.T32 = T32; b.Tb = T; b.M = p.M; b.N = p.N; b.r = p.r; b.rp = p.rp; b.s = scaling;
+    b.b_vec = (p.r % 8 == 0 && aligned16(B)) ? 1 : 0;
+    b.Upart = reinterpret_cast<float*>(wsb + p.off_Upart); b.US = p.US; b.rows_u = p.rows_u; b.dB = dB;
+    b.zero = reinterpret_cast<int*>(wsb + p.off_cnt); b.zero_n = (int)p.ncnt;
+    k_lora_bwd_small<<<(unsigned)(p.US + cdiv(p.N, kLoraThreads)), kLoraThreads, 0, st>>>(b);
+    note_launch();
+    rc = launch_status();
+    if (rc != QLORA_OK) return rc;
+    float* dxsum = reinterpret_cast<float*>(wsb + p.off_part);
+    rc = launch_tcs<true>(p, w, dY, nullptr, scaling, nullptr, dxsum, wsb, sms, st);
+    hook_after(st);
+    if (rc != QLORA_OK) return rc;
+    BwdEndArgs e{};
+    e.part = dxsum; e.S = 1; e.Upart = b.Upart; e.US = p.US; e.A = A; e.X = X;
+    e.M = p.M; e.K = p.K; e.r = p.r; e.rp = p.rp; e.s = scaling; e.dX = dX; e.dA = dA;
+    k_bwd_small_end<<<dim3((unsigned)cdiv(p.K, kLoraThreads), (unsigned)(p.M + p.r)), kLoraThreads, 0, st>>>(e);
+    note_launch();
+    return launch_status();
+}
+
 }  // namespace
 
 // ===========================================================================
@@ -529,28 +740,14 @@ int qlora_linear_fwd(const qlora_bf16* X, int64_t M, const nf4dq_weight* w, cons
     cudaStream_t st = (cudaStream_t)stream;
     uint8_t* wsb = static_cast<uint8_t*>(ws);
 
-    rc = compute_T(p, X, A, scaling, T_out, wsb, sms, st);
-    if (rc != QLORA_OK) return rc;
-
     if (M <= kSmallMaxM) {
-        SmallFwdArgs a{};
-        a.X = X; a.packed = w->packed; a.codes = w->codes; a.scale = w->scale; a.mean = w->mean;
-        a.T32 = reinterpret_cast<const float*>(wsb + p.off_T32); a.B = B; a.Y = Y;
-        a.part = reinterpret_cast<float*>(wsb + p.off_part);
-        a.counters = reinterpret_cast<int*>(wsb + p.off_cnt);
-        a.M = M; a.N = w->N; a.K = w->K; a.rp = p.rp; a.r = r; a.s = scaling; a.KS = p.KS; a.J = p.J;
-        const int64_t items = cdiv(w->N, 8) * p.KS;
-        const int64_t warps = items < 16LL * sms ? items : 16LL * sms;
-        const int grid = (int)cdiv(warps, kGemvThreads / 32);
-        hook_before(st);
-        if (M <= 16) k_fwd_gemv<1><<<grid, kGemvThreads, 0, st>>>(a, tables());
-        else k_fwd_gemv<2><<<grid, kGemvThreads, 0, st>>>(a, tables());
-        hook_after(st);
-        note_launch();
-        rc = launch_status();
+        rc = small_fwd(p, X, w, A, B, scaling, Y, T_out, wsb, sms, st);
         if (rc == QLORA_OK) t_last_path = 1;
         return rc;
     }
+    rc = compute_T(p, X, A, scaling, T_out, wsb, sms, st);
+    if (rc != QLORA_OK) return rc;
+
     // tcgen05 path: LoRA weight rows must be 16-byte granular (r % 8 == 0) or padded
     const uint16_t* lw = B;
     int64_t ldl = r;
@@ -597,6 +794,11 @@ int qlora_linear_bwd(const qlora_bf16* X, const qlora_bf16* dY, int64_t M, const
     if (ws_bytes < p.total) return QLORA_ERR_WORKSPACE;
     cudaStream_t st = (cudaStream_t)stream;
     uint8_t* wsb = static_cast<uint8_t*>(ws);
+    if (M <= kSmallMaxM) {
+        rc = small_bwd(p, X, dY, w, A, B, scaling, T, dX, dA, dB, wsb, sms, st);
+        if (rc == QLORA_OK) t_last_path = 1;
+        return rc;
+    }
     float* part = reinterpret_cast<float*>(wsb + p.off_part);
     uint16_t* Thl = reinterpret_cast<uint16_t*>(wsb + p.off_Tp);
     uint16_t* Uhl = reinterpret_cast<uint16_t*>(wsb + p.off_Ubf);
@@ -648,40 +850,18 @@ int qlora_linear_bwd(const qlora_bf16* X, const qlora_bf16* dY, int64_t M, const
         if (rc != QLORA_OK) return rc;
     }
     // dX = dY W' + s U A
-    if (M > kSmallMaxM) {
-        rc = ensure_tc_attrs();
-        if (rc != QLORA_OK) return rc;
-        const int pairs = current_pairs();
-        if (M > kPairMinM && pairs > 0) {
-            rc = launch_tc2<true>(w, dY, M, reinterpret_cast<const uint16_t*>(wsb + p.off_sU), p.rp64, A, K, r, dX,
-                                  pairs, st);
-            if (rc == QLORA_OK) t_last_path = 3;
-            return rc;
-        }
-        rc = launch_tc<true>(w, dY, M, reinterpret_cast<const uint16_t*>(wsb + p.off_sU), p.rp64, A, K, r, dX, sms,
-                             st);
-        if (rc == QLORA_OK) t_last_path = 2;
+    rc = ensure_tc_attrs();
+    if (rc != QLORA_OK) return rc;
+    const int pairs = current_pairs();
+    if (M > kPairMinM && pairs > 0) {
+        rc = launch_tc2<true>(w, dY, M, reinterpret_cast<const uint16_t*>(wsb + p.off_sU), p.rp64, A, K, r, dX,
+                              pairs, st);
+        if (rc == QLORA_OK) t_last_path = 3;
         return rc;
     }
-    {
-        SmallBwdArgs a{};
-        a.dY = dY; a.packed = w->packed; a.codes = w->codes; a.scale = w->scale; a.mean = w->mean;
-        a.part = part; a.M = M; a.N = N; a.K = K; a.rows_per_split = p.rows_per_split; a.S = p.S_bwd;
-        const int64_t units = (K / kBlock) * p.S_bwd;
-        const int grid = (int)(units < 2LL * sms ? units : 2LL * sms);
-        hook_before(st);
-        if (M <= 16) k_bwd_small<1><<<grid, kBwdThreads, bwd_small_smem_bytes<1>(), st>>>(a, tables());
-        else k_bwd_small<2><<<grid, kBwdThreads, bwd_small_smem_bytes<2>(), st>>>(a, tables());
-        hook_after(st);
-        note_launch();
-        k_bwd_small_finish<<<grid_for(M * K, 256, sms), 256, 0, st>>>(
-            part, p.S_bwd, M, K, reinterpret_cast<const float*>(wsb + p.off_U32), p.rp, A, r, scaling, dX);
-        note_launch();
-        rc = launch_status();
-        if (rc != QLORA_OK) return rc;
-    }
-    t_last_path = 1;
-    return QLORA_OK;
+    rc = launch_tc<true>(w, dY, M, reinterpret_cast<const uint16_t*>(wsb + p.off_sU), p.rp64, A, K, r, dX, sms, st);
+    if (rc == QLORA_OK) t_last_path = 2;
+    return rc;
 }
 
 

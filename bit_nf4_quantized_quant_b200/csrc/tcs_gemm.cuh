@@ -1,0 +1,446 @@
+// tcs_gemm.cuh -- fused NF4 dequant + GEMM on tcgen05 for a few tokens
+// (M <= 32): the decode / small-batch shape, where the layer is bound by the
+// exact dequantization of the 4.13-bit weight stream (integer-pipe work per
+// weight), not by tensor work.
+//
+//   forward : Y^T  [N, M] = W'   [N, K] . X^T  [K, M]    + s B T^T
+//   backward: dX^T [K, M] = W'^T [K, N] . dY^T [N, M]    (s A^T U^T added later)
+//
+// The weight is the MMA's A operand (M_mma = 128 rows of W, or 128 columns
+// of W in the backward) and the tokens are its N dimension (NT = 16 or 32,
+// zero rows beyond M come from the TMA's out-of-bound fill), so one
+// tcgen05.mma of 128 x NT x 16 does all the tensor work of 2048 weights.
+// Work unit = (output tile of 128, reduction step of 128).  The units of a
+// problem are split evenly over one CTA per SM in (tile, step) order
+// ("stream-K"), so every SM decodes the same number of weights; a tile whose
+// steps span several CTAs is finished, per TMEM lane quarter, by the warp
+// that arrives last on that quarter's counter, which sums the per-CTA
+// partials in CTA order (the result does not depend on arrival order).
+//
+// Warp roles (768 threads, one CTA per SM):
+//   warp 0      TMA producer of the activation tiles (NT x 128 bf16, two
+//               128-byte-swizzled boxes of 64 columns);
+//   warp 1      TMEM allocator and MMA issuer: 8 MMAs of 128 x NT x 16 per unit;
+//   warp 2      TMA producer of the packed NF4 tiles (128 rows x 64 B, 64-byte
+//               swizzle), 8 units ahead;
+//   warps 4-7   epilogue: the LoRA term of a tile while its MMAs run, then
+//               TMEM -> registers -> partial or finished output;
+//   warps 8-23  dequantizers, two groups of 8 warps taking alternate units (16
+//               warps keep the integer pipe busy while others wait): thread d
+//               of a group owns one 64-weight row-block per unit (row
+//               8 (d / 16) + d % 8, block (d / 8) % 2), exact bf16_rne(L[q] c')
+//               from the per-block register table, written into the swizzled
+//               A-operand layout (K-major in the forward, MN-major in the
+//               backward, where W's rows are the reduction).
+#pragma once
+#include "tc_gemm.cuh"
+
+namespace qnf4 {
+namespace tcs {
+
+constexpr int TR = 128;                    // output rows of a tile (MMA M)
+constexpr int KSTEP = 128;                 // reduction per step
+constexpr int SX = 3;                      // activation ring stages
+constexpr int SW = 4;                      // dequantized weight ring stages (2 per decoder group)
+constexpr int SP = 8;                      // packed weight ring stages (4 per decoder group)
+constexpr int X_BYTES_MAX = 32 * KSTEP * 2;        // 8192 (NT = 32)
+constexpr int W_BYTES = TR * KSTEP * 2;            // 32768
+constexpr int P_BYTES = TR * KSTEP / 2;            // 8192
+constexpr int kThreads = 768;
+constexpr int kGroupThreads = 256;         // one decoder group
+constexpr int kEpiThreads = 128;
+
+constexpr int OFF_X = 0;
+constexpr int OFF_W = OFF_X + SX * X_BYTES_MAX;
+constexpr int OFF_P = OFF_W + SW * W_BYTES;
+constexpr int OFF_BAR = OFF_P + SP * P_BYTES;
+// fullX[SX] emptyX[SX] fullW[SW] emptyW[SW] fullP[SP] emptyP[SP] tfull[2] tempty[2] drain
+constexpr int NBAR = 2 * SX + 2 * SW + 2 * SP + 4 + 1;
+constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
+constexpr int SMEM_BYTES = OFF_MISC + 16;
+constexpr int SMEM_ALLOC = SMEM_BYTES + 1024;
+
+struct Args {
+    const int8_t* codes;
+    const float* scale;
+    const float* mean;
+    int64_t M, N, K;           // W is [N, K]
+    int64_t n_out, n_red;      // forward: N, K;  backward: K, N
+    int tiles, nks;            // ceil(n_out / 128), ceil(n_red / 128)
+    int64_t units;             // tiles * nks
+    int ctas;                  // grid size
+    float* slots;              // [ctas + tiles][NT][128] fp32 partials
+    float* lslots;             // forward: [tiles][NT][128] fp32 LoRA terms
+    int* counters;             // [tiles][4] (per TMEM lane quarter), zero on entry, left zero
+    // forward finish: Y = acc + s T B^T
+    const float* T32;          // [M, rp]
+    int rp, r;
+    const uint16_t* lora_B;    // [N, r]
+    int b_vec;                 // rows of lora_B are 16-byte loadable
+    float s;
+    uint16_t* Y;               // [M, N]
+    // backward finish: the dY W' sum in fp32
+    float* dxsum;              // [M, K]
+};
+
+// First unit of CTA c, and the CTA that owns unit u, for an even split of U units over C CTAs.
+__host__ __device__ __forceinline__ int64_t unit_begin(int64_t c, int64_t U, int64_t C) { return c * U / C; }
+__host__ __device__ __forceinline__ int64_t unit_owner(int64_t u, int64_t U, int64_t C) {
+    return ((u + 1) * C + U - 1) / U - 1;
+}
+
+// Instruction descriptor: kind::f16, A = B = bf16, D = f32, M = 128, N = NT, A K- or MN-major.
+__host__ __device__ constexpr uint32_t make_idesc(bool a_mn_major, int nt) {
+    return (1u << 4) | (1u << 7) | (1u << 10) | ((a_mn_major ? 1u : 0u) << 15) | ((uint32_t)(nt >> 3) << 17) |
+           ((uint32_t)(TR >> 4) << 24);
+}
+
+#define TCS_LD16(taddr, r)                                                                                         \
+    asm volatile(                                                                                                  \
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"   \
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),        \
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])   \
+        : "r"(taddr))
+
+// Row-block of dequantizer thread d in a step: row 0..127 of the step and block 0..1.
+// A quarter-warp holds 8 consecutive rows of one block, so its packed reads
+// (64-byte swizzle) and its stores into the operand tile are conflict-free.
+__device__ __forceinline__ int deq_row(int d) { return 8 * (d >> 4) + (d & 7); }
+__device__ __forceinline__ int deq_blk(int d) { return (d >> 3) & 1; }
+
+// Byte offset of 16-byte chunk ch (8 weights) of thread d's row-block in the
+// operand tile.  Forward (K-major, two 64-column halves of 16 KB): half j, row
+// n, chunk ch ^ (n % 8).  Backward (MN-major: the tile's 128 rows are the
+// reduction, its 2 x 64 columns the MMA's M): atom column j 16 KB apart, 8-row
+// group n / 8 1 KB apart, row n % 8, chunk ch ^ (n % 8).
+template <bool BWD>
+__device__ __forceinline__ uint32_t w_chunk_offset(int d, int ch) {
+    const int n = deq_row(d), j = deq_blk(d);
+    if (!BWD) return (uint32_t)(j * 16384 + n * 128 + ((ch ^ (n & 7)) << 4));
+    return (uint32_t)(j * 16384 + (n >> 3) * 1024 + (n & 7) * 128 + ((ch ^ (n & 7)) << 4));
+}
+
+// Packed tile: 128 rows x 64 B (two blocks), 64-byte swizzle (chunk ^= (row / 2) % 4).
+__device__ __forceinline__ uint32_t p_chunk_offset(int d, int c) {
+    const int n = deq_row(d), j = deq_blk(d);
+    return (uint32_t)(n * 64 + (((2 * j + c) ^ ((n >> 1) & 3)) << 4));
+}
+
+// Advance a (tile, step) position by n units.
+__device__ __forceinline__ void unit_advance(int& tile, int& ks, int n, int nks) {
+    ks += n;
+    while (ks >= nks) { ks -= nks; ++tile; }
+}
+
+// ----------------------------------------------------------------------------
+template <bool BWD, int NT>
+__global__ void __launch_bounds__(kThreads, 1)
+k_tcs_gemm(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmP, Args a,
+           NF4Tables tab) {
+    constexpr int X_BYTES = NT * KSTEP * 2;
+    constexpr uint32_t kCols = NT == 16 ? 32 : 64;      // 2 accumulators of NT columns
+    extern __shared__ __align__(1024) uint8_t smem[];
+    uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem) + 1023) & ~(uintptr_t)1023);
+    const uint32_t sbase = smem_u32(base);
+    const uint32_t bar0 = sbase + OFF_BAR;
+    auto fullX = [&](int i) { return bar0 + 8 * i; };
+    auto emptyX = [&](int i) { return bar0 + 8 * (SX + i); };
+    auto fullW = [&](int i) { return bar0 + 8 * (2 * SX + i); };
+    auto emptyW = [&](int i) { return bar0 + 8 * (2 * SX + SW + i); };
+    auto fullP = [&](int i) { return bar0 + 8 * (2 * SX + 2 * SW + i); };
+    auto emptyP = [&](int i) { return bar0 + 8 * (2 * SX + 2 * SW + SP + i); };
+    auto tfull = [&](int i) { return bar0 + 8 * (2 * SX + 2 * SW + 2 * SP + i); };
+    auto tempty = [&](int i) { return bar0 + 8 * (2 * SX + 2 * SW + 2 * SP + 2 + i); };
+    const uint32_t drain = bar0 + 8 * (2 * SX + 2 * SW + 2 * SP + 4);
+    uint32_t* s_tmem = reinterpret_cast<uint32_t*>(base + OFF_MISC);
+    volatile int* s_abort = reinterpret_cast<volatile int*>(base + OFF_MISC + 4);
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int64_t U = a.units;
+    // this CTA's units [u0, u1) (fewer than 2^31: the weight has fewer than 2^38
+    // elements); unit i of the CTA is u0 + i, and loops walk (tile, step) incrementally
+    const int u0 = (int)unit_begin(blockIdx.x, U, a.ctas), u1 = (int)unit_begin(blockIdx.x + 1, U, a.ctas);
+    const int nu = u1 - u0;
+    const int nks = a.nks;
+    const int tile0 = u0 / nks, ks0 = u0 - tile0 * nks;
+    const int64_t nblk = a.K / kBlock;
+
+    if (tid == 0) {
+        for (int i = 0; i < SX; ++i) { tc::mbar_init(fullX(i), 1); tc::mbar_init(emptyX(i), 1); }
+        for (int i = 0; i < SW; ++i) { tc::mbar_init(fullW(i), kGroupThreads / 32); tc::mbar_init(emptyW(i), 1); }
+        for (int i = 0; i < SP; ++i) { tc::mbar_init(fullP(i), 1); tc::mbar_init(emptyP(i), kGroupThreads / 32); }
+        for (int i = 0; i < 2; ++i) { tc::mbar_init(tfull(i), 1); tc::mbar_init(tempty(i), kEpiThreads / 32); }
+        tc::mbar_init(drain, 1);
+        *s_abort = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(s_tmem)),
+                     "r"(kCols));
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+        tc::tc_fence_before();
+    }
+    __syncthreads();
+    tc::tc_fence_after();
+    const uint32_t tmem_base = *s_tmem;
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ TMA producer: activations
+        if (lane == 0) {
+            int sx = 0, px = 0, issued = 0;
+            bool ok = true;
+            for (int i = 0, ks = ks0; i < nu && ok; ++i, ks = (ks + 1 == nks) ? 0 : ks + 1) {
+                if (!(ok = tc::mbar_wait(emptyX(sx), px ^ 1, s_abort))) break;
+                tc::mbar_expect_tx(fullX(sx), X_BYTES);
+                const uint32_t dst = sbase + OFF_X + sx * X_BYTES_MAX;
+                tc::tma_load_2d(dst, &tmX, fullX(sx), ks * KSTEP, 0);
+                tc::tma_load_2d(dst + NT * 128, &tmX, fullX(sx), ks * KSTEP + 64, 0);
+                ++issued;
+                if (++sx == SX) { sx = 0; px ^= 1; }
+            }
+            if (!ok)
+                for (int k = 1; k <= SX && k <= issued; ++k)
+                    tc::mbar_drain(fullX((issued - k) % SX), ((issued - k) / SX) & 1);
+        }
+    } else if (warp == 2) {
+        // ------------------------------------------------------------ TMA producer: packed weights
+        if (lane == 0) {
+            int issued = 0, tile = tile0, ks = ks0;
+            bool ok = true;
+            for (int i = 0; i < nu && ok; ++i) {
+                const int sp = i & (SP - 1), pp = (i / SP) & 1;
+                if (!(ok = tc::mbar_wait(emptyP(sp), pp ^ 1, s_abort))) break;
+                tc::mbar_expect_tx(fullP(sp), P_BYTES);
+                const uint32_t dst = sbase + OFF_P + sp * P_BYTES;
+                if (!BWD) tc::tma_load_2d(dst, &tmP, fullP(sp), ks * (KSTEP / 2), tile * TR);
+                else tc::tma_load_2d(dst, &tmP, fullP(sp), tile * (TR / 2), ks * KSTEP);
+                ++issued;
+                unit_advance(tile, ks, 1, nks);
+            }
+            if (!ok)
+                for (int k = 1; k <= SP && k <= issued; ++k)
+                    tc::mbar_drain(fullP((issued - k) & (SP - 1)), ((issued - k) / SP) & 1);
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t idesc = make_idesc(BWD, NT);
+            int sx = 0, px = 0, seg = 0, buf = 0;
+            bool ok = true;
+            uint32_t d_tmem = tmem_base;
+            for (int i = 0, ks = ks0; i < nu && ok; ++i, ks = (ks + 1 == nks) ? 0 : ks + 1) {
+                const bool first = (i == 0) || ks == 0;
+                const bool last = (i == nu - 1) || ks == nks - 1;
+                if (first) {
+                    buf = seg & 1;
+                    if (!(ok = tc::mbar_wait(tempty(buf), ((seg >> 1) & 1) ^ 1, s_abort))) break;
+                    tc::tc_fence_after();
+                    d_tmem = tmem_base + (uint32_t)(buf * NT);
+                }
+                const int sw = i & (SW - 1), pw = (i / SW) & 1;
+                if (!(ok = tc::mbar_wait(fullX(sx), px, s_abort))) break;
+                if (!(ok = tc::mbar_wait(fullW(sw), pw, s_abort))) break;
+                tc::tc_fence_after();
+                const uint32_t x_addr = sbase + OFF_X + sx * X_BYTES_MAX;
+                const uint32_t w_addr = sbase + OFF_W + sw * W_BYTES;
+#pragma unroll
+                for (int q = 0; q < KSTEP / 16; ++q) {
+                    const int h = q >> 2, kk = q & 3;
+                    const uint64_t adesc = BWD ? tc::smem_desc_sw128(w_addr + q * 2048, 16384, 1024)
+                                               : tc::smem_desc_sw128(w_addr + h * 16384 + kk * 32, 16, 1024);
+                    const uint64_t bdesc = tc::smem_desc_sw128(x_addr + h * (NT * 128) + kk * 32, 16, 1024);
+                    tc::tc_mma(d_tmem, adesc, bdesc, idesc, (!first || q > 0) ? 1u : 0u);
+                }
+                tc::tc_commit(emptyX(sx));
+                tc::tc_commit(emptyW(sw));
+                if (++sx == SX) { sx = 0; px ^= 1; }
+                if (last) {
+                    tc::tc_commit(tfull(buf));
+                    ++seg;
+                }
+            }
+            tc::tc_commit(drain);
+            tc::mbar_drain(drain, 0);
+        }
+    } else if (warp >= 8) {
+        // ------------------------------------------------------------ dequantizers
+        const int grp = (warp - 8) >> 3;                 // group: units i = grp, grp + 2, ...
+        const int d = tid - 256 - kGroupThreads * grp;   // thread within the group
+        const int drow = deq_row(d), dblk = deq_blk(d);
+        bool ok = true;
+        // fetch position: the unit whose block-constant inputs are loaded next
+        int fi = grp, ft = tile0, fk = ks0;
+        unit_advance(ft, fk, grp, nks);
+        auto fetch = [&](int& code, float& sc, float& mu) {
+            code = 0; sc = 0.f; mu = 0.f;
+            const int tile = ft, ks = fk;
+            const bool in = fi < nu;
+            fi += 2;
+            unit_advance(ft, fk, 2, nks);
+            if (!in) return;
+            int64_t n, kb;
+            if (!BWD) { n = (int64_t)tile * TR + drow; kb = (int64_t)ks * 2 + dblk; }
+            else { n = (int64_t)ks * KSTEP + drow; kb = (int64_t)tile * 2 + dblk; }
+            if (n < a.N && kb < nblk) {
+                const int64_t b = n * nblk + kb;
+                code = __ldg(a.codes + b);
+                sc = __ldg(a.scale + (b >> 8));
+                mu = __ldg(a.mean + (b >> 8));
+            }
+        };
+        // unit i of this group; (code, sc, mu) hold its block-constant inputs and are
+        // refilled with those of unit i + 4 (two register slots alternate)
+        auto do_unit = [&](int i, int& code, float& sc, float& mu) {
+            const float c = __fmaf_rn((float)code, sc, mu);
+            fetch(code, sc, mu);
+            const int sp = i & (SP - 1), pp = (i / SP) & 1;
+            if (!(ok = tc::mbar_wait(fullP(sp), pp, s_abort))) return;
+            uint4 p0, p1;
+            const uint32_t pst = sbase + OFF_P + sp * P_BYTES;
+            const uint32_t src0 = pst + p_chunk_offset(d, 0), src1 = pst + p_chunk_offset(d, 1);
+            asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(p0.x), "=r"(p0.y), "=r"(p0.z), "=r"(p0.w) : "r"(src0));
+            asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(p1.x), "=r"(p1.y), "=r"(p1.z), "=r"(p1.w) : "r"(src1));
+            __syncwarp();
+            if (lane == 0) tc::mbar_arrive(emptyP(sp));
+            const BlockTable tb = make_block_table(tab, c);
+            const uint32_t pwd[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
+            const int sw = i & (SW - 1), pw = (i / SW) & 1;
+            if (!(ok = tc::mbar_wait(emptyW(sw), pw ^ 1, s_abort))) return;
+            const uint32_t wbase = sbase + OFF_W + sw * W_BYTES;
+#pragma unroll
+            for (int ch = 0; ch < 8; ++ch) {
+                uint32_t o[4];
+                decode8(tb, pwd[ch], o);
+                tc::st_shared_v4(wbase + w_chunk_offset<BWD>(d, ch), o[0], o[1], o[2], o[3]);
+            }
+            tc::fence_proxy_async();
+            __syncwarp();
+            if (lane == 0) tc::mbar_arrive(fullW(sw));
+        };
+        int codeA, codeB;
+        float scA, scB, muA, muB;
+        fetch(codeA, scA, muA);
+        fetch(codeB, scB, muB);
+        for (int i = grp; i < nu && ok; i += 4) {
+            do_unit(i, codeA, scA, muA);
+            if (ok && i + 2 < nu) do_unit(i + 2, codeB, scB, muB);
+        }
+    } else if (warp >= 4) {
+        // ------------------------------------------------------------ epilogue
+        const int q = warp & 3;                 // TMEM lane quarter of this warp
+        const int row = q * 32 + lane;
+        // T and the zeroed counters come from the kernel before this one, which may
+        // still be running (programmatic launch)
+        grid_dep_wait();
+        bool ok = true;
+        int seg = 0;
+        for (int u = u0, tile = tile0; u < u1 && ok; ++tile) {
+            const int tile_u0 = tile * nks, tile_u1 = tile_u0 + nks;
+            const int seg_end = tile_u1 < u1 ? tile_u1 : u1;
+            const bool starts = (u == tile_u0);
+            const bool whole = starts && (seg_end == tile_u1);
+            u = seg_end;
+            const int64_t o = (int64_t)tile * TR + row;     // output feature (forward) or column k (backward)
+            float* lp = BWD ? nullptr : a.lslots + (int64_t)tile * (NT * TR);
+            if (!BWD && starts && o < a.N) {
+                // the LoRA term s T B^T of this tile's rows, computed by the CTA that
+                // owns the tile's first step while the MMAs of the segment run
+                const uint16_t* br = a.lora_B + o * a.r;
+                for (int64_t m = 0; m < a.M; ++m) {
+                    const float* tr = a.T32 + m * a.rp;
+                    float l = 0.f;
+                    if (a.b_vec) {
+                        for (int i = 0; i < a.r; i += 8) {
+                            const uint4 bv = __ldg(reinterpret_cast<const uint4*>(br + i));
+                            const uint32_t bw[4] = {bv.x, bv.y, bv.z, bv.w};
+#pragma unroll
+                            for (int j = 0; j < 4; ++j) {
+                                l = __fmaf_rn(tr[i + 2 * j], bf16lo_to_f32(bw[j]), l);
+                                l = __fmaf_rn(tr[i + 2 * j + 1], bf16hi_to_f32(bw[j]), l);
+                            }
+                        }
+                    } else {
+                        for (int i = 0; i < a.r; ++i) l = __fmaf_rn(tr[i], bf16lo_to_f32(br[i]), l);
+                    }
+                    lp[m * TR + row] = a.s * l;
+                }
+            }
+            const int buf = seg & 1;
+            if (!(ok = tc::mbar_wait(tfull(buf), (seg >> 1) & 1, s_abort))) break;
+            ++seg;
+            tc::tc_fence_after();
+            float acc[NT];
+            {
+                uint32_t rr[16];
+                const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(buf * NT);
+#pragma unroll
+                for (int h = 0; h < NT / 16; ++h) {
+                    TCS_LD16(taddr + h * 16, rr);
+                    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) acc[h * 16 + j] = __uint_as_float(rr[j]);
+                }
+            }
+            tc::tc_fence_before();
+            __syncwarp();
+            if (lane == 0) tc::mbar_arrive(tempty(buf));
+            // a split tile: every epilogue warp publishes its 32 rows and arrives on the
+            // counter of (tile, its lane quarter); the last of them sums that quarter
+            bool finish = whole;
+            if (!whole) {
+                const int64_t slot = (int64_t)blockIdx.x + tile;
+                float* sp = a.slots + slot * (NT * TR);
+#pragma unroll
+                for (int m = 0; m < NT; ++m) sp[m * TR + row] = acc[m];
+                __threadfence();
+                __syncwarp();
+                const int64_t c_first = unit_owner(tile_u0, U, a.ctas);
+                const int64_t c_last = unit_owner(tile_u1 - 1, U, a.ctas);
+                int is_last = 0;
+                if (lane == 0) {
+                    int* cnt = a.counters + 4 * (int64_t)tile + q;
+                    is_last = atomicAdd(cnt, 1) == (int)(c_last - c_first);
+                    if (is_last) *cnt = 0;                      // ready for the next call
+                }
+                finish = __shfl_sync(0xffffffffu, is_last, 0) != 0;
+                if (finish) {
+                    __threadfence();
+#pragma unroll
+                    for (int m = 0; m < NT; ++m) acc[m] = 0.f;
+                    for (int64_t c2 = c_first; c2 <= c_last; ++c2) {
+                        const float* p2 = a.slots + (c2 + tile) * (NT * TR);
+#pragma unroll
+                        for (int m = 0; m < NT; ++m) acc[m] += __ldcg(p2 + m * TR + row);
+                    }
+                }
+            }
+            if (!finish) continue;
+            if (!BWD) {
+                if (o < a.N) {
+#pragma unroll
+                    for (int m = 0; m < NT; ++m) {
+                        if (m < a.M) {
+                            const float v = acc[m] + __ldcg(lp + m * TR + row);
+                            a.Y[(int64_t)m * a.N + o] = (uint16_t)(pack_bf16x2(v, 0.f) & 0xffffu);
+                        }
+                    }
+                }
+            } else {
+                if (o < a.K) {
+#pragma unroll
+                    for (int m = 0; m < NT; ++m)
+                        if (m < a.M) a.dxsum[(int64_t)m * a.K + o] = acc[m];
+                }
+            }
+        }
+    }
+
+    __syncthreads();
+    if (warp == 1) {
+        tc::tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(kCols));
+    }
+}
+
+}  // namespace tcs
+}  // namespace qnf4
