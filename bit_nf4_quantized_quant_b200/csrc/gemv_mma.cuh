@@ -17,11 +17,11 @@
 //    two whole blocks (rows g and g + 8) and builds two tables.
 //  * Work unit = (128 rows, 256 reduction) = 8 warps x 16 rows.  The units
 //    are split evenly over the CTAs in (tile, step) order; in a CTA two
-//    groups of 8 warps take alternate units.  Partial sums of a tile that
-//    spans several (CTA, group) pairs are written to per-pair slots; the warp
-//    that arrives last on the (tile, warp row-slice) counter sums them in
-//    (CTA, group) order -- the result does not depend on arrival order -- and
-//    adds s T B^T.
+//    groups of 8 warps take alternate units.  Every (CTA, group) pair writes
+//    its partial sum of each tile it touched to its own slot; the small
+//    k_nf4_gemv_finish kernel sums the slots of a tile in (CTA, group) order
+//    -- deterministic -- and adds s T B^T (no atomics or counters, so the
+//    fused kernel ends as soon as its last unit is done).
 //  * Warp 0 lane 0 loads each unit's packed tile (128 rows x 128 B, 128-byte
 //    swizzle) with TMA; the 32 lanes of warp 0 copy the unit's activation
 //    slice with cp.async into a fragment-native layout ([j][token][t] 16-byte
@@ -62,13 +62,7 @@ struct Args {
     int tiles, nks;            // ceil(N / 128), ceil(K / 256)
     int64_t units;             // tiles * nks
     int ctas;
-    float* slots;              // [(ctas + tiles) * 2][NT][128] fp32 partials
-    int* counters;             // [tiles][8], zero on entry, left zero
-    const float* T32;          // [M, rp] fp32 LoRA down-projection
-    int rp, r;
-    const uint16_t* lora_B;    // [N, r]
-    float s;
-    uint16_t* Y;               // [M, N]
+    float* slots;              // [(ctas + tiles) * 2][NT][128] fp32 partial tiles
 };
 
 __host__ __device__ __forceinline__ int64_t unit_begin(int64_t c, int64_t U, int64_t C) { return c * U / C; }
@@ -175,7 +169,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_nf4_gemv(const __grid_constant_
         const int w8 = (warp - 1) % kGroupWarps;         // rows 16 w8 .. 16 w8 + 15 of a unit
         const int g = lane >> 2, t = lane & 3;
         const int r0 = 16 * w8 + g;                      // rows r0 and r0 + 8 of the tile
-        bool ok = true, waited = false;
+        bool ok = true;
 
         // block-constant inputs of rows r0, r0 + 8, block 4 ks + t of the next unit to
         // fetch (zero beyond the weight); fetches run two group-units ahead
@@ -206,71 +200,19 @@ __global__ void __launch_bounds__(kThreads, 1) k_nf4_gemv(const __grid_constant_
 #pragma unroll
         for (int nt = 0; nt < NTT; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
 
-        // finish (or publish) this warp's 16 rows of `tile` after the group's last unit of it
-        auto fixup = [&](int tile) {
-            if (!waited) { grid_dep_wait(); waited = true; }   // T and the zeroed counters
-            const int64_t tu0 = (int64_t)tile * nks, tu1 = tu0 + nks;
-            const int64_t c_first = unit_owner(tu0, U, a.ctas), c_last = unit_owner(tu1 - 1, U, a.ctas);
-            int expected = 0;
-            for (int64_t c2 = c_first; c2 <= c_last; ++c2) expected += __popc(groups_in_tile(c2, U, a.ctas, tu0, tu1));
-            bool finish = expected == 1;
-            if (!finish) {
-                float* sp = a.slots + (((int64_t)blockIdx.x + tile) * 2 + grp) * (NT * TR);
+        // publish this warp's 16 rows x NT tokens of `tile` after the group's last unit of
+        // it: partial slot ((CTA + tile) * 2 + group), summed later by k_nf4_gemv_finish
+        auto publish = [&](int tile) {
+            float* sp = a.slots + (((int64_t)blockIdx.x + tile) * 2 + grp) * (NT * TR);
 #pragma unroll
-                for (int nt = 0; nt < NTT; ++nt) {
-                    const int m = 8 * nt + 2 * t;
-                    sp[m * TR + r0] = acc[nt][0];
-                    sp[(m + 1) * TR + r0] = acc[nt][1];
-                    sp[m * TR + r0 + 8] = acc[nt][2];
-                    sp[(m + 1) * TR + r0 + 8] = acc[nt][3];
-                }
-                __threadfence();
-                __syncwarp();
-                int last = 0;
-                if (lane == 0) {
-                    int* cnt = a.counters + (int64_t)tile * kGroupWarps + w8;
-                    last = atomicAdd(cnt, 1) == expected - 1;
-                    if (last) *cnt = 0;                        // ready for the next call
-                }
-                finish = __shfl_sync(0xffffffffu, last, 0) != 0;
-                if (finish) {
-                    __threadfence();
-#pragma unroll
-                    for (int nt = 0; nt < NTT; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
-                    for (int64_t c2 = c_first; c2 <= c_last; ++c2) {
-                        const int gm = groups_in_tile(c2, U, a.ctas, tu0, tu1);
-                        for (int g2 = 0; g2 < 2; ++g2) {
-                            if (!((gm >> g2) & 1)) continue;
-                            const float* p2 = a.slots + ((c2 + tile) * 2 + g2) * (NT * TR);
-#pragma unroll
-                            for (int nt = 0; nt < NTT; ++nt) {
-                                const int m = 8 * nt + 2 * t;
-                                acc[nt][0] += __ldcg(p2 + m * TR + r0);
-                                acc[nt][1] += __ldcg(p2 + (m + 1) * TR + r0);
-                                acc[nt][2] += __ldcg(p2 + m * TR + r0 + 8);
-                                acc[nt][3] += __ldcg(p2 + (m + 1) * TR + r0 + 8);
-                            }
-                        }
-                    }
-                }
+            for (int nt = 0; nt < NTT; ++nt) {
+                const int m = 8 * nt + 2 * t;
+                sp[m * TR + r0] = acc[nt][0];
+                sp[(m + 1) * TR + r0] = acc[nt][1];
+                sp[m * TR + r0 + 8] = acc[nt][2];
+                sp[(m + 1) * TR + r0 + 8] = acc[nt][3];
+                acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
             }
-            if (finish) {
-#pragma unroll
-                for (int e = 0; e < 4 * NTT; ++e) {
-                    const int nt = e >> 2, q = e & 3;
-                    const int64_t m = 8 * nt + 2 * t + (q & 1);
-                    const int64_t n = (int64_t)tile * TR + r0 + 8 * (q >> 1);
-                    if (m < a.M && n < a.N) {
-                        const float* tr = a.T32 + m * a.rp;
-                        const uint16_t* br = a.lora_B + n * a.r;
-                        float l = 0.f;
-                        for (int i = 0; i < a.r; ++i) l = __fmaf_rn(tr[i], bf16lo_to_f32(br[i]), l);
-                        a.Y[m * a.N + n] = (uint16_t)(pack_bf16x2(__fmaf_rn(a.s, l, acc[nt][q]), 0.f) & 0xffffu);
-                    }
-                }
-            }
-#pragma unroll
-            for (int nt = 0; nt < NTT; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
         };
 
         BC bA, bB;
@@ -318,10 +260,72 @@ __global__ void __launch_bounds__(kThreads, 1) k_nf4_gemv(const __grid_constant_
             // the group's next unit is i + 2: finish this tile's segment when it leaves the tile
             const int cur = tile;
             unit_advance(tile, ks, 2, nks);
-            if (tile != cur || i + 2 >= nu) fixup(cur);
+            if (tile != cur || i + 2 >= nu) publish(cur);
         }
     }
     __syncthreads();
+    // launched programmatically after the T kernel, which it does not read: it only
+    // may not complete before that kernel has (the finish kernel reads both)
+    if (tid == 0) grid_dep_wait();
+}
+
+// Sum of the partial tiles of every (CTA, group) pair that took units of
+// `tile`, in (CTA, group) order, plus s T B^T; CTA = (one 128-row tile, one
+// token), thread = one row n.  Launched programmatically after k_nf4_gemv: it
+// waits for that kernel (and so for the T kernel) first.
+struct FinishArgs {
+    const float* slots;
+    int64_t M, N;
+    int nks, ctas, NT;
+    int64_t units;
+    const float* T32;
+    int rp, r;
+    const uint16_t* lora_B;
+    int b_vec;
+    float s;
+    uint16_t* Y;
+};
+
+__global__ void __launch_bounds__(TR) k_nf4_gemv_finish(FinishArgs a) {
+    __shared__ int s_slot[2 * 148];     // contributing (CTA, group) slots of this tile, in order
+    __shared__ int s_n;
+    grid_dep_wait();
+    const int tile = blockIdx.x, row = threadIdx.x;
+    const int64_t m = blockIdx.y;
+    if (row == 0) {
+        const int64_t tu0 = (int64_t)tile * a.nks, tu1 = tu0 + a.nks;
+        const int64_t c_first = unit_owner(tu0, a.units, a.ctas), c_last = unit_owner(tu1 - 1, a.units, a.ctas);
+        int k = 0;
+        for (int64_t c = c_first; c <= c_last; ++c) {
+            const int gm = groups_in_tile(c, a.units, a.ctas, tu0, tu1);
+            for (int g2 = 0; g2 < 2; ++g2)
+                if ((gm >> g2) & 1) s_slot[k++] = (int)((c + tile) * 2 + g2);
+        }
+        s_n = k;
+    }
+    __syncthreads();
+    const int64_t n = (int64_t)tile * TR + row;
+    if (n >= a.N) return;
+    const int ns = s_n;
+    float v = 0.f;
+    for (int k = 0; k < ns; ++k) v += a.slots[(int64_t)s_slot[k] * (a.NT * TR) + m * TR + row];
+    const uint16_t* br = a.lora_B + n * a.r;
+    const float* tr = a.T32 + m * a.rp;
+    float l = 0.f;
+    if (a.b_vec) {
+        for (int i = 0; i < a.r; i += 8) {
+            const uint4 bv = __ldg(reinterpret_cast<const uint4*>(br + i));
+            const uint32_t bw[4] = {bv.x, bv.y, bv.z, bv.w};
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                l = __fmaf_rn(tr[i + 2 * j], bf16lo_to_f32(bw[j]), l);
+                l = __fmaf_rn(tr[i + 2 * j + 1], bf16hi_to_f32(bw[j]), l);
+            }
+        }
+    } else {
+        for (int i = 0; i < a.r; ++i) l = __fmaf_rn(tr[i], bf16lo_to_f32(br[i]), l);
+    }
+    a.Y[m * a.N + n] = (uint16_t)(pack_bf16x2(__fmaf_rn(a.s, l, v), 0.f) & 0xffffu);
 }
 
 }  // namespace gmv

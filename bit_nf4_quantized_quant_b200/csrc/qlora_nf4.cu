@@ -152,10 +152,9 @@ struct Plan {
     int64_t kT, kU, kA, kB;         // k per split
     int US;                         // small-path U = dY B: N splits
     int64_t rows_u;                 //   rows of B per split
-    int NT;                         // small-path token tile of the tcgen05 kernel (16 or 32)
-    int64_t ncnt;                   // arrival counters in the workspace
+    int NT;                         // small-path token tile (16 or 32; 8 more for the forward GEMV)
     // byte offsets
-    size_t off_slots, off_lslots, off_Upart, off_part, off_cnt, off_T32, off_U32, off_Tp, off_Ubf, off_sT, off_sU, off_Bp, total;
+    size_t off_slots, off_Upart, off_part, off_T32, off_U32, off_Tp, off_Ubf, off_sT, off_sU, off_Bp, total;
 };
 
 size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
@@ -227,35 +226,29 @@ Plan make_plan(int64_t M, int64_t N, int64_t K, int r, int sms) {
         upd(gemm_part_bytes(2 * p.rp, K, p.zA));
         upd(gemm_part_bytes(N, 2 * p.rp, p.zB));
     }
-    // small-path tcgen05 kernel: per-CTA partial tiles of 128 x NT fp32 (slot = CTA + tile)
-    // and one arrival counter per output tile, forward (tiles over N) and backward (over K)
-    size_t slots = 0, ncnt = (size_t)cdiv(N, 8);
+    // small path: partial tiles of the stream-K kernels, 128 x NT fp32 each, one per
+    // (CTA + tile) for the backward and per (CTA + tile, group) for the forward GEMV
+    size_t slots = 0;
     p.NT = M <= 16 ? 16 : 32;
     if (small) {
-        for (int bwd = 0; bwd < 2; ++bwd) {
-            const int64_t tiles = cdiv(bwd ? K : N, tcs::TR), units = tiles * cdiv(bwd ? N : K, tcs::KSTEP);
+        {
+            const int64_t tiles = cdiv(K, tcs::TR), units = tiles * cdiv(N, tcs::KSTEP);
             const int64_t ctas = units < kMaxCtas ? units : kMaxCtas;
-            const size_t b = (size_t)(ctas + tiles) * p.NT * tcs::TR * 4;
-            if (b > slots) slots = b;
-            if ((size_t)(4 * tiles) > ncnt) ncnt = (size_t)(4 * tiles);
+            slots = (size_t)(ctas + tiles) * p.NT * tcs::TR * 4;
         }
-        upd((size_t)M * K * 4);                    // backward dY W' sum
-        // forward GEMV: partial tiles of 128 x NT per (CTA + tile, group), counters [tiles][8]
-        const int64_t tiles = cdiv(N, gmv::TR), units = tiles * cdiv(K, gmv::KSTEP);
-        const int64_t ctas = units < kMaxCtas ? units : kMaxCtas;
-        const size_t b = (size_t)(ctas + tiles) * 2 * p.NT * gmv::TR * 4;
-        if (b > slots) slots = b;
-        if ((size_t)(tiles * gmv::kGroupWarps) > ncnt) ncnt = (size_t)(tiles * gmv::kGroupWarps);
+        {
+            const int64_t tiles = cdiv(N, gmv::TR), units = tiles * cdiv(K, gmv::KSTEP);
+            const int64_t ctas = units < kMaxCtas ? units : kMaxCtas;
+            const size_t b = (size_t)(ctas + tiles) * 2 * p.NT * gmv::TR * 4;
+            if (b > slots) slots = b;
+        }
     }
     const size_t big = small ? 0 : 1;
     size_t off = 0;
     auto take = [&](size_t b) { const size_t o = off; off = align256(off + b); return o; };
     p.off_slots = take(slots);
-    p.off_lslots = take(small ? (size_t)cdiv(N, tcs::TR) * p.NT * tcs::TR * 4 : 0);
     p.off_Upart = take(small ? (size_t)p.US * M * p.rp * 4 : 0);
     p.off_part = take(part);
-    p.off_cnt = take(ncnt * 4);
-    p.ncnt = (int64_t)ncnt;
     p.off_T32 = take((size_t)M * p.rp * 4);
     p.off_U32 = take(big * M * p.rp * 4);
     p.off_Tp = take(big * M * 2 * p.rp * 2);     // T hi | lo
@@ -363,13 +356,9 @@ int ensure_tc_attrs() {
                                  tc2::SMEM_ALLOC) != cudaSuccess ||
             cudaFuncSetAttribute(tc2::k_tc2_gemm<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  tc2::SMEM_ALLOC) != cudaSuccess ||
-            cudaFuncSetAttribute(tcs::k_tcs_gemm<false, 16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+            cudaFuncSetAttribute(tcs::k_tcs_gemm<16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  tcs::SMEM_ALLOC) != cudaSuccess ||
-            cudaFuncSetAttribute(tcs::k_tcs_gemm<false, 32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 tcs::SMEM_ALLOC) != cudaSuccess ||
-            cudaFuncSetAttribute(tcs::k_tcs_gemm<true, 16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 tcs::SMEM_ALLOC) != cudaSuccess ||
-            cudaFuncSetAttribute(tcs::k_tcs_gemm<true, 32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+            cudaFuncSetAttribute(tcs::k_tcs_gemm<32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  tcs::SMEM_ALLOC) != cudaSuccess)
             return QLORA_ERR_LAUNCH;
         // pairs of SMs that can hold one cluster each at the same time
@@ -478,7 +467,6 @@ int compute_T(const Plan& p, const uint16_t* X, const uint16_t* A, float s, uint
     f.J1 = p.r;
     f.hl = reinterpret_cast<uint16_t*>(ws + p.off_Tp); f.hl_ld = 2 * p.rp; f.hl_off = p.rp;
     f.o2 = reinterpret_cast<uint16_t*>(ws + p.off_sT); f.s2i = p.rp64; f.s2j = 1; f.J2 = p.r; f.J2pad = p.rp64; f.alpha2 = s;
-    f.zero = reinterpret_cast<int*>(ws + p.off_cnt); f.zero_n = cdiv(p.N, 8);
     int rc = run_gemm<true, true>(X, p.K, A, p.K, p.M, p.rp, p.K, p.M, p.r, p.zT, p.kT,
                                   reinterpret_cast<float*>(ws + p.off_part), f, sms, st);
     if (rc != QLORA_OK) return rc;
@@ -515,12 +503,11 @@ int launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaS
 }
 
 // Small-M T = X A^T into T32 (and the caller's bf16 T_out); clears `zero`.
-int small_T(const Plan& p, const uint16_t* X, const uint16_t* A, uint16_t* T_out, int* zero, int zero_n,
-            uint8_t* ws, cudaStream_t st) {
+int small_T(const Plan& p, const uint16_t* X, const uint16_t* A, uint16_t* T_out, uint8_t* ws, cudaStream_t st) {
     LoraDownArgs d{};
     d.X = X; d.A = A; d.M = p.M; d.K = p.K; d.r = p.r; d.rp = p.rp;
     d.T32 = reinterpret_cast<float*>(ws + p.off_T32);
-    d.T_out = T_out; d.zero = zero; d.zero_n = zero_n;
+    d.T_out = T_out;
     const int mg = p.M <= 1 ? 1 : p.M <= 2 ? 2 : p.M <= 4 ? 4 : 8;
     const dim3 grid((unsigned)p.r, (unsigned)cdiv(p.M, mg));
     switch (mg) {
@@ -533,39 +520,33 @@ int small_T(const Plan& p, const uint16_t* X, const uint16_t* A, uint16_t* T_out
     return launch_status();
 }
 
-// Small-M fused dequant-GEMM on tcgen05 (stream-K over one CTA per SM),
-// launched programmatically after the adapter kernel before it.
-template <bool BWD>
-int launch_tcs(const Plan& p, const nf4dq_weight* w, const uint16_t* act, const uint16_t* Bl, float s,
-               uint16_t* Y, float* dxsum, uint8_t* wsb, int sms, cudaStream_t st) {
+// Small-M backward dY W' on tcgen05 (stream-K over one CTA per SM), launched
+// programmatically after the U / dB kernel; it leaves partial tiles in the
+// workspace for k_bwd_small_end.
+int launch_tcs_bwd(const Plan& p, const nf4dq_weight* w, const uint16_t* dY, uint8_t* wsb, int sms, cudaStream_t st,
+                   tcs::Args* out) {
     int rc = ensure_tc_attrs();
     if (rc != QLORA_OK) return rc;
     const int64_t M = p.M, N = p.N, K = p.K;
-    const int64_t n_out = BWD ? K : N, n_red = BWD ? N : K;
     CUtensorMap tmX, tmP;
-    if (!make_map_2d(&tmX, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, act, n_red, M, n_red * 2, 64, p.NT,
-                     CU_TENSOR_MAP_SWIZZLE_128B) ||
+    if (!make_map_2d(&tmX, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, dY, N, M, N * 2, 64, p.NT, CU_TENSOR_MAP_SWIZZLE_128B) ||
         !make_map_2d(&tmP, CU_TENSOR_MAP_DATA_TYPE_UINT8, w->packed, K / 2, N, K / 2, 64, tcs::TR,
                      CU_TENSOR_MAP_SWIZZLE_64B))
         return QLORA_ERR_LAUNCH;
     tcs::Args a{};
     a.codes = w->codes; a.scale = w->scale; a.mean = w->mean;
-    a.M = M; a.N = N; a.K = K; a.n_out = n_out; a.n_red = n_red;
-    a.tiles = (int)cdiv(n_out, tcs::TR);
-    a.nks = (int)cdiv(n_red, tcs::KSTEP);
+    a.M = M; a.N = N; a.K = K;
+    a.tiles = (int)cdiv(K, tcs::TR);
+    a.nks = (int)cdiv(N, tcs::KSTEP);
     a.units = (int64_t)a.tiles * a.nks;
     int64_t ctas = sms < kMaxCtas ? sms : kMaxCtas;
     if (ctas > a.units) ctas = a.units;
     a.ctas = (int)ctas;
     a.slots = reinterpret_cast<float*>(wsb + p.off_slots);
-    a.lslots = reinterpret_cast<float*>(wsb + p.off_lslots);
-    a.counters = reinterpret_cast<int*>(wsb + p.off_cnt);
-    a.T32 = reinterpret_cast<const float*>(wsb + p.off_T32); a.rp = p.rp; a.r = p.r;
-    a.lora_B = Bl; a.s = s; a.Y = Y; a.dxsum = dxsum;
-    a.b_vec = (Bl != nullptr && p.r % 8 == 0 && aligned16(Bl)) ? 1 : 0;
+    *out = a;
     const dim3 grid((unsigned)ctas), block(tcs::kThreads);
-    if (p.NT == 16) return launch_pdl(tcs::k_tcs_gemm<BWD, 16>, grid, block, tcs::SMEM_ALLOC, st, tmX, tmP, a, tables());
-    return launch_pdl(tcs::k_tcs_gemm<BWD, 32>, grid, block, tcs::SMEM_ALLOC, st, tmX, tmP, a, tables());
+    if (p.NT == 16) return launch_pdl(tcs::k_tcs_gemm<16>, grid, block, tcs::SMEM_ALLOC, st, tmX, tmP, a, tables());
+    return launch_pdl(tcs::k_tcs_gemm<32>, grid, block, tcs::SMEM_ALLOC, st, tmX, tmP, a, tables());
 }
 
 // Small-M forward GEMV (mma.sync, stream-K over one CTA per SM), launched
@@ -599,11 +580,14 @@ int launch_gemv_ntt(const Plan& p, const nf4dq_weight* w, const uint16_t* X, con
     if (ctas > a.units) ctas = a.units;
     a.ctas = (int)ctas;
     a.slots = reinterpret_cast<float*>(wsb + p.off_slots);
-    a.counters = reinterpret_cast<int*>(wsb + p.off_cnt);
-    a.T32 = reinterpret_cast<const float*>(wsb + p.off_T32); a.rp = p.rp; a.r = p.r;
-    a.lora_B = B; a.s = s; a.Y = Y;
-    return launch_pdl(gmv::k_nf4_gemv<NTT>, dim3((unsigned)ctas), dim3(gmv::kThreads), (size_t)C::SMEM_ALLOC, st, tmP,
-                      a, tables());
+    int rc = launch_pdl(gmv::k_nf4_gemv<NTT>, dim3((unsigned)ctas), dim3(gmv::kThreads), (size_t)C::SMEM_ALLOC, st,
+                        tmP, a, tables());
+    if (rc != QLORA_OK) return rc;
+    gmv::FinishArgs f{};
+    f.slots = a.slots; f.M = p.M; f.N = N; f.nks = a.nks; f.ctas = a.ctas; f.NT = C::NT; f.units = a.units;
+    f.T32 = reinterpret_cast<const float*>(wsb + p.off_T32); f.rp = p.rp; f.r = p.r;
+    f.lora_B = B; f.b_vec = (p.r % 8 == 0 && aligned16(B)) ? 1 : 0; f.s = s; f.Y = Y;
+    return launch_pdl(gmv::k_nf4_gemv_finish, dim3((unsigned)a.tiles, (unsigned)p.M), dim3(gmv::TR), 0, st, f);
 }
 
 int launch_gemv(const Plan& p, const nf4dq_weight* w, const uint16_t* X, const uint16_t* B, float s, uint16_t* Y,
@@ -618,7 +602,7 @@ int launch_gemv(const Plan& p, const nf4dq_weight* w, const uint16_t* X, const u
 int small_fwd(const Plan& p, const uint16_t* X, const nf4dq_weight* w, const uint16_t* A, const uint16_t* B,
               float scaling, uint16_t* Y, uint16_t* T_out, uint8_t* wsb, int sms, cudaStream_t st) {
     hook_before(st);
-    int rc = small_T(p, X, A, T_out, reinterpret_cast<int*>(wsb + p.off_cnt), (int)p.ncnt, wsb, st);
+    int rc = small_T(p, X, A, T_out, wsb, st);
     if (rc != QLORA_OK) return rc;
     rc = launch_gemv(p, w, X, B, scaling, Y, wsb, sms, st);
     hook_after(st);
@@ -633,7 +617,7 @@ int small_bwd(const Plan& p, const uint16_t* X, const uint16_t* dY, const nf4dq_
     int rc = QLORA_OK;
     const float* T32 = nullptr;
     if (T == nullptr) {
-        rc = small_T(p, X, A, nullptr, nullptr, 0, wsb, st);
+        rc = small_T(p, X, A, nullptr, wsb, st);
         if (rc != QLORA_OK) return rc;
         T32 = reinterpret_cast<const float*>(wsb + p.off_T32);
     }
@@ -642,21 +626,20 @@ int small_bwd(const Plan& p, const uint16_t* X, const uint16_t* dY, const nf4dq_
     b.dY = dY; b.B = B; b.T32 = T32; b.Tb = T; b.M = p.M; b.N = p.N; b.r = p.r; b.rp = p.rp; b.s = scaling;
     b.b_vec = (p.r % 8 == 0 && aligned16(B)) ? 1 : 0;
     b.Upart = reinterpret_cast<float*>(wsb + p.off_Upart); b.US = p.US; b.rows_u = p.rows_u; b.dB = dB;
-    b.zero = reinterpret_cast<int*>(wsb + p.off_cnt); b.zero_n = (int)p.ncnt;
     k_lora_bwd_small<<<(unsigned)(p.US + cdiv(p.N, kLoraThreads)), kLoraThreads, 0, st>>>(b);
     note_launch();
     rc = launch_status();
     if (rc != QLORA_OK) return rc;
-    float* dxsum = reinterpret_cast<float*>(wsb + p.off_part);
-    rc = launch_tcs<true>(p, w, dY, nullptr, scaling, nullptr, dxsum, wsb, sms, st);
+    tcs::Args ta{};
+    rc = launch_tcs_bwd(p, w, dY, wsb, sms, st, &ta);
     hook_after(st);
     if (rc != QLORA_OK) return rc;
     BwdEndArgs e{};
-    e.part = dxsum; e.S = 1; e.Upart = b.Upart; e.US = p.US; e.A = A; e.X = X;
+    e.slots = ta.slots; e.NT = p.NT; e.nks = ta.nks; e.ctas = ta.ctas; e.units = ta.units;
+    e.Upart = b.Upart; e.US = p.US; e.A = A; e.X = X;
     e.M = p.M; e.K = p.K; e.r = p.r; e.rp = p.rp; e.s = scaling; e.dX = dX; e.dA = dA;
-    k_bwd_small_end<<<dim3((unsigned)cdiv(p.K, kLoraThreads), (unsigned)(p.M + p.r)), kLoraThreads, 0, st>>>(e);
-    note_launch();
-    return launch_status();
+    return launch_pdl(k_bwd_small_end, dim3((unsigned)cdiv(p.K, kLoraThreads), (unsigned)(p.M + p.r)),
+                      dim3(kLoraThreads), 0, st, e);
 }
 
 }  // namespace

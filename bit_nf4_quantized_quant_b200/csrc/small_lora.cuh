@@ -6,7 +6,7 @@
 //                      and token group; no cross-CTA reduction)
 //   k_lora_bwd_small   U = dY B as per-split partials, and dB = s dY^T T, in
 //                      one launch (the first CTAs take U, the rest dB)
-//   k_bwd_small_end    dX = (sum of the dY W' split partials) + s U A and
+//   k_bwd_small_end    dX = (sum of k_tcs_gemm's partial tiles) + s U A and
 //                      dA = s U^T X, each CTA first summing the U partials it
 //                      needs in a fixed order
 //
@@ -33,8 +33,6 @@ struct LoraDownArgs {
     int r, rp;
     float* T32;              // [M, rp] fp32 (columns >= r not written)
     uint16_t* T_out;         // [M, r] bf16 copy for the caller, or null
-    int* zero;               // ints to clear (the forward's arrival counters), or null
-    int zero_n;
 };
 
 __device__ __forceinline__ float dot8_bf16(const uint4& x, const uint4& y, float v) {
@@ -57,8 +55,6 @@ __global__ void __launch_bounds__(kLoraThreads) k_lora_down_small(LoraDownArgs a
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int i = blockIdx.x;
     const int64_t m0 = (int64_t)blockIdx.y * MG;
-    if (a.zero != nullptr && blockIdx.x == 0 && blockIdx.y == 0)
-        for (int e = tid; e < a.zero_n; e += kLoraThreads) a.zero[e] = 0;
     const uint4* ar = reinterpret_cast<const uint4*>(a.A + (int64_t)i * a.K);
     const uint4* xr[MG];
 #pragma unroll
@@ -109,8 +105,6 @@ struct LoraBwdArgs {
     int US;                  // N splits of U; CTAs [0, US) compute U
     int64_t rows_u;          // rows of B per split
     uint16_t* dB;            // [N, r] bf16
-    int* zero;               // ints to clear (the next kernel's arrival counters), or null
-    int zero_n;
 };
 
 constexpr int kUTok = 4;     // tokens per pass of a U split
@@ -144,8 +138,6 @@ __global__ void __launch_bounds__(kLoraThreads) k_lora_bwd_small(LoraBwdArgs a) 
     grid_dep_launch();
     __shared__ __align__(16) float smem[kSmemLoraBwd];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    if (a.zero != nullptr && blockIdx.x == 0)
-        for (int e = tid; e < a.zero_n; e += kLoraThreads) a.zero[e] = 0;
 
     if ((int)blockIdx.x < a.US) {
         // ---- U split b: rows n in [n0, n1); lane group c owns rank columns 8c .. 8c + 7
@@ -250,8 +242,9 @@ __global__ void __launch_bounds__(kLoraThreads) k_lora_bwd_small(LoraBwdArgs a) 
 // dX = sum_s part_s + s U A,   dA = s U^T X
 // ---------------------------------------------------------------------------
 struct BwdEndArgs {
-    const float* part;       // [S][M][K] fp32 partial dY W'
-    int S;
+    const float* slots;      // [ctas + tiles][NT][128] partial dY W' tiles of k_tcs_gemm
+    int NT, nks, ctas;       // that kernel's token width, steps per tile and grid
+    int64_t units;
     const float* Upart;      // [US][M][rp] fp32 partial U
     int US;
     const uint16_t* A;       // [r, K]
@@ -263,10 +256,19 @@ struct BwdEndArgs {
     uint16_t* dA;            // [r, K]
 };
 
+// First unit of CTA c, and the CTA that owns unit u, for k_tcs_gemm's even
+// split of U units over C CTAs.
+__device__ __forceinline__ int64_t end_unit_owner(int64_t u, int64_t U, int64_t C) {
+    return ((u + 1) * C + U - 1) / U - 1;
+}
+
 // grid (ceil(K / 256), M + r): row y < M writes dX[y, :], row M + i writes dA[i, :].
+// Launched programmatically after k_tcs_gemm: it waits for that kernel (and so
+// for the U / dB kernel before it) first.
 __global__ void __launch_bounds__(kLoraThreads) k_bwd_small_end(BwdEndArgs a) {
     __shared__ float s_q[kLoraThreads];
     __shared__ float s_u[kLoraThreads];
+    grid_dep_wait();
     const int tid = threadIdx.x;
     const int y = blockIdx.y;
     const bool is_dx = y < a.M;
@@ -295,8 +297,13 @@ __global__ void __launch_bounds__(kLoraThreads) k_bwd_small_end(BwdEndArgs a) {
     const int64_t k = (int64_t)blockIdx.x * kLoraThreads + tid;
     if (k >= a.K) return;
     if (is_dx) {
+        // dY W': the partial tiles of every CTA that took steps of column tile k / 128, in CTA order
+        const int64_t tile = k >> 7, row = k & 127;
+        const int64_t tu0 = tile * a.nks;
+        const int64_t c_first = end_unit_owner(tu0, a.units, a.ctas);
+        const int64_t c_last = end_unit_owner(tu0 + a.nks - 1, a.units, a.ctas);
         float v = 0.f;
-        for (int s2 = 0; s2 < a.S; ++s2) v += a.part[((int64_t)s2 * a.M + y) * a.K + k];
+        for (int64_t c = c_first; c <= c_last; ++c) v += a.slots[(c + tile) * (a.NT * 128) + (int64_t)y * 128 + row];
         float l = 0.f;
         for (int i = 0; i < a.r; ++i) l = __fmaf_rn(s_u[i], bf16lo_to_f32(a.A[(int64_t)i * a.K + k]), l);
         v = __fmaf_rn(a.s, l, v);

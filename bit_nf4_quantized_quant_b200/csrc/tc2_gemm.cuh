@@ -17,8 +17,8 @@
 //     transaction bytes complete on the leader's barrier (the leader arms it
 //     for both halves);
 //   - the dequantizers and the epilogue of both CTAs arrive on the leader's
-//     barriers (mapa + release at cluster scope); the leader's waits acquire
-//     at cluster scope;
+//     barriers: the peer's with release at cluster scope (mapa), the leader's
+//     own at CTA scope; the leader's waits acquire at cluster scope;
 //   - MMA completion is multicast to the "empty" and "accumulator full"
 //     barriers of both CTAs (tcgen05.commit ... multicast::cluster, mask 0b11).
 // No TMA load uses multicast.  All waits are bounded as in tc_gemm.cuh; a
@@ -373,7 +373,12 @@ k_tc2_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
                     tc::st_shared_v4(wbase + w_chunk_offset<BWD>(t, ch), o[ch][0], o[ch][1], o[ch][2], o[ch][3]);
                 tc::fence_proxy_async();                  // this thread's tile writes -> async proxy
                 __syncwarp();
-                if (lane == 0) mbar_arrive_cl(mapa(fullW(sw), 0));
+                // the leader's own warps release at CTA scope (same CTA as the MMA issuer);
+                // the peer's warps release at cluster scope on the leader's barrier
+                if (lane == 0) {
+                    if (leader) tc::mbar_arrive(fullW(sw));
+                    else mbar_arrive_cl(mapa(fullW(sw), 0));
+                }
             }
         }
     } else {
@@ -411,7 +416,10 @@ k_tc2_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
             }
             tc::tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive_cl(mapa(tempty(acc), 0));
+            if (lane == 0) {
+                if (leader) tc::mbar_arrive(tempty(acc));
+                else mbar_arrive_cl(mapa(tempty(acc), 0));
+            }
         }
     }
 

@@ -1,37 +1,32 @@
-// tcs_gemm.cuh -- fused NF4 dequant + GEMM on tcgen05 for a few tokens
-// (M <= 32): the decode / small-batch shape, where the layer is bound by the
-// exact dequantization of the 4.13-bit weight stream (integer-pipe work per
-// weight), not by tensor work.
+// tcs_gemm.cuh -- backward dX = dY W' for a few tokens (M <= 32) on tcgen05:
+// the fused exact NF4 dequant feeds the MMA's A operand, the tokens are its
+// N dimension.
 //
-//   forward : Y^T  [N, M] = W'   [N, K] . X^T  [K, M]    + s B T^T
-//   backward: dX^T [K, M] = W'^T [K, N] . dY^T [N, M]    (s A^T U^T added later)
+//   dX^T [K, M] = W'^T [K, N] . dY^T [N, M]      (s A^T U^T is added by k_bwd_small_end)
 //
-// The weight is the MMA's A operand (M_mma = 128 rows of W, or 128 columns
-// of W in the backward) and the tokens are its N dimension (NT = 16 or 32,
-// zero rows beyond M come from the TMA's out-of-bound fill), so one
-// tcgen05.mma of 128 x NT x 16 does all the tensor work of 2048 weights.
-// Work unit = (output tile of 128, reduction step of 128).  The units of a
-// problem are split evenly over one CTA per SM in (tile, step) order
-// ("stream-K"), so every SM decodes the same number of weights; a tile whose
-// steps span several CTAs is finished, per TMEM lane quarter, by the warp
-// that arrives last on that quarter's counter, which sums the per-CTA
-// partials in CTA order (the result does not depend on arrival order).
+// The weight is the MMA's A operand (M_mma = 128 columns of W; W's rows are
+// the reduction, so the dequantized tile is stored MN-major) and the tokens
+// are its N dimension (NT = 16 or 32, zero rows beyond M from the TMA's
+// out-of-bound fill).  Work unit = (128 output columns, 128 reduction rows).
+// The units are split evenly over one CTA per SM in (tile, step) order
+// ("stream-K"); every CTA writes its partial sum of each tile it touched to
+// its own slot (slot = CTA + tile, unique along the split), and
+// k_bwd_small_end sums the slots of a tile in CTA order (deterministic) when
+// it forms dX.
 //
 // Warp roles (768 threads, one CTA per SM):
-//   warp 0      TMA producer of the activation tiles (NT x 128 bf16, two
+//   warp 0      TMA producer of the dY tiles (NT x 128 bf16, two
 //               128-byte-swizzled boxes of 64 columns);
 //   warp 1      TMEM allocator and MMA issuer: 8 MMAs of 128 x NT x 16 per unit;
 //   warp 2      TMA producer of the packed NF4 tiles (128 rows x 64 B, 64-byte
 //               swizzle), 8 units ahead;
-//   warps 4-7   epilogue: the LoRA term of a tile while its MMAs run, then
-//               TMEM -> registers -> partial or finished output;
+//   warps 4-7   epilogue: TMEM -> registers -> partial slot;
 //   warps 8-23  dequantizers, two groups of 8 warps taking alternate units (16
 //               warps keep the integer pipe busy while others wait): thread d
 //               of a group owns one 64-weight row-block per unit (row
 //               8 (d / 16) + d % 8, block (d / 8) % 2), exact bf16_rne(L[q] c')
 //               from the per-block register table, written into the swizzled
-//               A-operand layout (K-major in the forward, MN-major in the
-//               backward, where W's rows are the reduction).
+//               MN-major A-operand layout.
 #pragma once
 #include "tc_gemm.cuh"
 
@@ -64,23 +59,11 @@ struct Args {
     const int8_t* codes;
     const float* scale;
     const float* mean;
-    int64_t M, N, K;           // W is [N, K]
-    int64_t n_out, n_red;      // forward: N, K;  backward: K, N
-    int tiles, nks;            // ceil(n_out / 128), ceil(n_red / 128)
+    int64_t M, N, K;           // W is [N, K]; the output has K columns, the reduction N rows
+    int tiles, nks;            // ceil(K / 128), ceil(N / 128)
     int64_t units;             // tiles * nks
     int ctas;                  // grid size
-    float* slots;              // [ctas + tiles][NT][128] fp32 partials
-    float* lslots;             // forward: [tiles][NT][128] fp32 LoRA terms
-    int* counters;             // [tiles][4] (per TMEM lane quarter), zero on entry, left zero
-    // forward finish: Y = acc + s T B^T
-    const float* T32;          // [M, rp]
-    int rp, r;
-    const uint16_t* lora_B;    // [N, r]
-    int b_vec;                 // rows of lora_B are 16-byte loadable
-    float s;
-    uint16_t* Y;               // [M, N]
-    // backward finish: the dY W' sum in fp32
-    float* dxsum;              // [M, K]
+    float* slots;              // [ctas + tiles][NT][128] fp32 partial tiles
 };
 
 // First unit of CTA c, and the CTA that owns unit u, for an even split of U units over C CTAs.
@@ -109,14 +92,11 @@ __device__ __forceinline__ int deq_row(int d) { return 8 * (d >> 4) + (d & 7); }
 __device__ __forceinline__ int deq_blk(int d) { return (d >> 3) & 1; }
 
 // Byte offset of 16-byte chunk ch (8 weights) of thread d's row-block in the
-// operand tile.  Forward (K-major, two 64-column halves of 16 KB): half j, row
-// n, chunk ch ^ (n % 8).  Backward (MN-major: the tile's 128 rows are the
-// reduction, its 2 x 64 columns the MMA's M): atom column j 16 KB apart, 8-row
-// group n / 8 1 KB apart, row n % 8, chunk ch ^ (n % 8).
-template <bool BWD>
+// MN-major operand tile (the tile's 128 rows are the reduction, its 2 x 64
+// columns the MMA's M): atom column j 16 KB apart, 8-row group n / 8 1 KB
+// apart, row n % 8, chunk ch ^ (n % 8).
 __device__ __forceinline__ uint32_t w_chunk_offset(int d, int ch) {
     const int n = deq_row(d), j = deq_blk(d);
-    if (!BWD) return (uint32_t)(j * 16384 + n * 128 + ((ch ^ (n & 7)) << 4));
     return (uint32_t)(j * 16384 + (n >> 3) * 1024 + (n & 7) * 128 + ((ch ^ (n & 7)) << 4));
 }
 
@@ -133,7 +113,7 @@ __device__ __forceinline__ void unit_advance(int& tile, int& ks, int n, int nks)
 }
 
 // ----------------------------------------------------------------------------
-template <bool BWD, int NT>
+template <int NT>
 __global__ void __launch_bounds__(kThreads, 1)
 k_tcs_gemm(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmP, Args a,
            NF4Tables tab) {
@@ -212,8 +192,7 @@ k_tcs_gemm(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUte
                 if (!(ok = tc::mbar_wait(emptyP(sp), pp ^ 1, s_abort))) break;
                 tc::mbar_expect_tx(fullP(sp), P_BYTES);
                 const uint32_t dst = sbase + OFF_P + sp * P_BYTES;
-                if (!BWD) tc::tma_load_2d(dst, &tmP, fullP(sp), ks * (KSTEP / 2), tile * TR);
-                else tc::tma_load_2d(dst, &tmP, fullP(sp), tile * (TR / 2), ks * KSTEP);
+                tc::tma_load_2d(dst, &tmP, fullP(sp), tile * (TR / 2), ks * KSTEP);
                 ++issued;
                 unit_advance(tile, ks, 1, nks);
             }
@@ -224,7 +203,7 @@ k_tcs_gemm(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUte
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
-            constexpr uint32_t idesc = make_idesc(BWD, NT);
+            constexpr uint32_t idesc = make_idesc(true, NT);
             int sx = 0, px = 0, seg = 0, buf = 0;
             bool ok = true;
             uint32_t d_tmem = tmem_base;
@@ -246,8 +225,7 @@ k_tcs_gemm(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUte
 #pragma unroll
                 for (int q = 0; q < KSTEP / 16; ++q) {
                     const int h = q >> 2, kk = q & 3;
-                    const uint64_t adesc = BWD ? tc::smem_desc_sw128(w_addr + q * 2048, 16384, 1024)
-                                               : tc::smem_desc_sw128(w_addr + h * 16384 + kk * 32, 16, 1024);
+                    const uint64_t adesc = tc::smem_desc_sw128(w_addr + q * 2048, 16384, 1024);
                     const uint64_t bdesc = tc::smem_desc_sw128(x_addr + h * (NT * 128) + kk * 32, 16, 1024);
                     tc::tc_mma(d_tmem, adesc, bdesc, idesc, (!first || q > 0) ? 1u : 0u);
                 }
@@ -278,9 +256,7 @@ k_tcs_gemm(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUte
             fi += 2;
             unit_advance(ft, fk, 2, nks);
             if (!in) return;
-            int64_t n, kb;
-            if (!BWD) { n = (int64_t)tile * TR + drow; kb = (int64_t)ks * 2 + dblk; }
-            else { n = (int64_t)ks * KSTEP + drow; kb = (int64_t)tile * 2 + dblk; }
+            const int64_t n = (int64_t)ks * KSTEP + drow, kb = (int64_t)tile * 2 + dblk;
             if (n < a.N && kb < nblk) {
                 const int64_t b = n * nblk + kb;
                 code = __ldg(a.codes + b);
@@ -311,7 +287,7 @@ k_tcs_gemm(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUte
             for (int ch = 0; ch < 8; ++ch) {
                 uint32_t o[4];
                 decode8(tb, pwd[ch], o);
-                tc::st_shared_v4(wbase + w_chunk_offset<BWD>(d, ch), o[0], o[1], o[2], o[3]);
+                tc::st_shared_v4(wbase + w_chunk_offset(d, ch), o[0], o[1], o[2], o[3]);
             }
             tc::fence_proxy_async();
             __syncwarp();
@@ -329,42 +305,11 @@ k_tcs_gemm(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUte
         // ------------------------------------------------------------ epilogue
         const int q = warp & 3;                 // TMEM lane quarter of this warp
         const int row = q * 32 + lane;
-        // T and the zeroed counters come from the kernel before this one, which may
-        // still be running (programmatic launch)
-        grid_dep_wait();
         bool ok = true;
         int seg = 0;
         for (int u = u0, tile = tile0; u < u1 && ok; ++tile) {
-            const int tile_u0 = tile * nks, tile_u1 = tile_u0 + nks;
-            const int seg_end = tile_u1 < u1 ? tile_u1 : u1;
-            const bool starts = (u == tile_u0);
-            const bool whole = starts && (seg_end == tile_u1);
-            u = seg_end;
-            const int64_t o = (int64_t)tile * TR + row;     // output feature (forward) or column k (backward)
-            float* lp = BWD ? nullptr : a.lslots + (int64_t)tile * (NT * TR);
-            if (!BWD && starts && o < a.N) {
-                // the LoRA term s T B^T of this tile's rows, computed by the CTA that
-                // owns the tile's first step while the MMAs of the segment run
-                const uint16_t* br = a.lora_B + o * a.r;
-                for (int64_t m = 0; m < a.M; ++m) {
-                    const float* tr = a.T32 + m * a.rp;
-                    float l = 0.f;
-                    if (a.b_vec) {
-                        for (int i = 0; i < a.r; i += 8) {
-                            const uint4 bv = __ldg(reinterpret_cast<const uint4*>(br + i));
-                            const uint32_t bw[4] = {bv.x, bv.y, bv.z, bv.w};
-#pragma unroll
-                            for (int j = 0; j < 4; ++j) {
-                                l = __fmaf_rn(tr[i + 2 * j], bf16lo_to_f32(bw[j]), l);
-                                l = __fmaf_rn(tr[i + 2 * j + 1], bf16hi_to_f32(bw[j]), l);
-                            }
-                        }
-                    } else {
-                        for (int i = 0; i < a.r; ++i) l = __fmaf_rn(tr[i], bf16lo_to_f32(br[i]), l);
-                    }
-                    lp[m * TR + row] = a.s * l;
-                }
-            }
+            const int tile_u1 = (tile + 1) * nks;
+            u = tile_u1 < u1 ? tile_u1 : u1;
             const int buf = seg & 1;
             if (!(ok = tc::mbar_wait(tfull(buf), (seg >> 1) & 1, s_abort))) break;
             ++seg;
@@ -384,54 +329,9 @@ k_tcs_gemm(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUte
             tc::tc_fence_before();
             __syncwarp();
             if (lane == 0) tc::mbar_arrive(tempty(buf));
-            // a split tile: every epilogue warp publishes its 32 rows and arrives on the
-            // counter of (tile, its lane quarter); the last of them sums that quarter
-            bool finish = whole;
-            if (!whole) {
-                const int64_t slot = (int64_t)blockIdx.x + tile;
-                float* sp = a.slots + slot * (NT * TR);
+            float* sp = a.slots + ((int64_t)blockIdx.x + tile) * (NT * TR);
 #pragma unroll
-                for (int m = 0; m < NT; ++m) sp[m * TR + row] = acc[m];
-                __threadfence();
-                __syncwarp();
-                const int64_t c_first = unit_owner(tile_u0, U, a.ctas);
-                const int64_t c_last = unit_owner(tile_u1 - 1, U, a.ctas);
-                int is_last = 0;
-                if (lane == 0) {
-                    int* cnt = a.counters + 4 * (int64_t)tile + q;
-                    is_last = atomicAdd(cnt, 1) == (int)(c_last - c_first);
-                    if (is_last) *cnt = 0;                      // ready for the next call
-                }
-                finish = __shfl_sync(0xffffffffu, is_last, 0) != 0;
-                if (finish) {
-                    __threadfence();
-#pragma unroll
-                    for (int m = 0; m < NT; ++m) acc[m] = 0.f;
-                    for (int64_t c2 = c_first; c2 <= c_last; ++c2) {
-                        const float* p2 = a.slots + (c2 + tile) * (NT * TR);
-#pragma unroll
-                        for (int m = 0; m < NT; ++m) acc[m] += __ldcg(p2 + m * TR + row);
-                    }
-                }
-            }
-            if (!finish) continue;
-            if (!BWD) {
-                if (o < a.N) {
-#pragma unroll
-                    for (int m = 0; m < NT; ++m) {
-                        if (m < a.M) {
-                            const float v = acc[m] + __ldcg(lp + m * TR + row);
-                            a.Y[(int64_t)m * a.N + o] = (uint16_t)(pack_bf16x2(v, 0.f) & 0xffffu);
-                        }
-                    }
-                }
-            } else {
-                if (o < a.K) {
-#pragma unroll
-                    for (int m = 0; m < NT; ++m)
-                        if (m < a.M) a.dxsum[(int64_t)m * a.K + o] = acc[m];
-                }
-            }
+            for (int m = 0; m < NT; ++m) sp[m * TR + row] = acc[m];
         }
     }
 
@@ -440,6 +340,9 @@ k_tcs_gemm(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUte
         tc::tc_fence_after();
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(kCols));
     }
+    // launched programmatically after the U / dB kernel, which it does not read: it
+    // only may not complete before that kernel has (k_bwd_small_end reads both)
+    if (tid == 0) grid_dep_wait();
 }
 
 }  // namespace tcs
