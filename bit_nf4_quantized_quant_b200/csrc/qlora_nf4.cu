@@ -302,6 +302,9 @@ int validate_weight(const nf4dq_weight* w) {
     if (w->N <= 0 || w->K <= 0 || (w->K % kBlock) != 0 || (w->N % 8) != 0) return QLORA_ERR_SHAPE;
     if (w->N > (int64_t)1 << 31 || w->K > (int64_t)1 << 31 || w->N * w->K >= ((int64_t)1 << 38)) return QLORA_ERR_SHAPE;
     if (!aligned16(w->packed)) return QLORA_ERR_ALIGN;
+    const uintptr_t lo = reinterpret_cast<uintptr_t>(w->codes) | reinterpret_cast<uintptr_t>(w->scale) |
+                         reinterpret_cast<uintptr_t>(w->mean);
+    if ((lo & 3u) != 0) return QLORA_ERR_ALIGN;
     return QLORA_OK;
 }
 

@@ -41,7 +41,7 @@ constexpr int SA = 5, SW = 5, SP = 8;
 constexpr int A_BYTES = HM * BK * 2;             // 16 KB
 constexpr int W_BYTES = HN * BK * 2;             // 16 KB
 constexpr int P_BYTES = HN * BK / 2;             // 4 KB
-constexpr int kThreads = 480;
+constexpr int kThreads = 512;
 constexpr int kGroupThreads = 128;               // dequantizers per step (one group of two)
 constexpr int kGroupWarps = kGroupThreads / 32;
 constexpr int kEpiWarps = 4;
@@ -51,9 +51,11 @@ constexpr int OFF_A = 0;
 constexpr int OFF_W = OFF_A + SA * A_BYTES;
 constexpr int OFF_P = OFF_W + SW * W_BYTES;
 constexpr int OFF_BAR = OFF_P + SP * P_BYTES;
-constexpr int NBAR = 2 * SA + 2 * SW + 2 * SP + 4 + 1;
+constexpr int NBAR = 2 * SA + 2 * SW + 2 * SP + 4 + 1 + SW;   // + peer-local fullWl[SW]
 constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
-constexpr int SMEM_BYTES = OFF_MISC + 16;
+// per dequantizer thread, 2 slots x (code word, scale, mean) of prefetched block-constant inputs
+constexpr int OFF_C = OFF_MISC + 16;
+constexpr int SMEM_BYTES = OFF_C + 2 * 3 * 2 * kGroupThreads * 4;
 constexpr int SMEM_ALLOC = SMEM_BYTES + 1024;
 
 __device__ __forceinline__ uint32_t cluster_rank() {
@@ -187,6 +189,7 @@ k_tc2_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
     auto tfull = [&](int i) { return bar0 + 8 * (2 * SA + 2 * SW + 2 * SP + i); };
     auto tempty = [&](int i) { return bar0 + 8 * (2 * SA + 2 * SW + 2 * SP + 2 + i); };
     const uint32_t drain = bar0 + 8 * (2 * SA + 2 * SW + 2 * SP + 4);
+    auto fullWl = [&](int i) { return bar0 + 8 * (2 * SA + 2 * SW + 2 * SP + 5 + i); };
     uint32_t* s_tmem = reinterpret_cast<uint32_t*>(base + OFF_MISC);
     volatile int* s_abort = reinterpret_cast<volatile int*>(base + OFF_MISC + 4);
 
@@ -202,7 +205,12 @@ k_tc2_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
 
     if (tid == 0) {
         for (int i = 0; i < SA; ++i) { tc::mbar_init(fullA(i), 1); tc::mbar_init(emptyA(i), 1); }
-        for (int i = 0; i < SW; ++i) { tc::mbar_init(fullW(i), 2 * kGroupWarps); tc::mbar_init(emptyW(i), 1); }
+        // leader: its own group's warps + one forwarded arrival from the peer; peer: its group's warps
+        for (int i = 0; i < SW; ++i) {
+            tc::mbar_init(fullW(i), kGroupWarps + 1);
+            tc::mbar_init(emptyW(i), 1);
+            tc::mbar_init(fullWl(i), kGroupWarps);
+        }
         for (int i = 0; i < SP; ++i) { tc::mbar_init(fullP(i), 1); tc::mbar_init(emptyP(i), kGroupWarps); }
         for (int i = 0; i < 2; ++i) { tc::mbar_init(tfull(i), 1); tc::mbar_init(tempty(i), 2 * kEpiWarps); }
         tc::mbar_init(drain, 1);
@@ -220,6 +228,24 @@ k_tc2_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
     __syncthreads();
     tc::tc_fence_after();
     const uint32_t tmem_base = *s_tmem;
+
+    // Peer CTA: pass the completion of each stage of the dequantized-weight ring on to
+    // the leader's barrier, for the steps of dequantizer group grp: one cluster-scope
+    // fence and one relaxed remote arrive per stage.
+    auto forward = [&](int grp) {
+        bool ok = true;
+        int it = 0;
+        for (int64_t tile = pair; tile < ntiles && ok; tile += npairs, ++it) {
+            for (int step = grp; step < nsteps && ok; step += 2) {
+                const int gs = it * nsteps + step;
+                const int sw = gs % SW, pw = (gs / SW) & 1;
+                if (!(ok = tc::mbar_wait(fullWl(sw), pw, s_abort))) break;
+                asm volatile("fence.acq_rel.cluster;" ::: "memory");
+                asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(mapa(fullW(sw), 0))
+                             : "memory");
+            }
+        }
+    };
 
     if (warp == 0) {
         // ------------------------------------------------------------ activations (both CTAs)
@@ -294,39 +320,62 @@ k_tc2_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
             }
             tc2_commit_local(drain);
             mbar_drain_cl(drain, 0);
+        } else if (!leader && lane == 0) {
+            forward(0);
         }
+    } else if (warp == 15) {
+        if (!leader && lane == 0) forward(1);
     } else if (warp < 10) {
         // ------------------------------------------------------------ dequantizers: two groups, alternate steps
         const int grp = (warp - 2) >> 2;               // 0: even steps, 1: odd steps
         const int t = ((warp - 2) & 3) * 32 + lane;    // 0..127
         const int drow = deq_row<BWD>(t), dblk = deq_blk<BWD>(t);
         bool ok = true;
-        auto fetch = [&](int64_t c0, int st, int& code, float& sc, float& mu) {
+        // Block-constant inputs (the code's aligned 32-bit word, scale, mean) of a step are
+        // copied with cp.async into this thread's slot two group-steps ahead.  Async
+        // copies are not waited for by the release arrives of the stage barriers, so
+        // their memory latency stays off the step; the thread waits for its own copies
+        // (cp.async.wait_group) just before it needs them.
+        const int dthr = (warp - 2) * 32 + lane;                     // 0..255
+        const uint32_t cbase = sbase + OFF_C + (uint32_t)dthr * 4;
+        auto cslot = [&](int slot, int wd) { return cbase + (uint32_t)((slot * 3 + wd) * 2 * kGroupThreads * 4); };
+        int shift0 = 0, shift1 = 0;                                  // byte of the code in its word
+        auto fetch = [&](int64_t c0, int st, int slot) {
             int64_t n, kb;
             if (!BWD) { n = c0 + drow; kb = st; }
             else { n = (int64_t)st * BK + drow; kb = c0 / kBlock + dblk; }
-            code = 0; sc = 0.f; mu = 0.f;
-            if (st < nks && n < a.N && kb < nblk) {
-                const int64_t b = n * nblk + kb;
-                const int64_t g = b >> 8;
-                code = __ldg(a.codes + b);
-                sc = __ldg(a.scale + g);
-                mu = __ldg(a.mean + g);
-            }
+            const bool v = st < nks && n < a.N && kb < nblk;
+            const int64_t b = v ? n * nblk + kb : 0;
+            const int sz = v ? 4 : 0;                                   // 0: zero-fill (constant 0)
+            if (slot) shift1 = (int)(b & 3) * 8;
+            else shift0 = (int)(b & 3) * 8;
+            asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(cslot(slot, 0)),
+                         "l"(a.codes + (b & ~(int64_t)3)), "r"(sz) : "memory");
+            asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(cslot(slot, 1)), "l"(a.scale + (b >> 8)),
+                         "r"(sz) : "memory");
+            asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(cslot(slot, 2)), "l"(a.mean + (b >> 8)),
+                         "r"(sz) : "memory");
+            asm volatile("cp.async.commit_group;" ::: "memory");
+        };
+        auto block_const = [&](int slot) {
+            asm volatile("cp.async.wait_group 1;" ::: "memory");       // this slot's copies have landed
+            const uint32_t wd = lds_u32(cslot(slot, 0));
+            const float sc = __uint_as_float(lds_u32(cslot(slot, 1))), mu = __uint_as_float(lds_u32(cslot(slot, 2)));
+            const int code = (int)(int8_t)(uint8_t)(wd >> (slot ? shift1 : shift0));
+            return __fmaf_rn((float)code, sc, mu);
         };
         int it = 0;
         for (int64_t tile = pair; tile < ntiles && ok; tile += npairs, ++it) {
             const int64_t c0 = (tile / mtiles) * BN + crank * HN;   // this CTA's first output column
-            int code;
-            float sc, mu;
-            fetch(c0, grp, code, sc, mu);
-            for (int step = grp; step < nsteps && ok; step += 2) {
+            fetch(c0, grp, 0);
+            fetch(c0, grp + 2, 1);
+            for (int step = grp, k = 0; step < nsteps && ok; step += 2, ++k) {
                 const int gs = it * nsteps + step;             // global step: W ring position
                 const int sw = gs % SW, pw = (gs / SW) & 1;
+                const int slot = k & 1;
                 uint32_t o[8][4];
                 if (step < nks) {
-                    const float c = __fmaf_rn((float)code, sc, mu);
-                    fetch(c0, step + 2, code, sc, mu);
+                    const float c = block_const(slot);
                     const int gp = it * nks + step;            // global main step: P ring position
                     const int sp = gp % SP, pp = (gp / SP) & 1;
                     if (!(ok = tc::mbar_wait(fullP(sp), pp, s_abort))) break;
@@ -375,12 +424,14 @@ k_tc2_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
                 __syncwarp();
                 // the leader's own warps release at CTA scope (same CTA as the MMA issuer);
                 // the peer's warps release at cluster scope on the leader's barrier
-                if (lane == 0) {
-                    if (leader) tc::mbar_arrive(fullW(sw));
-                    else mbar_arrive_cl(mapa(fullW(sw), 0));
-                }
+                // the leader's warps arrive on its own barrier; the peer's on a local one whose
+                // completion a forwarder passes on (a cluster-scope release per warp and step
+                // would cost each dequantizer a cluster fence, ~1000 cycles)
+                if (lane == 0) tc::mbar_arrive(leader ? fullW(sw) : fullWl(sw));
+                fetch(c0, step + 4, slot);                     // refill: the group's step after next
             }
         }
+        asm volatile("cp.async.wait_all;" ::: "memory");
     } else {
         // ------------------------------------------------------------ epilogue (own 128 tokens)
         const int q = warp & 3;

@@ -81,7 +81,10 @@ enum {
  *   scale  [G] fp32, mean [G] fp32, G = ceil(N*K/64 / 256): group g covers
  *                          blocks [256g, 256g+256) of the flattened weight.
  *   The constant of block b is c'_b = fmaf((float)codes[b], scale[b/256],
- *   mean[b/256]) and the dequantized weight is bf16_rne(L[nibble] * c'_b). */
+ *   mean[b/256]) and the dequantized weight is bf16_rne(L[nibble] * c'_b).
+ *   packed must be 16-byte aligned; codes, scale and mean 4-byte aligned (the
+ *   fused kernels copy the codes as whole 32-bit words: N % 8 == 0 makes the
+ *   code count a multiple of 8). */
 typedef struct {
     const uint8_t* packed;
     const int8_t* codes;
