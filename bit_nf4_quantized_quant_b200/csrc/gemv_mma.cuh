@@ -287,20 +287,29 @@ struct FinishArgs {
 };
 
 __global__ void __launch_bounds__(TR) k_nf4_gemv_finish(FinishArgs a) {
-    __shared__ int s_slot[2 * 148];     // contributing (CTA, group) slots of this tile, in order
+    __shared__ int s_mask[148];         // groups of CTA c_first + j that took units of this tile
+    __shared__ int s_slot[2 * 148];     // their slots, in (CTA, group) order
     __shared__ int s_n;
     grid_dep_wait();
     const int tile = blockIdx.x, row = threadIdx.x;
     const int64_t m = blockIdx.y;
+    // unit counts fit 32 bits and CTA * units < 2^32 (units < 2^24, at most 148 CTAs)
+    const uint32_t U = (uint32_t)a.units, C = (uint32_t)a.ctas;
+    const uint32_t tu0 = (uint32_t)tile * (uint32_t)a.nks, tu1 = tu0 + (uint32_t)a.nks;
+    const uint32_t c_first = ((tu0 + 1) * C + U - 1) / U - 1, c_last = (tu1 * C + U - 1) / U - 1;
+    const int ncta = (int)(c_last - c_first + 1);
+    for (int j = row; j < ncta; j += TR) {
+        const uint32_t c = c_first + (uint32_t)j;
+        const uint32_t b0 = c * U / C, b1 = (c + 1) * U / C;
+        const uint32_t lo = b0 > tu0 ? b0 : tu0, hi = b1 < tu1 ? b1 : tu1;
+        s_mask[j] = hi - lo >= 2 ? 3 : (hi - lo == 1 ? 1 << ((lo - b0) & 1) : 0);
+    }
+    __syncthreads();
     if (row == 0) {
-        const int64_t tu0 = (int64_t)tile * a.nks, tu1 = tu0 + a.nks;
-        const int64_t c_first = unit_owner(tu0, a.units, a.ctas), c_last = unit_owner(tu1 - 1, a.units, a.ctas);
         int k = 0;
-        for (int64_t c = c_first; c <= c_last; ++c) {
-            const int gm = groups_in_tile(c, a.units, a.ctas, tu0, tu1);
+        for (int j = 0; j < ncta; ++j)
             for (int g2 = 0; g2 < 2; ++g2)
-                if ((gm >> g2) & 1) s_slot[k++] = (int)((c + tile) * 2 + g2);
-        }
+                if ((s_mask[j] >> g2) & 1) s_slot[k++] = (int)(((int64_t)c_first + j + tile) * 2 + g2);
         s_n = k;
     }
     __syncthreads();

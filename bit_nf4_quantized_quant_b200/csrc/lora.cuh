@@ -46,13 +46,14 @@ struct GemmArgs {
 template <bool A_KMAJ, bool B_KMAJ, int BI, int BJ, int WI, int WJ>
 __global__ void __launch_bounds__(128) k_gemm_mma(GemmArgs p) {
     constexpr int BK = 32;
+    constexpr int ST = 4;                              // cp.async stages: 3 tiles in flight per CTA
     constexpr int TI = BI / WI, TJ = BJ / WJ;          // warp tile
     static_assert(WI * WJ == 4 && TI % 16 == 0 && TJ % 16 == 0, "tile");
     constexpr int A_ROWS = A_KMAJ ? BI : BK, A_COLS = A_KMAJ ? BK : BI;
     constexpr int B_ROWS = B_KMAJ ? BJ : BK, B_COLS = B_KMAJ ? BK : BJ;
     constexpr int A_LD = A_COLS + 8, B_LD = B_COLS + 8;  // +16 bytes: ldmatrix rows hit distinct banks
-    __shared__ __align__(16) uint16_t sA[2][A_ROWS * A_LD];
-    __shared__ __align__(16) uint16_t sB[2][B_ROWS * B_LD];
+    __shared__ __align__(16) uint16_t sA[ST][A_ROWS * A_LD];
+    __shared__ __align__(16) uint16_t sB[ST][B_ROWS * B_LD];
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int wi = warp / WJ, wj = warp % WJ;
@@ -90,12 +91,21 @@ __global__ void __launch_bounds__(128) k_gemm_mma(GemmArgs p) {
         for (int b = 0; b < TJ / 8; ++b) acc[a][b][0] = acc[a][b][1] = acc[a][b][2] = acc[a][b][3] = 0.f;
 
     const int nk = (int)cdiv(kend - kbeg, BK);
-    if (nk > 0) load_tile(0, kbeg);
+    // multistage pipeline: tiles kt+1 .. kt+ST-1 are in flight while tile kt is multiplied
+#pragma unroll
+    for (int s2 = 0; s2 < ST - 1; ++s2) {
+        if (s2 < nk) load_tile(s2, kbeg + (int64_t)s2 * BK);
+        else cp_async_commit();
+    }
     for (int kt = 0; kt < nk; ++kt) {
-        const int st = kt & 1;
-        if (kt + 1 < nk) { load_tile(st ^ 1, kbeg + (int64_t)(kt + 1) * BK); cp_async_wait<1>(); }
-        else cp_async_wait<0>();
-        __syncthreads();
+        const int st = kt % ST;
+        cp_async_wait<ST - 2>();
+        __syncthreads();                               // tile kt landed; stage (kt-1) % ST is free
+        {
+            const int nt = kt + ST - 1;
+            if (nt < nk) load_tile(nt % ST, kbeg + (int64_t)nt * BK);
+            else cp_async_commit();
+        }
 #pragma unroll
         for (int kk = 0; kk < BK; kk += 16) {
             uint32_t af[TI / 16][4], bfr[TJ / 8][2];
@@ -129,8 +139,8 @@ __global__ void __launch_bounds__(128) k_gemm_mma(GemmArgs p) {
                 for (int b = 0; b < TJ / 8; ++b)
                     mma_bf16_16816(acc[a][b], af[a][0], af[a][1], af[a][2], af[a][3], bfr[b][0], bfr[b][1]);
         }
-        __syncthreads();
     }
+    cp_async_wait<0>();
 
     float* C = p.C + (int64_t)blockIdx.z * p.I * p.J;
     const int g = lane >> 2, t = lane & 3;

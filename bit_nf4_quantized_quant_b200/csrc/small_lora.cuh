@@ -256,9 +256,9 @@ struct BwdEndArgs {
     uint16_t* dA;            // [r, K]
 };
 
-// First unit of CTA c, and the CTA that owns unit u, for k_tcs_gemm's even
-// split of U units over C CTAs.
-__device__ __forceinline__ int64_t end_unit_owner(int64_t u, int64_t U, int64_t C) {
+// The CTA that owns unit u under k_tcs_gemm's even split of U units over C
+// CTAs (U < 2^23 and C <= 148, so the products fit 32 bits).
+__device__ __forceinline__ uint32_t end_unit_owner(uint32_t u, uint32_t U, uint32_t C) {
     return ((u + 1) * C + U - 1) / U - 1;
 }
 
@@ -299,9 +299,9 @@ __global__ void __launch_bounds__(kLoraThreads) k_bwd_small_end(BwdEndArgs a) {
     if (is_dx) {
         // dY W': the partial tiles of every CTA that took steps of column tile k / 128, in CTA order
         const int64_t tile = k >> 7, row = k & 127;
-        const int64_t tu0 = tile * a.nks;
-        const int64_t c_first = end_unit_owner(tu0, a.units, a.ctas);
-        const int64_t c_last = end_unit_owner(tu0 + a.nks - 1, a.units, a.ctas);
+        const uint32_t tu0 = (uint32_t)tile * (uint32_t)a.nks;
+        const int64_t c_first = end_unit_owner(tu0, (uint32_t)a.units, (uint32_t)a.ctas);
+        const int64_t c_last = end_unit_owner(tu0 + (uint32_t)a.nks - 1, (uint32_t)a.units, (uint32_t)a.ctas);
         float v = 0.f;
         for (int64_t c = c_first; c <= c_last; ++c) v += a.slots[(c + tile) * (a.NT * 128) + (int64_t)y * 128 + row];
         float l = 0.f;
