@@ -22,6 +22,17 @@ struct NF4Tables {
     float pad;
 };
 
+// Encoder lookup: x in [-1, 1] falls in bucket b = round(64 x + 64) (0..128);
+// thr[b] is the one decision threshold within (1/64 + 2e-3) of that bucket's
+// range, or +inf if none, and qb[b] counts the thresholds below that range,
+// so the level is qb[b] + (x > thr[b]).  The thresholds are at least 0.08
+// apart, so no bucket range holds two.
+constexpr int kEncBuckets = 129;
+struct EncTables {
+    float thr[kEncBuckets];
+    uint32_t qb[kEncBuckets];
+};
+
 // Sticky per-device status word; kernels whose bounded waits give up set it.
 __device__ int g_status;
 

@@ -42,6 +42,7 @@ double inv_phi_bisect(double p) {
 }
 
 NF4Tables g_tables;
+EncTables g_enc;
 std::once_flag g_tables_once;
 
 void init_tables() {
@@ -57,6 +58,21 @@ void init_tables() {
     for (int i = 0; i < 16; ++i) g_tables.L[i] = (float)(v[i] / top);
     for (int i = 0; i < 15; ++i) g_tables.m[i] = (g_tables.L[i] + g_tables.L[i + 1]) * 0.5f;
     g_tables.pad = 0.f;
+    // encoder buckets: bucket b holds x with round(64 x + 64) = b, i.e. x in
+    // [(b - 64.5) / 64, (b - 63.5) / 64], widened by eps against rounding
+    const double eps = 1.0 / 512.0;
+    for (int b = 0; b < kEncBuckets; ++b) {
+        const double lo = (b - 64.5) / 64.0 - eps, hi = (b - 63.5) / 64.0 + eps;
+        uint32_t below = 0;
+        float thr = INFINITY;
+        for (int i = 0; i < 15; ++i) {
+            const double mi = g_tables.m[i];
+            if (mi < lo) ++below;
+            else if (mi <= hi) thr = g_tables.m[i];    // at most one (thresholds are >= 0.08 apart)
+        }
+        g_enc.thr[b] = thr;
+        g_enc.qb[b] = below;
+    }
 }
 
 const NF4Tables& tables() {
@@ -680,7 +696,7 @@ int nf4_quantize_dq(const qlora_bf16* W, int64_t N, int64_t K, uint8_t* packed, 
     if (rc != QLORA_OK) return rc;
     const NF4Tables& tab = tables();
     int grid = (int)(ng < (int64_t)sms * 8 ? ng : (int64_t)sms * 8);
-    k_quantize_dq<<<grid, 256, 0, (cudaStream_t)stream>>>(W, nb, packed, codes, scale, mean, tab);
+    k_quantize_dq<<<grid, 256, 0, (cudaStream_t)stream>>>(W, nb, packed, codes, scale, mean, tab, g_enc);
     note_launch();
     return launch_status();
 }

@@ -23,6 +23,21 @@ __device__ __forceinline__ uint32_t nf4_encode(float x, const NF4Tables& tab, co
     return q;
 }
 
+// The exact level of w in a block with absmax c (the slow path of the encoder
+// below): x = fl32(w / c) by IEEE division, then the 4-step search; c = 0
+// gives level 7.  Kept out of line: it runs for about one weight in 10^5.
+__device__ __noinline__ uint32_t nf4_encode_exact(float w, float c, float m3, float m7, float m11,
+                                                  const float* s_m) {
+    if (c == 0.f) return 7u;
+    const float x = __fdiv_rn(w, c);
+    uint32_t q = (x > m7) ? 8u : 0u;
+    const float t = q ? m11 : m3;
+    q += (x > t) ? 4u : 0u;
+    q += (x > s_m[q + 1]) ? 2u : 0u;
+    q += (x > s_m[q]) ? 1u : 0u;
+    return q;
+}
+
 // One CTA (8 warps) per double-quant group of 256 blocks (16384 weights),
 // grid-stride over groups.  Warp w owns blocks [32w, 32w+32) of the group; a
 // block is handled by 8 lanes of 8 weights each (16-byte loads, coalesced
@@ -33,11 +48,14 @@ __device__ __forceinline__ uint32_t nf4_encode(float x, const NF4Tables& tab, co
 __global__ void __launch_bounds__(256) k_quantize_dq(const uint16_t* __restrict__ W, int64_t nblocks,
                                                      uint8_t* __restrict__ packed, int8_t* __restrict__ codes,
                                                      float* __restrict__ scale, float* __restrict__ mean,
-                                                     NF4Tables tab) {
+                                                     NF4Tables tab, const __grid_constant__ EncTables enc) {
     __shared__ float s_c[kGroup];
     __shared__ float s_m[16];
+    __shared__ float2 s_enc[kEncBuckets];          // (threshold, levels below) per bucket
     if (threadIdx.x < 15) s_m[threadIdx.x] = tab.m[threadIdx.x];
     if (threadIdx.x == 15) s_m[15] = INFINITY;
+    for (int b = threadIdx.x; b < kEncBuckets; b += blockDim.x)
+        s_enc[b] = make_float2(enc.thr[b], __uint_as_float(enc.qb[b]));
     __syncthreads();
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -72,11 +90,27 @@ __global__ void __launch_bounds__(256) k_quantize_dq(const uint16_t* __restrict_
             c = fmaxf(c, __shfl_xor_sync(0xffffffffu, c, 2));
             c = fmaxf(c, __shfl_xor_sync(0xffffffffu, c, 4));
             if (bl < nb) {
+                // Fast path: x' = w * (1/c) is within 1.5 * 2^-23 of x = fl32(w / c) (|x| <= 1),
+                // so when x' is more than 2^-20 from its bucket's threshold, x and x' sit on the
+                // same side of it and the level is qb + (x' > thr).  Otherwise (or c = 0, a
+                // reciprocal that is not finite, NaN) the exact quotient takes the 4-step search.
+                const float rcp = __frcp_rn(c);
+                const bool fast_blk = c > 0.f && rcp < INFINITY;
                 uint32_t word = 0;
 #pragma unroll
                 for (int j = 0; j < 8; ++j) {
                     uint32_t q = 7u;
-                    if (c != 0.f) q = nf4_encode(__fdiv_rn(w[j], c), tab, s_m);
+                    bool slow = !fast_blk;
+                    if (fast_blk) {
+                        const float x = __fmul_rn(w[j], rcp);
+                        // round(64 x + 64) from the low bits of 64 x + 64 + 1.5 * 2^23
+                        const uint32_t b = min(__float_as_uint(__fmaf_rn(x, 64.f, 12582976.f)) - 0x4B400000u, 128u);
+                        const float2 e = s_enc[b];
+                        const float d = __fsub_rn(x, e.x);
+                        slow = !(fabsf(d) > 9.5367431640625e-07f);     // 2^-20 (also NaN)
+                        q = __float_as_uint(e.y) + (d > 0.f ? 1u : 0u);
+                    }
+                    if (slow) q = nf4_encode_exact(w[j], c, tab.m[3], tab.m[7], tab.m[11], s_m);
                     // element 2i -> high nibble of byte i (little-endian word)
                     word |= q << ((j >> 1) * 8 + ((j & 1) ? 0 : 4));
                 }

@@ -122,3 +122,38 @@ def test_bulk_mixture_layer_sampled(oracle_mod):
             assert np.array_equal(w.packed.view(-1)[lo // 2:hi // 2].cpu().numpy(), q["packed"].reshape(-1))
             assert np.array_equal(w.codes[g * 256:(g + 1) * 256].cpu().numpy(), q["codes"])
             assert np.array_equal(inputs.bf16_bits(Wd.view(-1)[lo:hi]), oracle_mod.dequant(q).reshape(-1))
+
+
+def test_quantize_near_thresholds(oracle_mod):
+    """Weights whose normalised value w / c lies within a few ulp of an NF4
+    decision threshold (and exactly on one where the division lands there):
+    every bf16 weight in a window of +-1.5 % around c * m_i, for every midpoint
+    m_i and block maxima c (every bf16 mantissa in [1, 2), and tiny and
+    subnormal ones), each block led
+    by +-c so that c is its absmax.  Bit-exact against the oracle, which
+    divides in IEEE fp32 -- this is where the kernel's reciprocal-and-bucket
+    fast path must hand over to the exact quotient."""
+    def bits_of(v):
+        return int(inputs.bf16_bits(torch.tensor([v], dtype=torch.float32).to(torch.bfloat16))[0])
+
+    blocks = []
+    maxima = [1.0 + k / 128.0 for k in range(128)] + [0.0234375, 3.0e-3, 7.25, 1.0e-30, 1.0e-39]
+    for c in maxima:
+        for mi in np.asarray(oracle_mod.midpoints(), dtype=np.float64):
+            centre = c * mi
+            a, b = bits_of(centre * 0.985), bits_of(centre * 1.015)
+            vals = np.arange(min(a, b), max(a, b) + 1, dtype=np.uint32).astype(np.uint16)
+            lead = np.uint16(bits_of(c) | (0x8000 if mi < 0 else 0))
+            for s0 in range(0, len(vals), 63):
+                blk = np.zeros(64, dtype=np.uint16)
+                blk[0] = lead
+                chunk = vals[s0:s0 + 63]
+                blk[1:1 + len(chunk)] = chunk
+                blocks.append(blk)
+    while len(blocks) % 64:                 # 8 rows of 8 blocks: N a multiple of 8
+        blocks.append(np.zeros(64, dtype=np.uint16))
+    bits = np.stack(blocks).reshape(-1, 512)
+    W = torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16)
+    q = oracle_mod.quantize_dq(inputs.bf16_bits(W))
+    w = _gpu_quant(W)
+    _assert_same_quant(w, q)
