@@ -37,7 +37,12 @@ using tc::Args;
 
 constexpr int BM = 256, BN = 256, BK = 64;       // pair tile
 constexpr int HM = 128, HN = 128;                // per-CTA halves
-constexpr int SA = 5, SW = 5, SP = 8;
+constexpr int SA = 5, SW = 6, SP = 8;
+// The W' and packed rings are split into one sub-ring per dequantizer group
+// (SW / 2 and SP / 2 stages), each filled and drained in that group's step
+// order, so every waiter is at most one phase ahead of the barrier it waits on
+// (a parity wait cannot tell phase k from phase k - 2).
+constexpr int SWH = SW / 2, SPH = SP / 2;
 constexpr int A_BYTES = HM * BK * 2;             // 16 KB
 constexpr int W_BYTES = HN * BK * 2;             // 16 KB
 constexpr int P_BYTES = HN * BK / 2;             // 4 KB
@@ -229,6 +234,19 @@ k_tc2_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
     tc::tc_fence_after();
     const uint32_t tmem_base = *s_tmem;
 
+    // Ring position of step `step` of this CTA's it-th tile: group g = step % 2 uses
+    // stages g * half .. g * half + half - 1 in its own step order.
+    auto wpos = [&](int it, int step, int& st, int& ph) {
+        const int g = step & 1, per = (nsteps + 1 - g) >> 1, j = it * per + (step >> 1);
+        st = g * SWH + j % SWH;
+        ph = (j / SWH) & 1;
+    };
+    auto ppos = [&](int it, int step, int& st, int& ph) {
+        const int g = step & 1, per = (nks + 1 - g) >> 1, j = it * per + (step >> 1);
+        st = g * SPH + j % SPH;
+        ph = (j / SPH) & 1;
+    };
+
     // Peer CTA: pass the completion of each stage of the dequantized-weight ring on to
     // the leader's barrier, for the steps of dequantizer group grp: one cluster-scope
     // fence and one relaxed remote arrive per stage.
@@ -237,8 +255,8 @@ k_tc2_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
         int it = 0;
         for (int64_t tile = pair; tile < ntiles && ok; tile += npairs, ++it) {
             for (int step = grp; step < nsteps && ok; step += 2) {
-                const int gs = it * nsteps + step;
-                const int sw = gs % SW, pw = (gs / SW) & 1;
+                int sw, pw;
+                wpos(it, step, sw, pw);
                 if (!(ok = tc::mbar_wait(fullWl(sw), pw, s_abort))) break;
                 asm volatile("fence.acq_rel.cluster;" ::: "memory");
                 asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(mapa(fullW(sw), 0))
@@ -270,27 +288,32 @@ k_tc2_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
     } else if (warp == 14) {
         // ------------------------------------------------------------ packed weights (own half)
         if (lane == 0) {
-            int sp = 0, pp = 0, issued = 0;
+            int last_ph[SP];                             // phase of each stage's last issued copy
+#pragma unroll
+            for (int i = 0; i < SP; ++i) last_ph[i] = -1;
             bool ok = true;
-            for (int64_t tile = pair; tile < ntiles && ok; tile += npairs) {
+            int it = 0;
+            for (int64_t tile = pair; tile < ntiles && ok; tile += npairs, ++it) {
                 const int c0 = (int)((tile / mtiles) * BN + crank * HN);
                 for (int step = 0; step < nks && ok; ++step) {
+                    int sp, pp;
+                    ppos(it, step, sp, pp);
                     if (!(ok = tc::mbar_wait(emptyP(sp), pp ^ 1, s_abort))) break;
                     tc::mbar_expect_tx(fullP(sp), P_BYTES);
                     if (!BWD) tc::tma_load_2d(sbase + OFF_P + sp * P_BYTES, &tmP, fullP(sp), step * (BK / 2), c0);
                     else tc::tma_load_2d(sbase + OFF_P + sp * P_BYTES, &tmP, fullP(sp), c0 / 2, step * BK);
-                    ++issued;
-                    if (++sp == SP) { sp = 0; pp ^= 1; }
+                    last_ph[sp] = pp;
                 }
             }
-            if (!ok)
-                for (int i = 1; i <= SP && i <= issued; ++i) tc::mbar_drain(fullP((issued - i) % SP), ((issued - i) / SP) & 1);
+            if (!ok)                                     // wait for the copies in flight
+                for (int i = 0; i < SP; ++i)
+                    if (last_ph[i] >= 0) tc::mbar_drain(fullP(i), last_ph[i]);
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer (leader only)
         if (leader && lane == 0) {
             constexpr uint32_t idesc = make_idesc2(BWD);
-            int sa = 0, pa = 0, sw = 0, pw = 0;
+            int sa = 0, pa = 0;
             bool ok = true;
             int it = 0;
             for (int64_t tile = pair; tile < ntiles && ok; tile += npairs, ++it) {
@@ -299,6 +322,8 @@ k_tc2_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
                 tc::tc_fence_after();
                 const uint32_t d_tmem = tmem_base + acc * BN;
                 for (int step = 0; step < nsteps && ok; ++step) {
+                    int sw, pw;
+                    wpos(it, step, sw, pw);
                     if (!(ok = mbar_wait_cl(fullA(sa), pa, s_abort))) break;
                     if (!(ok = mbar_wait_cl(fullW(sw), pw, s_abort))) break;
                     tc::tc_fence_after();
@@ -314,7 +339,6 @@ k_tc2_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
                     tc2_commit_both(emptyA(sa));
                     tc2_commit_both(emptyW(sw));
                     if (++sa == SA) { sa = 0; pa ^= 1; }
-                    if (++sw == SW) { sw = 0; pw ^= 1; }
                 }
                 if (ok) tc2_commit_both(tfull(acc));
             }
@@ -370,14 +394,14 @@ k_tc2_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
             fetch(c0, grp, 0);
             fetch(c0, grp + 2, 1);
             for (int step = grp, k = 0; step < nsteps && ok; step += 2, ++k) {
-                const int gs = it * nsteps + step;             // global step: W ring position
-                const int sw = gs % SW, pw = (gs / SW) & 1;
+                int sw, pw;
+                wpos(it, step, sw, pw);
                 const int slot = k & 1;
                 uint32_t o[8][4];
                 if (step < nks) {
                     const float c = block_const(slot);
-                    const int gp = it * nks + step;            // global main step: P ring position
-                    const int sp = gp % SP, pp = (gp / SP) & 1;
+                    int sp, pp;
+                    ppos(it, step, sp, pp);
                     if (!(ok = tc::mbar_wait(fullP(sp), pp, s_abort))) break;
                     uint4 p0, p1;
                     const uint32_t pst = sbase + OFF_P + sp * P_BYTES;
