@@ -44,7 +44,13 @@ struct GemmArgs {
 };
 
 template <bool A_KMAJ, bool B_KMAJ, int BI, int BJ, int WI, int WJ>
+// The adapter kernels run as a chain on one stream with programmatic launch:
+// each lets the next one start launching at once, then waits for the one
+// before it (whose outputs it may read, or whose inputs it may overwrite)
+// before touching global memory.
 __global__ void __launch_bounds__(128) k_gemm_mma(GemmArgs p) {
+    grid_dep_launch();
+    grid_dep_wait();
     constexpr int BK = 32;
     constexpr int ST = 4;                              // cp.async stages: 3 tiles in flight per CTA
     constexpr int TI = BI / WI, TJ = BJ / WJ;          // warp tile
@@ -187,6 +193,8 @@ struct FinishArgs {
 };
 
 __global__ void __launch_bounds__(256) k_gemm_finish(FinishArgs f) {
+    grid_dep_launch();
+    grid_dep_wait();
     if (f.zero)
         for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < f.zero_n; e += (int64_t)gridDim.x * blockDim.x)
             f.zero[e] = 0;
@@ -219,6 +227,8 @@ __global__ void __launch_bounds__(256) k_gemm_finish(FinishArgs f) {
 // dst [rows, dcols] bf16 = src [rows, scols] zero-padded (dcols >= scols).
 __global__ void k_pad_cols(const uint16_t* __restrict__ src, int64_t rows, int64_t scols, uint16_t* __restrict__ dst,
                            int64_t dcols) {
+    grid_dep_launch();
+    grid_dep_wait();
     const int64_t total = rows * dcols;
     for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < total; e += (int64_t)gridDim.x * blockDim.x) {
         const int64_t i = e / dcols, j = e % dcols;

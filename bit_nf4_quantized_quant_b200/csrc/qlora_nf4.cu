@@ -156,6 +156,27 @@ int launch_status() {
     return e == cudaSuccess ? QLORA_OK : QLORA_ERR_LAUNCH;
 }
 
+// Launch with programmatic stream serialization: the kernel may start while
+// the kernel before it on the stream is still running (that kernel calls
+// grid_dep_launch() first; this one calls grid_dep_wait() before it reads
+// anything the other writes).
+template <typename... KArgs, typename... Args>
+int launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st, Args... args) {
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    at[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, args...);
+    note_launch();
+    return e == cudaSuccess ? QLORA_OK : QLORA_ERR_LAUNCH;
+}
+
 // ---------------------------------------------------------------------------
 // Workspace plan: every region 256-byte aligned; regions used one after the
 // other on a stream may share the "partials" region.
@@ -297,15 +318,14 @@ int run_gemm(const uint16_t* A, int64_t lda, const uint16_t* B, int64_t ldb, int
     gemm_tile(I, J, &bi, &bj);
     g.I = rup(I, bi); g.J = rup(J, bj);
     dim3 grid((unsigned)(g.I / bi), (unsigned)(g.J / bj), (unsigned)z);
-    if (bj == 16) k_gemm_mma<AK, BK, 64, 16, 4, 1><<<grid, 128, 0, st>>>(g);
-    else if (bi == 16) k_gemm_mma<AK, BK, 16, 64, 1, 4><<<grid, 128, 0, st>>>(g);
-    else k_gemm_mma<AK, BK, 64, 64, 2, 2><<<grid, 128, 0, st>>>(g);
-    note_launch();
+    int rc;
+    if (bj == 16) rc = launch_pdl(k_gemm_mma<AK, BK, 64, 16, 4, 1>, grid, dim3(128), 0, st, g);
+    else if (bi == 16) rc = launch_pdl(k_gemm_mma<AK, BK, 16, 64, 1, 4>, grid, dim3(128), 0, st, g);
+    else rc = launch_pdl(k_gemm_mma<AK, BK, 64, 64, 2, 2>, grid, dim3(128), 0, st, g);
+    if (rc != QLORA_OK) return rc;
     f.I = g.I; f.J = g.J;
     if (f.Iout > I) f.Iout = I;
-    k_gemm_finish<<<grid_for(f.Iout * f.Jiter, 256, sms), 256, 0, st>>>(f);
-    note_launch();
-    return launch_status();
+    return launch_pdl(k_gemm_finish, dim3((unsigned)grid_for(f.Iout * f.Jiter, 256, sms)), dim3(256), 0, st, f);
 }
 
 FinishArgs fin_none() {
@@ -486,42 +506,15 @@ int compute_T(const Plan& p, const uint16_t* X, const uint16_t* A, float s, uint
     f.J1 = p.r;
     f.hl = reinterpret_cast<uint16_t*>(ws + p.off_Tp); f.hl_ld = 2 * p.rp; f.hl_off = p.rp;
     f.o2 = reinterpret_cast<uint16_t*>(ws + p.off_sT); f.s2i = p.rp64; f.s2j = 1; f.J2 = p.r; f.J2pad = p.rp64; f.alpha2 = s;
-    int rc = run_gemm<true, true>(X, p.K, A, p.K, p.M, p.rp, p.K, p.M, p.r, p.zT, p.kT,
-                                  reinterpret_cast<float*>(ws + p.off_part), f, sms, st);
-    if (rc != QLORA_OK) return rc;
-    if (T_out) {
-        // bf16 T in the caller's [M, r] layout: the hi half of Thl
-        k_pad_cols<<<grid_for(p.M * p.r, 256, sms), 256, 0, st>>>(reinterpret_cast<uint16_t*>(ws + p.off_Tp), p.M,
-                                                                   2 * p.rp, T_out, p.r);
-        note_launch();
-        rc = launch_status();
+    if (T_out) {   // the caller's bf16 T [M, r]: the same rounding as the hi half of Thl
+        f.o1 = T_out; f.s1i = p.r; f.s1j = 1; f.J1pad = p.r; f.alpha1 = 1.f;
     }
-    return rc;
+    return run_gemm<true, true>(X, p.K, A, p.K, p.M, p.rp, p.K, p.M, p.r, p.zT, p.kT,
+                                reinterpret_cast<float*>(ws + p.off_part), f, sms, st);
 }
 
 
-// Launch with programmatic stream serialization: the kernel may start while
-// the kernel before it on the stream is still running (that kernel calls
-// grid_dep_launch() first; this one calls grid_dep_wait() before it reads
-// anything the other writes).
-template <typename... KArgs, typename... Args>
-int launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st, Args... args) {
-    cudaLaunchConfig_t cfg{};
-    cfg.gridDim = grid;
-    cfg.blockDim = block;
-    cfg.dynamicSmemBytes = smem;
-    cfg.stream = st;
-    cudaLaunchAttribute at[1];
-    at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    at[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = at;
-    cfg.numAttrs = 1;
-    const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, args...);
-    note_launch();
-    return e == cudaSuccess ? QLORA_OK : QLORA_ERR_LAUNCH;
-}
-
-// Small-M T = X A^T into T32 (and the caller's bf16 T_out); clears `zero`.
+// Small-M T = X A^T into T32 (and the caller's bf16 T_out).
 int small_T(const Plan& p, const uint16_t* X, const uint16_t* A, uint16_t* T_out, uint8_t* ws, cudaStream_t st) {
     LoraDownArgs d{};
     d.X = X; d.A = A; d.M = p.M; d.K = p.K; d.r = p.r; d.rp = p.rp;
@@ -755,8 +748,9 @@ int qlora_linear_fwd(const qlora_bf16* X, int64_t M, const nf4dq_weight* w, cons
     int64_t ldl = r;
     if (r % 8 != 0) {
         uint16_t* Bp = reinterpret_cast<uint16_t*>(wsb + p.off_Bp);
-        k_pad_cols<<<grid_for(w->N * p.rp, 256, sms), 256, 0, st>>>(B, w->N, r, Bp, p.rp);
-        note_launch();
+        rc = launch_pdl(k_pad_cols, dim3((unsigned)grid_for(w->N * p.rp, 256, sms)), dim3(256), 0, st, B, w->N,
+                        (int64_t)r, Bp, (int64_t)p.rp);
+        if (rc != QLORA_OK) return rc;
         lw = Bp;
         ldl = p.rp;
     } else if (!aligned16(B)) {
@@ -806,13 +800,15 @@ int qlora_linear_bwd(const qlora_bf16* X, const qlora_bf16* dY, int64_t M, const
     uint16_t* Uhl = reinterpret_cast<uint16_t*>(wsb + p.off_Ubf);
     uint16_t* Bp = reinterpret_cast<uint16_t*>(wsb + p.off_Bp);
 
-    // T: recompute (hi + lo pair), or take the caller's bf16 copy as it is (lo = 0)
+    // T: recompute (hi + lo pair), or take the caller's bf16 copy as it is -- read in
+    // place by the dB product when its rows are 16-byte granular, else padded to [M, 2 rp]
+    // with a zero lo half
+    const bool t_direct = T != nullptr && r % 8 == 0 && aligned16(T);
     if (T == nullptr) {
         rc = compute_T(p, X, A, scaling, nullptr, wsb, sms, st);
-    } else {
-        k_pad_cols<<<grid_for(M * 2 * p.rp, 256, sms), 256, 0, st>>>(T, M, r, Thl, 2 * p.rp);
-        note_launch();
-        rc = launch_status();
+    } else if (!t_direct) {
+        rc = launch_pdl(k_pad_cols, dim3((unsigned)grid_for(M * 2 * p.rp, 256, sms)), dim3(256), 0, st, T, M,
+                        (int64_t)r, Thl, (int64_t)(2 * p.rp));
     }
     if (rc != QLORA_OK) return rc;
 
@@ -820,8 +816,9 @@ int qlora_linear_bwd(const qlora_bf16* X, const qlora_bf16* dY, int64_t M, const
     const uint16_t* Bop = B;
     int64_t ldb = r;
     if (r % 8 != 0 || !aligned16(B)) {
-        k_pad_cols<<<grid_for(N * p.rp, 256, sms), 256, 0, st>>>(B, N, r, Bp, p.rp);
-        note_launch();
+        rc = launch_pdl(k_pad_cols, dim3((unsigned)grid_for(N * p.rp, 256, sms)), dim3(256), 0, st, B, N, (int64_t)r,
+                        Bp, (int64_t)p.rp);
+        if (rc != QLORA_OK) return rc;
         Bop = Bp; ldb = p.rp;
     }
     {
@@ -835,12 +832,16 @@ int qlora_linear_bwd(const qlora_bf16* X, const qlora_bf16* dY, int64_t M, const
         rc = run_gemm<true, false>(dY, N, Bop, ldb, M, p.rp, N, M, r, p.zU, p.kU, part, f, sms, st);
         if (rc != QLORA_OK) return rc;
     }
-    // dB = s dY^T T  [N, r]   (T as hi | lo columns, summed in the finish)
+    // dB = s dY^T T  [N, r]   (T as hi | lo columns, summed in the finish, or the caller's T)
     {
         FinishArgs f = fin_none();
-        f.Iout = N; f.Jiter = r; f.col_pair = p.rp;
+        f.Iout = N; f.Jiter = r; f.col_pair = t_direct ? 0 : p.rp;
         f.o1 = dB; f.s1i = r; f.s1j = 1; f.J1 = r; f.J1pad = r; f.alpha1 = scaling;
-        rc = run_gemm<false, false>(dY, N, Thl, 2 * p.rp, N, 2 * p.rp, M, N, 2 * p.rp, p.zB, p.kB, part, f, sms, st);
+        if (t_direct)
+            rc = run_gemm<false, false>(dY, N, T, r, N, p.rp, M, N, r, p.zB, p.kB, part, f, sms, st);
+        else
+            rc = run_gemm<false, false>(dY, N, Thl, 2 * p.rp, N, 2 * p.rp, M, N, 2 * p.rp, p.zB, p.kB, part, f, sms,
+                                        st);
         if (rc != QLORA_OK) return rc;
     }
     // dA = s U^T X  [r, K]   (U as hi | lo rows, summed in the finish)

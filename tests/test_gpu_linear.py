@@ -59,6 +59,9 @@ CASES = [
     (129, 256, 512, 16),
     (640, 1280, 1024, 32),
     (1000, 520, 1088, 64),
+    (2, 256, 512, 256),         # maximum rank on each path
+    (64, 256, 512, 256),
+    (130, 256, 512, 256),
 ]
 
 
