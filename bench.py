@@ -239,8 +239,11 @@ def run_ours(args, rank, world, local_rank):
         dist.barrier()
 
     # ---- timed region: one CUDA graph per timed step (the library calls are
-    # asynchronous and allocation-free, so a step captures as is); each graph
-    # records its own per-launch events around the fused dequant-GEMM kernels
+    # asynchronous and allocation-free, so a step captures as is).  The last
+    # timed step also records the library's per-launch events around the fused
+    # dequant-GEMM kernels: an event between two kernels ends the overlap that
+    # programmatic launch gives them, so the other steps carry none.
+    ev_step = args.steps - 1
     kev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
             for _ in range(2 * len(layers))] for _ in range(args.steps)]
     for evs in kev:                 # torch creates the CUDA events lazily: record once so they exist
@@ -253,7 +256,7 @@ def run_ours(args, rank, world, local_rank):
         for k in range(args.steps):
             g = torch.cuda.CUDAGraph()
             with torch.cuda.graph(g):
-                step(kev[k], collective=False)
+                step(kev[k] if k == ev_step else None, collective=False)
             graphs.append(g)
         for g in graphs:            # upload + warm
             g.replay()
@@ -277,7 +280,7 @@ def run_ours(args, rank, world, local_rank):
             if world > 1 and bwd:
                 dist.all_reduce(gbuf)
         else:
-            step(kev[k])
+            step(kev[k] if k == ev_step else None)
     t1.record(stream)
     torch.cuda.nvtx.range_pop()
     torch.cuda.synchronize()
@@ -311,22 +314,22 @@ def run_ours(args, rank, world, local_rank):
     kbytes = 0
     kev_src = "graph replay" if graphs else "timed steps"
     try:
-        kev[0][0][0].elapsed_time(kev[0][0][1])
+        kev[ev_step][0][0].elapsed_time(kev[ev_step][0][1])
     except RuntimeError:
         # events inside a replayed graph could not be timed: time the kernels
-        # over the same number of steps launched eagerly on the same stream
+        # of one step launched eagerly on the same stream
         torch.cuda.synchronize()
-        for k in range(args.steps):
-            step(kev[k], collective=False)
+        step(kev[ev_step], collective=False)
         torch.cuda.synchronize()
         kev_src = "eager pass after the timed steps"
-    for k in range(args.steps):
+    for k in (ev_step,):
         for j, L in enumerate(layers):
             N_, K_ = L["p"].N, L["p"].K
             f_fwd, f_bwd = main_kernel_flops(M, N_, K_, r)
-            # small M: the timed pair in the forward is T = X A^T + the GEMV (NF4 weight, X, A, B
-            # read, Y and T written once); in the backward the U / dB kernel + the dX GEMV
-            # (NF4 weight, dY, B and T read, dB written once; split partials not counted)
+            # small M: the timed pair in the forward is the GEMV (which also computes T = X A^T)
+            # + its finish kernel (NF4 weight, X, A, B read, Y and T written once); in the
+            # backward the U / dB kernel + the dX GEMV (NF4 weight, dY, B and T read, dB
+            # written once; split partials not counted)
             b_fwd = nf4_bytes(N_, K_) + 2 * (M * K_ + M * N_ + r * K_ + N_ * r + M * r)
             b_bwd = nf4_bytes(N_, K_) + 2 * (M * N_ + 2 * N_ * r + M * r)
             for h, f, bb in ((0, f_fwd, b_fwd), (1, f_bwd, b_bwd))[:npass]:
@@ -347,7 +350,7 @@ def run_ours(args, rank, world, local_rank):
     roof.update({"achieved": round(achieved, 2), "peak": peak, "frac": round(achieved / peak, 4),
                  "traffic": tr["bytes_per_launch"] if tr and tr.get("src") == src_hash() else None,
                  "peak_source": f"{peak_src} ({'hbm copy' if small else 'cuBLAS bf16 sustained'})",
-                 "kernel": ("k_lora_down_small + k_nf4_gemv / k_lora_bwd_small + k_tcs_gemm (programmatic-launch pairs)"
+                 "kernel": ("k_nf4_gemv + k_nf4_gemv_finish / k_lora_bwd_small + k_tcs_gemm (programmatic-launch pairs)"
                             if small else "k_tc_gemm / k_tc2_gemm (fwd + bwd dX)"),
                  "launches_timed": nlaunch, "avg_launch_us": round(kms / nlaunch * 1e3, 2),
                  "events_from": kev_src})

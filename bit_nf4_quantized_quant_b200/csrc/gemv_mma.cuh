@@ -17,22 +17,31 @@
 //    two whole blocks (rows g and g + 8) and builds two tables.
 //  * Work unit = (128 rows, 256 reduction) = 8 warps x 16 rows.  The units
 //    are split evenly over the CTAs in (tile, step) order; in a CTA two
-//    groups of 8 warps take alternate units.  Every (CTA, group) pair writes
+//    groups of 8 warps take alternate units, each group with its own producer
+//    warp and its own half of the stage ring.  Every (CTA, group) pair writes
 //    its partial sum of each tile it touched to its own slot; the small
 //    k_nf4_gemv_finish kernel sums the slots of a tile in (CTA, group) order
 //    -- deterministic -- and adds s T B^T (no atomics or counters, so the
 //    fused kernel ends as soon as its last unit is done).
-//  * Warp 0 lane 0 loads each unit's packed tile (128 rows x 128 B, 128-byte
-//    swizzle) with TMA; the 32 lanes of warp 0 copy the unit's activation
-//    slice with cp.async into a fragment-native layout ([j][token][t] 16-byte
+//  * A producer warp's lane 0 loads each unit's packed tile (128 rows x 128 B,
+//    128-byte swizzle) with TMA; its 32 lanes copy the unit's activation slice
+//    with cp.async into a fragment-native layout ([j][token][t] 16-byte
 //    chunks: the 16 bytes lane (g, t) feeds to MMAs 2j and 2j+1), so the
 //    consumers' shared loads are conflict-free; both complete on the stage's
 //    mbarrier.  Rows of the slice beyond M are zeroed once and never copied.
+//  * Three programmatic launches make the forward: this kernel, then the
+//    small T = X A^T kernel (which runs beside it on the SMs' spare registers
+//    and ends only after it), then the finish kernel.  Before it waits for
+//    the kernel ahead of it on the stream, the GEMV only sets up its barriers
+//    and warms L2 with its first packed tiles (an L2 prefetch cannot return
+//    stale data: L2 is the point of coherence); everything it reads is read
+//    after the wait, and it releases the T kernel right after it.
 #pragma once
 #include <cuda.h>
 #include "common.cuh"
 #include "nf4_decode.cuh"
 #include "tc_gemm.cuh"
+#include "small_lora.cuh"
 
 namespace qnf4 {
 namespace gmv {
@@ -41,14 +50,16 @@ constexpr int TR = 128;                          // rows of a unit
 constexpr int KSTEP = 256;                       // reduction of a unit
 constexpr int P_BYTES = TR * KSTEP / 2;          // 16384
 constexpr int kGroupWarps = 8;
-constexpr int kThreads = 32 * (1 + 2 * kGroupWarps);   // 544
+constexpr int kFirstMath = 2;                    // warps 0, 1: producers of groups 0, 1; 2 .. 17: decode + MMA
+constexpr int kThreads = 32 * (kFirstMath + 2 * kGroupWarps);   // 576
 
 template <int NTT>
 struct Cfg {
     static constexpr int NT = 8 * NTT;                  // token columns (zero beyond M)
     static constexpr int X_BYTES = NT * KSTEP * 2;      // 4096 * NTT
     static constexpr int STAGE = P_BYTES + X_BYTES;     // a multiple of 1024
-    static constexpr int SP = NTT == 4 ? 4 : 8;         // stages (half per group), a power of 2
+    static constexpr int SP = NTT == 4 ? 4 : 8;         // stages, a power of 2
+    static constexpr int SPG = SP / 2;                  // stages of each group's ring
     static constexpr int OFF_BAR = SP * STAGE;
     static constexpr int SMEM_ALLOC = OFF_BAR + 2 * SP * 8 + 16 + 1024;
 };
@@ -89,12 +100,18 @@ __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, int sr
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
 }
 
+__device__ __forceinline__ void tma_prefetch_l2(const CUtensorMap* map, int x, int y) {
+    asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];"
+                 ::"l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y) : "memory");
+}
+
 template <int NTT>
 __global__ void __launch_bounds__(kThreads, 1) k_nf4_gemv(const __grid_constant__ CUtensorMap tmP, Args a,
                                                         NF4Tables tab) {
     using C = Cfg<NTT>;
     constexpr int NT = C::NT;
     constexpr int SP = C::SP;
+    constexpr int SPG = C::SPG;
     extern __shared__ __align__(1024) uint8_t smem[];
     uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem) + 1023) & ~(uintptr_t)1023);
     const uint32_t sbase = smem_u32(base);
@@ -120,6 +137,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_nf4_gemv(const __grid_constant_
         }
     }
     if (tid == 0) {
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmP)) : "memory");
         for (int i = 0; i < SP; ++i) {
             tc::mbar_init(full(i), 1 + 32);              // TMA expect-tx arrival + 32 cp.async arrivals
             tc::mbar_init(empty(i), kGroupWarps);
@@ -129,13 +147,29 @@ __global__ void __launch_bounds__(kThreads, 1) k_nf4_gemv(const __grid_constant_
     }
     __syncthreads();
 
-    if (warp == 0) {
-        // ------------------------------------------------------------ producer
-        int tile = tile0, ks = ks0, issued = 0;
+    // CTA-local unit i belongs to group i & 1; its group-local index q = i >> 1
+    // selects stage (group, q mod SPG) with parity (q / SPG) & 1.
+    if (warp < kFirstMath) {
+        // ------------------------------------------------------------ producer of group `warp`
+        const int grp = warp;
+        const int nq = nu > grp ? (nu - grp + 1) / 2 : 0;
+        int tile = tile0, ks = ks0;
+        unit_advance(tile, ks, grp, nks);
+        if (lane == 0) {            // warm L2 with the group's first packed tiles
+            int pt = tile, pk = ks;
+            for (int q = 0; q < nq && q < 2 * SPG; ++q) {
+                tma_prefetch_l2(&tmP, pk * (KSTEP / 2), pt * TR);
+                unit_advance(pt, pk, 2, nks);
+            }
+        }
+        grid_dep_wait();
+        // X is complete: the T kernel launched behind this one may start (and read it)
+        if (grp == 0 && lane == 0) grid_dep_launch();
+        int issued = 0;
         bool ok = true;
         const int64_t mrows = a.M < NT ? a.M : NT;
-        for (int i = 0; i < nu; ++i) {
-            const int st = i % SP, ph = (i / SP) & 1;
+        for (int q = 0; q < nq; ++q) {
+            const int st = grp * SPG + q % SPG, ph = (q / SPG) & 1;
             int w_ok = 1;
             if (lane == 0) w_ok = tc::mbar_wait(empty(st), ph ^ 1, s_abort) ? 1 : 0;
             ok = __shfl_sync(0xffffffffu, w_ok, 0) != 0;
@@ -156,20 +190,21 @@ __global__ void __launch_bounds__(kThreads, 1) k_nf4_gemv(const __grid_constant_
             }
             asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(full(st)) : "memory");
             ++issued;
-            unit_advance(tile, ks, 1, nks);
+            unit_advance(tile, ks, 2, nks);
         }
         // on abort: let the copies in flight land before the CTA exits
         asm volatile("cp.async.wait_all;" ::: "memory");
         if (!ok && lane == 0)
-            for (int k = 1; k <= SP && k <= issued; ++k)
-                tc::mbar_drain(full((issued - k) % SP), ((issued - k) / SP) & 1);
+            for (int k = 1; k <= SPG && k <= issued; ++k)
+                tc::mbar_drain(full(grp * SPG + (issued - k) % SPG), ((issued - k) / SPG) & 1);
     } else {
         // ------------------------------------------------------------ decode + MMA warps
-        const int grp = (warp - 1) / kGroupWarps;        // units i = grp, grp + 2, ...
-        const int w8 = (warp - 1) % kGroupWarps;         // rows 16 w8 .. 16 w8 + 15 of a unit
+        const int grp = (warp - kFirstMath) / kGroupWarps;    // units i = grp, grp + 2, ...
+        const int w8 = (warp - kFirstMath) % kGroupWarps;     // rows 16 w8 .. 16 w8 + 15 of a unit
         const int g = lane >> 2, t = lane & 3;
         const int r0 = 16 * w8 + g;                      // rows r0 and r0 + 8 of the tile
         bool ok = true;
+        grid_dep_wait();
 
         // block-constant inputs of rows r0, r0 + 8, block 4 ks + t of the next unit to
         // fetch (zero beyond the weight); fetches run two group-units ahead
@@ -223,10 +258,10 @@ __global__ void __launch_bounds__(kThreads, 1) k_nf4_gemv(const __grid_constant_
         // swizzled offsets of this lane's packed chunks (row r0; row r0 + 8 has the same swizzle)
         const uint32_t pch0 = (uint32_t)(r0 * 128 + (((2 * t) ^ (r0 & 7)) << 4));
         const uint32_t pch1 = (uint32_t)(r0 * 128 + (((2 * t + 1) ^ (r0 & 7)) << 4));
-        auto do_unit = [&](int i, BC& b) {
+        auto do_unit = [&](int q, BC& b) {
             const float c0 = __fmaf_rn((float)b.c0, b.s0, b.m0), c1 = __fmaf_rn((float)b.c1, b.s1, b.m1);
             fetch(b);
-            const int st = i % SP, ph = (i / SP) & 1;
+            const int st = grp * SPG + q % SPG, ph = (q / SPG) & 1;
             if (!(ok = tc::mbar_wait(full(st), ph, s_abort))) return;
             const uint32_t sst = sbase + st * C::STAGE;
             uint32_t pa[8], pb[8];
@@ -254,8 +289,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_nf4_gemv(const __grid_constant_
             __syncwarp();
             if (lane == 0) tc::mbar_arrive(empty(st));
         };
-        for (int i = grp; i < nu && ok; i += 2) {
-            do_unit(i, ((i >> 1) & 1) ? bB : bA);
+        for (int i = grp, q = 0; i < nu && ok; i += 2, ++q) {
+            do_unit(q, (q & 1) ? bB : bA);
             if (!ok) break;
             // the group's next unit is i + 2: finish this tile's segment when it leaves the tile
             const int cur = tile;
@@ -263,36 +298,42 @@ __global__ void __launch_bounds__(kThreads, 1) k_nf4_gemv(const __grid_constant_
             if (tile != cur || i + 2 >= nu) publish(cur);
         }
     }
-    __syncthreads();
-    // launched programmatically after the T kernel, which it does not read: it only
-    // may not complete before that kernel has (the finish kernel reads both)
-    if (tid == 0) grid_dep_wait();
 }
 
 // Sum of the partial tiles of every (CTA, group) pair that took units of
-// `tile`, in (CTA, group) order, plus s T B^T; CTA = (one 128-row tile, one
-// token), thread = one row n.  Launched programmatically after k_nf4_gemv: it
-// waits for that kernel (and so for the T kernel) first.
+// `tile`, in (CTA, group) order, plus s T B^T; CTA = (one 128-row tile, 8
+// tokens), thread = one row n.  T is first summed over its K splits, in split
+// order, into shared memory (tile 0 also hands the caller its bf16 copy).
+// Launched programmatically after the T kernel: it lets the next kernel on the
+// stream launch, then waits for the T kernel, which completes only after the
+// GEMV has.
+constexpr int kFinTok = 8;
+
 struct FinishArgs {
     const float* slots;
     int64_t M, N;
     int nks, ctas, NT;
     int64_t units;
-    const float* T32;
-    int rp, r;
+    const float* Tpart;        // [kc][M, rp] fp32 split sums of T = X A^T
+    int kc, rp, r;
     const uint16_t* lora_B;
     int b_vec;
     float s;
     uint16_t* Y;
+    uint16_t* T_out;           // [M, r] bf16 copy of T for the caller, or null
 };
 
-__global__ void __launch_bounds__(TR) k_nf4_gemv_finish(FinishArgs a) {
+__global__ void __launch_bounds__(TR, 16) k_nf4_gemv_finish(FinishArgs a) {
+    __shared__ float s_T[kFinTok * 256];  // [kFinTok][r], r <= 256
     __shared__ int s_mask[148];         // groups of CTA c_first + j that took units of this tile
     __shared__ int s_slot[2 * 148];     // their slots, in (CTA, group) order
     __shared__ int s_n;
+    grid_dep_launch();
     grid_dep_wait();
     const int tile = blockIdx.x, row = threadIdx.x;
-    const int64_t m = blockIdx.y;
+    const int r = a.r;
+    const int m0 = blockIdx.y * kFinTok;
+    const int mn = a.M - m0 < kFinTok ? (int)a.M - m0 : kFinTok;
     // unit counts fit 32 bits and CTA * units < 2^32 (units < 2^24, at most 148 CTAs)
     const uint32_t U = (uint32_t)a.units, C = (uint32_t)a.ctas;
     const uint32_t tu0 = (uint32_t)tile * (uint32_t)a.nks, tu1 = tu0 + (uint32_t)a.nks;
@@ -303,6 +344,14 @@ __global__ void __launch_bounds__(TR) k_nf4_gemv_finish(FinishArgs a) {
         const uint32_t b0 = c * U / C, b1 = (c + 1) * U / C;
         const uint32_t lo = b0 > tu0 ? b0 : tu0, hi = b1 < tu1 ? b1 : tu1;
         s_mask[j] = hi - lo >= 2 ? 3 : (hi - lo == 1 ? 1 << ((lo - b0) & 1) : 0);
+    }
+    for (int e = row; e < mn * r; e += TR) {
+        const int mm = e / r, i = e - mm * r;
+        float t = 0.f;
+        for (int z = 0; z < a.kc; ++z) t += a.Tpart[((int64_t)z * a.M + m0 + mm) * a.rp + i];
+        s_T[e] = t;
+        if (tile == 0 && a.T_out != nullptr)
+            a.T_out[(int64_t)(m0 + mm) * r + i] = (uint16_t)(pack_bf16x2(t, 0.f) & 0xffffu);
     }
     __syncthreads();
     if (row == 0) {
@@ -315,26 +364,50 @@ __global__ void __launch_bounds__(TR) k_nf4_gemv_finish(FinishArgs a) {
     __syncthreads();
     const int64_t n = (int64_t)tile * TR + row;
     if (n >= a.N) return;
+    // partial tiles: the loads of one slot for all the CTA's tokens are issued together
+    float v[kFinTok];
+#pragma unroll
+    for (int mm = 0; mm < kFinTok; ++mm) v[mm] = 0.f;
     const int ns = s_n;
-    float v = 0.f;
-    for (int k = 0; k < ns; ++k) v += a.slots[(int64_t)s_slot[k] * (a.NT * TR) + m * TR + row];
-    const uint16_t* br = a.lora_B + n * a.r;
-    const float* tr = a.T32 + m * a.rp;
-    float l = 0.f;
+    for (int k = 0; k < ns; ++k) {
+        const float* sp = a.slots + (int64_t)s_slot[k] * (a.NT * TR) + (int64_t)m0 * TR + row;
+#pragma unroll
+        for (int mm = 0; mm < kFinTok; ++mm)
+            if (mm < mn) v[mm] += sp[mm * TR];
+    }
+    // s T B^T
+    const uint16_t* br = a.lora_B + n * r;
+    float l[kFinTok];
+#pragma unroll
+    for (int mm = 0; mm < kFinTok; ++mm) l[mm] = 0.f;
     if (a.b_vec) {
-        for (int i = 0; i < a.r; i += 8) {
+        for (int i = 0; i < r; i += 8) {
             const uint4 bv = __ldg(reinterpret_cast<const uint4*>(br + i));
             const uint32_t bw[4] = {bv.x, bv.y, bv.z, bv.w};
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                l = __fmaf_rn(tr[i + 2 * j], bf16lo_to_f32(bw[j]), l);
-                l = __fmaf_rn(tr[i + 2 * j + 1], bf16hi_to_f32(bw[j]), l);
+            for (int mm = 0; mm < kFinTok; ++mm) {
+                if (mm < mn) {
+                    const float* tm = s_T + mm * r + i;
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        l[mm] = __fmaf_rn(tm[2 * j], bf16lo_to_f32(bw[j]), l[mm]);
+                        l[mm] = __fmaf_rn(tm[2 * j + 1], bf16hi_to_f32(bw[j]), l[mm]);
+                    }
+                }
             }
         }
     } else {
-        for (int i = 0; i < a.r; ++i) l = __fmaf_rn(tr[i], bf16lo_to_f32(br[i]), l);
+        for (int i = 0; i < r; ++i) {
+            const float b = bf16lo_to_f32(br[i]);
+#pragma unroll
+            for (int mm = 0; mm < kFinTok; ++mm)
+                if (mm < mn) l[mm] = __fmaf_rn(s_T[mm * r + i], b, l[mm]);
+        }
     }
-    a.Y[m * a.N + n] = (uint16_t)(pack_bf16x2(__fmaf_rn(a.s, l, v), 0.f) & 0xffffu);
+#pragma unroll
+    for (int mm = 0; mm < kFinTok; ++mm)
+        if (mm < mn)
+            a.Y[(int64_t)(m0 + mm) * a.N + n] = (uint16_t)(pack_bf16x2(__fmaf_rn(a.s, l[mm], v[mm]), 0.f) & 0xffffu);
 }
 
 }  // namespace gmv

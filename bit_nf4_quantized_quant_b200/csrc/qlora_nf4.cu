@@ -132,7 +132,7 @@ int check_device(int* sm_count) {
                 // which need most of shared memory: keep the SM in its shared-memory-heavy
                 // configuration so that the next kernel's CTAs need no reconfiguration
                 const void* smalls[] = {(const void*)k_lora_down_small<1>, (const void*)k_lora_down_small<2>,
-                                        (const void*)k_lora_down_small<4>, (const void*)k_lora_down_small<8>,
+                                        (const void*)k_lora_down_small<4>, (const void*)gmv::k_nf4_gemv_finish,
                                         (const void*)k_lora_bwd_small, (const void*)k_bwd_small_end};
                 for (const void* f : smalls)
                     if (r == cudaSuccess)
@@ -190,6 +190,7 @@ struct Plan {
     int US;                         // small-path U = dY B: N splits
     int64_t rows_u;                 //   rows of B per split
     int NT;                         // small-path token tile (16 or 32; 8 more for the forward GEMV)
+    int TKC;                        // small-path forward: K splits of T = X A^T
     // byte offsets
     size_t off_slots, off_Upart, off_part, off_T32, off_U32, off_Tp, off_Ubf, off_sT, off_sU, off_Bp, total;
 };
@@ -286,7 +287,8 @@ Plan make_plan(int64_t M, int64_t N, int64_t K, int r, int sms) {
     p.off_slots = take(slots);
     p.off_Upart = take(small ? (size_t)p.US * M * p.rp * 4 : 0);
     p.off_part = take(part);
-    p.off_T32 = take((size_t)M * p.rp * 4);
+    p.TKC = small ? (int)down_splits(K) : 1;
+    p.off_T32 = take((size_t)p.TKC * M * p.rp * 4);
     p.off_U32 = take(big * M * p.rp * 4);
     p.off_Tp = take(big * M * 2 * p.rp * 2);     // T hi | lo
     p.off_Ubf = take(big * M * 2 * p.rp * 2);    // U hi | lo
@@ -514,20 +516,21 @@ int compute_T(const Plan& p, const uint16_t* X, const uint16_t* A, float s, uint
 }
 
 
-// Small-M T = X A^T into T32 (and the caller's bf16 T_out).
-int small_T(const Plan& p, const uint16_t* X, const uint16_t* A, uint16_t* T_out, uint8_t* ws, cudaStream_t st) {
+// Small-M T = X A^T into T32 (and the caller's bf16 T_out): programmatic
+// launch behind the forward GEMV, plain launch in the backward's recompute.
+int small_T(const Plan& p, const uint16_t* X, const uint16_t* A, uint16_t* T_out, uint8_t* ws, cudaStream_t st,
+            bool pdl) {
     LoraDownArgs d{};
     d.X = X; d.A = A; d.M = p.M; d.K = p.K; d.r = p.r; d.rp = p.rp;
+    d.kc = pdl ? p.TKC : 1;             // the forward's split sums are added by the finish kernel
     d.T32 = reinterpret_cast<float*>(ws + p.off_T32);
-    d.T_out = T_out;
-    const int mg = p.M <= 1 ? 1 : p.M <= 2 ? 2 : p.M <= 4 ? 4 : 8;
-    const dim3 grid((unsigned)p.r, (unsigned)cdiv(p.M, mg));
-    switch (mg) {
-        case 1: k_lora_down_small<1><<<grid, kLoraThreads, 0, st>>>(d); break;
-        case 2: k_lora_down_small<2><<<grid, kLoraThreads, 0, st>>>(d); break;
-        case 4: k_lora_down_small<4><<<grid, kLoraThreads, 0, st>>>(d); break;
-        default: k_lora_down_small<8><<<grid, kLoraThreads, 0, st>>>(d); break;
-    }
+    d.T_out = pdl ? nullptr : T_out;
+    const int mg = p.M <= 1 ? 1 : p.M <= 2 ? 2 : 4;
+    const dim3 grid((unsigned)p.r, (unsigned)d.kc, (unsigned)cdiv(p.M, mg)), block(kDownThreads);
+    void (*kern)(LoraDownArgs) = mg == 1 ? k_lora_down_small<1> : mg == 2 ? k_lora_down_small<2>
+                                : k_lora_down_small<4>;
+    if (pdl) return launch_pdl(kern, grid, block, 0, st, d);
+    kern<<<grid, block, 0, st>>>(d);
     note_launch();
     return launch_status();
 }
@@ -561,11 +564,11 @@ int launch_tcs_bwd(const Plan& p, const nf4dq_weight* w, const uint16_t* dY, uin
     return launch_pdl(tcs::k_tcs_gemm<32>, grid, block, tcs::SMEM_ALLOC, st, tmX, tmP, a, tables());
 }
 
-// Small-M forward GEMV (mma.sync, stream-K over one CTA per SM), launched
-// programmatically after the T kernel.
+// Small-M forward: the GEMV (mma.sync, stream-K over one CTA per SM), the
+// T = X A^T kernel and the finish kernel, all launched programmatically.
 template <int NTT>
-int launch_gemv_ntt(const Plan& p, const nf4dq_weight* w, const uint16_t* X, const uint16_t* B, float s, uint16_t* Y,
-                    uint8_t* wsb, int sms, cudaStream_t st) {
+int launch_gemv_ntt(const Plan& p, const nf4dq_weight* w, const uint16_t* X, const uint16_t* A, const uint16_t* B,
+                    float s, uint16_t* Y, uint16_t* T_out, uint8_t* wsb, int sms, cudaStream_t st) {
     using C = gmv::Cfg<NTT>;
     static bool attr_set[64];
     int dev = 0;
@@ -595,28 +598,25 @@ int launch_gemv_ntt(const Plan& p, const nf4dq_weight* w, const uint16_t* X, con
     int rc = launch_pdl(gmv::k_nf4_gemv<NTT>, dim3((unsigned)ctas), dim3(gmv::kThreads), (size_t)C::SMEM_ALLOC, st,
                         tmP, a, tables());
     if (rc != QLORA_OK) return rc;
+    rc = small_T(p, X, A, nullptr, wsb, st, true);
+    if (rc != QLORA_OK) return rc;
     gmv::FinishArgs f{};
     f.slots = a.slots; f.M = p.M; f.N = N; f.nks = a.nks; f.ctas = a.ctas; f.NT = C::NT; f.units = a.units;
-    f.T32 = reinterpret_cast<const float*>(wsb + p.off_T32); f.rp = p.rp; f.r = p.r;
-    f.lora_B = B; f.b_vec = (p.r % 8 == 0 && aligned16(B)) ? 1 : 0; f.s = s; f.Y = Y;
-    return launch_pdl(gmv::k_nf4_gemv_finish, dim3((unsigned)a.tiles, (unsigned)p.M), dim3(gmv::TR), 0, st, f);
+    f.Tpart = reinterpret_cast<const float*>(wsb + p.off_T32); f.kc = p.TKC; f.rp = p.rp; f.r = p.r;
+    f.lora_B = B; f.b_vec = (p.r % 8 == 0 && aligned16(B)) ? 1 : 0; f.s = s; f.Y = Y; f.T_out = T_out;
+    return launch_pdl(gmv::k_nf4_gemv_finish, dim3((unsigned)a.tiles, (unsigned)cdiv(p.M, gmv::kFinTok)),
+                      dim3(gmv::TR), 0, st, f);
 }
 
-int launch_gemv(const Plan& p, const nf4dq_weight* w, const uint16_t* X, const uint16_t* B, float s, uint16_t* Y,
-                uint8_t* wsb, int sms, cudaStream_t st) {
-    if (p.M <= 8) return launch_gemv_ntt<1>(p, w, X, B, s, Y, wsb, sms, st);
-    if (p.M <= 16) return launch_gemv_ntt<2>(p, w, X, B, s, Y, wsb, sms, st);
-    return launch_gemv_ntt<4>(p, w, X, B, s, Y, wsb, sms, st);
-}
-
-// Small-M forward: T = X A^T, then the fused GEMV, which overlaps the T
-// kernel and adds s T B^T when it finishes a tile.
+// Small-M forward: fused GEMV, T = X A^T beside it, then the finish kernel
+// (partial tiles summed, s T B^T added).
 int small_fwd(const Plan& p, const uint16_t* X, const nf4dq_weight* w, const uint16_t* A, const uint16_t* B,
               float scaling, uint16_t* Y, uint16_t* T_out, uint8_t* wsb, int sms, cudaStream_t st) {
     hook_before(st);
-    int rc = small_T(p, X, A, T_out, wsb, st);
-    if (rc != QLORA_OK) return rc;
-    rc = launch_gemv(p, w, X, B, scaling, Y, wsb, sms, st);
+    int rc;
+    if (p.M <= 8) rc = launch_gemv_ntt<1>(p, w, X, A, B, scaling, Y, T_out, wsb, sms, st);
+    else if (p.M <= 16) rc = launch_gemv_ntt<2>(p, w, X, A, B, scaling, Y, T_out, wsb, sms, st);
+    else rc = launch_gemv_ntt<4>(p, w, X, A, B, scaling, Y, T_out, wsb, sms, st);
     hook_after(st);
     return rc;
 }
@@ -629,7 +629,7 @@ int small_bwd(const Plan& p, const uint16_t* X, const uint16_t* dY, const nf4dq_
     int rc = QLORA_OK;
     const float* T32 = nullptr;
     if (T == nullptr) {
-        rc = small_T(p, X, A, nullptr, wsb, st);
+        rc = small_T(p, X, A, nullptr, wsb, st, false);
         if (rc != QLORA_OK) return rc;
         T32 = reinterpret_cast<const float*>(wsb + p.off_T32);
     }
@@ -703,9 +703,9 @@ int nf4_dequant(const nf4dq_weight* w, qlora_bf16* W_out, qlora_stream_t stream)
     int sms = 0;
     rc = check_device(&sms);
     if (rc != QLORA_OK) return rc;
-    const int64_t nchunks = w->N * w->K / 32;
-    k_dequant<<<grid_for(nchunks, 256, sms), 256, 0, (cudaStream_t)stream>>>(w->packed, w->codes, w->scale, w->mean,
-                                                                            nchunks, W_out, tables());
+    const int64_t nwords = w->N * w->K / 8;                    // 8 weights per packed 32-bit word
+    k_dequant<<<grid_for(nwords, 8 * kDqWarpWords, sms, 4), 256, 0, (cudaStream_t)stream>>>(
+        w->packed, w->codes, w->scale, w->mean, nwords, W_out, tables());
     note_launch();
     return launch_status();
 }

@@ -45,7 +45,7 @@ __device__ __noinline__ uint32_t nf4_encode_exact(float w, float c, float m3, fl
 // quantization with the fp64 pairwise tree held in registers: lane l keeps
 // slots l, l+32, ..., l+224, so strides 128, 64, 32 are in-register adds and
 // strides 16..1 are shuffles -- the same association order as the definition.
-__global__ void __launch_bounds__(256) k_quantize_dq(const uint16_t* __restrict__ W, int64_t nblocks,
+__global__ void __launch_bounds__(256, 4) k_quantize_dq(const uint16_t* __restrict__ W, int64_t nblocks,
                                                      uint8_t* __restrict__ packed, int8_t* __restrict__ codes,
                                                      float* __restrict__ scale, float* __restrict__ mean,
                                                      NF4Tables tab, const __grid_constant__ EncTables enc) {
@@ -96,23 +96,29 @@ __global__ void __launch_bounds__(256) k_quantize_dq(const uint16_t* __restrict_
                 // reciprocal that is not finite, NaN) the exact quotient takes the 4-step search.
                 const float rcp = __frcp_rn(c);
                 const bool fast_blk = c > 0.f && rcp < INFINITY;
-                uint32_t word = 0;
+                uint32_t word = 0, slow = fast_blk ? 0u : 0xffu;
 #pragma unroll
                 for (int j = 0; j < 8; ++j) {
-                    uint32_t q = 7u;
-                    bool slow = !fast_blk;
-                    if (fast_blk) {
-                        const float x = __fmul_rn(w[j], rcp);
-                        // round(64 x + 64) from the low bits of 64 x + 64 + 1.5 * 2^23
-                        const uint32_t b = min(__float_as_uint(__fmaf_rn(x, 64.f, 12582976.f)) - 0x4B400000u, 128u);
-                        const float2 e = s_enc[b];
-                        const float d = __fsub_rn(x, e.x);
-                        slow = !(fabsf(d) > 9.5367431640625e-07f);     // 2^-20 (also NaN)
-                        q = __float_as_uint(e.y) + (d > 0.f ? 1u : 0u);
-                    }
-                    if (slow) q = nf4_encode_exact(w[j], c, tab.m[3], tab.m[7], tab.m[11], s_m);
+                    const float x = __fmul_rn(w[j], rcp);
+                    // round(64 x + 64) from the low bits of 64 x + 64 + 1.5 * 2^23
+                    const uint32_t b = min(__float_as_uint(__fmaf_rn(x, 64.f, 12582976.f)) - 0x4B400000u, 128u);
+                    const float2 e = s_enc[b];
+                    const float d = __fsub_rn(x, e.x);
+                    if (!(fabsf(d) > 9.5367431640625e-07f)) slow |= 1u << j;     // 2^-20 (also NaN)
+                    const uint32_t q = __float_as_uint(e.y) + (d > 0.f ? 1u : 0u);
                     // element 2i -> high nibble of byte i (little-endian word)
                     word |= q << ((j >> 1) * 8 + ((j & 1) ? 0 : 4));
+                }
+                // rare: weights near a threshold (or a block the fast path cannot take)
+                if (slow) {
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) {
+                        if ((slow >> j) & 1u) {
+                            const int sh = (j >> 1) * 8 + ((j & 1) ? 0 : 4);
+                            const uint32_t q = nf4_encode_exact(w[j], c, tab.m[3], tab.m[7], tab.m[11], s_m);
+                            word = (word & ~(15u << sh)) | (q << sh);
+                        }
+                    }
                 }
                 *reinterpret_cast<uint32_t*>(packed + ((b0 + bl) * kBlock + part * 8) / 2) = word;
                 if (part == 0) s_c[bl] = c;
@@ -170,38 +176,58 @@ __global__ void __launch_bounds__(256) k_quantize_dq(const uint16_t* __restrict_
     }
 }
 
-// Dense dequantization: one thread per 16 packed bytes (32 weights = half a
-// block), grid-stride.  W' = bf16_rne(L[q] * c'_b), c'_b = fmaf(code, scale, mean).
+// Dense dequantization, coalesced on both sides: a warp takes a segment of
+// 256 packed 32-bit words (2048 weights) per iteration, lane l the words
+// l + 32 k (k = 0..7), so each of its eight 4-byte loads and eight 16-byte
+// stores (8 weights of word w go to bytes [16 w, 16 w + 16) of the output)
+// covers one contiguous stretch across the warp; all loads of a segment are
+// issued before the first store.  W' = bf16_rne(L[q] * c'_b),
+// c'_b = fmaf(code_b, scale_g, mean_g).
+constexpr int kDqWarpWords = 256;
+
 __global__ void __launch_bounds__(256) k_dequant(const uint8_t* __restrict__ packed,
                                                  const int8_t* __restrict__ codes,
                                                  const float* __restrict__ scale, const float* __restrict__ mean,
-                                                 int64_t nchunks, uint16_t* __restrict__ out, NF4Tables tab) {
+                                                 int64_t nwords, uint16_t* __restrict__ out, NF4Tables tab) {
     __shared__ float s_L[16];
     if (threadIdx.x < 16) s_L[threadIdx.x] = tab.L[threadIdx.x];
     __syncthreads();
-    for (int64_t ch = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; ch < nchunks;
-         ch += (int64_t)gridDim.x * blockDim.x) {
-        const uint4 p = ldg_nc_v4(packed + ch * 16);
-        const int64_t b = ch >> 1;
-        const int64_t g = b / kGroup;
-        const float cp = __fmaf_rn((float)codes[b], __ldg(scale + g), __ldg(mean + g));
-        const uint32_t pw[4] = {p.x, p.y, p.z, p.w};
-        uint32_t o[16];
+    const int lane = threadIdx.x & 31;
+    const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
+    const uint32_t* pw = reinterpret_cast<const uint32_t*>(packed);
+    for (int64_t seg = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5; seg * kDqWarpWords < nwords;
+         seg += nwarps) {
+        const int64_t w0 = seg * kDqWarpWords + lane;
+        uint32_t v[8];
+        int cd[8];
+        float sc[8], mn[8];
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                const uint32_t byte = (pw[j] >> (8 * k)) & 0xffu;
-                const float hi = __fmul_rn(s_L[byte >> 4], cp);     // element 2i
-                const float lo = __fmul_rn(s_L[byte & 15u], cp);    // element 2i+1
-                o[j * 4 + k] = pack_bf16x2(hi, lo);
+        for (int k = 0; k < 8; ++k) {
+            const int64_t wi = w0 + 32 * k;                 // 8 weights: block wi / 8, group wi / 2048
+            v[k] = 0u; cd[k] = 0; sc[k] = 0.f; mn[k] = 0.f;
+            if (wi < nwords) {
+                v[k] = ldg_nc_u32(pw + wi);
+                cd[k] = __ldg(codes + (wi >> 3));
+                sc[k] = __ldg(scale + (wi >> 11));
+                mn[k] = __ldg(mean + (wi >> 11));
             }
         }
-        uint4* dst = reinterpret_cast<uint4*>(out + ch * 32);
-        dst[0] = make_uint4(o[0], o[1], o[2], o[3]);
-        dst[1] = make_uint4(o[4], o[5], o[6], o[7]);
-        dst[2] = make_uint4(o[8], o[9], o[10], o[11]);
-        dst[3] = make_uint4(o[12], o[13], o[14], o[15]);
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+            const int64_t wi = w0 + 32 * k;
+            if (wi < nwords) {
+                const float cp = __fmaf_rn((float)cd[k], sc[k], mn[k]);
+                uint32_t o[4];
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const uint32_t byte = (v[k] >> (8 * j)) & 0xffu;
+                    const float hi = __fmul_rn(s_L[byte >> 4], cp);     // element 2j
+                    const float lo = __fmul_rn(s_L[byte & 15u], cp);    // element 2j+1
+                    o[j] = pack_bf16x2(hi, lo);
+                }
+                *reinterpret_cast<uint4*>(out + wi * 8) = make_uint4(o[0], o[1], o[2], o[3]);
+            }
+        }
     }
 }
 

@@ -1,6 +1,6 @@
 // small_lora.cuh -- the LoRA adapter products of the small-M path (M <= 32
-// tokens), written so that a decode-sized forward is two launches and the
-// backward three (four when T is recomputed):
+// tokens).  A decode-sized forward is three launches (fused GEMV, T, finish)
+// and the backward three (four when T is recomputed):
 //
 //   k_lora_down_small  T = X A^T over the whole K (one CTA per rank column
 //                      and token group; no cross-CTA reduction)
@@ -31,9 +31,13 @@ struct LoraDownArgs {
     const uint16_t* A;       // [r, K] bf16, 16-byte aligned
     int64_t M, K;            // K % 64 == 0
     int r, rp;
-    float* T32;              // [M, rp] fp32 (columns >= r not written)
-    uint16_t* T_out;         // [M, r] bf16 copy for the caller, or null
+    int kc;                  // K splits: split z sums the 8-wide chunks [z nch / kc, (z + 1) nch / kc)
+    float* T32;              // [kc][M, rp] fp32 partial sums (columns >= r not written)
+    uint16_t* T_out;         // [M, r] bf16 copy for the caller (kc == 1 only), or null
 };
+
+// K splits of the forward's T: about two 8-wide chunks per thread and split.
+inline int64_t down_splits(int64_t K) { return (K / 8 + 255) / 256; }
 
 __device__ __forceinline__ float dot8_bf16(const uint4& x, const uint4& y, float v) {
     const uint32_t xw[4] = {x.x, x.y, x.z, x.w}, yw[4] = {y.x, y.y, y.z, y.w};
@@ -45,31 +49,38 @@ __device__ __forceinline__ float dot8_bf16(const uint4& x, const uint4& y, float
     return v;
 }
 
-// CTA (i, mg) computes T[mg MG .. mg MG + MG, i]; thread t takes the 8-wide K
-// chunks t, t + 256, ...; fixed-order warp and block reductions.  It lets the
-// next kernel (launched with programmatic serialization) start at once.
+// CTA (i, z, mg) computes split z of T[mg MG .. mg MG + MG, i]; thread t takes
+// the split's 8-wide K chunks t, t + 128, ...; fixed-order warp and block
+// reductions.  Small enough (128 threads, at most 32 registers) to run beside
+// a fused GEMV CTA on its SM.  In the forward it is launched programmatically
+// right behind the GEMV, which releases it only once the kernel ahead of the
+// GEMV (the writer of X) has completed, so X is read at once, through L2; it
+// lets the finish kernel launch at once, and its first CTA waits for the
+// GEMV before it ends, so that this grid's completion implies the GEMV's
+// (the other CTAs exit as soon as their sums are written).  Launched plainly
+// (the backward's recompute, one split) the wait returns at once.
+constexpr int kDownThreads = 128;
+
 template <int MG>
-__global__ void __launch_bounds__(kLoraThreads) k_lora_down_small(LoraDownArgs a) {
+__global__ void __launch_bounds__(kDownThreads, 16) k_lora_down_small(LoraDownArgs a) {
     grid_dep_launch();
-    __shared__ float s_red[kLoraThreads / 32][MG];
+    __shared__ float s_red[kDownThreads / 32][MG];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int i = blockIdx.x;
-    const int64_t m0 = (int64_t)blockIdx.y * MG;
+    const int i = blockIdx.x, z = blockIdx.y;
+    const int64_t m0 = (int64_t)blockIdx.z * MG;
+    const int64_t nch = a.K / 8;
+    const int64_t c0 = z * nch / a.kc, c1 = (z + 1) * nch / a.kc;
     const uint4* ar = reinterpret_cast<const uint4*>(a.A + (int64_t)i * a.K);
-    const uint4* xr[MG];
-#pragma unroll
-    for (int mm = 0; mm < MG; ++mm) {
-        const int64_t m = m0 + mm < a.M ? m0 + mm : a.M - 1;
-        xr[mm] = reinterpret_cast<const uint4*>(a.X + m * a.K);
-    }
+    const uint4* xr = reinterpret_cast<const uint4*>(a.X + m0 * a.K);
+    const int mn = a.M - m0 < MG ? (int)(a.M - m0) : MG;
     float acc[MG];
 #pragma unroll
     for (int mm = 0; mm < MG; ++mm) acc[mm] = 0.f;
-    const int64_t nch = a.K / 8;
-    for (int64_t c = tid; c < nch; c += kLoraThreads) {
-        const uint4 av = ldg_nc_v4(ar + c);
+    for (int64_t c = c0 + tid; c < c1; c += kDownThreads) {
+        const uint4 av = ldg_cg_v4(ar + c);
 #pragma unroll
-        for (int mm = 0; mm < MG; ++mm) acc[mm] = dot8_bf16(ldg_nc_v4(xr[mm] + c), av, acc[mm]);
+        for (int mm = 0; mm < MG; ++mm)
+            if (mm < mn) acc[mm] = dot8_bf16(ldg_cg_v4(xr + mm * nch + c), av, acc[mm]);
     }
 #pragma unroll
     for (int mm = 0; mm < MG; ++mm) {
@@ -79,14 +90,15 @@ __global__ void __launch_bounds__(kLoraThreads) k_lora_down_small(LoraDownArgs a
         if (lane == 0) s_red[warp][mm] = v;
     }
     __syncthreads();
-    if (tid < MG && m0 + tid < a.M) {
+    if (tid < mn) {
         float v = 0.f;
 #pragma unroll
-        for (int w = 0; w < kLoraThreads / 32; ++w) v += s_red[w][tid];
+        for (int w = 0; w < kDownThreads / 32; ++w) v += s_red[w][tid];
         const int64_t m = m0 + tid;
-        a.T32[m * a.rp + i] = v;
+        a.T32[((int64_t)z * a.M + m) * a.rp + i] = v;
         if (a.T_out != nullptr) a.T_out[m * a.r + i] = (uint16_t)(pack_bf16x2(v, 0.f) & 0xffffu);
     }
+    if (blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0) grid_dep_wait();
 }
 
 // ---------------------------------------------------------------------------
@@ -263,11 +275,13 @@ __device__ __forceinline__ uint32_t end_unit_owner(uint32_t u, uint32_t U, uint3
 }
 
 // grid (ceil(K / 256), M + r): row y < M writes dX[y, :], row M + i writes dA[i, :].
-// Launched programmatically after k_tcs_gemm: it waits for that kernel (and so
-// for the U / dB kernel before it) first.
+// Launched programmatically after k_tcs_gemm: it lets the next kernel on the
+// stream launch, then waits for that kernel (and so for the U / dB kernel
+// before it).
 __global__ void __launch_bounds__(kLoraThreads) k_bwd_small_end(BwdEndArgs a) {
     __shared__ float s_q[kLoraThreads];
     __shared__ float s_u[kLoraThreads];
+    grid_dep_launch();
     grid_dep_wait();
     const int tid = threadIdx.x;
     const int y = blockIdx.y;
