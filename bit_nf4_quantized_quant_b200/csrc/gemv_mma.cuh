@@ -33,9 +33,9 @@
 //    small T = X A^T kernel (which runs beside it on the SMs' spare registers
 //    and ends only after it), then the finish kernel.  Before it waits for
 //    the kernel ahead of it on the stream, the GEMV only sets up its barriers
-//    and warms L2 with its first packed tiles (an L2 prefetch cannot return
-//    stale data: L2 is the point of coherence); everything it reads is read
-//    after the wait, and it releases the T kernel right after it.
+//    and warms L2 with each group's first packed tile (an L2 prefetch cannot
+//    return stale data: L2 is the point of coherence); everything it reads is
+//    read after the wait, and it releases the T kernel right after it.
 #pragma once
 #include <cuda.h>
 #include "common.cuh"
@@ -155,13 +155,9 @@ __global__ void __launch_bounds__(kThreads, 1) k_nf4_gemv(const __grid_constant_
         const int nq = nu > grp ? (nu - grp + 1) / 2 : 0;
         int tile = tile0, ks = ks0;
         unit_advance(tile, ks, grp, nks);
-        if (lane == 0) {            // warm L2 with the group's first packed tiles
-            int pt = tile, pk = ks;
-            for (int q = 0; q < nq && q < 2 * SPG; ++q) {
-                tma_prefetch_l2(&tmP, pk * (KSTEP / 2), pt * TR);
-                unit_advance(pt, pk, 2, nks);
-            }
-        }
+        // warm L2 with the group's first packed tile only: every CTA's first tile is then
+        // at the front of the memory queue (the rest streams through the stage ring)
+        if (lane == 0 && nq > 0) tma_prefetch_l2(&tmP, ks * (KSTEP / 2), tile * TR);
         grid_dep_wait();
         // X is complete: the T kernel launched behind this one may start (and read it)
         if (grp == 0 && lane == 0) grid_dep_launch();
@@ -301,14 +297,13 @@ __global__ void __launch_bounds__(kThreads, 1) k_nf4_gemv(const __grid_constant_
 }
 
 // Sum of the partial tiles of every (CTA, group) pair that took units of
-// `tile`, in (CTA, group) order, plus s T B^T; CTA = (one 128-row tile, 8
-// tokens), thread = one row n.  T is first summed over its K splits, in split
+// `tile`, in (CTA, group) order, plus s T B^T; CTA = (one 128-row tile, MT
+// tokens), thread = one row n.  T is summed over its K splits, in split
 // order, into shared memory (tile 0 also hands the caller its bf16 copy).
 // Launched programmatically after the T kernel: it lets the next kernel on the
 // stream launch, then waits for the T kernel, which completes only after the
-// GEMV has.
-constexpr int kFinTok = 8;
-
+// GEMV has.  After the wait, the partial-tile, B-row and T loads are all
+// issued before the first of them is used (one round trip to L2).
 struct FinishArgs {
     const float* slots;
     int64_t M, N;
@@ -323,17 +318,24 @@ struct FinishArgs {
     uint16_t* T_out;           // [M, r] bf16 copy of T for the caller, or null
 };
 
-__global__ void __launch_bounds__(TR, 16) k_nf4_gemv_finish(FinishArgs a) {
-    __shared__ float s_T[kFinTok * 256];  // [kFinTok][r], r <= 256
+constexpr int kFinSlots = 4;   // partial tiles loaded per batch
+constexpr int kFinB = 4;       // 8-wide chunks of the B row held in registers (r <= 32)
+
+template <int MT>
+__global__ void __launch_bounds__(TR, 8) k_nf4_gemv_finish(FinishArgs a) {
+    __shared__ float s_T[MT * 256];     // [MT][r], r <= 256
     __shared__ int s_mask[148];         // groups of CTA c_first + j that took units of this tile
     __shared__ int s_slot[2 * 148];     // their slots, in (CTA, group) order
     __shared__ int s_n;
     grid_dep_launch();
-    grid_dep_wait();
     const int tile = blockIdx.x, row = threadIdx.x;
     const int r = a.r;
-    const int m0 = blockIdx.y * kFinTok;
-    const int mn = a.M - m0 < kFinTok ? (int)a.M - m0 : kFinTok;
+    const int m0 = blockIdx.y * MT;
+    const int mn = a.M - m0 < MT ? (int)a.M - m0 : MT;
+    const int64_t n = (int64_t)tile * TR + row;
+    const bool live = n < a.N;
+    // Before the wait: what depends on the split only (integer arithmetic), and an
+    // L2 prefetch of this row of B.
     // unit counts fit 32 bits and CTA * units < 2^32 (units < 2^24, at most 148 CTAs)
     const uint32_t U = (uint32_t)a.units, C = (uint32_t)a.ctas;
     const uint32_t tu0 = (uint32_t)tile * (uint32_t)a.nks, tu1 = tu0 + (uint32_t)a.nks;
@@ -345,14 +347,8 @@ __global__ void __launch_bounds__(TR, 16) k_nf4_gemv_finish(FinishArgs a) {
         const uint32_t lo = b0 > tu0 ? b0 : tu0, hi = b1 < tu1 ? b1 : tu1;
         s_mask[j] = hi - lo >= 2 ? 3 : (hi - lo == 1 ? 1 << ((lo - b0) & 1) : 0);
     }
-    for (int e = row; e < mn * r; e += TR) {
-        const int mm = e / r, i = e - mm * r;
-        float t = 0.f;
-        for (int z = 0; z < a.kc; ++z) t += a.Tpart[((int64_t)z * a.M + m0 + mm) * a.rp + i];
-        s_T[e] = t;
-        if (tile == 0 && a.T_out != nullptr)
-            a.T_out[(int64_t)(m0 + mm) * r + i] = (uint16_t)(pack_bf16x2(t, 0.f) & 0xffffu);
-    }
+    const uint16_t* br = a.lora_B + (live ? n : 0) * r;
+    if (live) asm volatile("prefetch.global.L2 [%0];" ::"l"(br));
     __syncthreads();
     if (row == 0) {
         int k = 0;
@@ -362,50 +358,88 @@ __global__ void __launch_bounds__(TR, 16) k_nf4_gemv_finish(FinishArgs a) {
         s_n = k;
     }
     __syncthreads();
-    const int64_t n = (int64_t)tile * TR + row;
-    if (n >= a.N) return;
-    // partial tiles: the loads of one slot for all the CTA's tokens are issued together
-    float v[kFinTok];
-#pragma unroll
-    for (int mm = 0; mm < kFinTok; ++mm) v[mm] = 0.f;
     const int ns = s_n;
-    for (int k = 0; k < ns; ++k) {
-        const float* sp = a.slots + (int64_t)s_slot[k] * (a.NT * TR) + (int64_t)m0 * TR + row;
+    grid_dep_wait();
+
+    // partial tiles, kFinSlots at a time, summed in slot order
+    float v[MT];
 #pragma unroll
-        for (int mm = 0; mm < kFinTok; ++mm)
-            if (mm < mn) v[mm] += sp[mm * TR];
+    for (int mm = 0; mm < MT; ++mm) v[mm] = 0.f;
+    const bool bregs = live && a.b_vec && r <= 8 * kFinB;
+    uint4 bq[kFinB];
+    if (live) {
+        for (int k0 = 0; k0 < ns; k0 += kFinSlots) {
+            float t[kFinSlots][MT];
+#pragma unroll
+            for (int k = 0; k < kFinSlots; ++k) {
+                const float* sp = a.slots + (int64_t)s_slot[k0 + k < ns ? k0 + k : k0] * (a.NT * TR) +
+                                  (int64_t)m0 * TR + row;
+#pragma unroll
+                for (int mm = 0; mm < MT; ++mm) t[k][mm] = (k0 + k < ns && mm < mn) ? sp[mm * TR] : 0.f;
+            }
+            if (k0 == 0 && bregs) {
+#pragma unroll
+                for (int c = 0; c < kFinB; ++c) bq[c] = 8 * c < r ? ldg_cg_v4(br + 8 * c) : make_uint4(0, 0, 0, 0);
+            }
+#pragma unroll
+            for (int k = 0; k < kFinSlots; ++k)
+#pragma unroll
+                for (int mm = 0; mm < MT; ++mm)
+                    if (k0 + k < ns) v[mm] += t[k][mm];
+        }
     }
+    // T over its K splits, in split order
+    for (int e = row; e < mn * r; e += TR) {
+        const int mm = e / r, i = e - mm * r;
+        const float* tp = a.Tpart + ((int64_t)m0 + mm) * a.rp + i;
+        const int64_t zs = a.M * a.rp;
+        float t = 0.f;
+        int z = 0;
+        for (; z + 4 <= a.kc; z += 4) {
+            const float t0 = tp[z * zs], t1 = tp[(z + 1) * zs], t2 = tp[(z + 2) * zs], t3 = tp[(z + 3) * zs];
+            t += t0; t += t1; t += t2; t += t3;
+        }
+        for (; z < a.kc; ++z) t += tp[z * zs];
+        s_T[e] = t;
+        if (tile == 0 && a.T_out != nullptr)
+            a.T_out[(int64_t)(m0 + mm) * r + i] = (uint16_t)(pack_bf16x2(t, 0.f) & 0xffffu);
+    }
+    __syncthreads();
+    if (!live) return;
     // s T B^T
-    const uint16_t* br = a.lora_B + n * r;
-    float l[kFinTok];
+    float l[MT];
 #pragma unroll
-    for (int mm = 0; mm < kFinTok; ++mm) l[mm] = 0.f;
-    if (a.b_vec) {
-        for (int i = 0; i < r; i += 8) {
-            const uint4 bv = __ldg(reinterpret_cast<const uint4*>(br + i));
-            const uint32_t bw[4] = {bv.x, bv.y, bv.z, bv.w};
+    for (int mm = 0; mm < MT; ++mm) l[mm] = 0.f;
+    auto chunk = [&](const uint4& bv, int i) {
+        const uint32_t bw[4] = {bv.x, bv.y, bv.z, bv.w};
 #pragma unroll
-            for (int mm = 0; mm < kFinTok; ++mm) {
-                if (mm < mn) {
-                    const float* tm = s_T + mm * r + i;
+        for (int mm = 0; mm < MT; ++mm) {
+            if (mm < mn) {
+                const float* tm = s_T + mm * r + i;
 #pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        l[mm] = __fmaf_rn(tm[2 * j], bf16lo_to_f32(bw[j]), l[mm]);
-                        l[mm] = __fmaf_rn(tm[2 * j + 1], bf16hi_to_f32(bw[j]), l[mm]);
-                    }
+                for (int j = 0; j < 4; ++j) {
+                    l[mm] = __fmaf_rn(tm[2 * j], bf16lo_to_f32(bw[j]), l[mm]);
+                    l[mm] = __fmaf_rn(tm[2 * j + 1], bf16hi_to_f32(bw[j]), l[mm]);
                 }
             }
         }
+    };
+    if (bregs) {
+#pragma unroll
+        for (int c = 0; c < kFinB; ++c)
+            if (8 * c < r) chunk(bq[c], 8 * c);
+    } else if (a.b_vec) {
+        for (int i = 0; i < r; i += 8) chunk(ldg_cg_v4(br + i), i);
     } else {
         for (int i = 0; i < r; ++i) {
             const float b = bf16lo_to_f32(br[i]);
 #pragma unroll
-            for (int mm = 0; mm < kFinTok; ++mm)
+            for (int mm = 0; mm < MT; ++mm)
                 if (mm < mn) l[mm] = __fmaf_rn(s_T[mm * r + i], b, l[mm]);
         }
     }
 #pragma unroll
-    for (int mm = 0; mm < kFinTok; ++mm)
+    for (int mm = 0; mm < MT; ++mm)
         if (mm < mn)
             a.Y[(int64_t)(m0 + mm) * a.N + n] = (uint16_t)(pack_bf16x2(__fmaf_rn(a.s, l[mm], v[mm]), 0.f) & 0xffffu);
 }

@@ -132,7 +132,9 @@ int check_device(int* sm_count) {
                 // which need most of shared memory: keep the SM in its shared-memory-heavy
                 // configuration so that the next kernel's CTAs need no reconfiguration
                 const void* smalls[] = {(const void*)k_lora_down_small<1>, (const void*)k_lora_down_small<2>,
-                                        (const void*)k_lora_down_small<4>, (const void*)gmv::k_nf4_gemv_finish,
+                                        (const void*)k_lora_down_small<4>, (const void*)gmv::k_nf4_gemv_finish<1>,
+                                        (const void*)gmv::k_nf4_gemv_finish<2>, (const void*)gmv::k_nf4_gemv_finish<4>,
+                                        (const void*)gmv::k_nf4_gemv_finish<8>,
                                         (const void*)k_lora_bwd_small, (const void*)k_bwd_small_end};
                 for (const void* f : smalls)
                     if (r == cudaSuccess)
@@ -575,8 +577,12 @@ int launch_gemv_ntt(const Plan& p, const nf4dq_weight* w, const uint16_t* X, con
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return QLORA_ERR_DEVICE;
     if (!attr_set[dev]) {
         std::lock_guard<std::mutex> lk(g_tc_mu);
+        // the same (shared-memory-heavy) carveout as the small kernels launched beside it,
+        // so that their CTAs can share its SMs
         if (cudaFuncSetAttribute(gmv::k_nf4_gemv<NTT>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_ALLOC) !=
-            cudaSuccess)
+                cudaSuccess ||
+            cudaFuncSetAttribute(gmv::k_nf4_gemv<NTT>, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                 (int)cudaSharedmemCarveoutMaxShared) != cudaSuccess)
             return QLORA_ERR_LAUNCH;
         attr_set[dev] = true;
     }
@@ -604,8 +610,10 @@ int launch_gemv_ntt(const Plan& p, const nf4dq_weight* w, const uint16_t* X, con
     f.slots = a.slots; f.M = p.M; f.N = N; f.nks = a.nks; f.ctas = a.ctas; f.NT = C::NT; f.units = a.units;
     f.Tpart = reinterpret_cast<const float*>(wsb + p.off_T32); f.kc = p.TKC; f.rp = p.rp; f.r = p.r;
     f.lora_B = B; f.b_vec = (p.r % 8 == 0 && aligned16(B)) ? 1 : 0; f.s = s; f.Y = Y; f.T_out = T_out;
-    return launch_pdl(gmv::k_nf4_gemv_finish, dim3((unsigned)a.tiles, (unsigned)cdiv(p.M, gmv::kFinTok)),
-                      dim3(gmv::TR), 0, st, f);
+    const int mt = p.M <= 1 ? 1 : p.M <= 2 ? 2 : p.M <= 4 ? 4 : 8;
+    void (*fin)(gmv::FinishArgs) = mt == 1 ? gmv::k_nf4_gemv_finish<1> : mt == 2 ? gmv::k_nf4_gemv_finish<2>
+                                 : mt == 4 ? gmv::k_nf4_gemv_finish<4> : gmv::k_nf4_gemv_finish<8>;
+    return launch_pdl(fin, dim3((unsigned)a.tiles, (unsigned)cdiv(p.M, mt)), dim3(gmv::TR), 0, st, f);
 }
 
 // Small-M forward: fused GEMV, T = X A^T beside it, then the finish kernel
