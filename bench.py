@@ -37,14 +37,14 @@ if ROOT not in sys.path:
 METRIC = "QLoRA linear fwd+bwd TFLOP/s & NF4 weight-stream GB/s; % of roofline, 1×B200"
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
-# dram__bytes_read.sum + dram__bytes_write.sum per launch of the fused
-# dequant-GEMM, from an ncu capture (see profiles/), keyed by the hash of the
-# CUDA sources it was taken on; null once the kernel sources change.
 # dram__bytes_read.sum + dram__bytes_write.sum of the dominant kernel, averaged over its launches
-# in one timed step (ncu --metrics ... --nvtx-include "timed/" python bench.py --steps 1 ...), and the
-# hash of the kernel sources it was taken on (a later source change makes the figure stale: null)
+# in one timed step (ncu --metrics ... --nvtx-include "timed/" python bench.py --steps 1 ..., see
+# profiles/), and the hash of the kernel sources it was taken on (a later source change makes the
+# figure stale: null)
 TRAFFIC = {
-    "workload3_M2048": {"bytes_per_launch": 41907931, "src": "802eb498c217"},
+    "workload3_M2048": {"bytes_per_launch": 41658990, "src": "dc43a81efa36"},
+    # small M: one forward chain (GEMV + T + finish) per projection
+    "workload2_M1": {"bytes_per_launch": 24058752, "src": "dc43a81efa36"},
 }
 
 

@@ -41,7 +41,6 @@
 #include "common.cuh"
 #include "nf4_decode.cuh"
 #include "tc_gemm.cuh"
-#include "small_lora.cuh"
 
 namespace qnf4 {
 namespace gmv {
