@@ -39,19 +39,21 @@ PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 
 # dram__bytes_read.sum + dram__bytes_write.sum of the dominant kernel, averaged over its launches
 # in one timed step (ncu --metrics ... --nvtx-include "timed/" python bench.py --steps 1 ..., see
-# profiles/), and the hash of the kernel sources it was taken on (a later source change makes the
-# figure stale: null)
+# profiles/), with the hash of the sources that define those kernels and their launches when the
+# counters were taken (a later change to any of them makes the figure stale: null)
+_PAIR_SRC = ("common.cuh", "nf4_decode.cuh", "tc_gemm.cuh", "tc2_gemm.cuh", "qlora_nf4.cu")
+_GEMV_SRC = ("common.cuh", "nf4_decode.cuh", "tc_gemm.cuh", "gemv_mma.cuh", "small_lora.cuh", "qlora_nf4.cu")
 TRAFFIC = {
-    "workload3_M2048": {"bytes_per_launch": 41658990, "src": "dc43a81efa36"},
+    "workload3_M2048": {"bytes_per_launch": 41658990, "files": _PAIR_SRC, "src": "bea19313b8e6"},
     # small M: one forward chain (GEMV + T + finish) per projection
-    "workload2_M1": {"bytes_per_launch": 24058752, "src": "dc43a81efa36"},
+    "workload2_M1": {"bytes_per_launch": 24058752, "files": _GEMV_SRC, "src": "77fe13572d82"},
 }
 
 
-def src_hash() -> str:
+def src_hash(files=None) -> str:
     h = hashlib.sha1()
     d = os.path.join(ROOT, "bit_nf4_quantized_quant_b200", "csrc")
-    for f in sorted(os.listdir(d)):
+    for f in sorted(files if files is not None else os.listdir(d)):
         with open(os.path.join(d, f), "rb") as fh:
             h.update(f.encode())
             h.update(fh.read())
@@ -348,7 +350,7 @@ def run_ours(args, rank, world, local_rank):
         roof = {"bound": "tensor", "unit": "TFLOP/s"}
     tr = TRAFFIC.get(f"workload{args.workload}_M{M}")
     roof.update({"achieved": round(achieved, 2), "peak": peak, "frac": round(achieved / peak, 4),
-                 "traffic": tr["bytes_per_launch"] if tr and tr.get("src") == src_hash() else None,
+                 "traffic": tr["bytes_per_launch"] if tr and tr.get("src") == src_hash(tr["files"]) else None,
                  "peak_source": f"{peak_src} ({'hbm copy' if small else 'cuBLAS bf16 sustained'})",
                  "kernel": ("k_nf4_gemv + k_nf4_gemv_finish / k_lora_bwd_small + k_tcs_gemm (programmatic-launch pairs)"
                             if small else "k_tc_gemm / k_tc2_gemm (fwd + bwd dX)"),

@@ -33,6 +33,40 @@
 namespace qnf4 {
 namespace tcs {
 
+// L2 cache policies.  The block constants of a row are 2 bytes per column tile
+// in 32-byte sectors shared by 16 tiles, which different CTAs reach at
+// different times: kept in L2 (evict_last) they are read from DRAM once,
+// instead of once per tile after the streamed weight has pushed them out.
+// The packed weight itself is read once (evict_first).
+__device__ __forceinline__ uint64_t l2_policy_evict_last() {
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
+    return p;
+}
+__device__ __forceinline__ uint64_t l2_policy_evict_first() {
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+    return p;
+}
+__device__ __forceinline__ int ldg_s8_keep(const int8_t* ptr, uint64_t pol) {
+    int v;
+    asm volatile("ld.global.nc.L2::cache_hint.s8 %0, [%1], %2;" : "=r"(v) : "l"(ptr), "l"(pol));
+    return v;
+}
+__device__ __forceinline__ float ldg_f32_keep(const float* ptr, uint64_t pol) {
+    float v;
+    asm volatile("ld.global.nc.L2::cache_hint.f32 %0, [%1], %2;" : "=f"(v) : "l"(ptr), "l"(pol));
+    return v;
+}
+__device__ __forceinline__ void tma_load_2d_hint(uint32_t dst, const CUtensorMap* map, uint32_t bar, int x, int y,
+                                                 uint64_t pol) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+        " [%0], [%1, {%2, %3}], [%4], %5;"
+        ::"r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar), "l"(pol)
+        : "memory");
+}
+
 constexpr int TR = 128;                    // output rows of a tile (MMA M)
 constexpr int KSTEP = 128;                 // reduction per step
 constexpr int SX = 3;                      // activation ring stages
@@ -187,12 +221,13 @@ k_tcs_gemm(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUte
         if (lane == 0) {
             int issued = 0, tile = tile0, ks = ks0;
             bool ok = true;
+            const uint64_t stream_pol = l2_policy_evict_first();
             for (int i = 0; i < nu && ok; ++i) {
                 const int sp = i & (SP - 1), pp = (i / SP) & 1;
                 if (!(ok = tc::mbar_wait(emptyP(sp), pp ^ 1, s_abort))) break;
                 tc::mbar_expect_tx(fullP(sp), P_BYTES);
                 const uint32_t dst = sbase + OFF_P + sp * P_BYTES;
-                tc::tma_load_2d(dst, &tmP, fullP(sp), tile * (TR / 2), ks * KSTEP);
+                tma_load_2d_hint(dst, &tmP, fullP(sp), tile * (TR / 2), ks * KSTEP, stream_pol);
                 ++issued;
                 unit_advance(tile, ks, 1, nks);
             }
@@ -249,6 +284,7 @@ k_tcs_gemm(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUte
         // fetch position: the unit whose block-constant inputs are loaded next
         int fi = grp, ft = tile0, fk = ks0;
         unit_advance(ft, fk, grp, nks);
+        const uint64_t keep_pol = l2_policy_evict_last();
         auto fetch = [&](int& code, float& sc, float& mu) {
             code = 0; sc = 0.f; mu = 0.f;
             const int tile = ft, ks = fk;
@@ -259,9 +295,9 @@ k_tcs_gemm(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUte
             const int64_t n = (int64_t)ks * KSTEP + drow, kb = (int64_t)tile * 2 + dblk;
             if (n < a.N && kb < nblk) {
                 const int64_t b = n * nblk + kb;
-                code = __ldg(a.codes + b);
-                sc = __ldg(a.scale + (b >> 8));
-                mu = __ldg(a.mean + (b >> 8));
+                code = ldg_s8_keep(a.codes + b, keep_pol);
+                sc = ldg_f32_keep(a.scale + (b >> 8), keep_pol);
+                mu = ldg_f32_keep(a.mean + (b >> 8), keep_pol);
             }
         };
         // unit i of this group; (code, sc, mu) hold its block-constant inputs and are
