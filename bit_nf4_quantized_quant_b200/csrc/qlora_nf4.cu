@@ -229,7 +229,7 @@ Plan make_plan(int64_t M, int64_t N, int64_t K, int r, int sms) {
     p.M = M; p.N = N; p.K = K; p.r = r;
     p.rp = (int)rup(r, 16);
     p.rp64 = (int)rup(r, 64);
-    const int64_t target = 2 * (int64_t)sms;
+    const int64_t target = 4 * (int64_t)sms;      // split-K: ~4 CTAs of the memory-bound adapter GEMMs per SM
     const int64_t bj = p.rp == 16 ? 16 : 64;
     // T = X A^T: I = M (BI 64), J = rp, Kd = K
     p.zT = choose_splits(cdiv(M, 64) * cdiv(p.rp, bj), K, target);

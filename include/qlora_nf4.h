@@ -28,7 +28,12 @@
  *     except a per-process copy of the codebook it computes on first use.
  *   - Work is enqueued on `stream` (NULL = the legacy default stream) and
  *     the call returns without synchronizing.  Results are valid once the
- *     stream reaches that point.
+ *     stream reaches that point.  Inputs may be written by work enqueued
+ *     just before the call on the same stream: kernels launched with
+ *     programmatic dependent launch, which may start while the kernel ahead
+ *     of them is still running, read none of the caller's memory before that
+ *     kernel has completed (before it they only prefetch into L2, which is
+ *     coherent).
  *   - The return value is QLORA_OK (0) or a negative QLORA_ERR_* code.  All
  *     argument checks run before anything is launched; a rejected call
  *     launches nothing and writes nothing.  No C++ exception crosses the ABI.

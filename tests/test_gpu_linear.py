@@ -115,6 +115,49 @@ def test_repeatable(oracle_mod):
         assert torch.equal(a, b)        # fixed reduction orders: bit-identical reruns
 
 
+@pytest.mark.parametrize("M", [1, 5, 17, 64, 200])
+def test_inputs_written_just_before_each_call(M):
+    """Every input of every call is written by the kernels queued right before it on the same
+    stream, with no synchronisation: the weights by nf4_quantize_dq, the adapters and dY by torch
+    copies, and layer 1's X is layer 0's Y.  The kernels that start before the one ahead of them
+    has finished (programmatic launch) must read none of it early, so the outputs must equal, bit
+    for bit, those of a run that synchronises after every call."""
+    N0, K0, r, s = 512, 1024, 16, 2.0
+    shapes = [(N0, K0), (K0, N0)]          # layer 1 maps layer 0's output back to K0
+    W = [inputs.weight(90 + i, 0, n, k, 0.02).cuda() for i, (n, k) in enumerate(shapes)]
+    X0 = inputs.normal(92, (M, K0), 1.0).cuda()
+    A = [inputs.uniform(93 + i, (r, k), 1.0 / np.sqrt(k)).cuda() for i, (n, k) in enumerate(shapes)]
+    B = [inputs.normal(95 + i, (n, r), 0.1).cuda() for i, (n, k) in enumerate(shapes)]
+    dY = [inputs.normal(97 + i, (M, n), 1.0).cuda() for i, (n, k) in enumerate(shapes)]
+
+    def run(sync):
+        outs = []
+        x = X0.clone()
+        for i in range(2):
+            w = ops.nf4_quantize_dq(W[i])
+            a, b, dy = A[i].clone(), B[i].clone(), dY[i].clone()
+            if sync:
+                torch.cuda.synchronize()
+            T = torch.empty((M, r), dtype=torch.bfloat16, device="cuda")
+            y = ops.qlora_linear_fwd(x, w, a, b, s, T_out=T)
+            if sync:
+                torch.cuda.synchronize()
+            dx, da, db = ops.qlora_linear_bwd(x, dy, w, a, b, s, T=T)
+            if sync:
+                torch.cuda.synchronize()
+            outs += [y, T, dx, da, db]
+            x = y
+        torch.cuda.synchronize()
+        assert ops.qlora_device_status() == 0
+        return [t.cpu() for t in outs]
+
+    ref = run(True)
+    for _ in range(3):
+        got = run(False)
+        for g, e in zip(got, ref):
+            assert torch.equal(g, e)
+
+
 def _sampled_rows_parity(oracle_mod, wl, proj, M, rows_n=16, bwd=True):
     p = wl.projections[proj]
     s = wl.scaling
