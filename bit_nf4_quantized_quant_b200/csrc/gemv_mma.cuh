@@ -76,23 +76,9 @@ struct Args {
 };
 
 __host__ __device__ __forceinline__ int64_t unit_begin(int64_t c, int64_t U, int64_t C) { return c * U / C; }
-__host__ __device__ __forceinline__ int64_t unit_owner(int64_t u, int64_t U, int64_t C) {
-    return ((u + 1) * C + U - 1) / U - 1;
-}
 __device__ __forceinline__ void unit_advance(int& tile, int& ks, int n, int nks) {
     ks += n;
     while (ks >= nks) { ks -= nks; ++tile; }
-}
-
-// Units of CTA c inside tile [tu0, tu1), and which of its two groups took
-// them: bit 0 = group 0, bit 1 = group 1 (its CTA-local unit indices are even
-// for group 0 and odd for group 1).
-__device__ __forceinline__ int groups_in_tile(int64_t c, int64_t U, int64_t C, int64_t tu0, int64_t tu1) {
-    const int64_t b0 = unit_begin(c, U, C), b1 = unit_begin(c + 1, U, C);
-    const int64_t lo = b0 > tu0 ? b0 : tu0, hi = b1 < tu1 ? b1 : tu1;
-    if (hi - lo >= 2) return 3;
-    if (hi - lo == 1) return 1 << ((lo - b0) & 1);
-    return 0;
 }
 
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, int src_bytes) {

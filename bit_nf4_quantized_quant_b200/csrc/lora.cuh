@@ -188,16 +188,11 @@ struct FinishArgs {
     uint16_t* o2;
     int64_t s2i, s2j, J2, J2pad;
     float alpha2;
-    int* zero;               // optional: zero[0 .. zero_n) = 0 (counters for a later kernel)
-    int64_t zero_n;
 };
 
 __global__ void __launch_bounds__(256) k_gemm_finish(FinishArgs f) {
     grid_dep_launch();
     grid_dep_wait();
-    if (f.zero)
-        for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < f.zero_n; e += (int64_t)gridDim.x * blockDim.x)
-            f.zero[e] = 0;
     const int64_t total = f.Iout * f.Jiter;
     for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < total; e += (int64_t)gridDim.x * blockDim.x) {
         const int64_t i = e / f.Jiter, j = e % f.Jiter;

@@ -102,9 +102,6 @@ struct Args {
 
 // First unit of CTA c, and the CTA that owns unit u, for an even split of U units over C CTAs.
 __host__ __device__ __forceinline__ int64_t unit_begin(int64_t c, int64_t U, int64_t C) { return c * U / C; }
-__host__ __device__ __forceinline__ int64_t unit_owner(int64_t u, int64_t U, int64_t C) {
-    return ((u + 1) * C + U - 1) / U - 1;
-}
 
 // Instruction descriptor: kind::f16, A = B = bf16, D = f32, M = 128, N = NT, A K- or MN-major.
 __host__ __device__ constexpr uint32_t make_idesc(bool a_mn_major, int nt) {
