@@ -190,6 +190,19 @@ struct FinishArgs {
     float alpha2;
 };
 
+// v + p[0] + p[stride] + ... + p[(n - 1) stride], added in that order; four
+// loads are issued before they are added, so a thread waits for memory about
+// n / 4 times instead of n.
+__device__ __forceinline__ float split_sum(const float* p, int64_t stride, int n, float v) {
+    int z = 0;
+    for (; z + 4 <= n; z += 4) {
+        const float a0 = p[z * stride], a1 = p[(z + 1) * stride], a2 = p[(z + 2) * stride], a3 = p[(z + 3) * stride];
+        v += a0; v += a1; v += a2; v += a3;
+    }
+    for (; z < n; ++z) v += p[z * stride];
+    return v;
+}
+
 __global__ void __launch_bounds__(256) k_gemm_finish(FinishArgs f) {
     grid_dep_launch();
     grid_dep_wait();
@@ -198,11 +211,9 @@ __global__ void __launch_bounds__(256) k_gemm_finish(FinishArgs f) {
         const int64_t i = e / f.Jiter, j = e % f.Jiter;
         float v = 0.f;
         if (j < f.J) {
-            for (int z = 0; z < f.splits; ++z) v += f.C[(z * f.I + i) * f.J + j];
-            if (f.row_pair > 0)
-                for (int z = 0; z < f.splits; ++z) v += f.C[(z * f.I + i + f.row_pair) * f.J + j];
-            if (f.col_pair > 0)
-                for (int z = 0; z < f.splits; ++z) v += f.C[(z * f.I + i) * f.J + j + f.col_pair];
+            v = split_sum(f.C + i * f.J + j, f.I * f.J, f.splits, v);
+            if (f.row_pair > 0) v = split_sum(f.C + (i + f.row_pair) * f.J + j, f.I * f.J, f.splits, v);
+            if (f.col_pair > 0) v = split_sum(f.C + i * f.J + j + f.col_pair, f.I * f.J, f.splits, v);
         }
         if (f.f32 && j < f.Jf) f.f32[i * f.ld_f32 + j] = v;
         if (f.hl && j < f.hl_off) {
