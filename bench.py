@@ -21,6 +21,7 @@ from __future__ import annotations
 
 import argparse
 import hashlib
+import re
 import json
 import math
 import os
@@ -39,24 +40,28 @@ PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 
 # dram__bytes_read.sum + dram__bytes_write.sum of the dominant kernel, averaged over its launches
 # in one timed step (ncu --metrics ... --nvtx-include "timed/" python bench.py --steps 1 ..., see
-# profiles/), with the hash of the sources that define those kernels and their launches when the
-# counters were taken (a later change to any of them makes the figure stale: null)
+# profiles/), with the hash of the code (comments aside) of the sources that define those kernels
+# and their launches when the counters were taken (a later code change to any of them makes the
+# figure stale: null)
 _PAIR_SRC = ("common.cuh", "nf4_decode.cuh", "tc_gemm.cuh", "tc2_gemm.cuh", "qlora_nf4.cu")
 _GEMV_SRC = ("common.cuh", "nf4_decode.cuh", "tc_gemm.cuh", "gemv_mma.cuh", "small_lora.cuh", "qlora_nf4.cu")
 TRAFFIC = {
-    "workload3_M2048": {"bytes_per_launch": 40918528, "files": _PAIR_SRC, "src": "b829ec39600b"},
+    "workload3_M2048": {"bytes_per_launch": 40918528, "files": _PAIR_SRC, "src": "702092635744"},
     # small M: one forward chain (GEMV + T + finish) per projection
-    "workload2_M1": {"bytes_per_launch": 24058624, "files": _GEMV_SRC, "src": "63a8d12f13ef"},
+    "workload2_M1": {"bytes_per_launch": 24058624, "files": _GEMV_SRC, "src": "5632ff290ad1"},
 }
 
 
 def src_hash(files=None) -> str:
+    """Hash of the code (comments and blank lines dropped) of the given CUDA sources."""
     h = hashlib.sha1()
     d = os.path.join(ROOT, "bit_nf4_quantized_quant_b200", "csrc")
     for f in sorted(files if files is not None else os.listdir(d)):
-        with open(os.path.join(d, f), "rb") as fh:
-            h.update(f.encode())
-            h.update(fh.read())
+        with open(os.path.join(d, f), encoding="utf-8") as fh:
+            text = re.sub(r"/\*.*?\*/", "", fh.read(), flags=re.S)
+        code = [ln.split("//", 1)[0].rstrip() for ln in text.splitlines()]
+        h.update(f.encode())
+        h.update("\n".join(ln for ln in code if ln).encode())
     return h.hexdigest()[:12]
 
 

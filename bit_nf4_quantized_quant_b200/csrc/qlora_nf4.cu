@@ -629,8 +629,8 @@ int small_fwd(const Plan& p, const uint16_t* X, const nf4dq_weight* w, const uin
     return rc;
 }
 
-// Small-M backward: [T], U partials + dB (and the counters cleared), the fused
-// dY W' kernel (overlapping the U / dB kernel), then dX = dY W' + s U A and dA.
+// Small-M backward: [T], U partials + dB, the fused dY W' kernel (overlapping
+// the U / dB kernel), then dX = dY W' + s U A and dA.
 int small_bwd(const Plan& p, const uint16_t* X, const uint16_t* dY, const nf4dq_weight* w, const uint16_t* A,
               const uint16_t* B, float scaling, const uint16_t* T, uint16_t* dX, uint16_t* dA, uint16_t* dB,
               uint8_t* wsb, int sms, cudaStream_t st) {
