@@ -340,6 +340,7 @@ FinishArgs fin_none() {
 int validate_weight(const nf4dq_weight* w) {
     if (!w || !w->packed || !w->codes || !w->scale || !w->mean) return QLORA_ERR_NULL;
     if (w->N <= 0 || w->K <= 0 || (w->K % kBlock) != 0 || (w->N % 8) != 0) return QLORA_ERR_SHAPE;
+    if (w->K > QLORA_MAX_K) return QLORA_ERR_SHAPE;      // grid y of the K-wide adapter products
     if (w->N > (int64_t)1 << 31 || w->K > (int64_t)1 << 31 || w->N * w->K >= ((int64_t)1 << 38)) return QLORA_ERR_SHAPE;
     if (!aligned16(w->packed)) return QLORA_ERR_ALIGN;
     const uintptr_t lo = reinterpret_cast<uintptr_t>(w->codes) | reinterpret_cast<uintptr_t>(w->scale) |
@@ -719,7 +720,7 @@ int nf4_dequant(const nf4dq_weight* w, qlora_bf16* W_out, qlora_stream_t stream)
 }
 
 size_t qlora_workspace_bytes(int64_t M, int64_t N, int64_t K, int r) {
-    if (M <= 0 || N <= 0 || K <= 0 || (K % kBlock) != 0 || (N % 8) != 0) return 0;
+    if (M <= 0 || N <= 0 || K <= 0 || (K % kBlock) != 0 || (N % 8) != 0 || K > QLORA_MAX_K) return 0;
     if (r < 1 || r > QLORA_MAX_RANK) return 0;
     return make_plan(M, N, K, r, 148).total;
 }

@@ -63,11 +63,14 @@ typedef struct CUstream_st* qlora_stream_t;   /* a cudaStream_t */
 #define QLORA_NF4_BLOCK 64              /* weights per absmax block */
 #define QLORA_DQ_GROUP 256              /* block constants per double-quant group */
 #define QLORA_MAX_RANK 256              /* largest LoRA rank accepted */
+#define QLORA_MAX_K (1 << 21)           /* largest K (input features) of the linear layer: keeps every
+                                           launch's grid within CUDA's limits */
 
 enum {
     QLORA_OK = 0,
     QLORA_ERR_NULL = -1,        /* a required pointer is NULL */
-    QLORA_ERR_SHAPE = -2,       /* M, N or K <= 0, K % 64 != 0, or a size overflows */
+    QLORA_ERR_SHAPE = -2,       /* M, N or K <= 0, K % 64 != 0, K > QLORA_MAX_K (linear layer), or a
+                                   size overflows */
     QLORA_ERR_RANK = -3,        /* r outside [1, QLORA_MAX_RANK] */
     QLORA_ERR_ALIGN = -4,       /* a pointer is not 16-byte aligned */
     QLORA_ERR_WORKSPACE = -5,   /* workspace NULL or smaller than qlora_workspace_bytes() */
@@ -144,7 +147,8 @@ QLORA_API size_t qlora_workspace_bytes(int64_t M, int64_t N, int64_t K, int r);
  * T_out [M, r] bf16 may be NULL; when given it receives bf16(T) for reuse
  * by the backward.  s = scaling (alpha / r).  ws: device workspace of at
  * least qlora_workspace_bytes(M, N, K, r) bytes, 256-byte aligned.
- * X, Y must be 16-byte aligned. */
+ * X, Y must be 16-byte aligned.  Requires K % 64 == 0, K <= QLORA_MAX_K and
+ * N % 8 == 0. */
 QLORA_API int qlora_linear_fwd(const qlora_bf16* X, int64_t M, const nf4dq_weight* w, const qlora_bf16* A,
                      const qlora_bf16* B, int r, float scaling, qlora_bf16* Y, qlora_bf16* T_out,
                      void* ws, size_t ws_bytes, qlora_stream_t stream);

@@ -91,6 +91,14 @@ def test_argument_errors_before_any_launch(lib):
     assert lib.qlora_linear_fwd(fake, 4, ctypes.byref(wbad), fake, fake, 16, 2.0, fake, None, fake, 1 << 30,
                                 None) == -2
     assert lib.qlora_linear_fwd(fake, 0, ctypes.byref(w), fake, fake, 16, 2.0, fake, None, fake, 1 << 30, None) == -2
+    # K beyond QLORA_MAX_K (2^21): rejected before any launch, no workspace size
+    wbig = ops._Weight(0x1000, 0x1000, 0x1000, 0x1000, 64, (1 << 21) + 64)
+    assert lib.qlora_linear_fwd(fake, 4, ctypes.byref(wbig), fake, fake, 16, 2.0, fake, None, fake, 1 << 40,
+                                None) == -2
+    assert lib.qlora_linear_bwd(fake, fake, 4, ctypes.byref(wbig), fake, fake, 16, 2.0, None, fake, fake, fake, fake,
+                                1 << 40, None) == -2
+    assert lib.qlora_workspace_bytes(4, 64, (1 << 21) + 64, 16) == 0
+    assert lib.qlora_workspace_bytes(4, 64, 1 << 21, 16) > 0
     # rank
     assert lib.qlora_linear_fwd(fake, 4, ctypes.byref(w), fake, fake, 0, 2.0, fake, None, fake, 1 << 30, None) == -3
     assert lib.qlora_linear_fwd(fake, 4, ctypes.byref(w), fake, fake, 300, 2.0, fake, None, fake, 1 << 30,
