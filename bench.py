@@ -731,6 +731,9 @@ def main():
         torch.cuda.set_device(local_rank)
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=torch.device("cuda", local_rank))
+        if rank == 0:                 # one rank (re)builds the in-tree library if a source is newer
+            build_lib()
+        dist.barrier()
     build_lib()
     try:
         out = run_bulk(args, rank, world, local_rank) if args.workload == 5 else run_ours(args, rank, world, local_rank)

@@ -41,12 +41,13 @@ def stale() -> bool:
 def build(force: bool = False, verbose: bool = False, extra=None) -> str:
     if not force and not stale():
         return LIB
-    cmd = [_nvcc(), *NVCC_FLAGS, *(extra or []), MAIN, "-o", LIB + ".tmp"]
+    tmp = f"{LIB}.tmp{os.getpid()}"            # per process: concurrent builds never share a file
+    cmd = [_nvcc(), *NVCC_FLAGS, *(extra or []), MAIN, "-o", tmp]
     if verbose:
         cmd.insert(1, "-Xptxas=-v")
         print(" ".join(cmd), flush=True)
     subprocess.check_call(cmd)
-    os.replace(LIB + ".tmp", LIB)
+    os.replace(tmp, LIB)
     return LIB
 
 
