@@ -187,7 +187,11 @@ QLORA_API int qlora_last_path(void);
  * process so far (all threads).  qlora_set_kernel_events: the next
  * qlora_linear_fwd / qlora_linear_bwd call on this thread records `before`
  * (a cudaEvent_t) on its stream right before its fused dequant-GEMM kernel
- * and `after` right after it, then forgets both; pass NULL, NULL to clear. */
+ * and `after` right after it, then forgets both; pass NULL, NULL to clear.
+ * For M <= 32 the pair brackets the fused kernel together with the small
+ * kernels chained to it (forward: GEMV, T, finish; backward: U / dB, then
+ * dY W').  An event between two kernels ends the programmatic-launch overlap
+ * between them, so a timed call runs a little slower than an untimed one. */
 QLORA_API long long qlora_launch_count(void);
 QLORA_API int qlora_set_kernel_events(void* before, void* after);
 
@@ -207,10 +211,12 @@ QLORA_API int qlora_set_kernel_events(void* before, void* after);
  *     before any stream capture.
  *   - Calls whose workspace need (qlora_workspace_bytes) exceeds
  *     QLORA_NOALLOC_SCRATCH_BYTES return QLORA_ERR_SCRATCH and launch
- *     nothing; decode-sized calls (M <= 32 with 70B-model projections) fit.
+ *     nothing.  Decode-sized calls fit: M <= 16 with 70B-model projections
+ *     (up to 28672 x 8192, r <= 64), M <= 32 up to 11008 x 4096; M = 32 with
+ *     a 28672-row weight needs ~12 MiB and is rejected.
  *   - All calls share the one array: calls that overlap on the GPU (other
  *     streams, other host threads) race on it and must be serialized by the
- *     caller.  What the forward needs zeroed it zeroes itself each call.
+ *     caller.  Nothing in the scratch needs to be zeroed between calls.
  * Arguments, layouts and the other errors are those of qlora_linear_fwd. */
 #define QLORA_NOALLOC_SCRATCH_BYTES (8u << 20)
 QLORA_API int qlora_linear_fwd_noalloc(const qlora_bf16* X, int64_t M, const nf4dq_weight* w, const qlora_bf16* A,
