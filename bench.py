@@ -179,7 +179,7 @@ def run_ours(args, rank, world, local_rank):
 
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
-    wl = inputs.WORKLOADS[args.workload]
+    wl = inputs.WORKLOADS[args.workload or 3]
     M = args.M or (wl.Ms[-1] if wl.Ms else 0)
     r, s = wl.r, wl.scaling
     projs = wl.projections
@@ -306,16 +306,7 @@ def run_ours(args, rank, world, local_rank):
     ms_per_step = ms / args.steps
 
     npass = 2 if bwd else 1
-    flops_step = sum(flops_fwd_bwd(M, L["p"].N, L["p"].K, r) if bwd else
-                     2 * M * L["p"].N * L["p"].K + 2 * M * r * (L["p"].K + L["p"].N) for L in layers)
-    # algorithmic HBM bytes of one step: the NF4 weight once per pass, plus the
-    # activations, adapters and outputs each pass reads or writes once
-    bytes_step = 0
-    for L in layers:
-        N_, K_ = L["p"].N, L["p"].K
-        bytes_step += npass * nf4_bytes(N_, K_) + 2 * (M * K_ + r * K_ + N_ * r + M * N_)      # fwd: X, A, B, Y
-        if bwd:
-            bytes_step += 2 * (M * N_ + M * K_ + M * K_ + r * K_ + N_ * r + M * r)           # dY, X, dX, dA, dB, T
+    flops_step, bytes_step = step_work(wl, M)
     # roofline of the dominant kernel (the fused dequant-GEMM), from its own launch events
     kflops, kms, nlaunch = 0.0, 0.0, 0
     kbytes = 0
@@ -351,12 +342,14 @@ def run_ours(args, rank, world, local_rank):
         roof = {"bound": "hbm", "unit": "GB/s"}
     else:
         achieved = kflops / (kms * 1e-3) / 1e12
-        peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
+        peak = peaks["bf16_tflops"]
         roof = {"bound": "tensor", "unit": "TFLOP/s"}
-    tr = TRAFFIC.get(f"workload{args.workload}_M{M}")
+        if "bf16_tflops_sustained" in peaks:
+            roof["frac_of_sustained"] = round(achieved / peaks["bf16_tflops_sustained"], 4)
+    tr = TRAFFIC.get(f"workload{wl.index}_M{M}")
     roof.update({"achieved": round(achieved, 2), "peak": peak, "frac": round(achieved / peak, 4),
                  "traffic": tr["bytes_per_launch"] if tr and tr.get("src") == src_hash(tr["files"]) else None,
-                 "peak_source": f"{peak_src} ({'hbm copy' if small else 'cuBLAS bf16 sustained'})",
+                 "peak_source": f"{peak_src} ({'hbm copy' if small else 'cuBLAS bf16 burst'})",
                  "kernel": ("k_nf4_gemv + k_nf4_gemv_finish / k_lora_bwd_small + k_tcs_gemm (programmatic-launch pairs)"
                             if small else "k_tc_gemm / k_tc2_gemm (fwd + bwd dX)"),
                  "launches_timed": nlaunch, "avg_launch_us": round(kms / nlaunch * 1e3, 2),
@@ -587,7 +580,7 @@ def run_bulk(args, rank, world, local_rank):
     p7 = sum(W.numel() for W, _, _ in tensors[:7])
     q7 = sum(w.packed.numel() + w.codes.numel() + 8 * w.scale.numel() for _, w, _ in tensors[:7])
     e2e = 2 * (2 * p7 + q7) / (e0.elapsed_time(e1) / args.steps * 1e-3) / 1e9
-    return {"metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+    out = {"metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": round(ms, 4), "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16 -> NF4 + int8/fp32 constants -> bf16", "data": "synthetic (seeded)",
             "config": {"workload": wl.name, "tensors": len(tensors), "params": params,
@@ -597,106 +590,190 @@ def run_bulk(args, rank, world, local_rank):
             "e2e": {"value": round(e2e, 1), "unit": "GB/s", "h2d_bytes_per_step": 2 * p7,
                     "d2h_bytes_per_step": 2 * p7 + sum(w.packed.numel() + w.codes.numel() for _, w, _ in tensors[:7])},
             "gpu_launches": launches, "clocks": clk}
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        out["cpu_baseline"] = bulk_cpu_baseline(wl)
+    return out
 
 
 def _threads():
     try:
         from threadpoolctl import threadpool_info
-        n = [i.get("num_threads", 1) for i in threadpool_info()]
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
         return max(n + [1])
     except Exception:
         return os.cpu_count() or 1
 
 
-def oracle_sample_step(wl, proj, rows, state):
-    """One bounded sample of a step on the CPU oracle: dequantize the
-    projection's full weight, then fp64 forward + backward on `rows` tokens.
-    Returns the algorithmic flops of the sampled rows."""
-    import numpy as np
+def step_work(wl, M):
+    """Algorithmic work of one step of a workload at M tokens: (flops, bytes).
 
-    import oracle
-    from bit_nf4_quantized_quant_b200 import inputs
-
-    p = wl.projections[proj]
-    if proj not in state:
-        W = inputs.layer_weight(wl, proj)
-        q = oracle.quantize_dq(inputs.bf16_bits(W))
-        X, A, B, dY = inputs.layer_inputs(wl, proj, rows)
-        state[proj] = (q, inputs.to_f64(X), inputs.to_f64(A), inputs.to_f64(B), inputs.to_f64(dY))
-    q, X, A, B, dY = state[proj]
-    Wd = oracle.bf16_to_f32(oracle.dequant(q)).astype(np.float64)
-    oracle.linear_fwd(X, Wd, A, B, wl.scaling)
-    oracle.linear_bwd(X, dY, Wd, A, B, wl.scaling)
-    return flops_fwd_bwd(rows, p.N, p.K, wl.r)
-
-
-def _distinct_shapes(wl):
-    seen, out = set(), []
-    for i, p in enumerate(wl.projections):
-        if (p.N, p.K) not in seen:
-            seen.add((p.N, p.K))
-            out.append(i)
-    return out
+    flops: 4MNK + 6Mr(K+N) per projection for forward + backward, 2MNK + 2Mr(K+N)
+    for the forward alone.  bytes: the NF4 weight once per pass (4.12890625 bit per
+    parameter) plus every activation, adapter and output tensor read or written once.
+    """
+    r = wl.r
+    flops = bytes_ = 0
+    for p in wl.projections:
+        N_, K_ = p.N, p.K
+        if wl.backward:
+            flops += flops_fwd_bwd(M, N_, K_, r)
+            bytes_ += 2 * nf4_bytes(N_, K_) + 2 * (M * K_ + r * K_ + N_ * r + M * N_)
+            bytes_ += 2 * (M * N_ + M * K_ + M * K_ + r * K_ + N_ * r + M * r)
+        else:
+            flops += 2 * M * N_ * K_ + 2 * M * r * (K_ + N_)
+            bytes_ += nf4_bytes(N_, K_) + 2 * (M * K_ + r * K_ + N_ * r + M * N_)
+    return flops, bytes_
 
 
-def _sample_value(wl, M, projs_done, flops, dt):
-    if M <= 32:
-        b = sum(2 * nf4_bytes(wl.projections[i].N, wl.projections[i].K) for i in projs_done)
-        return b / dt / 1e9, "GB/s"
-    return flops / dt / 1e12, "TFLOP/s"
+class OracleStep:
+    """One step of a workload on the CPU oracle, timed on the host cores.
+
+    Per projection: the oracle's dequantization of the whole NF4 weight (C, run
+    over row ranges on a thread pool of all host cores: ctypes releases the GIL)
+    and its widening to fp64, charged once per step as a layer call would; then
+    the fp64 forward (+ backward) on `rows` of the M tokens (numpy, BLAS on all
+    host cores), whose time is scaled by M / rows -- every token costs the same
+    in these products, so the extrapolation is linear and is labelled as such.
+    Quantization happens once before timing, as at model load."""
+
+    def __init__(self, wl, M, rows=64):
+        import numpy as np
+        from concurrent.futures import ThreadPoolExecutor
+
+        import oracle
+        from bit_nf4_quantized_quant_b200 import inputs
+        self.wl, self.M = wl, M
+        self.rows = min(rows, M)
+        self.ncores = os.cpu_count() or 1
+        self.pool = ThreadPoolExecutor(self.ncores)
+        self.state = []
+        for i, p in enumerate(wl.projections):
+            W = inputs.layer_weight(wl, i)
+            q = oracle.quantize_dq(inputs.bf16_bits(W))
+            X, A, B, dY = inputs.layer_inputs(wl, i, self.rows, with_dy=wl.backward)
+            self.state.append((q, inputs.to_f64(X), inputs.to_f64(A), inputs.to_f64(B),
+                               inputs.to_f64(dY) if dY is not None else None,
+                               np.array_split(np.arange(p.N), self.ncores)))
+        self.flops, self.bytes = step_work(wl, M)
+
+    def run(self):
+        """Returns the step's time in seconds, extrapolated to M tokens."""
+        import numpy as np
+
+        import oracle
+        total = 0.0
+        s = self.wl.scaling
+        for q, X, A, B, dY, chunks in self.state:
+            t0 = time.perf_counter()
+            parts = list(self.pool.map(lambda rr: oracle.dequant_rows(q, rr), chunks))
+            Wd = oracle.bf16_to_f32(np.concatenate(parts)).astype(np.float64)
+            t1 = time.perf_counter()
+            oracle.linear_fwd(X, Wd, A, B, s)
+            if dY is not None:
+                oracle.linear_bwd(X, dY, Wd, A, B, s)
+            t2 = time.perf_counter()
+            total += (t1 - t0) + (t2 - t1) * self.M / self.rows
+        return total
+
+    def value(self, seconds):
+        if self.M <= 32:
+            return self.bytes / seconds / 1e9, "GB/s"
+        return self.flops / seconds / 1e12, "TFLOP/s"
+
+    def sample_text(self, nsteps):
+        return (f"{nsteps} oracle step(s) of all {len(self.wl.projections)} projections: dequant of each full NF4 "
+                f"weight (C, {self.ncores} threads over row ranges) + fp64 fwd{'+bwd' if self.wl.backward else ''} "
+                f"(numpy, {_threads()} BLAS threads) on {self.rows} of {self.M} tokens, the product time scaled "
+                f"by {self.M}/{self.rows} (extrapolated); quantization once, untimed")
 
 
 def cpu_baseline(wl, M, budget_s=20.0):
     """The oracle, as it stands, on the host cores over a bounded sample."""
-    rows = min(64, max(1, M))
-    shapes = _distinct_shapes(wl)
-    state = {}
-    for i in shapes:                               # quantize + inputs: load time, untimed
-        oracle_sample_step(wl, i, rows, state)
+    if wl.index == 5:
+        return bulk_cpu_baseline(wl)
+    st = OracleStep(wl, M)
+    st.run()                                     # warm: first touch of the fp64 buffers
     t0 = time.perf_counter()
-    flops, done = 0, []
-    while True:
-        i = shapes[len(done) % len(shapes)]
-        flops += oracle_sample_step(wl, i, rows, state)
-        done.append(i)
-        if len(done) >= len(shapes) and time.perf_counter() - t0 > budget_s / 2:
-            break
-    dt = time.perf_counter() - t0
-    v, unit = _sample_value(wl, M, done, flops, dt)
-    return {"value": round(v, 6), "unit": unit, "cores": _threads(), "kind": "oracle",
-            "sample": f"{len(done)} projection passes over the {len(shapes)} distinct shapes: oracle dequant of the "
-                      f"full NF4 weight (C, 1 thread) + fp64 fwd+bwd (numpy) on {rows} of {M} tokens; {dt:.1f} s"}
+    times = []
+    while not times or time.perf_counter() - t0 < budget_s / 2:
+        times.append(st.run())
+    v, unit = st.value(statistics.mean(times))
+    return {"value": round(v, 6), "unit": unit, "cores": st.ncores, "kind": "oracle",
+            "sample": st.sample_text(len(times))}
+
+
+def bulk_cpu_baseline(wl):
+    """Workload 5 on the oracle: quantize + double-quantize then dequantize one
+    7-tensor layer (the tensors in parallel on host threads); GB/s of the same
+    byte accounting as the GPU line (read 2 B + write 0.516 B per parameter, each way)."""
+    from concurrent.futures import ThreadPoolExecutor
+
+    import oracle
+    from bit_nf4_quantized_quant_b200 import inputs
+    Ws = [inputs.bf16_bits(inputs.layer_weight(wl, i)) for i in range(len(wl.projections))]
+
+    def one(Wb):
+        q = oracle.quantize_dq(Wb)
+        oracle.dequant(q)
+        return Wb.size
+
+    with ThreadPoolExecutor(len(Ws)) as pool:
+        t0 = time.perf_counter()
+        params = sum(pool.map(one, Ws))
+        dt = time.perf_counter() - t0
+    qbytes = sum(nf4_bytes(p.N, p.K) for p in wl.projections)
+    v = 2 * (2 * params + qbytes) / dt / 1e9
+    return {"value": round(v, 3), "unit": "GB/s", "cores": len(Ws), "kind": "oracle",
+            "sample": f"one layer (7 tensors, {params} params) quantized + dequantized by the C oracle, one thread "
+                      f"per tensor; {dt:.1f} s; the rate stands for the whole 32-layer set"}
 
 
 def run_reference(args):
     """The oracle as the reference arm: host cores, one bounded sample per step."""
     from bit_nf4_quantized_quant_b200 import inputs
-    wl = inputs.WORKLOADS[args.workload]
-    M = args.M or (wl.Ms[-1] if wl.Ms else 0)
-    rows = min(64, max(1, M))
-    shapes = _distinct_shapes(wl)
-    state = {}
-    for i in shapes:
-        oracle_sample_step(wl, i, rows, state)
-    for k in range(args.warmup):
-        oracle_sample_step(wl, shapes[k % len(shapes)], rows, state)
-    t0 = time.perf_counter()
-    flops, done = 0, []
-    for k in range(args.steps):
-        i = shapes[k % len(shapes)]
-        flops += oracle_sample_step(wl, i, rows, state)
-        done.append(i)
-    dt = time.perf_counter() - t0
-    value, unit = _sample_value(wl, M, done, flops, dt)
-    sample = (f"each step: one projection shape (rotating over {len(shapes)}): oracle dequant of its full NF4 "
-              f"weight + fp64 fwd+bwd on {rows} of {M} tokens")
+    wl = inputs.WORKLOADS[args.workload or 3]
+    if wl.index == 5:
+        cb = bulk_cpu_baseline(wl)
+        value, unit, ms, sample = cb["value"], cb["unit"], None, cb["sample"]
+        cores = cb["cores"]
+    else:
+        M = args.M or wl.Ms[-1]
+        st = OracleStep(wl, M)
+        for _ in range(args.warmup):
+            st.run()
+        times = [st.run() for _ in range(args.steps)]
+        ms = statistics.mean(times) * 1e3
+        value, unit = st.value(statistics.mean(times))
+        sample, cores = st.sample_text(args.steps), st.ncores
+    cfg = {"workload": wl.name, "M": args.M or (wl.Ms[-1] if wl.Ms else 0), "r": wl.r, "alpha": wl.alpha}
     return {"impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": unit, "n_gpus": 1,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(dt / args.steps * 1e3, 3),
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 3) if ms else None,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64 (oracle)",
-            "data": "synthetic (seeded)", "config": {"workload": wl.name, "M": M, "r": wl.r, "alpha": wl.alpha},
-            "cpu_baseline": {"value": round(value, 6), "unit": unit, "cores": _threads(), "kind": "oracle",
+            "data": "synthetic (seeded)", "config": cfg,
+            "cpu_baseline": {"value": round(value, 6), "unit": unit, "cores": cores, "kind": "oracle",
                              "sample": sample},
             "e2e": {"value": round(value, 6), "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def sub_results(args, rank, world, local_rank):
+    """The memory-bound half of the metric, measured in the same process after the
+    headline line: decode GEMV (workload 2, M = 1), the single 4096^2 linear
+    (workload 1, M = 16, fwd+bwd) and the bulk quantize + dequantize round trip
+    (workload 5), each with its own roofline entry, clocks and CPU baseline."""
+    import copy
+
+    import torch
+    subs = []
+    for wlx, M in ((2, 1), (1, 16), (5, 0)):
+        torch.cuda.empty_cache()
+        a = copy.copy(args)
+        a.workload, a.M = wlx, M
+        a.cpu_seconds = min(args.cpu_seconds, 8.0)
+        o = run_bulk(a, rank, world, local_rank) if wlx == 5 else run_ours(a, rank, world, local_rank)
+        o.pop("metric", None)
+        o["config"]["M"] = M
+        subs.append(o)
+    return subs
 
 
 def main():
@@ -705,7 +782,10 @@ def main():
     ap.add_argument("--steps", type=int, default=10)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", type=int, default=3, choices=[1, 2, 3, 4, 5])
+    ap.add_argument("--workload", type=int, default=0, choices=[0, 1, 2, 3, 4, 5],
+                    help="0 (default): the 7B block at M = 2048 as the headline line, with the decode GEMV (M = 1), "
+                         "the single 4096^2 linear (M = 16) and the bulk quantize round trip as sub_results")
+    ap.add_argument("--no-sub", action="store_true", help="default workload: skip the sub_results")
     ap.add_argument("--layers", type=int, default=0, help="workload 5: number of 7-tensor layers (default 32)")
     ap.add_argument("--M", type=int, default=0, help="tokens per GPU (default: the workload's largest)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -737,6 +817,8 @@ def main():
     build_lib()
     try:
         out = run_bulk(args, rank, world, local_rank) if args.workload == 5 else run_ours(args, rank, world, local_rank)
+        if args.workload == 0 and world == 1 and not args.no_sub:
+            out["sub_results"] = sub_results(args, rank, world, local_rank)
         if rank == 0:
             print(json.dumps(out), flush=True)
     finally:

@@ -21,7 +21,7 @@
  *     per block.
  *   - "QLoRA: The 4-bit Revolution" (shshell.com), section "2. Double
  *     Quantization": the scaling factors go from 32-bit to 8-bit.
- * Readings taken where the pages are silent (each listed in the design doc):
+ * Readings taken where the pages are silent:
  *   R1 codebook construction (asymmetric 8 positive / 7 negative quantiles,
  *      offset delta = ((1-1/32)+(1-1/30))/2, normalised by the largest level);
  *   R2 nearest level with ties to the lower index, via fp32 midpoints;

@@ -40,3 +40,34 @@ def test_src_hash_ignores_comments_only(tmp_path, monkeypatch):
     assert bench.src_hash(["k.cuh"]) == h0
     (csrc / "k.cuh").write_text("int a = 1;\nint b = 3;\n")
     assert bench.src_hash(["k.cuh"]) != h0
+
+
+def test_step_work_sums_the_projections():
+    from bit_nf4_quantized_quant_b200 import inputs
+    wl = inputs.WORKLOADS[3]
+    f, b = bench.step_work(wl, 2048)
+    assert f == sum(bench.flops_fwd_bwd(2048, p.N, p.K, wl.r) for p in wl.projections)
+    # fwd+bwd streams every NF4 weight twice
+    assert b > 2 * sum(bench.nf4_bytes(p.N, p.K) for p in wl.projections)
+    wl2 = inputs.WORKLOADS[2]
+    f2, b2 = bench.step_work(wl2, 1)
+    assert f2 == sum(2 * p.N * p.K + 2 * wl2.r * (p.N + p.K) for p in wl2.projections)
+    assert b2 == sum(bench.nf4_bytes(p.N, p.K) + 2 * (p.K + wl2.r * p.K + p.N * wl2.r + p.N)
+                     for p in wl2.projections)
+
+
+def test_reference_arm_runs_on_the_host(capsys):
+    """The reference arm (the oracle on the host cores) prints one JSON line with the
+    reference keys, on the single-linear workload."""
+    import json
+    import sys
+    argv = sys.argv
+    try:
+        sys.argv = ["bench.py", "--impl", "reference", "--workload", "1", "--steps", "1", "--warmup", "0"]
+        bench.main()
+    finally:
+        sys.argv = argv
+    line = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
+    assert line["impl"] == "reference" and line["unit"] == "GB/s" and line["value"] > 0
+    assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] >= 1
+    assert line["e2e"]["h2d_bytes_per_step"] == 0

@@ -62,6 +62,13 @@ CASES = [
     (2, 256, 512, 256),         # maximum rank on each path
     (64, 256, 512, 256),
     (130, 256, 512, 256),
+    # more tiles than persistent CTAs (148) or SM pairs (74), so that a CTA or pair runs
+    # several tiles through its double-buffered accumulator: forward tiles span N,
+    # backward tiles span K
+    (64, 38912, 256, 16),       # single-SM kernel: 152 forward tiles
+    (100, 256, 38912, 8),       # single-SM kernel: 152 backward tiles
+    (512, 11008, 1024, 16),     # SM pairs: 86 forward pair tiles
+    (520, 1024, 11008, 32),     # SM pairs: 3 x 43 = 129 backward pair tiles, ragged M
 ]
 
 
@@ -70,13 +77,15 @@ def test_fwd_bwd_parity(oracle_mod, M, N, K, r):
     s = 32.0 / r
     W, X, A, B, dY, Wd, w = _setup(oracle_mod, M, N, K, r, seed=M + N + K + r)
     Xc, Ac, Bc, dYc = X.cuda(), A.cuda(), B.cuda(), dY.cuda()
+    X64, A64, B64, dY64 = (inputs.to_f64(t) for t in (X, A, B, dY))
+    # the backward with T given takes T as an input: feed it the oracle's T rounded to bf16
+    T_in = torch.from_numpy(X64 @ A64.T).to(torch.bfloat16)
     T_out = torch.empty((M, r), dtype=torch.bfloat16, device="cuda")
     Y = ops.qlora_linear_fwd(Xc, w, Ac, Bc, s, T_out=T_out)
     dX, dA, dB = ops.qlora_linear_bwd(Xc, dYc, w, Ac, Bc, s)
-    dX2, dA2, dB2 = ops.qlora_linear_bwd(Xc, dYc, w, Ac, Bc, s, T=T_out)
+    dX2, dA2, dB2 = ops.qlora_linear_bwd(Xc, dYc, w, Ac, Bc, s, T=T_in.cuda())
     torch.cuda.synchronize()
     assert ops.qlora_device_status() == 0
-    X64, A64, B64, dY64 = (inputs.to_f64(t) for t in (X, A, B, dY))
     Yr, Tr = oracle_mod.linear_fwd(X64, Wd, A64, B64, s)
     dXr, dAr, dBr = oracle_mod.linear_bwd(X64, dY64, Wd, A64, B64, s)
     _close(inputs.to_f64(Y), Yr, "Y")
@@ -85,7 +94,7 @@ def test_fwd_bwd_parity(oracle_mod, M, N, K, r):
     _close(inputs.to_f64(dA), dAr, "dA")
     _close(inputs.to_f64(dB), dBr, "dB")
     # with T supplied, the bf16 T is an input of the backward: dB = s dY^T T_given
-    dBr_given = s * (dY64.T @ inputs.to_f64(T_out))
+    dBr_given = s * (dY64.T @ inputs.to_f64(T_in))
     _close(inputs.to_f64(dX2), dXr, "dX (T given)")
     _close(inputs.to_f64(dA2), dAr, "dA (T given)")
     _close(inputs.to_f64(dB2), dBr_given, "dB (T given)")
