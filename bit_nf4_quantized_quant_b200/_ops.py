@@ -29,9 +29,14 @@ class QLoRAError(RuntimeError):
         super().__init__(f"{fn} failed: {code} ({status_string(code)})")
 
 
+QLORA_QUANT_NF4 = 0
+QLORA_QUANT_FP4 = 1
+
+
 class _Weight(ctypes.Structure):
     _fields_ = [("packed", ctypes.c_void_p), ("codes", ctypes.c_void_p), ("scale", ctypes.c_void_p),
-                ("mean", ctypes.c_void_p), ("N", ctypes.c_int64), ("K", ctypes.c_int64)]
+                ("mean", ctypes.c_void_p), ("N", ctypes.c_int64), ("K", ctypes.c_int64),
+                ("quant_type", ctypes.c_int32)]
 
 
 def lib():
@@ -46,6 +51,9 @@ def lib():
         WP = ctypes.POINTER(_Weight)
         sig = {
             "nf4_codebook": (i32, [P]),
+            "quant4_codebook": (i32, [i32, P]),
+            "quant4_quantize_dq": (i32, [P, i64, i64, i32, P, P, P, P, P]),
+            "nf4_dequant_merge": (i32, [WP, P, P, i32, f32, P, P]),
             "nf4dq_sizes": (i32, [i64, i64, P, P, P]),
             "nf4_quantize_dq": (i32, [P, i64, i64, P, P, P, P, P]),
             "nf4_dequant": (i32, [WP, P, P]),
@@ -102,23 +110,30 @@ class NF4Weight:
     mean: torch.Tensor     # fp32 [G]
     N: int
     K: int
+    quant_type: int = QLORA_QUANT_NF4
 
     def c_struct(self) -> _Weight:
         return _Weight(self.packed.data_ptr(), self.codes.data_ptr(), self.scale.data_ptr(),
-                       self.mean.data_ptr(), self.N, self.K)
+                       self.mean.data_ptr(), self.N, self.K, self.quant_type)
 
     @staticmethod
-    def empty(N: int, K: int, device="cuda") -> "NF4Weight":
+    def empty(N: int, K: int, device="cuda", quant_type: int = QLORA_QUANT_NF4) -> "NF4Weight":
         pb, nb, ng = nf4dq_sizes(N, K)
         return NF4Weight(torch.empty((N, K // 2), dtype=torch.uint8, device=device),
                          torch.empty(nb, dtype=torch.int8, device=device),
                          torch.empty(ng, dtype=torch.float32, device=device),
-                         torch.empty(ng, dtype=torch.float32, device=device), N, K)
+                         torch.empty(ng, dtype=torch.float32, device=device), N, K, quant_type)
 
 
 def nf4_codebook() -> list:
     out = (ctypes.c_float * 16)()
     _check("nf4_codebook", lib().nf4_codebook(out))
+    return list(out)
+
+
+def quant4_codebook(quant_type: int) -> list:
+    out = (ctypes.c_float * 16)()
+    _check("quant4_codebook", lib().quant4_codebook(int(quant_type), out))
     return list(out)
 
 
@@ -136,6 +151,30 @@ def nf4_quantize_dq(W: torch.Tensor, out: NF4Weight | None = None, stream=None) 
         out = NF4Weight.empty(N, K, W.device)
     _check("nf4_quantize_dq", lib().nf4_quantize_dq(_ptr(W), N, K, _ptr(out.packed), _ptr(out.codes),
                                                     _ptr(out.scale), _ptr(out.mean), _stream(stream)))
+    return out
+
+
+def quant4_quantize_dq(W: torch.Tensor, quant_type: int, out: NF4Weight | None = None, stream=None) -> NF4Weight:
+    """bf16 W [N, K] (device) -> NF4Weight of the given quant type (NF4 or FP4)."""
+    W = _bits(W)
+    N, K = W.shape
+    if out is None:
+        out = NF4Weight.empty(N, K, W.device, quant_type)
+    out.quant_type = int(quant_type)
+    _check("quant4_quantize_dq", lib().quant4_quantize_dq(_ptr(W), N, K, int(quant_type), _ptr(out.packed),
+                                                          _ptr(out.codes), _ptr(out.scale), _ptr(out.mean),
+                                                          _stream(stream)))
+    return out
+
+
+def nf4_dequant_merge(w: NF4Weight, A, B, scaling: float, out: torch.Tensor | None = None,
+                      stream=None) -> torch.Tensor:
+    """Dense bf16 W' + scaling * B A (the merged weight of the adapted layer)."""
+    if out is None:
+        out = torch.empty((w.N, w.K), dtype=torch.bfloat16, device=w.packed.device)
+    st = w.c_struct()
+    _check("nf4_dequant_merge", lib().nf4_dequant_merge(ctypes.byref(st), _ptr(_bits(A)), _ptr(_bits(B)),
+                                                        A.shape[0], float(scaling), _ptr(out), _stream(stream)))
     return out
 
 

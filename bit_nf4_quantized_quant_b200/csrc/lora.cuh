@@ -188,6 +188,9 @@ struct FinishArgs {
     uint16_t* o2;
     int64_t s2i, s2j, J2, J2pad;
     float alpha2;
+    // o2_lo > 0: o2 holds alpha2 * v as a bf16 hi + lo pair, hi in column j and
+    // lo in column o2_lo + j for j < o2_lo, zero in columns [2 o2_lo, J2pad)
+    int64_t o2_lo;
 };
 
 // v + p[0] + p[stride] + ... + p[(n - 1) stride], added in that order; four
@@ -226,7 +229,22 @@ __global__ void __launch_bounds__(256) k_gemm_finish(FinishArgs f) {
             f.hl[i * f.hl_ld + f.hl_off + j] = lo;
         }
         if (f.o1 && j < f.J1pad) f.o1[i * f.s1i + j * f.s1j] = (j < f.J1) ? (uint16_t)(pack_bf16x2(f.alpha1 * v, 0.f) & 0xffffu) : (uint16_t)0;
-        if (f.o2 && j < f.J2pad) f.o2[i * f.s2i + j * f.s2j] = (j < f.J2) ? (uint16_t)(pack_bf16x2(f.alpha2 * v, 0.f) & 0xffffu) : (uint16_t)0;
+        if (f.o2 && j < f.J2pad) {
+            if (f.o2_lo == 0) {
+                f.o2[i * f.s2i + j * f.s2j] = (j < f.J2) ? (uint16_t)(pack_bf16x2(f.alpha2 * v, 0.f) & 0xffffu) : (uint16_t)0;
+            } else if (j < f.o2_lo) {
+                uint16_t hi = 0, lo = 0;
+                if (j < f.J2) {
+                    const float sv = f.alpha2 * v;
+                    hi = (uint16_t)(pack_bf16x2(sv, 0.f) & 0xffffu);
+                    lo = (uint16_t)(pack_bf16x2(sv - bf16lo_to_f32(hi), 0.f) & 0xffffu);
+                }
+                f.o2[i * f.s2i + j * f.s2j] = hi;
+                f.o2[i * f.s2i + (f.o2_lo + j) * f.s2j] = lo;
+            } else if (j >= 2 * f.o2_lo) {
+                f.o2[i * f.s2i + j * f.s2j] = 0;
+            }
+        }
     }
 }
 

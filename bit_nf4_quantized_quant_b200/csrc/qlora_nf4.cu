@@ -19,6 +19,7 @@
 #include "lora.cuh"
 #include "tc_gemm.cuh"
 #include "tc2_gemm.cuh"
+#include "merge.cuh"
 
 using namespace qnf4;
 
@@ -41,11 +42,37 @@ double inv_phi_bisect(double p) {
     return 0.5 * (lo + hi);
 }
 
-NF4Tables g_tables;
-EncTables g_enc;
+// Tables of the two quant types: [0] NF4, [1] FP4 (E2M1).
+NF4Tables g_tables[2];
+EncTables g_enc[2];
 std::once_flag g_tables_once;
 
+// Decision thresholds of a codebook and the encoder buckets over them.
+// `sorted` lists the n distinct levels in ascending order; thresholds beyond
+// the n - 1 real ones are +inf (the encoder then returns the level's rank,
+// which the quantize kernel maps to its nibble).
+void build_encoder(NF4Tables& t, EncTables& e, const float* sorted, int n) {
+    for (int i = 0; i < 15; ++i) t.m[i] = (i + 1 < n) ? (sorted[i] + sorted[i + 1]) * 0.5f : INFINITY;
+    t.pad = 0.f;
+    // encoder buckets: bucket b holds x with round(64 x + 64) = b, i.e. x in
+    // [(b - 64.5) / 64, (b - 63.5) / 64], widened by eps against rounding
+    const double eps = 1.0 / 512.0;
+    for (int b = 0; b < kEncBuckets; ++b) {
+        const double lo = (b - 64.5) / 64.0 - eps, hi = (b - 63.5) / 64.0 + eps;
+        uint32_t below = 0;
+        float thr = INFINITY;
+        for (int i = 0; i + 1 < n; ++i) {
+            const double mi = t.m[i];
+            if (mi < lo) ++below;
+            else if (mi <= hi) thr = t.m[i];    // at most one (thresholds are >= 0.08 apart)
+        }
+        e.thr[b] = thr;
+        e.qb[b] = below;
+    }
+}
+
 void init_tables() {
+    // NF4: the nibble is the level's rank
     const double delta = 0.5 * ((1.0 - 1.0 / 32.0) + (1.0 - 1.0 / 30.0));
     double pos[8], neg[7];
     for (int i = 0; i < 8; ++i) pos[i] = inv_phi_bisect(delta - (delta - 0.5) * i / 8.0);   // descending
@@ -55,29 +82,31 @@ void init_tables() {
     v[7] = 0.0;
     for (int i = 0; i < 8; ++i) v[8 + i] = pos[7 - i];
     const double top = v[15];
-    for (int i = 0; i < 16; ++i) g_tables.L[i] = (float)(v[i] / top);
-    for (int i = 0; i < 15; ++i) g_tables.m[i] = (g_tables.L[i] + g_tables.L[i + 1]) * 0.5f;
-    g_tables.pad = 0.f;
-    // encoder buckets: bucket b holds x with round(64 x + 64) = b, i.e. x in
-    // [(b - 64.5) / 64, (b - 63.5) / 64], widened by eps against rounding
-    const double eps = 1.0 / 512.0;
-    for (int b = 0; b < kEncBuckets; ++b) {
-        const double lo = (b - 64.5) / 64.0 - eps, hi = (b - 63.5) / 64.0 + eps;
-        uint32_t below = 0;
-        float thr = INFINITY;
-        for (int i = 0; i < 15; ++i) {
-            const double mi = g_tables.m[i];
-            if (mi < lo) ++below;
-            else if (mi <= hi) thr = g_tables.m[i];    // at most one (thresholds are >= 0.08 apart)
-        }
-        g_enc.thr[b] = thr;
-        g_enc.qb[b] = below;
+    for (int i = 0; i < 16; ++i) g_tables[QLORA_QUANT_NF4].L[i] = (float)(v[i] / top);
+    build_encoder(g_tables[QLORA_QUANT_NF4], g_enc[QLORA_QUANT_NF4], g_tables[QLORA_QUANT_NF4].L, 16);
+    // FP4: nibble = E2M1 bit pattern (bit 3 sign, bits 2..1 exponent with bias 1, bit 0
+    // mantissa; exponent 0 is subnormal), divided by the largest magnitude, 6
+    float* L = g_tables[QLORA_QUANT_FP4].L;
+    for (int code = 0; code < 16; ++code) {
+        const int e = (code >> 1) & 3, m = code & 1;
+        const double mag = e == 0 ? 0.5 * m : std::ldexp(1.0 + 0.5 * m, e - 1);
+        L[code] = (float)((code & 8 ? -mag : mag) / 6.0);
     }
+    float sorted[15];
+    int n = 0;
+    for (int code = 15; code >= 9; --code) sorted[n++] = L[code];    // -1 .. -1/12
+    for (int code = 0; code <= 7; ++code) sorted[n++] = L[code];     // 0 .. 1
+    build_encoder(g_tables[QLORA_QUANT_FP4], g_enc[QLORA_QUANT_FP4], sorted, n);
 }
 
-const NF4Tables& tables() {
+const NF4Tables& tables(int qt = QLORA_QUANT_NF4) {
     std::call_once(g_tables_once, init_tables);
-    return g_tables;
+    return g_tables[qt == QLORA_QUANT_FP4 ? 1 : 0];
+}
+
+const EncTables& enc_tables(int qt) {
+    std::call_once(g_tables_once, init_tables);
+    return g_enc[qt == QLORA_QUANT_FP4 ? 1 : 0];
 }
 
 thread_local int t_last_path = 0;
@@ -185,7 +214,7 @@ int launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaS
 // ---------------------------------------------------------------------------
 struct Plan {
     int64_t M, N, K;
-    int r, rp, rp64;
+    int r, rp, lw;                  // lw: columns of the scaled hi | lo LoRA activation
     // split-K choices
     int zT, zU, zA, zB;
     int64_t kT, kU, kA, kB;         // k per split
@@ -228,7 +257,7 @@ Plan make_plan(int64_t M, int64_t N, int64_t K, int r, int sms) {
     Plan p{};
     p.M = M; p.N = N; p.K = K; p.r = r;
     p.rp = (int)rup(r, 16);
-    p.rp64 = (int)rup(r, 64);
+    p.lw = (int)rup(2 * p.rp, 64);
     const int64_t target = 4 * (int64_t)sms;      // split-K: ~4 CTAs of the memory-bound adapter GEMMs per SM
     const int64_t bj = p.rp == 16 ? 16 : 64;
     // T = X A^T: I = M (BI 64), J = rp, Kd = K
@@ -294,8 +323,8 @@ Plan make_plan(int64_t M, int64_t N, int64_t K, int r, int sms) {
     p.off_U32 = take(big * M * p.rp * 4);
     p.off_Tp = take(big * M * 2 * p.rp * 2);     // T hi | lo
     p.off_Ubf = take(big * M * 2 * p.rp * 2);    // U hi | lo
-    p.off_sT = take(big * M * p.rp64 * 2);
-    p.off_sU = take(big * M * p.rp64 * 2);
+    p.off_sT = take(big * M * p.lw * 2);
+    p.off_sU = take(big * M * p.lw * 2);
     p.off_Bp = take(big * N * p.rp * 2);
     p.total = off;
     return p;
@@ -339,6 +368,7 @@ FinishArgs fin_none() {
 
 int validate_weight(const nf4dq_weight* w) {
     if (!w || !w->packed || !w->codes || !w->scale || !w->mean) return QLORA_ERR_NULL;
+    if (w->quant_type != QLORA_QUANT_NF4 && w->quant_type != QLORA_QUANT_FP4) return QLORA_ERR_VALUE;
     if (w->N <= 0 || w->K <= 0 || (w->K % kBlock) != 0 || (w->N % 8) != 0) return QLORA_ERR_SHAPE;
     if (w->K > QLORA_MAX_K) return QLORA_ERR_SHAPE;      // grid y of the K-wide adapter products
     if (w->N > (int64_t)1 << 31 || w->K > (int64_t)1 << 31 || w->N * w->K >= ((int64_t)1 << 38)) return QLORA_ERR_SHAPE;
@@ -432,10 +462,11 @@ int ensure_tc_attrs() {
 }
 
 // Fused dequant-GEMM on the tcgen05 path.  act [M, n_red] bf16 activations,
-// lact [M, rp64] bf16 scaled LoRA activations, lora_w / ldl the LoRA weight
+// lact [M, lw] bf16 scaled LoRA activations as hi | lo halves of rp = rup(r, 16)
+// columns each (lw = rup(2 rp, 64)), lora_w / ldl the LoRA weight
 // rows (B for the forward, A for the backward).
 template <bool BWD>
-int launch_tc(const nf4dq_weight* w, const uint16_t* act, int64_t M, const uint16_t* lact, int rp64,
+int launch_tc(const nf4dq_weight* w, const uint16_t* act, int64_t M, const uint16_t* lact, int lw,
               const uint16_t* lora_w, int64_t ldl, int r, uint16_t* out, int sms, cudaStream_t st) {
     int rc = ensure_tc_attrs();
     if (rc != QLORA_OK) return rc;
@@ -444,19 +475,19 @@ int launch_tc(const nf4dq_weight* w, const uint16_t* act, int64_t M, const uint1
     CUtensorMap tmA, tmL, tmP;
     if (!make_map_2d(&tmA, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, act, n_red, M, n_red * 2, 64, 128,
                      CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !make_map_2d(&tmL, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, lact, rp64, M, (uint64_t)rp64 * 2, 64, 128,
+        !make_map_2d(&tmL, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, lact, lw, M, (uint64_t)lw * 2, 64, 128,
                      CU_TENSOR_MAP_SWIZZLE_128B) ||
         !make_map_2d(&tmP, CU_TENSOR_MAP_DATA_TYPE_UINT8, w->packed, K / 2, N, K / 2, BWD ? 128 : 32,
                      BWD ? 64 : 256, BWD ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_32B))
         return QLORA_ERR_LAUNCH;
     tc::Args a{};
     a.codes = w->codes; a.scale = w->scale; a.mean = w->mean;
-    a.lora_w = lora_w; a.ldl = ldl; a.r = r; a.nlora = (int)cdiv(r, 64);
+    a.lora_w = lora_w; a.ldl = ldl; a.r = r; a.lper = (int)rup(r, 16); a.nlora = (int)cdiv(lw, 64);
     a.out = out; a.M = M; a.N = N; a.K = K; a.n_out = n_out; a.n_red = n_red;
     const int64_t ntiles = cdiv(M, tc::BM) * cdiv(n_out, tc::BN);
     const int grid = (int)(ntiles < sms ? ntiles : sms);
     hook_before(st);
-    tc::k_tc_gemm<BWD><<<grid, tc::kThreads, tc::SMEM_ALLOC, st>>>(tmA, tmL, tmP, a, tables());
+    tc::k_tc_gemm<BWD><<<grid, tc::kThreads, tc::SMEM_ALLOC, st>>>(tmA, tmL, tmP, a, tables(w->quant_type));
     hook_after(st);
     note_launch();
     return launch_status();
@@ -464,26 +495,26 @@ int launch_tc(const nf4dq_weight* w, const uint16_t* act, int64_t M, const uint1
 
 // The same on SM pairs (cta_group::2), 256 x 256 tiles.
 template <bool BWD>
-int launch_tc2(const nf4dq_weight* w, const uint16_t* act, int64_t M, const uint16_t* lact, int rp64,
+int launch_tc2(const nf4dq_weight* w, const uint16_t* act, int64_t M, const uint16_t* lact, int lw,
                const uint16_t* lora_w, int64_t ldl, int r, uint16_t* out, int pairs, cudaStream_t st) {
     const int64_t N = w->N, K = w->K;
     const int64_t n_red = BWD ? N : K, n_out = BWD ? K : N;
     CUtensorMap tmA, tmL, tmP;
     if (!make_map_2d(&tmA, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, act, n_red, M, n_red * 2, 64, 128,
                      CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !make_map_2d(&tmL, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, lact, rp64, M, (uint64_t)rp64 * 2, 64, 128,
+        !make_map_2d(&tmL, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, lact, lw, M, (uint64_t)lw * 2, 64, 128,
                      CU_TENSOR_MAP_SWIZZLE_128B) ||
         !make_map_2d(&tmP, CU_TENSOR_MAP_DATA_TYPE_UINT8, w->packed, K / 2, N, K / 2, BWD ? 64 : 32,
                      BWD ? 64 : 128, BWD ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B))
         return QLORA_ERR_LAUNCH;
     tc::Args a{};
     a.codes = w->codes; a.scale = w->scale; a.mean = w->mean;
-    a.lora_w = lora_w; a.ldl = ldl; a.r = r; a.nlora = (int)cdiv(r, 64);
+    a.lora_w = lora_w; a.ldl = ldl; a.r = r; a.lper = (int)rup(r, 16); a.nlora = (int)cdiv(lw, 64);
     a.out = out; a.M = M; a.N = N; a.K = K; a.n_out = n_out; a.n_red = n_red;
     const int64_t ntiles = cdiv(M, tc2::BM) * cdiv(n_out, tc2::BN);
     const int np = (int)(ntiles < pairs ? ntiles : pairs);
     hook_before(st);
-    tc2::k_tc2_gemm<BWD><<<2 * np, tc2::kThreads, tc2::SMEM_ALLOC, st>>>(tmA, tmL, tmP, a, tables());
+    tc2::k_tc2_gemm<BWD><<<2 * np, tc2::kThreads, tc2::SMEM_ALLOC, st>>>(tmA, tmL, tmP, a, tables(w->quant_type));
     hook_after(st);
     note_launch();
     return launch_status();
@@ -501,16 +532,17 @@ int current_pairs() {
 // Tokens at or below this count take the small-M (GEMV-shaped) kernels.
 constexpr int64_t kSmallMaxM = 32;
 
-// T = X A^T: T32 (fp32 [M, rp]), Thl (bf16 hi|lo [M, 2 rp]), sT (bf16 s*T, [M, rp64]),
+// T = X A^T: T32 (fp32 [M, rp]), Thl (bf16 hi|lo [M, 2 rp]), sT (bf16 s*T as hi | lo, [M, lw]),
 // and the caller's T_out (bf16 [M, r]) when given.
 int compute_T(const Plan& p, const uint16_t* X, const uint16_t* A, float s, uint16_t* T_out, uint8_t* ws, int sms,
               cudaStream_t st) {
     FinishArgs f = fin_none();
-    f.Iout = p.M; f.Jiter = p.rp64;
+    f.Iout = p.M; f.Jiter = p.lw;
     f.f32 = reinterpret_cast<float*>(ws + p.off_T32); f.ld_f32 = p.rp; f.Jf = p.rp;
     f.J1 = p.r;
     f.hl = reinterpret_cast<uint16_t*>(ws + p.off_Tp); f.hl_ld = 2 * p.rp; f.hl_off = p.rp;
-    f.o2 = reinterpret_cast<uint16_t*>(ws + p.off_sT); f.s2i = p.rp64; f.s2j = 1; f.J2 = p.r; f.J2pad = p.rp64; f.alpha2 = s;
+    f.o2 = reinterpret_cast<uint16_t*>(ws + p.off_sT); f.s2i = p.lw; f.s2j = 1; f.J2 = p.r; f.J2pad = p.lw; f.alpha2 = s;
+    f.o2_lo = p.rp;
     if (T_out) {   // the caller's bf16 T [M, r]: the same rounding as the hi half of Thl
         f.o1 = T_out; f.s1i = p.r; f.s1j = 1; f.J1pad = p.r; f.alpha1 = 1.f;
     }
@@ -563,8 +595,9 @@ int launch_tcs_bwd(const Plan& p, const nf4dq_weight* w, const uint16_t* dY, uin
     a.slots = reinterpret_cast<float*>(wsb + p.off_slots);
     *out = a;
     const dim3 grid((unsigned)ctas), block(tcs::kThreads);
-    if (p.NT == 16) return launch_pdl(tcs::k_tcs_gemm<16>, grid, block, tcs::SMEM_ALLOC, st, tmX, tmP, a, tables());
-    return launch_pdl(tcs::k_tcs_gemm<32>, grid, block, tcs::SMEM_ALLOC, st, tmX, tmP, a, tables());
+    const NF4Tables& tab = tables(w->quant_type);
+    if (p.NT == 16) return launch_pdl(tcs::k_tcs_gemm<16>, grid, block, tcs::SMEM_ALLOC, st, tmX, tmP, a, tab);
+    return launch_pdl(tcs::k_tcs_gemm<32>, grid, block, tcs::SMEM_ALLOC, st, tmX, tmP, a, tab);
 }
 
 // Small-M forward: the GEMV (mma.sync, stream-K over one CTA per SM), the
@@ -603,7 +636,7 @@ int launch_gemv_ntt(const Plan& p, const nf4dq_weight* w, const uint16_t* X, con
     a.ctas = (int)ctas;
     a.slots = reinterpret_cast<float*>(wsb + p.off_slots);
     int rc = launch_pdl(gmv::k_nf4_gemv<NTT>, dim3((unsigned)ctas), dim3(gmv::kThreads), (size_t)C::SMEM_ALLOC, st,
-                        tmP, a, tables());
+                        tmP, a, tables(w->quant_type));
     if (rc != QLORA_OK) return rc;
     rc = small_T(p, X, A, nullptr, wsb, st, true);
     if (rc != QLORA_OK) return rc;
@@ -687,26 +720,45 @@ int nf4dq_sizes(int64_t N, int64_t K, int64_t* packed_bytes, int64_t* n_blocks, 
     return QLORA_OK;
 }
 
-int nf4_quantize_dq(const qlora_bf16* W, int64_t N, int64_t K, uint8_t* packed, int8_t* codes, float* scale,
-                    float* mean, qlora_stream_t stream) {
+int quant4_codebook(int quant_type, float out16[16]) {
+    if (!out16) return QLORA_ERR_NULL;
+    if (quant_type != QLORA_QUANT_NF4 && quant_type != QLORA_QUANT_FP4) return QLORA_ERR_VALUE;
+    const NF4Tables& t = tables(quant_type);
+    for (int i = 0; i < 16; ++i) out16[i] = t.L[i];
+    return QLORA_OK;
+}
+
+int quant4_quantize_dq(const qlora_bf16* W, int64_t N, int64_t K, int quant_type, uint8_t* packed, int8_t* codes,
+                       float* scale, float* mean, qlora_stream_t stream) {
     if (!W || !packed || !codes || !scale || !mean) return QLORA_ERR_NULL;
+    if (quant_type != QLORA_QUANT_NF4 && quant_type != QLORA_QUANT_FP4) return QLORA_ERR_VALUE;
     int64_t nb = 0, ng = 0;
     if (nf4dq_sizes(N, K, nullptr, &nb, &ng) != QLORA_OK) return QLORA_ERR_SHAPE;
     if (!aligned16(W) || !aligned16(packed)) return QLORA_ERR_ALIGN;
     int sms = 0;
     int rc = check_device(&sms);
     if (rc != QLORA_OK) return rc;
-    const NF4Tables& tab = tables();
+    const NF4Tables& tab = tables(quant_type);
+    const EncTables& enc = enc_tables(quant_type);
     int grid = (int)(ng < (int64_t)sms * 8 ? ng : (int64_t)sms * 8);
-    k_quantize_dq<<<grid, 256, 0, (cudaStream_t)stream>>>(W, nb, packed, codes, scale, mean, tab, g_enc);
+    if (quant_type == QLORA_QUANT_FP4)
+        k_quantize_dq<true><<<grid, 256, 0, (cudaStream_t)stream>>>(W, nb, packed, codes, scale, mean, tab, enc);
+    else
+        k_quantize_dq<false><<<grid, 256, 0, (cudaStream_t)stream>>>(W, nb, packed, codes, scale, mean, tab, enc);
     note_launch();
     return launch_status();
+}
+
+int nf4_quantize_dq(const qlora_bf16* W, int64_t N, int64_t K, uint8_t* packed, int8_t* codes, float* scale,
+                    float* mean, qlora_stream_t stream) {
+    return quant4_quantize_dq(W, N, K, QLORA_QUANT_NF4, packed, codes, scale, mean, stream);
 }
 
 int nf4_dequant(const nf4dq_weight* w, qlora_bf16* W_out, qlora_stream_t stream) {
     int rc = (!w || !W_out) ? QLORA_ERR_NULL : QLORA_OK;
     if (rc != QLORA_OK) return rc;
     if (!w->packed || !w->codes || !w->scale || !w->mean) return QLORA_ERR_NULL;
+    if (w->quant_type != QLORA_QUANT_NF4 && w->quant_type != QLORA_QUANT_FP4) return QLORA_ERR_VALUE;
     if (nf4dq_sizes(w->N, w->K, nullptr, nullptr, nullptr) != QLORA_OK) return QLORA_ERR_SHAPE;
     if (!aligned16(w->packed) || !aligned16(W_out)) return QLORA_ERR_ALIGN;
     int sms = 0;
@@ -714,7 +766,38 @@ int nf4_dequant(const nf4dq_weight* w, qlora_bf16* W_out, qlora_stream_t stream)
     if (rc != QLORA_OK) return rc;
     const int64_t nwords = w->N * w->K / 8;                    // 8 weights per packed 32-bit word
     k_dequant<<<grid_for(nwords, 8 * kDqWarpWords, sms, 4), 256, 0, (cudaStream_t)stream>>>(
-        w->packed, w->codes, w->scale, w->mean, nwords, W_out, tables());
+        w->packed, w->codes, w->scale, w->mean, nwords, W_out, tables(w->quant_type));
+    note_launch();
+    return launch_status();
+}
+
+int nf4_dequant_merge(const nf4dq_weight* w, const qlora_bf16* A, const qlora_bf16* B, int r, float scaling,
+                      qlora_bf16* W_out, qlora_stream_t stream) {
+    if (!w || !A || !B || !W_out) return QLORA_ERR_NULL;
+    if (!w->packed || !w->codes || !w->scale || !w->mean) return QLORA_ERR_NULL;
+    if (w->quant_type != QLORA_QUANT_NF4 && w->quant_type != QLORA_QUANT_FP4) return QLORA_ERR_VALUE;
+    if (nf4dq_sizes(w->N, w->K, nullptr, nullptr, nullptr) != QLORA_OK || w->K > QLORA_MAX_K) return QLORA_ERR_SHAPE;
+    if (r < 1 || r > QLORA_MAX_RANK) return QLORA_ERR_RANK;
+    if (!std::isfinite(scaling)) return QLORA_ERR_VALUE;
+    if (!aligned16(w->packed) || !aligned16(A) || !aligned16(W_out)) return QLORA_ERR_ALIGN;
+    int sms = 0;
+    int rc = check_device(&sms);
+    if (rc != QLORA_OK) return rc;
+    static bool attr_set[64];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return QLORA_ERR_DEVICE;
+    if (!attr_set[dev]) {
+        std::lock_guard<std::mutex> lk(g_tc_mu);
+        if (cudaFuncSetAttribute(merge::k_dequant_merge, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 merge::SMEM_BYTES) != cudaSuccess)
+            return QLORA_ERR_LAUNCH;
+        attr_set[dev] = true;
+    }
+    merge::Args a{};
+    a.packed = w->packed; a.codes = w->codes; a.scale = w->scale; a.mean = w->mean;
+    a.A = A; a.B = B; a.out = W_out; a.N = w->N; a.K = w->K; a.r = r; a.s = scaling;
+    const dim3 grid((unsigned)cdiv(w->N, merge::TM), (unsigned)cdiv(w->K, merge::TK));
+    merge::k_dequant_merge<<<grid, merge::kThreads, merge::SMEM_BYTES, (cudaStream_t)stream>>>(a, tables(w->quant_type));
     note_launch();
     return launch_status();
 }
@@ -769,12 +852,12 @@ int qlora_linear_fwd(const qlora_bf16* X, int64_t M, const nf4dq_weight* w, cons
     if (rc != QLORA_OK) return rc;
     const int pairs = current_pairs();
     if (M > kPairMinM && pairs > 0) {
-        rc = launch_tc2<false>(w, X, M, reinterpret_cast<const uint16_t*>(wsb + p.off_sT), p.rp64, lw, ldl, r, Y,
+        rc = launch_tc2<false>(w, X, M, reinterpret_cast<const uint16_t*>(wsb + p.off_sT), p.lw, lw, ldl, r, Y,
                                pairs, st);
         if (rc == QLORA_OK) t_last_path = 3;
         return rc;
     }
-    rc = launch_tc<false>(w, X, M, reinterpret_cast<const uint16_t*>(wsb + p.off_sT), p.rp64, lw, ldl, r, Y, sms, st);
+    rc = launch_tc<false>(w, X, M, reinterpret_cast<const uint16_t*>(wsb + p.off_sT), p.lw, lw, ldl, r, Y, sms, st);
     if (rc == QLORA_OK) t_last_path = 2;
     return rc;
 }
@@ -821,7 +904,7 @@ int qlora_linear_bwd(const qlora_bf16* X, const qlora_bf16* dY, int64_t M, const
     }
     if (rc != QLORA_OK) return rc;
 
-    // U = dY B  ->  U32 (fp32), Uhl (bf16 hi | lo), sU (bf16 s*U, [M, rp64])
+    // U = dY B  ->  U32 (fp32), Uhl (bf16 hi | lo), sU (bf16 s*U as hi | lo, [M, lw])
     const uint16_t* Bop = B;
     int64_t ldb = r;
     if (r % 8 != 0 || !aligned16(B)) {
@@ -832,11 +915,12 @@ int qlora_linear_bwd(const qlora_bf16* X, const qlora_bf16* dY, int64_t M, const
     }
     {
         FinishArgs f = fin_none();
-        f.Iout = M; f.Jiter = p.rp64;
+        f.Iout = M; f.Jiter = p.lw;
         f.f32 = reinterpret_cast<float*>(wsb + p.off_U32); f.ld_f32 = p.rp; f.Jf = p.rp;
         f.J1 = r;
         f.hl = Uhl; f.hl_ld = 2 * p.rp; f.hl_off = p.rp;
-        f.o2 = reinterpret_cast<uint16_t*>(wsb + p.off_sU); f.s2i = p.rp64; f.s2j = 1; f.J2 = r; f.J2pad = p.rp64;
+        f.o2 = reinterpret_cast<uint16_t*>(wsb + p.off_sU); f.s2i = p.lw; f.s2j = 1; f.J2 = r; f.J2pad = p.lw;
+        f.o2_lo = p.rp;
         f.alpha2 = scaling;
         rc = run_gemm<true, false>(dY, N, Bop, ldb, M, p.rp, N, M, r, p.zU, p.kU, part, f, sms, st);
         if (rc != QLORA_OK) return rc;
@@ -866,12 +950,12 @@ int qlora_linear_bwd(const qlora_bf16* X, const qlora_bf16* dY, int64_t M, const
     if (rc != QLORA_OK) return rc;
     const int pairs = current_pairs();
     if (M > kPairMinM && pairs > 0) {
-        rc = launch_tc2<true>(w, dY, M, reinterpret_cast<const uint16_t*>(wsb + p.off_sU), p.rp64, A, K, r, dX,
+        rc = launch_tc2<true>(w, dY, M, reinterpret_cast<const uint16_t*>(wsb + p.off_sU), p.lw, A, K, r, dX,
                               pairs, st);
         if (rc == QLORA_OK) t_last_path = 3;
         return rc;
     }
-    rc = launch_tc<true>(w, dY, M, reinterpret_cast<const uint16_t*>(wsb + p.off_sU), p.rp64, A, K, r, dX, sms, st);
+    rc = launch_tc<true>(w, dY, M, reinterpret_cast<const uint16_t*>(wsb + p.off_sU), p.lw, A, K, r, dX, sms, st);
     if (rc == QLORA_OK) t_last_path = 2;
     return rc;
 }

@@ -25,7 +25,7 @@ __device__ __forceinline__ uint32_t nf4_encode(float x, const NF4Tables& tab, co
 
 // The exact level of w in a block with absmax c (the slow path of the encoder
 // below): x = fl32(w / c) by IEEE division, then the 4-step search; c = 0
-// gives level 7.  Kept out of line: it runs for about one weight in 10^5.
+// gives rank 7, the zero level of both codebooks.  Kept out of line: it runs for about one weight in 10^5.
 __device__ __noinline__ uint32_t nf4_encode_exact(float w, float c, float m3, float m7, float m11,
                                                   const float* s_m) {
     if (c == 0.f) return 7u;
@@ -45,6 +45,18 @@ __device__ __noinline__ uint32_t nf4_encode_exact(float w, float c, float m3, fl
 // quantization with the fp64 pairwise tree held in registers: lane l keeps
 // slots l, l+32, ..., l+224, so strides 128, 64, 32 are in-register adds and
 // strides 16..1 are shuffles -- the same association order as the definition.
+//
+// FP4 (kFP4): the same search yields the level's rank among the 15 distinct
+// FP4 levels in ascending order (threshold 14 is +inf); its nibble is the
+// E2M1 bit pattern of that level: ranks 0..6 are -1 .. -1/12 (codes 15..9),
+// rank 7 is +0 (code 0), ranks 8..14 are 1/12 .. 1 (codes 1..7).
+template <bool kFP4>
+__device__ __forceinline__ uint32_t rank_to_nibble(uint32_t q) {
+    if (!kFP4) return q;
+    return q < 7u ? 15u - q : q - 7u;
+}
+
+template <bool kFP4>
 __global__ void __launch_bounds__(256, 4) k_quantize_dq(const uint16_t* __restrict__ W, int64_t nblocks,
                                                      uint8_t* __restrict__ packed, int8_t* __restrict__ codes,
                                                      float* __restrict__ scale, float* __restrict__ mean,
@@ -105,7 +117,7 @@ __global__ void __launch_bounds__(256, 4) k_quantize_dq(const uint16_t* __restri
                     const float2 e = s_enc[b];
                     const float d = __fsub_rn(x, e.x);
                     if (!(fabsf(d) > 9.5367431640625e-07f)) slow |= 1u << j;     // 2^-20 (also NaN)
-                    const uint32_t q = __float_as_uint(e.y) + (d > 0.f ? 1u : 0u);
+                    const uint32_t q = rank_to_nibble<kFP4>(__float_as_uint(e.y) + (d > 0.f ? 1u : 0u));
                     // element 2i -> high nibble of byte i (little-endian word)
                     word |= q << ((j >> 1) * 8 + ((j & 1) ? 0 : 4));
                 }
@@ -115,7 +127,8 @@ __global__ void __launch_bounds__(256, 4) k_quantize_dq(const uint16_t* __restri
                     for (int j = 0; j < 8; ++j) {
                         if ((slow >> j) & 1u) {
                             const int sh = (j >> 1) * 8 + ((j & 1) ? 0 : 4);
-                            const uint32_t q = nf4_encode_exact(w[j], c, tab.m[3], tab.m[7], tab.m[11], s_m);
+                            const uint32_t q =
+                                rank_to_nibble<kFP4>(nf4_encode_exact(w[j], c, tab.m[3], tab.m[7], tab.m[11], s_m));
                             word = (word & ~(15u << sh)) | (q << sh);
                         }
                     }

@@ -364,11 +364,20 @@ k_tc2_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
         const uint32_t cbase = sbase + OFF_C + (uint32_t)dthr * 4;
         auto cslot = [&](int slot, int wd) { return cbase + (uint32_t)((slot * 3 + wd) * 2 * kGroupThreads * 4); };
         int shift0 = 0, shift1 = 0;                                  // byte of the code in its word
+        // A step past the tile's last dequantization step (a LoRA step, or beyond the
+        // tile) reads no constants: it copies nothing and commits an empty group.  Such
+        // steps are the last fetches of a tile, and the next tile's first fetches write
+        // the same slots before anyone waits for these; two copies in flight to one
+        // address may land in either order, so none of them may be a copy.
         auto fetch = [&](int64_t c0, int st, int slot) {
+            if (st >= nks) {
+                asm volatile("cp.async.commit_group;" ::: "memory");
+                return;
+            }
             int64_t n, kb;
             if (!BWD) { n = c0 + drow; kb = st; }
             else { n = (int64_t)st * BK + drow; kb = c0 / kBlock + dblk; }
-            const bool v = st < nks && n < a.N && kb < nblk;
+            const bool v = n < a.N && kb < nblk;
             const int64_t b = v ? n * nblk + kb : 0;
             const int sz = v ? 4 : 0;                                   // 0: zero-fill (constant 0)
             if (slot) shift1 = (int)(b & 3) * 8;
@@ -398,18 +407,18 @@ k_tc2_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
                 wpos(it, step, sw, pw);
                 const int slot = k & 1;
                 uint32_t o[8][4];
+                int rel = -1;               // packed stage to release once its data is consumed
                 if (step < nks) {
                     const float c = block_const(slot);
                     int sp, pp;
                     ppos(it, step, sp, pp);
+                    rel = sp;
                     if (!(ok = tc::mbar_wait(fullP(sp), pp, s_abort))) break;
                     uint4 p0, p1;
                     const uint32_t pst = sbase + OFF_P + sp * P_BYTES;
                     const uint32_t src0 = pst + p_chunk_offset<BWD>(t, 0), src1 = pst + p_chunk_offset<BWD>(t, 1);
                     asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(p0.x), "=r"(p0.y), "=r"(p0.z), "=r"(p0.w) : "r"(src0));
                     asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(p1.x), "=r"(p1.y), "=r"(p1.z), "=r"(p1.w) : "r"(src1));
-                    __syncwarp();
-                    if (lane == 0) tc::mbar_arrive(emptyP(sp));
                     const BlockTable tb = make_block_table(tab, c);
                     const uint32_t pwd[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
 #pragma unroll
@@ -425,15 +434,22 @@ k_tc2_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
                         src = a.lora_w + n * a.ldl;
                         col0 = (int64_t)lc * BK;
                     } else {
-                        const int64_t i = (int64_t)lc * BK + drow;
-                        rowok = i < a.r;
+                        const int64_t ip = (int64_t)lc * BK + drow, i = ip >= a.lper ? ip - a.lper : ip;
+                        rowok = ip < 2 * a.lper && i < a.r;
                         src = a.lora_w + i * a.ldl;
                         col0 = c0 + dblk * 64;
                     }
 #pragma unroll
                     for (int ch = 0; ch < 8; ++ch) {
-                        const int64_t col = col0 + ch * 8;
-                        const bool v = rowok && (BWD ? (col < a.K) : (col < a.r));
+                        int64_t col = col0 + ch * 8;
+                        bool v;
+                        if (BWD) {
+                            v = rowok && col < a.K;
+                        } else {                    // rank index: the same B columns for hi and lo
+                            v = rowok && col < 2 * a.lper;
+                            if (col >= a.lper) col -= a.lper;
+                            v = v && col < a.r;
+                        }
                         uint4 q = make_uint4(0, 0, 0, 0);
                         if (v) q = __ldg(reinterpret_cast<const uint4*>(src + col));
                         o[ch][0] = q.x; o[ch][1] = q.y; o[ch][2] = q.z; o[ch][3] = q.w;
@@ -451,7 +467,13 @@ k_tc2_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
                 // the leader's warps arrive on its own barrier; the peer's on a local one whose
                 // completion a forwarder passes on (a cluster-scope release per warp and step
                 // would cost each dequantizer a cluster fence, ~1000 cycles)
-                if (lane == 0) tc::mbar_arrive(leader ? fullW(sw) : fullWl(sw));
+                // the packed stage is released only after the stores above, which consume
+                // the values decoded from it: a release right after the shared loads were
+                // issued let the next TMA copy overwrite the stage under loads in flight
+                if (lane == 0) {
+                    tc::mbar_arrive(leader ? fullW(sw) : fullWl(sw));
+                    if (rel >= 0) tc::mbar_arrive(emptyP(rel));
+                }
                 fetch(c0, step + 4, slot);                     // refill: the group's step after next
             }
         }

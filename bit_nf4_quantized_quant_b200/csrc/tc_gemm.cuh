@@ -68,7 +68,12 @@ struct Args {
     const uint16_t* lora_w;   // forward: B [N, ldl]; backward: A [r, ldl]
     int64_t ldl;              // row stride of lora_w in elements (multiple of 8)
     int r;                    // LoRA rank
-    int nlora;                // ceil(r / 64) extra reduction steps
+    // The LoRA term enters as extra reduction steps over a scaled activation
+    // (s T forward, s U backward) held as a bf16 hi + lo pair, [hi | lo] with
+    // each half `lper` columns wide (r rounded up to 16, zero beyond r): LoRA
+    // reduction index j' pairs with rank index j' mod lper, for j' < 2 lper.
+    int lper;
+    int nlora;                // ceil(2 lper / 64) extra reduction steps
     uint16_t* out;            // Y [M, N] or dX [M, K]
     int64_t M, N, K;          // W is [N, K]
     int64_t n_out;            // N (forward) or K (backward)
@@ -367,6 +372,7 @@ k_tc_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
         // loads have two steps to land before anything reads the registers)
         auto do_step = [&](int64_t c0, int step, int& code, float& sc, float& mu) {
             uint32_t o[8][4];
+            int rel = -1;                   // packed stage to release once its data is consumed
             if (step < nks) {
                 const float c = __fmaf_rn((float)code, sc, mu);
                 fetch(c0, step + 2, code, sc, mu);
@@ -376,8 +382,7 @@ k_tc_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
                 const uint32_t src0 = pst + p_chunk_offset<BWD>(d, 0), src1 = pst + p_chunk_offset<BWD>(d, 1);
                 asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(p0.x), "=r"(p0.y), "=r"(p0.z), "=r"(p0.w) : "r"(src0));
                 asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(p1.x), "=r"(p1.y), "=r"(p1.z), "=r"(p1.w) : "r"(src1));
-                __syncwarp();
-                if (lane == 0) mbar_arrive(emptyP(sp));
+                rel = sp;
                 if (++sp == SP) { sp = 0; pp ^= 1; }
                 const BlockTable tb = make_block_table(tab, c);
                 const uint32_t pwd[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
@@ -393,17 +398,24 @@ k_tc_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
                     const int64_t n = c0 + drow;
                     rowok = n < a.N;
                     src = a.lora_w + n * a.ldl;
-                    col0 = (int64_t)lc * BK;        // rank index of chunk 0
+                    col0 = (int64_t)lc * BK;        // LoRA reduction index of chunk 0
                 } else {
-                    const int64_t i = (int64_t)lc * BK + drow;
-                    rowok = i < a.r;
+                    const int64_t ip = (int64_t)lc * BK + drow, i = ip >= a.lper ? ip - a.lper : ip;
+                    rowok = ip < 2 * a.lper && i < a.r;
                     src = a.lora_w + i * a.ldl;
                     col0 = c0 + dblk * 64;          // output column of chunk 0
                 }
 #pragma unroll
                 for (int ch = 0; ch < 8; ++ch) {
-                    const int64_t col = col0 + ch * 8;
-                    const bool v = rowok && (BWD ? (col < a.K) : (col < a.r));
+                    int64_t col = col0 + ch * 8;
+                    bool v;
+                    if (BWD) {
+                        v = rowok && col < a.K;
+                    } else {                        // rank index: the same B columns for hi and lo
+                        v = rowok && col < 2 * a.lper;
+                        if (col >= a.lper) col -= a.lper;
+                        v = v && col < a.r;
+                    }
                     uint4 q = make_uint4(0, 0, 0, 0);
                     if (v) q = __ldg(reinterpret_cast<const uint4*>(src + col));
                     o[ch][0] = q.x; o[ch][1] = q.y; o[ch][2] = q.z; o[ch][3] = q.w;
@@ -416,7 +428,14 @@ k_tc_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
                 st_shared_v4(wbase + w_chunk_offset<BWD>(d, ch), o[ch][0], o[ch][1], o[ch][2], o[ch][3]);
             fence_proxy_async();
             __syncwarp();
-            if (lane == 0) mbar_arrive(fullW(sw));
+            // The packed stage is released only now: the stores above consume the values
+            // decoded from it, so every lane's shared loads of it have returned.  A release
+            // right after the loads were issued let the next TMA copy overwrite the stage
+            // while some lanes' loads were still in flight.
+            if (lane == 0) {
+                mbar_arrive(fullW(sw));
+                if (rel >= 0) mbar_arrive(emptyP(rel));
+            }
             if (++sw == SW) { sw = 0; pw ^= 1; }
         };
         for (int64_t tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {

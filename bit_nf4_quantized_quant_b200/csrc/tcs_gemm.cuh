@@ -309,8 +309,6 @@ k_tcs_gemm(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUte
             const uint32_t src0 = pst + p_chunk_offset(d, 0), src1 = pst + p_chunk_offset(d, 1);
             asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(p0.x), "=r"(p0.y), "=r"(p0.z), "=r"(p0.w) : "r"(src0));
             asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(p1.x), "=r"(p1.y), "=r"(p1.z), "=r"(p1.w) : "r"(src1));
-            __syncwarp();
-            if (lane == 0) tc::mbar_arrive(emptyP(sp));
             const BlockTable tb = make_block_table(tab, c);
             const uint32_t pwd[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
             const int sw = i & (SW - 1), pw = (i / SW) & 1;
@@ -324,7 +322,13 @@ k_tcs_gemm(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUte
             }
             tc::fence_proxy_async();
             __syncwarp();
-            if (lane == 0) tc::mbar_arrive(fullW(sw));
+            // the packed stage is released only after the stores above, which consume the
+            // values decoded from it (a release right after the shared loads were issued let
+            // the next TMA copy overwrite the stage under loads still in flight)
+            if (lane == 0) {
+                tc::mbar_arrive(fullW(sw));
+                tc::mbar_arrive(emptyP(sp));
+            }
         };
         int codeA, codeB;
         float scA, scB, muA, muB;

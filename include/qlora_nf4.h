@@ -77,14 +77,20 @@ enum {
     QLORA_ERR_DEVICE = -6,      /* current device is not compute capability 10.0 */
     QLORA_ERR_LAUNCH = -7,      /* a CUDA launch or runtime call failed */
     QLORA_ERR_TIMEOUT = -8,     /* a device-side bounded wait gave up (see qlora_device_status) */
-    QLORA_ERR_VALUE = -9,       /* a scalar argument is not finite */
+    QLORA_ERR_VALUE = -9,       /* a scalar argument is not finite, or an unknown quant_type */
     QLORA_ERR_SCRATCH = -10     /* needs more than QLORA_NOALLOC_SCRATCH_BYTES (no-alloc entry point) */
 };
+
+/* 4-bit quant types ("Qlora Expert", Hyperparameter Guidance: the 4-bit
+ * quant type is "nf4" or "fp4"; "QLoRA Guide", FAQs: NF4 vs FP4). */
+#define QLORA_QUANT_NF4 0   /* NormalFloat: 16 levels at N(0,1) quantiles (nf4_codebook) */
+#define QLORA_QUANT_FP4 1   /* E2M1 4-bit float over its largest magnitude (quant4_codebook) */
 
 /* Quantized weight: all device pointers, caller-owned.
  *   packed [N, K/2] uint8: byte j of row n holds element 2j in its high
  *                          nibble and element 2j+1 in its low nibble; a
- *                          nibble is the index of an NF4 level (0..15).
+ *                          nibble indexes the quant type's 16-entry table L
+ *                          (nf4_codebook / quant4_codebook).
  *   codes  [N*K/64] int8 : code of block b = flat weights [64b, 64b+64)
  *   scale  [G] fp32, mean [G] fp32, G = ceil(N*K/64 / 256): group g covers
  *                          blocks [256g, 256g+256) of the flattened weight.
@@ -100,6 +106,8 @@ typedef struct {
     const float* mean;
     int64_t N;
     int64_t K;
+    int32_t quant_type;     /* QLORA_QUANT_NF4 or QLORA_QUANT_FP4: which 16-entry table L the nibbles
+                               index; any other value is rejected with QLORA_ERR_VALUE */
 } nf4dq_weight;
 
 /* The 16 NF4 levels in fp32, ascending (out16[0] = -1, out16[7] = 0,
@@ -109,6 +117,15 @@ typedef struct {
  * largest (the pages give only "levels at N(0,1) quantiles"; this is the
  * construction of the QLoRA paper they cite).  Host memory; no GPU needed. */
 QLORA_API int nf4_codebook(float out16[16]);
+
+/* The 16 levels of a quant type in fp32, indexed by nibble.  NF4: as
+ * nf4_codebook.  FP4 (a reading: the pages name the type but give no
+ * values): the E2M1 value of the nibble's bit pattern (bit 3 sign, bits 2..1
+ * exponent with bias 1, bit 0 mantissa; exponent 0 is subnormal: 0 or 0.5),
+ * divided by the largest magnitude 6 in double and rounded once to fp32:
+ * +-{0, 1/12, 1/6, 1/4, 1/3, 1/2, 2/3, 1}; nibbles 0 and 8 are +0 and -0.
+ * Host memory; returns QLORA_ERR_VALUE for another quant_type. */
+QLORA_API int quant4_codebook(int quant_type, float out16[16]);
 
 /* Element counts of a quantized [N, K] weight (host only, no GPU needed).
  * Any output pointer may be NULL. */
@@ -128,10 +145,38 @@ QLORA_API int nf4dq_sizes(int64_t N, int64_t K, int64_t* packed_bytes, int64_t* 
 QLORA_API int nf4_quantize_dq(const qlora_bf16* W, int64_t N, int64_t K, uint8_t* packed, int8_t* codes,
                     float* scale, float* mean, qlora_stream_t stream);
 
+/* nf4_quantize_dq for either quant type.  The encoder is the same nearest-
+ * level rule over that type's distinct levels in ascending order (thresholds
+ * halfway between neighbours, in fp32; exactly on a threshold goes to the
+ * lower level); the nibble written is the level's index in the table of
+ * quant4_codebook.  For FP4 a zero (and every weight of an all-zero block)
+ * is written as +0 (nibble 0).  quant_type other than NF4 / FP4:
+ * QLORA_ERR_VALUE. */
+QLORA_API int quant4_quantize_dq(const qlora_bf16* W, int64_t N, int64_t K, int quant_type, uint8_t* packed,
+                                 int8_t* codes, float* scale, float* mean, qlora_stream_t stream);
+
 /* Dequantize to a dense bf16 W' [N, K] (device, 16-byte aligned)
  * ("QLORA: Efficient Finetuning of Quantized LLMs", Notes: dequantize to
  * BF16).  Bit-exact with the definition under nf4dq_weight. */
 QLORA_API int nf4_dequant(const nf4dq_weight* w, qlora_bf16* W_out, qlora_stream_t stream);
+
+/* Dequantize-and-merge ("Qlora Expert", When to Use and Common Pitfalls: a
+ * dense model is obtained by dequantize-and-merge, since merging into the
+ * 4-bit weight is impossible -- merging requires dequantization; "QLoRA
+ * Implementation Details (2025 Edition)", Step 7: merge for inference).
+ * The dense bf16 weight of the adapted layer:
+ *   W_out[n, k] = bf16_rne( fmaf(scaling, d[n, k], w'[n, k]) )
+ *   d[n, k]     = sum over j = 0 .. r-1 of B[n, j] * A[j, k], accumulated in
+ *                 fp32 as d = fmaf(B[n, j], A[j, k], d) from d = 0 in
+ *                 increasing j (a fixed order, so the result is reproducible
+ *                 bit for bit)
+ *   w'[n, k]    = the dequantized weight bf16_rne(L[q] * c'_b) of nf4_dequant.
+ * A [r, K] bf16 (16-byte aligned), B [N, r] bf16, W_out [N, K] bf16
+ * (16-byte aligned), all device.  1 <= r <= QLORA_MAX_RANK; any N >= 1;
+ * K % 64 == 0, K <= QLORA_MAX_K.  With B = 0 the result equals nf4_dequant's
+ * in value.  Non-finite scaling: QLORA_ERR_VALUE. */
+QLORA_API int nf4_dequant_merge(const nf4dq_weight* w, const qlora_bf16* A, const qlora_bf16* B, int r,
+                                float scaling, qlora_bf16* W_out, qlora_stream_t stream);
 
 /* Bytes of device workspace that qlora_linear_fwd / qlora_linear_bwd need
  * for these sizes (0 is never returned for valid sizes; returns 0 for

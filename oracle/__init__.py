@@ -87,6 +87,18 @@ def lib():
         L.oracle_dequant.argtypes = [P, P, P, P, i64, i64, P]
         L.oracle_dequant_rows.restype = ctypes.c_int
         L.oracle_dequant_rows.argtypes = [P, P, P, P, i64, i64, P, i64, P]
+        i32 = ctypes.c_int
+        L.oracle_fp4_codebook.argtypes = [P, P]
+        L.oracle_codebook.restype = i32
+        L.oracle_codebook.argtypes = [i32, P]
+        L.oracle_encode_value_qt.restype = i32
+        L.oracle_encode_value_qt.argtypes = [i32, ctypes.c_float]
+        L.oracle_quantize_dq_qt.restype = i32
+        L.oracle_quantize_dq_qt.argtypes = [i32, P, i64, i64, P, P, P, P, P]
+        L.oracle_dequant_qt.restype = i32
+        L.oracle_dequant_qt.argtypes = [i32, P, P, P, P, i64, i64, P, i64, P]
+        L.oracle_dequant_merge.restype = i32
+        L.oracle_dequant_merge.argtypes = [i32, P, P, P, P, i64, i64, P, P, i32, ctypes.c_float, P, i64, P]
         _lib = L
     return _lib
 
@@ -193,6 +205,92 @@ def dequant_rows(q: dict, rows) -> np.ndarray:
                                    N, K, _ptr(rows), rows.size, _ptr(out))
     if rc != 0:
         raise ValueError("oracle_dequant_rows rejected its arguments")
+    return out
+
+
+# --------------------------------------------------------------------------
+# quant types: NF4 (the default) and the FP4 (E2M1) variant
+# --------------------------------------------------------------------------
+QUANT_NF4 = 0
+QUANT_FP4 = 1
+
+
+def codebook_qt(qt: int) -> np.ndarray:
+    """The nibble-indexed 16-entry fp32 table of a quant type."""
+    L = np.zeros(16, np.float32)
+    if lib().oracle_codebook(int(qt), _ptr(L)) == 0:
+        raise ValueError(f"unknown quant type {qt}")
+    return L
+
+
+def fp4_codebook():
+    """The FP4 (E2M1 / 6) table: (fp64 before rounding, fp32 as used)."""
+    v64 = np.zeros(16, np.float64)
+    v32 = np.zeros(16, np.float32)
+    lib().oracle_fp4_codebook(_ptr(v64), _ptr(v32))
+    return v64, v32
+
+
+def encode_value_qt(qt: int, x: float) -> int:
+    return int(lib().oracle_encode_value_qt(int(qt), ctypes.c_float(float(x))))
+
+
+def quantize_dq_qt(W_bits: np.ndarray, qt: int):
+    """quantize_dq for any quant type (NF4 or FP4)."""
+    W_bits = np.ascontiguousarray(W_bits, np.uint16)
+    N, K = W_bits.shape
+    nblocks = N * K // NF4_BLOCK
+    G = (nblocks + DQ_GROUP - 1) // DQ_GROUP
+    packed = np.zeros((N, K // 2), np.uint8)
+    codes = np.zeros(nblocks, np.int8)
+    scale = np.zeros(G, np.float32)
+    mean = np.zeros(G, np.float32)
+    absmax = np.zeros(nblocks, np.float32)
+    rc = lib().oracle_quantize_dq_qt(int(qt), _ptr(W_bits), N, K, _ptr(packed), _ptr(codes), _ptr(scale),
+                                     _ptr(mean), _ptr(absmax))
+    if rc != 0:
+        raise ValueError(f"oracle_quantize_dq_qt rejected its arguments ({rc})")
+    return dict(packed=packed, codes=codes, scale=scale, mean=mean, absmax=absmax, N=N, K=K, qt=int(qt))
+
+
+def dequant_qt(q: dict, rows=None) -> np.ndarray:
+    """bf16 W' (raw bits) of a quantized weight of any quant type, all rows or the listed ones."""
+    N, K = q["N"], q["K"]
+    qt = q.get("qt", QUANT_NF4)
+    if rows is None:
+        out = np.zeros((N, K), np.uint16)
+        rc = lib().oracle_dequant_qt(qt, _ptr(q["packed"]), _ptr(q["codes"]), _ptr(q["scale"]), _ptr(q["mean"]),
+                                     N, K, None, 0, _ptr(out))
+    else:
+        rows = np.ascontiguousarray(np.asarray(rows, np.int64))
+        out = np.zeros((rows.size, K), np.uint16)
+        rc = lib().oracle_dequant_qt(qt, _ptr(q["packed"]), _ptr(q["codes"]), _ptr(q["scale"]), _ptr(q["mean"]),
+                                     N, K, _ptr(rows), rows.size, _ptr(out))
+    if rc != 0:
+        raise ValueError(f"oracle_dequant_qt rejected its arguments ({rc})")
+    return out
+
+
+def dequant_merge(q: dict, A_bits: np.ndarray, B_bits: np.ndarray, s: float, rows=None) -> np.ndarray:
+    """Dequantize-and-merge: bf16 bits of W' + s B A, one fma per LoRA term in fp32
+    (see oracle_dequant_merge), for all rows or the listed ones."""
+    N, K = q["N"], q["K"]
+    A_bits = np.ascontiguousarray(A_bits, np.uint16)
+    B_bits = np.ascontiguousarray(B_bits, np.uint16)
+    r = A_bits.shape[0]
+    assert A_bits.shape == (r, K) and B_bits.shape == (N, r)
+    qt = q.get("qt", QUANT_NF4)
+    if rows is None:
+        out = np.zeros((N, K), np.uint16)
+        rp, nr = None, 0
+    else:
+        rows = np.ascontiguousarray(np.asarray(rows, np.int64))
+        out = np.zeros((rows.size, K), np.uint16)
+        rp, nr = _ptr(rows), rows.size
+    rc = lib().oracle_dequant_merge(qt, _ptr(q["packed"]), _ptr(q["codes"]), _ptr(q["scale"]), _ptr(q["mean"]),
+                                    N, K, _ptr(A_bits), _ptr(B_bits), r, ctypes.c_float(s), rp, nr, _ptr(out))
+    if rc != 0:
+        raise ValueError(f"oracle_dequant_merge rejected its arguments ({rc})")
     return out
 
 

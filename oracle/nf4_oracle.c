@@ -303,3 +303,168 @@ int oracle_dequant_rows(const uint8_t* packed, const int8_t* codes, const float*
     }
     return 0;
 }
+
+/* ===========================================================================
+ * The FP4 codebook variant ("Qlora Expert", Hyperparameter Guidance: the
+ * 4-bit quant type is "nf4" or "fp4"; "QLoRA Guide", FAQs: NF4 vs FP4).
+ * The pages give no FP4 values.  Reading: the 4-bit float E2M1 (1 sign,
+ * 2 exponent, 1 mantissa bit; magnitudes 0, 0.5, 1, 1.5, 2, 3, 4, 6), the
+ * nibble being the E2M1 bit pattern itself (sign in bit 3), normalised to
+ * [-1, 1] by dividing by the largest magnitude 6 in fp64 and rounding once
+ * to fp32.  Codes 0 and 8 are +0 and -0; the encoder only emits +0.
+ * Everything else (blocks of 64, absmax, the double quantization, the
+ * dequantized weight bf16_rne(L[q] * c')) is the same as for NF4; only the
+ * 16-entry table and the encoder's level order change.
+ * ========================================================================= */
+#define QUANT_NF4 0
+#define QUANT_FP4 1
+
+void oracle_fp4_codebook(double out64[16], float out32[16])
+{
+    static const double mag[8] = {0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0};
+    for (int code = 0; code < 16; ++code) {
+        double v = mag[code & 7] / 6.0;
+        if (code & 8) v = -v;
+        out64[code] = v;
+        out32[code] = (float)v;
+    }
+}
+
+/* The levels of a quant type as nibble-indexed table L, and its distinct
+ * levels in ascending order as nibble codes (nlev of them). */
+static int codebook_of(int qt, float L[16], int sorted_code[16])
+{
+    double L64[16];
+    if (qt == QUANT_NF4) {
+        oracle_nf4_codebook(L64, L);
+        for (int i = 0; i < 16; ++i) sorted_code[i] = i;
+        return 16;
+    }
+    if (qt == QUANT_FP4) {
+        oracle_fp4_codebook(L64, L);
+        int n = 0;
+        for (int code = 15; code >= 9; --code) sorted_code[n++] = code;   /* -1 .. -1/12 */
+        for (int code = 0; code <= 7; ++code) sorted_code[n++] = code;    /* 0 .. 1 */
+        return n;                                                          /* 15: -0 is not emitted */
+    }
+    return 0;
+}
+
+/* The 16-entry table of a quant type (nibble-indexed); returns the number of
+ * distinct levels, 0 for an unknown type. */
+int oracle_codebook(int qt, float out32[16])
+{
+    int sc[16];
+    return codebook_of(qt, out32, sc);
+}
+
+/* Reading R2 for any codebook: thresholds between neighbouring distinct
+ * levels m_i = fl32((s_i + s_{i+1}) / 2); the level is the number of
+ * thresholds x lies strictly above; its nibble is that level's code. */
+int oracle_encode_value_qt(int qt, float x)
+{
+    float L[16], m[15];
+    int sc[16];
+    int n = codebook_of(qt, L, sc);
+    for (int i = 0; i + 1 < n; ++i) m[i] = (L[sc[i]] + L[sc[i + 1]]) * 0.5f;
+    int q = 0;
+    for (int i = 0; i + 1 < n; ++i)
+        if (x > m[i]) ++q;
+    return sc[q];
+}
+
+/* Quantize + double-quantize with the given quant type (see oracle_quantize_dq). */
+int oracle_quantize_dq_qt(int qt, const uint16_t* W, int64_t N, int64_t K, uint8_t* packed, int8_t* codes,
+                          float* scale, float* mean, float* absmax_scratch)
+{
+    if (N <= 0 || K <= 0 || (K % NF4_BLOCK) != 0) return -1;
+    float L[16], m[15];
+    int sc[16];
+    int n = codebook_of(qt, L, sc);
+    if (n == 0) return -3;
+    for (int i = 0; i + 1 < n; ++i) m[i] = (L[sc[i]] + L[sc[i + 1]]) * 0.5f;
+    int zero_code = -1;
+    for (int i = 0; i < n; ++i)
+        if (L[sc[i]] == 0.0f) { zero_code = sc[i]; break; }
+    int64_t nblocks = N * K / NF4_BLOCK;
+    oracle_block_absmax(W, nblocks, absmax_scratch);
+    for (int64_t b = 0; b < nblocks; ++b) {
+        float c = absmax_scratch[b];
+        for (int j = 0; j < NF4_BLOCK; j += 2) {
+            int q[2];
+            for (int h = 0; h < 2; ++h) {
+                if (c == 0.0f) {
+                    q[h] = zero_code;
+                } else {
+                    float x = oracle_bf16_to_f32(W[b * NF4_BLOCK + j + h]) / c;
+                    int k = 0;
+                    for (int i = 0; i + 1 < n; ++i)
+                        if (x > m[i]) ++k;
+                    q[h] = sc[k];
+                }
+            }
+            packed[(b * NF4_BLOCK + j) / 2] = (uint8_t)((q[0] << 4) | q[1]);
+        }
+    }
+    oracle_double_quant(absmax_scratch, nblocks, codes, scale, mean);
+    return 0;
+}
+
+/* W' = bf16_rne(L[q] * c'_b) for the listed rows, with the given quant type
+ * (rows = NULL: every row, in order). */
+int oracle_dequant_qt(int qt, const uint8_t* packed, const int8_t* codes, const float* scale, const float* mean,
+                      int64_t N, int64_t K, const int64_t* rows, int64_t nrows, uint16_t* Wout)
+{
+    if (N <= 0 || K <= 0 || (K % NF4_BLOCK) != 0) return -1;
+    float L[16];
+    int sc[16];
+    if (codebook_of(qt, L, sc) == 0) return -3;
+    if (rows == NULL) nrows = N;
+    for (int64_t ri = 0; ri < nrows; ++ri) {
+        int64_t n = rows ? rows[ri] : ri;
+        if (n < 0 || n >= N) return -2;
+        for (int64_t k = 0; k < K; ++k) {
+            int64_t e = n * K + k;
+            int64_t b = e / NF4_BLOCK;
+            int64_t g = b / DQ_GROUP;
+            float cp = oracle_block_constant(codes[b], scale[g], mean[g]);
+            uint8_t byte = packed[e / 2];
+            int q = (e % 2 == 0) ? (byte >> 4) : (byte & 0x0f);
+            Wout[ri * K + k] = oracle_f32_to_bf16(L[q] * cp);
+        }
+    }
+    return 0;
+}
+
+/* ===========================================================================
+ * Dequantize-and-merge ("Qlora Expert", When to Use / Common Pitfalls: a
+ * dense model needs dequantize-and-merge, since merging requires
+ * dequantization; "QLoRA Implementation Details (2025 Edition)", Step 7:
+ * merge for inference).  The dense weight of the trained layer is the
+ * dequantized base plus the scaled LoRA product:
+ *   W_merged[n, k] = bf16_rne( fmaf(s, d[n, k], w'[n, k]) ),
+ *   d[n, k] = sum_j B[n, j] A[j, k]   in fp32, j = 0, 1, ..., r-1, one fmaf
+ *             per term starting from 0 (the first term is exact),
+ *   w'[n, k] the dequantized weight (bf16, as the forward multiplies with it).
+ * A [r, K] and B [N, r] are bf16; rows = NULL merges every row in order.
+ * ========================================================================= */
+int oracle_dequant_merge(int qt, const uint8_t* packed, const int8_t* codes, const float* scale, const float* mean,
+                         int64_t N, int64_t K, const uint16_t* A, const uint16_t* B, int r, float s,
+                         const int64_t* rows, int64_t nrows, uint16_t* Wout)
+{
+    if (r < 1) return -4;
+    int rc = oracle_dequant_qt(qt, packed, codes, scale, mean, N, K, rows, nrows, Wout);
+    if (rc != 0) return rc;
+    if (rows == NULL) nrows = N;
+    for (int64_t ri = 0; ri < nrows; ++ri) {
+        int64_t n = rows ? rows[ri] : ri;
+        for (int64_t k = 0; k < K; ++k) {
+            float d = 0.0f;
+            for (int j = 0; j < r; ++j)
+                d = fmaf(oracle_bf16_to_f32(B[n * r + j]), oracle_bf16_to_f32(A[(int64_t)j * K + k]), d);
+            float w = oracle_bf16_to_f32(Wout[ri * K + k]);
+            Wout[ri * K + k] = oracle_f32_to_bf16(fmaf(s, d, w));
+        }
+    }
+    return 0;
+}

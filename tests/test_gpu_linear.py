@@ -208,3 +208,62 @@ def test_workload1_full(oracle_mod, proj):
 @pytest.mark.parametrize("proj,M", [(0, 1), (0, 4), (1, 8), (1, 32)])
 def test_workload2_decode(oracle_mod, proj, M):
     _sampled_rows_parity(oracle_mod, inputs.WORKLOADS[2], proj, M, rows_n=M, bwd=False)
+
+
+@pytest.mark.parametrize("M,N,K,r", [(512, 28672, 1024, 64), (384, 1024, 11008, 16)])
+def test_multi_tile_pair_kernel_repeats_bit_identically(oracle_mod, M, N, K, r):
+    """Several SM-pair tiles per pair, two LoRA steps per tile (r = 64): five runs of the
+    forward and backward must agree bit for bit (the reduction orders are fixed, so any
+    difference is a race) and the first must match the oracle."""
+    s = 16.0 / r
+    W, X, A, B, dY, Wd, w = _setup(oracle_mod, M, N, K, r, seed=7)
+    Xc, Ac, Bc, dYc = X.cuda(), A.cuda(), B.cuda(), dY.cuda()
+    outs = []
+    for _ in range(5):
+        Y = ops.qlora_linear_fwd(Xc, w, Ac, Bc, s)
+        dX, dA, dB = ops.qlora_linear_bwd(Xc, dYc, w, Ac, Bc, s)
+        outs.append([t.cpu() for t in (Y, dX, dA, dB)])
+    torch.cuda.synchronize()
+    assert ops.qlora_device_status() == 0
+    assert ops.qlora_last_path() == 3
+    for o in outs[1:]:
+        for a, b in zip(outs[0], o):
+            assert torch.equal(a, b)
+    X64, A64, B64, dY64 = (inputs.to_f64(t) for t in (X, A, B, dY))
+    Yr, _ = oracle_mod.linear_fwd(X64, Wd, A64, B64, s)
+    dXr, dAr, dBr = oracle_mod.linear_bwd(X64, dY64, Wd, A64, B64, s)
+    for name, got, ref in zip(("Y", "dX", "dA", "dB"), outs[0], (Yr, dXr, dAr, dBr)):
+        _close(inputs.to_f64(got), ref, name)
+
+
+@pytest.mark.parametrize("M,N,K,r,bwd", [(512, 28672, 1024, 16, False),   # SM pairs, 224 tiles
+                                         (512, 4096, 11008, 64, True),    # SM pairs, backward over 11008
+                                         (100, 38912, 256, 16, False),    # single SM, 152 tiles
+                                         (64, 512, 38912, 8, True),       # single SM, backward, 152 tiles
+                                         (16, 4096, 28672, 64, True)])    # small-M backward (tcgen05)
+def test_fused_kernels_repeat_bit_identically(M, N, K, r, bwd):
+    """Fifty back-to-back calls give bit-identical outputs.  Every reduction order is fixed,
+    so a difference can only come from a race between a stage's producer and its consumers
+    (this caught packed stages being released while their shared loads were in flight)."""
+    s = 16.0 / r
+    W = inputs.weight(57, 0, N, K, 0.02, device="cuda")
+    X = inputs.normal(67, (M, K), 1.0, "cuda")
+    A = inputs.uniform(68, (r, K), 1.0 / np.sqrt(K), "cuda")
+    B = inputs.normal(69, (N, r), 0.1, "cuda")
+    dY = inputs.normal(70, (M, N), 1.0, "cuda")
+    w = ops.nf4_quantize_dq(W)
+    ws = ops.workspace(M, N, K, r)
+    first = None
+    same = torch.ones((), dtype=torch.bool, device="cuda")
+    for _ in range(50):
+        if bwd:
+            out = ops.qlora_linear_bwd(X, dY, w, A, B, s, ws=ws)[0]
+        else:
+            out = ops.qlora_linear_fwd(X, w, A, B, s, ws=ws)
+        if first is None:
+            first = out.clone()
+        else:
+            same &= torch.equal(out, first)
+    torch.cuda.synchronize()
+    assert ops.qlora_device_status() == 0
+    assert bool(same)
