@@ -36,6 +36,9 @@ if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
 METRIC = "QLoRA linear fwd+bwd TFLOP/s & NF4 weight-stream GB/s; % of roofline, 1×B200"
+QUANT = {"nf4": 0, "fp4": 1}
+# fp32 fused multiply-adds per cycle per SM of B200 (4 sub-partitions x 32 lanes)
+FMA_PER_SM_CYCLE = 128
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 # dram__bytes_read.sum + dram__bytes_write.sum of the dominant kernel, averaged over its launches
@@ -196,8 +199,8 @@ def run_ours(args, rank, world, local_rank):
     layers = []
     for i, p in enumerate(projs):
         W = inputs.layer_weight(wl, i, device=dev)
-        w = ops.nf4_quantize_dq(W)
-        ws_copies = [w] + [ops.nf4_quantize_dq(W) for _ in range(copies - 1)]
+        w = ops.quant4_quantize_dq(W, QUANT[args.quant])
+        ws_copies = [w] + [ops.quant4_quantize_dq(W, QUANT[args.quant]) for _ in range(copies - 1)]
         del W
         _, A, B, _ = inputs.layer_inputs(wl, i, M, device=dev, with_dy=False)
         X, dY = rank_batch(wl, i, M, rank, world, dev)
@@ -470,7 +473,8 @@ def run_ours(args, rank, world, local_rank):
         ems = float(tt.item())
     e2e_val = (flops_step if not small else bytes_step) * world / (ems / args.steps * 1e-3) / (1e12 if not small else 1e9)
 
-    cfg = {"workload": wl.name, "projections": [f"{p.name} {p.N}x{p.K}" for p in projs], "M_per_gpu": M,
+    cfg = {"workload": wl.name, "quant_type": args.quant,
+           "projections": [f"{p.name} {p.N}x{p.K}" for p in projs], "M_per_gpu": M,
            "global_batch_tokens": M * world, "r": r, "alpha": wl.alpha, "weights": "NF4 + double-quant (64/256)",
            "step": "qlora_linear_fwd + qlora_linear_bwd for every projection" +
                    (" + NCCL all-reduce of dA,dB" if world > 1 else ""),
@@ -487,7 +491,7 @@ def run_ours(args, rank, world, local_rank):
                               "in order on the compute stream") + "; all inside the timed region"},
            "gpu_launches": launches, "clocks": clk}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        out["cpu_baseline"] = cpu_baseline(wl, M, budget_s=args.cpu_seconds)
+        out["cpu_baseline"] = cpu_baseline(wl, M, budget_s=args.cpu_seconds, quant=args.quant)
     return out
 
 
@@ -595,6 +599,112 @@ def run_bulk(args, rank, world, local_rank):
     return out
 
 
+def run_merge(args, rank, world, local_rank):
+    """Dequantize-and-merge of the 7 projections of the 7B block (r = 16, s = 2):
+    W' + s B A in bf16, one nf4_dequant_merge per projection per step.  Each rank
+    merges its own copy (weak scaling)."""
+    import torch
+
+    from bit_nf4_quantized_quant_b200 import _ops as ops
+    from bit_nf4_quantized_quant_b200 import inputs
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    wl = inputs.WORKLOADS[3]
+    peaks, peak_src = load_peaks()
+    r, s = wl.r, wl.scaling
+    layers = []
+    for i, p in enumerate(wl.projections):
+        W = inputs.layer_weight(wl, i, device=dev)
+        w = ops.quant4_quantize_dq(W, QUANT[args.quant])
+        del W
+        _, A, B, _ = inputs.layer_inputs(wl, i, 1, device=dev, with_dy=False)
+        layers.append((w, A, B, torch.empty((p.N, p.K), dtype=torch.bfloat16, device=dev)))
+    stream = torch.cuda.current_stream()
+
+    def step(ev=None):
+        for j, (w, A, B, out) in enumerate(layers):
+            if ev: ev[j][0].record(stream)
+            ops.nf4_dequant_merge(w, A, B, s, out=out)
+            if ev: ev[j][1].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in layers]
+    torch.cuda.synchronize()
+    clocks = ClockSampler(local_rank)
+    clocks.start()
+    l0 = ops.qlora_launch_count()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for k in range(args.steps):
+        step(ev if k == args.steps - 1 else None)
+    t1.record(stream)
+    torch.cuda.synchronize()
+    launches = ops.qlora_launch_count() - l0
+    clk = clocks.stop()
+    assert ops.qlora_device_status() == 0
+    ms = t0.elapsed_time(t1) / args.steps
+    params = sum(p.N * p.K for p in wl.projections)
+    step_bytes = sum(nf4_bytes(p.N, p.K) + 2 * p.N * p.K + 2 * r * (p.N + p.K) for p in wl.projections)
+    step_flops = sum(2 * p.N * p.K * r for p in wl.projections)
+    kms = sum(a.elapsed_time(b) for a, b in ev)
+    mhz = peaks.get("sm_max_mhz", 1965.0)
+    fma_peak = 148 * FMA_PER_SM_CYCLE * 2 * mhz * 1e6 / 1e12
+    achieved = step_flops / (kms * 1e-3) / 1e12
+    roof = {"bound": "alu", "unit": "TFLOP/s", "achieved": round(achieved, 2), "peak": round(fma_peak, 1),
+            "frac": round(achieved / fma_peak, 4), "traffic": None,
+            "peak_source": f"fp32 fma pipe: 148 SMs x {FMA_PER_SM_CYCLE} fma/cycle x 2 flop x {mhz:.0f} MHz "
+                           f"(sm_max_mhz, {peak_src})",
+            "kernel": "k_dequant_merge", "launches_timed": len(layers),
+            "avg_launch_us": round(kms / len(layers) * 1e3, 2),
+            "hbm": {"achieved_GBps": round(step_bytes / (kms * 1e-3) / 1e9, 1), "peak": peaks["hbm_gbs"],
+                    "frac": round(step_bytes / (kms * 1e-3) / 1e9 / peaks["hbm_gbs"], 4)}}
+    out = {"metric": METRIC, "value": round(step_bytes / (ms * 1e-3) / 1e9, 1), "unit": "GB/s", "n_gpus": world,
+           "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 4), "higher_is_better": True,
+           "scaling": "weak", "vs_baseline": None, "dtype": "NF4/FP4 + bf16 adapters -> bf16 (fp32 fma chain)",
+           "data": "synthetic (seeded)",
+           "config": {"workload": "dequantize-and-merge llama7b block (7 projections)", "quant_type": args.quant,
+                      "r": r, "alpha": wl.alpha, "params": params,
+                      "step": "nf4_dequant_merge of every projection",
+                      "l2": f"inputs larger than L2: {step_bytes / 1e6:.0f} MB per step"},
+           "roofline": roof, "gpu_launches": launches, "clocks": clk}
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        out["cpu_baseline"] = merge_cpu_baseline(wl, args.quant)
+    return out
+
+
+def merge_cpu_baseline(wl, quant, rows=64):
+    """The oracle's dequantize-and-merge on `rows` rows of each projection (C, one
+    thread per projection), scaled to the whole weight (every row costs the same)."""
+    from concurrent.futures import ThreadPoolExecutor
+
+    import numpy as np
+
+    import oracle
+    from bit_nf4_quantized_quant_b200 import inputs
+    jobs = []
+    for i, p in enumerate(wl.projections):
+        W = inputs.layer_weight(wl, i)
+        q = oracle.quantize_dq_qt(inputs.bf16_bits(W), QUANT[quant])
+        _, A, B, _ = inputs.layer_inputs(wl, i, 1, with_dy=False)
+        jobs.append((q, inputs.bf16_bits(A), inputs.bf16_bits(B), np.arange(rows) * (p.N // rows)))
+
+    def one(job):
+        q, A, B, rr = job
+        t0 = time.perf_counter()
+        oracle.dequant_merge(q, A, B, wl.scaling, rows=rr)
+        return time.perf_counter() - t0
+
+    with ThreadPoolExecutor(len(jobs)) as pool:
+        times = list(pool.map(one, jobs))
+    full = sum(t * p.N / rows for t, p in zip(times, wl.projections))      # serial-equivalent seconds
+    step_bytes = sum(nf4_bytes(p.N, p.K) + 2 * p.N * p.K + 2 * wl.r * (p.N + p.K) for p in wl.projections)
+    return {"value": round(step_bytes / full / 1e9, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
+            "sample": f"{rows} rows of each of the 7 projections merged by the C oracle ({sum(times):.1f} s), "
+                      f"time scaled by N/{rows} per projection (extrapolated), one core per projection counted serially"}
+
+
 def _threads():
     try:
         from threadpoolctl import threadpool_info
@@ -636,7 +746,7 @@ class OracleStep:
     in these products, so the extrapolation is linear and is labelled as such.
     Quantization happens once before timing, as at model load."""
 
-    def __init__(self, wl, M, rows=64):
+    def __init__(self, wl, M, rows=64, quant="nf4"):
         import numpy as np
         from concurrent.futures import ThreadPoolExecutor
 
@@ -649,7 +759,7 @@ class OracleStep:
         self.state = []
         for i, p in enumerate(wl.projections):
             W = inputs.layer_weight(wl, i)
-            q = oracle.quantize_dq(inputs.bf16_bits(W))
+            q = oracle.quantize_dq_qt(inputs.bf16_bits(W), QUANT[quant])
             X, A, B, dY = inputs.layer_inputs(wl, i, self.rows, with_dy=wl.backward)
             self.state.append((q, inputs.to_f64(X), inputs.to_f64(A), inputs.to_f64(B),
                                inputs.to_f64(dY) if dY is not None else None,
@@ -665,7 +775,7 @@ class OracleStep:
         s = self.wl.scaling
         for q, X, A, B, dY, chunks in self.state:
             t0 = time.perf_counter()
-            parts = list(self.pool.map(lambda rr: oracle.dequant_rows(q, rr), chunks))
+            parts = list(self.pool.map(lambda rr: oracle.dequant_qt(q, rr), chunks))
             Wd = oracle.bf16_to_f32(np.concatenate(parts)).astype(np.float64)
             t1 = time.perf_counter()
             oracle.linear_fwd(X, Wd, A, B, s)
@@ -687,11 +797,11 @@ class OracleStep:
                 f"by {self.M}/{self.rows} (extrapolated); quantization once, untimed")
 
 
-def cpu_baseline(wl, M, budget_s=20.0):
+def cpu_baseline(wl, M, budget_s=20.0, quant="nf4"):
     """The oracle, as it stands, on the host cores over a bounded sample."""
     if wl.index == 5:
         return bulk_cpu_baseline(wl)
-    st = OracleStep(wl, M)
+    st = OracleStep(wl, M, quant=quant)
     st.run()                                     # warm: first touch of the fp64 buffers
     t0 = time.perf_counter()
     times = []
@@ -764,12 +874,16 @@ def sub_results(args, rank, world, local_rank):
 
     import torch
     subs = []
-    for wlx, M in ((2, 1), (1, 16), (5, 0)):
+    for wlx, M, op, quant in ((2, 1, "linear", "nf4"), (1, 16, "linear", "nf4"), (5, 0, "linear", "nf4"),
+                              (2, 1, "linear", "fp4"), (3, 0, "merge", "nf4")):
         torch.cuda.empty_cache()
         a = copy.copy(args)
-        a.workload, a.M = wlx, M
+        a.workload, a.M, a.op, a.quant = wlx, M, op, quant
         a.cpu_seconds = min(args.cpu_seconds, 8.0)
-        o = run_bulk(a, rank, world, local_rank) if wlx == 5 else run_ours(a, rank, world, local_rank)
+        if op == "merge":
+            o = run_merge(a, rank, world, local_rank)
+        else:
+            o = run_bulk(a, rank, world, local_rank) if wlx == 5 else run_ours(a, rank, world, local_rank)
         o.pop("metric", None)
         o["config"]["M"] = M
         subs.append(o)
@@ -786,6 +900,9 @@ def main():
                     help="0 (default): the 7B block at M = 2048 as the headline line, with the decode GEMV (M = 1), "
                          "the single 4096^2 linear (M = 16) and the bulk quantize round trip as sub_results")
     ap.add_argument("--no-sub", action="store_true", help="default workload: skip the sub_results")
+    ap.add_argument("--quant", choices=["nf4", "fp4"], default="nf4", help="4-bit quant type of the frozen weights")
+    ap.add_argument("--op", choices=["linear", "merge"], default="linear",
+                    help="merge: time nf4_dequant_merge over the 7B block's projections instead")
     ap.add_argument("--layers", type=int, default=0, help="workload 5: number of 7-tensor layers (default 32)")
     ap.add_argument("--M", type=int, default=0, help="tokens per GPU (default: the workload's largest)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -816,8 +933,13 @@ def main():
         dist.barrier()
     build_lib()
     try:
-        out = run_bulk(args, rank, world, local_rank) if args.workload == 5 else run_ours(args, rank, world, local_rank)
-        if args.workload == 0 and world == 1 and not args.no_sub:
+        if args.op == "merge":
+            out = run_merge(args, rank, world, local_rank)
+        elif args.workload == 5:
+            out = run_bulk(args, rank, world, local_rank)
+        else:
+            out = run_ours(args, rank, world, local_rank)
+        if args.workload == 0 and args.op == "linear" and world == 1 and not args.no_sub:
             out["sub_results"] = sub_results(args, rank, world, local_rank)
         if rank == 0:
             print(json.dumps(out), flush=True)

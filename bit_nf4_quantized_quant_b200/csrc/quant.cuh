@@ -64,7 +64,11 @@ __global__ void __launch_bounds__(256, 4) k_quantize_dq(const uint16_t* __restri
     __shared__ float s_c[kGroup];
     __shared__ float s_m[16];
     __shared__ float2 s_enc[kEncBuckets];          // (threshold, levels below) per bucket
-    if (threadIdx.x < 15) s_m[threadIdx.x] = tab.m[threadIdx.x];
+    // constant indices (a thread-dependent index into the by-value table would make every
+    // thread copy the whole parameter to local memory first)
+#pragma unroll
+    for (int q = 0; q < 15; ++q)
+        if (threadIdx.x == q) s_m[q] = tab.m[q];
     if (threadIdx.x == 15) s_m[15] = INFINITY;
     for (int b = threadIdx.x; b < kEncBuckets; b += blockDim.x)
         s_enc[b] = make_float2(enc.thr[b], __uint_as_float(enc.qb[b]));
