@@ -97,6 +97,16 @@ def lib():
         L.oracle_quantize_dq_qt.argtypes = [i32, P, i64, i64, P, P, P, P, P]
         L.oracle_dequant_qt.restype = i32
         L.oracle_dequant_qt.argtypes = [i32, P, P, P, P, i64, i64, P, i64, P]
+        L.oracle_e4m3_to_f32.restype = ctypes.c_float
+        L.oracle_e4m3_to_f32.argtypes = [ctypes.c_uint8]
+        L.oracle_f32_to_e4m3.restype = ctypes.c_uint8
+        L.oracle_f32_to_e4m3.argtypes = [ctypes.c_float]
+        L.oracle_adamw8_step.restype = i32
+        L.oracle_adamw8_step.argtypes = [P, P, i64, P, P, P, P, i64, ctypes.c_float, ctypes.c_float, ctypes.c_float,
+                                         ctypes.c_float, ctypes.c_float]
+        L.oracle_philox4x64.argtypes = [P, P, P]
+        L.oracle_dropout_mask.restype = i32
+        L.oracle_dropout_mask.argtypes = [ctypes.c_uint64, ctypes.c_uint64, i64, i64, ctypes.c_float, P]
         L.oracle_dequant_merge.restype = i32
         L.oracle_dequant_merge.argtypes = [i32, P, P, P, P, i64, i64, P, P, i32, ctypes.c_float, P, i64, P]
         _lib = L
@@ -295,6 +305,67 @@ def dequant_merge(q: dict, A_bits: np.ndarray, B_bits: np.ndarray, s: float, row
 
 
 # --------------------------------------------------------------------------
+# 8-bit AdamW step of the adapters (E4M3 states, blocks of 256)
+# --------------------------------------------------------------------------
+ADAM_BLOCK = 256
+
+
+def e4m3_to_f32(code: int) -> float:
+    return float(lib().oracle_e4m3_to_f32(ctypes.c_uint8(int(code))))
+
+
+def f32_to_e4m3(x: float) -> int:
+    return int(lib().oracle_f32_to_e4m3(ctypes.c_float(float(x))))
+
+
+def adamw8_state(n: int):
+    """Zero 8-bit moment states for n parameters: (m_code, m_scale, v_code, v_scale)."""
+    nb = (n + ADAM_BLOCK - 1) // ADAM_BLOCK
+    return (np.zeros(n, np.uint8), np.zeros(nb, np.float32), np.zeros(n, np.uint8), np.zeros(nb, np.float32))
+
+
+def adamw8_step(p_bits: np.ndarray, g_bits: np.ndarray, state, step: int, lr: float, b1: float, b2: float,
+                eps: float, wd: float):
+    """One AdamW step in place: p_bits (bf16 bits, updated), state (updated)."""
+    m_code, m_scale, v_code, v_scale = state
+    for a in (p_bits, g_bits, m_code, m_scale, v_code, v_scale):
+        assert a.flags["C_CONTIGUOUS"]
+    n = p_bits.size
+    assert g_bits.size == n and m_code.size == n and v_code.size == n
+    rc = lib().oracle_adamw8_step(_ptr(p_bits), _ptr(g_bits), n, _ptr(m_code), _ptr(m_scale), _ptr(v_code),
+                                  _ptr(v_scale), int(step), ctypes.c_float(lr), ctypes.c_float(b1),
+                                  ctypes.c_float(b2), ctypes.c_float(eps), ctypes.c_float(wd))
+    if rc != 0:
+        raise ValueError(f"oracle_adamw8_step rejected its arguments ({rc})")
+
+
+# --------------------------------------------------------------------------
+# LoRA dropout: Philox4x64-10 keep mask of the LoRA branch's input
+# --------------------------------------------------------------------------
+def philox4x64(counter, key) -> np.ndarray:
+    c = np.ascontiguousarray(np.asarray(counter, np.uint64))
+    k = np.ascontiguousarray(np.asarray(key, np.uint64))
+    out = np.zeros(4, np.uint64)
+    lib().oracle_philox4x64(_ptr(c), _ptr(k), _ptr(out))
+    return out
+
+
+def dropout_mask(seed: int, offset: int, M: int, K: int, p: float) -> np.ndarray:
+    """Keep mask [M, K] (bool) of the LoRA dropout with rate p."""
+    keep = np.zeros((M, K), np.uint8)
+    rc = lib().oracle_dropout_mask(ctypes.c_uint64(seed), ctypes.c_uint64(offset), M, K, ctypes.c_float(p),
+                                   _ptr(keep))
+    if rc != 0:
+        raise ValueError("oracle_dropout_mask rejected its arguments")
+    return keep.astype(bool)
+
+
+def dropout_scale(p: float) -> float:
+    """The scale of kept values, fl32(1 / (1 - p)) for the fp32 rate p."""
+    return float(np.float32(1.0 / (1.0 - float(np.float32(p)))))
+
+
+# --------------------------------------------------------------------------
 # linear layer forward / backward, fp64 definitions
 # --------------------------------------------------------------------------
 def lora_scaling(r: int, alpha: float) -> float:
@@ -337,3 +408,31 @@ def linear_bwd_adapters(X, dY, A, B, s):
     T = X @ np.asarray(A, np.float64).T
     U = dY @ np.asarray(B, np.float64)
     return s * (U.T @ X), s * (dY.T @ T)
+
+
+def linear_fwd_dropout(X, Wd, A, B, s, keep, c):
+    """Forward with LoRA dropout on the branch input: Y = X W'^T + s (Xd A^T) B^T,
+    Xd = X * keep * c (keep the mask, c the scale of kept values); returns (Y, T)."""
+    X = np.asarray(X, np.float64)
+    Xd = X * np.asarray(keep, np.float64) * c
+    T = Xd @ np.asarray(A, np.float64).T
+    Y = X @ np.asarray(Wd, np.float64).T + s * (T @ np.asarray(B, np.float64).T)
+    return Y, T
+
+
+def linear_bwd_dropout(X, dY, Wd, A, B, s, keep, c):
+    """Gradients of <Y, dY> for linear_fwd_dropout with the mask held fixed:
+    U = dY B, dX = dY W' + s (U A) * keep * c, dA = s U^T Xd, dB = s dY^T T."""
+    X = np.asarray(X, np.float64)
+    dY = np.asarray(dY, np.float64)
+    A = np.asarray(A, np.float64)
+    B = np.asarray(B, np.float64)
+    km = np.asarray(keep, np.float64) * c
+    Xd = X * km
+    T = Xd @ A.T
+    U = dY @ B
+    dX = dY @ np.asarray(Wd, np.float64) + s * (U @ A) * km
+    dA = s * (U.T @ Xd)
+    dB = s * (dY.T @ T)
+    return dX, dA, dB
+

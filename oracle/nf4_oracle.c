@@ -468,3 +468,180 @@ int oracle_dequant_merge(int qt, const uint8_t* packed, const int8_t* codes, con
     }
     return 0;
 }
+
+/* ===========================================================================
+ * 8-bit AdamW step for the LoRA adapters ("Qlora Expert", Hyperparameter
+ * Guidance and Memory Math: paged_adamw_8bit, 8-bit Adam to cut optimizer
+ * memory; "QLoRA Implementation Details (2025 Edition)", Step 5: Paged
+ * Optimizer).  The paging (unified memory) is driver behaviour and not part
+ * of the step.  The pages name the optimizer but give no state encoding.
+ * Reading: both moments are stored blockwise like the weights -- blocks of
+ * 256 consecutive parameters, one fp32 scale per block, and one 8-bit code
+ * per parameter, the code being an FP8 E4M3 number (1 sign, 4 exponent bits
+ * with bias 7, 3 mantissa bits, largest finite 448), so that
+ *   state value = fl32(e4m3(code) * scale_b),  scale_b = fl32(absmax_b / 448),
+ *   code        = e4m3_rne_saturating(fl32(x * inv_b)), inv_b = fl32(448 / absmax_b),
+ *                 0 if absmax_b = 0.
+ * The update is AdamW with decoupled weight decay, every operation one IEEE
+ * fp32 rounding in this order (g, p are bf16 widened exactly):
+ *   m  = b1 * m + omb1 * g                 (two products, then the sum)
+ *   v  = b2 * v + omb2 * (g * g)
+ *   mh = m * rbc1,  vh = v * rbc2
+ *   u  = mh / (sqrt(vh) + eps) + wd * p
+ *   p  = bf16_rne(p - lr * u)
+ * with omb1 = fl32(1 - b1), omb2 = fl32(1 - b2), rbc1 = fl32(1 / (1 - b1^t)),
+ * rbc2 = fl32(1 / (1 - b2^t)) computed in double from the fp32 b1, b2 and the
+ * step t (the bias corrections and the block scales enter as reciprocals, so
+ * that one division and one square root per parameter remain).  The new m, v
+ * of a block are then requantized with that block's new absmax.
+ * ========================================================================= */
+#define ADAM_BLOCK 256
+#define E4M3_MAX 448.0f
+
+/* Value of an E4M3 code (the 0x7f / 0xff NaN patterns are never produced). */
+float oracle_e4m3_to_f32(uint8_t c)
+{
+    int s = c >> 7, e = (c >> 3) & 15, m = c & 7;
+    double v = (e == 0) ? ldexp((double)m / 8.0, -6) : ldexp(1.0 + (double)m / 8.0, e - 7);
+    return (float)(s ? -v : v);
+}
+
+/* Nearest E4M3 value of a finite fp32 x, ties to even mantissa, magnitudes
+ * above 448 saturating to 448 (no infinities in E4M3). */
+uint8_t oracle_f32_to_e4m3(float x)
+{
+    uint8_t s = (x < 0.0f || (x == 0.0f && signbit(x))) ? 0x80 : 0;
+    double a = fabs((double)x);
+    if (a >= 448.0) return (uint8_t)(s | 0x7e);                 /* 1.75 * 2^8 */
+    int e;
+    frexp(a, &e);                                               /* a = f * 2^e, f in [0.5, 1) */
+    int ex = e - 1;                                             /* a in [2^ex, 2^(ex+1)) */
+    if (ex < -6) ex = -6;                                       /* subnormal range: fixed quantum */
+    double quantum = ldexp(1.0, ex - 3);
+    double q = a / quantum;                                     /* exact: a power-of-two scaling */
+    double r = rint(q);                                         /* ties to even */
+    double v = r * quantum;
+    if (v >= 448.0) return (uint8_t)(s | 0x7e);
+    if (v == 0.0) return s;
+    int ve;
+    frexp(v, &ve);
+    int vex = ve - 1;
+    if (vex < -6) {                                             /* subnormal: m * 2^-9 */
+        return (uint8_t)(s | (uint8_t)(v / ldexp(1.0, -9)));
+    }
+    int mant = (int)((v / ldexp(1.0, vex) - 1.0) * 8.0);
+    return (uint8_t)(s | (uint8_t)((vex + 7) << 3) | (uint8_t)mant);
+}
+
+/* Blockwise quantization of one block of fp32 values into codes + scale. */
+static void quant_block8(const float* x, int n, uint8_t* code, float* scale)
+{
+    float amax = 0.0f;
+    for (int i = 0; i < n; ++i)
+        if (fabsf(x[i]) > amax) amax = fabsf(x[i]);
+    *scale = amax / E4M3_MAX;
+    float inv = (amax == 0.0f) ? 0.0f : E4M3_MAX / amax;
+    for (int i = 0; i < n; ++i) code[i] = (amax == 0.0f) ? 0 : oracle_f32_to_e4m3(x[i] * inv);
+}
+
+/* One AdamW step over n parameters (see the block comment above).  p, g: bf16
+ * [n]; m_code, v_code: [n]; m_scale, v_scale: [ceil(n / 256)].  All in-out
+ * except g.  Returns 0, or -1 for n <= 0 or step < 1. */
+int oracle_adamw8_step(uint16_t* p, const uint16_t* g, int64_t n, uint8_t* m_code, float* m_scale,
+                       uint8_t* v_code, float* v_scale, int64_t step, float lr, float b1, float b2, float eps,
+                       float wd)
+{
+    if (n <= 0 || step < 1) return -1;
+    const float omb1 = (float)(1.0 - (double)b1), omb2 = (float)(1.0 - (double)b2);
+    const float rbc1 = (float)(1.0 / (1.0 - pow((double)b1, (double)step)));
+    const float rbc2 = (float)(1.0 / (1.0 - pow((double)b2, (double)step)));
+    float mnew[ADAM_BLOCK], vnew[ADAM_BLOCK];
+    for (int64_t b0 = 0; b0 < n; b0 += ADAM_BLOCK) {
+        int64_t blk = b0 / ADAM_BLOCK;
+        int cnt = (int)((n - b0) < ADAM_BLOCK ? (n - b0) : ADAM_BLOCK);
+        for (int i = 0; i < cnt; ++i) {
+            int64_t e = b0 + i;
+            float gf = oracle_bf16_to_f32(g[e]);
+            float pf = oracle_bf16_to_f32(p[e]);
+            float mo = oracle_e4m3_to_f32(m_code[e]) * m_scale[blk];
+            float vo = oracle_e4m3_to_f32(v_code[e]) * v_scale[blk];
+            float t1 = b1 * mo, t2 = omb1 * gf;
+            float mn = t1 + t2;
+            float gg = gf * gf;
+            float t3 = b2 * vo, t4 = omb2 * gg;
+            float vn = t3 + t4;
+            float mh = mn * rbc1, vh = vn * rbc2;
+            float den = sqrtf(vh) + eps;
+            float u = mh / den;
+            float dec = wd * pf;
+            u = u + dec;
+            float st = lr * u;
+            p[e] = oracle_f32_to_bf16(pf - st);
+            mnew[i] = mn;
+            vnew[i] = vn;
+        }
+        quant_block8(mnew, cnt, m_code + b0, &m_scale[blk]);
+        quant_block8(vnew, cnt, v_code + b0, &v_scale[blk]);
+    }
+    return 0;
+}
+
+/* ===========================================================================
+ * LoRA dropout ("Qlora Expert", Implementation Pattern: lora_dropout=0.05;
+ * "QLoRA Implementation Details (2025 Edition)", Step 4: lora_dropout=0.1).
+ * Reading (the pages give only the rate): dropout on the LoRA branch's input
+ * X, the base path unchanged; element (m, k) of X is kept with probability
+ * about 1 - p and kept values are scaled by 1 / (1 - p).  The mask comes
+ * from the counter-based generator Philox4x64-10 (Salmon, Moraes, Dror and
+ * Shaw, "Parallel random numbers: as easy as 1, 2, 3", SC 2011), written
+ * here from that definition:
+ *   round:  (hi0, lo0) = M0 * c0,  (hi1, lo1) = M1 * c2  (128-bit products)
+ *           c = (hi1 ^ c1 ^ k0, lo1, hi0 ^ c3 ^ k1, lo0)
+ *   key:    (k0, k1) += (W0, W1) between rounds; 10 rounds.
+ * Element e = m K + k uses 32-bit word (e mod 8) of the 256-bit output for
+ * counter (e div 8, offset, 0, 0) and key (seed, 0), words in little-endian
+ * order (word 2i is the low half of output i); it is kept iff
+ * (word >> 8) >= t, t = llrint(p * 2^24).
+ * ========================================================================= */
+static const uint64_t PHILOX_M0 = 0xD2E7470EE14C6C93ull, PHILOX_M1 = 0xCA5A826395121157ull;
+static const uint64_t PHILOX_W0 = 0x9E3779B97F4A7C15ull, PHILOX_W1 = 0xBB67AE8584CAA73Bull;
+
+static void mulhilo64(uint64_t a, uint64_t b, uint64_t* hi, uint64_t* lo)
+{
+    unsigned __int128 p = (unsigned __int128)a * (unsigned __int128)b;
+    *hi = (uint64_t)(p >> 64);
+    *lo = (uint64_t)p;
+}
+
+void oracle_philox4x64(const uint64_t ctr_in[4], const uint64_t key_in[2], uint64_t out[4])
+{
+    uint64_t c[4] = {ctr_in[0], ctr_in[1], ctr_in[2], ctr_in[3]};
+    uint64_t k0 = key_in[0], k1 = key_in[1];
+    for (int round = 0; round < 10; ++round) {
+        if (round > 0) { k0 += PHILOX_W0; k1 += PHILOX_W1; }
+        uint64_t hi0, lo0, hi1, lo1;
+        mulhilo64(PHILOX_M0, c[0], &hi0, &lo0);
+        mulhilo64(PHILOX_M1, c[2], &hi1, &lo1);
+        uint64_t n0 = hi1 ^ c[1] ^ k0, n1 = lo1, n2 = hi0 ^ c[3] ^ k1, n3 = lo0;
+        c[0] = n0; c[1] = n1; c[2] = n2; c[3] = n3;
+    }
+    for (int i = 0; i < 4; ++i) out[i] = c[i];
+}
+
+/* Keep mask [M, K] (1 = kept) of the LoRA dropout above. */
+int oracle_dropout_mask(uint64_t seed, uint64_t offset, int64_t M, int64_t K, float p, uint8_t* keep)
+{
+    if (M <= 0 || K <= 0 || !(p >= 0.0f && p < 1.0f)) return -1;
+    const uint32_t t = (uint32_t)llrint((double)p * 16777216.0);
+    const uint64_t key[2] = {seed, 0};
+    for (int64_t e8 = 0; e8 * 8 < M * K; ++e8) {
+        const uint64_t ctr[4] = {(uint64_t)e8, offset, 0, 0};
+        uint64_t o[4];
+        oracle_philox4x64(ctr, key, o);
+        for (int j = 0; j < 8 && e8 * 8 + j < M * K; ++j) {
+            uint32_t word = (uint32_t)(o[j / 2] >> (32 * (j % 2)));
+            keep[e8 * 8 + j] = (uint8_t)((word >> 8) >= t);
+        }
+    }
+    return 0;
+}
