@@ -37,6 +37,7 @@ if ROOT not in sys.path:
 
 METRIC = "QLoRA linear fwd+bwd TFLOP/s & NF4 weight-stream GB/s; % of roofline, 1×B200"
 QUANT = {"nf4": 0, "fp4": 1}
+DROPOUT_SEED = 20251
 # fp32 fused multiply-adds per cycle per SM of B200 (4 sub-partitions x 32 lanes)
 FMA_PER_SM_CYCLE = 128
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
@@ -215,12 +216,27 @@ def run_ours(args, rank, world, local_rank):
     for L, (oa, ob) in zip(layers, offs):
         L["dA"] = gbuf[oa:oa + r * L["p"].K].view(r, L["p"].K)
         L["dB"] = gbuf[ob:ob + L["p"].N * r].view(L["p"].N, r)
-    ws = torch.empty(max(ops.qlora_workspace_bytes(M, L["p"].N, L["p"].K, r) for L in layers), dtype=torch.uint8,
-                     device=dev)
+    wsb = ops.qlora_dropout_workspace_bytes if args.dropout > 0 else ops.qlora_workspace_bytes
+    ws = torch.empty(max(wsb(M, L["p"].N, L["p"].K, r) for L in layers), dtype=torch.uint8, device=dev)
     torch.cuda.synchronize()
     stream = torch.cuda.current_stream()
 
     it = [0]
+
+    def fwd_call(L, w, off):
+        if args.dropout > 0:
+            ops.qlora_linear_fwd_dropout(L["X"], w, L["A"], L["B"], s, args.dropout, DROPOUT_SEED, off,
+                                         Y=L["Y"], T_out=L["T"], ws=ws)
+        else:
+            ops.qlora_linear_fwd(L["X"], w, L["A"], L["B"], s, Y=L["Y"], T_out=L["T"], ws=ws)
+
+    def bwd_call(L, w, off):
+        if args.dropout > 0:
+            ops.qlora_linear_bwd_dropout(L["X"], L["dY"], w, L["A"], L["B"], s, args.dropout, DROPOUT_SEED, off,
+                                         T=L["T"], dX=L["dX"], dA=L["dA"], dB=L["dB"], ws=ws)
+        else:
+            ops.qlora_linear_bwd(L["X"], L["dY"], w, L["A"], L["B"], s, T=L["T"], dX=L["dX"], dA=L["dA"],
+                                 dB=L["dB"], ws=ws)
 
     def step(events=None, collective=True):
         c = it[0] % copies
@@ -229,13 +245,13 @@ def run_ours(args, rank, world, local_rank):
             w = L["wc"][c]
             if events is not None:
                 ops.qlora_set_kernel_events(*events[2 * j])
-            ops.qlora_linear_fwd(L["X"], w, L["A"], L["B"], s, Y=L["Y"], T_out=L["T"], ws=ws)
+            off = (it[0] - 1) * len(layers) + j   # dropout: a fresh mask per step and projection
+            fwd_call(L, w, off)
             if not bwd:
                 continue
             if events is not None:
                 ops.qlora_set_kernel_events(*events[2 * j + 1])
-            ops.qlora_linear_bwd(L["X"], L["dY"], w, L["A"], L["B"], s, T=L["T"], dX=L["dX"], dA=L["dA"],
-                                 dB=L["dB"], ws=ws)
+            bwd_call(L, w, off)
         if world > 1 and bwd and collective:
             dist.all_reduce(gbuf)
 
@@ -400,11 +416,10 @@ def run_ours(args, rank, world, local_rank):
             L["X"].copy_(hX[j], non_blocking=True)
             if bwd:
                 L["dY"].copy_(hdY[j], non_blocking=True)
-            ops.qlora_linear_fwd(L["X"], L["w"], L["A"], L["B"], s, Y=L["Y"], T_out=L["T"], ws=ws)
+            fwd_call(L, L["w"], j)
             hout[j][0].copy_(L["Y"], non_blocking=True)
             if bwd:
-                ops.qlora_linear_bwd(L["X"], L["dY"], L["w"], L["A"], L["B"], s, T=L["T"], dX=L["dX"],
-                                     dA=L["dA"], dB=L["dB"], ws=ws)
+                bwd_call(L, L["w"], j)
                 hout[j][1].copy_(L["dX"], non_blocking=True)
         if world > 1 and bwd:
             dist.all_reduce(gbuf)
@@ -427,12 +442,11 @@ def run_ours(args, rank, world, local_rank):
             comp.wait_event(ev_in[j])
             if primed[0]:
                 comp.wait_event(ev_out[j])
-            ops.qlora_linear_fwd(L["X"], L["w"], L["A"], L["B"], s, Y=L["Y"], T_out=L["T"], ws=ws)
+            fwd_call(L, L["w"], j)
             if bwd:
                 if j == 0 and primed[0]:
                     comp.wait_event(ev_gout)          # the gradient buffer was copied out
-                ops.qlora_linear_bwd(L["X"], L["dY"], L["w"], L["A"], L["B"], s, T=L["T"], dX=L["dX"],
-                                     dA=L["dA"], dB=L["dB"], ws=ws)
+                bwd_call(L, L["w"], j)
             ev_done[j].record(comp)
             with torch.cuda.stream(s_out):
                 s_out.wait_event(ev_done[j])
@@ -473,7 +487,7 @@ def run_ours(args, rank, world, local_rank):
         ems = float(tt.item())
     e2e_val = (flops_step if not small else bytes_step) * world / (ems / args.steps * 1e-3) / (1e12 if not small else 1e9)
 
-    cfg = {"workload": wl.name, "quant_type": args.quant,
+    cfg = {"workload": wl.name, "quant_type": args.quant, "lora_dropout": args.dropout,
            "projections": [f"{p.name} {p.N}x{p.K}" for p in projs], "M_per_gpu": M,
            "global_batch_tokens": M * world, "r": r, "alpha": wl.alpha, "weights": "NF4 + double-quant (64/256)",
            "step": "qlora_linear_fwd + qlora_linear_bwd for every projection" +
@@ -491,7 +505,7 @@ def run_ours(args, rank, world, local_rank):
                               "in order on the compute stream") + "; all inside the timed region"},
            "gpu_launches": launches, "clocks": clk}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        out["cpu_baseline"] = cpu_baseline(wl, M, budget_s=args.cpu_seconds, quant=args.quant)
+        out["cpu_baseline"] = cpu_baseline(wl, M, budget_s=args.cpu_seconds, quant=args.quant, dropout=args.dropout)
     return out
 
 
@@ -674,6 +688,86 @@ def run_merge(args, rank, world, local_rank):
     return out
 
 
+def run_adamw(args, rank, world, local_rank):
+    """One 8-bit AdamW step over every LoRA adapter of a 32-layer 7B model (the 7
+    projections per layer at r = 16: 40.0M bf16 parameters in one flat buffer, more
+    than twice L2 with its states)."""
+    import torch
+
+    from bit_nf4_quantized_quant_b200 import _ops as ops
+    from bit_nf4_quantized_quant_b200 import inputs
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    wl = inputs.WORKLOADS[3]
+    peaks, peak_src = load_peaks()
+    n = 32 * sum(wl.r * (p.N + p.K) for p in wl.projections)
+    p = inputs.normal(5000, (n,), 0.01, device=dev)
+    g = inputs.normal(5001, (n,), 1e-3, device=dev)
+    st = ops.AdamW8State.zeros(n, device=dev)
+    stream = torch.cuda.current_stream()
+    k = [0]
+
+    def step():
+        k[0] += 1
+        ops.adamw_8bit_step(p, g, st, k[0], 2e-4, 0.9, 0.999, 1e-8, 0.01)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(local_rank)
+    clocks.start()
+    l0 = ops.qlora_launch_count()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for _ in range(args.steps):
+        step()
+    t1.record(stream)
+    torch.cuda.synchronize()
+    launches = ops.qlora_launch_count() - l0
+    clk = clocks.stop()
+    ms = t0.elapsed_time(t1) / args.steps
+    nblk = math.ceil(n / 256)
+    step_bytes = n * (2 + 2 + 1 + 1) + n * (2 + 1 + 1) + nblk * 16   # read p, g, codes; write p, codes; scales
+    gbs = step_bytes / (ms * 1e-3) / 1e9
+    roof = {"bound": "hbm", "unit": "GB/s", "achieved": round(gbs, 1), "peak": peaks["hbm_gbs"],
+            "frac": round(gbs / peaks["hbm_gbs"], 4), "traffic": None, "peak_source": f"{peak_src} (hbm copy)",
+            "kernel": "k_adamw8", "launches_timed": args.steps, "avg_launch_us": round(ms * 1e3, 2)}
+    out = {"metric": METRIC, "value": round(gbs, 1), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+           "warmup": args.warmup, "ms_per_step": round(ms, 4), "higher_is_better": True, "scaling": "weak",
+           "vs_baseline": None, "dtype": "bf16 params/grads, E4M3 moment codes + fp32 block scales, fp32 update",
+           "data": "synthetic (seeded)",
+           "config": {"workload": "8-bit AdamW step, all LoRA adapters of a 32-layer 7B model (r=16, 7 projections)",
+                      "params": n, "block": 256,
+                      "l2": f"inputs larger than L2: {step_bytes / 1e6:.0f} MB per step"},
+           "roofline": roof, "gpu_launches": launches, "clocks": clk}
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        out["cpu_baseline"] = adamw_cpu_baseline(n // 32)
+    return out
+
+
+def adamw_cpu_baseline(n):
+    """The oracle's AdamW step (C, one thread) on one layer's adapters, as GB/s of the
+    same byte accounting (the rate stands for the whole model)."""
+    import numpy as np
+
+    import oracle
+    from bit_nf4_quantized_quant_b200 import inputs
+    p = inputs.bf16_bits(inputs.normal(5000, (n,), 0.01)).copy()
+    g = inputs.bf16_bits(inputs.normal(5001, (n,), 1e-3)).copy()
+    st = oracle.adamw8_state(n)
+    t0 = time.perf_counter()
+    k = 0
+    while k < 3 or time.perf_counter() - t0 < 2.0:
+        k += 1
+        oracle.adamw8_step(p, g, st, k, 2e-4, 0.9, 0.999, 1e-8, 0.01)
+    dt = (time.perf_counter() - t0) / k
+    step_bytes = n * 10 + math.ceil(n / 256) * 16
+    return {"value": round(step_bytes / dt / 1e9, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
+            "sample": f"{k} oracle steps over one layer's adapters ({n} params), C, one thread; "
+                      f"{dt * 1e3:.1f} ms per step; the rate stands for all 32 layers"}
+
+
 def merge_cpu_baseline(wl, quant, rows=64):
     """The oracle's dequantize-and-merge on `rows` rows of each projection (C, one
     thread per projection), scaled to the whole weight (every row costs the same)."""
@@ -746,7 +840,7 @@ class OracleStep:
     in these products, so the extrapolation is linear and is labelled as such.
     Quantization happens once before timing, as at model load."""
 
-    def __init__(self, wl, M, rows=64, quant="nf4"):
+    def __init__(self, wl, M, rows=64, quant="nf4", dropout=0.0):
         import numpy as np
         from concurrent.futures import ThreadPoolExecutor
 
@@ -754,6 +848,7 @@ class OracleStep:
         from bit_nf4_quantized_quant_b200 import inputs
         self.wl, self.M = wl, M
         self.rows = min(rows, M)
+        self.dropout = dropout
         self.ncores = os.cpu_count() or 1
         self.pool = ThreadPoolExecutor(self.ncores)
         self.state = []
@@ -778,9 +873,16 @@ class OracleStep:
             parts = list(self.pool.map(lambda rr: oracle.dequant_qt(q, rr), chunks))
             Wd = oracle.bf16_to_f32(np.concatenate(parts)).astype(np.float64)
             t1 = time.perf_counter()
-            oracle.linear_fwd(X, Wd, A, B, s)
-            if dY is not None:
-                oracle.linear_bwd(X, dY, Wd, A, B, s)
+            if self.dropout > 0:
+                keep = oracle.dropout_mask(DROPOUT_SEED, 0, X.shape[0], X.shape[1], self.dropout)
+                c = oracle.dropout_scale(self.dropout)
+                oracle.linear_fwd_dropout(X, Wd, A, B, s, keep, c)
+                if dY is not None:
+                    oracle.linear_bwd_dropout(X, dY, Wd, A, B, s, keep, c)
+            else:
+                oracle.linear_fwd(X, Wd, A, B, s)
+                if dY is not None:
+                    oracle.linear_bwd(X, dY, Wd, A, B, s)
             t2 = time.perf_counter()
             total += (t1 - t0) + (t2 - t1) * self.M / self.rows
         return total
@@ -797,11 +899,11 @@ class OracleStep:
                 f"by {self.M}/{self.rows} (extrapolated); quantization once, untimed")
 
 
-def cpu_baseline(wl, M, budget_s=20.0, quant="nf4"):
+def cpu_baseline(wl, M, budget_s=20.0, quant="nf4", dropout=0.0):
     """The oracle, as it stands, on the host cores over a bounded sample."""
     if wl.index == 5:
         return bulk_cpu_baseline(wl)
-    st = OracleStep(wl, M, quant=quant)
+    st = OracleStep(wl, M, quant=quant, dropout=dropout)
     st.run()                                     # warm: first touch of the fp64 buffers
     t0 = time.perf_counter()
     times = []
@@ -874,14 +976,18 @@ def sub_results(args, rank, world, local_rank):
 
     import torch
     subs = []
-    for wlx, M, op, quant in ((2, 1, "linear", "nf4"), (1, 16, "linear", "nf4"), (5, 0, "linear", "nf4"),
-                              (2, 1, "linear", "fp4"), (3, 0, "merge", "nf4")):
+    for wlx, M, op, quant, dropout in ((2, 1, "linear", "nf4", 0.0), (1, 16, "linear", "nf4", 0.0),
+                                       (5, 0, "linear", "nf4", 0.0), (2, 1, "linear", "fp4", 0.0),
+                                       (3, 0, "merge", "nf4", 0.0), (3, 0, "adamw", "nf4", 0.0),
+                                       (3, 2048, "linear", "nf4", 0.05)):
         torch.cuda.empty_cache()
         a = copy.copy(args)
-        a.workload, a.M, a.op, a.quant = wlx, M, op, quant
+        a.workload, a.M, a.op, a.quant, a.dropout = wlx, M, op, quant, dropout
         a.cpu_seconds = min(args.cpu_seconds, 8.0)
         if op == "merge":
             o = run_merge(a, rank, world, local_rank)
+        elif op == "adamw":
+            o = run_adamw(a, rank, world, local_rank)
         else:
             o = run_bulk(a, rank, world, local_rank) if wlx == 5 else run_ours(a, rank, world, local_rank)
         o.pop("metric", None)
@@ -901,8 +1007,10 @@ def main():
                          "the single 4096^2 linear (M = 16) and the bulk quantize round trip as sub_results")
     ap.add_argument("--no-sub", action="store_true", help="default workload: skip the sub_results")
     ap.add_argument("--quant", choices=["nf4", "fp4"], default="nf4", help="4-bit quant type of the frozen weights")
-    ap.add_argument("--op", choices=["linear", "merge"], default="linear",
-                    help="merge: time nf4_dequant_merge over the 7B block's projections instead")
+    ap.add_argument("--dropout", type=float, default=0.0, help="LoRA dropout rate of the linear-layer step")
+    ap.add_argument("--op", choices=["linear", "merge", "adamw"], default="linear",
+                    help="merge: time nf4_dequant_merge over the 7B block's projections; adamw: one 8-bit AdamW "
+                         "step over every adapter of a 32-layer 7B model")
     ap.add_argument("--layers", type=int, default=0, help="workload 5: number of 7-tensor layers (default 32)")
     ap.add_argument("--M", type=int, default=0, help="tokens per GPU (default: the workload's largest)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -935,6 +1043,8 @@ def main():
     try:
         if args.op == "merge":
             out = run_merge(args, rank, world, local_rank)
+        elif args.op == "adamw":
+            out = run_adamw(args, rank, world, local_rank)
         elif args.workload == 5:
             out = run_bulk(args, rank, world, local_rank)
         else:

@@ -48,12 +48,19 @@ def lib():
                                "`python -m bit_nf4_quantized_quant_b200.build`")
         L = ctypes.CDLL(LIB_PATH)
         P, i64, i32, f32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_float
+        u64 = ctypes.c_uint64
         WP = ctypes.POINTER(_Weight)
         sig = {
             "nf4_codebook": (i32, [P]),
             "quant4_codebook": (i32, [i32, P]),
             "quant4_quantize_dq": (i32, [P, i64, i64, i32, P, P, P, P, P]),
             "nf4_dequant_merge": (i32, [WP, P, P, i32, f32, P, P]),
+            "adamw_8bit_step": (i32, [P, P, i64, P, P, P, P, i64, f32, f32, f32, f32, f32, P]),
+            "qlora_dropout_workspace_bytes": (ctypes.c_size_t, [i64, i64, i64, i32]),
+            "qlora_linear_fwd_dropout": (i32, [P, i64, WP, P, P, i32, f32, f32, u64, u64, P, P, P,
+                                               ctypes.c_size_t, P]),
+            "qlora_linear_bwd_dropout": (i32, [P, P, i64, WP, P, P, i32, f32, f32, u64, u64, P, P, P, P, P,
+                                               ctypes.c_size_t, P]),
             "nf4dq_sizes": (i32, [i64, i64, P, P, P]),
             "nf4_quantize_dq": (i32, [P, i64, i64, P, P, P, P, P]),
             "nf4_dequant": (i32, [WP, P, P]),
@@ -178,6 +185,37 @@ def nf4_dequant_merge(w: NF4Weight, A, B, scaling: float, out: torch.Tensor | No
     return out
 
 
+QLORA_ADAM_BLOCK = 256
+
+
+@dataclass
+class AdamW8State:
+    """8-bit moment states of n parameters (E4M3 codes + one fp32 scale per 256)."""
+    m_code: torch.Tensor   # uint8 [n]
+    m_scale: torch.Tensor  # fp32 [ceil(n / 256)]
+    v_code: torch.Tensor   # uint8 [n]
+    v_scale: torch.Tensor  # fp32 [ceil(n / 256)]
+
+    @staticmethod
+    def zeros(n: int, device="cuda") -> "AdamW8State":
+        nb = (n + QLORA_ADAM_BLOCK - 1) // QLORA_ADAM_BLOCK
+        return AdamW8State(torch.zeros(n, dtype=torch.uint8, device=device),
+                           torch.zeros(nb, dtype=torch.float32, device=device),
+                           torch.zeros(n, dtype=torch.uint8, device=device),
+                           torch.zeros(nb, dtype=torch.float32, device=device))
+
+
+def adamw_8bit_step(p: torch.Tensor, g: torch.Tensor, state: AdamW8State, step: int, lr: float,
+                    beta1: float = 0.9, beta2: float = 0.999, eps: float = 1e-8, weight_decay: float = 0.0,
+                    stream=None) -> None:
+    """In-place AdamW step of the bf16 parameters p with gradient g and 8-bit states."""
+    p, g = _bits(p), _bits(g)
+    _check("adamw_8bit_step", lib().adamw_8bit_step(
+        _ptr(p), _ptr(g), p.numel(), _ptr(state.m_code), _ptr(state.m_scale), _ptr(state.v_code),
+        _ptr(state.v_scale), int(step), float(lr), float(beta1), float(beta2), float(eps), float(weight_decay),
+        _stream(stream)))
+
+
 def nf4_dequant(w: NF4Weight, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
     if out is None:
         out = torch.empty((w.N, w.K), dtype=torch.bfloat16, device=w.packed.device)
@@ -229,6 +267,54 @@ def qlora_linear_bwd(X, dY, w: NF4Weight, A, B, scaling: float, T=None, dX=None,
     _check("qlora_linear_bwd", lib().qlora_linear_bwd(
         _ptr(_bits(X)), _ptr(_bits(dY)), M, ctypes.byref(st), _ptr(_bits(A)), _ptr(_bits(B)), r, float(scaling),
         _ptr(T), _ptr(dX), _ptr(dA), _ptr(dB), _ptr(ws), ws.numel(), _stream(stream)))
+    return dX, dA, dB
+
+
+def qlora_dropout_workspace_bytes(M: int, N: int, K: int, r: int) -> int:
+    return int(lib().qlora_dropout_workspace_bytes(M, N, K, r))
+
+
+def dropout_workspace(M: int, N: int, K: int, r: int, device="cuda") -> torch.Tensor:
+    n = qlora_dropout_workspace_bytes(M, N, K, r)
+    if n == 0:
+        raise QLoRAError("qlora_dropout_workspace_bytes", -2)
+    return torch.empty(n, dtype=torch.uint8, device=device)
+
+
+def qlora_linear_fwd_dropout(X, w: NF4Weight, A, B, scaling: float, dropout_p: float, seed: int, offset: int,
+                             Y=None, T_out=None, ws=None, stream=None):
+    """qlora_linear_fwd with LoRA dropout on the branch input (mask from (seed, offset))."""
+    M = X.shape[0]
+    if Y is None:
+        Y = torch.empty((M, w.N), dtype=torch.bfloat16, device=X.device)
+    if ws is None:
+        ws = dropout_workspace(M, w.N, w.K, A.shape[0], X.device)
+    st = w.c_struct()
+    _check("qlora_linear_fwd_dropout", lib().qlora_linear_fwd_dropout(
+        _ptr(_bits(X)), M, ctypes.byref(st), _ptr(_bits(A)), _ptr(_bits(B)), A.shape[0], float(scaling),
+        float(dropout_p), int(seed), int(offset), _ptr(Y), _ptr(T_out), _ptr(ws), ws.numel(), _stream(stream)))
+    return Y
+
+
+def qlora_linear_bwd_dropout(X, dY, w: NF4Weight, A, B, scaling: float, dropout_p: float, seed: int, offset: int,
+                             T=None, dX=None, dA=None, dB=None, ws=None, stream=None):
+    """qlora_linear_bwd under the same LoRA dropout mask as the forward; returns (dX, dA, dB)."""
+    M = X.shape[0]
+    r = A.shape[0]
+    dev = X.device
+    if dX is None:
+        dX = torch.empty((M, w.K), dtype=torch.bfloat16, device=dev)
+    if dA is None:
+        dA = torch.empty((r, w.K), dtype=torch.bfloat16, device=dev)
+    if dB is None:
+        dB = torch.empty((w.N, r), dtype=torch.bfloat16, device=dev)
+    if ws is None:
+        ws = dropout_workspace(M, w.N, w.K, r, dev)
+    st = w.c_struct()
+    _check("qlora_linear_bwd_dropout", lib().qlora_linear_bwd_dropout(
+        _ptr(_bits(X)), _ptr(_bits(dY)), M, ctypes.byref(st), _ptr(_bits(A)), _ptr(_bits(B)), r, float(scaling),
+        float(dropout_p), int(seed), int(offset), _ptr(T), _ptr(dX), _ptr(dA), _ptr(dB), _ptr(ws), ws.numel(),
+        _stream(stream)))
     return dX, dA, dB
 
 

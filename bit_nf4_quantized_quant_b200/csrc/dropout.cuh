@@ -1,0 +1,123 @@
+// dropout.cuh -- LoRA dropout on the branch input X (the base path is left
+// unchanged): the keep mask, the dropped copy X * keep (exact in bf16; the
+// scale c of kept values is applied in fp32 where T, dA and the LoRA term of
+// dX are formed), and the masked LoRA term of dX.
+//
+// Element e = m K + k of X is kept iff (word >> 8) >= t, t = llrint(p 2^24),
+// where word is 32-bit word (e mod 8) of the Philox4x64-10 output for counter
+// (e div 8, offset, 0, 0) and key (seed, 0) (Salmon, Moraes, Dror and Shaw,
+// SC 2011: per round (hi0, lo0) = M0 c0, (hi1, lo1) = M1 c2 as 128-bit
+// products, c = (hi1 ^ c1 ^ k0, lo1, hi0 ^ c3 ^ k1, lo0), and the key adds
+// the Weyl increments between rounds).  Kept values are scaled by
+// c = fl32(1 / (1 - p)).  One generator call serves the 8 consecutive
+// elements a thread handles (K % 64 == 0 keeps every 8-element group in one
+// row).
+#pragma once
+#include "common.cuh"
+
+namespace qnf4 {
+namespace drop {
+
+struct Params {
+    uint64_t seed, offset;
+    uint32_t t;        // keep iff (word >> 8) >= t
+    float c;           // scale of kept values
+};
+
+__device__ __forceinline__ void philox4x64(uint64_t c0, uint64_t c1, uint64_t k0, uint64_t out[4]) {
+    constexpr uint64_t M0 = 0xD2E7470EE14C6C93ull, M1 = 0xCA5A826395121157ull;
+    constexpr uint64_t W0 = 0x9E3779B97F4A7C15ull, W1 = 0xBB67AE8584CAA73Bull;
+    uint64_t c2 = 0, c3 = 0, k1 = 0;
+#pragma unroll
+    for (int round = 0; round < 10; ++round) {
+        if (round > 0) { k0 += W0; k1 += W1; }
+        const uint64_t hi0 = __umul64hi(M0, c0), lo0 = M0 * c0;
+        const uint64_t hi1 = __umul64hi(M1, c2), lo1 = M1 * c2;
+        const uint64_t n0 = hi1 ^ c1 ^ k0, n2 = hi0 ^ c3 ^ k1;
+        c0 = n0; c1 = lo1; c2 = n2; c3 = lo0;
+    }
+    out[0] = c0; out[1] = c1; out[2] = c2; out[3] = c3;
+}
+
+// keep bits of elements 8 e8 .. 8 e8 + 7 (bit j = element 8 e8 + j)
+__device__ __forceinline__ uint32_t keep8(const Params& d, uint64_t e8) {
+    uint64_t o[4];
+    philox4x64(e8, d.offset, d.seed, o);
+    uint32_t bits = 0;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        const uint32_t word = (uint32_t)(o[j >> 1] >> (32 * (j & 1)));
+        bits |= ((word >> 8) >= d.t ? 1u : 0u) << j;
+    }
+    return bits;
+}
+
+// Xd [M, K] = X where kept, 0 where dropped (exact; the scale c of kept values is applied in
+// fp32 where T and dA are formed); one thread per 8 elements.
+__global__ void __launch_bounds__(256) k_dropout_x(const uint16_t* __restrict__ X, int64_t total8,
+                                                   uint16_t* __restrict__ Xd, Params d) {
+    for (int64_t e8 = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e8 < total8;
+         e8 += (int64_t)gridDim.x * blockDim.x) {
+        const uint32_t keep = keep8(d, (uint64_t)e8);
+        const uint4 x = ldg_nc_v4(X + 8 * e8);
+        const uint32_t xw[4] = {x.x, x.y, x.z, x.w};
+        uint32_t o[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const uint32_t lo = (keep >> (2 * j)) & 1u ? (xw[j] & 0xffffu) : 0u;
+            const uint32_t hi = (keep >> (2 * j + 1)) & 1u ? (xw[j] & 0xffff0000u) : 0u;
+            o[j] = lo | hi;
+        }
+        *reinterpret_cast<uint4*>(Xd + 8 * e8) = make_uint4(o[0], o[1], o[2], o[3]);
+    }
+}
+
+// dX [M, K] += masked LoRA term, in place on the bf16 base dY W' (written by
+// the fused kernel with its LoRA steps switched off):
+//   l  = sum_j U[m, j] A[j, k]   (fp32, increasing j)
+//   dX = bf16_rne(fmaf(sc, l, fl32(dX)))  where kept, dX unchanged where dropped,
+//   sc = fl32(s c).  One thread per 8 consecutive k of one row.
+struct DxArgs {
+    uint16_t* dX;          // [M, K]
+    const float* U;        // [M, ldu] fp32
+    int64_t ldu;
+    const uint16_t* A;     // [r, K]
+    int64_t M, K;
+    int r;
+    float sc;
+};
+
+__global__ void __launch_bounds__(256) k_dx_lora_dropout(const DxArgs a, Params d) {
+    const int64_t total8 = a.M * a.K / 8;
+    for (int64_t e8 = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e8 < total8;
+         e8 += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t m = (8 * e8) / a.K, k = (8 * e8) % a.K;
+        const uint32_t keep = keep8(d, (uint64_t)e8);
+        float l[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        for (int j = 0; j < a.r; ++j) {
+            const float u = __ldg(a.U + m * a.ldu + j);
+            const uint4 av = ldg_nc_v4(a.A + (int64_t)j * a.K + k);
+            const uint32_t aw[4] = {av.x, av.y, av.z, av.w};
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                l[2 * q] = __fmaf_rn(u, bf16lo_to_f32(aw[q]), l[2 * q]);
+                l[2 * q + 1] = __fmaf_rn(u, bf16hi_to_f32(aw[q]), l[2 * q + 1]);
+            }
+        }
+        uint4* p = reinterpret_cast<uint4*>(a.dX + 8 * e8);
+        const uint4 b = *p;
+        const uint32_t bw[4] = {b.x, b.y, b.z, b.w};
+        uint32_t o[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            float lo = bf16lo_to_f32(bw[q]), hi = bf16hi_to_f32(bw[q]);
+            if ((keep >> (2 * q)) & 1u) lo = __fmaf_rn(a.sc, l[2 * q], lo);
+            if ((keep >> (2 * q + 1)) & 1u) hi = __fmaf_rn(a.sc, l[2 * q + 1], hi);
+            o[q] = pack_bf16x2(lo, hi);
+        }
+        *p = make_uint4(o[0], o[1], o[2], o[3]);
+    }
+}
+
+}  // namespace drop
+}  // namespace qnf4

@@ -299,6 +299,7 @@ struct FinishArgs {
     const uint16_t* lora_B;
     int b_vec;
     float s;
+    float tscale;              // T = tscale * (sum of the splits); 1 except under LoRA dropout
     uint16_t* Y;
     uint16_t* T_out;           // [M, r] bf16 copy of T for the caller, or null
 };
@@ -385,6 +386,7 @@ __global__ void __launch_bounds__(TR, 8) k_nf4_gemv_finish(FinishArgs a) {
             t += t0; t += t1; t += t2; t += t3;
         }
         for (; z < a.kc; ++z) t += tp[z * zs];
+        t = __fmul_rn(t, a.tscale);
         s_T[e] = t;
         if (tile == 0 && a.T_out != nullptr)
             a.T_out[(int64_t)(m0 + mm) * r + i] = (uint16_t)(pack_bf16x2(t, 0.f) & 0xffffu);

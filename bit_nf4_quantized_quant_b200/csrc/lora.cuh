@@ -191,6 +191,7 @@ struct FinishArgs {
     // o2_lo > 0: o2 holds alpha2 * v as a bf16 hi + lo pair, hi in column j and
     // lo in column o2_lo + j for j < o2_lo, zero in columns [2 o2_lo, J2pad)
     int64_t o2_lo;
+    float pre;               // every output is of pre * (the split sum); 1 except under LoRA dropout
 };
 
 // v + p[0] + p[stride] + ... + p[(n - 1) stride], added in that order; four
@@ -217,6 +218,7 @@ __global__ void __launch_bounds__(256) k_gemm_finish(FinishArgs f) {
             v = split_sum(f.C + i * f.J + j, f.I * f.J, f.splits, v);
             if (f.row_pair > 0) v = split_sum(f.C + (i + f.row_pair) * f.J + j, f.I * f.J, f.splits, v);
             if (f.col_pair > 0) v = split_sum(f.C + i * f.J + j + f.col_pair, f.I * f.J, f.splits, v);
+            v = __fmul_rn(v, f.pre);
         }
         if (f.f32 && j < f.Jf) f.f32[i * f.ld_f32 + j] = v;
         if (f.hl && j < f.hl_off) {

@@ -20,6 +20,7 @@
 #include "tc_gemm.cuh"
 #include "tc2_gemm.cuh"
 #include "merge.cuh"
+#include "adamw8.cuh"
 
 using namespace qnf4;
 
@@ -363,6 +364,7 @@ int run_gemm(const uint16_t* A, int64_t lda, const uint16_t* B, int64_t ldb, int
 
 FinishArgs fin_none() {
     FinishArgs f{};
+    f.pre = 1.f;
     return f;
 }
 
@@ -467,7 +469,8 @@ int ensure_tc_attrs() {
 // rows (B for the forward, A for the backward).
 template <bool BWD>
 int launch_tc(const nf4dq_weight* w, const uint16_t* act, int64_t M, const uint16_t* lact, int lw,
-              const uint16_t* lora_w, int64_t ldl, int r, uint16_t* out, int sms, cudaStream_t st) {
+              const uint16_t* lora_w, int64_t ldl, int r, uint16_t* out, int sms, cudaStream_t st,
+              bool lora = true) {
     int rc = ensure_tc_attrs();
     if (rc != QLORA_OK) return rc;
     const int64_t N = w->N, K = w->K;
@@ -482,7 +485,7 @@ int launch_tc(const nf4dq_weight* w, const uint16_t* act, int64_t M, const uint1
         return QLORA_ERR_LAUNCH;
     tc::Args a{};
     a.codes = w->codes; a.scale = w->scale; a.mean = w->mean;
-    a.lora_w = lora_w; a.ldl = ldl; a.r = r; a.lper = (int)rup(r, 16); a.nlora = (int)cdiv(lw, 64);
+    a.lora_w = lora_w; a.ldl = ldl; a.r = r; a.lper = (int)rup(r, 16); a.nlora = lora ? (int)cdiv(lw, 64) : 0;
     a.out = out; a.M = M; a.N = N; a.K = K; a.n_out = n_out; a.n_red = n_red;
     const int64_t ntiles = cdiv(M, tc::BM) * cdiv(n_out, tc::BN);
     const int grid = (int)(ntiles < sms ? ntiles : sms);
@@ -496,7 +499,8 @@ int launch_tc(const nf4dq_weight* w, const uint16_t* act, int64_t M, const uint1
 // The same on SM pairs (cta_group::2), 256 x 256 tiles.
 template <bool BWD>
 int launch_tc2(const nf4dq_weight* w, const uint16_t* act, int64_t M, const uint16_t* lact, int lw,
-               const uint16_t* lora_w, int64_t ldl, int r, uint16_t* out, int pairs, cudaStream_t st) {
+               const uint16_t* lora_w, int64_t ldl, int r, uint16_t* out, int pairs, cudaStream_t st,
+               bool lora = true) {
     const int64_t N = w->N, K = w->K;
     const int64_t n_red = BWD ? N : K, n_out = BWD ? K : N;
     CUtensorMap tmA, tmL, tmP;
@@ -509,7 +513,7 @@ int launch_tc2(const nf4dq_weight* w, const uint16_t* act, int64_t M, const uint
         return QLORA_ERR_LAUNCH;
     tc::Args a{};
     a.codes = w->codes; a.scale = w->scale; a.mean = w->mean;
-    a.lora_w = lora_w; a.ldl = ldl; a.r = r; a.lper = (int)rup(r, 16); a.nlora = (int)cdiv(lw, 64);
+    a.lora_w = lora_w; a.ldl = ldl; a.r = r; a.lper = (int)rup(r, 16); a.nlora = lora ? (int)cdiv(lw, 64) : 0;
     a.out = out; a.M = M; a.N = N; a.K = K; a.n_out = n_out; a.n_red = n_red;
     const int64_t ntiles = cdiv(M, tc2::BM) * cdiv(n_out, tc2::BN);
     const int np = (int)(ntiles < pairs ? ntiles : pairs);
@@ -535,8 +539,9 @@ constexpr int64_t kSmallMaxM = 32;
 // T = X A^T: T32 (fp32 [M, rp]), Thl (bf16 hi|lo [M, 2 rp]), sT (bf16 s*T as hi | lo, [M, lw]),
 // and the caller's T_out (bf16 [M, r]) when given.
 int compute_T(const Plan& p, const uint16_t* X, const uint16_t* A, float s, uint16_t* T_out, uint8_t* ws, int sms,
-              cudaStream_t st) {
+              cudaStream_t st, float tscale = 1.f) {
     FinishArgs f = fin_none();
+    f.pre = tscale;
     f.Iout = p.M; f.Jiter = p.lw;
     f.f32 = reinterpret_cast<float*>(ws + p.off_T32); f.ld_f32 = p.rp; f.Jf = p.rp;
     f.J1 = p.r;
@@ -603,8 +608,9 @@ int launch_tcs_bwd(const Plan& p, const nf4dq_weight* w, const uint16_t* dY, uin
 // Small-M forward: the GEMV (mma.sync, stream-K over one CTA per SM), the
 // T = X A^T kernel and the finish kernel, all launched programmatically.
 template <int NTT>
-int launch_gemv_ntt(const Plan& p, const nf4dq_weight* w, const uint16_t* X, const uint16_t* A, const uint16_t* B,
-                    float s, uint16_t* Y, uint16_t* T_out, uint8_t* wsb, int sms, cudaStream_t st) {
+int launch_gemv_ntt(const Plan& p, const nf4dq_weight* w, const uint16_t* X, const uint16_t* Xl, const uint16_t* A,
+                    const uint16_t* B, float s, uint16_t* Y, uint16_t* T_out, uint8_t* wsb, int sms, cudaStream_t st,
+                    float tscale) {
     using C = gmv::Cfg<NTT>;
     static bool attr_set[64];
     int dev = 0;
@@ -638,12 +644,13 @@ int launch_gemv_ntt(const Plan& p, const nf4dq_weight* w, const uint16_t* X, con
     int rc = launch_pdl(gmv::k_nf4_gemv<NTT>, dim3((unsigned)ctas), dim3(gmv::kThreads), (size_t)C::SMEM_ALLOC, st,
                         tmP, a, tables(w->quant_type));
     if (rc != QLORA_OK) return rc;
-    rc = small_T(p, X, A, nullptr, wsb, st, true);
+    rc = small_T(p, Xl, A, nullptr, wsb, st, true);
     if (rc != QLORA_OK) return rc;
     gmv::FinishArgs f{};
     f.slots = a.slots; f.M = p.M; f.N = N; f.nks = a.nks; f.ctas = a.ctas; f.NT = C::NT; f.units = a.units;
     f.Tpart = reinterpret_cast<const float*>(wsb + p.off_T32); f.kc = p.TKC; f.rp = p.rp; f.r = p.r;
-    f.lora_B = B; f.b_vec = (p.r % 8 == 0 && aligned16(B)) ? 1 : 0; f.s = s; f.Y = Y; f.T_out = T_out;
+    f.lora_B = B; f.b_vec = (p.r % 8 == 0 && aligned16(B)) ? 1 : 0; f.s = s; f.tscale = tscale; f.Y = Y;
+    f.T_out = T_out;
     const int mt = p.M <= 1 ? 1 : p.M <= 2 ? 2 : p.M <= 4 ? 4 : 8;
     void (*fin)(gmv::FinishArgs) = mt == 1 ? gmv::k_nf4_gemv_finish<1> : mt == 2 ? gmv::k_nf4_gemv_finish<2>
                                  : mt == 4 ? gmv::k_nf4_gemv_finish<4> : gmv::k_nf4_gemv_finish<8>;
@@ -652,32 +659,34 @@ int launch_gemv_ntt(const Plan& p, const nf4dq_weight* w, const uint16_t* X, con
 
 // Small-M forward: fused GEMV, T = X A^T beside it, then the finish kernel
 // (partial tiles summed, s T B^T added).
-int small_fwd(const Plan& p, const uint16_t* X, const nf4dq_weight* w, const uint16_t* A, const uint16_t* B,
-              float scaling, uint16_t* Y, uint16_t* T_out, uint8_t* wsb, int sms, cudaStream_t st) {
+int small_fwd(const Plan& p, const uint16_t* X, const uint16_t* Xl, const nf4dq_weight* w, const uint16_t* A,
+              const uint16_t* B, float scaling, uint16_t* Y, uint16_t* T_out, uint8_t* wsb, int sms, cudaStream_t st,
+              float tscale) {
     hook_before(st);
     int rc;
-    if (p.M <= 8) rc = launch_gemv_ntt<1>(p, w, X, A, B, scaling, Y, T_out, wsb, sms, st);
-    else if (p.M <= 16) rc = launch_gemv_ntt<2>(p, w, X, A, B, scaling, Y, T_out, wsb, sms, st);
-    else rc = launch_gemv_ntt<4>(p, w, X, A, B, scaling, Y, T_out, wsb, sms, st);
+    if (p.M <= 8) rc = launch_gemv_ntt<1>(p, w, X, Xl, A, B, scaling, Y, T_out, wsb, sms, st, tscale);
+    else if (p.M <= 16) rc = launch_gemv_ntt<2>(p, w, X, Xl, A, B, scaling, Y, T_out, wsb, sms, st, tscale);
+    else rc = launch_gemv_ntt<4>(p, w, X, Xl, A, B, scaling, Y, T_out, wsb, sms, st, tscale);
     hook_after(st);
     return rc;
 }
 
 // Small-M backward: [T], U partials + dB, the fused dY W' kernel (overlapping
 // the U / dB kernel), then dX = dY W' + s U A and dA.
-int small_bwd(const Plan& p, const uint16_t* X, const uint16_t* dY, const nf4dq_weight* w, const uint16_t* A,
+int small_bwd(const Plan& p, const uint16_t* Xl, const uint16_t* dY, const nf4dq_weight* w, const uint16_t* A,
               const uint16_t* B, float scaling, const uint16_t* T, uint16_t* dX, uint16_t* dA, uint16_t* dB,
-              uint8_t* wsb, int sms, cudaStream_t st) {
+              uint8_t* wsb, int sms, cudaStream_t st, const drop::Params* dp) {
     int rc = QLORA_OK;
     const float* T32 = nullptr;
     if (T == nullptr) {
-        rc = small_T(p, X, A, nullptr, wsb, st, false);
+        rc = small_T(p, Xl, A, nullptr, wsb, st, false);
         if (rc != QLORA_OK) return rc;
         T32 = reinterpret_cast<const float*>(wsb + p.off_T32);
     }
     hook_before(st);
     LoraBwdArgs b{};
     b.dY = dY; b.B = B; b.T32 = T32; b.Tb = T; b.M = p.M; b.N = p.N; b.r = p.r; b.rp = p.rp; b.s = scaling;
+    b.tscale = dp ? dp->c : 1.f;
     b.b_vec = (p.r % 8 == 0 && aligned16(B)) ? 1 : 0;
     b.Upart = reinterpret_cast<float*>(wsb + p.off_Upart); b.US = p.US; b.rows_u = p.rows_u; b.dB = dB;
     k_lora_bwd_small<<<(unsigned)(p.US + cdiv(p.N, kLoraThreads)), kLoraThreads, 0, st>>>(b);
@@ -690,10 +699,34 @@ int small_bwd(const Plan& p, const uint16_t* X, const uint16_t* dY, const nf4dq_
     if (rc != QLORA_OK) return rc;
     BwdEndArgs e{};
     e.slots = ta.slots; e.NT = p.NT; e.nks = ta.nks; e.ctas = ta.ctas; e.units = ta.units;
-    e.Upart = b.Upart; e.US = p.US; e.A = A; e.X = X;
+    e.Upart = b.Upart; e.US = p.US; e.A = A; e.X = Xl;
+    if (dp) { e.dropout = 1; e.dp = *dp; }
     e.M = p.M; e.K = p.K; e.r = p.r; e.rp = p.rp; e.s = scaling; e.dX = dX; e.dA = dA;
+    e.s_da = dp ? (float)((double)scaling * (double)dp->c) : scaling;
     return launch_pdl(k_bwd_small_end, dim3((unsigned)cdiv(p.K, kLoraThreads), (unsigned)(p.M + p.r)),
                       dim3(kLoraThreads), 0, st, e);
+}
+
+// Bytes of the dropped copy of X that the dropout entry points need past the
+// regular workspace plan.
+size_t dropout_bytes(int64_t M, int64_t K) { return align256((size_t)M * (size_t)K * 2); }
+
+int dropout_params(float p, uint64_t seed, uint64_t offset, drop::Params* d) {
+    if (!(p >= 0.f && p < 1.f)) return QLORA_ERR_VALUE;
+    d->seed = seed;
+    d->offset = offset;
+    d->t = (uint32_t)std::llrint((double)p * 16777216.0);
+    d->c = (float)(1.0 / (1.0 - (double)p));
+    return QLORA_OK;
+}
+
+// Xd = the dropped and scaled copy of X [M, K] (into the workspace).
+int launch_dropout_x(const uint16_t* X, int64_t M, int64_t K, uint8_t* dst, const drop::Params& d, int sms,
+                     cudaStream_t st) {
+    const int64_t total8 = M * K / 8;
+    drop::k_dropout_x<<<grid_for(total8, 256, sms), 256, 0, st>>>(X, total8, reinterpret_cast<uint16_t*>(dst), d);
+    note_launch();
+    return launch_status();
 }
 
 }  // namespace
@@ -802,15 +835,48 @@ int nf4_dequant_merge(const nf4dq_weight* w, const qlora_bf16* A, const qlora_bf
     return launch_status();
 }
 
+int adamw_8bit_step(qlora_bf16* p, const qlora_bf16* g, int64_t n, uint8_t* m_code, float* m_scale,
+                    uint8_t* v_code, float* v_scale, int64_t step, float lr, float beta1, float beta2, float eps,
+                    float weight_decay, qlora_stream_t stream) {
+    if (!p || !g || !m_code || !m_scale || !v_code || !v_scale) return QLORA_ERR_NULL;
+    if (n <= 0 || n > ((int64_t)1 << 40)) return QLORA_ERR_SHAPE;
+    if (step < 1 || !std::isfinite(lr) || !std::isfinite(eps) || !std::isfinite(weight_decay) ||
+        !(beta1 >= 0.f && beta1 < 1.f) || !(beta2 >= 0.f && beta2 < 1.f))
+        return QLORA_ERR_VALUE;
+    if (!aligned16(p) || !aligned16(g) || (reinterpret_cast<uintptr_t>(m_code) & 7u) != 0 ||
+        (reinterpret_cast<uintptr_t>(v_code) & 7u) != 0 || (reinterpret_cast<uintptr_t>(m_scale) & 3u) != 0 ||
+        (reinterpret_cast<uintptr_t>(v_scale) & 3u) != 0)
+        return QLORA_ERR_ALIGN;
+    int sms = 0;
+    int rc = check_device(&sms);
+    if (rc != QLORA_OK) return rc;
+    adam::Args a{};
+    a.p = p; a.g = g; a.n = n; a.m_code = m_code; a.m_scale = m_scale; a.v_code = v_code; a.v_scale = v_scale;
+    a.lr = lr; a.b1 = beta1; a.b2 = beta2; a.eps = eps; a.wd = weight_decay;
+    // host constants, each rounded once to fp32 from a double computation
+    a.omb1 = (float)(1.0 - (double)beta1);
+    a.omb2 = (float)(1.0 - (double)beta2);
+    a.rbc1 = (float)(1.0 / (1.0 - std::pow((double)beta1, (double)step)));
+    a.rbc2 = (float)(1.0 / (1.0 - std::pow((double)beta2, (double)step)));
+    if (!std::isfinite(a.rbc1) || !std::isfinite(a.rbc2)) return QLORA_ERR_VALUE;
+    const int64_t nblocks = cdiv(n, adam::kBlockParams);
+    const int grid = grid_for(nblocks, adam::kThreads / 32, sms, 8);
+    adam::k_adamw8<<<grid, adam::kThreads, 0, (cudaStream_t)stream>>>(a);
+    note_launch();
+    return launch_status();
+}
+
 size_t qlora_workspace_bytes(int64_t M, int64_t N, int64_t K, int r) {
     if (M <= 0 || N <= 0 || K <= 0 || (K % kBlock) != 0 || (N % 8) != 0 || K > QLORA_MAX_K) return 0;
     if (r < 1 || r > QLORA_MAX_RANK) return 0;
     return make_plan(M, N, K, r, 148).total;
 }
 
-int qlora_linear_fwd(const qlora_bf16* X, int64_t M, const nf4dq_weight* w, const qlora_bf16* A,
-                     const qlora_bf16* B, int r, float scaling, qlora_bf16* Y, qlora_bf16* T_out, void* ws,
-                     size_t ws_bytes, qlora_stream_t stream) {
+// The forward with the LoRA branch reading Xl (X, or its dropped copy in the
+// workspace past the regular plan when dp is given).
+static int fwd_impl(const qlora_bf16* X, int64_t M, const nf4dq_weight* w, const qlora_bf16* A,
+                    const qlora_bf16* B, int r, float scaling, qlora_bf16* Y, qlora_bf16* T_out, void* ws,
+                    size_t ws_bytes, qlora_stream_t stream, const drop::Params* dp) {
     if (!X || !A || !B || !Y) return QLORA_ERR_NULL;
     int rc = validate_weight(w);
     if (rc != QLORA_OK) return rc;
@@ -823,16 +889,22 @@ int qlora_linear_fwd(const qlora_bf16* X, int64_t M, const nf4dq_weight* w, cons
     rc = check_device(&sms);
     if (rc != QLORA_OK) return rc;
     const Plan p = make_plan(M, w->N, w->K, r, 148);
-    if (ws_bytes < p.total) return QLORA_ERR_WORKSPACE;
+    if (ws_bytes < p.total + (dp ? dropout_bytes(M, w->K) : 0)) return QLORA_ERR_WORKSPACE;
     cudaStream_t st = (cudaStream_t)stream;
     uint8_t* wsb = static_cast<uint8_t*>(ws);
+    const uint16_t* Xl = X;
+    if (dp) {
+        rc = launch_dropout_x(X, M, w->K, wsb + p.total, *dp, sms, st);
+        if (rc != QLORA_OK) return rc;
+        Xl = reinterpret_cast<const uint16_t*>(wsb + p.total);
+    }
 
     if (M <= kSmallMaxM) {
-        rc = small_fwd(p, X, w, A, B, scaling, Y, T_out, wsb, sms, st);
+        rc = small_fwd(p, X, Xl, w, A, B, scaling, Y, T_out, wsb, sms, st, dp ? dp->c : 1.f);
         if (rc == QLORA_OK) t_last_path = 1;
         return rc;
     }
-    rc = compute_T(p, X, A, scaling, T_out, wsb, sms, st);
+    rc = compute_T(p, Xl, A, scaling, T_out, wsb, sms, st, dp ? dp->c : 1.f);
     if (rc != QLORA_OK) return rc;
 
     // tcgen05 path: LoRA weight rows must be 16-byte granular (r % 8 == 0) or padded
@@ -862,10 +934,12 @@ int qlora_linear_fwd(const qlora_bf16* X, int64_t M, const nf4dq_weight* w, cons
     return rc;
 }
 
-int qlora_linear_bwd(const qlora_bf16* X, const qlora_bf16* dY, int64_t M, const nf4dq_weight* w,
-                     const qlora_bf16* A, const qlora_bf16* B, int r, float scaling, const qlora_bf16* T,
-                     qlora_bf16* dX, qlora_bf16* dA, qlora_bf16* dB, void* ws, size_t ws_bytes,
-                     qlora_stream_t stream) {
+// The backward; with dp the LoRA branch reads the dropped copy of X and the
+// LoRA term of dX is masked (keep * c).
+static int bwd_impl(const qlora_bf16* X, const qlora_bf16* dY, int64_t M, const nf4dq_weight* w,
+                    const qlora_bf16* A, const qlora_bf16* B, int r, float scaling, const qlora_bf16* T,
+                    qlora_bf16* dX, qlora_bf16* dA, qlora_bf16* dB, void* ws, size_t ws_bytes,
+                    qlora_stream_t stream, const drop::Params* dp) {
     if (!X || !dY || !A || !B || !dX || !dA || !dB) return QLORA_ERR_NULL;
     int rc = validate_weight(w);
     if (rc != QLORA_OK) return rc;
@@ -879,11 +953,17 @@ int qlora_linear_bwd(const qlora_bf16* X, const qlora_bf16* dY, int64_t M, const
     if (rc != QLORA_OK) return rc;
     const int64_t N = w->N, K = w->K;
     const Plan p = make_plan(M, N, K, r, 148);
-    if (ws_bytes < p.total) return QLORA_ERR_WORKSPACE;
+    if (ws_bytes < p.total + (dp ? dropout_bytes(M, K) : 0)) return QLORA_ERR_WORKSPACE;
     cudaStream_t st = (cudaStream_t)stream;
     uint8_t* wsb = static_cast<uint8_t*>(ws);
+    const uint16_t* Xl = X;
+    if (dp) {
+        rc = launch_dropout_x(X, M, K, wsb + p.total, *dp, sms, st);
+        if (rc != QLORA_OK) return rc;
+        Xl = reinterpret_cast<const uint16_t*>(wsb + p.total);
+    }
     if (M <= kSmallMaxM) {
-        rc = small_bwd(p, X, dY, w, A, B, scaling, T, dX, dA, dB, wsb, sms, st);
+        rc = small_bwd(p, Xl, dY, w, A, B, scaling, T, dX, dA, dB, wsb, sms, st, dp);
         if (rc == QLORA_OK) t_last_path = 1;
         return rc;
     }
@@ -897,7 +977,7 @@ int qlora_linear_bwd(const qlora_bf16* X, const qlora_bf16* dY, int64_t M, const
     // with a zero lo half
     const bool t_direct = T != nullptr && r % 8 == 0 && aligned16(T);
     if (T == nullptr) {
-        rc = compute_T(p, X, A, scaling, nullptr, wsb, sms, st);
+        rc = compute_T(p, Xl, A, scaling, nullptr, wsb, sms, st, dp ? dp->c : 1.f);
     } else if (!t_direct) {
         rc = launch_pdl(k_pad_cols, dim3((unsigned)grid_for(M * 2 * p.rp, 256, sms)), dim3(256), 0, st, T, M,
                         (int64_t)r, Thl, (int64_t)(2 * p.rp));
@@ -941,23 +1021,74 @@ int qlora_linear_bwd(const qlora_bf16* X, const qlora_bf16* dY, int64_t M, const
     {
         FinishArgs f = fin_none();
         f.Iout = r; f.Jiter = K; f.row_pair = p.rp;
-        f.o1 = dA; f.s1i = K; f.s1j = 1; f.J1 = K; f.J1pad = K; f.alpha1 = scaling;
-        rc = run_gemm<false, false>(Uhl, 2 * p.rp, X, K, 2 * p.rp, K, M, 2 * p.rp, K, p.zA, p.kA, part, f, sms, st);
+        f.o1 = dA; f.s1i = K; f.s1j = 1; f.J1 = K; f.J1pad = K;
+        f.alpha1 = dp ? (float)((double)scaling * (double)dp->c) : scaling;
+        rc = run_gemm<false, false>(Uhl, 2 * p.rp, Xl, K, 2 * p.rp, K, M, 2 * p.rp, K, p.zA, p.kA, part, f, sms, st);
         if (rc != QLORA_OK) return rc;
     }
-    // dX = dY W' + s U A
+    // dX = dY W' + s U A (with dropout: the fused kernel computes dY W' alone, then the
+    // masked LoRA term is added in place)
     rc = ensure_tc_attrs();
     if (rc != QLORA_OK) return rc;
     const int pairs = current_pairs();
+    const bool fused_lora = dp == nullptr;
+    const uint16_t* sU = reinterpret_cast<const uint16_t*>(wsb + p.off_sU);
+    int path;
     if (M > kPairMinM && pairs > 0) {
-        rc = launch_tc2<true>(w, dY, M, reinterpret_cast<const uint16_t*>(wsb + p.off_sU), p.lw, A, K, r, dX,
-                              pairs, st);
-        if (rc == QLORA_OK) t_last_path = 3;
-        return rc;
+        rc = launch_tc2<true>(w, dY, M, sU, p.lw, A, K, r, dX, pairs, st, fused_lora);
+        path = 3;
+    } else {
+        rc = launch_tc<true>(w, dY, M, sU, p.lw, A, K, r, dX, sms, st, fused_lora);
+        path = 2;
     }
-    rc = launch_tc<true>(w, dY, M, reinterpret_cast<const uint16_t*>(wsb + p.off_sU), p.lw, A, K, r, dX, sms, st);
-    if (rc == QLORA_OK) t_last_path = 2;
+    if (rc == QLORA_OK && dp) {
+        drop::DxArgs d{};
+        d.dX = dX; d.U = reinterpret_cast<const float*>(wsb + p.off_U32); d.ldu = p.rp; d.A = A;
+        d.M = M; d.K = K; d.r = r; d.sc = (float)((double)scaling * (double)dp->c);
+        drop::k_dx_lora_dropout<<<grid_for(M * K / 8, 256, sms), 256, 0, st>>>(d, *dp);
+        note_launch();
+        rc = launch_status();
+    }
+    if (rc == QLORA_OK) t_last_path = path;
     return rc;
+}
+
+int qlora_linear_fwd(const qlora_bf16* X, int64_t M, const nf4dq_weight* w, const qlora_bf16* A,
+                     const qlora_bf16* B, int r, float scaling, qlora_bf16* Y, qlora_bf16* T_out, void* ws,
+                     size_t ws_bytes, qlora_stream_t stream) {
+    return fwd_impl(X, M, w, A, B, r, scaling, Y, T_out, ws, ws_bytes, stream, nullptr);
+}
+
+int qlora_linear_bwd(const qlora_bf16* X, const qlora_bf16* dY, int64_t M, const nf4dq_weight* w,
+                     const qlora_bf16* A, const qlora_bf16* B, int r, float scaling, const qlora_bf16* T,
+                     qlora_bf16* dX, qlora_bf16* dA, qlora_bf16* dB, void* ws, size_t ws_bytes,
+                     qlora_stream_t stream) {
+    return bwd_impl(X, dY, M, w, A, B, r, scaling, T, dX, dA, dB, ws, ws_bytes, stream, nullptr);
+}
+
+size_t qlora_dropout_workspace_bytes(int64_t M, int64_t N, int64_t K, int r) {
+    const size_t b = qlora_workspace_bytes(M, N, K, r);
+    return b == 0 ? 0 : b + dropout_bytes(M, K);
+}
+
+int qlora_linear_fwd_dropout(const qlora_bf16* X, int64_t M, const nf4dq_weight* w, const qlora_bf16* A,
+                             const qlora_bf16* B, int r, float scaling, float dropout_p, uint64_t seed,
+                             uint64_t offset, qlora_bf16* Y, qlora_bf16* T_out, void* ws, size_t ws_bytes,
+                             qlora_stream_t stream) {
+    drop::Params d{};
+    const int rc = dropout_params(dropout_p, seed, offset, &d);
+    if (rc != QLORA_OK) return rc;
+    return fwd_impl(X, M, w, A, B, r, scaling, Y, T_out, ws, ws_bytes, stream, &d);
+}
+
+int qlora_linear_bwd_dropout(const qlora_bf16* X, const qlora_bf16* dY, int64_t M, const nf4dq_weight* w,
+                             const qlora_bf16* A, const qlora_bf16* B, int r, float scaling, float dropout_p,
+                             uint64_t seed, uint64_t offset, const qlora_bf16* T, qlora_bf16* dX, qlora_bf16* dA,
+                             qlora_bf16* dB, void* ws, size_t ws_bytes, qlora_stream_t stream) {
+    drop::Params d{};
+    const int rc = dropout_params(dropout_p, seed, offset, &d);
+    if (rc != QLORA_OK) return rc;
+    return bwd_impl(X, dY, M, w, A, B, r, scaling, T, dX, dA, dB, ws, ws_bytes, stream, &d);
 }
 
 

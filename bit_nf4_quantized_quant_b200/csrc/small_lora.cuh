@@ -18,6 +18,7 @@
 // 16-byte loads suffice; U and T stay in fp32 end to end.
 #pragma once
 #include "common.cuh"
+#include "dropout.cuh"
 
 namespace qnf4 {
 
@@ -112,6 +113,7 @@ struct LoraBwdArgs {
     int64_t M, N;
     int r, rp;
     float s;
+    float tscale;            // scale of the T32 values (1 except under LoRA dropout; Tb is taken as is)
     int b_vec;               // B rows are 16-byte loadable (r % 8 == 0, B 16-byte aligned)
     float* Upart;            // [US][M][rp] fp32 partial U (columns >= r not written)
     int US;                  // N splits of U; CTAs [0, US) compute U
@@ -216,7 +218,7 @@ __global__ void __launch_bounds__(kLoraThreads) k_lora_bwd_small(LoraBwdArgs a) 
             const int mm = e / kDbCols, j = e % kDbCols;
             float tv = 0.f;
             if (j < ic)
-                tv = a.T32 != nullptr ? a.T32[(int64_t)mm * a.rp + i0 + j]
+                tv = a.T32 != nullptr ? __fmul_rn(a.T32[(int64_t)mm * a.rp + i0 + j], a.tscale)
                                       : bf16lo_to_f32(a.Tb[(int64_t)mm * a.r + i0 + j]);
             s_T[e] = tv;
         }
@@ -264,8 +266,11 @@ struct BwdEndArgs {
     int64_t M, K;
     int r, rp;
     float s;
+    float s_da;              // scale of dA: s, or fl32(s c) under LoRA dropout
     uint16_t* dX;            // [M, K]
     uint16_t* dA;            // [r, K]
+    int dropout;             // 1: the LoRA term of dX is masked (keep * c); X above is then X * keep
+    drop::Params dp;
 };
 
 // The CTA that owns unit u under k_tcs_gemm's even split of U units over C
@@ -320,13 +325,17 @@ __global__ void __launch_bounds__(kLoraThreads) k_bwd_small_end(BwdEndArgs a) {
         for (int64_t c = c_first; c <= c_last; ++c) v += a.slots[(c + tile) * (a.NT * 128) + (int64_t)y * 128 + row];
         float l = 0.f;
         for (int i = 0; i < a.r; ++i) l = __fmaf_rn(s_u[i], bf16lo_to_f32(a.A[(int64_t)i * a.K + k]), l);
+        if (a.dropout) {                    // d Xd / d X = keep * c
+            const uint64_t e = (uint64_t)y * (uint64_t)a.K + (uint64_t)k;
+            l = ((drop::keep8(a.dp, e >> 3) >> (e & 7)) & 1u) ? __fmul_rn(l, a.dp.c) : 0.f;
+        }
         v = __fmaf_rn(a.s, l, v);
         a.dX[(int64_t)y * a.K + k] = (uint16_t)(pack_bf16x2(v, 0.f) & 0xffffu);
     } else {
         const int i = y - (int)a.M;
         float v = 0.f;
         for (int64_t m = 0; m < a.M; ++m) v = __fmaf_rn(s_u[m], bf16lo_to_f32(a.X[m * a.K + k]), v);
-        a.dA[(int64_t)i * a.K + k] = (uint16_t)(pack_bf16x2(a.s * v, 0.f) & 0xffffu);
+        a.dA[(int64_t)i * a.K + k] = (uint16_t)(pack_bf16x2(a.s_da * v, 0.f) & 0xffffu);
     }
 }
 

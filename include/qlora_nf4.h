@@ -178,6 +178,35 @@ QLORA_API int nf4_dequant(const nf4dq_weight* w, qlora_bf16* W_out, qlora_stream
 QLORA_API int nf4_dequant_merge(const nf4dq_weight* w, const qlora_bf16* A, const qlora_bf16* B, int r,
                                 float scaling, qlora_bf16* W_out, qlora_stream_t stream);
 
+/* One AdamW step of LoRA adapter parameters with 8-bit moment states
+ * ("Qlora Expert", Hyperparameter Guidance: paged_adamw_8bit, 8-bit Adam to
+ * cut optimizer memory; "QLoRA Implementation Details (2025 Edition)", Step
+ * 5: Paged Optimizer).  The paging itself (unified memory) is left to the
+ * caller's allocator; this is the step.  The pages give no state encoding;
+ * this library's reading:
+ *   - states m and v are stored per block of QLORA_ADAM_BLOCK consecutive
+ *     parameters as one fp32 scale and one FP8 E4M3 code per parameter
+ *     (1 sign, 4 exponent bits with bias 7, 3 mantissa bits, largest 448):
+ *     value = fl32(e4m3(code) * scale), scale = fl32(absmax / 448),
+ *     code = e4m3 round-to-nearest-even of fl32(value * fl32(448 / absmax)),
+ *     saturating at 448; code 0 when absmax = 0.  All-zero codes and scales
+ *     are the initial (zero) state.
+ *   - the update, every operation one IEEE fp32 rounding in this order:
+ *       m = b1*m + omb1*g;  v = b2*v + omb2*(g*g);  mh = m*rbc1;  vh = v*rbc2;
+ *       u = mh/(sqrt(vh) + eps) + weight_decay*p;  p = bf16_rne(p - lr*u)
+ *     with omb = fl32(1 - b), rbc = fl32(1 / (1 - b^step)) computed in double
+ *     on the host; then each block's m and v are requantized with its new
+ *     absmax.
+ * p [n] bf16 (in/out, 16-byte aligned), g [n] bf16 gradient (16-byte
+ * aligned), m_code, v_code [n] (in/out, 8-byte aligned), m_scale, v_scale
+ * [ceil(n / QLORA_ADAM_BLOCK)] fp32 (in/out), all device.  step >= 1 is the
+ * 1-based step count.  Errors: non-finite lr/eps/weight_decay or a beta
+ * outside [0, 1) -> QLORA_ERR_VALUE; n <= 0 -> QLORA_ERR_SHAPE. */
+#define QLORA_ADAM_BLOCK 256
+QLORA_API int adamw_8bit_step(qlora_bf16* p, const qlora_bf16* g, int64_t n, uint8_t* m_code, float* m_scale,
+                              uint8_t* v_code, float* v_scale, int64_t step, float lr, float beta1, float beta2,
+                              float eps, float weight_decay, qlora_stream_t stream);
+
 /* Bytes of device workspace that qlora_linear_fwd / qlora_linear_bwd need
  * for these sizes (0 is never returned for valid sizes; returns 0 for
  * invalid ones).  The same workspace may be reused by calls that run one
@@ -212,6 +241,37 @@ QLORA_API int qlora_linear_bwd(const qlora_bf16* X, const qlora_bf16* dY, int64_
                      const qlora_bf16* A, const qlora_bf16* B, int r, float scaling, const qlora_bf16* T,
                      qlora_bf16* dX, qlora_bf16* dA, qlora_bf16* dB, void* ws, size_t ws_bytes,
                      qlora_stream_t stream);
+
+/* LoRA dropout ("Qlora Expert", Implementation Pattern: lora_dropout=0.05;
+ * "QLoRA Implementation Details (2025 Edition)", Step 4: lora_dropout=0.1).
+ * The pages give only the rate; this library's reading: dropout on the LoRA
+ * branch's input, the base path unchanged,
+ *   Y  = X W'^T + s (Xd A^T) B^T,  T = Xd A^T,  Xd = X * keep * c,
+ *   c  = fl32(1 / (1 - p)),
+ * and its backward under the same mask:
+ *   U = dY B,  dX = dY W' + s (U A) * keep * c,  dA = s U^T Xd,  dB = s dY^T T.
+ * The kernels keep X * keep (exact in bf16) and apply c in fp32 to the
+ * accumulated T and dA and to the LoRA term of dX.
+ * Element e = m K + k of X is kept iff (word >> 8) >= llrint(p * 2^24), word
+ * being 32-bit word (e mod 8) (word 2i = the low half of output i) of the
+ * Philox4x64-10 output (Salmon et al., SC 2011) for counter
+ * (e div 8, offset, 0, 0) and key (seed, 0).  The forward and the backward
+ * of one step must be given the same (dropout_p, seed, offset); T given to
+ * the backward is the T_out of that forward.
+ * Arguments, layouts and errors are those of qlora_linear_fwd / _bwd, plus:
+ * 0 <= dropout_p < 1 (else QLORA_ERR_VALUE; 0 drops nothing), and the
+ * workspace must hold qlora_dropout_workspace_bytes(M, N, K, r) bytes (the
+ * regular workspace plus the dropped copy of X). */
+QLORA_API size_t qlora_dropout_workspace_bytes(int64_t M, int64_t N, int64_t K, int r);
+QLORA_API int qlora_linear_fwd_dropout(const qlora_bf16* X, int64_t M, const nf4dq_weight* w, const qlora_bf16* A,
+                                       const qlora_bf16* B, int r, float scaling, float dropout_p, uint64_t seed,
+                                       uint64_t offset, qlora_bf16* Y, qlora_bf16* T_out, void* ws, size_t ws_bytes,
+                                       qlora_stream_t stream);
+QLORA_API int qlora_linear_bwd_dropout(const qlora_bf16* X, const qlora_bf16* dY, int64_t M, const nf4dq_weight* w,
+                                       const qlora_bf16* A, const qlora_bf16* B, int r, float scaling,
+                                       float dropout_p, uint64_t seed, uint64_t offset, const qlora_bf16* T,
+                                       qlora_bf16* dX, qlora_bf16* dA, qlora_bf16* dB, void* ws, size_t ws_bytes,
+                                       qlora_stream_t stream);
 
 /* Human-readable text for a status code (static storage). */
 QLORA_API const char* qlora_status_string(int status);
