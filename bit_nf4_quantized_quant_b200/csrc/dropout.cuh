@@ -76,7 +76,12 @@ __global__ void __launch_bounds__(256) k_dropout_x(const uint16_t* __restrict__ 
 // the fused kernel with its LoRA steps switched off):
 //   l  = sum_j U[m, j] A[j, k]   (fp32, increasing j)
 //   dX = bf16_rne(fmaf(sc, l, fl32(dX)))  where kept, dX unchanged where dropped,
-//   sc = fl32(s c).  One thread per 8 consecutive k of one row.
+//   sc = fl32(s c).
+// A CTA takes 32 rows x 256 columns; thread (warp w, lane l) owns rows
+// 4w..4w+3 and columns 8l..8l+7.  Chunks of 64 LoRA terms are staged in
+// shared memory: A[j, tile columns] as bf16 by cp.async (read as one 16-byte
+// vector per lane), U[tile rows, j] transposed to fp32 [j][row] (a broadcast
+// read), so each A element is read from L2 once per 32 rows.
 struct DxArgs {
     uint16_t* dX;          // [M, K]
     const float* U;        // [M, ldu] fp32
@@ -87,32 +92,68 @@ struct DxArgs {
     float sc;
 };
 
-__global__ void __launch_bounds__(256) k_dx_lora_dropout(const DxArgs a, Params d) {
-    const int64_t total8 = a.M * a.K / 8;
-    for (int64_t e8 = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e8 < total8;
-         e8 += (int64_t)gridDim.x * blockDim.x) {
-        const int64_t m = (8 * e8) / a.K, k = (8 * e8) % a.K;
-        const uint32_t keep = keep8(d, (uint64_t)e8);
-        float l[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-        for (int j = 0; j < a.r; ++j) {
-            const float u = __ldg(a.U + m * a.ldu + j);
-            const uint4 av = ldg_nc_v4(a.A + (int64_t)j * a.K + k);
-            const uint32_t aw[4] = {av.x, av.y, av.z, av.w};
+constexpr int DX_TM = 32, DX_TK = 256, DX_JC = 64, DX_THREADS = 256;
+constexpr int DX_SMEM = DX_JC * DX_TK * 2 + DX_JC * DX_TM * 4;
+
+__global__ void __launch_bounds__(DX_THREADS) k_dx_lora_dropout(const DxArgs a, Params d) {
+    extern __shared__ __align__(16) uint8_t smem[];
+    float* sU = reinterpret_cast<float*>(smem + DX_JC * DX_TK * 2);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int64_t m0 = (int64_t)blockIdx.x * DX_TM, k0 = (int64_t)blockIdx.y * DX_TK;
+    float acc[4][8];
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                l[2 * q] = __fmaf_rn(u, bf16lo_to_f32(aw[q]), l[2 * q]);
-                l[2 * q + 1] = __fmaf_rn(u, bf16hi_to_f32(aw[q]), l[2 * q + 1]);
-            }
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int c = 0; c < 8; ++c) acc[i][c] = 0.f;
+    for (int j0 = 0; j0 < a.r; j0 += DX_JC) {
+        const int jc = min(DX_JC, a.r - j0);
+        if (j0 > 0) __syncthreads();
+        for (int i = tid; i < jc * (DX_TK / 8); i += DX_THREADS) {
+            const int jj = i / (DX_TK / 8), v = i % (DX_TK / 8);
+            const int64_t k = k0 + 8 * v;
+            const bool ok = k < a.K;
+            const uint16_t* src = ok ? a.A + (int64_t)(j0 + jj) * a.K + k : a.A;
+            const uint32_t dst = smem_u32(smem + (jj * DX_TK + 8 * v) * 2);
+            asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(ok ? 16 : 0)
+                         : "memory");
         }
-        uint4* p = reinterpret_cast<uint4*>(a.dX + 8 * e8);
+        asm volatile("cp.async.commit_group;" ::: "memory");
+        for (int i = tid; i < jc * DX_TM; i += DX_THREADS) {
+            const int jj = i / DX_TM, row = i % DX_TM;
+            const int64_t m = m0 + row;
+            sU[jj * DX_TM + row] = m < a.M ? __ldg(a.U + m * a.ldu + j0 + jj) : 0.f;
+        }
+        asm volatile("cp.async.wait_all;" ::: "memory");
+        __syncthreads();
+        for (int jj = 0; jj < jc; ++jj) {
+            const uint4 x = *reinterpret_cast<const uint4*>(smem + (jj * DX_TK + 8 * lane) * 2);
+            const float4 u = *reinterpret_cast<const float4*>(sU + jj * DX_TM + 4 * warp);
+            const float av[8] = {bf16lo_to_f32(x.x), bf16hi_to_f32(x.x), bf16lo_to_f32(x.y), bf16hi_to_f32(x.y),
+                                 bf16lo_to_f32(x.z), bf16hi_to_f32(x.z), bf16lo_to_f32(x.w), bf16hi_to_f32(x.w)};
+            const float uv[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+#pragma unroll
+                for (int c = 0; c < 8; ++c) acc[i][c] = __fmaf_rn(uv[i], av[c], acc[i][c]);
+        }
+    }
+    const int64_t k = k0 + 8 * lane;
+    if (k >= a.K) return;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const int64_t m = m0 + 4 * warp + i;
+        if (m >= a.M) break;
+        const int64_t e8 = (m * a.K + k) >> 3;
+        const uint32_t keep = keep8(d, (uint64_t)e8);
+        uint4* p = reinterpret_cast<uint4*>(a.dX + m * a.K + k);
         const uint4 b = *p;
         const uint32_t bw[4] = {b.x, b.y, b.z, b.w};
         uint32_t o[4];
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
             float lo = bf16lo_to_f32(bw[q]), hi = bf16hi_to_f32(bw[q]);
-            if ((keep >> (2 * q)) & 1u) lo = __fmaf_rn(a.sc, l[2 * q], lo);
-            if ((keep >> (2 * q + 1)) & 1u) hi = __fmaf_rn(a.sc, l[2 * q + 1], hi);
+            if ((keep >> (2 * q)) & 1u) lo = __fmaf_rn(a.sc, acc[i][2 * q], lo);
+            if ((keep >> (2 * q + 1)) & 1u) hi = __fmaf_rn(a.sc, acc[i][2 * q + 1], hi);
             o[q] = pack_bf16x2(lo, hi);
         }
         *p = make_uint4(o[0], o[1], o[2], o[3]);

@@ -1045,7 +1045,18 @@ static int bwd_impl(const qlora_bf16* X, const qlora_bf16* dY, int64_t M, const 
         drop::DxArgs d{};
         d.dX = dX; d.U = reinterpret_cast<const float*>(wsb + p.off_U32); d.ldu = p.rp; d.A = A;
         d.M = M; d.K = K; d.r = r; d.sc = (float)((double)scaling * (double)dp->c);
-        drop::k_dx_lora_dropout<<<grid_for(M * K / 8, 256, sms), 256, 0, st>>>(d, *dp);
+        static bool dx_attr[64];
+        int dev = 0;
+        if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return QLORA_ERR_DEVICE;
+        if (!dx_attr[dev]) {
+            std::lock_guard<std::mutex> lk(g_tc_mu);
+            if (cudaFuncSetAttribute(drop::k_dx_lora_dropout, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     drop::DX_SMEM) != cudaSuccess)
+                return QLORA_ERR_LAUNCH;
+            dx_attr[dev] = true;
+        }
+        const dim3 grid((unsigned)cdiv(M, drop::DX_TM), (unsigned)cdiv(K, drop::DX_TK));
+        drop::k_dx_lora_dropout<<<grid, drop::DX_THREADS, drop::DX_SMEM, st>>>(d, *dp);
         note_launch();
         rc = launch_status();
     }
