@@ -86,8 +86,9 @@ class ClockSampler:
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, gpu_index: int):
+    def __init__(self, gpu_index: int, period_ms: int = 200):
         self.gpu = gpu_index
+        self.period_ms = period_ms
         self.proc = None
         self.path = None
 
@@ -96,7 +97,7 @@ class ClockSampler:
         os.close(fd)
         try:
             self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
-                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                          "--format=csv,noheader,nounits", "-lms", str(self.period_ms)],
                                          stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
         except Exception:
             self.proc = None
@@ -125,7 +126,9 @@ class ClockSampler:
         reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower().startswith("active")})
         loaded = [v for v in sm if mx and v >= 0.5 * max(mx)] or sm
         return {"sm_mhz": statistics.median(loaded) if loaded else None,
-                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons, "samples": len(rows)}
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons, "samples": len(rows),
+                "sm_mhz_min": min(sm) if sm else None,
+                "power_w_max": max((float(r[3]) for r in rows if r[3].replace(".", "").isdigit()), default=None)}
 
 
 # ---------------------------------------------------------------------------
@@ -290,7 +293,7 @@ def run_ours(args, rank, world, local_rank):
                 dist.all_reduce(gbuf)
         torch.cuda.synchronize()
         stream = torch.cuda.current_stream()
-    clocks = ClockSampler(local_rank)
+    clocks = ClockSampler(local_rank, args.clock_ms)
     clocks.start()
     launches0 = ops.qlora_launch_count()
     t0 = torch.cuda.Event(enable_timing=True)
@@ -1016,6 +1019,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-graph", action="store_true", help="launch the timed steps eagerly instead of as CUDA graphs")
     ap.add_argument("--cpu-seconds", type=float, default=20.0)
+    ap.add_argument("--clock-ms", type=int, default=200, help="nvidia-smi clock sampling period during the timed region")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
 

@@ -3,15 +3,16 @@
 // scale c of kept values is applied in fp32 where T, dA and the LoRA term of
 // dX are formed), and the masked LoRA term of dX.
 //
-// Element e = m K + k of X is kept iff (word >> 8) >= t, t = llrint(p 2^24),
-// where word is 32-bit word (e mod 8) of the Philox4x64-10 output for counter
-// (e div 8, offset, 0, 0) and key (seed, 0) (Salmon, Moraes, Dror and Shaw,
+// Element e = m K + k of X is kept iff field >= t, t = llrint(p 2^16), where
+// field is 16-bit field (e mod 16) of the Philox4x64-10 output for counter
+// (e div 16, offset, 0, 0) and key (seed, 0) (Salmon, Moraes, Dror and Shaw,
 // SC 2011: per round (hi0, lo0) = M0 c0, (hi1, lo1) = M1 c2 as 128-bit
 // products, c = (hi1 ^ c1 ^ k0, lo1, hi0 ^ c3 ^ k1, lo0), and the key adds
-// the Weyl increments between rounds).  Kept values are scaled by
-// c = fl32(1 / (1 - p)).  One generator call serves the 8 consecutive
-// elements a thread handles (K % 64 == 0 keeps every 8-element group in one
-// row).
+// the Weyl increments between rounds); field 4i + j is bits 16j..16j+15 of
+// output i.  Kept values are scaled by c = fl32(1 / (1 - p)).  One generator
+// call serves 16 consecutive elements (K % 64 == 0 keeps every group in one
+// row); the backward generates the mask once, as a bitmask (bit e % 16 of
+// 16-bit word e / 16) that its later kernels read.
 #pragma once
 #include "common.cuh"
 
@@ -20,7 +21,7 @@ namespace drop {
 
 struct Params {
     uint64_t seed, offset;
-    uint32_t t;        // keep iff (word >> 8) >= t
+    uint32_t t;        // keep iff field >= t
     float c;           // scale of kept values
 };
 
@@ -39,37 +40,46 @@ __device__ __forceinline__ void philox4x64(uint64_t c0, uint64_t c1, uint64_t k0
     out[0] = c0; out[1] = c1; out[2] = c2; out[3] = c3;
 }
 
-// keep bits of elements 8 e8 .. 8 e8 + 7 (bit j = element 8 e8 + j)
-__device__ __forceinline__ uint32_t keep8(const Params& d, uint64_t e8) {
+// keep bits of elements 16 e16 .. 16 e16 + 15 (bit j = element 16 e16 + j)
+__device__ __forceinline__ uint32_t keep16(const Params& d, uint64_t e16) {
     uint64_t o[4];
-    philox4x64(e8, d.offset, d.seed, o);
+    philox4x64(e16, d.offset, d.seed, o);
     uint32_t bits = 0;
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-        const uint32_t word = (uint32_t)(o[j >> 1] >> (32 * (j & 1)));
-        bits |= ((word >> 8) >= d.t ? 1u : 0u) << j;
+    for (int j = 0; j < 16; ++j) {
+        const uint32_t field = (uint32_t)(o[j >> 2] >> (16 * (j & 3))) & 0xffffu;
+        bits |= (field >= d.t ? 1u : 0u) << j;
     }
     return bits;
 }
 
-// Xd [M, K] = X where kept, 0 where dropped (exact; the scale c of kept values is applied in
-// fp32 where T and dA are formed); one thread per 8 elements.
-__global__ void __launch_bounds__(256) k_dropout_x(const uint16_t* __restrict__ X, int64_t total8,
-                                                   uint16_t* __restrict__ Xd, Params d) {
-    for (int64_t e8 = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e8 < total8;
-         e8 += (int64_t)gridDim.x * blockDim.x) {
-        const uint32_t keep = keep8(d, (uint64_t)e8);
-        const uint4 x = ldg_nc_v4(X + 8 * e8);
-        const uint32_t xw[4] = {x.x, x.y, x.z, x.w};
-        uint32_t o[4];
+// Xd [M, K] = X where kept, 0 where dropped; when mask is given, also its
+// keep bits (one 16-bit word per 16 elements).  One thread per 16 elements.
+__global__ void __launch_bounds__(256) k_dropout_x(const uint16_t* __restrict__ X, int64_t total16,
+                                                   uint16_t* __restrict__ Xd, uint16_t* __restrict__ mask,
+                                                   Params d) {
+    for (int64_t e16 = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e16 < total16;
+         e16 += (int64_t)gridDim.x * blockDim.x) {
+        const uint32_t keep = keep16(d, (uint64_t)e16);
+        const uint4 x0 = ldg_nc_v4(X + 16 * e16), x1 = ldg_nc_v4(X + 16 * e16 + 8);
+        const uint32_t xw[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+        uint32_t o[8];
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
+        for (int j = 0; j < 8; ++j) {
             const uint32_t lo = (keep >> (2 * j)) & 1u ? (xw[j] & 0xffffu) : 0u;
             const uint32_t hi = (keep >> (2 * j + 1)) & 1u ? (xw[j] & 0xffff0000u) : 0u;
             o[j] = lo | hi;
         }
-        *reinterpret_cast<uint4*>(Xd + 8 * e8) = make_uint4(o[0], o[1], o[2], o[3]);
+        uint4* dst = reinterpret_cast<uint4*>(Xd + 16 * e16);
+        dst[0] = make_uint4(o[0], o[1], o[2], o[3]);
+        dst[1] = make_uint4(o[4], o[5], o[6], o[7]);
+        if (mask) mask[e16] = (uint16_t)keep;
     }
+}
+
+// keep bit of element e from the bitmask
+__device__ __forceinline__ uint32_t mask_bit(const uint16_t* mask, uint64_t e) {
+    return ((uint32_t)__ldg(mask + (e >> 4)) >> (e & 15)) & 1u;
 }
 
 // dX [M, K] += masked LoRA term, in place on the bf16 base dY W' (written by
@@ -87,6 +97,7 @@ struct DxArgs {
     const float* U;        // [M, ldu] fp32
     int64_t ldu;
     const uint16_t* A;     // [r, K]
+    const uint16_t* mask;  // keep bits of [M, K] (k_dropout_x)
     int64_t M, K;
     int r;
     float sc;
@@ -95,7 +106,7 @@ struct DxArgs {
 constexpr int DX_TM = 32, DX_TK = 256, DX_JC = 64, DX_THREADS = 256;
 constexpr int DX_SMEM = DX_JC * DX_TK * 2 + DX_JC * DX_TM * 4;
 
-__global__ void __launch_bounds__(DX_THREADS) k_dx_lora_dropout(const DxArgs a, Params d) {
+__global__ void __launch_bounds__(DX_THREADS) k_dx_lora_dropout(const DxArgs a) {
     extern __shared__ __align__(16) uint8_t smem[];
     float* sU = reinterpret_cast<float*>(smem + DX_JC * DX_TK * 2);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -143,8 +154,8 @@ __global__ void __launch_bounds__(DX_THREADS) k_dx_lora_dropout(const DxArgs a, 
     for (int i = 0; i < 4; ++i) {
         const int64_t m = m0 + 4 * warp + i;
         if (m >= a.M) break;
-        const int64_t e8 = (m * a.K + k) >> 3;
-        const uint32_t keep = keep8(d, (uint64_t)e8);
+        const uint64_t e = (uint64_t)(m * a.K + k);     // a multiple of 8: bits e % 16 .. e % 16 + 7
+        const uint32_t keep = ((uint32_t)__ldg(a.mask + (e >> 4)) >> (e & 15)) & 0xffu;
         uint4* p = reinterpret_cast<uint4*>(a.dX + m * a.K + k);
         const uint4 b = *p;
         const uint32_t bw[4] = {b.x, b.y, b.z, b.w};

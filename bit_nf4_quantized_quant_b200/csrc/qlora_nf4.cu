@@ -675,7 +675,7 @@ int small_fwd(const Plan& p, const uint16_t* X, const uint16_t* Xl, const nf4dq_
 // the U / dB kernel), then dX = dY W' + s U A and dA.
 int small_bwd(const Plan& p, const uint16_t* Xl, const uint16_t* dY, const nf4dq_weight* w, const uint16_t* A,
               const uint16_t* B, float scaling, const uint16_t* T, uint16_t* dX, uint16_t* dA, uint16_t* dB,
-              uint8_t* wsb, int sms, cudaStream_t st, const drop::Params* dp) {
+              uint8_t* wsb, int sms, cudaStream_t st, const drop::Params* dp, const uint16_t* mask) {
     int rc = QLORA_OK;
     const float* T32 = nullptr;
     if (T == nullptr) {
@@ -700,7 +700,7 @@ int small_bwd(const Plan& p, const uint16_t* Xl, const uint16_t* dY, const nf4dq
     BwdEndArgs e{};
     e.slots = ta.slots; e.NT = p.NT; e.nks = ta.nks; e.ctas = ta.ctas; e.units = ta.units;
     e.Upart = b.Upart; e.US = p.US; e.A = A; e.X = Xl;
-    if (dp) { e.dropout = 1; e.dp = *dp; }
+    if (dp) { e.mask = mask; e.c = dp->c; }
     e.M = p.M; e.K = p.K; e.r = p.r; e.rp = p.rp; e.s = scaling; e.dX = dX; e.dA = dA;
     e.s_da = dp ? (float)((double)scaling * (double)dp->c) : scaling;
     return launch_pdl(k_bwd_small_end, dim3((unsigned)cdiv(p.K, kLoraThreads), (unsigned)(p.M + p.r)),
@@ -709,22 +709,25 @@ int small_bwd(const Plan& p, const uint16_t* Xl, const uint16_t* dY, const nf4dq
 
 // Bytes of the dropped copy of X that the dropout entry points need past the
 // regular workspace plan.
-size_t dropout_bytes(int64_t M, int64_t K) { return align256((size_t)M * (size_t)K * 2); }
+size_t dropout_bytes(int64_t M, int64_t K) {
+    return align256((size_t)M * (size_t)K * 2) + align256((size_t)M * (size_t)K / 8);
+}
 
 int dropout_params(float p, uint64_t seed, uint64_t offset, drop::Params* d) {
     if (!(p >= 0.f && p < 1.f)) return QLORA_ERR_VALUE;
     d->seed = seed;
     d->offset = offset;
-    d->t = (uint32_t)std::llrint((double)p * 16777216.0);
+    d->t = (uint32_t)std::llrint((double)p * 65536.0);
     d->c = (float)(1.0 / (1.0 - (double)p));
     return QLORA_OK;
 }
 
-// Xd = the dropped and scaled copy of X [M, K] (into the workspace).
-int launch_dropout_x(const uint16_t* X, int64_t M, int64_t K, uint8_t* dst, const drop::Params& d, int sms,
-                     cudaStream_t st) {
-    const int64_t total8 = M * K / 8;
-    drop::k_dropout_x<<<grid_for(total8, 256, sms), 256, 0, st>>>(X, total8, reinterpret_cast<uint16_t*>(dst), d);
+// Xd = X * keep [M, K] into the workspace, and (mask non-null) its keep bits.
+int launch_dropout_x(const uint16_t* X, int64_t M, int64_t K, uint8_t* dst, uint16_t* mask, const drop::Params& d,
+                     int sms, cudaStream_t st) {
+    const int64_t total16 = M * K / 16;
+    drop::k_dropout_x<<<grid_for(total16, 256, sms), 256, 0, st>>>(X, total16, reinterpret_cast<uint16_t*>(dst),
+                                                                   mask, d);
     note_launch();
     return launch_status();
 }
@@ -894,7 +897,7 @@ static int fwd_impl(const qlora_bf16* X, int64_t M, const nf4dq_weight* w, const
     uint8_t* wsb = static_cast<uint8_t*>(ws);
     const uint16_t* Xl = X;
     if (dp) {
-        rc = launch_dropout_x(X, M, w->K, wsb + p.total, *dp, sms, st);
+        rc = launch_dropout_x(X, M, w->K, wsb + p.total, nullptr, *dp, sms, st);
         if (rc != QLORA_OK) return rc;
         Xl = reinterpret_cast<const uint16_t*>(wsb + p.total);
     }
@@ -957,13 +960,15 @@ static int bwd_impl(const qlora_bf16* X, const qlora_bf16* dY, int64_t M, const 
     cudaStream_t st = (cudaStream_t)stream;
     uint8_t* wsb = static_cast<uint8_t*>(ws);
     const uint16_t* Xl = X;
+    uint16_t* mask = nullptr;
     if (dp) {
-        rc = launch_dropout_x(X, M, K, wsb + p.total, *dp, sms, st);
+        mask = reinterpret_cast<uint16_t*>(wsb + p.total + align256((size_t)M * (size_t)K * 2));
+        rc = launch_dropout_x(X, M, K, wsb + p.total, mask, *dp, sms, st);
         if (rc != QLORA_OK) return rc;
         Xl = reinterpret_cast<const uint16_t*>(wsb + p.total);
     }
     if (M <= kSmallMaxM) {
-        rc = small_bwd(p, Xl, dY, w, A, B, scaling, T, dX, dA, dB, wsb, sms, st, dp);
+        rc = small_bwd(p, Xl, dY, w, A, B, scaling, T, dX, dA, dB, wsb, sms, st, dp, mask);
         if (rc == QLORA_OK) t_last_path = 1;
         return rc;
     }
@@ -1043,7 +1048,7 @@ static int bwd_impl(const qlora_bf16* X, const qlora_bf16* dY, int64_t M, const 
     }
     if (rc == QLORA_OK && dp) {
         drop::DxArgs d{};
-        d.dX = dX; d.U = reinterpret_cast<const float*>(wsb + p.off_U32); d.ldu = p.rp; d.A = A;
+        d.dX = dX; d.U = reinterpret_cast<const float*>(wsb + p.off_U32); d.ldu = p.rp; d.A = A; d.mask = mask;
         d.M = M; d.K = K; d.r = r; d.sc = (float)((double)scaling * (double)dp->c);
         static bool dx_attr[64];
         int dev = 0;
@@ -1056,7 +1061,7 @@ static int bwd_impl(const qlora_bf16* X, const qlora_bf16* dY, int64_t M, const 
             dx_attr[dev] = true;
         }
         const dim3 grid((unsigned)cdiv(M, drop::DX_TM), (unsigned)cdiv(K, drop::DX_TK));
-        drop::k_dx_lora_dropout<<<grid, drop::DX_THREADS, drop::DX_SMEM, st>>>(d, *dp);
+        drop::k_dx_lora_dropout<<<grid, drop::DX_THREADS, drop::DX_SMEM, st>>>(d);
         note_launch();
         rc = launch_status();
     }

@@ -269,8 +269,9 @@ struct BwdEndArgs {
     float s_da;              // scale of dA: s, or fl32(s c) under LoRA dropout
     uint16_t* dX;            // [M, K]
     uint16_t* dA;            // [r, K]
-    int dropout;             // 1: the LoRA term of dX is masked (keep * c); X above is then X * keep
-    drop::Params dp;
+    const uint16_t* mask;    // LoRA dropout: keep bits of [M, K] (the LoRA term of dX is masked, keep * c,
+                             // and X above is then X * keep); null without dropout
+    float c;                 // scale of kept values
 };
 
 // The CTA that owns unit u under k_tcs_gemm's even split of U units over C
@@ -325,10 +326,8 @@ __global__ void __launch_bounds__(kLoraThreads) k_bwd_small_end(BwdEndArgs a) {
         for (int64_t c = c_first; c <= c_last; ++c) v += a.slots[(c + tile) * (a.NT * 128) + (int64_t)y * 128 + row];
         float l = 0.f;
         for (int i = 0; i < a.r; ++i) l = __fmaf_rn(s_u[i], bf16lo_to_f32(a.A[(int64_t)i * a.K + k]), l);
-        if (a.dropout) {                    // d Xd / d X = keep * c
-            const uint64_t e = (uint64_t)y * (uint64_t)a.K + (uint64_t)k;
-            l = ((drop::keep8(a.dp, e >> 3) >> (e & 7)) & 1u) ? __fmul_rn(l, a.dp.c) : 0.f;
-        }
+        if (a.mask)                         // d Xd / d X = keep * c
+            l = drop::mask_bit(a.mask, (uint64_t)y * (uint64_t)a.K + (uint64_t)k) ? __fmul_rn(l, a.c) : 0.f;
         v = __fmaf_rn(a.s, l, v);
         a.dX[(int64_t)y * a.K + k] = (uint16_t)(pack_bf16x2(v, 0.f) & 0xffffu);
     } else {

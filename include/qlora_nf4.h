@@ -252,16 +252,16 @@ QLORA_API int qlora_linear_bwd(const qlora_bf16* X, const qlora_bf16* dY, int64_
  *   U = dY B,  dX = dY W' + s (U A) * keep * c,  dA = s U^T Xd,  dB = s dY^T T.
  * The kernels keep X * keep (exact in bf16) and apply c in fp32 to the
  * accumulated T and dA and to the LoRA term of dX.
- * Element e = m K + k of X is kept iff (word >> 8) >= llrint(p * 2^24), word
- * being 32-bit word (e mod 8) (word 2i = the low half of output i) of the
- * Philox4x64-10 output (Salmon et al., SC 2011) for counter
- * (e div 8, offset, 0, 0) and key (seed, 0).  The forward and the backward
+ * Element e = m K + k of X is kept iff field >= llrint(p * 2^16), field
+ * being 16-bit field (e mod 16) (field 4i + j = bits 16j..16j+15 of output
+ * i) of the Philox4x64-10 output (Salmon et al., SC 2011) for counter
+ * (e div 16, offset, 0, 0) and key (seed, 0).  The forward and the backward
  * of one step must be given the same (dropout_p, seed, offset); T given to
  * the backward is the T_out of that forward.
  * Arguments, layouts and errors are those of qlora_linear_fwd / _bwd, plus:
  * 0 <= dropout_p < 1 (else QLORA_ERR_VALUE; 0 drops nothing), and the
  * workspace must hold qlora_dropout_workspace_bytes(M, N, K, r) bytes (the
- * regular workspace plus the dropped copy of X). */
+ * regular workspace plus the dropped copy of X and its keep bitmask). */
 QLORA_API size_t qlora_dropout_workspace_bytes(int64_t M, int64_t N, int64_t K, int r);
 QLORA_API int qlora_linear_fwd_dropout(const qlora_bf16* X, int64_t M, const nf4dq_weight* w, const qlora_bf16* A,
                                        const qlora_bf16* B, int r, float scaling, float dropout_p, uint64_t seed,

@@ -598,10 +598,10 @@ int oracle_adamw8_step(uint16_t* p, const uint16_t* g, int64_t n, uint8_t* m_cod
  *   round:  (hi0, lo0) = M0 * c0,  (hi1, lo1) = M1 * c2  (128-bit products)
  *           c = (hi1 ^ c1 ^ k0, lo1, hi0 ^ c3 ^ k1, lo0)
  *   key:    (k0, k1) += (W0, W1) between rounds; 10 rounds.
- * Element e = m K + k uses 32-bit word (e mod 8) of the 256-bit output for
- * counter (e div 8, offset, 0, 0) and key (seed, 0), words in little-endian
- * order (word 2i is the low half of output i); it is kept iff
- * (word >> 8) >= t, t = llrint(p * 2^24).
+ * Element e = m K + k uses 16-bit field (e mod 16) of the 256-bit output for
+ * counter (e div 16, offset, 0, 0) and key (seed, 0), fields in little-endian
+ * order (field 4i + j is bits 16j .. 16j + 15 of output i); it is kept iff
+ * field >= t, t = llrint(p * 2^16).
  * ========================================================================= */
 static const uint64_t PHILOX_M0 = 0xD2E7470EE14C6C93ull, PHILOX_M1 = 0xCA5A826395121157ull;
 static const uint64_t PHILOX_W0 = 0x9E3779B97F4A7C15ull, PHILOX_W1 = 0xBB67AE8584CAA73Bull;
@@ -632,15 +632,15 @@ void oracle_philox4x64(const uint64_t ctr_in[4], const uint64_t key_in[2], uint6
 int oracle_dropout_mask(uint64_t seed, uint64_t offset, int64_t M, int64_t K, float p, uint8_t* keep)
 {
     if (M <= 0 || K <= 0 || !(p >= 0.0f && p < 1.0f)) return -1;
-    const uint32_t t = (uint32_t)llrint((double)p * 16777216.0);
+    const uint32_t t = (uint32_t)llrint((double)p * 65536.0);
     const uint64_t key[2] = {seed, 0};
-    for (int64_t e8 = 0; e8 * 8 < M * K; ++e8) {
-        const uint64_t ctr[4] = {(uint64_t)e8, offset, 0, 0};
+    for (int64_t e16 = 0; e16 * 16 < M * K; ++e16) {
+        const uint64_t ctr[4] = {(uint64_t)e16, offset, 0, 0};
         uint64_t o[4];
         oracle_philox4x64(ctr, key, o);
-        for (int j = 0; j < 8 && e8 * 8 + j < M * K; ++j) {
-            uint32_t word = (uint32_t)(o[j / 2] >> (32 * (j % 2)));
-            keep[e8 * 8 + j] = (uint8_t)((word >> 8) >= t);
+        for (int j = 0; j < 16 && e16 * 16 + j < M * K; ++j) {
+            uint32_t field = (uint32_t)((o[j / 4] >> (16 * (j % 4))) & 0xffffu);
+            keep[e16 * 16 + j] = (uint8_t)(field >= t);
         }
     }
     return 0;

@@ -38,7 +38,7 @@ def test_mask_determinism_and_offsets(oracle_mod):
     assert not np.array_equal(a, oracle_mod.dropout_mask(7, 4, 16, 256, 0.1))
     assert not np.array_equal(a, oracle_mod.dropout_mask(8, 3, 16, 256, 0.1))
     assert oracle_mod.dropout_mask(7, 3, 16, 256, 0.0).all()
-    # element e uses word e % 8 of block e // 8: a row-major [M, K] mask is one flat stream
+    # element e uses field e % 16 of block e // 16: a row-major [M, K] mask is one flat stream
     flat = oracle_mod.dropout_mask(7, 3, 1, 16 * 256, 0.1).reshape(16, 256)
     assert np.array_equal(a, flat)
 
