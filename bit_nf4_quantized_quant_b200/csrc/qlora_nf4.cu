@@ -428,10 +428,14 @@ int ensure_tc_attrs() {
                 cudaSuccess ||
             cudaFuncSetAttribute(tc::k_tc_gemm<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, tc::SMEM_ALLOC) !=
                 cudaSuccess ||
-            cudaFuncSetAttribute(tc2::k_tc2_gemm<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 tc2::SMEM_ALLOC) != cudaSuccess ||
-            cudaFuncSetAttribute(tc2::k_tc2_gemm<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 tc2::SMEM_ALLOC) != cudaSuccess ||
+            cudaFuncSetAttribute(tc2::k_tc2_gemm<false, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 tc2::Lay<1>::SMEM_ALLOC) != cudaSuccess ||
+            cudaFuncSetAttribute(tc2::k_tc2_gemm<true, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 tc2::Lay<1>::SMEM_ALLOC) != cudaSuccess ||
+            cudaFuncSetAttribute(tc2::k_tc2_gemm<false, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 tc2::Lay<2>::SMEM_ALLOC) != cudaSuccess ||
+            cudaFuncSetAttribute(tc2::k_tc2_gemm<true, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 tc2::Lay<2>::SMEM_ALLOC) != cudaSuccess ||
             cudaFuncSetAttribute(tcs::k_tcs_gemm<16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  tcs::SMEM_ALLOC) != cudaSuccess ||
             cudaFuncSetAttribute(tcs::k_tcs_gemm<32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -444,15 +448,15 @@ int ensure_tc_attrs() {
         attr.val.clusterDim.x = 2; attr.val.clusterDim.y = 1; attr.val.clusterDim.z = 1;
         cfg.gridDim = dim3(2 * 74, 1, 1);
         cfg.blockDim = dim3(tc2::kThreads, 1, 1);
-        cfg.dynamicSmemBytes = tc2::SMEM_ALLOC;
+        cfg.dynamicSmemBytes = tc2::Lay<1>::SMEM_ALLOC;
         cfg.attrs = nullptr;
         cfg.numAttrs = 0;               // the kernel carries its cluster shape (__cluster_dims__)
         int nclusters = 0;
-        if (cudaOccupancyMaxActiveClusters(&nclusters, tc2::k_tc2_gemm<false>, &cfg) != cudaSuccess) {
+        if (cudaOccupancyMaxActiveClusters(&nclusters, tc2::k_tc2_gemm<false, 1>, &cfg) != cudaSuccess) {
             cudaGetLastError();
             cfg.attrs = &attr;
             cfg.numAttrs = 1;
-            if (cudaOccupancyMaxActiveClusters(&nclusters, tc2::k_tc2_gemm<false>, &cfg) != cudaSuccess) {
+            if (cudaOccupancyMaxActiveClusters(&nclusters, tc2::k_tc2_gemm<false, 1>, &cfg) != cudaSuccess) {
                 cudaGetLastError();
                 nclusters = 0;
             }
@@ -496,6 +500,18 @@ int launch_tc(const nf4dq_weight* w, const uint16_t* act, int64_t M, const uint1
     return launch_status();
 }
 
+// Token tiles of 256 per SM-pair tile: 2 when a decoded W' stage can feed two
+// of them (halving the decode work per flop) without losing more to wave
+// quantization than that gains.  Measured on the 7B block at M = 2048: a
+// two-tile tile runs 1.2x the flop rate of a one-tile tile, so a wave of them
+// costs about 5/3 of a one-tile wave.
+int tc2_token_tiles(int64_t M, int64_t n_out, int pairs) {
+    const int64_t m1 = cdiv(M, tc2::BM), m2 = cdiv(M, 2 * tc2::BM), nt = cdiv(n_out, tc2::BN);
+    if (m1 < 2 || pairs <= 0) return 1;
+    const int64_t w1 = cdiv(m1 * nt, pairs), w2 = cdiv(m2 * nt, pairs);
+    return 5 * w2 <= 3 * w1 ? 2 : 1;
+}
+
 // The same on SM pairs (cta_group::2), 256 x 256 tiles.
 template <bool BWD>
 int launch_tc2(const nf4dq_weight* w, const uint16_t* act, int64_t M, const uint16_t* lact, int lw,
@@ -515,10 +531,16 @@ int launch_tc2(const nf4dq_weight* w, const uint16_t* act, int64_t M, const uint
     a.codes = w->codes; a.scale = w->scale; a.mean = w->mean;
     a.lora_w = lora_w; a.ldl = ldl; a.r = r; a.lper = (int)rup(r, 16); a.nlora = lora ? (int)cdiv(lw, 64) : 0;
     a.out = out; a.M = M; a.N = N; a.K = K; a.n_out = n_out; a.n_red = n_red;
-    const int64_t ntiles = cdiv(M, tc2::BM) * cdiv(n_out, tc2::BN);
+    const int mt = tc2_token_tiles(M, n_out, pairs);
+    const int64_t ntiles = cdiv(M, (int64_t)tc2::BM * mt) * cdiv(n_out, tc2::BN);
     const int np = (int)(ntiles < pairs ? ntiles : pairs);
     hook_before(st);
-    tc2::k_tc2_gemm<BWD><<<2 * np, tc2::kThreads, tc2::SMEM_ALLOC, st>>>(tmA, tmL, tmP, a, tables(w->quant_type));
+    if (mt == 2)
+        tc2::k_tc2_gemm<BWD, 2><<<2 * np, tc2::kThreads, tc2::Lay<2>::SMEM_ALLOC, st>>>(tmA, tmL, tmP, a,
+                                                                                        tables(w->quant_type));
+    else
+        tc2::k_tc2_gemm<BWD, 1><<<2 * np, tc2::kThreads, tc2::Lay<1>::SMEM_ALLOC, st>>>(tmA, tmL, tmP, a,
+                                                                                        tables(w->quant_type));
     hook_after(st);
     note_launch();
     return launch_status();

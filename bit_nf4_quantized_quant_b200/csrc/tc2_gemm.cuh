@@ -37,12 +37,6 @@ using tc::Args;
 
 constexpr int BM = 256, BN = 256, BK = 64;       // pair tile
 constexpr int HM = 128, HN = 128;                // per-CTA halves
-constexpr int SA = 5, SW = 6, SP = 8;
-// The W' and packed rings are split into one sub-ring per dequantizer group
-// (SW / 2 and SP / 2 stages), each filled and drained in that group's step
-// order, so every waiter is at most one phase ahead of the barrier it waits on
-// (a parity wait cannot tell phase k from phase k - 2).
-constexpr int SWH = SW / 2, SPH = SP / 2;
 constexpr int A_BYTES = HM * BK * 2;             // 16 KB
 constexpr int W_BYTES = HN * BK * 2;             // 16 KB
 constexpr int P_BYTES = HN * BK / 2;             // 4 KB
@@ -52,16 +46,33 @@ constexpr int kGroupWarps = kGroupThreads / 32;
 constexpr int kEpiWarps = 4;
 constexpr int kTmemCols = 512;
 
-constexpr int OFF_A = 0;
-constexpr int OFF_W = OFF_A + SA * A_BYTES;
-constexpr int OFF_P = OFF_W + SW * W_BYTES;
-constexpr int OFF_BAR = OFF_P + SP * P_BYTES;
-constexpr int NBAR = 2 * SA + 2 * SW + 2 * SP + 4 + 1 + SW;   // + peer-local fullWl[SW]
-constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
-// per dequantizer thread, 2 slots x (code word, scale, mean) of prefetched block-constant inputs
-constexpr int OFF_C = OFF_MISC + 16;
-constexpr int SMEM_BYTES = OFF_C + 2 * 3 * 2 * kGroupThreads * 4;
-constexpr int SMEM_ALLOC = SMEM_BYTES + 1024;
+// Shared-memory layout for MT token tiles of 256 per pair tile.  MT = 1: one
+// accumulator per tile, two in TMEM so the epilogue of a tile overlaps the next
+// tile's main loop.  MT = 2: each decoded W' stage feeds the MMAs of two token
+// tiles (two accumulators, all of TMEM), which halves the decode work per
+// flop; the epilogue then drains both before the next tile starts.
+//   SA: activation slots (one token tile's 128 x 64 half each; a step takes MT)
+//   SW / SP: W' and packed stages, split into one sub-ring per dequantizer
+//   group (SW / 2 and SP / 2 stages), each filled and drained in that group's
+//   step order, so every waiter is at most one phase ahead of the barrier it
+//   waits on (a parity wait cannot tell phase k from phase k - 2).
+template <int MT>
+struct Lay {
+    static constexpr int SA = MT == 1 ? 5 : 6, SW = 6, SP = MT == 1 ? 8 : 4;
+    static constexpr int SWH = SW / 2, SPH = SP / 2;
+    static constexpr int NACC = 2 / MT;          // accumulator buffers (TMEM holds 2 x 256 columns)
+    static constexpr int OFF_A = 0;
+    static constexpr int OFF_W = OFF_A + SA * A_BYTES;
+    static constexpr int OFF_P = OFF_W + SW * W_BYTES;
+    static constexpr int OFF_BAR = OFF_P + SP * P_BYTES;
+    static constexpr int NBAR = 2 * SA + 2 * SW + 2 * SP + 4 + 1 + SW;   // + peer-local fullWl[SW]
+    static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
+    // per dequantizer thread, 2 slots x (code word, scale, mean) of prefetched block-constant inputs
+    static constexpr int OFF_C = OFF_MISC + 16;
+    static constexpr int SMEM_BYTES = OFF_C + 2 * 3 * 2 * kGroupThreads * 4;
+    static constexpr int SMEM_ALLOC = SMEM_BYTES + 1024;
+};
+static_assert(Lay<1>::SMEM_ALLOC <= 232448 && Lay<2>::SMEM_ALLOC <= 232448, "shared memory");
 
 __device__ __forceinline__ uint32_t cluster_rank() {
     uint32_t r;
@@ -177,10 +188,14 @@ __device__ __forceinline__ uint32_t p_chunk_offset(int t, int c) {
     return (uint32_t)(n * 64 + (((2 * j + c) ^ ((n >> 1) & 3)) << 4));
 }
 
-template <bool BWD>
+template <bool BWD, int MT>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 k_tc2_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmL,
            const __grid_constant__ CUtensorMap tmP, Args a, NF4Tables tab) {
+    using L = Lay<MT>;
+    constexpr int SA = L::SA, SW = L::SW, SP = L::SP, SWH = L::SWH, SPH = L::SPH, NACC = L::NACC;
+    constexpr int OFF_A = L::OFF_A, OFF_W = L::OFF_W, OFF_P = L::OFF_P, OFF_BAR = L::OFF_BAR;
+    constexpr int OFF_MISC = L::OFF_MISC, OFF_C = L::OFF_C;
     extern __shared__ __align__(1024) uint8_t smem[];
     uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem) + 1023) & ~(uintptr_t)1023);
     const uint32_t sbase = smem_u32(base);
@@ -202,7 +217,7 @@ k_tc2_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
     const uint32_t crank = cluster_rank();
     const bool leader = crank == 0;
     const int64_t pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
-    const int64_t mtiles = cdiv(a.M, BM), ntiles_n = cdiv(a.n_out, BN);
+    const int64_t mtiles = cdiv(a.M, (int64_t)BM * MT), ntiles_n = cdiv(a.n_out, BN);   // token groups
     const int64_t ntiles = mtiles * ntiles_n;
     const int nks = (int)cdiv(a.n_red, BK);
     const int nsteps = nks + a.nlora;
@@ -271,15 +286,18 @@ k_tc2_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
             int sa = 0, pa = 0, issued = 0;
             bool ok = true;
             for (int64_t tile = pair; tile < ntiles && ok; tile += npairs) {
-                const int m0 = (int)((tile % mtiles) * BM + crank * HM);
+                const int m0 = (int)((tile % mtiles) * BM * MT + crank * HM);
                 for (int step = 0; step < nsteps && ok; ++step) {
-                    if (!(ok = tc::mbar_wait(emptyA(sa), pa ^ 1, s_abort))) break;
-                    if (leader) tc::mbar_expect_tx(fullA(sa), 2 * A_BYTES);     // both halves land here
-                    const uint32_t bar = mapa(fullA(sa), 0);
-                    if (step < nks) tma_load_2d_pair(sbase + OFF_A + sa * A_BYTES, &tmA, bar, step * BK, m0);
-                    else tma_load_2d_pair(sbase + OFF_A + sa * A_BYTES, &tmL, bar, (step - nks) * BK, m0);
-                    ++issued;
-                    if (++sa == SA) { sa = 0; pa ^= 1; }
+#pragma unroll
+                    for (int u = 0; u < MT && ok; ++u) {          // token tile u of the group
+                        if (!(ok = tc::mbar_wait(emptyA(sa), pa ^ 1, s_abort))) break;
+                        if (leader) tc::mbar_expect_tx(fullA(sa), 2 * A_BYTES);     // both halves land here
+                        const uint32_t bar = mapa(fullA(sa), 0);
+                        if (step < nks) tma_load_2d_pair(sbase + OFF_A + sa * A_BYTES, &tmA, bar, step * BK, m0 + u * BM);
+                        else tma_load_2d_pair(sbase + OFF_A + sa * A_BYTES, &tmL, bar, (step - nks) * BK, m0 + u * BM);
+                        ++issued;
+                        if (++sa == SA) { sa = 0; pa ^= 1; }
+                    }
                 }
             }
             if (!ok && leader)
@@ -317,28 +335,31 @@ k_tc2_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
             bool ok = true;
             int it = 0;
             for (int64_t tile = pair; tile < ntiles && ok; tile += npairs, ++it) {
-                const int acc = it & 1, aph = (it >> 1) & 1;
+                const int acc = it % NACC, aph = (it / NACC) & 1;
                 if (!(ok = mbar_wait_cl(tempty(acc), aph ^ 1, s_abort))) break;
                 tc::tc_fence_after();
-                const uint32_t d_tmem = tmem_base + acc * BN;
                 for (int step = 0; step < nsteps && ok; ++step) {
                     int sw, pw;
                     wpos(it, step, sw, pw);
-                    if (!(ok = mbar_wait_cl(fullA(sa), pa, s_abort))) break;
                     if (!(ok = mbar_wait_cl(fullW(sw), pw, s_abort))) break;
-                    tc::tc_fence_after();
-                    const uint32_t a_addr = sbase + OFF_A + sa * A_BYTES;
                     const uint32_t w_addr = sbase + OFF_W + sw * W_BYTES;
 #pragma unroll
-                    for (int kk = 0; kk < BK / 16; ++kk) {
-                        const uint64_t adesc = tc::smem_desc_sw128(a_addr + kk * 32, 16, 1024);
-                        const uint64_t bdesc = BWD ? tc::smem_desc_sw128(w_addr + kk * 2048, 8192, 1024)
-                                                   : tc::smem_desc_sw128(w_addr + kk * 32, 16, 1024);
-                        tc2_mma(d_tmem, adesc, bdesc, idesc, (step > 0 || kk > 0) ? 1u : 0u);
+                    for (int u = 0; u < MT && ok; ++u) {          // one W' stage, MT token tiles
+                        if (!(ok = mbar_wait_cl(fullA(sa), pa, s_abort))) break;
+                        tc::tc_fence_after();
+                        const uint32_t a_addr = sbase + OFF_A + sa * A_BYTES;
+                        const uint32_t d_tmem = tmem_base + (acc * MT + u) * BN;
+#pragma unroll
+                        for (int kk = 0; kk < BK / 16; ++kk) {
+                            const uint64_t adesc = tc::smem_desc_sw128(a_addr + kk * 32, 16, 1024);
+                            const uint64_t bdesc = BWD ? tc::smem_desc_sw128(w_addr + kk * 2048, 8192, 1024)
+                                                       : tc::smem_desc_sw128(w_addr + kk * 32, 16, 1024);
+                            tc2_mma(d_tmem, adesc, bdesc, idesc, (step > 0 || kk > 0) ? 1u : 0u);
+                        }
+                        tc2_commit_both(emptyA(sa));
+                        if (++sa == SA) { sa = 0; pa ^= 1; }
                     }
-                    tc2_commit_both(emptyA(sa));
-                    tc2_commit_both(emptyW(sw));
-                    if (++sa == SA) { sa = 0; pa ^= 1; }
+                    if (ok) tc2_commit_both(emptyW(sw));
                 }
                 if (ok) tc2_commit_both(tfull(acc));
             }
@@ -485,15 +506,17 @@ k_tc2_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
         bool ok = true;
         int it = 0;
         for (int64_t tile = pair; tile < ntiles && ok; tile += npairs, ++it) {
-            const int acc = it & 1, aph = (it >> 1) & 1;
-            const int64_t m = (tile % mtiles) * BM + crank * HM + row;
+            const int acc = it % NACC, aph = (it / NACC) & 1;
             const int64_t c0 = (tile / mtiles) * BN;
             if (!(ok = tc::mbar_wait(tfull(acc), aph, s_abort))) break;
             tc::tc_fence_after();
 #pragma unroll 1
-            for (int cc = 0; cc < BN / 32; ++cc) {
+            for (int ucc = 0; ucc < MT * (BN / 32); ++ucc) {
+                const int u = ucc / (BN / 32), cc = ucc % (BN / 32);
+                const int64_t m = (tile % mtiles) * BM * MT + u * BM + crank * HM + row;
                 uint32_t r[32];
-                const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN + cc * 32);
+                const uint32_t taddr =
+                    tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)((acc * MT + u) * BN + cc * 32);
                 TC_LD32(taddr, r);
                 asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
                 if (m < a.M) {
