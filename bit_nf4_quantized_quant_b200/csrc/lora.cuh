@@ -207,6 +207,38 @@ __device__ __forceinline__ float split_sum(const float* p, int64_t stride, int n
     return v;
 }
 
+// The outputs of element (i, j) whose reduced value is v (the stores of the
+// finish, shared with the cluster-reduced adapter kernels).
+__device__ __forceinline__ void finish_store(const FinishArgs& f, int64_t i, int64_t j, float v) {
+    if (f.f32 && j < f.Jf) f.f32[i * f.ld_f32 + j] = v;
+    if (f.hl && j < f.hl_off) {
+        uint16_t hi = 0, lo = 0;
+        if (j < f.J1) {
+            hi = (uint16_t)(pack_bf16x2(v, 0.f) & 0xffffu);
+            lo = (uint16_t)(pack_bf16x2(v - bf16lo_to_f32(hi), 0.f) & 0xffffu);
+        }
+        f.hl[i * f.hl_ld + j] = hi;
+        f.hl[i * f.hl_ld + f.hl_off + j] = lo;
+    }
+    if (f.o1 && j < f.J1pad) f.o1[i * f.s1i + j * f.s1j] = (j < f.J1) ? (uint16_t)(pack_bf16x2(f.alpha1 * v, 0.f) & 0xffffu) : (uint16_t)0;
+    if (f.o2 && j < f.J2pad) {
+        if (f.o2_lo == 0) {
+            f.o2[i * f.s2i + j * f.s2j] = (j < f.J2) ? (uint16_t)(pack_bf16x2(f.alpha2 * v, 0.f) & 0xffffu) : (uint16_t)0;
+        } else if (j < f.o2_lo) {
+            uint16_t hi = 0, lo = 0;
+            if (j < f.J2) {
+                const float sv = f.alpha2 * v;
+                hi = (uint16_t)(pack_bf16x2(sv, 0.f) & 0xffffu);
+                lo = (uint16_t)(pack_bf16x2(sv - bf16lo_to_f32(hi), 0.f) & 0xffffu);
+            }
+            f.o2[i * f.s2i + j * f.s2j] = hi;
+            f.o2[i * f.s2i + (f.o2_lo + j) * f.s2j] = lo;
+        } else if (j >= 2 * f.o2_lo) {
+            f.o2[i * f.s2i + j * f.s2j] = 0;
+        }
+    }
+}
+
 __global__ void __launch_bounds__(256) k_gemm_finish(FinishArgs f) {
     grid_dep_launch();
     grid_dep_wait();
@@ -220,33 +252,7 @@ __global__ void __launch_bounds__(256) k_gemm_finish(FinishArgs f) {
             if (f.col_pair > 0) v = split_sum(f.C + i * f.J + j + f.col_pair, f.I * f.J, f.splits, v);
             v = __fmul_rn(v, f.pre);
         }
-        if (f.f32 && j < f.Jf) f.f32[i * f.ld_f32 + j] = v;
-        if (f.hl && j < f.hl_off) {
-            uint16_t hi = 0, lo = 0;
-            if (j < f.J1) {
-                hi = (uint16_t)(pack_bf16x2(v, 0.f) & 0xffffu);
-                lo = (uint16_t)(pack_bf16x2(v - bf16lo_to_f32(hi), 0.f) & 0xffffu);
-            }
-            f.hl[i * f.hl_ld + j] = hi;
-            f.hl[i * f.hl_ld + f.hl_off + j] = lo;
-        }
-        if (f.o1 && j < f.J1pad) f.o1[i * f.s1i + j * f.s1j] = (j < f.J1) ? (uint16_t)(pack_bf16x2(f.alpha1 * v, 0.f) & 0xffffu) : (uint16_t)0;
-        if (f.o2 && j < f.J2pad) {
-            if (f.o2_lo == 0) {
-                f.o2[i * f.s2i + j * f.s2j] = (j < f.J2) ? (uint16_t)(pack_bf16x2(f.alpha2 * v, 0.f) & 0xffffu) : (uint16_t)0;
-            } else if (j < f.o2_lo) {
-                uint16_t hi = 0, lo = 0;
-                if (j < f.J2) {
-                    const float sv = f.alpha2 * v;
-                    hi = (uint16_t)(pack_bf16x2(sv, 0.f) & 0xffffu);
-                    lo = (uint16_t)(pack_bf16x2(sv - bf16lo_to_f32(hi), 0.f) & 0xffffu);
-                }
-                f.o2[i * f.s2i + j * f.s2j] = hi;
-                f.o2[i * f.s2i + (f.o2_lo + j) * f.s2j] = lo;
-            } else if (j >= 2 * f.o2_lo) {
-                f.o2[i * f.s2i + j * f.s2j] = 0;
-            }
-        }
+        finish_store(f, i, j, v);
     }
 }
 

@@ -21,6 +21,7 @@
 #include "tc2_gemm.cuh"
 #include "merge.cuh"
 #include "adamw8.cuh"
+#include "skinny.cuh"
 
 using namespace qnf4;
 
@@ -555,6 +556,138 @@ int current_pairs() {
     return g_pairs[dev];
 }
 
+// ---------------------------------------------------------------------------
+// Cluster-reduced adapter products (sk::k_rowk / sk::k_colk, padded rank <= 64)
+// ---------------------------------------------------------------------------
+bool g_sk_attr_set[64];
+
+int ensure_sk_attrs() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return QLORA_ERR_DEVICE;
+    std::lock_guard<std::mutex> lk(g_tc_mu);
+    if (!g_sk_attr_set[dev]) {
+        const cudaFuncAttribute at = cudaFuncAttributeMaxDynamicSharedMemorySize;
+        if (cudaFuncSetAttribute(sk::k_rowk<0, 16>, at, sk::Lay<16>::SMEM_ALLOC) != cudaSuccess ||
+            cudaFuncSetAttribute(sk::k_rowk<0, 32>, at, sk::Lay<32>::SMEM_ALLOC) != cudaSuccess ||
+            cudaFuncSetAttribute(sk::k_rowk<0, 64>, at, sk::Lay<64>::SMEM_ALLOC) != cudaSuccess ||
+            cudaFuncSetAttribute(sk::k_rowk<1, 16>, at, sk::Lay<16>::SMEM_ALLOC) != cudaSuccess ||
+            cudaFuncSetAttribute(sk::k_rowk<1, 32>, at, sk::Lay<32>::SMEM_ALLOC) != cudaSuccess ||
+            cudaFuncSetAttribute(sk::k_rowk<1, 64>, at, sk::Lay<64>::SMEM_ALLOC) != cudaSuccess ||
+            cudaFuncSetAttribute(sk::k_colk<16>, at, sk::Lay<16>::SMEM_ALLOC) != cudaSuccess ||
+            cudaFuncSetAttribute(sk::k_colk<32>, at, sk::Lay<32>::SMEM_ALLOC) != cudaSuccess ||
+            cudaFuncSetAttribute(sk::k_colk<64>, at, sk::Lay<64>::SMEM_ALLOC) != cudaSuccess ||
+            cudaFuncSetAttribute(sk::k_colk<128>, at, sk::Lay<128>::SMEM_ALLOC) != cudaSuccess)
+            return QLORA_ERR_LAUNCH;
+        g_sk_attr_set[dev] = true;
+    }
+    return QLORA_OK;
+}
+
+// Padded ranks the cluster-reduced kernels take (larger ones: split-K + finish).
+constexpr int kSkMaxRp = 64;
+
+int sk_jq(int64_t cols) { return cols <= 16 ? 16 : cols <= 32 ? 32 : cols <= 64 ? 64 : 128; }
+
+CUtensorMapSwizzle sk_swizzle(int span) {
+    return span >= 128 ? CU_TENSOR_MAP_SWIZZLE_128B : span == 64 ? CU_TENSOR_MAP_SWIZZLE_64B
+                                                                 : CU_TENSOR_MAP_SWIZZLE_32B;
+}
+
+// Cluster size: at most one wave of CTAs (smem_per_cta decides how many an SM
+// holds, at most 3), and at least 4 reduction tiles per rank.
+int sk_cluster(int64_t tiles, int64_t nred, int smem_per_cta, int sms) {
+    int per_sm = 232448 / smem_per_cta;
+    if (per_sm > 3) per_sm = 3;
+    if (per_sm < 1) per_sm = 1;
+    const int64_t slots = (int64_t)sms * per_sm;
+    int z = sk::kMaxCluster;
+    while (z > 1 && (tiles * z > slots || cdiv(nred, z) < 4)) z >>= 1;
+    return z;
+}
+
+template <typename... KArgs>
+int launch_sk(void (*kern)(KArgs...), int z, int64_t tiles, int smem, cudaStream_t st, const CUtensorMap& tmP,
+              const CUtensorMap& tmQ, const sk::Args& a) {
+    const int64_t ctas = tiles * z;
+    if (ctas > 0x7fffffffLL) return QLORA_ERR_SHAPE;
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3((unsigned)ctas, 1, 1);
+    cfg.blockDim = dim3(sk::kThreads, 1, 1);
+    cfg.dynamicSmemBytes = (size_t)smem;
+    cfg.stream = st;
+    cudaLaunchAttribute at[2];
+    at[0].id = cudaLaunchAttributeClusterDimension;
+    at[0].val.clusterDim.x = (unsigned)z; at[0].val.clusterDim.y = 1; at[0].val.clusterDim.z = 1;
+    at[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    at[1].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = 2;
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, tmP, tmQ, a);
+    note_launch();
+    return e == cudaSuccess ? QLORA_OK : QLORA_ERR_LAUNCH;
+}
+
+// out [M, rp] = P [M, L] . Q with the outputs of f (rows i < M, columns
+// j < f.Jiter; f.J = rp).  qt 0: Q^T = A [qn, L] (A's rows, pitch ldq);
+// qt 1: Q = B [L, qn] (qn columns, pitch ldq).
+int run_rowk(const uint16_t* P, int64_t M, int64_t L, const uint16_t* Q, int qt, int64_t qn, int64_t ldq, int rp,
+             FinishArgs f, int sms, cudaStream_t st) {
+    int rc = ensure_sk_attrs();
+    if (rc != QLORA_OK) return rc;
+    const int jq = sk_jq(rp);
+    CUtensorMap tmP, tmQ;
+    bool ok = make_map_2d(&tmP, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, P, L, M, L * 2, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B);
+    if (qt == 0)
+        ok = ok && make_map_2d(&tmQ, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, Q, L, qn, ldq * 2, 64, jq,
+                               CU_TENSOR_MAP_SWIZZLE_128B);
+    else
+        ok = ok && make_map_2d(&tmQ, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, Q, qn, L, ldq * 2, jq, 64,
+                               sk_swizzle(jq * 2));
+    if (!ok) return QLORA_ERR_LAUNCH;
+    f.J = rp;
+    sk::Args a{};
+    a.M = M; a.L = L; a.nred = cdiv(L, sk::TILE); a.f = f;
+    const int64_t tiles = cdiv(M, sk::TILE);
+    const int smem = jq == 16 ? sk::Lay<16>::SMEM_ALLOC : jq == 32 ? sk::Lay<32>::SMEM_ALLOC : sk::Lay<64>::SMEM_ALLOC;
+    const int z = sk_cluster(tiles, a.nred, smem, sms);
+    a.ns = (int)cdiv(a.nred, z);
+    if (qt == 0) {
+        if (jq == 16) return launch_sk(sk::k_rowk<0, 16>, z, tiles, smem, st, tmP, tmQ, a);
+        if (jq == 32) return launch_sk(sk::k_rowk<0, 32>, z, tiles, smem, st, tmP, tmQ, a);
+        return launch_sk(sk::k_rowk<0, 64>, z, tiles, smem, st, tmP, tmQ, a);
+    }
+    if (jq == 16) return launch_sk(sk::k_rowk<1, 16>, z, tiles, smem, st, tmP, tmQ, a);
+    if (jq == 32) return launch_sk(sk::k_rowk<1, 32>, z, tiles, smem, st, tmP, tmQ, a);
+    return launch_sk(sk::k_rowk<1, 64>, z, tiles, smem, st, tmP, tmQ, a);
+}
+
+// out (l, j) = sum_m P [m, l] Q [m, j] (+ the same at column j + pair) for
+// j < jout, written by finish_store as element (l, j), or (j, l) with trans_out.
+// Q [M, qn] with pitch ldq; qn <= 128.
+int run_colk(const uint16_t* P, int64_t M, int64_t L, const uint16_t* Q, int64_t qn, int64_t ldq, int pair,
+             int jout, bool trans_out, FinishArgs f, int sms, cudaStream_t st) {
+    int rc = ensure_sk_attrs();
+    if (rc != QLORA_OK) return rc;
+    const int jq = sk_jq(qn);
+    const int box = jq > 64 ? 64 : jq;
+    CUtensorMap tmP, tmQ;
+    if (!make_map_2d(&tmP, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, P, L, M, L * 2, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_map_2d(&tmQ, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, Q, qn, M, ldq * 2, box, 64, sk_swizzle(box * 2)))
+        return QLORA_ERR_LAUNCH;
+    sk::Args a{};
+    a.M = M; a.L = L; a.nred = cdiv(M, sk::TILE); a.pair = pair; a.jout = jout; a.trans_out = trans_out ? 1 : 0;
+    a.f = f;
+    const int64_t tiles = cdiv(L, sk::TILE);
+    const int smem = jq == 16 ? sk::Lay<16>::SMEM_ALLOC : jq == 32 ? sk::Lay<32>::SMEM_ALLOC
+                   : jq == 64 ? sk::Lay<64>::SMEM_ALLOC : sk::Lay<128>::SMEM_ALLOC;
+    const int z = sk_cluster(tiles, a.nred, smem, sms);
+    a.ns = (int)cdiv(a.nred, z);
+    if (jq == 16) return launch_sk(sk::k_colk<16>, z, tiles, smem, st, tmP, tmQ, a);
+    if (jq == 32) return launch_sk(sk::k_colk<32>, z, tiles, smem, st, tmP, tmQ, a);
+    if (jq == 64) return launch_sk(sk::k_colk<64>, z, tiles, smem, st, tmP, tmQ, a);
+    return launch_sk(sk::k_colk<128>, z, tiles, smem, st, tmP, tmQ, a);
+}
+
 // Tokens at or below this count take the small-M (GEMV-shaped) kernels.
 constexpr int64_t kSmallMaxM = 32;
 
@@ -573,6 +706,7 @@ int compute_T(const Plan& p, const uint16_t* X, const uint16_t* A, float s, uint
     if (T_out) {   // the caller's bf16 T [M, r]: the same rounding as the hi half of Thl
         f.o1 = T_out; f.s1i = p.r; f.s1j = 1; f.J1pad = p.r; f.alpha1 = 1.f;
     }
+    if (p.rp <= kSkMaxRp) return run_rowk(X, p.M, p.K, A, 0, p.r, p.K, p.rp, f, sms, st);
     return run_gemm<true, true>(X, p.K, A, p.K, p.M, p.rp, p.K, p.M, p.r, p.zT, p.kT,
                                 reinterpret_cast<float*>(ws + p.off_part), f, sms, st);
 }
@@ -1029,7 +1163,8 @@ static int bwd_impl(const qlora_bf16* X, const qlora_bf16* dY, int64_t M, const 
         f.o2 = reinterpret_cast<uint16_t*>(wsb + p.off_sU); f.s2i = p.lw; f.s2j = 1; f.J2 = r; f.J2pad = p.lw;
         f.o2_lo = p.rp;
         f.alpha2 = scaling;
-        rc = run_gemm<true, false>(dY, N, Bop, ldb, M, p.rp, N, M, r, p.zU, p.kU, part, f, sms, st);
+        if (p.rp <= kSkMaxRp) rc = run_rowk(dY, M, N, Bop, 1, ldb, ldb, p.rp, f, sms, st);
+        else rc = run_gemm<true, false>(dY, N, Bop, ldb, M, p.rp, N, M, r, p.zU, p.kU, part, f, sms, st);
         if (rc != QLORA_OK) return rc;
     }
     // dB = s dY^T T  [N, r]   (T as hi | lo columns, summed in the finish, or the caller's T)
@@ -1037,7 +1172,11 @@ static int bwd_impl(const qlora_bf16* X, const qlora_bf16* dY, int64_t M, const 
         FinishArgs f = fin_none();
         f.Iout = N; f.Jiter = r; f.col_pair = t_direct ? 0 : p.rp;
         f.o1 = dB; f.s1i = r; f.s1j = 1; f.J1 = r; f.J1pad = r; f.alpha1 = scaling;
-        if (t_direct)
+        if (p.rp <= kSkMaxRp && t_direct)
+            rc = run_colk(dY, M, N, T, r, r, 0, r, false, f, sms, st);
+        else if (p.rp <= kSkMaxRp)
+            rc = run_colk(dY, M, N, Thl, 2 * p.rp, 2 * p.rp, p.rp, r, false, f, sms, st);
+        else if (t_direct)
             rc = run_gemm<false, false>(dY, N, T, r, N, p.rp, M, N, r, p.zB, p.kB, part, f, sms, st);
         else
             rc = run_gemm<false, false>(dY, N, Thl, 2 * p.rp, N, 2 * p.rp, M, N, 2 * p.rp, p.zB, p.kB, part, f, sms,
@@ -1050,7 +1189,11 @@ static int bwd_impl(const qlora_bf16* X, const qlora_bf16* dY, int64_t M, const 
         f.Iout = r; f.Jiter = K; f.row_pair = p.rp;
         f.o1 = dA; f.s1i = K; f.s1j = 1; f.J1 = K; f.J1pad = K;
         f.alpha1 = dp ? (float)((double)scaling * (double)dp->c) : scaling;
-        rc = run_gemm<false, false>(Uhl, 2 * p.rp, Xl, K, 2 * p.rp, K, M, 2 * p.rp, K, p.zA, p.kA, part, f, sms, st);
+        if (p.rp <= kSkMaxRp)
+            rc = run_colk(Xl, M, K, Uhl, 2 * p.rp, 2 * p.rp, p.rp, r, true, f, sms, st);
+        else
+            rc = run_gemm<false, false>(Uhl, 2 * p.rp, Xl, K, 2 * p.rp, K, M, 2 * p.rp, K, p.zA, p.kA, part, f, sms,
+                                        st);
         if (rc != QLORA_OK) return rc;
     }
     // dX = dY W' + s U A (with dropout: the fused kernel computes dY W' alone, then the
