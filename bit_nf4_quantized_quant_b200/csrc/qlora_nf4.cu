@@ -665,7 +665,7 @@ int run_rowk(const uint16_t* P, int64_t M, int64_t L, const uint16_t* Q, int qt,
 // j < jout, written by finish_store as element (l, j), or (j, l) with trans_out.
 // Q [M, qn] with pitch ldq; qn <= 128.
 int run_colk(const uint16_t* P, int64_t M, int64_t L, const uint16_t* Q, int64_t qn, int64_t ldq, int pair,
-             int jout, bool trans_out, FinishArgs f, int sms, cudaStream_t st) {
+             int jout, bool trans_out, FinishArgs f, int sms, cudaStream_t st, bool wait_end = false) {
     int rc = ensure_sk_attrs();
     if (rc != QLORA_OK) return rc;
     const int jq = sk_jq(qn);
@@ -676,6 +676,7 @@ int run_colk(const uint16_t* P, int64_t M, int64_t L, const uint16_t* Q, int64_t
         return QLORA_ERR_LAUNCH;
     sk::Args a{};
     a.M = M; a.L = L; a.nred = cdiv(M, sk::TILE); a.pair = pair; a.jout = jout; a.trans_out = trans_out ? 1 : 0;
+    a.wait_end = wait_end ? 1 : 0;
     a.f = f;
     const int64_t tiles = cdiv(L, sk::TILE);
     const int smem = jq == 16 ? sk::Lay<16>::SMEM_ALLOC : jq == 32 ? sk::Lay<32>::SMEM_ALLOC
@@ -1167,35 +1168,6 @@ static int bwd_impl(const qlora_bf16* X, const qlora_bf16* dY, int64_t M, const 
         else rc = run_gemm<true, false>(dY, N, Bop, ldb, M, p.rp, N, M, r, p.zU, p.kU, part, f, sms, st);
         if (rc != QLORA_OK) return rc;
     }
-    // dB = s dY^T T  [N, r]   (T as hi | lo columns, summed in the finish, or the caller's T)
-    {
-        FinishArgs f = fin_none();
-        f.Iout = N; f.Jiter = r; f.col_pair = t_direct ? 0 : p.rp;
-        f.o1 = dB; f.s1i = r; f.s1j = 1; f.J1 = r; f.J1pad = r; f.alpha1 = scaling;
-        if (p.rp <= kSkMaxRp && t_direct)
-            rc = run_colk(dY, M, N, T, r, r, 0, r, false, f, sms, st);
-        else if (p.rp <= kSkMaxRp)
-            rc = run_colk(dY, M, N, Thl, 2 * p.rp, 2 * p.rp, p.rp, r, false, f, sms, st);
-        else if (t_direct)
-            rc = run_gemm<false, false>(dY, N, T, r, N, p.rp, M, N, r, p.zB, p.kB, part, f, sms, st);
-        else
-            rc = run_gemm<false, false>(dY, N, Thl, 2 * p.rp, N, 2 * p.rp, M, N, 2 * p.rp, p.zB, p.kB, part, f, sms,
-                                        st);
-        if (rc != QLORA_OK) return rc;
-    }
-    // dA = s U^T X  [r, K]   (U as hi | lo rows, summed in the finish)
-    {
-        FinishArgs f = fin_none();
-        f.Iout = r; f.Jiter = K; f.row_pair = p.rp;
-        f.o1 = dA; f.s1i = K; f.s1j = 1; f.J1 = K; f.J1pad = K;
-        f.alpha1 = dp ? (float)((double)scaling * (double)dp->c) : scaling;
-        if (p.rp <= kSkMaxRp)
-            rc = run_colk(Xl, M, K, Uhl, 2 * p.rp, 2 * p.rp, p.rp, r, true, f, sms, st);
-        else
-            rc = run_gemm<false, false>(Uhl, 2 * p.rp, Xl, K, 2 * p.rp, K, M, 2 * p.rp, K, p.zA, p.kA, part, f, sms,
-                                        st);
-        if (rc != QLORA_OK) return rc;
-    }
     // dX = dY W' + s U A (with dropout: the fused kernel computes dY W' alone, then the
     // masked LoRA term is added in place)
     rc = ensure_tc_attrs();
@@ -1211,6 +1183,42 @@ static int bwd_impl(const qlora_bf16* X, const qlora_bf16* dY, int64_t M, const 
         rc = launch_tc<true>(w, dY, M, sU, p.lw, A, K, r, dX, sms, st, fused_lora);
         path = 2;
     }
+    if (rc != QLORA_OK) return rc;
+    // dB and dA read dY, X, T and U (complete: the fused kernel starts after the
+    // kernel computing U has completed) and nothing the fused kernel writes, so
+    // they run beside it (wait_end) on the SMs it leaves free
+    const bool beside = p.rp <= kSkMaxRp;
+    // dB = s dY^T T  [N, r]   (T as hi | lo columns, summed in the finish, or the caller's T)
+    {
+        FinishArgs f = fin_none();
+        f.Iout = N; f.Jiter = r; f.col_pair = t_direct ? 0 : p.rp;
+        f.o1 = dB; f.s1i = r; f.s1j = 1; f.J1 = r; f.J1pad = r; f.alpha1 = scaling;
+        if (p.rp <= kSkMaxRp && t_direct)
+            rc = run_colk(dY, M, N, T, r, r, 0, r, false, f, sms, st, beside);
+        else if (p.rp <= kSkMaxRp)
+            rc = run_colk(dY, M, N, Thl, 2 * p.rp, 2 * p.rp, p.rp, r, false, f, sms, st, beside);
+        else if (t_direct)
+            rc = run_gemm<false, false>(dY, N, T, r, N, p.rp, M, N, r, p.zB, p.kB, part, f, sms, st);
+        else
+            rc = run_gemm<false, false>(dY, N, Thl, 2 * p.rp, N, 2 * p.rp, M, N, 2 * p.rp, p.zB, p.kB, part, f, sms,
+                                        st);
+        if (rc != QLORA_OK) return rc;
+    }
+    // dA = s U^T X  [r, K]   (U as hi | lo rows, summed in the finish)
+    {
+        FinishArgs f = fin_none();
+        f.Iout = r; f.Jiter = K; f.row_pair = p.rp;
+        f.o1 = dA; f.s1i = K; f.s1j = 1; f.J1 = K; f.J1pad = K;
+        f.alpha1 = dp ? (float)((double)scaling * (double)dp->c) : scaling;
+        if (p.rp <= kSkMaxRp)
+            rc = run_colk(Xl, M, K, Uhl, 2 * p.rp, 2 * p.rp, p.rp, r, true, f, sms, st, beside);
+        else
+            rc = run_gemm<false, false>(Uhl, 2 * p.rp, Xl, K, 2 * p.rp, K, M, 2 * p.rp, K, p.zA, p.kA, part, f, sms,
+                                        st);
+        if (rc != QLORA_OK) return rc;
+    }
+    // with dropout, the masked LoRA term of dX (a plain launch: it starts after dA has
+    // completed, and so after the fused kernel)
     if (rc == QLORA_OK && dp) {
         drop::DxArgs d{};
         d.dX = dX; d.U = reinterpret_cast<const float*>(wsb + p.off_U32); d.ldu = p.rp; d.A = A; d.mask = mask;

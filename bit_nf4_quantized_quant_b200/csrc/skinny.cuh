@@ -23,7 +23,12 @@
 //    go through HBM or a second kernel.
 //  * Programmatic launch: the kernel lets the next one launch at once and
 //    waits for the one before it before the producer's first load and before
-//    any store.
+//    any store -- or, with wait_end, where every input is known complete and
+//    the kernel before it touches neither the inputs nor the outputs (dB and
+//    dA launched behind the fused backward kernel, which starts only after the
+//    kernel computing U has completed), not at all at the start: the kernel
+//    then runs beside the one before it on the SMs that one leaves free, and
+//    one CTA waits for it before exiting, so this grid completes after it.
 //  * Every mbarrier wait is bounded (an expired wait raises the CTA's abort
 //    flag and the device status); every thread still takes both cluster
 //    barriers, so an aborting CTA never strands its cluster.
@@ -63,6 +68,8 @@ struct Args {
     int pair;           // column kernel: column offset of a lo half added to its hi half (0: none)
     int jout;           // column kernel: output columns j < jout
     int trans_out;      // column kernel: element (l, j) is output (j, l) (dA) instead of (l, j) (dB)
+    int wait_end;       // 1: the inputs are complete before launch (see below): no wait before the
+                        // loads; the grid's last CTA waits for the kernel before it before exiting
     FinishArgs f;       // the outputs (f.C, f.splits and the split-sum fields are unused)
 };
 
@@ -127,7 +134,7 @@ __device__ __forceinline__ void run(const CUtensorMap* tmP, const CUtensorMap* t
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     __syncthreads();
-    grid_dep_wait();
+    if (!a.wait_end) grid_dep_wait();
 
     if (warp == kCons) {
         // ---------------------------------------------------------------- producer
@@ -276,6 +283,7 @@ __device__ __forceinline__ void run(const CUtensorMap* tmP, const CUtensorMap* t
         }
     }
     cluster_sync();                       // no CTA leaves while its partial tile may still be read
+    if (a.wait_end && blockIdx.x == gridDim.x - 1 && tid == 0) grid_dep_wait();
 }
 
 template <int QT, int JQ>

@@ -196,6 +196,9 @@ k_tc2_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
     uint32_t* s_tmem = reinterpret_cast<uint32_t*>(base + OFF_MISC);
     volatile int* s_abort = reinterpret_cast<volatile int*>(base + OFF_MISC + 4);
 
+    // kernels launched behind this one with programmatic serialization (the
+    // adapter products dB and dA, which read nothing this kernel writes) may start
+    grid_dep_launch();
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const uint32_t crank = cluster_rank();
     const bool leader = crank == 0;

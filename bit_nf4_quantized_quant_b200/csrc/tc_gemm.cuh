@@ -247,6 +247,9 @@ k_tc_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
     uint32_t* s_tmem = reinterpret_cast<uint32_t*>(base + OFF_MISC);
     volatile int* s_abort = reinterpret_cast<volatile int*>(base + OFF_MISC + 4);
 
+    // kernels launched behind this one with programmatic serialization (the
+    // adapter products dB and dA, which read nothing this kernel writes) may start
+    grid_dep_launch();
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int64_t mtiles = cdiv(a.M, BM), ntiles_n = cdiv(a.n_out, BN);
     const int64_t ntiles = mtiles * ntiles_n;
