@@ -16,11 +16,14 @@
 //  * The reduction is split over the z CTAs of a thread-block cluster (z <= 8,
 //    the reduction tiles dealt out in contiguous runs).  After the loop each
 //    CTA leaves its fp32 partial tile in shared memory; after a cluster
-//    barrier, CTA q sums rows [64 q / z, 64 (q + 1) / z) of the tile over the
+//    barrier, CTA q sums the q-th of z equal runs of the tile's outputs over the
 //    ranks in rank order through distributed shared memory and writes every
 //    output of those elements itself (fp32, bf16, hi + lo pairs, scaled
-//    copies: finish_store).  The result is deterministic and no partial sums
-//    go through HBM or a second kernel.
+//    copies), 8 consecutive elements per thread: two 16-byte loads per rank
+//    and one 16-byte store per output array (dA's partial tile is stored
+//    transposed so that its 8 elements are contiguous too).  One store per
+//    element and array cost more than the rest of the kernel.  The result is
+//    deterministic and no partial sums go through HBM or a second kernel.
 //  * Programmatic launch: the kernel lets the next one launch at once and
 //    waits for the one before it before the producer's first load and before
 //    any store -- or, with wait_end, where every input is known complete and
@@ -52,9 +55,11 @@ template <int JQ>
 struct Lay {
     static constexpr int Q_BYTES = JQ * 128;              // 64 x JQ bf16 (or JQ x 64)
     static constexpr int STAGE = P_BYTES + Q_BYTES;       // a multiple of 1024
-    static constexpr int RED_LD = JQ + 4;                 // fp32 pitch of the partial tile
+    static constexpr int RED_LD = JQ + 4;                 // fp32 pitch of the partial tile [64][JQ]
+    static constexpr int RT_LD = TILE + 4;                // ... stored transposed [JQ][64] (dA)
+    static constexpr int RED_FLOATS = TILE * RED_LD > JQ * RT_LD ? TILE * RED_LD : JQ * RT_LD;
     static constexpr int OFF_RED = kStages * STAGE;
-    static constexpr int OFF_BAR = OFF_RED + TILE * RED_LD * 4;
+    static constexpr int OFF_BAR = OFF_RED + RED_FLOATS * 4;
     static constexpr int SMEM = OFF_BAR + 2 * kStages * 8 + 16;
     static constexpr int SMEM_ALLOC = SMEM + 1024;        // slack for 1024-byte alignment
 };
@@ -212,73 +217,162 @@ __device__ __forceinline__ void run(const CUtensorMap* tmP, const CUtensorMap* t
             __syncwarp();
             if (lane == 0) tc::mbar_arrive(empty(st));
         }
-        // partial tile: rows 16 warp + g (+ 8), columns 8 t + 2 q (+ 1)
+        // partial tile: rows 16 warp + g (+ 8), columns 8 t + 2 q (+ 1); transposed for dA
         const int g = lane >> 2, q = lane & 3;
+        if (COL && a.trans_out) {
 #pragma unroll
-        for (int t = 0; t < JQ / 8; ++t) {
-            float* r0 = red + (16 * warp + g) * LY::RED_LD + 8 * t + 2 * q;
-            *reinterpret_cast<float2*>(r0) = make_float2(acc[t][0], acc[t][1]);
-            *reinterpret_cast<float2*>(r0 + 8 * LY::RED_LD) = make_float2(acc[t][2], acc[t][3]);
+            for (int t = 0; t < JQ / 8; ++t) {
+                float* r0 = red + (8 * t + 2 * q) * LY::RT_LD + 16 * warp + g;
+                r0[0] = acc[t][0];
+                r0[LY::RT_LD] = acc[t][1];
+                r0[8] = acc[t][2];
+                r0[LY::RT_LD + 8] = acc[t][3];
+            }
+        } else {
+#pragma unroll
+            for (int t = 0; t < JQ / 8; ++t) {
+                float* r0 = red + (16 * warp + g) * LY::RED_LD + 8 * t + 2 * q;
+                *reinterpret_cast<float2*>(r0) = make_float2(acc[t][0], acc[t][1]);
+                *reinterpret_cast<float2*>(r0 + 8 * LY::RED_LD) = make_float2(acc[t][2], acc[t][3]);
+            }
         }
     }
     __syncthreads();
     cluster_sync();                       // every partial tile of the cluster is in place
 
     // ---------------------------------------------------------------- reduction + outputs
-    const int r_lo = (int)(TILE * rank / z), r_hi = (int)(TILE * (rank + 1) / z);
+    // Output groups of 8 consecutive elements, dealt out to the ranks in contiguous runs;
+    // a group is 8 partial values of every rank (two 16-byte loads each) summed in rank
+    // order, then 16-byte stores.
     const uint32_t red_s = smem_u32(red);
     const FinishArgs& f = a.f;
+    auto sum8 = [&](uint32_t off, float (&v)[8]) {
+        float4 lo[kMaxCluster], hi[kMaxCluster];
+#pragma unroll
+        for (int p = 0; p < kMaxCluster; ++p)
+            if (p < z) {
+                const uint32_t ad = mapa(off, (uint32_t)p);
+                lo[p] = ld_dsmem_v4(ad);
+                hi[p] = ld_dsmem_v4(ad + 16);
+            }
+#pragma unroll
+        for (int p = 0; p < kMaxCluster; ++p)
+            if (p < z) {
+                v[0] += lo[p].x; v[1] += lo[p].y; v[2] += lo[p].z; v[3] += lo[p].w;
+                v[4] += hi[p].x; v[5] += hi[p].y; v[6] += hi[p].z; v[7] += hi[p].w;
+            }
+    };
     if (!COL) {
-        // rows of the output = tokens t0 + row; columns j < f.Jiter (JQ and beyond read as 0)
-        const int jq4 = (int)(f.Jiter / 4);
-        for (int e = tid; e < (r_hi - r_lo) * jq4; e += kThreads) {
-            const int row = r_lo + e / jq4, j = 4 * (e % jq4);
+        // row i = t0 + row; value groups j0 = 8 gi < rp (f.J), then the zero columns
+        // [2 rp, J2pad) of the s-scaled hi | lo copy
+        const int vg = (int)(f.J / 8);
+        const int zg = f.o2 ? (int)((f.J2pad - 2 * f.o2_lo) / 8) : 0;
+        const int gpr = vg + zg;
+        const int G = TILE * gpr;
+        const int g_lo = (int)((int64_t)G * rank / z), g_hi = (int)((int64_t)G * (rank + 1) / z);
+        const bool o1vec = f.o1 && f.s1i % 8 == 0 && (reinterpret_cast<uintptr_t>(f.o1) & 15) == 0;
+        for (int e = g_lo + tid; e < g_hi; e += kThreads) {
+            const int row = e / gpr, gi = e - row * gpr;
             const int64_t i = t0 + row;
             if (i >= a.M) continue;
-            float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-            if (j < JQ) {
-                const uint32_t off = red_s + (uint32_t)((row * LY::RED_LD + j) * 4);
-                float4 pv[kMaxCluster];
-#pragma unroll
-                for (int p = 0; p < kMaxCluster; ++p)
-                    if (p < z) pv[p] = ld_dsmem_v4(mapa(off, (uint32_t)p));
-#pragma unroll
-                for (int p = 0; p < kMaxCluster; ++p)
-                    if (p < z) { v.x += pv[p].x; v.y += pv[p].y; v.z += pv[p].z; v.w += pv[p].w; }
+            if (gi >= vg) {
+                *reinterpret_cast<uint4*>(f.o2 + i * f.s2i + 2 * f.o2_lo + 8 * (gi - vg)) = make_uint4(0, 0, 0, 0);
+                continue;
             }
-            const float vv[4] = {v.x, v.y, v.z, v.w};
+            const int j0 = 8 * gi;
+            float v[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+            sum8(red_s + (uint32_t)((row * LY::RED_LD + j0) * 4), v);
+#pragma unroll
+            for (int c = 0; c < 8; ++c) v[c] = __fmul_rn(v[c], f.pre);
+            if (f.f32) {
+                float4* d = reinterpret_cast<float4*>(f.f32 + i * f.ld_f32 + j0);
+                d[0] = make_float4(v[0], v[1], v[2], v[3]);
+                d[1] = make_float4(v[4], v[5], v[6], v[7]);
+            }
+            uint32_t h[4], l[4], sh[4], sl[4], b[4];
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
-                const int64_t jj = j + c;
-                finish_store(f, i, jj, jj < f.J ? __fmul_rn(vv[c], f.pre) : 0.f);
+                const bool in0 = j0 + 2 * c < f.J1, in1 = j0 + 2 * c + 1 < f.J1;
+                const float x0 = in0 ? v[2 * c] : 0.f, x1 = in1 ? v[2 * c + 1] : 0.f;
+                h[c] = pack_bf16x2(x0, x1);
+                l[c] = pack_bf16x2(x0 - bf16lo_to_f32(h[c]), x1 - bf16hi_to_f32(h[c]));
+                const float s0 = in0 ? __fmul_rn(f.alpha2, v[2 * c]) : 0.f;
+                const float s1 = in1 ? __fmul_rn(f.alpha2, v[2 * c + 1]) : 0.f;
+                sh[c] = pack_bf16x2(s0, s1);
+                sl[c] = pack_bf16x2(s0 - bf16lo_to_f32(sh[c]), s1 - bf16hi_to_f32(sh[c]));
+                b[c] = pack_bf16x2(in0 ? __fmul_rn(f.alpha1, v[2 * c]) : 0.f, in1 ? __fmul_rn(f.alpha1, v[2 * c + 1]) : 0.f);
+            }
+            if (f.hl) {
+                *reinterpret_cast<uint4*>(f.hl + i * f.hl_ld + j0) = make_uint4(h[0], h[1], h[2], h[3]);
+                *reinterpret_cast<uint4*>(f.hl + i * f.hl_ld + f.hl_off + j0) = make_uint4(l[0], l[1], l[2], l[3]);
+            }
+            if (f.o2) {
+                *reinterpret_cast<uint4*>(f.o2 + i * f.s2i + j0) = make_uint4(sh[0], sh[1], sh[2], sh[3]);
+                *reinterpret_cast<uint4*>(f.o2 + i * f.s2i + f.o2_lo + j0) = make_uint4(sl[0], sl[1], sl[2], sl[3]);
+            }
+            if (f.o1 && j0 < f.J1pad) {
+                if (o1vec && j0 + 8 <= f.J1pad) {
+                    *reinterpret_cast<uint4*>(f.o1 + i * f.s1i + j0) = make_uint4(b[0], b[1], b[2], b[3]);
+                } else {
+#pragma unroll
+                    for (int c = 0; c < 8; ++c)
+                        if (j0 + c < f.J1pad)
+                            f.o1[i * f.s1i + (j0 + c) * f.s1j] =
+                                (uint16_t)((c & 1) ? (b[c >> 1] >> 16) : (b[c >> 1] & 0xffffu));
+                }
             }
         }
     } else {
-        // rows of the tile = columns l = t0 + row of P; output columns j < a.jout
-        const int jo4 = (a.jout + 3) / 4;
-        for (int e = tid; e < (r_hi - r_lo) * jo4; e += kThreads) {
-            const int row = r_lo + e / jo4, j = 4 * (e % jo4);
-            const int64_t l = t0 + row;
-            if (l >= a.L) continue;
-            float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-            for (int h = 0; h < (a.pair > 0 ? 2 : 1); ++h) {
-                const uint32_t off = red_s + (uint32_t)((row * LY::RED_LD + j + h * a.pair) * 4);
-                float4 pv[kMaxCluster];
-#pragma unroll
-                for (int p = 0; p < kMaxCluster; ++p)
-                    if (p < z) pv[p] = ld_dsmem_v4(mapa(off, (uint32_t)p));
-#pragma unroll
-                for (int p = 0; p < kMaxCluster; ++p)
-                    if (p < z) { v.x += pv[p].x; v.y += pv[p].y; v.z += pv[p].z; v.w += pv[p].w; }
+        // out (l, j) = alpha1 * pre * (sum over ranks of the partial at (l, j) [+ at (l, j + pair)]),
+        // stored at o1[l * s1i + j] (dB) or o1[j * s1i + l] (dA, from the transposed tile)
+        const bool tr = a.trans_out != 0;
+        const int jg = (a.jout + 7) / 8;
+        const int G = tr ? a.jout * (TILE / 8) : TILE * jg;
+        const int g_lo = (int)((int64_t)G * rank / z), g_hi = (int)((int64_t)G * (rank + 1) / z);
+        const bool vec = f.s1i % 8 == 0 && (reinterpret_cast<uintptr_t>(f.o1) & 15) == 0;
+        for (int e = g_lo + tid; e < g_hi; e += kThreads) {
+            int j, l_loc;
+            uint32_t off, off2;
+            if (tr) {
+                j = e / (TILE / 8);
+                l_loc = 8 * (e - j * (TILE / 8));
+                off = red_s + (uint32_t)((j * LY::RT_LD + l_loc) * 4);
+                off2 = off + (uint32_t)(a.pair * LY::RT_LD * 4);
+            } else {
+                l_loc = e / jg;
+                j = 8 * (e - l_loc * jg);
+                off = red_s + (uint32_t)((l_loc * LY::RED_LD + j) * 4);
+                off2 = off + (uint32_t)(a.pair * 4);
             }
-            const float vv[4] = {v.x, v.y, v.z, v.w};
+            float v[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+            sum8(off, v);
+            if (a.pair > 0) sum8(off2, v);
+            uint32_t b[4];
 #pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                const int jj = j + c;
-                if (jj >= a.jout) break;
-                const float w = __fmul_rn(vv[c], f.pre);
-                if (a.trans_out) finish_store(f, jj, l, w);
-                else finish_store(f, l, jj, w);
+            for (int c = 0; c < 4; ++c)
+                b[c] = pack_bf16x2(__fmul_rn(f.alpha1, __fmul_rn(v[2 * c], f.pre)),
+                                   __fmul_rn(f.alpha1, __fmul_rn(v[2 * c + 1], f.pre)));
+            if (tr) {
+                const int64_t l0 = t0 + l_loc;
+                uint16_t* d = f.o1 + (int64_t)j * f.s1i + l0;
+                if (vec && l0 + 8 <= a.L) {
+                    *reinterpret_cast<uint4*>(d) = make_uint4(b[0], b[1], b[2], b[3]);
+                } else {
+#pragma unroll
+                    for (int c = 0; c < 8; ++c)
+                        if (l0 + c < a.L) d[c] = (uint16_t)((c & 1) ? (b[c >> 1] >> 16) : (b[c >> 1] & 0xffffu));
+                }
+            } else {
+                const int64_t l = t0 + l_loc;
+                if (l >= a.L) continue;
+                uint16_t* d = f.o1 + l * f.s1i + j;
+                if (vec && j + 8 <= a.jout) {
+                    *reinterpret_cast<uint4*>(d) = make_uint4(b[0], b[1], b[2], b[3]);
+                } else {
+#pragma unroll
+                    for (int c = 0; c < 8; ++c)
+                        if (j + c < a.jout) d[c] = (uint16_t)((c & 1) ? (b[c >> 1] >> 16) : (b[c >> 1] & 0xffffu));
+                }
             }
         }
     }

@@ -167,6 +167,85 @@ def test_inputs_written_just_before_each_call(M):
             assert torch.equal(g, e)
 
 
+@pytest.mark.parametrize("M", [64, 200, 600])
+@pytest.mark.parametrize("given_T", [True, False])
+@pytest.mark.parametrize("dropout", [0.0, 0.1])
+def test_layer_chain_on_one_workspace(M, given_T, dropout):
+    """Two layers' forward, then their backward in reverse order (layer 0's dY is layer 1's dX),
+    on one stream and ONE workspace, with the adapter gradients copied by torch right after the
+    last call: no synchronisation anywhere.  In the backward, dB and dA run beside the fused dX
+    kernel (they skip the wait on it), and every next call's kernels overwrite the workspace that
+    the previous call's kernels read; the results must equal, bit for bit, a run that synchronises
+    after every call -- run eagerly, and replayed as a CUDA graph."""
+    N0, K0, r, s = 768, 1024, 16, 2.0
+    shapes = [(N0, K0), (K0, N0)]                 # layer 1 maps layer 0's output back to K0
+    W = [inputs.weight(70 + i, 0, n, k, 0.02).cuda() for i, (n, k) in enumerate(shapes)]
+    w = [ops.nf4_quantize_dq(Wi) for Wi in W]
+    X0 = inputs.normal(72, (M, K0), 1.0).cuda()
+    A = [inputs.uniform(73 + i, (r, k), 1.0 / np.sqrt(k)).cuda() for i, (n, k) in enumerate(shapes)]
+    B = [inputs.normal(75 + i, (n, r), 0.1).cuda() for i, (n, k) in enumerate(shapes)]
+    dY1 = inputs.normal(77, (M, K0), 1.0).cuda()
+    nbytes = max((ops.qlora_dropout_workspace_bytes if dropout else ops.qlora_workspace_bytes)(M, n, k, r)
+                 for n, k in shapes)
+    ws = torch.empty(nbytes, dtype=torch.uint8, device="cuda")
+    Ts = [torch.empty((M, r), dtype=torch.bfloat16, device="cuda") for _ in range(2)]
+    Ys = [torch.empty((M, n), dtype=torch.bfloat16, device="cuda") for n, k in shapes]
+    dXs = [torch.empty((M, k), dtype=torch.bfloat16, device="cuda") for n, k in shapes]
+    dAs = [torch.empty((r, k), dtype=torch.bfloat16, device="cuda") for n, k in shapes]
+    dBs = [torch.empty((n, r), dtype=torch.bfloat16, device="cuda") for n, k in shapes]
+    copies = [torch.empty_like(t) for t in dAs + dBs]
+
+    def fwd(i, x):
+        if dropout:
+            ops.qlora_linear_fwd_dropout(x, w[i], A[i], B[i], s, dropout, 5, i, Y=Ys[i], T_out=Ts[i], ws=ws)
+        else:
+            ops.qlora_linear_fwd(x, w[i], A[i], B[i], s, Y=Ys[i], T_out=Ts[i], ws=ws)
+
+    def bwd(i, x, dy):
+        T = Ts[i] if given_T else None
+        if dropout:
+            ops.qlora_linear_bwd_dropout(x, dy, w[i], A[i], B[i], s, dropout, 5, i, T=T, dX=dXs[i], dA=dAs[i],
+                                         dB=dBs[i], ws=ws)
+        else:
+            ops.qlora_linear_bwd(x, dy, w[i], A[i], B[i], s, T=T, dX=dXs[i], dA=dAs[i], dB=dBs[i], ws=ws)
+
+    def seq(sync):
+        for i, x in ((0, X0), (1, Ys[0])):
+            fwd(i, x)
+            if sync:
+                torch.cuda.synchronize()
+        for i, x, dy in ((1, Ys[0], dY1), (0, X0, dXs[1])):
+            bwd(i, x, dy)
+            if sync:
+                torch.cuda.synchronize()
+        for c, t in zip(copies, dAs + dBs):
+            c.copy_(t)
+
+    def results():
+        torch.cuda.synchronize()
+        assert ops.qlora_device_status() == 0
+        return [t.cpu() for t in Ys + Ts + dXs + copies]
+
+    seq(True)
+    ref = results()
+    for _ in range(2):
+        for t in Ys + Ts + dXs + dAs + dBs + copies:
+            t.zero_()
+        seq(False)
+        for g, e in zip(results(), ref):
+            assert torch.equal(g, e)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        seq(False)
+    for _ in range(2):
+        for t in Ys + Ts + dXs + dAs + dBs + copies:
+            t.zero_()
+        g.replay()
+        for gt, e in zip(results(), ref):
+            assert torch.equal(gt, e)
+    del g
+
+
 def _sampled_rows_parity(oracle_mod, wl, proj, M, rows_n=16, bwd=True):
     p = wl.projections[proj]
     s = wl.scaling
