@@ -18,7 +18,9 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libqlora_nf4.so")
 
 QLORA_OK = 0
+QLORA_ERR_NULL = -1
 QLORA_ERR_TIMEOUT = -8
+QLORA_ERR_VALUE = -9
 
 _lib = None
 
@@ -70,6 +72,8 @@ def lib():
             "qlora_status_string": (ctypes.c_char_p, [i32]),
             "qlora_device_status": (i32, [i32]),
             "qlora_last_path": (i32, []),
+            "qlora_pair_schedule": (i32, [i64, i64, i32, i32, P, P, P]),
+            "qlora_pair_spans": (i32, [i64, i32, i32, i32, P, i32]),
             "qlora_launch_count": (ctypes.c_longlong, []),
             "qlora_set_kernel_events": (i32, [P, P]),
             "qlora_linear_fwd_noalloc": (i32, [P, i64, WP, P, P, i32, f32, P, P, P]),
@@ -347,3 +351,21 @@ def qlora_linear_fwd_noalloc(X, w: NF4Weight, A, B, scaling: float, Y=None, T_ou
         _ptr(_bits(X)), M, ctypes.byref(st), _ptr(_bits(A)), _ptr(_bits(B)), A.shape[0], float(scaling),
         _ptr(Y), _ptr(T_out), _stream(stream)))
     return Y
+
+
+def pair_schedule(M: int, n_out: int, pairs: int, bwd: bool):
+    """(token tiles per weight stage, tile count, stream-K) of the SM-pair kernel."""
+    mt, nt, sk = ctypes.c_int(0), ctypes.c_int64(0), ctypes.c_int(0)
+    _check("qlora_pair_schedule", lib().qlora_pair_schedule(M, n_out, pairs, int(bwd), ctypes.byref(mt),
+                                                            ctypes.byref(nt), ctypes.byref(sk)))
+    return mt.value, nt.value, bool(sk.value)
+
+
+def pair_spans(ntiles: int, nsteps: int, pair: int, npairs: int):
+    """The stream-K spans [(tile, first step, end step), ...] of one pair, in the order it takes them."""
+    buf = (ctypes.c_int64 * 3 * 64)()
+    n = lib().qlora_pair_spans(ntiles, nsteps, pair, npairs, buf, 64)
+    if n < 0:
+        _check("qlora_pair_spans", n)
+    assert n <= 64
+    return [(buf[i][0], buf[i][1], buf[i][2]) for i in range(n)]

@@ -226,6 +226,8 @@ struct Plan {
     int TKC;                        // small-path forward: K splits of T = X A^T
     // byte offsets
     size_t off_slots, off_Upart, off_part, off_T32, off_U32, off_Tp, off_Ubf, off_sT, off_sU, off_Bp, total;
+    // stream-K SM-pair kernel: partial tiles and per-(tile, CTA, warp) counters
+    size_t off_skpart, sk_part_bytes, off_skflags, sk_flag_bytes;
 };
 
 size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
@@ -251,6 +253,51 @@ int choose_splits(int64_t tiles, int64_t kd, int64_t target) {
     if (z < 1) z = 1;
     return (int)z;
 }
+
+// Token tiles of 256 per SM-pair tile: 2 when a decoded W' stage can feed two
+// of them (halving the decode work per flop) without losing more to wave
+// quantization than that gains.  Measured on the 7B block at M = 2048: a
+// two-tile tile runs 1.2x the flop rate of a one-tile tile, so a wave of them
+// costs about 5/3 of a one-tile wave.
+int tc2_token_tiles(int64_t M, int64_t n_out, int pairs) {
+    const int64_t m1 = cdiv(M, tc2::BM), m2 = cdiv(M, 2 * tc2::BM), nt = cdiv(n_out, tc2::BN);
+    if (m1 < 2 || pairs <= 0) return 1;
+    const int64_t w1 = cdiv(m1 * nt, pairs), w2 = cdiv(m2 * nt, pairs);
+    return 5 * w2 <= 3 * w1 ? 2 : 1;
+}
+
+// SM pairs of a B200; the stream-K workspace is sized for this many.
+constexpr int kSkMaxPairs = 74;
+
+// Padded ranks the cluster-reduced adapter kernels take (larger ones: split-K + finish).
+constexpr int kSkMaxRp = 64;
+
+// Schedule of the SM-pair kernel for an n_out-wide output on `pairs` pairs: token
+// tiles per W' stage (mt) and whether the (tile, step) units are dealt stream-K.
+// Stream-K when whole tiles would leave a partial wave, there are at least half as
+// many tiles as pairs (fewer: more partial-sum traffic than gain), and, in the
+// backward, more tiles than pairs: with fewer, the pairs left free run dB and dA.
+struct Tc2Sched {
+    int mt;
+    bool sk;
+    int64_t ntiles;
+};
+
+Tc2Sched tc2_schedule(int64_t M, int64_t n_out, int pairs, bool bwd) {
+    Tc2Sched sc{};
+    sc.mt = tc2_token_tiles(M, n_out, pairs);
+    sc.ntiles = cdiv(M, (int64_t)tc2::BM * sc.mt) * cdiv(n_out, tc2::BN);
+    sc.sk = pairs > 0 && pairs <= kSkMaxPairs && sc.ntiles % pairs != 0 && 2 * sc.ntiles >= pairs &&
+            (!bwd || sc.ntiles > pairs);
+    return sc;
+}
+
+// Stream-K workspace of one schedule: partial tiles (one slot per pair, 2 CTAs x
+// mt x 128 rows x 256 fp32) and counters (tile x 2 CTAs x 4 epilogue warps).
+size_t sk_part_bytes(const Tc2Sched& sc, int pairs) {
+    return sc.sk ? (size_t)pairs * 2 * sc.mt * tc2::HM * tc2::BN * 4 : 0;
+}
+size_t sk_flag_bytes(const Tc2Sched& sc) { return sc.sk ? (size_t)sc.ntiles * 8 * 4 : 0; }
 
 // CTAs of the small-M tcgen05 kernel: at most one per SM of a B200.
 constexpr int64_t kMaxCtas = 148;
@@ -328,6 +375,15 @@ Plan make_plan(int64_t M, int64_t N, int64_t K, int r, int sms) {
     p.off_sT = take(big * M * p.lw * 2);
     p.off_sU = take(big * M * p.lw * 2);
     p.off_Bp = take(big * N * p.rp * 2);
+    p.sk_part_bytes = p.sk_flag_bytes = 0;
+    if (M > 128) {                      // the SM-pair kernel's path (kPairMinM)
+        for (const Tc2Sched& sc : {tc2_schedule(M, N, kSkMaxPairs, false), tc2_schedule(M, K, kSkMaxPairs, true)}) {
+            if (sk_part_bytes(sc, kSkMaxPairs) > p.sk_part_bytes) p.sk_part_bytes = sk_part_bytes(sc, kSkMaxPairs);
+            if (sk_flag_bytes(sc) > p.sk_flag_bytes) p.sk_flag_bytes = sk_flag_bytes(sc);
+        }
+    }
+    p.off_skpart = take(p.sk_part_bytes);
+    p.off_skflags = take(p.sk_flag_bytes);
     p.total = off;
     return p;
 }
@@ -501,23 +557,12 @@ int launch_tc(const nf4dq_weight* w, const uint16_t* act, int64_t M, const uint1
     return launch_status();
 }
 
-// Token tiles of 256 per SM-pair tile: 2 when a decoded W' stage can feed two
-// of them (halving the decode work per flop) without losing more to wave
-// quantization than that gains.  Measured on the 7B block at M = 2048: a
-// two-tile tile runs 1.2x the flop rate of a one-tile tile, so a wave of them
-// costs about 5/3 of a one-tile wave.
-int tc2_token_tiles(int64_t M, int64_t n_out, int pairs) {
-    const int64_t m1 = cdiv(M, tc2::BM), m2 = cdiv(M, 2 * tc2::BM), nt = cdiv(n_out, tc2::BN);
-    if (m1 < 2 || pairs <= 0) return 1;
-    const int64_t w1 = cdiv(m1 * nt, pairs), w2 = cdiv(m2 * nt, pairs);
-    return 5 * w2 <= 3 * w1 ? 2 : 1;
-}
 
 // The same on SM pairs (cta_group::2), 256 x 256 tiles.
 template <bool BWD>
 int launch_tc2(const nf4dq_weight* w, const uint16_t* act, int64_t M, const uint16_t* lact, int lw,
                const uint16_t* lora_w, int64_t ldl, int r, uint16_t* out, int pairs, cudaStream_t st,
-               bool lora = true) {
+               bool lora, const Plan& p, uint8_t* wsb) {
     const int64_t N = w->N, K = w->K;
     const int64_t n_red = BWD ? N : K, n_out = BWD ? K : N;
     CUtensorMap tmA, tmL, tmP;
@@ -532,9 +577,17 @@ int launch_tc2(const nf4dq_weight* w, const uint16_t* act, int64_t M, const uint
     a.codes = w->codes; a.scale = w->scale; a.mean = w->mean;
     a.lora_w = lora_w; a.ldl = ldl; a.r = r; a.lper = (int)rup(r, 16); a.nlora = lora ? (int)cdiv(lw, 64) : 0;
     a.out = out; a.M = M; a.N = N; a.K = K; a.n_out = n_out; a.n_red = n_red;
-    const int mt = tc2_token_tiles(M, n_out, pairs);
-    const int64_t ntiles = cdiv(M, (int64_t)tc2::BM * mt) * cdiv(n_out, tc2::BN);
-    const int np = (int)(ntiles < pairs ? ntiles : pairs);
+    Tc2Sched sc = tc2_schedule(M, n_out, pairs, BWD);
+    // the counters were zeroed by the kernel before this one (the T or U product), or below
+    if (sc.sk && (sk_part_bytes(sc, pairs) > p.sk_part_bytes || sk_flag_bytes(sc) > p.sk_flag_bytes)) sc.sk = false;
+    a.sk = sc.sk ? 1 : 0;
+    a.part = reinterpret_cast<float*>(wsb + p.off_skpart);
+    a.flags = reinterpret_cast<int*>(wsb + p.off_skflags);
+    if (sc.sk && p.rp > kSkMaxRp &&         // the split-K adapter kernels do not zero the counters
+        cudaMemsetAsync(a.flags, 0, sk_flag_bytes(sc), st) != cudaSuccess)
+        return QLORA_ERR_LAUNCH;
+    const int mt = sc.mt;
+    const int np = sc.sk ? pairs : (int)(sc.ntiles < pairs ? sc.ntiles : pairs);
     hook_before(st);
     if (mt == 2)
         tc2::k_tc2_gemm<BWD, 2><<<2 * np, tc2::kThreads, tc2::Lay<2>::SMEM_ALLOC, st>>>(tmA, tmL, tmP, a,
@@ -583,8 +636,6 @@ int ensure_sk_attrs() {
     return QLORA_OK;
 }
 
-// Padded ranks the cluster-reduced kernels take (larger ones: split-K + finish).
-constexpr int kSkMaxRp = 64;
 
 int sk_jq(int64_t cols) { return cols <= 16 ? 16 : cols <= 32 ? 32 : cols <= 64 ? 64 : 128; }
 
@@ -631,7 +682,7 @@ int launch_sk(void (*kern)(KArgs...), int z, int64_t tiles, int smem, cudaStream
 // j < f.Jiter; f.J = rp).  qt 0: Q^T = A [qn, L] (A's rows, pitch ldq);
 // qt 1: Q = B [L, qn] (qn columns, pitch ldq).
 int run_rowk(const uint16_t* P, int64_t M, int64_t L, const uint16_t* Q, int qt, int64_t qn, int64_t ldq, int rp,
-             FinishArgs f, int sms, cudaStream_t st) {
+             FinishArgs f, int sms, cudaStream_t st, int* zero = nullptr, int64_t nzero = 0) {
     int rc = ensure_sk_attrs();
     if (rc != QLORA_OK) return rc;
     const int jq = sk_jq(rp);
@@ -647,6 +698,7 @@ int run_rowk(const uint16_t* P, int64_t M, int64_t L, const uint16_t* Q, int qt,
     f.J = rp;
     sk::Args a{};
     a.M = M; a.L = L; a.nred = cdiv(L, sk::TILE); a.f = f;
+    a.zero = zero; a.nzero = zero ? nzero : 0;
     const int64_t tiles = cdiv(M, sk::TILE);
     const int smem = jq == 16 ? sk::Lay<16>::SMEM_ALLOC : jq == 32 ? sk::Lay<32>::SMEM_ALLOC : sk::Lay<64>::SMEM_ALLOC;
     const int z = sk_cluster(tiles, a.nred, smem, sms);
@@ -707,7 +759,9 @@ int compute_T(const Plan& p, const uint16_t* X, const uint16_t* A, float s, uint
     if (T_out) {   // the caller's bf16 T [M, r]: the same rounding as the hi half of Thl
         f.o1 = T_out; f.s1i = p.r; f.s1j = 1; f.J1pad = p.r; f.alpha1 = 1.f;
     }
-    if (p.rp <= kSkMaxRp) return run_rowk(X, p.M, p.K, A, 0, p.r, p.K, p.rp, f, sms, st);
+    if (p.rp <= kSkMaxRp)
+        return run_rowk(X, p.M, p.K, A, 0, p.r, p.K, p.rp, f, sms, st, reinterpret_cast<int*>(ws + p.off_skflags),
+                        (int64_t)(p.sk_flag_bytes / 4));
     return run_gemm<true, true>(X, p.K, A, p.K, p.M, p.rp, p.K, p.M, p.r, p.zT, p.kT,
                                 reinterpret_cast<float*>(ws + p.off_part), f, sms, st);
 }
@@ -1085,7 +1139,7 @@ static int fwd_impl(const qlora_bf16* X, int64_t M, const nf4dq_weight* w, const
     const int pairs = current_pairs();
     if (M > kPairMinM && pairs > 0) {
         rc = launch_tc2<false>(w, X, M, reinterpret_cast<const uint16_t*>(wsb + p.off_sT), p.lw, lw, ldl, r, Y,
-                               pairs, st);
+                               pairs, st, true, p, wsb);
         if (rc == QLORA_OK) t_last_path = 3;
         return rc;
     }
@@ -1164,7 +1218,9 @@ static int bwd_impl(const qlora_bf16* X, const qlora_bf16* dY, int64_t M, const 
         f.o2 = reinterpret_cast<uint16_t*>(wsb + p.off_sU); f.s2i = p.lw; f.s2j = 1; f.J2 = r; f.J2pad = p.lw;
         f.o2_lo = p.rp;
         f.alpha2 = scaling;
-        if (p.rp <= kSkMaxRp) rc = run_rowk(dY, M, N, Bop, 1, ldb, ldb, p.rp, f, sms, st);
+        if (p.rp <= kSkMaxRp)
+            rc = run_rowk(dY, M, N, Bop, 1, ldb, ldb, p.rp, f, sms, st, reinterpret_cast<int*>(wsb + p.off_skflags),
+                          (int64_t)(p.sk_flag_bytes / 4));
         else rc = run_gemm<true, false>(dY, N, Bop, ldb, M, p.rp, N, M, r, p.zU, p.kU, part, f, sms, st);
         if (rc != QLORA_OK) return rc;
     }
@@ -1177,7 +1233,7 @@ static int bwd_impl(const qlora_bf16* X, const qlora_bf16* dY, int64_t M, const 
     const uint16_t* sU = reinterpret_cast<const uint16_t*>(wsb + p.off_sU);
     int path;
     if (M > kPairMinM && pairs > 0) {
-        rc = launch_tc2<true>(w, dY, M, sU, p.lw, A, K, r, dX, pairs, st, fused_lora);
+        rc = launch_tc2<true>(w, dY, M, sU, p.lw, A, K, r, dX, pairs, st, fused_lora, p, wsb);
         path = 3;
     } else {
         rc = launch_tc<true>(w, dY, M, sU, p.lw, A, K, r, dX, sms, st, fused_lora);
@@ -1310,6 +1366,34 @@ int qlora_device_status(int reset) {
 }
 
 int qlora_last_path(void) { return t_last_path; }
+
+int qlora_pair_schedule(int64_t M, int64_t n_out, int pairs, int bwd, int* mt, int64_t* ntiles, int* stream_k) {
+    if (!mt || !ntiles || !stream_k) return QLORA_ERR_NULL;
+    if (M <= 0 || n_out <= 0 || pairs <= 0) return QLORA_ERR_VALUE;
+    const Tc2Sched sc = tc2_schedule(M, n_out, pairs, bwd != 0);
+    *mt = sc.mt;
+    *ntiles = sc.ntiles;
+    *stream_k = sc.sk ? 1 : 0;
+    return QLORA_OK;
+}
+
+int qlora_pair_spans(int64_t ntiles, int nsteps, int pair, int npairs, int64_t* out, int max_spans) {
+    if (!out) return QLORA_ERR_NULL;
+    if (ntiles <= 0 || nsteps <= 0 || npairs <= 0 || pair < 0 || pair >= npairs || max_spans < 0)
+        return QLORA_ERR_VALUE;
+    tc2::Spans spn(true, pair, npairs, ntiles, nsteps);
+    int64_t tile;
+    int s0, s1, n = 0;
+    while (spn.next(tile, s0, s1)) {
+        if (n < max_spans) {
+            out[3 * n] = tile;
+            out[3 * n + 1] = s0;
+            out[3 * n + 2] = s1;
+        }
+        ++n;
+    }
+    return n;
+}
 
 long long qlora_launch_count(void) { return g_launches.load(); }
 

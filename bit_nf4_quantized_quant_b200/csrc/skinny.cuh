@@ -75,6 +75,8 @@ struct Args {
     int trans_out;      // column kernel: element (l, j) is output (j, l) (dA) instead of (l, j) (dB)
     int wait_end;       // 1: the inputs are complete before launch (see below): no wait before the
                         // loads; the grid's last CTA waits for the kernel before it before exiting
+    int* zero;          // row kernel: nzero ints set to 0 (the stream-K counters of the fused
+    int64_t nzero;      // kernel launched next, which starts after this one has completed)
     FinishArgs f;       // the outputs (f.C, f.splits and the split-sum fields are unused)
 };
 
@@ -376,6 +378,9 @@ __device__ __forceinline__ void run(const CUtensorMap* tmP, const CUtensorMap* t
             }
         }
     }
+    if (!COL)
+        for (int64_t i = (int64_t)blockIdx.x * kThreads + tid; i < a.nzero; i += (int64_t)gridDim.x * kThreads)
+            a.zero[i] = 0;
     cluster_sync();                       // no CTA leaves while its partial tile may still be read
     if (a.wait_end && blockIdx.x == gridDim.x - 1 && tid == 0) grid_dep_wait();
 }

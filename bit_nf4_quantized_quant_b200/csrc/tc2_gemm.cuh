@@ -74,6 +74,19 @@ struct Lay {
 };
 static_assert(Lay<1>::SMEM_ALLOC <= 232448 && Lay<2>::SMEM_ALLOC <= 232448, "shared memory");
 
+// Stream-K partial tiles: per (pair, CTA rank) MT x 8 chunks of 32 columns, each as
+// 8 pieces of 4 columns x 128 rows x 16 bytes (row-fastest), so that a warp's 32 rows
+// of one piece are 512 contiguous bytes for the contributor's stores and the owner's
+// copies.  The owner streams them through kFixD 4 KB buffers per epilogue warp in the
+// activation and weight rings, idle by then (the span that adds partials is always
+// the pair's last).
+constexpr int kFixD = 8;
+static_assert((BN / 32) % 2 == 0, "epilogue chunk pairs");
+static_assert(4 * kFixD * 4096 <= Lay<1>::OFF_P && 4 * kFixD * 4096 <= Lay<2>::OFF_P, "fix-up staging");
+__host__ __device__ constexpr int64_t part_off(int64_t slot, int nchunks, int ucc, int j, int row) {
+    return (((slot * nchunks + ucc) * 8 + j) * 128 + row) * 4;
+}
+
 __device__ __forceinline__ bool mbar_try_cl(uint32_t bar, uint32_t parity) {
     uint32_t ok;
     asm volatile(
@@ -171,6 +184,50 @@ __device__ __forceinline__ uint32_t p_chunk_offset(int t, int c) {
     return (uint32_t)(n * 64 + (((2 * j + c) ^ ((n >> 1) & 3)) << 4));
 }
 
+// The spans (tile, reduction steps [s0, s1)) a pair takes, in the order it takes them.
+// Round-robin: whole tiles pair, pair + npairs, ...  Stream-K: the pair's run
+// [u0, u1) of the ntiles x nsteps units (tile-major), walked from its END back, so
+// its first span is the head of a tile that a later pair finishes and its last span
+// the tail of a tile it finishes itself.  The pair that takes a tile's last step owns
+// the tile: it adds the partial sums of the lower pairs that took the tile's head,
+// which they computed first, so an owner waits only for lower pairs, and for little.
+struct Spans {
+    int64_t u0, u, nsteps, next_tile, ntiles, npairs;
+    bool sk;
+    __host__ __device__ Spans(bool sk_, int64_t pair, int64_t npairs_, int64_t ntiles_, int nsteps_)
+        : nsteps(nsteps_), next_tile(pair), ntiles(ntiles_), npairs(npairs_), sk(sk_) {
+        const int64_t U = ntiles_ * nsteps_;
+        u0 = pair * U / npairs_;
+        u = (pair + 1) * U / npairs_;
+    }
+    __host__ __device__ bool next(int64_t& tile, int& s0, int& s1) {
+        if (!sk) {
+            if (next_tile >= ntiles) return false;
+            tile = next_tile;
+            s0 = 0;
+            s1 = (int)nsteps;
+            next_tile += npairs;
+            return true;
+        }
+        if (u <= u0) return false;
+        tile = (u - 1) / nsteps;
+        const int64_t tb = tile * nsteps;
+        s1 = (int)(u - tb);
+        s0 = (int)((u0 > tb ? u0 : tb) - tb);
+        u = tb + s0;
+        return true;
+    }
+};
+
+// Steps s in [a, b) with s % 2 == g (a <= b).
+__device__ __forceinline__ int count_par(int a, int b, int g) { return ((b + 1 - g) >> 1) - ((a + 1 - g) >> 1); }
+
+__device__ __forceinline__ int ld_acquire_gpu(const int* p) {
+    int v;
+    asm volatile("ld.acquire.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
 template <bool BWD, int MT>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 k_tc2_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmL,
@@ -235,34 +292,38 @@ k_tc2_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
     tc::tc_fence_after();
     const uint32_t tmem_base = *s_tmem;
 
-    // Ring position of step `step` of this CTA's it-th tile: group g = step % 2 uses
-    // stages g * half .. g * half + half - 1 in its own step order.
-    auto wpos = [&](int it, int step, int& st, int& ph) {
-        const int g = step & 1, per = (nsteps + 1 - g) >> 1, j = it * per + (step >> 1);
+    // Ring position of the j-th step (counted over this CTA's spans so far) of
+    // dequantizer group g = step % 2: the group uses stages g * half .. g * half +
+    // half - 1 in its own step order.
+    auto wpos = [&](int j, int g, int& st, int& ph) {
         st = g * SWH + j % SWH;
         ph = (j / SWH) & 1;
     };
-    auto ppos = [&](int it, int step, int& st, int& ph) {
-        const int g = step & 1, per = (nks + 1 - g) >> 1, j = it * per + (step >> 1);
+    auto ppos = [&](int j, int g, int& st, int& ph) {
         st = g * SPH + j % SPH;
         ph = (j / SPH) & 1;
     };
+    const bool skm = a.sk != 0;
 
     // Peer CTA: pass the completion of each stage of the dequantized-weight ring on to
     // the leader's barrier, for the steps of dequantizer group grp: one cluster-scope
     // fence and one relaxed remote arrive per stage.
     auto forward = [&](int grp) {
         bool ok = true;
-        int it = 0;
-        for (int64_t tile = pair; tile < ntiles && ok; tile += npairs, ++it) {
-            for (int step = grp; step < nsteps && ok; step += 2) {
+        int jw = 0;
+        Spans spn(skm, pair, npairs, ntiles, nsteps);
+        int64_t tile;
+        int s0, s1;
+        while (ok && spn.next(tile, s0, s1)) {
+            for (int step = s0 + ((s0 & 1) != grp ? 1 : 0), k = 0; step < s1 && ok; step += 2, ++k) {
                 int sw, pw;
-                wpos(it, step, sw, pw);
+                wpos(jw + k, grp, sw, pw);
                 if (!(ok = tc::mbar_wait(fullWl(sw), pw, s_abort))) break;
                 asm volatile("fence.acq_rel.cluster;" ::: "memory");
                 asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(mapa(fullW(sw), 0))
                              : "memory");
             }
+            jw += count_par(s0, s1, grp);
         }
     };
 
@@ -271,9 +332,12 @@ k_tc2_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
         if (lane == 0) {
             int sa = 0, pa = 0, issued = 0;
             bool ok = true;
-            for (int64_t tile = pair; tile < ntiles && ok; tile += npairs) {
+            Spans spn(skm, pair, npairs, ntiles, nsteps);
+            int64_t tile;
+            int s0, s1;
+            while (ok && spn.next(tile, s0, s1)) {
                 const int m0 = (int)((tile % mtiles) * BM * MT + crank * HM);
-                for (int step = 0; step < nsteps && ok; ++step) {
+                for (int step = s0; step < s1 && ok; ++step) {
 #pragma unroll
                     for (int u = 0; u < MT && ok; ++u) {          // token tile u of the group
                         if (!(ok = tc::mbar_wait(emptyA(sa), pa ^ 1, s_abort))) break;
@@ -296,17 +360,26 @@ k_tc2_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
 #pragma unroll
             for (int i = 0; i < SP; ++i) last_ph[i] = -1;
             bool ok = true;
-            int it = 0;
-            for (int64_t tile = pair; tile < ntiles && ok; tile += npairs, ++it) {
+            int jp0 = 0, jp1 = 0;
+            Spans spn(skm, pair, npairs, ntiles, nsteps);
+            int64_t tile;
+            int s0, s1;
+            while (ok && spn.next(tile, s0, s1)) {
                 const int c0 = (int)((tile / mtiles) * BN + crank * HN);
-                for (int step = 0; step < nks && ok; ++step) {
+                const int e = s1 < nks ? s1 : nks;
+                for (int step = s0; step < e && ok; ++step) {
+                    const int g = step & 1;
                     int sp, pp;
-                    ppos(it, step, sp, pp);
+                    ppos((g ? jp1 : jp0) + count_par(s0, step, g), g, sp, pp);
                     if (!(ok = tc::mbar_wait(emptyP(sp), pp ^ 1, s_abort))) break;
                     tc::mbar_expect_tx(fullP(sp), P_BYTES);
                     if (!BWD) tc::tma_load_2d(sbase + OFF_P + sp * P_BYTES, &tmP, fullP(sp), step * (BK / 2), c0);
                     else tc::tma_load_2d(sbase + OFF_P + sp * P_BYTES, &tmP, fullP(sp), c0 / 2, step * BK);
                     last_ph[sp] = pp;
+                }
+                if (s0 < e) {
+                    jp0 += count_par(s0, e, 0);
+                    jp1 += count_par(s0, e, 1);
                 }
             }
             if (!ok)                                     // wait for the copies in flight
@@ -319,14 +392,18 @@ k_tc2_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
             constexpr uint32_t idesc = make_idesc2(BWD);
             int sa = 0, pa = 0;
             bool ok = true;
-            int it = 0;
-            for (int64_t tile = pair; tile < ntiles && ok; tile += npairs, ++it) {
+            int it = 0, jw0 = 0, jw1 = 0;
+            Spans spn(skm, pair, npairs, ntiles, nsteps);
+            int64_t tile;
+            int s0, s1;
+            while (ok && spn.next(tile, s0, s1)) {
                 const int acc = it % NACC, aph = (it / NACC) & 1;
                 if (!(ok = mbar_wait_cl(tempty(acc), aph ^ 1, s_abort))) break;
                 tc::tc_fence_after();
-                for (int step = 0; step < nsteps && ok; ++step) {
+                for (int step = s0; step < s1 && ok; ++step) {
+                    const int g = step & 1;
                     int sw, pw;
-                    wpos(it, step, sw, pw);
+                    wpos((g ? jw1 : jw0) + count_par(s0, step, g), g, sw, pw);
                     if (!(ok = mbar_wait_cl(fullW(sw), pw, s_abort))) break;
                     const uint32_t w_addr = sbase + OFF_W + sw * W_BYTES;
 #pragma unroll
@@ -340,7 +417,7 @@ k_tc2_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
                             const uint64_t adesc = tc::smem_desc_sw128(a_addr + kk * 32, 16, 1024);
                             const uint64_t bdesc = BWD ? tc::smem_desc_sw128(w_addr + kk * 2048, 8192, 1024)
                                                        : tc::smem_desc_sw128(w_addr + kk * 32, 16, 1024);
-                            tc2_mma(d_tmem, adesc, bdesc, idesc, (step > 0 || kk > 0) ? 1u : 0u);
+                            tc2_mma(d_tmem, adesc, bdesc, idesc, (step > s0 || kk > 0) ? 1u : 0u);
                         }
                         tc2_commit_both(emptyA(sa));
                         if (++sa == SA) { sa = 0; pa ^= 1; }
@@ -348,6 +425,9 @@ k_tc2_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
                     if (ok) tc2_commit_both(emptyW(sw));
                 }
                 if (ok) tc2_commit_both(tfull(acc));
+                jw0 += count_par(s0, s1, 0);
+                jw1 += count_par(s0, s1, 1);
+                ++it;
             }
             tc2_commit_local(drain);
             mbar_drain_cl(drain, 0);
@@ -376,8 +456,8 @@ k_tc2_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
         // steps are the last fetches of a tile, and the next tile's first fetches write
         // the same slots before anyone waits for these; two copies in flight to one
         // address may land in either order, so none of them may be a copy.
-        auto fetch = [&](int64_t c0, int st, int slot) {
-            if (st >= nks) {
+        auto fetch = [&](int64_t c0, int st, int slot, int lim) {
+            if (st >= lim) {
                 asm volatile("cp.async.commit_group;" ::: "memory");
                 return;
             }
@@ -404,21 +484,26 @@ k_tc2_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
             const int code = (int)(int8_t)(uint8_t)(wd >> (slot ? shift1 : shift0));
             return __fmaf_rn((float)code, sc, mu);
         };
-        int it = 0;
-        for (int64_t tile = pair; tile < ntiles && ok; tile += npairs, ++it) {
+        int jw = 0, jp = 0;
+        Spans spn(skm, pair, npairs, ntiles, nsteps);
+        int64_t tile;
+        int s0, s1;
+        while (ok && spn.next(tile, s0, s1)) {
             const int64_t c0 = (tile / mtiles) * BN + crank * HN;   // this CTA's first output column
-            fetch(c0, grp, 0);
-            fetch(c0, grp + 2, 1);
-            for (int step = grp, k = 0; step < nsteps && ok; step += 2, ++k) {
+            const int lim = s1 < nks ? s1 : nks;                     // dequantization steps of the span end here
+            const int f0 = s0 + ((s0 & 1) != grp ? 1 : 0);           // the group's first step of the span
+            fetch(c0, f0, 0, lim);
+            fetch(c0, f0 + 2, 1, lim);
+            for (int step = f0, k = 0; step < s1 && ok; step += 2, ++k) {
                 int sw, pw;
-                wpos(it, step, sw, pw);
+                wpos(jw + k, grp, sw, pw);
                 const int slot = k & 1;
                 uint32_t o[8][4];
                 int rel = -1;               // packed stage to release once its data is consumed
                 if (step < nks) {
                     const float c = block_const(slot);
                     int sp, pp;
-                    ppos(it, step, sp, pp);
+                    ppos(jp + k, grp, sp, pp);
                     rel = sp;
                     if (!(ok = tc::mbar_wait(fullP(sp), pp, s_abort))) break;
                     uint4 p0, p1;
@@ -481,30 +566,108 @@ k_tc2_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
                     tc::mbar_arrive(leader ? fullW(sw) : fullWl(sw));
                     if (rel >= 0) tc::mbar_arrive(emptyP(rel));
                 }
-                fetch(c0, step + 4, slot);                     // refill: the group's step after next
+                fetch(c0, step + 4, slot, lim);                // refill: the group's step after next
             }
+            jw += count_par(s0, s1, grp);
+            jp += count_par(s0, s0 > lim ? s0 : lim, grp);
         }
         asm volatile("cp.async.wait_all;" ::: "memory");
     } else {
         // ------------------------------------------------------------ epilogue (own 128 tokens)
+        // Stream-K: a span that does not end its tile leaves its fp32 partial sums in this
+        // pair's slot of a.part, then (per warp, after its lanes' stores) counts itself in
+        // a.flags[tile][rank][warp]; the span that ends the tile waits, per warp, for the
+        // counts of the lower pairs pf .. pair - 1 that took the tile's head and adds their
+        // partials to its accumulator in pair order.  No barrier across warps: every wait
+        // is a bounded poll.
         const int q = warp & 3;
         const int row = q * 32 + lane;
         bool ok = true;
         int it = 0;
-        for (int64_t tile = pair; tile < ntiles && ok; tile += npairs, ++it) {
+        const int64_t U = ntiles * (int64_t)nsteps;
+        Spans spn(skm, pair, npairs, ntiles, nsteps);
+        int64_t tile;
+        int s0, s1;
+        while (ok && spn.next(tile, s0, s1)) {
             const int acc = it % NACC, aph = (it / NACC) & 1;
+            ++it;
             const int64_t c0 = (tile / mtiles) * BN;
+            const bool contrib = skm && s1 < nsteps;
+            int64_t pf = pair;                               // first pair whose partials this span adds
+            if (skm && s1 == nsteps && s0 > 0) {
+                const int64_t tb = tile * (int64_t)nsteps;
+                pf = pair - 1;
+                while (pf > 0 && pf * U / npairs > tb) --pf;
+            }
+            int* fq = skm ? a.flags + ((tile * 2 + crank) * 4 + q) : nullptr;
             if (!(ok = tc::mbar_wait(tfull(acc), aph, s_abort))) break;
             tc::tc_fence_after();
-#pragma unroll 1
-            for (int ucc = 0; ucc < MT * (BN / 32); ++ucc) {
+            if (pf < pair) {
+                const int want = (int)(pair - pf);
+                if (ld_acquire_gpu(fq) < want) {
+                    const uint64_t t0 = tc::globaltimer();
+                    while (ld_acquire_gpu(fq) < want) {
+                        if (*s_abort) { ok = false; break; }
+                        if (tc::globaltimer() - t0 > tc::kWaitTimeoutNs) {
+                            *s_abort = 1;
+                            report_timeout();
+                            ok = false;
+                            break;
+                        }
+                    }
+                }
+                ok = __all_sync(0xffffffffu, ok);
+                if (!ok) break;
+            }
+            // owner: item i = (chunk i / nc, lower pair pf + i % nc) of the partials, copied by
+            // each lane for its own row (pieces j = 0..7) into buffer i % kFixD of its warp
+            const int nc = (int)(pair - pf);
+            const int nitems = nc * MT * (BN / 32);
+            const uint32_t fbase = sbase + OFF_A + (uint32_t)(q * kFixD * 4096);
+            auto fix_buf = [&](int i) { return fbase + (uint32_t)((i % kFixD) * 4096); };
+            auto fix_issue = [&](int i) {
+                if (i < nitems) {
+                    const int ucc = i / nc, c = i - ucc * nc;
+                    const float* src = a.part + part_off((pf + c) * 2 + crank, MT * (BN / 32), ucc, 0, row);
+#pragma unroll
+                    for (int j = 0; j < 8; ++j)
+                        asm volatile("cp.async.cg.shared.global [%0], [%1], 16;"
+                                     ::"r"(fix_buf(i) + (uint32_t)((j * 32 + lane) * 16)), "l"(src + j * 128 * 4)
+                                     : "memory");
+                }
+                asm volatile("cp.async.commit_group;" ::: "memory");
+            };
+            int fi = 0;
+            if (nc > 0)
+                for (int i = 0; i < kFixD; ++i) fix_issue(i);
+            // one 32-column chunk of this warp's 32 rows, its accumulator values in r
+            auto emit = [&](int ucc, uint32_t (&r)[32]) {
                 const int u = ucc / (BN / 32), cc = ucc % (BN / 32);
                 const int64_t m = (tile % mtiles) * BM * MT + u * BM + crank * HM + row;
-                uint32_t r[32];
-                const uint32_t taddr =
-                    tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)((acc * MT + u) * BN + cc * 32);
-                TC_LD32(taddr, r);
-                asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+                if (contrib) {
+                    float* dst = a.part + part_off(pair * 2 + crank, MT * (BN / 32), ucc, 0, row);
+#pragma unroll
+                    for (int j = 0; j < 8; ++j)
+                        *reinterpret_cast<float4*>(dst + j * 128 * 4) =
+                            make_float4(__uint_as_float(r[4 * j]), __uint_as_float(r[4 * j + 1]),
+                                        __uint_as_float(r[4 * j + 2]), __uint_as_float(r[4 * j + 3]));
+                    return;
+                }
+                for (int c = 0; c < nc; ++c, ++fi) {
+                    asm volatile("cp.async.wait_group %0;" ::"n"(kFixD - 1) : "memory");
+                    const uint32_t buf = fix_buf(fi);
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) {
+                        uint32_t v0, v1, v2, v3;
+                        asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];"
+                                     : "=r"(v0), "=r"(v1), "=r"(v2), "=r"(v3) : "r"(buf + (uint32_t)((j * 32 + lane) * 16)));
+                        r[4 * j] = __float_as_uint(__uint_as_float(r[4 * j]) + __uint_as_float(v0));
+                        r[4 * j + 1] = __float_as_uint(__uint_as_float(r[4 * j + 1]) + __uint_as_float(v1));
+                        r[4 * j + 2] = __float_as_uint(__uint_as_float(r[4 * j + 2]) + __uint_as_float(v2));
+                        r[4 * j + 3] = __float_as_uint(__uint_as_float(r[4 * j + 3]) + __uint_as_float(v3));
+                    }
+                    fix_issue(fi + kFixD);               // this lane's buffer is read: refill it
+                }
                 if (m < a.M) {
                     uint16_t* dst = a.out + m * a.n_out + c0 + cc * 32;
 #pragma unroll
@@ -519,12 +682,30 @@ k_tc2_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
                         }
                     }
                 }
+            };
+            // two chunks per wait for the tensor-memory loads (one wait per chunk left the
+            // epilogue bound by their latency)
+#pragma unroll 1
+            for (int ucc = 0; ucc < MT * (BN / 32); ucc += 2) {
+                uint32_t r0[32], r1[32];
+                const uint32_t t0 = tmem_base + ((uint32_t)(q * 32) << 16) +
+                                    (uint32_t)((acc * MT + ucc / (BN / 32)) * BN + (ucc % (BN / 32)) * 32);
+                TC_LD32(t0, r0);
+                TC_LD32(t0 + 32, r1);                    // chunk ucc + 1: the next 32 columns (BN / 32 is even)
+                asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+                emit(ucc, r0);
+                emit(ucc + 1, r1);
             }
+            if (nc > 0) asm volatile("cp.async.wait_all;" ::: "memory");
             tc::tc_fence_before();
             __syncwarp();
             if (lane == 0) {
                 if (leader) tc::mbar_arrive(tempty(acc));
                 else mbar_arrive_cl(mapa(tempty(acc), 0));
+                if (contrib) {                   // this warp's partial rows are written: count them
+                    __threadfence();
+                    atomicAdd(fq, 1);
+                }
             }
         }
     }

@@ -78,6 +78,11 @@ struct Args {
     int64_t M, N, K;          // W is [N, K]
     int64_t n_out;            // N (forward) or K (backward)
     int64_t n_red;            // K (forward) or N (backward)
+    // stream-K (SM-pair kernel only): the (tile, reduction step) units are dealt to the
+    // pairs in equal contiguous runs instead of whole tiles round-robin
+    int sk;
+    float* part;              // fp32 partial tiles, one slot per pair: [pairs][2 CTAs][MT x 128 rows][256]
+    int* flags;               // per (tile, CTA rank): partial tiles written so far; zero at launch
 };
 
 // ----------------------------------------------------------------------------

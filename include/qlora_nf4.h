@@ -287,6 +287,20 @@ QLORA_API int qlora_device_status(int reset);
  * (32 < M <= 128), 3 = the same on SM pairs (cta_group::2, M > 128). */
 QLORA_API int qlora_last_path(void);
 
+/* Schedule of the SM-pair kernel (no counterpart on the pages; for tests; no
+ * device work).  qlora_pair_schedule: for M tokens, an n_out-wide output
+ * (N forward, K backward), `pairs` SM pairs and the direction (bwd != 0),
+ * writes the token tiles of 256 per weight stage (*mt), the tile count
+ * (*ntiles) and 1 to *stream_k when the (tile, reduction step) units are dealt
+ * to the pairs stream-K, else 0.  qlora_pair_spans: the spans that pair `pair`
+ * of `npairs` takes of ntiles x nsteps units under stream-K, in the order it
+ * takes them: out[3 i] = tile, out[3 i + 1] = first step, out[3 i + 2] = end
+ * step (exclusive); writes at most max_spans and returns the span count.
+ * Both return QLORA_ERR_VALUE (or QLORA_ERR_NULL) on a bad argument. */
+QLORA_API int qlora_pair_schedule(int64_t M, int64_t n_out, int pairs, int bwd, int* mt, int64_t* ntiles,
+                                  int* stream_k);
+QLORA_API int qlora_pair_spans(int64_t ntiles, int nsteps, int pair, int npairs, int64_t* out, int max_spans);
+
 /* Measurement hooks (no counterpart on the pages; used by benchmarks).
  * qlora_launch_count: number of kernels this library has launched in this
  * process so far (all threads).  qlora_set_kernel_events: the next

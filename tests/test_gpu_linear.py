@@ -167,17 +167,20 @@ def test_inputs_written_just_before_each_call(M):
             assert torch.equal(g, e)
 
 
-@pytest.mark.parametrize("M", [64, 200, 600])
+@pytest.mark.parametrize("M,N0,K0", [(64, 768, 1024), (200, 768, 1024), (600, 768, 1024), (2048, 4096, 4096),
+                                     (2048, 11008, 4096)])
 @pytest.mark.parametrize("given_T", [True, False])
 @pytest.mark.parametrize("dropout", [0.0, 0.1])
-def test_layer_chain_on_one_workspace(M, given_T, dropout):
+def test_layer_chain_on_one_workspace(M, N0, K0, given_T, dropout):
     """Two layers' forward, then their backward in reverse order (layer 0's dY is layer 1's dX),
     on one stream and ONE workspace, with the adapter gradients copied by torch right after the
     last call: no synchronisation anywhere.  In the backward, dB and dA run beside the fused dX
     kernel (they skip the wait on it), and every next call's kernels overwrite the workspace that
     the previous call's kernels read; the results must equal, bit for bit, a run that synchronises
-    after every call -- run eagerly, and replayed as a CUDA graph."""
-    N0, K0, r, s = 768, 1024, 16, 2.0
+    after every call -- run eagerly, and replayed as a CUDA graph.  At 2048 tokens the SM-pair
+    kernel runs stream-K (partial tiles and counters in the workspace) in the forward of both
+    shapes and in the backward of the 11008-wide dX."""
+    r, s = 16, 2.0
     shapes = [(N0, K0), (K0, N0)]                 # layer 1 maps layer 0's output back to K0
     W = [inputs.weight(70 + i, 0, n, k, 0.02).cuda() for i, (n, k) in enumerate(shapes)]
     w = [ops.nf4_quantize_dq(Wi) for Wi in W]
@@ -315,8 +318,9 @@ def test_multi_tile_pair_kernel_repeats_bit_identically(oracle_mod, M, N, K, r):
         _close(inputs.to_f64(got), ref, name)
 
 
-@pytest.mark.parametrize("M,N,K,r,bwd", [(512, 28672, 1024, 16, False),   # SM pairs, 224 tiles
+@pytest.mark.parametrize("M,N,K,r,bwd", [(512, 28672, 1024, 16, False),   # SM pairs, 112 tiles stream-K
                                          (512, 4096, 11008, 64, True),    # SM pairs, backward over 11008
+                                         (1024, 4096, 11008, 16, True),   # SM pairs, backward, 172 tiles stream-K
                                          (100, 38912, 256, 16, False),    # single SM, 152 tiles
                                          (64, 512, 38912, 8, True),       # single SM, backward, 152 tiles
                                          (16, 4096, 28672, 64, True)])    # small-M backward (tcgen05)
