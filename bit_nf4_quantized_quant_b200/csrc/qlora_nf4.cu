@@ -588,16 +588,27 @@ int launch_tc2(const nf4dq_weight* w, const uint16_t* act, int64_t M, const uint
         return QLORA_ERR_LAUNCH;
     const int mt = sc.mt;
     const int np = sc.sk ? pairs : (int)(sc.ntiles < pairs ? sc.ntiles : pairs);
+    // launched with programmatic serialization behind the T or U row kernel (see the
+    // kernel), which lets it start only after its own wait; the split-K adapter kernels
+    // of larger ranks let the next kernel start before theirs, so there it is a plain launch
+    const bool pdl = p.rp <= kSkMaxRp;
     hook_before(st);
-    if (mt == 2)
-        tc2::k_tc2_gemm<BWD, 2><<<2 * np, tc2::kThreads, tc2::Lay<2>::SMEM_ALLOC, st>>>(tmA, tmL, tmP, a,
-                                                                                        tables(w->quant_type));
-    else
-        tc2::k_tc2_gemm<BWD, 1><<<2 * np, tc2::kThreads, tc2::Lay<1>::SMEM_ALLOC, st>>>(tmA, tmL, tmP, a,
-                                                                                        tables(w->quant_type));
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3((unsigned)(2 * np));
+    cfg.blockDim = dim3(tc2::kThreads);
+    cfg.dynamicSmemBytes = mt == 2 ? tc2::Lay<2>::SMEM_ALLOC : tc2::Lay<1>::SMEM_ALLOC;
+    cfg.stream = st;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    at[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = pdl ? 1 : 0;
+    const NF4Tables tb = tables(w->quant_type);
+    const cudaError_t e = mt == 2 ? cudaLaunchKernelEx(&cfg, tc2::k_tc2_gemm<BWD, 2>, tmA, tmL, tmP, a, tb)
+                                  : cudaLaunchKernelEx(&cfg, tc2::k_tc2_gemm<BWD, 1>, tmA, tmL, tmP, a, tb);
     hook_after(st);
     note_launch();
-    return launch_status();
+    return e == cudaSuccess ? QLORA_OK : QLORA_ERR_LAUNCH;
 }
 
 // Tokens above this count use the SM-pair kernel.

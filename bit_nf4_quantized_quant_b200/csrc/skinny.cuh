@@ -24,9 +24,9 @@
 //    transposed so that its 8 elements are contiguous too).  One store per
 //    element and array cost more than the rest of the kernel.  The result is
 //    deterministic and no partial sums go through HBM or a second kernel.
-//  * Programmatic launch: the kernel lets the next one launch at once and
-//    waits for the one before it before the producer's first load and before
-//    any store -- or, with wait_end, where every input is known complete and
+//  * Programmatic launch: the kernel waits for the one before it before the
+//    producer's first load and any store, then lets the next one launch -- or,
+//    with wait_end, where every input is known complete and
 //    the kernel before it touches neither the inputs nor the outputs (dB and
 //    dA launched behind the fused backward kernel, which starts only after the
 //    kernel computing U has completed), not at all at the start: the kernel
@@ -129,7 +129,7 @@ __device__ __forceinline__ void run(const CUtensorMap* tmP, const CUtensorMap* t
     const int64_t s_begin = (int64_t)rank * a.ns;
     const int n = (int)(s_begin >= a.nred ? 0 : (a.nred - s_begin < a.ns ? a.nred - s_begin : a.ns));
 
-    grid_dep_launch();
+    if (a.wait_end) grid_dep_launch();
     if (tid == 0) {
         asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(tmP)) : "memory");
         asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(tmQ)) : "memory");
@@ -141,7 +141,13 @@ __device__ __forceinline__ void run(const CUtensorMap* tmP, const CUtensorMap* t
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     __syncthreads();
-    if (!a.wait_end) grid_dep_wait();
+    if (!a.wait_end) {
+        // the next kernel (the fused one, itself launched programmatically) may start once
+        // everything before this one has completed: it then reads only inputs that are ready,
+        // except this kernel's outputs, for which it waits
+        grid_dep_wait();
+        grid_dep_launch();
+    }
 
     if (warp == kCons) {
         // ---------------------------------------------------------------- producer

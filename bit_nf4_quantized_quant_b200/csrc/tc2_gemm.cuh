@@ -253,10 +253,16 @@ k_tc2_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
     uint32_t* s_tmem = reinterpret_cast<uint32_t*>(base + OFF_MISC);
     volatile int* s_abort = reinterpret_cast<volatile int*>(base + OFF_MISC + 4);
 
-    // kernels launched behind this one with programmatic serialization (the
-    // adapter products dB and dA, which read nothing this kernel writes) may start
-    grid_dep_launch();
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    // Programmatic launch.  This kernel is launched behind the T or U product,
+    // which lets it start once everything before that product has completed: the
+    // activations, the weight and the LoRA weights of the caller are ready, the
+    // product's own outputs (the scaled LoRA activation, the padded LoRA weight,
+    // the zeroed stream-K counters) are not, and every role waits before its
+    // first use of them.  The kernels behind this one (dB and dA, which read U
+    // and nothing this kernel writes) start once every CTA has let them: the
+    // peer CTA at once, the leader's idle warp 15 after waiting for the product.
+    if (cluster_rank() != 0 && tid == 0) grid_dep_launch();
     const uint32_t crank = cluster_rank();
     const bool leader = crank == 0;
     const int64_t pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
@@ -343,8 +349,12 @@ k_tc2_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
                         if (!(ok = tc::mbar_wait(emptyA(sa), pa ^ 1, s_abort))) break;
                         if (leader) tc::mbar_expect_tx(fullA(sa), 2 * A_BYTES);     // both halves land here
                         const uint32_t bar = mapa(fullA(sa), 0);
-                        if (step < nks) tma_load_2d_pair(sbase + OFF_A + sa * A_BYTES, &tmA, bar, step * BK, m0 + u * BM);
-                        else tma_load_2d_pair(sbase + OFF_A + sa * A_BYTES, &tmL, bar, (step - nks) * BK, m0 + u * BM);
+                        if (step < nks) {
+                            tma_load_2d_pair(sbase + OFF_A + sa * A_BYTES, &tmA, bar, step * BK, m0 + u * BM);
+                        } else {
+                            grid_dep_wait();                   // the scaled LoRA activation is complete
+                            tma_load_2d_pair(sbase + OFF_A + sa * A_BYTES, &tmL, bar, (step - nks) * BK, m0 + u * BM);
+                        }
                         ++issued;
                         if (++sa == SA) { sa = 0; pa ^= 1; }
                     }
@@ -436,6 +446,10 @@ k_tc2_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
         }
     } else if (warp == 15) {
         if (!leader && lane == 0) forward(1);
+        if (leader && lane == 0) {
+            grid_dep_wait();
+            grid_dep_launch();
+        }
     } else if (warp < 10) {
         // ------------------------------------------------------------ dequantizers: two groups, alternate steps
         const int grp = (warp - 2) >> 2;               // 0: even steps, 1: odd steps
@@ -516,6 +530,7 @@ k_tc2_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
 #pragma unroll
                     for (int ch = 0; ch < 8; ++ch) decode8(tb, pwd[ch], o[ch]);
                 } else {
+                    grid_dep_wait();                           // the LoRA weight rows (maybe padded) are complete
                     const int lc = step - nks;
                     const uint16_t* src;
                     int64_t col0;
@@ -602,6 +617,7 @@ k_tc2_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
             int* fq = skm ? a.flags + ((tile * 2 + crank) * 4 + q) : nullptr;
             if (!(ok = tc::mbar_wait(tfull(acc), aph, s_abort))) break;
             tc::tc_fence_after();
+            if (skm) grid_dep_wait();                          // the counters are zeroed
             if (pf < pair) {
                 const int want = (int)(pair - pf);
                 if (ld_acquire_gpu(fq) < want) {
