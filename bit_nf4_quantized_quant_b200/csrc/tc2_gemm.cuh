@@ -60,6 +60,7 @@ template <int MT>
 struct Lay {
     static constexpr int SA = MT == 1 ? 5 : 6, SW = 6, SP = MT == 1 ? 8 : 4;
     static constexpr int SWH = SW / 2, SPH = SP / 2;
+    static constexpr int SAS = SA / MT;          // activation stages (MT slots each)
     static constexpr int NACC = 2 / MT;          // accumulator buffers (TMEM holds 2 x 256 columns)
     static constexpr int OFF_A = 0;
     static constexpr int OFF_W = OFF_A + SA * A_BYTES;
@@ -233,7 +234,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 k_tc2_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmL,
            const __grid_constant__ CUtensorMap tmP, Args a, NF4Tables tab) {
     using L = Lay<MT>;
-    constexpr int SA = L::SA, SW = L::SW, SP = L::SP, SWH = L::SWH, SPH = L::SPH, NACC = L::NACC;
+    constexpr int SA = L::SA, SW = L::SW, SP = L::SP, SWH = L::SWH, SPH = L::SPH, NACC = L::NACC, SAS = L::SAS;
+    static_assert(SA % MT == 0, "activation stages");
     constexpr int OFF_A = L::OFF_A, OFF_W = L::OFF_W, OFF_P = L::OFF_P, OFF_BAR = L::OFF_BAR;
     constexpr int OFF_MISC = L::OFF_MISC, OFF_C = L::OFF_C;
     extern __shared__ __align__(1024) uint8_t smem[];
@@ -344,24 +346,25 @@ k_tc2_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
             while (ok && spn.next(tile, s0, s1)) {
                 const int m0 = (int)((tile % mtiles) * BM * MT + crank * HM);
                 for (int step = s0; step < s1 && ok; ++step) {
+                    // one stage = the step's MT token tiles (slots MT sa .. MT sa + MT - 1), one
+                    // barrier pair: the issuing thread tests and commits once per step
+                    if (!(ok = tc::mbar_wait(emptyA(sa), pa ^ 1, s_abort))) break;
+                    if (leader) tc::mbar_expect_tx(fullA(sa), MT * 2 * A_BYTES);    // both halves land here
+                    const uint32_t bar = mapa(fullA(sa), 0);
+                    if (step >= nks) grid_dep_wait();              // the scaled LoRA activation is complete
 #pragma unroll
-                    for (int u = 0; u < MT && ok; ++u) {          // token tile u of the group
-                        if (!(ok = tc::mbar_wait(emptyA(sa), pa ^ 1, s_abort))) break;
-                        if (leader) tc::mbar_expect_tx(fullA(sa), 2 * A_BYTES);     // both halves land here
-                        const uint32_t bar = mapa(fullA(sa), 0);
-                        if (step < nks) {
-                            tma_load_2d_pair(sbase + OFF_A + sa * A_BYTES, &tmA, bar, step * BK, m0 + u * BM);
-                        } else {
-                            grid_dep_wait();                   // the scaled LoRA activation is complete
-                            tma_load_2d_pair(sbase + OFF_A + sa * A_BYTES, &tmL, bar, (step - nks) * BK, m0 + u * BM);
-                        }
-                        ++issued;
-                        if (++sa == SA) { sa = 0; pa ^= 1; }
+                    for (int u = 0; u < MT; ++u) {                 // token tile u of the group
+                        const uint32_t dst = sbase + OFF_A + (sa * MT + u) * A_BYTES;
+                        if (step < nks) tma_load_2d_pair(dst, &tmA, bar, step * BK, m0 + u * BM);
+                        else tma_load_2d_pair(dst, &tmL, bar, (step - nks) * BK, m0 + u * BM);
                     }
+                    ++issued;
+                    if (++sa == SAS) { sa = 0; pa ^= 1; }
                 }
             }
             if (!ok && leader)
-                for (int i = 1; i <= SA && i <= issued; ++i) mbar_drain_cl(fullA((issued - i) % SA), ((issued - i) / SA) & 1);
+                for (int i = 1; i <= SAS && i <= issued; ++i)
+                    mbar_drain_cl(fullA((issued - i) % SAS), ((issued - i) / SAS) & 1);
         }
     } else if (warp == 14) {
         // ------------------------------------------------------------ packed weights (own half)
@@ -416,23 +419,29 @@ k_tc2_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
                     wpos((g ? jw1 : jw0) + count_par(s0, step, g), g, sw, pw);
                     if (!(ok = mbar_wait_cl(fullW(sw), pw, s_abort))) break;
                     const uint32_t w_addr = sbase + OFF_W + sw * W_BYTES;
+                    // descriptors of the stage's k-slices differ only in their start-address
+                    // field (address / 16, 14 bits, no carry for these offsets): one is built,
+                    // the others are it plus a constant (the issuing thread's instructions are
+                    // on the tensor pipe's critical path)
+                    const uint64_t bd0 = BWD ? tc::smem_desc_sw128(w_addr, 8192, 1024)
+                                             : tc::smem_desc_sw128(w_addr, 16, 1024);
+                    if (!(ok = mbar_wait_cl(fullA(sa), pa, s_abort))) break;
+                    tc::tc_fence_after();
 #pragma unroll
-                    for (int u = 0; u < MT && ok; ++u) {          // one W' stage, MT token tiles
-                        if (!(ok = mbar_wait_cl(fullA(sa), pa, s_abort))) break;
-                        tc::tc_fence_after();
-                        const uint32_t a_addr = sbase + OFF_A + sa * A_BYTES;
+                    for (int u = 0; u < MT; ++u) {                 // one W' stage, MT token tiles
+                        const uint32_t a_addr = sbase + OFF_A + (sa * MT + u) * A_BYTES;
                         const uint32_t d_tmem = tmem_base + (acc * MT + u) * BN;
+                        const uint64_t ad0 = tc::smem_desc_sw128(a_addr, 16, 1024);
 #pragma unroll
                         for (int kk = 0; kk < BK / 16; ++kk) {
-                            const uint64_t adesc = tc::smem_desc_sw128(a_addr + kk * 32, 16, 1024);
-                            const uint64_t bdesc = BWD ? tc::smem_desc_sw128(w_addr + kk * 2048, 8192, 1024)
-                                                       : tc::smem_desc_sw128(w_addr + kk * 32, 16, 1024);
+                            const uint64_t adesc = ad0 + (uint64_t)((kk * 32) >> 4);
+                            const uint64_t bdesc = bd0 + (uint64_t)((BWD ? kk * 2048 : kk * 32) >> 4);
                             tc2_mma(d_tmem, adesc, bdesc, idesc, (step > s0 || kk > 0) ? 1u : 0u);
                         }
-                        tc2_commit_both(emptyA(sa));
-                        if (++sa == SA) { sa = 0; pa ^= 1; }
                     }
-                    if (ok) tc2_commit_both(emptyW(sw));
+                    tc2_commit_both(emptyA(sa));
+                    if (++sa == SAS) { sa = 0; pa ^= 1; }
+                    tc2_commit_both(emptyW(sw));
                 }
                 if (ok) tc2_commit_both(tfull(acc));
                 jw0 += count_par(s0, s1, 0);

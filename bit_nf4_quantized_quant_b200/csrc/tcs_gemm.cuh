@@ -17,7 +17,10 @@
 // Warp roles (768 threads, one CTA per SM):
 //   warp 0      TMA producer of the dY tiles (NT x 128 bf16, two
 //               128-byte-swizzled boxes of 64 columns);
-//   warp 1      TMEM allocator and MMA issuer: 8 MMAs of 128 x NT x 16 per unit;
+//   warp 1      TMEM allocator and MMA issuer of decoder group 0's units, warp 3
+//               the issuer of group 1's units: 8 MMAs of 128 x NT x 16 per unit,
+//               each issuer into its own accumulator (two issuers double the
+//               rate: issuing one such MMA costs the issuing thread ~77 cycles);
 //   warp 2      TMA producer of the packed NF4 tiles (128 rows x 64 B, 64-byte
 //               swizzle), 8 units ahead;
 //   warps 4-7   epilogue: TMEM -> registers -> partial slot;
@@ -149,7 +152,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 k_tcs_gemm(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmP, Args a,
            NF4Tables tab) {
     constexpr int X_BYTES = NT * KSTEP * 2;
-    constexpr uint32_t kCols = NT == 16 ? 32 : 64;      // 2 accumulators of NT columns
+    constexpr uint32_t kCols = NT == 16 ? 64 : 128;     // 2 buffers x 2 issuers x NT columns
     extern __shared__ __align__(1024) uint8_t smem[];
     uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem) + 1023) & ~(uintptr_t)1023);
     const uint32_t sbase = smem_u32(base);
@@ -180,8 +183,9 @@ k_tcs_gemm(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUte
         for (int i = 0; i < SX; ++i) { tc::mbar_init(fullX(i), 1); tc::mbar_init(emptyX(i), 1); }
         for (int i = 0; i < SW; ++i) { tc::mbar_init(fullW(i), kGroupThreads / 32); tc::mbar_init(emptyW(i), 1); }
         for (int i = 0; i < SP; ++i) { tc::mbar_init(fullP(i), 1); tc::mbar_init(emptyP(i), kGroupThreads / 32); }
-        for (int i = 0; i < 2; ++i) { tc::mbar_init(tfull(i), 1); tc::mbar_init(tempty(i), kEpiThreads / 32); }
-        tc::mbar_init(drain, 1);
+        // tfull: one commit from each MMA issuer per segment; drain: one from each at the end
+        for (int i = 0; i < 2; ++i) { tc::mbar_init(tfull(i), 2); tc::mbar_init(tempty(i), kEpiThreads / 32); }
+        tc::mbar_init(drain, 2);
         *s_abort = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
@@ -232,12 +236,21 @@ k_tcs_gemm(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUte
                 for (int k = 1; k <= SP && k <= issued; ++k)
                     tc::mbar_drain(fullP((issued - k) & (SP - 1)), ((issued - k) / SP) & 1);
         }
-    } else if (warp == 1) {
-        // ------------------------------------------------------------ MMA issuer
+    } else if (warp == 1 || warp == 3) {
+        // ------------------------------------------------------------ MMA issuers
+        // Issuer iss = 0 (warp 1) takes the units of decoder group 0 (even i), issuer 1
+        // (warp 3) those of group 1, each into its own accumulator (buffer buf, columns
+        // (2 buf + iss) NT): one thread issuing a 128 x NT x 16 MMA spends ~77 cycles on it,
+        // so two issuers double the rate.  Both walk every unit so that they agree on the
+        // segments (a segment = this CTA's units of one tile): each waits for the
+        // segment's buffer to be free and commits the segment's "full" barrier once (the
+        // epilogue waits for both commits and adds the accumulators of the issuers that
+        // had units in the segment).
+        const int iss = warp == 1 ? 0 : 1;
         if (lane == 0) {
             constexpr uint32_t idesc = make_idesc(true, NT);
-            int sx = 0, px = 0, seg = 0, buf = 0;
-            bool ok = true;
+            int seg = 0, buf = 0;
+            bool ok = true, started = false;
             uint32_t d_tmem = tmem_base;
             for (int i = 0, ks = ks0; i < nu && ok; ++i, ks = (ks + 1 == nks) ? 0 : ks + 1) {
                 const bool first = (i == 0) || ks == 0;
@@ -246,30 +259,33 @@ k_tcs_gemm(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUte
                     buf = seg & 1;
                     if (!(ok = tc::mbar_wait(tempty(buf), ((seg >> 1) & 1) ^ 1, s_abort))) break;
                     tc::tc_fence_after();
-                    d_tmem = tmem_base + (uint32_t)(buf * NT);
+                    d_tmem = tmem_base + (uint32_t)((2 * buf + iss) * NT);
+                    started = false;
                 }
-                const int sw = i & (SW - 1), pw = (i / SW) & 1;
-                if (!(ok = tc::mbar_wait(fullX(sx), px, s_abort))) break;
-                if (!(ok = tc::mbar_wait(fullW(sw), pw, s_abort))) break;
-                tc::tc_fence_after();
-                const uint32_t x_addr = sbase + OFF_X + sx * X_BYTES_MAX;
-                const uint32_t w_addr = sbase + OFF_W + sw * W_BYTES;
-                // the 16 descriptors of a unit differ only in their start-address field
-                // (address / 16, 14 bits; every offset keeps it below 2^14): each is the
-                // stage's base descriptor plus a constant (building each in full cost ~200
-                // of the ~1600 cycles the issuing thread spends per unit, measured)
-                const uint64_t a0 = tc::smem_desc_sw128(w_addr, 16384, 1024);
-                const uint64_t b0 = tc::smem_desc_sw128(x_addr, 16, 1024);
+                if ((i & 1) == iss) {
+                    const int sx = i % SX, px = (i / SX) & 1;
+                    const int sw = i & (SW - 1), pw = (i / SW) & 1;
+                    if (!(ok = tc::mbar_wait(fullX(sx), px, s_abort))) break;
+                    if (!(ok = tc::mbar_wait(fullW(sw), pw, s_abort))) break;
+                    tc::tc_fence_after();
+                    const uint32_t x_addr = sbase + OFF_X + sx * X_BYTES_MAX;
+                    const uint32_t w_addr = sbase + OFF_W + sw * W_BYTES;
+                    // the 16 descriptors of a unit differ only in their start-address field
+                    // (address / 16, 14 bits; every offset keeps it below 2^14): each is the
+                    // stage's base descriptor plus a constant
+                    const uint64_t a0 = tc::smem_desc_sw128(w_addr, 16384, 1024);
+                    const uint64_t b0 = tc::smem_desc_sw128(x_addr, 16, 1024);
 #pragma unroll
-                for (int q = 0; q < KSTEP / 16; ++q) {
-                    const int h = q >> 2, kk = q & 3;
-                    const uint64_t adesc = a0 + (uint64_t)((q * 2048) >> 4);
-                    const uint64_t bdesc = b0 + (uint64_t)((h * (NT * 128) + kk * 32) >> 4);
-                    tc::tc_mma(d_tmem, adesc, bdesc, idesc, (!first || q > 0) ? 1u : 0u);
+                    for (int q = 0; q < KSTEP / 16; ++q) {
+                        const int h = q >> 2, kk = q & 3;
+                        const uint64_t adesc = a0 + (uint64_t)((q * 2048) >> 4);
+                        const uint64_t bdesc = b0 + (uint64_t)((h * (NT * 128) + kk * 32) >> 4);
+                        tc::tc_mma(d_tmem, adesc, bdesc, idesc, (started || q > 0) ? 1u : 0u);
+                    }
+                    started = true;
+                    tc::tc_commit(emptyX(sx));
+                    tc::tc_commit(emptyW(sw));
                 }
-                tc::tc_commit(emptyX(sx));
-                tc::tc_commit(emptyW(sw));
-                if (++sx == SX) { sx = 0; px ^= 1; }
                 if (last) {
                     tc::tc_commit(tfull(buf));
                     ++seg;
@@ -352,21 +368,31 @@ k_tcs_gemm(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUte
         int seg = 0;
         for (int u = u0, tile = tile0; u < u1 && ok; ++tile) {
             const int tile_u1 = (tile + 1) * nks;
+            const int seg_u0 = u;
             u = tile_u1 < u1 ? tile_u1 : u1;
             const int buf = seg & 1;
             if (!(ok = tc::mbar_wait(tfull(buf), (seg >> 1) & 1, s_abort))) break;
             ++seg;
             tc::tc_fence_after();
+            // the segment's units are CTA-local indices [seg_i0, seg_i1): issuer 0 took the even
+            // ones, issuer 1 the odd ones; the sum is issuer 0's accumulator plus issuer 1's
+            const int seg_i1 = u - u0, seg_i0 = (seg_u0 - u0);
+            const bool has0 = seg_i1 - seg_i0 >= 2 || (seg_i0 & 1) == 0;
+            const bool has1 = seg_i1 - seg_i0 >= 2 || (seg_i0 & 1) == 1;
             float acc[NT];
-            {
+#pragma unroll
+            for (int m = 0; m < NT; ++m) acc[m] = 0.f;
+#pragma unroll
+            for (int is = 0; is < 2; ++is) {
+                if (is == 0 ? !has0 : !has1) continue;
                 uint32_t rr[16];
-                const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(buf * NT);
+                const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)((2 * buf + is) * NT);
 #pragma unroll
                 for (int h = 0; h < NT / 16; ++h) {
                     TCS_LD16(taddr + h * 16, rr);
                     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 #pragma unroll
-                    for (int j = 0; j < 16; ++j) acc[h * 16 + j] = __uint_as_float(rr[j]);
+                    for (int j = 0; j < 16; ++j) acc[h * 16 + j] += __uint_as_float(rr[j]);
                 }
             }
             tc::tc_fence_before();
