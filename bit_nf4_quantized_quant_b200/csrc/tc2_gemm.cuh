@@ -236,6 +236,11 @@ k_tc2_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
     using L = Lay<MT>;
     constexpr int SA = L::SA, SW = L::SW, SP = L::SP, SWH = L::SWH, SPH = L::SPH, NACC = L::NACC, SAS = L::SAS;
     static_assert(SA % MT == 0, "activation stages");
+    // MMA-issuing threads of the leader, one per token tile of a step (warp 1, and warp 15
+    // for the second).  Each commits its own MMAs, so the barriers that those commits
+    // arrive on (both CTAs' activation and weight stage releases, accumulator full, the
+    // final drain) count NISS arrivals.
+    constexpr int NISS = MT;
     constexpr int OFF_A = L::OFF_A, OFF_W = L::OFF_W, OFF_P = L::OFF_P, OFF_BAR = L::OFF_BAR;
     constexpr int OFF_MISC = L::OFF_MISC, OFF_C = L::OFF_C;
     extern __shared__ __align__(1024) uint8_t smem[];
@@ -263,7 +268,8 @@ k_tc2_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
     // the zeroed stream-K counters) are not, and every role waits before its
     // first use of them.  The kernels behind this one (dB and dA, which read U
     // and nothing this kernel writes) start once every CTA has let them: the
-    // peer CTA at once, the leader's idle warp 15 after waiting for the product.
+    // peer CTA at once, the leader's first epilogue warp (idle until its first
+    // accumulator is full) after waiting for the product.
     if (cluster_rank() != 0 && tid == 0) grid_dep_launch();
     const uint32_t crank = cluster_rank();
     const bool leader = crank == 0;
@@ -275,16 +281,16 @@ k_tc2_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
     const int64_t nblk = a.K / kBlock;
 
     if (tid == 0) {
-        for (int i = 0; i < SA; ++i) { tc::mbar_init(fullA(i), 1); tc::mbar_init(emptyA(i), 1); }
+        for (int i = 0; i < SA; ++i) { tc::mbar_init(fullA(i), 1); tc::mbar_init(emptyA(i), NISS); }
         // leader: its own group's warps + one forwarded arrival from the peer; peer: its group's warps
         for (int i = 0; i < SW; ++i) {
             tc::mbar_init(fullW(i), kGroupWarps + 1);
-            tc::mbar_init(emptyW(i), 1);
+            tc::mbar_init(emptyW(i), NISS);
             tc::mbar_init(fullWl(i), kGroupWarps);
         }
         for (int i = 0; i < SP; ++i) { tc::mbar_init(fullP(i), 1); tc::mbar_init(emptyP(i), kGroupWarps); }
-        for (int i = 0; i < 2; ++i) { tc::mbar_init(tfull(i), 1); tc::mbar_init(tempty(i), 2 * kEpiWarps); }
-        tc::mbar_init(drain, 1);
+        for (int i = 0; i < 2; ++i) { tc::mbar_init(tfull(i), NISS); tc::mbar_init(tempty(i), 2 * kEpiWarps); }
+        tc::mbar_init(drain, NISS);
         *s_abort = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
@@ -333,6 +339,60 @@ k_tc2_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
             }
             jw += count_par(s0, s1, grp);
         }
+    };
+
+    // MMA issuer iss (leader only): token tile u = iss of every step (all of them when
+    // NISS = 1) into its accumulator columns.  Both issuers wait on the same stage
+    // barriers (a wait does not consume a phase) and each commits its own MMAs.
+    auto issue = [&](const int iss) {
+        constexpr uint32_t idesc = make_idesc2(BWD);
+        int sa = 0, pa = 0;
+        bool ok = true;
+        int it = 0, jw0 = 0, jw1 = 0;
+        Spans spn(skm, pair, npairs, ntiles, nsteps);
+        int64_t tile;
+        int s0, s1;
+        while (ok && spn.next(tile, s0, s1)) {
+            const int acc = it % NACC, aph = (it / NACC) & 1;
+            if (!(ok = mbar_wait_cl(tempty(acc), aph ^ 1, s_abort))) break;
+            tc::tc_fence_after();
+            for (int step = s0; step < s1 && ok; ++step) {
+                const int g = step & 1;
+                int sw, pw;
+                wpos((g ? jw1 : jw0) + count_par(s0, step, g), g, sw, pw);
+                if (!(ok = mbar_wait_cl(fullW(sw), pw, s_abort))) break;
+                const uint32_t w_addr = sbase + OFF_W + sw * W_BYTES;
+                // descriptors of the stage's k-slices differ only in their start-address
+                // field (address / 16, 14 bits, no carry for these offsets): one is built,
+                // the others are it plus a constant (the issuing thread's instructions are
+                // on the tensor pipe's critical path)
+                const uint64_t bd0 = BWD ? tc::smem_desc_sw128(w_addr, 8192, 1024)
+                                         : tc::smem_desc_sw128(w_addr, 16, 1024);
+                if (!(ok = mbar_wait_cl(fullA(sa), pa, s_abort))) break;
+                tc::tc_fence_after();
+#pragma unroll
+                for (int u = iss; u < MT; u += NISS) {         // one W' stage, this thread's token tiles
+                    const uint32_t a_addr = sbase + OFF_A + (sa * MT + u) * A_BYTES;
+                    const uint32_t d_tmem = tmem_base + (acc * MT + u) * BN;
+                    const uint64_t ad0 = tc::smem_desc_sw128(a_addr, 16, 1024);
+#pragma unroll
+                    for (int kk = 0; kk < BK / 16; ++kk) {
+                        const uint64_t adesc = ad0 + (uint64_t)((kk * 32) >> 4);
+                        const uint64_t bdesc = bd0 + (uint64_t)((BWD ? kk * 2048 : kk * 32) >> 4);
+                        tc2_mma(d_tmem, adesc, bdesc, idesc, (step > s0 || kk > 0) ? 1u : 0u);
+                    }
+                }
+                tc2_commit_both(emptyA(sa));
+                if (++sa == SAS) { sa = 0; pa ^= 1; }
+                tc2_commit_both(emptyW(sw));
+            }
+            if (ok) tc2_commit_both(tfull(acc));
+            jw0 += count_par(s0, s1, 0);
+            jw1 += count_par(s0, s1, 1);
+            ++it;
+        }
+        tc2_commit_local(drain);
+        mbar_drain_cl(drain, 0);
     };
 
     if (warp == 0) {
@@ -400,65 +460,13 @@ k_tc2_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
                     if (last_ph[i] >= 0) tc::mbar_drain(fullP(i), last_ph[i]);
         }
     } else if (warp == 1) {
-        // ------------------------------------------------------------ MMA issuer (leader only)
-        if (leader && lane == 0) {
-            constexpr uint32_t idesc = make_idesc2(BWD);
-            int sa = 0, pa = 0;
-            bool ok = true;
-            int it = 0, jw0 = 0, jw1 = 0;
-            Spans spn(skm, pair, npairs, ntiles, nsteps);
-            int64_t tile;
-            int s0, s1;
-            while (ok && spn.next(tile, s0, s1)) {
-                const int acc = it % NACC, aph = (it / NACC) & 1;
-                if (!(ok = mbar_wait_cl(tempty(acc), aph ^ 1, s_abort))) break;
-                tc::tc_fence_after();
-                for (int step = s0; step < s1 && ok; ++step) {
-                    const int g = step & 1;
-                    int sw, pw;
-                    wpos((g ? jw1 : jw0) + count_par(s0, step, g), g, sw, pw);
-                    if (!(ok = mbar_wait_cl(fullW(sw), pw, s_abort))) break;
-                    const uint32_t w_addr = sbase + OFF_W + sw * W_BYTES;
-                    // descriptors of the stage's k-slices differ only in their start-address
-                    // field (address / 16, 14 bits, no carry for these offsets): one is built,
-                    // the others are it plus a constant (the issuing thread's instructions are
-                    // on the tensor pipe's critical path)
-                    const uint64_t bd0 = BWD ? tc::smem_desc_sw128(w_addr, 8192, 1024)
-                                             : tc::smem_desc_sw128(w_addr, 16, 1024);
-                    if (!(ok = mbar_wait_cl(fullA(sa), pa, s_abort))) break;
-                    tc::tc_fence_after();
-#pragma unroll
-                    for (int u = 0; u < MT; ++u) {                 // one W' stage, MT token tiles
-                        const uint32_t a_addr = sbase + OFF_A + (sa * MT + u) * A_BYTES;
-                        const uint32_t d_tmem = tmem_base + (acc * MT + u) * BN;
-                        const uint64_t ad0 = tc::smem_desc_sw128(a_addr, 16, 1024);
-#pragma unroll
-                        for (int kk = 0; kk < BK / 16; ++kk) {
-                            const uint64_t adesc = ad0 + (uint64_t)((kk * 32) >> 4);
-                            const uint64_t bdesc = bd0 + (uint64_t)((BWD ? kk * 2048 : kk * 32) >> 4);
-                            tc2_mma(d_tmem, adesc, bdesc, idesc, (step > s0 || kk > 0) ? 1u : 0u);
-                        }
-                    }
-                    tc2_commit_both(emptyA(sa));
-                    if (++sa == SAS) { sa = 0; pa ^= 1; }
-                    tc2_commit_both(emptyW(sw));
-                }
-                if (ok) tc2_commit_both(tfull(acc));
-                jw0 += count_par(s0, s1, 0);
-                jw1 += count_par(s0, s1, 1);
-                ++it;
-            }
-            tc2_commit_local(drain);
-            mbar_drain_cl(drain, 0);
-        } else if (!leader && lane == 0) {
-            forward(0);
-        }
+        // ------------------------------------------------------------ MMA issuer 0 (leader)
+        if (leader && lane == 0) issue(0);
+        else if (!leader && lane == 0) forward(0);
     } else if (warp == 15) {
+        // ------------------------------------------------------------ MMA issuer 1 (leader)
         if (!leader && lane == 0) forward(1);
-        if (leader && lane == 0) {
-            grid_dep_wait();
-            grid_dep_launch();
-        }
+        if (NISS > 1 && leader && lane == 0) issue(1);
     } else if (warp < 10) {
         // ------------------------------------------------------------ dequantizers: two groups, alternate steps
         const int grp = (warp - 2) >> 2;               // 0: even steps, 1: odd steps
@@ -606,6 +614,13 @@ k_tc2_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
         // is a bounded poll.
         const int q = warp & 3;
         const int row = q * 32 + lane;
+        if (leader && warp == 10) {
+            if (lane == 0) {
+                grid_dep_wait();
+                grid_dep_launch();
+            }
+            __syncwarp();
+        }
         bool ok = true;
         int it = 0;
         const int64_t U = ntiles * (int64_t)nsteps;
