@@ -46,22 +46,28 @@ constexpr int kGroupWarps = kGroupThreads / 32;
 constexpr int kEpiWarps = 4;
 constexpr int kTmemCols = 512;
 
-// Shared-memory layout for MT token tiles of 256 per pair tile.  MT = 1: one
-// accumulator per tile, two in TMEM so the epilogue of a tile overlaps the next
-// tile's main loop.  MT = 2: each decoded W' stage feeds the MMAs of two token
-// tiles (two accumulators, all of TMEM), which halves the decode work per
-// flop; the epilogue then drains both before the next tile starts.
-//   SA: activation slots (one token tile's 128 x 64 half each; a step takes MT)
+// Shared-memory layout for MT token tiles of 256 per pair tile.  Two threads of
+// the leader issue the MMAs (one thread spends ~77 cycles issuing one, about as
+// long as a 256 x 256 x 16 MMA takes the pair's tensor cores to run, so one
+// thread cannot keep them busy).  MT = 2: each decoded W' stage feeds the MMAs of
+// two token tiles, one per issuer (two accumulators, all of TMEM), which halves
+// the decode work per flop.  MT = 1: issuer g takes the steps of parity g into its
+// own accumulator (all of TMEM again) and the epilogue adds the two.  Either way
+// the epilogue drains TMEM before the next tile starts.
+//   SA: activation slots (one token tile's 128 x 64 half each; a step takes MT);
+//   MT = 1 splits them into one sub-ring per step parity, so that each stage is
+//   only ever waited on by the issuer of that parity
 //   SW / SP: W' and packed stages, split into one sub-ring per dequantizer
 //   group (SW / 2 and SP / 2 stages), each filled and drained in that group's
 //   step order, so every waiter is at most one phase ahead of the barrier it
 //   waits on (a parity wait cannot tell phase k from phase k - 2).
 template <int MT>
 struct Lay {
-    static constexpr int SA = MT == 1 ? 5 : 6, SW = 6, SP = MT == 1 ? 8 : 4;
+    static constexpr int SA = MT == 1 ? 4 : 6, SW = 6, SP = MT == 1 ? 8 : 4;
     static constexpr int SWH = SW / 2, SPH = SP / 2;
     static constexpr int SAS = SA / MT;          // activation stages (MT slots each)
-    static constexpr int NACC = 2 / MT;          // accumulator buffers (TMEM holds 2 x 256 columns)
+    static constexpr int SAH = SA / 2;           // MT = 1: stages per step-parity sub-ring
+    static constexpr int NACC = 1;               // accumulator sets (TMEM holds 2 x 256 columns)
     static constexpr int OFF_A = 0;
     static constexpr int OFF_W = OFF_A + SA * A_BYTES;
     static constexpr int OFF_P = OFF_W + SW * W_BYTES;
@@ -235,12 +241,13 @@ k_tc2_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
            const __grid_constant__ CUtensorMap tmP, Args a, NF4Tables tab) {
     using L = Lay<MT>;
     constexpr int SA = L::SA, SW = L::SW, SP = L::SP, SWH = L::SWH, SPH = L::SPH, NACC = L::NACC, SAS = L::SAS;
-    static_assert(SA % MT == 0, "activation stages");
-    // MMA-issuing threads of the leader, one per token tile of a step (warp 1, and warp 15
-    // for the second).  Each commits its own MMAs, so the barriers that those commits
-    // arrive on (both CTAs' activation and weight stage releases, accumulator full, the
-    // final drain) count NISS arrivals.
-    constexpr int NISS = MT;
+    constexpr int SAH = L::SAH;
+    static_assert(SA % MT == 0 && SA % 2 == 0, "activation stages");
+    // MMA-issuing threads of the leader: warp 1 (issuer 0) and warp 15 (issuer 1).  Each
+    // commits its own MMAs.  MT = 2: both read every stage, so the stage releases count
+    // two arrivals; MT = 1: a stage is read by one issuer (NREL = 1).  Accumulator full
+    // and the final drain count one arrival per issuer.
+    constexpr int NISS = 2, NREL = MT;
     constexpr int OFF_A = L::OFF_A, OFF_W = L::OFF_W, OFF_P = L::OFF_P, OFF_BAR = L::OFF_BAR;
     constexpr int OFF_MISC = L::OFF_MISC, OFF_C = L::OFF_C;
     extern __shared__ __align__(1024) uint8_t smem[];
@@ -281,11 +288,11 @@ k_tc2_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
     const int64_t nblk = a.K / kBlock;
 
     if (tid == 0) {
-        for (int i = 0; i < SA; ++i) { tc::mbar_init(fullA(i), 1); tc::mbar_init(emptyA(i), NISS); }
+        for (int i = 0; i < SA; ++i) { tc::mbar_init(fullA(i), 1); tc::mbar_init(emptyA(i), NREL); }
         // leader: its own group's warps + one forwarded arrival from the peer; peer: its group's warps
         for (int i = 0; i < SW; ++i) {
             tc::mbar_init(fullW(i), kGroupWarps + 1);
-            tc::mbar_init(emptyW(i), NISS);
+            tc::mbar_init(emptyW(i), NREL);
             tc::mbar_init(fullWl(i), kGroupWarps);
         }
         for (int i = 0; i < SP; ++i) { tc::mbar_init(fullP(i), 1); tc::mbar_init(emptyP(i), kGroupWarps); }
@@ -317,6 +324,17 @@ k_tc2_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
         st = g * SPH + j % SPH;
         ph = (j / SPH) & 1;
     };
+    // Activation stage of a step: MT = 2, one ring in step order (jall = this CTA's steps
+    // so far); MT = 1, the sub-ring of the step's parity g (jg = its steps of parity g).
+    auto apos = [&](int jall, int jg, int g, int& st, int& ph) {
+        if (MT == 2) {
+            st = jall % SAS;
+            ph = (jall / SAS) & 1;
+        } else {
+            st = g * SAH + jg % SAH;
+            ph = (jg / SAH) & 1;
+        }
+    };
     const bool skm = a.sk != 0;
 
     // Peer CTA: pass the completion of each stage of the dequantized-weight ring on to
@@ -341,14 +359,15 @@ k_tc2_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
         }
     };
 
-    // MMA issuer iss (leader only): token tile u = iss of every step (all of them when
-    // NISS = 1) into its accumulator columns.  Both issuers wait on the same stage
-    // barriers (a wait does not consume a phase) and each commits its own MMAs.
+    // MMA issuer iss (leader only).  MT = 2: token tile u = iss of every step into its
+    // accumulator columns; both issuers wait on the same stage barriers (a wait does not
+    // consume a phase).  MT = 1: the steps of parity iss into accumulator iss.
     auto issue = [&](const int iss) {
         constexpr uint32_t idesc = make_idesc2(BWD);
-        int sa = 0, pa = 0;
+        constexpr int sstep = MT == 2 ? 1 : 2;
+        const int u = MT == 2 ? iss : 0;
         bool ok = true;
-        int it = 0, jw0 = 0, jw1 = 0;
+        int it = 0, jw0 = 0, jw1 = 0, ja = 0;
         Spans spn(skm, pair, npairs, ntiles, nsteps);
         int64_t tile;
         int s0, s1;
@@ -356,10 +375,13 @@ k_tc2_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
             const int acc = it % NACC, aph = (it / NACC) & 1;
             if (!(ok = mbar_wait_cl(tempty(acc), aph ^ 1, s_abort))) break;
             tc::tc_fence_after();
-            for (int step = s0; step < s1 && ok; ++step) {
+            const uint32_t d_tmem = tmem_base + (uint32_t)(iss * BN);
+            const int first = (MT == 1 && (s0 & 1) != iss) ? s0 + 1 : s0;
+            for (int step = first; step < s1 && ok; step += sstep) {
                 const int g = step & 1;
-                int sw, pw;
+                int sw, pw, sa, pa;
                 wpos((g ? jw1 : jw0) + count_par(s0, step, g), g, sw, pw);
+                apos(ja + (step - s0), (g ? jw1 : jw0) + count_par(s0, step, g), g, sa, pa);
                 if (!(ok = mbar_wait_cl(fullW(sw), pw, s_abort))) break;
                 const uint32_t w_addr = sbase + OFF_W + sw * W_BYTES;
                 // descriptors of the stage's k-slices differ only in their start-address
@@ -370,25 +392,24 @@ k_tc2_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
                                          : tc::smem_desc_sw128(w_addr, 16, 1024);
                 if (!(ok = mbar_wait_cl(fullA(sa), pa, s_abort))) break;
                 tc::tc_fence_after();
+                const uint32_t a_addr = sbase + OFF_A + (sa * MT + u) * A_BYTES;
+                const uint64_t ad0 = tc::smem_desc_sw128(a_addr, 16, 1024);
 #pragma unroll
-                for (int u = iss; u < MT; u += NISS) {         // one W' stage, this thread's token tiles
-                    const uint32_t a_addr = sbase + OFF_A + (sa * MT + u) * A_BYTES;
-                    const uint32_t d_tmem = tmem_base + (acc * MT + u) * BN;
-                    const uint64_t ad0 = tc::smem_desc_sw128(a_addr, 16, 1024);
-#pragma unroll
-                    for (int kk = 0; kk < BK / 16; ++kk) {
-                        const uint64_t adesc = ad0 + (uint64_t)((kk * 32) >> 4);
-                        const uint64_t bdesc = bd0 + (uint64_t)((BWD ? kk * 2048 : kk * 32) >> 4);
-                        tc2_mma(d_tmem, adesc, bdesc, idesc, (step > s0 || kk > 0) ? 1u : 0u);
-                    }
+                for (int kk = 0; kk < BK / 16; ++kk) {
+                    const uint64_t adesc = ad0 + (uint64_t)((kk * 32) >> 4);
+                    const uint64_t bdesc = bd0 + (uint64_t)((BWD ? kk * 2048 : kk * 32) >> 4);
+                    tc2_mma(d_tmem, adesc, bdesc, idesc, (step > first || kk > 0) ? 1u : 0u);
                 }
                 tc2_commit_both(emptyA(sa));
-                if (++sa == SAS) { sa = 0; pa ^= 1; }
                 tc2_commit_both(emptyW(sw));
             }
+            // both issuers commit every span (an MT = 1 issuer with no step in a one-step
+            // span commits nothing new: its arrival comes at once); the epilogue adds only
+            // the accumulators that received a step
             if (ok) tc2_commit_both(tfull(acc));
             jw0 += count_par(s0, s1, 0);
             jw1 += count_par(s0, s1, 1);
+            ja += s1 - s0;
             ++it;
         }
         tc2_commit_local(drain);
@@ -398,7 +419,10 @@ k_tc2_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
     if (warp == 0) {
         // ------------------------------------------------------------ activations (both CTAs)
         if (lane == 0) {
-            int sa = 0, pa = 0, issued = 0;
+            int last_ph[SA];                             // phase of each stage's last issued copy
+#pragma unroll
+            for (int i = 0; i < SA; ++i) last_ph[i] = -1;
+            int ja = 0, ja0 = 0, ja1 = 0;
             bool ok = true;
             Spans spn(skm, pair, npairs, ntiles, nsteps);
             int64_t tile;
@@ -407,7 +431,10 @@ k_tc2_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
                 const int m0 = (int)((tile % mtiles) * BM * MT + crank * HM);
                 for (int step = s0; step < s1 && ok; ++step) {
                     // one stage = the step's MT token tiles (slots MT sa .. MT sa + MT - 1), one
-                    // barrier pair: the issuing thread tests and commits once per step
+                    // barrier pair: an issuing thread tests and commits once per step
+                    const int g = step & 1;
+                    int sa, pa;
+                    apos(ja + (step - s0), (g ? ja1 : ja0) + count_par(s0, step, g), g, sa, pa);
                     if (!(ok = tc::mbar_wait(emptyA(sa), pa ^ 1, s_abort))) break;
                     if (leader) tc::mbar_expect_tx(fullA(sa), MT * 2 * A_BYTES);    // both halves land here
                     const uint32_t bar = mapa(fullA(sa), 0);
@@ -418,13 +445,15 @@ k_tc2_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
                         if (step < nks) tma_load_2d_pair(dst, &tmA, bar, step * BK, m0 + u * BM);
                         else tma_load_2d_pair(dst, &tmL, bar, (step - nks) * BK, m0 + u * BM);
                     }
-                    ++issued;
-                    if (++sa == SAS) { sa = 0; pa ^= 1; }
+                    last_ph[sa] = pa;
                 }
+                ja += s1 - s0;
+                ja0 += count_par(s0, s1, 0);
+                ja1 += count_par(s0, s1, 1);
             }
-            if (!ok && leader)
-                for (int i = 1; i <= SAS && i <= issued; ++i)
-                    mbar_drain_cl(fullA((issued - i) % SAS), ((issued - i) / SAS) & 1);
+            if (!ok && leader)                           // wait for the copies in flight
+                for (int i = 0; i < SA; ++i)
+                    if (last_ph[i] >= 0) mbar_drain_cl(fullA(i), last_ph[i]);
         }
     } else if (warp == 14) {
         // ------------------------------------------------------------ packed weights (own half)
@@ -723,18 +752,37 @@ k_tc2_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
                     }
                 }
             };
-            // two chunks per wait for the tensor-memory loads (one wait per chunk left the
-            // epilogue bound by their latency)
+            // MT = 1: issuer g's accumulator (columns g BN) holds the span's steps of parity
+            // g; the tile's sum is issuer 0's plus issuer 1's (a one-step span fills one)
+            const bool has0 = MT == 2 || count_par(s0, s1, 0) > 0;
+            const bool has1 = MT == 2 || count_par(s0, s1, 1) > 0;
+            const uint32_t trow = tmem_base + ((uint32_t)(q * 32) << 16);
+            if (MT == 2 || !(has0 && has1)) {
+                // two chunks per wait for the tensor-memory loads (one wait per chunk left
+                // the epilogue bound by their latency)
+                const uint32_t cb = (MT == 1 && !has0) ? (uint32_t)BN : 0u;
 #pragma unroll 1
-            for (int ucc = 0; ucc < MT * (BN / 32); ucc += 2) {
-                uint32_t r0[32], r1[32];
-                const uint32_t t0 = tmem_base + ((uint32_t)(q * 32) << 16) +
-                                    (uint32_t)((acc * MT + ucc / (BN / 32)) * BN + (ucc % (BN / 32)) * 32);
-                TC_LD32(t0, r0);
-                TC_LD32(t0 + 32, r1);                    // chunk ucc + 1: the next 32 columns (BN / 32 is even)
-                asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-                emit(ucc, r0);
-                emit(ucc + 1, r1);
+                for (int ucc = 0; ucc < MT * (BN / 32); ucc += 2) {
+                    uint32_t r0[32], r1[32];
+                    const uint32_t t0 = trow + cb + (uint32_t)((ucc / (BN / 32)) * BN + (ucc % (BN / 32)) * 32);
+                    TC_LD32(t0, r0);
+                    TC_LD32(t0 + 32, r1);                // chunk ucc + 1: the next 32 columns (BN / 32 is even)
+                    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+                    emit(ucc, r0);
+                    emit(ucc + 1, r1);
+                }
+            } else {
+#pragma unroll 1
+                for (int ucc = 0; ucc < BN / 32; ++ucc) {
+                    uint32_t r0[32], r1[32];
+                    const uint32_t t0 = trow + (uint32_t)(ucc * 32);
+                    TC_LD32(t0, r0);
+                    TC_LD32(t0 + BN, r1);                // the same 32 columns of issuer 1's accumulator
+                    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) r0[j] = __float_as_uint(__uint_as_float(r0[j]) + __uint_as_float(r1[j]));
+                    emit(ucc, r0);
+                }
             }
             if (nc > 0) asm volatile("cp.async.wait_all;" ::: "memory");
             tc::tc_fence_before();
