@@ -277,6 +277,12 @@ constexpr int kSkMaxRp = 64;
 // Stream-K when whole tiles would leave a partial wave, there are at least half as
 // many tiles as pairs (fewer: more partial-sum traffic than gain), and, in the
 // backward, more tiles than pairs: with fewer, the pairs left free run dB and dA.
+// A forward that the wave rule leaves at one token tile takes two, and stream-K,
+// where two-token-tile tiles still number at least a third of the pairs: a
+// one-token-tile step is bound by its decode (each decoded stage feeds one token
+// tile; 0.49 of the burst peak against 0.75 with two, measured), which costs more
+// than the partial sums of tiles split two or three ways (70B projections at 512
+// tokens: 1040 -> 1091 TFLOP/s on one box).
 struct Tc2Sched {
     int mt;
     bool sk;
@@ -286,8 +292,12 @@ struct Tc2Sched {
 Tc2Sched tc2_schedule(int64_t M, int64_t n_out, int pairs, bool bwd) {
     Tc2Sched sc{};
     sc.mt = tc2_token_tiles(M, n_out, pairs);
-    sc.ntiles = cdiv(M, (int64_t)tc2::BM * sc.mt) * cdiv(n_out, tc2::BN);
-    sc.sk = pairs > 0 && pairs <= kSkMaxPairs && sc.ntiles % pairs != 0 && 2 * sc.ntiles >= pairs &&
+    const int64_t nt = cdiv(n_out, tc2::BN);
+    const bool promote = !bwd && pairs > 0 && sc.mt == 1 && cdiv(M, (int64_t)tc2::BM) >= 2 &&
+                         3 * cdiv(M, 2 * (int64_t)tc2::BM) * nt >= pairs;
+    if (promote) sc.mt = 2;
+    sc.ntiles = cdiv(M, (int64_t)tc2::BM * sc.mt) * nt;
+    sc.sk = pairs > 0 && pairs <= kSkMaxPairs && sc.ntiles % pairs != 0 && (promote ? 3 : 2) * sc.ntiles >= pairs &&
             (!bwd || sc.ntiles > pairs);
     return sc;
 }
