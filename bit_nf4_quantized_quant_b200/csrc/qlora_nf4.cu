@@ -277,12 +277,14 @@ constexpr int kSkMaxRp = 64;
 // Stream-K when whole tiles would leave a partial wave, there are at least half as
 // many tiles as pairs (fewer: more partial-sum traffic than gain), and, in the
 // backward, more tiles than pairs: with fewer, the pairs left free run dB and dA.
-// A forward that the wave rule leaves at one token tile takes two, and stream-K,
-// where two-token-tile tiles still number at least a third of the pairs: a
-// one-token-tile step is bound by its decode (each decoded stage feeds one token
-// tile; 0.49 of the burst peak against 0.75 with two, measured), which costs more
-// than the partial sums of tiles split two or three ways (70B projections at 512
-// tokens: 1040 -> 1091 TFLOP/s on one box).
+// A product that the wave rule leaves at one token tile takes two, and stream-K
+// over all pairs, where two-token-tile tiles still number at least a third of the
+// pairs: a one-token-tile step is bound by its decode (each decoded stage feeds one
+// token tile; 0.49 of the burst peak against 0.75 with two, measured), which costs
+// more than the partial sums of tiles split two or three ways and, in the backward,
+// than running dB and dA after the fused kernel instead of beside it (70B
+// projections at 512 tokens on one box: 1040 -> 1091 TFLOP/s with the forward
+// promoted, 1091 -> 1180 with the backward too).
 struct Tc2Sched {
     int mt;
     bool sk;
@@ -293,12 +295,12 @@ Tc2Sched tc2_schedule(int64_t M, int64_t n_out, int pairs, bool bwd) {
     Tc2Sched sc{};
     sc.mt = tc2_token_tiles(M, n_out, pairs);
     const int64_t nt = cdiv(n_out, tc2::BN);
-    const bool promote = !bwd && pairs > 0 && sc.mt == 1 && cdiv(M, (int64_t)tc2::BM) >= 2 &&
+    const bool promote = pairs > 0 && sc.mt == 1 && cdiv(M, (int64_t)tc2::BM) >= 2 &&
                          3 * cdiv(M, 2 * (int64_t)tc2::BM) * nt >= pairs;
     if (promote) sc.mt = 2;
     sc.ntiles = cdiv(M, (int64_t)tc2::BM * sc.mt) * nt;
     sc.sk = pairs > 0 && pairs <= kSkMaxPairs && sc.ntiles % pairs != 0 && (promote ? 3 : 2) * sc.ntiles >= pairs &&
-            (!bwd || sc.ntiles > pairs);
+            (!bwd || promote || sc.ntiles > pairs);
     return sc;
 }
 

@@ -60,8 +60,8 @@ def test_stream_k_spans(M, N, K, r, bwd, pairs):
         assert ntiles % pairs == 0 or 2 * ntiles < pairs or (bwd and ntiles <= pairs)
         return
     if 2 * ntiles < pairs:
-        # a forward promoted to two token tiles: tiles split two or three ways
-        assert not bwd and mt == 2 and 3 * ntiles >= pairs
+        # promoted to two token tiles: tiles split two or three ways
+        assert mt == 2 and 3 * ntiles >= pairs
     rp = cdiv(r, 16) * 16
     nsteps = cdiv(n_red, 64) + cdiv(cdiv(2 * rp, 64) * 64, 64)
     taken = {}
@@ -102,11 +102,10 @@ def test_schedule_of_the_default_workload():
     assert ops.pair_schedule(2048, 11008, 74, False) == (2, 172, True)
     assert ops.pair_schedule(2048, 11008, 74, True) == (2, 172, True)
     assert ops.pair_schedule(160, 1024, 74, False)[2] is False
-    # 70B 8192-wide outputs at 512 tokens: 64 one-token-tile tiles, or 32 of two; the
-    # forward takes two (decode-bound otherwise) with tiles split over two or three
-    # pairs, the backward one (64 tiles, ten pairs left to dB and dA)
+    # 70B 8192-wide outputs at 512 tokens: 64 one-token-tile tiles, or 32 of two; both
+    # directions take two (decode-bound otherwise) with tiles split over two or three pairs
     assert ops.pair_schedule(512, 8192, 74, False) == (2, 32, True)
-    assert ops.pair_schedule(512, 8192, 74, True) == (1, 64, False)
+    assert ops.pair_schedule(512, 8192, 74, True) == (2, 32, True)
     assert ops.pair_schedule(512, 1024, 74, False) == (1, 8, False)
 
 
