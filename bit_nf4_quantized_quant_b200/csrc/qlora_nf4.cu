@@ -274,9 +274,11 @@ constexpr int kSkMaxRp = 64;
 
 // Schedule of the SM-pair kernel for an n_out-wide output on `pairs` pairs: token
 // tiles per W' stage (mt) and whether the (tile, step) units are dealt stream-K.
-// Stream-K when whole tiles would leave a partial wave, there are at least half as
-// many tiles as pairs (fewer: more partial-sum traffic than gain), and, in the
-// backward, more tiles than pairs: with fewer, the pairs left free run dB and dA.
+// Stream-K when whole tiles would leave a partial wave and there are at least a
+// third as many tiles as pairs (fewer: tiles split more than three ways, whose
+// owner adds more partial sums than the split gains).  The backward keeps whole
+// tiles where they fill at least three quarters of the pairs without covering
+// them: the pairs left free run dB and dA beside it.
 // A product that the wave rule leaves at one token tile takes two, and stream-K
 // over all pairs, where two-token-tile tiles still number at least a third of the
 // pairs: a one-token-tile step is bound by its decode (each decoded stage feeds one
@@ -299,8 +301,8 @@ Tc2Sched tc2_schedule(int64_t M, int64_t n_out, int pairs, bool bwd) {
                          3 * cdiv(M, 2 * (int64_t)tc2::BM) * nt >= pairs;
     if (promote) sc.mt = 2;
     sc.ntiles = cdiv(M, (int64_t)tc2::BM * sc.mt) * nt;
-    sc.sk = pairs > 0 && pairs <= kSkMaxPairs && sc.ntiles % pairs != 0 && (promote ? 3 : 2) * sc.ntiles >= pairs &&
-            (!bwd || promote || sc.ntiles > pairs);
+    sc.sk = pairs > 0 && pairs <= kSkMaxPairs && sc.ntiles % pairs != 0 && 3 * sc.ntiles >= pairs &&
+            (!bwd || promote || sc.ntiles > pairs || 4 * sc.ntiles < 3 * (int64_t)pairs);
     return sc;
 }
 

@@ -69,6 +69,8 @@ CASES = [
     (100, 256, 38912, 8),       # single-SM kernel: 152 backward tiles
     (512, 11008, 1024, 16),     # SM pairs: 86 forward pair tiles
     (520, 1024, 11008, 32),     # SM pairs: 3 x 43 = 129 backward pair tiles, ragged M
+    (512, 4096, 4096, 16),      # SM pairs, one token tile per step, stream-K both ways (32 tiles)
+    (500, 5120, 1024, 16),      # SM pairs, one token tile, stream-K forward (40 tiles), ragged M
 ]
 
 
@@ -319,6 +321,8 @@ def test_multi_tile_pair_kernel_repeats_bit_identically(oracle_mod, M, N, K, r):
 
 
 @pytest.mark.parametrize("M,N,K,r,bwd", [(512, 28672, 1024, 16, False),   # SM pairs, 112 tiles stream-K
+                                         (512, 4096, 4096, 16, False),    # SM pairs, one token tile, stream-K
+                                         (512, 4096, 4096, 16, True),
                                          (512, 4096, 11008, 64, True),    # SM pairs, backward over 11008
                                          (1024, 4096, 11008, 16, True),   # SM pairs, backward, 172 tiles stream-K
                                          (100, 38912, 256, 16, False),    # single SM, 152 tiles
