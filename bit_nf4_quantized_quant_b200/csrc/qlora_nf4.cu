@@ -276,9 +276,12 @@ constexpr int kSkMaxRp = 64;
 // tiles per W' stage (mt) and whether the (tile, step) units are dealt stream-K.
 // Stream-K when whole tiles would leave a partial wave and there are at least a
 // third as many tiles as pairs (fewer: tiles split more than three ways, whose
-// owner adds more partial sums than the split gains).  The backward keeps whole
-// tiles where they fill at least three quarters of the pairs without covering
-// them: the pairs left free run dB and dA beside it.
+// owner adds more partial sums than the split gains), but whole tiles are kept
+// where they fill at least three quarters of the pairs without covering them: the
+// drain of a split tile's partial sums and the owner's fix-up cost more than the
+// idle pairs (7B block at 2048 tokens, 64 tiles of its 4096-wide forwards on 74
+// pairs: 1.477 -> 1.430 ms a step on one box), and in the backward the pairs left
+// free run dB and dA beside it.
 // A product that the wave rule leaves at one token tile takes two, and stream-K
 // over all pairs, where two-token-tile tiles still number at least a third of the
 // pairs: a one-token-tile step is bound by its decode (each decoded stage feeds one
@@ -302,7 +305,7 @@ Tc2Sched tc2_schedule(int64_t M, int64_t n_out, int pairs, bool bwd) {
     if (promote) sc.mt = 2;
     sc.ntiles = cdiv(M, (int64_t)tc2::BM * sc.mt) * nt;
     sc.sk = pairs > 0 && pairs <= kSkMaxPairs && sc.ntiles % pairs != 0 && 3 * sc.ntiles >= pairs &&
-            (!bwd || promote || sc.ntiles > pairs || 4 * sc.ntiles < 3 * (int64_t)pairs);
+            (promote || sc.ntiles > pairs || 4 * sc.ntiles < 3 * (int64_t)pairs);
     return sc;
 }
 

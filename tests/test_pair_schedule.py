@@ -56,8 +56,8 @@ def test_stream_k_spans(M, N, K, r, bwd, pairs):
     mt, ntiles, sk = ops.pair_schedule(M, n_out, pairs, bwd)
     assert ntiles == cdiv(M, 256 * mt) * cdiv(n_out, 256)
     if not sk:
-        # whole waves, too few tiles, or (backward) whole tiles on at least 3/4 of the pairs
-        assert ntiles % pairs == 0 or 3 * ntiles < pairs or (bwd and 3 * pairs <= 4 * ntiles <= 4 * pairs)
+        # whole waves, too few tiles, or whole tiles on at least 3/4 of the pairs
+        assert ntiles % pairs == 0 or 3 * ntiles < pairs or 3 * pairs <= 4 * ntiles <= 4 * pairs
         return
     assert 3 * ntiles >= pairs                        # tiles split at most three ways
     rp = cdiv(r, 16) * 16
@@ -94,8 +94,8 @@ def test_stream_k_spans(M, N, K, r, bwd, pairs):
 
 def test_schedule_of_the_default_workload():
     # 7B block at 2048 tokens on 74 pairs: 4096-wide outputs are 64 two-token-tile tiles
-    # (stream-K forward; backward leaves 10 pairs to dB and dA), 11008-wide ones 172
-    assert ops.pair_schedule(2048, 4096, 74, False) == (2, 64, True)
+    # (whole tiles; the backward leaves 10 pairs to dB and dA), 11008-wide ones 172
+    assert ops.pair_schedule(2048, 4096, 74, False) == (2, 64, False)
     assert ops.pair_schedule(2048, 4096, 74, True) == (2, 64, False)
     assert ops.pair_schedule(2048, 11008, 74, False) == (2, 172, True)
     assert ops.pair_schedule(2048, 11008, 74, True) == (2, 172, True)
