@@ -51,9 +51,9 @@ _PAIR_SRC = ("common.cuh", "nf4_decode.cuh", "tc_gemm.cuh", "tc2_gemm.cuh", "qlo
 _GEMV_SRC = ("common.cuh", "nf4_decode.cuh", "tc_gemm.cuh", "gemv_mma.cuh", "small_lora.cuh", "dropout.cuh",
              "qlora_nf4.cu")
 TRAFFIC = {
-    "workload3_M2048": {"bytes_per_launch": 57498642, "files": _PAIR_SRC, "src": "46b5045a2de9"},
+    "workload3_M2048": {"bytes_per_launch": 54590446, "files": _PAIR_SRC, "src": "0706f491eb5d"},
     # small M: one forward chain (GEMV + T + finish) per projection
-    "workload2_M1": {"bytes_per_launch": 24059008, "files": _GEMV_SRC, "src": "484a198816e0"},
+    "workload2_M1": {"bytes_per_launch": 24058496, "files": _GEMV_SRC, "src": "0853182519f5"},
 }
 
 
