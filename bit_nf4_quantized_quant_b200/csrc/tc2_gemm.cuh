@@ -3,7 +3,8 @@
 //
 // Same computation as tc_gemm.cuh (forward Y = X W'^T + s T B^T, backward
 // dX = dY W' + s U A), but a cluster of two CTAs computes one 256-token x
-// 256-output tile with 256 x 256 x 16 MMAs issued by the leader CTA (rank 0):
+// 256-output tile with 256 x 256 x 16 MMAs issued by two threads of the leader
+// CTA (rank 0; one thread's issue cost is about one MMA's tensor time):
 //   - each CTA holds its 128 tokens of the activation tile (A operand) and
 //     its 128 output features of the weight tile (B operand) in its own
 //     shared memory, at the same offsets;
