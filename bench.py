@@ -234,13 +234,15 @@ def run_ours(args, rank, world, local_rank):
         else:
             ops.qlora_linear_fwd(L["X"], w, L["A"], L["B"], s, Y=L["Y"], T_out=L["T"], ws=ws)
 
-    def bwd_call(L, w, off):
+    def bwd_call(L, w, off, g=""):
+        # g selects the gradient buffer: "" the main one, "2" the second one the end-to-end
+        # pipeline alternates with
+        dA, dB = L["dA" + g], L["dB" + g]
         if args.dropout > 0:
             ops.qlora_linear_bwd_dropout(L["X"], L["dY"], w, L["A"], L["B"], s, args.dropout, DROPOUT_SEED, off,
-                                         T=L["T"], dX=L["dX"], dA=L["dA"], dB=L["dB"], ws=ws)
+                                         T=L["T"], dX=L["dX"], dA=dA, dB=dB, ws=ws)
         else:
-            ops.qlora_linear_bwd(L["X"], L["dY"], w, L["A"], L["B"], s, T=L["T"], dX=L["dX"], dA=L["dA"],
-                                 dB=L["dB"], ws=ws)
+            ops.qlora_linear_bwd(L["X"], L["dY"], w, L["A"], L["B"], s, T=L["T"], dX=L["dX"], dA=dA, dB=dB, ws=ws)
 
     def step(events=None, collective=True):
         c = it[0] % copies
@@ -407,13 +409,23 @@ def run_ours(args, rank, world, local_rank):
     # Events keep each buffer's order: layer j's inputs are overwritten only after
     # the previous step's compute has read them, and its outputs (and the
     # gradient buffer) only after the previous step's copy-out has read them.
+    # The adapter gradients alternate between two device buffers by step, so a step's
+    # first backward does not wait for the previous step's gradients to reach the host
+    # (only for those of the step before it, long since copied).
     comp = stream
     s_in, s_out = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
     ev_in = [torch.cuda.Event() for _ in layers]      # layer j's inputs have landed
     ev_done = [torch.cuda.Event() for _ in layers]    # layer j's calls are done
     ev_out = [torch.cuda.Event() for _ in layers]     # layer j's outputs are on the host
-    ev_grad, ev_gout = torch.cuda.Event(), torch.cuda.Event()
+    ev_grad = torch.cuda.Event()
+    ev_gout = [torch.cuda.Event(), torch.cuda.Event()]  # gradient buffer g is on the host
+    gbufs = [gbuf, torch.empty_like(gbuf) if bwd else gbuf]
+    if bwd:
+        for L, (oa, ob) in zip(layers, offs):
+            L["dA2"] = gbufs[1][oa:oa + r * L["p"].K].view(r, L["p"].K)
+            L["dB2"] = gbufs[1][ob:ob + L["p"].N * r].view(L["p"].N, r)
     primed = [False]
+    nstep = [0]
 
     def e2e_step_serial():
         for j, L in enumerate(layers):
@@ -435,6 +447,8 @@ def run_ours(args, rank, world, local_rank):
     def e2e_step():
         if not pipelined:
             return e2e_step_serial()
+        g = nstep[0] & 1
+        gb = gbufs[g]
         for j, L in enumerate(layers):
             with torch.cuda.stream(s_in):
                 if primed[0]:
@@ -448,9 +462,9 @@ def run_ours(args, rank, world, local_rank):
                 comp.wait_event(ev_out[j])
             fwd_call(L, L["w"], j)
             if bwd:
-                if j == 0 and primed[0]:
-                    comp.wait_event(ev_gout)          # the gradient buffer was copied out
-                bwd_call(L, L["w"], j)
+                if j == 0 and nstep[0] >= 2:
+                    comp.wait_event(ev_gout[g])       # this buffer's gradients of two steps ago are out
+                bwd_call(L, L["w"], j, "2" if g else "")
             ev_done[j].record(comp)
             with torch.cuda.stream(s_out):
                 s_out.wait_event(ev_done[j])
@@ -459,14 +473,15 @@ def run_ours(args, rank, world, local_rank):
                     hout[j][1].copy_(L["dX"], non_blocking=True)
                 ev_out[j].record(s_out)
         if world > 1 and bwd:
-            dist.all_reduce(gbuf)
+            dist.all_reduce(gb)
         if bwd:
             ev_grad.record(comp)
             with torch.cuda.stream(s_out):
                 s_out.wait_event(ev_grad)
-                hg.copy_(gbuf, non_blocking=True)
-                ev_gout.record(s_out)
+                hg.copy_(gb, non_blocking=True)
+                ev_gout[g].record(s_out)
         primed[0] = True
+        nstep[0] += 1
 
     for _ in range(max(1, args.warmup // 2)):
         e2e_step()
